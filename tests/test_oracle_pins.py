@@ -1,0 +1,425 @@
+"""Pins of the CPU oracle to what the pages and the mathematics fix.
+
+None of these tests re-types the oracle's formulas: each checks a printed
+worked example, a closed form, an invariant, a special case that reduces to a
+library routine (torch / numpy), or brute force over tiny inputs, chosen so a
+dropped term, a wrong sign or index or a transposed operand fails one of them.
+"""
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from conftest import read_golden
+from workload import stored_numpy
+
+pytestmark = pytest.mark.filterwarnings("ignore::RuntimeWarning")
+
+
+# ----------------------------------------------------------------------
+# storage formats
+# ----------------------------------------------------------------------
+
+def test_e4m3_decode_all_codes_match_library():
+    codes = np.arange(256, dtype=np.uint8)
+    ours = oracle.e4m3_decode(codes)
+    lib = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    nan = np.isnan(lib)
+    assert np.array_equal(np.isnan(ours), nan)
+    assert nan.sum() == 2  # S.1111.111 for both signs
+    assert np.array_equal(ours[~nan], lib[~nan])
+    assert ours[~nan].max() == 448.0 and ours[~nan].min() == -448.0
+    assert oracle.e4m3_decode([0x01])[0] == 2.0 ** -9  # smallest subnormal
+
+
+def test_e4m3_encode_roundtrip_and_rounding():
+    codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], dtype=np.uint8)
+    assert np.array_equal(oracle.e4m3_encode(oracle.e4m3_decode(codes)), codes)
+    rng = np.random.default_rng(0)
+    vals = np.concatenate([rng.normal(0, 50, 3000), rng.normal(0, 0.01, 1000)]).astype(np.float32)
+    # midpoints between neighbouring codes exercise ties-to-even
+    pos = np.sort(oracle.e4m3_decode(np.arange(0, 0x7F, dtype=np.uint8)))
+    mids = ((pos[:-1] + pos[1:]) / 2).astype(np.float32)
+    vals = np.concatenate([vals, mids, -mids]).astype(np.float32)
+    vals = vals[np.abs(vals) <= 448]
+    lib = torch.from_numpy(vals).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    ours = oracle.e4m3_encode(vals.astype(np.float64))
+    assert np.array_equal(ours, lib)
+    assert oracle.e4m3_encode([1e6])[0] == 0x7E and oracle.e4m3_encode([-1e6])[0] == 0xFE
+
+
+def test_bf16_decode_all_codes_match_library():
+    codes = np.arange(65536, dtype=np.uint16)
+    ours = oracle.decode(codes)
+    lib = torch.from_numpy(codes.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    nan = np.isnan(lib)
+    assert np.array_equal(np.isnan(ours), nan)
+    assert np.array_equal(ours[~nan], lib[~nan])
+
+
+def test_bf16_encode_matches_library_rne():
+    rng = np.random.default_rng(1)
+    vals = np.concatenate([rng.normal(0, 1, 4000), rng.normal(0, 1e-30, 200), rng.normal(0, 1e30, 200)])
+    vals = vals.astype(np.float32)  # exactly representable: no double rounding on the library side
+    lib = torch.from_numpy(vals).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(oracle.bf16_encode(vals.astype(np.float64)), lib)
+
+
+# ----------------------------------------------------------------------
+# compressor
+# ----------------------------------------------------------------------
+
+def test_compress_worked_example(golden_dir):
+    g = read_golden(os.path.join(golden_dir, "compress_worked_example.txt"))
+    C = np.array([g[f"C{i}"] for i in range(4)], dtype=np.float32)
+    S = np.array([g[f"S{i}"] for i in range(4)], dtype=np.float64)
+    assert np.allclose(S.sum(axis=0), 1.0)
+    Z = np.log(S).astype(np.float32)
+    out = oracle.compress(C[None], Z[None], m=4)
+    assert out.shape == (1, 1, 3)
+    assert np.allclose(out[0, 0], g["EXPECTED"], atol=1e-6)
+
+
+def test_compress_m1_is_identity():
+    rng = np.random.default_rng(2)
+    x = rng.normal(size=(2, 37, 24)).astype(np.float32)
+    z = rng.normal(size=(2, 37, 24)).astype(np.float32)
+    assert np.array_equal(oracle.compress(x, z, m=1), x.astype(np.float64))
+
+
+def test_compress_equal_logits_give_chunk_mean():
+    rng = np.random.default_rng(3)
+    x = rng.normal(size=(1, 4 * 9, 16)).astype(np.float32)
+    z = np.full_like(x, 0.37)
+    out = oracle.compress(x, z, m=4)
+    mean = x.astype(np.float64).reshape(1, 9, 4, 16).mean(axis=2)
+    assert np.allclose(out, mean, atol=1e-12)
+    # the tail (tokens of an incomplete chunk) is not compressed
+    out2 = oracle.compress(x[:, :35], z[:, :35], m=4)
+    assert out2.shape == (1, 8, 16) and np.allclose(out2, mean[:, :8], atol=1e-12)
+
+
+def test_compress_dominant_gate_selects_that_token_per_channel():
+    """A gate logit far above the others in one channel makes the entry equal
+    to that token's value in that channel: pins the token/chunk/channel
+    indexing and that the softmax runs over tokens, not channels."""
+    rng = np.random.default_rng(4)
+    B, n_ent, m, C = 2, 6, 8, 5
+    x = rng.normal(size=(B, n_ent * m, C)).astype(np.float32)
+    z = rng.normal(size=(B, n_ent * m, C)).astype(np.float32)
+    pick = rng.integers(0, m, size=(B, n_ent, C))
+    for b, s, c in itertools.product(range(B), range(n_ent), range(C)):
+        z[b, s * m + pick[b, s, c], c] = 200.0
+    out = oracle.compress(x, z, m=m)
+    for b, s, c in itertools.product(range(B), range(n_ent), range(C)):
+        assert out[b, s, c] == pytest.approx(float(x[b, s * m + pick[b, s, c], c]), abs=1e-12)
+
+
+def test_compress_shift_invariance_and_bf16_input():
+    rng = np.random.default_rng(5)
+    x = rng.normal(size=(1, 128, 8)).astype(np.float32)
+    z = rng.normal(size=(1, 128, 8)).astype(np.float32)
+    a = oracle.compress(x, z, m=128)
+    b = oracle.compress(x, (z + 3.0).astype(np.float32), m=128)
+    assert np.allclose(a, b, atol=1e-6)
+    # two-token closed form: weight of token 0 is sigmoid(z0 - z1)
+    x2 = np.array([[[2.0], [-1.0]]], dtype=np.float32)
+    z2 = np.array([[[0.25], [-0.5]]], dtype=np.float32)
+    s = 1.0 / (1.0 + math.exp(-(0.25 + 0.5)))
+    assert oracle.compress(x2, z2, m=2)[0, 0, 0] == pytest.approx(s * 2.0 + (1 - s) * -1.0, abs=1e-12)
+    xb = torch.from_numpy(x).to(torch.bfloat16)
+    zb = torch.from_numpy(z).to(torch.bfloat16)
+    ob = oracle.compress(stored_numpy(xb), stored_numpy(zb), m=128)
+    of = oracle.compress(xb.float().numpy(), zb.float().numpy(), m=128)
+    assert np.allclose(ob, of, atol=1e-12)
+
+
+def test_quantize_rows_bounds():
+    rng = np.random.default_rng(6)
+    v = rng.normal(size=(50, 128))
+    v[3] = 0.0
+    codes, scales = oracle.quantize_e4m3_rows(v)
+    assert scales[3] == 1.0 and np.all(codes[3] == 0)
+    deq = oracle.e4m3_decode(codes) * scales[:, None]
+    amax = np.abs(v).max(axis=1)
+    assert np.allclose(np.abs(deq).max(axis=1), amax, rtol=1e-12)  # the row max maps to exactly 448
+    # nearest-code error: at most half a step of the e4m3 grid (relative 2^-4 for normals)
+    rel = np.abs(deq - v) / np.maximum(np.abs(v), 2.0 ** -6 * scales[:, None])
+    assert rel.max() <= 2.0 ** -4 + 1e-12
+
+
+# ----------------------------------------------------------------------
+# visibility and counts
+# ----------------------------------------------------------------------
+
+def test_page_counts(golden_dir):
+    g = read_golden(os.path.join(golden_dir, "page_counts.txt"))
+    L, m, n = g["HCA"]
+    assert oracle.n_visible(int(L) - 1, int(m)) == int(n)
+    L, m, n = g["CSA"]
+    assert oracle.n_visible(int(L) - 1, int(m)) == int(n)
+    k, n, pct = g["TOPK_FRACTION_PERCENT"]
+    assert round(100.0 * k / n, 2) == pct
+    w, mh = g["WINDOW_EQUALS_HCA_RATE"]
+    assert w == mh
+    # the workloads' own counts
+    assert oracle.n_visible(4095, 4) == 1024 and oracle.n_visible(4095, 128) == 32
+    assert oracle.n_visible(1048575, 4) == 262144 and oracle.n_visible(1048575, 128) == 8192
+    assert oracle.n_visible(126976 - 1, 4) == 31744 and oracle.n_visible(131071, 4) == 32768
+
+
+def test_visibility_coverage_invariant():
+    """With n_win = m' = 128, every token 0..t lies in a visible HCA entry or
+    in the window, and no visible entry reaches past t."""
+    m, W = 128, 128
+    for t in list(range(0, 600)) + [1048575, 1048574, 1048448, 1048447]:
+        nvis = oracle.n_visible(t, m)
+        covered_hi = nvis * m  # entries cover [0, covered_hi)
+        assert covered_hi <= t + 1
+        win_lo = max(0, t - W + 1)
+        assert win_lo <= covered_hi  # no gap between entries and window
+    # a block ending exactly at t is visible; one ending at t+1 is not
+    assert oracle.n_visible(3, 4) == 1 and oracle.n_visible(2, 4) == 0
+
+
+# ----------------------------------------------------------------------
+# Lightning indexer
+# ----------------------------------------------------------------------
+
+def _idx_case(rng, B, T, L, m, HI, DI):
+    q = rng.normal(size=(B, T, HI, DI)).astype(np.float32)
+    w = rng.uniform(size=(B, T, HI)).astype(np.float32)
+    k = rng.normal(size=(B, L // m, DI)).astype(np.float32)
+    return q, w, k
+
+
+def test_index_single_head_unit_weight_is_relu_dot():
+    rng = np.random.default_rng(7)
+    q, _, k = _idx_case(rng, 1, 1, 64, 4, 1, 32)
+    w = np.ones((1, 1, 1), dtype=np.float32)
+    s = oracle.index_scores(q, w, k, None, ctx_len=64, m=4)
+    dots = k[0].astype(np.float64) @ q[0, 0, 0].astype(np.float64)
+    assert np.allclose(s[0, 0], np.maximum(dots, 0.0), atol=1e-12)
+    # ReLU closed form: score(q) + score(-q) = |q.k|
+    s_neg = oracle.index_scores(-q, w, k, None, ctx_len=64, m=4)
+    assert np.allclose(s[0, 0] + s_neg[0, 0], np.abs(dots), atol=1e-12)
+
+
+def test_index_heads_add_and_contribute_nonnegatively():
+    rng = np.random.default_rng(8)
+    q, w, k = _idx_case(rng, 2, 1, 256, 4, 4, 16)
+    full = oracle.index_scores(q, w, k, None, ctx_len=256, m=4)
+    parts = [oracle.index_scores(q[:, :, h:h + 1], w[:, :, h:h + 1], k, None, ctx_len=256, m=4) for h in range(4)]
+    assert np.allclose(full, sum(parts), atol=1e-10)
+    assert all((p >= 0).all() for p in parts)  # w >= 0: a head can only add relevance
+    # raising one head's query along a key that it already matches cannot lower the score
+    q2 = q.copy()
+    q2[0, 0, 1] += 0.5 * k[0, 5]
+    s2 = oracle.index_scores(q2, w, k, None, ctx_len=256, m=4)
+    assert s2[0, 0, 5] >= full[0, 0, 5]
+    # w scales linearly
+    s3 = oracle.index_scores(q, (2 * w).astype(np.float32), k, None, ctx_len=256, m=4)
+    assert np.allclose(s3, 2 * full, atol=1e-10)
+
+
+def test_index_scale_and_fp8_keys():
+    rng = np.random.default_rng(9)
+    q, w, k = _idx_case(rng, 1, 1, 128, 4, 3, 16)
+    codes, scales = oracle.quantize_e4m3_rows(k[0].astype(np.float64))
+    sc32 = scales.astype(np.float32)[None]
+    s8 = oracle.index_scores(q, w, codes[None], sc32, ctx_len=128, m=4)
+    s8_unit = oracle.index_scores(q, w, codes[None], np.ones_like(sc32), ctx_len=128, m=4)
+    # the per-entry scale multiplies that entry's score
+    assert np.allclose(s8, s8_unit * sc32.astype(np.float64)[:, None, :], rtol=1e-14, atol=0)
+    # e4m3 values are exact in float32: coded keys score like their decoded values
+    dec32 = oracle.e4m3_decode(codes).astype(np.float32)[None]
+    assert np.array_equal(s8_unit, oracle.index_scores(q, w, dec32, None, ctx_len=128, m=4))
+    # a NULL scale means 1
+    assert np.array_equal(s8_unit, oracle.index_scores(q, w, codes[None], None, ctx_len=128, m=4))
+
+
+def test_index_visibility_boundary():
+    rng = np.random.default_rng(10)
+    L, m, T = 40, 4, 7
+    q, w, k = _idx_case(rng, 1, T, L, m, 2, 8)
+    s = oracle.index_scores(q, w, k, None, ctx_len=L, m=m)
+    for j in range(T):
+        t = L - T + j
+        nvis = (t + 1) // m
+        assert np.all(np.isfinite(s[0, j, :nvis]))
+        assert np.all(np.isneginf(s[0, j, nvis:]))
+
+
+# ----------------------------------------------------------------------
+# top-k
+# ----------------------------------------------------------------------
+
+def _better(a, b):
+    """(score, index) a ranks before b: higher score, then lower index."""
+    return a[0] > b[0] or (a[0] == b[0] and a[1] < b[1])
+
+
+@pytest.mark.parametrize("n", [1, 5, 9])
+def test_topk_brute_force_over_subsets(n):
+    rng = np.random.default_rng(11 + n)
+    for trial in range(6):
+        # few distinct values -> many exact ties
+        scores = rng.integers(0, 4, size=n).astype(np.float64) if trial % 2 else rng.normal(size=n)
+        for k in range(1, n + 2):
+            idx, sel, kth = oracle.select_row(scores, n, k)
+            take = min(k, n)
+            want = None
+            for comb in itertools.combinations(range(n), take):
+                inside = [(scores[i], i) for i in comb]
+                outside = [(scores[i], i) for i in range(n) if i not in comb]
+                if all(_better(a, b) for a in inside for b in outside):
+                    assert want is None  # the defining property has one solution
+                    want = list(comb)
+            assert list(idx[:take]) == want
+            assert list(idx[take:]) == [-1] * (k - take)
+            assert np.all(np.diff(idx[:take]) > 0)  # ascending index order
+            assert kth == (min(scores[i] for i in want) if take == k else -math.inf)
+            assert np.array_equal(sel[:take], scores[idx[:take]])
+
+
+def test_topk_ties_prefer_lower_index_and_pad():
+    scores = np.array([5, 7, 7, 7, 1, 7, 0], dtype=np.float64)
+    idx, _, kth = oracle.select_row(scores, 7, 3)
+    assert list(idx) == [1, 2, 3] and kth == 7
+    idx, _, _ = oracle.select_row(scores, 4, 6)  # only 4 visible
+    assert list(idx) == [0, 1, 2, 3, -1, -1]
+
+
+def test_topk_end_to_end_matches_library_sort():
+    rng = np.random.default_rng(12)
+    B, T, L, m, HI, DI, k = 2, 3, 200, 4, 2, 8, 11
+    q, w, kk = _idx_case(rng, B, T, L, m, HI, DI)
+    r = oracle.topk(q, w, kk, None, ctx_len=L, m=m, k=k, want_scores=True)
+    sc = r["scores"]
+    for b, j in itertools.product(range(B), range(T)):
+        t = L - T + j
+        nvis = (t + 1) // m
+        order = sorted(range(nvis), key=lambda s: (-sc[b, j, s], s))[:k]  # library sort
+        assert list(r["idx"][b, j]) == sorted(order) + [-1] * (k - len(order))
+
+
+# ----------------------------------------------------------------------
+# attention
+# ----------------------------------------------------------------------
+
+def _att_case(rng, B, T, L, m, H, d, W, fmt="f32"):
+    q = rng.normal(size=(B, T, H, d)) / math.sqrt(d)
+    ent = rng.normal(size=(B, L // m, d))
+    p0 = max(0, L - T - W + 1)
+    tok = rng.normal(size=(B, L - p0, d))
+    cast = (lambda a: a.astype(np.float32)) if fmt == "f32" else \
+        (lambda a: stored_numpy(torch.from_numpy(a).to(torch.bfloat16)))
+    return cast(q), cast(ent), cast(tok), p0
+
+
+def test_short_context_hca_is_textbook_window_attention():
+    """Context shorter than one HCA chunk: no visible entry, so HCA is plain
+    softmax attention over the window rows (library SDPA in fp64)."""
+    rng = np.random.default_rng(13)
+    for L, W in [(100, 128), (127, 128), (90, 32)]:
+        B, T, H, d = 2, 3, 4, 16
+        q, ent, tok, p0 = _att_case(rng, B, T, max(L, 128), 128, H, d, W)
+        ent = ent[:, : L // 128]
+        tok = rng.normal(size=(B, L - max(0, L - T - W + 1), d)).astype(np.float32)
+        p0 = max(0, L - T - W + 1)
+        out = oracle.attend(q, ent if ent.shape[1] else np.zeros((B, 0, d), np.float32), None, tok, p0, L, 128, W)
+        for j in range(T):
+            t = L - T + j
+            lo = max(0, t - W + 1)
+            rows = torch.from_numpy(tok[:, lo - p0: t - p0 + 1].astype(np.float64))  # [B][n][d]
+            qq = torch.from_numpy(q[:, j].astype(np.float64))[:, :, None, :]  # [B][H][1][d]
+            kv = rows[:, None].expand(B, H, -1, d)
+            ref = torch.nn.functional.scaled_dot_product_attention(qq, kv, kv)[:, :, 0]
+            assert np.allclose(out[:, j], ref.numpy(), atol=1e-12)
+
+
+def test_topk_covering_all_entries_equals_dense():
+    rng = np.random.default_rng(14)
+    B, T, L, m, H, d, W = 2, 5, 64, 4, 3, 8, 8
+    q, ent, tok, p0 = _att_case(rng, B, T, L, m, H, d, W)
+    N = L // m
+    idx = np.full((B, T, N + 3), -1, dtype=np.int32)
+    for j in range(T):
+        nvis = (L - T + j + 1) // m
+        for b in range(B):
+            idx[b, j, :nvis] = rng.permutation(nvis)  # order must not matter
+    sparse = oracle.attend(q, ent, idx, tok, p0, L, m, W)
+    dense = oracle.attend(q, ent, None, tok, p0, L, m, W)
+    assert np.allclose(sparse, dense, atol=1e-12)
+
+
+def test_attention_weights_sum_to_one_and_two_candidate_closed_form():
+    rng = np.random.default_rng(15)
+    B, T, L, m, H, d, W = 1, 2, 48, 4, 2, 8, 4
+    q, ent, tok, p0 = _att_case(rng, B, T, L, m, H, d, W)
+    for j, h in itertools.product(range(T), range(H)):
+        wts = oracle.attend_weights(q, ent, None, tok, p0, L, m, W, 0, j, h)
+        assert wts.shape[0] == (L - T + j + 1) // m + W
+        assert abs(wts.sum() - 1.0) < 1e-12 and (wts > 0).all()
+    # exactly two candidates (context 2, window 2, no entry visible with m = 4):
+    # weight of token 0 = sigmoid((q.x0 - q.x1)/sqrt(d))
+    q2 = rng.normal(size=(1, 1, 1, 8)).astype(np.float32)
+    tok2 = rng.normal(size=(1, 2, 8)).astype(np.float32)
+    ent2 = np.zeros((1, 0, 8), np.float32)
+    wts = oracle.attend_weights(q2, ent2, None, tok2, 0, 2, 4, 2, 0, 0, 0)
+    z = float(np.dot(q2[0, 0, 0].astype(np.float64), tok2[0, 0].astype(np.float64) - tok2[0, 1].astype(np.float64))) / math.sqrt(8)
+    assert wts[0] == pytest.approx(1.0 / (1.0 + math.exp(-z)), abs=1e-14)
+    out = oracle.attend(q2, ent2, None, tok2, 0, 2, 4, 2)
+    assert np.allclose(out[0, 0, 0], wts[0] * tok2[0, 0] + wts[1] * tok2[0, 1], atol=1e-12)
+
+
+def test_single_candidate_returns_that_row_and_duplicates_count_twice():
+    rng = np.random.default_rng(16)
+    d = 16
+    q = rng.normal(size=(1, 1, 2, d)).astype(np.float32)
+    tok = rng.normal(size=(1, 1, d)).astype(np.float32)
+    ent = np.zeros((1, 0, d), np.float32)
+    out = oracle.attend(q, ent, None, tok, 0, 1, 4, 1)  # context of one token, window 1
+    assert np.allclose(out[0, 0], np.broadcast_to(tok[0, 0], (2, d)), atol=1e-15)
+    # a candidate listed twice gets twice the weight: with e = entry 0 listed
+    # twice and the window token once, weight(e) = 2a/(2a+b)
+    ent1 = rng.normal(size=(1, 1, d)).astype(np.float32)
+    tok1 = rng.normal(size=(1, 4, d)).astype(np.float32)
+    idx = np.array([[[0, 0]]], dtype=np.int32)
+    o = oracle.attend(q[:, :, :1], ent1, idx, tok1, 0, 4, 4, 1)
+    a = math.exp(float(np.dot(q[0, 0, 0].astype(np.float64), ent1[0, 0].astype(np.float64))) / math.sqrt(d))
+    bb = math.exp(float(np.dot(q[0, 0, 0].astype(np.float64), tok1[0, 3].astype(np.float64))) / math.sqrt(d))
+    we = 2 * a / (2 * a + bb)
+    assert np.allclose(o[0, 0, 0], we * ent1[0, 0] + (1 - we) * tok1[0, 3], atol=1e-12)
+
+
+def test_visibility_boundary_in_attention():
+    """An entry whose block ends exactly at the query position is attended;
+    the next one (block not yet complete) is not."""
+    d, m = 8, 4
+    q = np.zeros((1, 1, 1, d), np.float32)
+    q[0, 0, 0, 0] = 60.0
+    ent = np.zeros((1, 3, d), np.float32)
+    ent[0, 1, 0] = 10.0  # block [4, 8): visible to t = 7, not to t = 6
+    ent[0, 2, 0] = 20.0  # block [8, 12)
+    tok = np.zeros((1, 12, d), np.float32)
+    o7 = oracle.attend(q, ent, None, tok[:, :8], 0, 8, m, 1)
+    assert o7[0, 0, 0, 0] == pytest.approx(10.0, rel=1e-9)
+    o6 = oracle.attend(q, ent[:, :1], None, tok[:, :7], 0, 7, m, 1)
+    assert o6[0, 0, 0, 0] == pytest.approx(0.0, abs=1e-9)
+    idx = np.array([[[1, 2]]], dtype=np.int32)
+    with pytest.raises(ValueError):
+        oracle.attend(q, ent[:, :2], idx, tok[:, :8], 0, 8, m, 1)  # entry 2 is not visible at t = 7
+
+
+def test_bf16_attention_matches_fp32_of_same_values():
+    rng = np.random.default_rng(17)
+    q, ent, tok, p0 = _att_case(rng, 1, 2, 256, 4, 4, 32, 16, fmt="bf16")
+    o_b = oracle.attend(q, ent, None, tok, p0, 256, 4, 16)
+    f = lambda a: oracle.decode(a).astype(np.float32)
+    o_f = oracle.attend(f(q), f(ent), None, f(tok), p0, 256, 4, 16)
+    assert np.allclose(o_b, o_f, atol=1e-12)
