@@ -1,0 +1,491 @@
+"""Benchmark: one decode step of the hybrid compressed-attention layer pair at
+a 1,048,576-token context on B200.
+
+A step is the whole path for the token at position t = L-1 of every sequence:
+  CSA layer (batch 4, 262,144 entries of d=512 bf16, FP8-e4m3 indexer keys
+  16 x 128 with per-entry scales, top-1024, window 128):
+    compress the chunk completing at t (K=V entry + fp8 indexer key),
+    Lightning-indexer scores + top-k select, sparse attention + split combine;
+  HCA layer (batch 32, 8,192 entries, window 128):
+    compress the 128-token chunk completing at t, dense attention + combine.
+Metric: decode tokens/s per layer = (4 + 32) sequence-layer decodes / step
+time.  The device-side value replays the step as a CUDA graph with every input
+resident in HBM; `e2e` calls the public API eagerly with the step's inputs
+(queries, indexer queries/weights, the new chunk's rows and gates) copied from
+pinned host memory and the attention outputs copied back, every step.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Under torchrun each rank runs its own replica (no data-path collective); the
+step time is the max over ranks and `value` counts every rank's tokens.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+METRIC = "CSA/HCA decode tokens/s per layer at 1M ctx"
+UNIT = "tokens/s"
+WORKLOAD = ("1M-ctx decode step: CSA layer (batch 4, 262,144 entries, fp8 indexer keys, top-1024) + "
+            "HCA layer (batch 32, 8,192 entries), d=512, 64 heads, window 128")
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=400)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=20.0, help="budget of the oracle sample")
+    return p.parse_args()
+
+
+# ----------------------------------------------------------------------
+# distributed plumbing
+# ----------------------------------------------------------------------
+
+def dist_init(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() and args.impl == "ours" else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if dist.get_backend() == "nccl" else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------
+# clocks during the timed region
+# ----------------------------------------------------------------------
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                                          "-i", str(self.gpu), "-lms", "100"], stdout=self.f,
+                                         stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None:
+            return None
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(parts[1]), smax=float(parts[2]), power=float(parts[3]),
+                                 hw=parts[5], hwt=parts[6], swt=parts[7], swp=parts[8]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        reasons = set()
+        for r in rows:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"), ("swt", "sw_thermal_slowdown"),
+                              ("swp", "sw_power_cap")):
+                if r[key].lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in rows), "sm_max_mhz": max(r["smax"] for r in rows),
+                "reasons": sorted(reasons), "samples": len(rows),
+                "power_w_max": max(r["power"] for r in rows)}
+
+
+# ----------------------------------------------------------------------
+# the step
+# ----------------------------------------------------------------------
+
+class Step:
+    """Device buffers and the calls of one decode step (both layers)."""
+
+    def __init__(self, seed_offset: int = 0):
+        import compressed_sparse_long_v4a_b200 as v4a
+        import workload as wl
+
+        self.v4a = v4a
+        cw = wl.csa_decode("csa_l1m_fp8", seed=wl.CONFIGS["csa_l1m_fp8"]["seed"] + seed_offset)
+        hw = wl.hca_decode("hca_l1m", seed=wl.CONFIGS["hca_l1m"]["seed"] + seed_offset)
+        self.cc, self.hc = cw["cfg"], hw["cfg"]
+        dv = lambda t: None if t is None else t.cuda()
+        # CSA layer
+        self.c_q, self.c_tok, self.c_ent = dv(cw["q"]), dv(cw["token_kv"]), dv(cw["entries"])
+        self.c_qi, self.c_w, self.c_ki, self.c_ks = dv(cw["q_i"]), dv(cw["w"]), dv(cw["k_i"]), dv(cw["k_scale"])
+        self.c_gate, self.c_xi, self.c_gi = dv(cw["gate_tail"]), dv(cw["xi_tail"]), dv(cw["gate_i_tail"])
+        self.c_pos0 = cw["tok_pos0"]
+        # HCA layer
+        self.h_q, self.h_tok, self.h_ent, self.h_gate = dv(hw["q"]), dv(hw["token_kv"]), dv(hw["entries"]), \
+            dv(hw["gate_tail"])
+        self.h_pos0 = hw["tok_pos0"]
+        # host copies of the per-step inputs (pinned) for the end-to-end measurement
+        self.host_in = {name: t.pin_memory() for name, t in (
+            ("c_q", cw["q"]), ("c_qi", cw["q_i"]), ("c_w", cw["w"]), ("c_gate", cw["gate_tail"]),
+            ("c_xi", cw["xi_tail"]), ("c_gi", cw["gate_i_tail"]), ("c_newtok", cw["token_kv"][:, -1:].contiguous()),
+            ("h_q", hw["q"]), ("h_gate", hw["gate_tail"]), ("h_newtok", hw["token_kv"][:, -1:].contiguous()))}
+        self.cw_host, self.hw_host = cw, hw
+        c, h = self.cc, self.hc
+        self.Bc, self.Bh = c["batch"], h["batch"]
+        self.Lc, self.Lh = c["ctx_len"], h["ctx_len"]
+        self.Nc, self.Nh = self.Lc // c["m"], self.Lh // h["m"]
+        self.idx = torch.empty((self.Bc, 1, c["k"]), dtype=torch.int32, device="cuda")
+        self.c_out = torch.empty((self.Bc, 1, c["heads"], c["d"]), dtype=torch.float32, device="cuda")
+        self.h_out = torch.empty((self.Bh, 1, h["heads"], h["d"]), dtype=torch.float32, device="cuda")
+        self.status = torch.zeros((1,), dtype=torch.int32, device="cuda")
+        ws = lambda n: torch.empty(max(n, 256), dtype=torch.uint8, device="cuda")
+        self.ws_topk = ws(v4a.v4a_workspace_size("topk", batch=self.Bc, m=c["m"], k=c["k"], ctx_len=self.Lc,
+                                                 heads_i=c["heads_i"], d_i=c["d_i"]))
+        self.ws_csa = ws(v4a.v4a_workspace_size("csa_attend", batch=self.Bc, heads=c["heads"], d=c["d"], m=c["m"],
+                                                k=c["k"], window=c["window"], ctx_len=self.Lc))
+        self.ws_hca = ws(v4a.v4a_workspace_size("hca_attend", batch=self.Bh, heads=h["heads"], d=h["d"], m=h["m"],
+                                                window=h["window"], ctx_len=self.Lh))
+
+    # the four ops -----------------------------------------------------
+    def compress_csa(self):
+        c, m, lt = self.cc, self.cc["m"], self.c_tok.shape[1]
+        self.v4a.v4a_compress(self.c_tok[:, lt - m:], self.c_gate, self.c_ent[:, self.Nc - 1:], m=m,
+                              xi=self.c_xi, gate_i=self.c_gi, out_i=self.c_ki[:, self.Nc - 1:],
+                              out_i_scale=self.c_ks[:, self.Nc - 1:])
+
+    def compress_hca(self):
+        m, lt = self.hc["m"], self.h_tok.shape[1]
+        self.v4a.v4a_compress(self.h_tok[:, lt - m:], self.h_gate, self.h_ent[:, self.Nh - 1:], m=m)
+
+    def topk(self):
+        c = self.cc
+        self.v4a.v4a_topk(self.c_qi, self.c_w, self.c_ki, self.c_ks, self.idx, m=c["m"], k=c["k"], ctx_len=self.Lc,
+                          workspace=self.ws_topk)
+
+    def csa_attend(self):
+        c = self.cc
+        self.v4a.v4a_csa_attend(self.c_q, self.c_ent, self.idx, self.c_tok, self.c_pos0, self.c_out, m=c["m"],
+                                window=c["window"], ctx_len=self.Lc, workspace=self.ws_csa, dev_status=self.status)
+
+    def hca_attend(self):
+        h = self.hc
+        self.v4a.v4a_hca_attend(self.h_q, self.h_ent, self.h_tok, self.h_pos0, self.h_out, m=h["m"],
+                                window=h["window"], ctx_len=self.Lh, workspace=self.ws_hca)
+
+    def run(self):
+        self.compress_csa()
+        self.compress_hca()
+        self.topk()
+        self.csa_attend()
+        self.hca_attend()
+
+    # bytes ------------------------------------------------------------
+    def algorithmic_bytes(self):
+        """Bytes the method must read per step (indexer keys + scales, selected
+        entries + window rows; HCA: every entry + window rows)."""
+        c, h = self.cc, self.hc
+        idx_b = self.Bc * self.Nc * (c["d_i"] * 1 + 4)
+        csa_b = self.Bc * (c["k"] + c["window"]) * c["d"] * 2
+        hca_b = self.Bh * (self.Nh + h["window"]) * h["d"] * 2
+        return dict(topk=idx_b, csa_attend=csa_b, hca_attend=hca_b, total=idx_b + csa_b + hca_b)
+
+    def units(self):
+        return self.Bc + self.Bh
+
+
+def kernel_nodes(graph) -> int | None:
+    """Kernel nodes in a captured graph (cudaGraphGetNodes + cudaGraphNodeGetType)."""
+    try:
+        import ctypes
+
+        import torch.cuda
+        raw = graph.raw_cuda_graph()
+        rt = None
+        for name in ("libcudart.so.12", "libcudart.so"):
+            try:
+                rt = ctypes.CDLL(name)
+                break
+            except OSError:
+                continue
+        if rt is None:
+            return None
+        n = ctypes.c_size_t(0)
+        if rt.cudaGraphGetNodes(ctypes.c_void_p(raw), None, ctypes.byref(n)) != 0:
+            return None
+        nodes = (ctypes.c_void_p * n.value)()
+        if rt.cudaGraphGetNodes(ctypes.c_void_p(raw), nodes, ctypes.byref(n)) != 0:
+            return None
+        kinds = 0
+        for i in range(n.value):
+            t = ctypes.c_int(-1)
+            rt.cudaGraphNodeGetType(ctypes.c_void_p(nodes[i]), ctypes.byref(t))
+            kinds += 1 if t.value == 0 else 0  # cudaGraphNodeTypeKernel
+        return kinds
+    except Exception:
+        return None
+
+
+def time_op(fn, reps: int, flush: torch.Tensor) -> float:
+    """Mean device ms of one call of fn, L2 flushed (memset of a buffer larger
+    than L2) before each timed call, outside its events."""
+    s = torch.cuda.current_stream()
+    evs = []
+    for _ in range(reps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(s)
+        fn()
+        b.record(s)
+        evs.append((a, b))
+    torch.cuda.synchronize()
+    return statistics.mean(a.elapsed_time(b) for a, b in evs)
+
+
+# ----------------------------------------------------------------------
+# CPU oracle (the reference arm and the cpu_baseline object)
+# ----------------------------------------------------------------------
+
+def oracle_sample(budget_s: float, step: "Step | None" = None):
+    """Time the CPU oracle on a bounded sample of the same workload: all 4 CSA
+    sequences (indexer + top-k + attention) and as many HCA sequences as fit the
+    budget.  Returns (tokens/s for the workload's 4:32 mix, threads, sample text)."""
+    import numpy as np
+
+    import oracle
+    import workload as wl
+
+    if step is not None:
+        cw, hw = step.cw_host, step.hw_host
+    else:
+        cw = wl.csa_decode("csa_l1m_fp8", with_tail=False)
+        hw = wl.hca_decode("hca_l1m", with_tail=False)
+    c, h = cw["cfg"], hw["cfg"]
+    h_ = wl.stored_numpy
+    t0 = time.perf_counter()
+    top = oracle.topk(h_(cw["q_i"]), h_(cw["w"]), h_(cw["k_i"]), h_(cw["k_scale"]), c["ctx_len"], c["m"], c["k"])
+    oracle.attend(h_(cw["q"]), h_(cw["entries"]), top["idx"], h_(cw["token_kv"]), cw["tok_pos0"], c["ctx_len"],
+                  c["m"], c["window"])
+    t_csa = (time.perf_counter() - t0) / c["batch"]
+    n_h = 0
+    t1 = time.perf_counter()
+    per = max(1, oracle.get_threads() // 8)
+    while n_h < h["batch"]:
+        bs = list(range(n_h, min(h["batch"], n_h + per)))
+        oracle.attend(h_(hw["q"][bs]), h_(hw["entries"][bs]), None, h_(hw["token_kv"][bs]), hw["tok_pos0"],
+                      h["ctx_len"], h["m"], h["window"])
+        n_h += len(bs)
+        if time.perf_counter() - t1 > budget_s:
+            break
+    t_hca = (time.perf_counter() - t1) / n_h
+    step_s = c["batch"] * t_csa + h["batch"] * t_hca
+    value = (c["batch"] + h["batch"]) / step_s
+    sample = (f"oracle (fp64 C, {oracle.get_threads()} threads) on all {c['batch']} CSA sequences "
+              f"(indexer+top-k+attention) and {n_h} of {h['batch']} HCA sequences; per-sequence times "
+              f"{t_csa:.3f} s (CSA) / {t_hca:.3f} s (HCA) combined in the step's 4:32 mix")
+    return value, oracle.get_threads(), sample, dict(csa_s_per_seq=t_csa, hca_s_per_seq=t_hca, hca_seqs=n_h)
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    import numpy as np  # noqa: F401
+
+    value, threads, sample, detail = oracle_sample(args.cpu_seconds)
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1000.0 * 36 / value, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": WORKLOAD, "parallelism": "replicas", "sample": sample},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------
+# main
+# ----------------------------------------------------------------------
+
+def main():
+    args = parse()
+    world, rank, local = dist_init(args)
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return
+    assert torch.cuda.is_available(), "bench.py needs a CUDA device"
+    args.warmup = max(3, args.warmup)
+    step = Step(seed_offset=rank)
+    s = torch.cuda.current_stream()
+
+    # warm-up (also loads every kernel before capture)
+    for _ in range(args.warmup):
+        step.run()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step.run()
+    for _ in range(args.warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    launches_per_step = kernel_nodes(g)
+
+    # timed region: K graph replays, inputs (416 MB streamed per step) larger than L2
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        for _ in range(args.steps):
+            g.replay()
+        e1.record(s)
+        torch.cuda.synchronize()
+    barrier(world)
+    ms = e0.elapsed_time(e1) / args.steps
+    ms = max_over_ranks(ms, world)
+    units = step.units() * world
+    value = units / (ms / 1000.0)
+
+    # per-op device times (L2 flushed before each), for the roofline of the dominant kernel
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    reps = 20
+    op_ms = {name: time_op(getattr(step, name), reps, flush)
+             for name in ("compress_csa", "compress_hca", "topk", "csa_attend", "hca_attend")}
+    ab = step.algorithmic_bytes()
+    dom = max(("topk", "csa_attend", "hca_attend"), key=lambda n: op_ms[n])
+    peaks = {}
+    try:
+        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+    except Exception:
+        pass
+    peak = float(peaks.get("hbm_gbs", 6650.0))
+    achieved = ab[dom] / (op_ms[dom] / 1000.0) / 1e9
+    traffic = None
+    try:
+        tr = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))
+        traffic = tr.get(dom)
+    except Exception:
+        pass
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "traffic": traffic,
+                "peak_source": "measured" if "hbm_gbs" in peaks else "fallback",
+                "algorithmic_bytes": ab[dom], "ms": op_ms[dom]}
+
+    # end to end through the public API: per-step inputs from pinned host memory, outputs back
+    hin = step.host_in
+    c_out_h = torch.empty(step.c_out.shape, dtype=torch.float32, pin_memory=True)
+    h_out_h = torch.empty(step.h_out.shape, dtype=torch.float32, pin_memory=True)
+    lt_c, lt_h = step.c_tok.shape[1], step.h_tok.shape[1]
+
+    def e2e_step():
+        step.c_q.copy_(hin["c_q"], non_blocking=True)
+        step.c_qi.copy_(hin["c_qi"], non_blocking=True)
+        step.c_w.copy_(hin["c_w"], non_blocking=True)
+        step.c_gate.copy_(hin["c_gate"], non_blocking=True)
+        step.c_xi.copy_(hin["c_xi"], non_blocking=True)
+        step.c_gi.copy_(hin["c_gi"], non_blocking=True)
+        step.c_tok[:, lt_c - 1:].copy_(hin["c_newtok"], non_blocking=True)
+        step.h_q.copy_(hin["h_q"], non_blocking=True)
+        step.h_gate.copy_(hin["h_gate"], non_blocking=True)
+        step.h_tok[:, lt_h - 1:].copy_(hin["h_newtok"], non_blocking=True)
+        step.run()
+        c_out_h.copy_(step.c_out, non_blocking=True)
+        h_out_h.copy_(step.h_out, non_blocking=True)
+
+    h2d = sum(t.numel() * t.element_size() for t in hin.values())
+    d2h = c_out_h.numel() * 4 + h_out_h.numel() * 4
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    e2e_steps = max(20, min(args.steps, 200))
+    barrier(world)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for _ in range(e2e_steps):
+        e2e_step()
+    torch.cuda.synchronize()
+    e2e_s = max_over_ranks((time.perf_counter() - t0) / e2e_steps, world)
+    e2e = {"value": units / e2e_s, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+           "ms_per_step": e2e_s * 1000.0, "how": "eager API calls, pinned copies in, outputs out, host wall clock"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, threads, sample, _ = oracle_sample(args.cpu_seconds, step)
+        cpu = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample}
+
+    clocks = clk.summary()
+    if rank == 0:
+        total_bytes = ab["total"] * world
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": WORKLOAD, "csa": "csa_l1m_fp8", "hca": "hca_l1m",
+                           "parallelism": f"replicas x{world}",
+                           "l2": "inputs larger than L2 (416 MB streamed per step; 126 MB L2)",
+                           "step_algorithmic_bytes": ab["total"],
+                           "step_hbm_gbs": total_bytes / (ms / 1000.0) / 1e9 / world,
+                           "op_ms": op_ms,
+                           "per_layer_tokens_per_s": {"csa": step.Bc / (op_ms["compress_csa"] + op_ms["topk"] +
+                                                                        op_ms["csa_attend"]) * 1000.0,
+                                                      "hca": step.Bh / (op_ms["compress_hca"] +
+                                                                        op_ms["hca_attend"]) * 1000.0}},
+                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": (launches_per_step * args.steps) if launches_per_step else None,
+                "gpu_launches_per_step": launches_per_step,
+                "clocks": clocks}
+        print(json.dumps(line), flush=True)
+    del g
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

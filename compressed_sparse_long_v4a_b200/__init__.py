@@ -1,0 +1,223 @@
+"""Python binding of libv4a.so, the B200 compressed-attention library.
+
+The functions here carry the C ABI's names (``include/v4a.h``) and only
+marshal arguments: they read pointers, sizes and strides off torch tensors,
+pass the current CUDA stream, and raise ``V4AError`` with the library's
+one-line reason when a call returns a non-OK status.  Every step of the
+computation runs in the library's CUDA kernels; there is no other path.  If
+the shared library has not been built, importing this package fails.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "V4AError", "F32", "BF16", "FP8E4M3", "lib", "library_path",
+    "v4a_compress", "v4a_index_scores", "v4a_topk", "v4a_csa_attend", "v4a_hca_attend",
+    "v4a_workspace_size", "v4a_status_string", "v4a_version", "n_entries", "window_rows",
+]
+
+F32, BF16, FP8E4M3 = 0, 1, 2
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libv4a.so")
+
+
+class V4AError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"v4a status {status}: {message}")
+        self.status = status
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int), ("n_q", ctypes.c_int), ("heads", ctypes.c_int), ("d", ctypes.c_int),
+                ("m", ctypes.c_int), ("k", ctypes.c_int), ("window", ctypes.c_int), ("ctx_len", ctypes.c_longlong)]
+
+
+class CompressIO(ctypes.Structure):
+    _fields_ = [("x", ctypes.c_void_p), ("gate", ctypes.c_void_p), ("out", ctypes.c_void_p),
+                ("out_scale", ctypes.c_void_p), ("channels", ctypes.c_int), ("in_dtype", ctypes.c_int),
+                ("out_dtype", ctypes.c_int), ("x_batch_stride", ctypes.c_longlong),
+                ("gate_batch_stride", ctypes.c_longlong), ("out_batch_stride", ctypes.c_longlong),
+                ("scale_batch_stride", ctypes.c_longlong)]
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def _load():
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(f"libv4a.so is not built at {_LIB_PATH}; run __graft_entry__.build() "
+                          "(python -c 'import __graft_entry__ as g; g.build()')")
+    L = ctypes.CDLL(_LIB_PATH)
+    vp, i32, ll, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong, ctypes.c_size_t
+    P = ctypes.POINTER
+    L.v4a_compress.restype = i32
+    L.v4a_compress.argtypes = [P(CompressIO), P(CompressIO), i32, ll, i32, vp]
+    L.v4a_index_scores.restype = i32
+    L.v4a_index_scores.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, P(Shape), vp]
+    L.v4a_topk.restype = i32
+    L.v4a_topk.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, sz, P(Shape), vp]
+    L.v4a_csa_attend.restype = i32
+    L.v4a_csa_attend.argtypes = [vp, vp, vp, vp, ll, ll, vp, i32, vp, sz, vp, P(Shape), vp]
+    L.v4a_hca_attend.restype = i32
+    L.v4a_hca_attend.argtypes = [vp, vp, vp, ll, ll, vp, i32, vp, sz, P(Shape), vp]
+    L.v4a_workspace_size.restype = sz
+    L.v4a_workspace_size.argtypes = [ctypes.c_char_p, P(Shape), i32, i32]
+    L.v4a_status_string.restype = ctypes.c_char_p
+    L.v4a_status_string.argtypes = [i32]
+    L.v4a_last_error.restype = ctypes.c_char_p
+    L.v4a_last_error.argtypes = []
+    L.v4a_version.restype = i32
+    L.v4a_version.argtypes = []
+    return L
+
+
+lib = _load()
+
+
+def _check(status: int) -> None:
+    if status != 0:
+        raise V4AError(status, lib.v4a_last_error().decode() or lib.v4a_status_string(status).decode())
+
+
+def _dtype(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return F32
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype in (torch.uint8, torch.float8_e4m3fn):
+        return FP8E4M3
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libv4a takes CUDA tensors")
+    return t.data_ptr()
+
+
+def _contig(t: torch.Tensor, name: str) -> None:
+    if t is not None and not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def n_entries(ctx_len: int, m: int) -> int:
+    return ctx_len // m
+
+
+def window_rows(ctx_len: int, n_q: int, window: int):
+    """(tok_pos0, l_tok): the token rows that every query's window needs."""
+    p0 = max(0, ctx_len - n_q - window + 1)
+    return p0, ctx_len - p0
+
+
+def _shape(batch=0, n_q=1, heads=0, d=0, m=1, k=0, window=0, ctx_len=1) -> Shape:
+    return Shape(int(batch), int(n_q), int(heads), int(d), int(m), int(k), int(window), int(ctx_len))
+
+
+def v4a_workspace_size(op: str, *, batch, n_q=1, heads=0, d=0, m=1, k=0, window=0, ctx_len=1, heads_i=0,
+                       d_i=0) -> int:
+    s = _shape(batch, n_q, heads, d, m, k, window, ctx_len)
+    return int(lib.v4a_workspace_size(op.encode(), ctypes.byref(s), int(heads_i), int(d_i)))
+
+
+def v4a_status_string(status: int) -> str:
+    return lib.v4a_status_string(int(status)).decode()
+
+
+def v4a_version() -> int:
+    return int(lib.v4a_version())
+
+
+def _workspace(nbytes: int, device) -> torch.Tensor:
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def _io(x, gate, out, out_scale) -> CompressIO:
+    for t, name in ((x, "x"), (gate, "gate"), (out, "out")):
+        if t.dim() != 3 or t.stride(2) != 1 or t.stride(1) != t.shape[2]:
+            raise ValueError(f"{name} must be [batch][rows][channels] with dense rows")
+    sc_stride = 0
+    if out_scale is not None:
+        if out_scale.dim() != 2 or out_scale.stride(1) != 1:
+            raise ValueError("out_scale must be [batch][entries] with dense rows")
+        sc_stride = out_scale.stride(0)
+    return CompressIO(_ptr(x), _ptr(gate), _ptr(out), _ptr(out_scale), int(x.shape[2]), _dtype(x), _dtype(out),
+                      x.stride(0), gate.stride(0), out.stride(0), sc_stride)
+
+
+def v4a_compress(x, gate, out, *, m: int, n_tok: int | None = None, out_scale=None, xi=None, gate_i=None,
+                 out_i=None, out_i_scale=None, stream=None) -> None:
+    """Compress complete m-token chunks of x (gated by `gate`) into `out`;
+    optionally the indexer-key stream (xi, gate_i -> out_i [, out_i_scale]) in
+    the same launch.  Tensors are [batch][rows][channels] (views into larger
+    buffers are fine: the batch stride is read off the tensor)."""
+    n = x.shape[1] if n_tok is None else int(n_tok)
+    kv = _io(x, gate, out, out_scale)
+    idx = None
+    if xi is not None:
+        idx = _io(xi, gate_i, out_i, out_i_scale)
+    _check(lib.v4a_compress(ctypes.byref(kv), ctypes.byref(idx) if idx is not None else None, int(x.shape[0]), n,
+                            int(m), _stream(stream)))
+
+
+def v4a_index_scores(q_i, w, k_i, k_scale, scores, *, m: int, ctx_len: int, stream=None) -> None:
+    for t, n in ((q_i, "q_i"), (w, "w"), (k_i, "k_i"), (k_scale, "k_scale"), (scores, "scores")):
+        _contig(t, n)
+    B, T, HI, DI = q_i.shape
+    s = _shape(batch=B, n_q=T, m=m, ctx_len=ctx_len)
+    _check(lib.v4a_index_scores(_ptr(q_i), _ptr(w), _ptr(k_i), _ptr(k_scale), _ptr(scores), HI, DI, _dtype(q_i),
+                                _dtype(k_i), ctypes.byref(s), _stream(stream)))
+
+
+def v4a_topk(q_i, w, k_i, k_scale, idx_out, score_out=None, *, m: int, k: int, ctx_len: int, workspace=None,
+             stream=None) -> None:
+    for t, n in ((q_i, "q_i"), (w, "w"), (k_i, "k_i"), (k_scale, "k_scale"), (idx_out, "idx_out"),
+                 (score_out, "score_out")):
+        _contig(t, n)
+    B, T, HI, DI = q_i.shape
+    s = _shape(batch=B, n_q=T, m=m, k=k, ctx_len=ctx_len)
+    if workspace is None:
+        workspace = _workspace(lib.v4a_workspace_size(b"topk", ctypes.byref(s), HI, DI), q_i.device)
+    _check(lib.v4a_topk(_ptr(q_i), _ptr(w), _ptr(k_i), _ptr(k_scale), _ptr(idx_out), _ptr(score_out), HI, DI,
+                        _dtype(q_i), _dtype(k_i), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                        ctypes.byref(s), _stream(stream)))
+
+
+def v4a_csa_attend(q, entries, idx, token_kv, tok_pos0: int, out, *, m: int, window: int, ctx_len: int,
+                   workspace=None, dev_status=None, stream=None) -> None:
+    for t, n in ((q, "q"), (entries, "entries"), (idx, "idx"), (token_kv, "token_kv"), (out, "out")):
+        _contig(t, n)
+    B, T, H, d = q.shape
+    s = _shape(batch=B, n_q=T, heads=H, d=d, m=m, k=idx.shape[-1], window=window, ctx_len=ctx_len)
+    if workspace is None:
+        workspace = _workspace(lib.v4a_workspace_size(b"csa_attend", ctypes.byref(s), 0, 0), q.device)
+    _check(lib.v4a_csa_attend(_ptr(q), _ptr(entries), _ptr(idx), _ptr(token_kv), int(tok_pos0),
+                              int(token_kv.shape[1]), _ptr(out), _dtype(q), _ptr(workspace),
+                              workspace.numel() * workspace.element_size(), _ptr(dev_status), ctypes.byref(s),
+                              _stream(stream)))
+
+
+def v4a_hca_attend(q, entries, token_kv, tok_pos0: int, out, *, m: int, window: int, ctx_len: int, workspace=None,
+                   stream=None) -> None:
+    for t, n in ((q, "q"), (entries, "entries"), (token_kv, "token_kv"), (out, "out")):
+        _contig(t, n)
+    B, T, H, d = q.shape
+    s = _shape(batch=B, n_q=T, heads=H, d=d, m=m, window=window, ctx_len=ctx_len)
+    if workspace is None:
+        workspace = _workspace(lib.v4a_workspace_size(b"hca_attend", ctypes.byref(s), 0, 0), q.device)
+    _check(lib.v4a_hca_attend(_ptr(q), _ptr(entries), _ptr(token_kv), int(tok_pos0), int(token_kv.shape[1]),
+                              _ptr(out), _dtype(q), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                              ctypes.byref(s), _stream(stream)))

@@ -1,0 +1,128 @@
+// common.cuh -- device helpers shared by the libv4a kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "v4a.h"
+
+namespace v4a {
+
+constexpr int kNumSMs = 148;  // B200: two dies of 74 SMs
+
+// ---------------------------------------------------------------------
+// element loads: 8 consecutive elements (16 bytes of bf16, 32 of fp32)
+// ---------------------------------------------------------------------
+
+__device__ __forceinline__ float bf16_bits_to_float(uint32_t h16) { return __uint_as_float(h16 << 16); }
+
+__device__ __forceinline__ void unpack_bf16x8(const uint4& v, float f[8]) {
+    f[0] = __uint_as_float(v.x << 16);
+    f[1] = __uint_as_float(v.x & 0xffff0000u);
+    f[2] = __uint_as_float(v.y << 16);
+    f[3] = __uint_as_float(v.y & 0xffff0000u);
+    f[4] = __uint_as_float(v.z << 16);
+    f[5] = __uint_as_float(v.z & 0xffff0000u);
+    f[6] = __uint_as_float(v.w << 16);
+    f[7] = __uint_as_float(v.w & 0xffff0000u);
+}
+
+template <typename T>
+struct Vec8;
+
+template <>
+struct Vec8<float> {
+    static __device__ __forceinline__ void load(const float* p, float f[8]) {
+        float4 a = *reinterpret_cast<const float4*>(p);
+        float4 b = *reinterpret_cast<const float4*>(p + 4);
+        f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+        f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+    }
+    static __device__ __forceinline__ void load_nc(const float* p, float f[8]) {
+        float4 a = __ldg(reinterpret_cast<const float4*>(p));
+        float4 b = __ldg(reinterpret_cast<const float4*>(p + 4));
+        f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+        f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+    }
+    static __device__ __forceinline__ void store(float* p, const float f[8]) {
+        *reinterpret_cast<float4*>(p) = make_float4(f[0], f[1], f[2], f[3]);
+        *reinterpret_cast<float4*>(p + 4) = make_float4(f[4], f[5], f[6], f[7]);
+    }
+};
+
+template <>
+struct Vec8<__nv_bfloat16> {
+    static __device__ __forceinline__ void load(const __nv_bfloat16* p, float f[8]) {
+        uint4 v = *reinterpret_cast<const uint4*>(p);
+        unpack_bf16x8(v, f);
+    }
+    static __device__ __forceinline__ void load_nc(const __nv_bfloat16* p, float f[8]) {
+        uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
+        unpack_bf16x8(v, f);
+    }
+    static __device__ __forceinline__ void store(__nv_bfloat16* p, const float f[8]) {
+        __nv_bfloat162 h[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+        *reinterpret_cast<uint4*>(p) = *reinterpret_cast<uint4*>(h);
+    }
+};
+
+// 8 e4m3 codes (8 bytes) -> 8 floats (exact: every e4m3 value is a float)
+__device__ __forceinline__ void unpack_e4m3x8(const uint2& v, float f[8]) {
+    const uint32_t w[2] = {v.x, v.y};
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[i] & 0xffffu), __NV_E4M3);
+        __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[i] >> 16), __NV_E4M3);
+        float2 a = __half22float2(*reinterpret_cast<__half2*>(&lo));
+        float2 b = __half22float2(*reinterpret_cast<__half2*>(&hi));
+        f[4 * i + 0] = a.x;
+        f[4 * i + 1] = a.y;
+        f[4 * i + 2] = b.x;
+        f[4 * i + 3] = b.y;
+    }
+}
+
+// two floats -> two e4m3 codes (round to nearest even, saturate to +-448)
+__device__ __forceinline__ uint16_t pack_e4m3x2(float a, float b) {
+    return (uint16_t)__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+}
+
+// ---------------------------------------------------------------------
+// order-preserving float -> uint32 (larger float -> larger key); -0 == +0
+// ---------------------------------------------------------------------
+__device__ __forceinline__ uint32_t float_to_ordered(float f) {
+    f += 0.0f;  // -0 -> +0
+    uint32_t u = __float_as_uint(f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float ordered_to_float(uint32_t k) {
+    uint32_t u = (k & 0x80000000u) ? (k & 0x7fffffffu) : ~k;
+    return __uint_as_float(u);
+}
+
+// ---------------------------------------------------------------------
+// warp reductions
+// ---------------------------------------------------------------------
+template <int WIDTH>
+__device__ __forceinline__ float group_max(float v) {
+#pragma unroll
+    for (int o = WIDTH / 2; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+template <int WIDTH>
+__device__ __forceinline__ float group_sum(float v) {
+#pragma unroll
+    for (int o = WIDTH / 2; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+__host__ __device__ __forceinline__ long long n_visible(long long t, int m) { return (t + 1) / m; }
+
+}  // namespace v4a

@@ -1,0 +1,142 @@
+// compress.cu -- chunk compression of token rows into compressed entries.
+//
+// "DeepSeek-V4 的暗线之一：分层记忆比输入框更关键" (blog.xieydd.top), section 3:
+// an entry is the per-channel softmax (over the chunk's m tokens, from the gate
+// logits Z) weighted sum of the content rows C.  One launch compresses both the
+// K=V stream and, optionally, the indexer-key stream of the same chunks.
+//
+// Mapping: one thread owns 8 consecutive channels of one entry and streams the
+// chunk's m tokens with 16-byte vector loads (two for fp32), keeping a running
+// max / denominator / numerator per channel in registers (online softmax).
+// The threads of one entry are consecutive lanes of one warp, so an FP8 output
+// finds the entry's amax with warp shuffles.
+#include "common.cuh"
+#include "internal.h"
+
+namespace v4a {
+namespace {
+
+struct StreamDesc {
+    const void* x;
+    const void* gate;
+    void* out;
+    float* out_scale;
+    int channels, groups;  // groups = channels / 8
+    int in_dtype, out_dtype;
+    long long x_bs, gate_bs, out_bs, scale_bs;
+};
+
+template <typename T>
+__device__ __forceinline__ void compress_group(const StreamDesc& d, int b, long long s, int grp, int m,
+                                               float out[8]) {
+    const T* xp = static_cast<const T*>(d.x) + (long long)b * d.x_bs + s * m * d.channels + grp * 8;
+    const T* zp = static_cast<const T*>(d.gate) + (long long)b * d.gate_bs + s * m * d.channels + grp * 8;
+    float mx[8], den[8], num[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        mx[e] = -INFINITY;
+        den[e] = 0.f;
+        num[e] = 0.f;
+    }
+    for (int i = 0; i < m; ++i) {
+        float xv[8], zv[8];
+        Vec8<T>::load_nc(xp + (long long)i * d.channels, xv);
+        Vec8<T>::load_nc(zp + (long long)i * d.channels, zv);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            float nm = fmaxf(mx[e], zv[e]);
+            float a = expf(mx[e] - nm);  // rescale of what was accumulated so far
+            float p = expf(zv[e] - nm);
+            den[e] = den[e] * a + p;
+            num[e] = num[e] * a + p * xv[e];
+            mx[e] = nm;
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) out[e] = num[e] / den[e];
+}
+
+__global__ void __launch_bounds__(256) compress_kernel(StreamDesc s0, StreamDesc s1, int batch, long long n_ent,
+                                                       int m) {
+    const StreamDesc& d = blockIdx.y == 0 ? s0 : s1;
+    long long total = (long long)batch * n_ent * d.groups;
+    long long g = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    bool active = g < total;
+    long long gg = active ? g : 0;
+    int b = (int)(gg / (n_ent * d.groups));
+    long long rem = gg % (n_ent * d.groups);
+    long long s = rem / d.groups;
+    int grp = (int)(rem % d.groups);
+
+    float out[8];
+    if (active) {
+        if (d.in_dtype == V4A_BF16)
+            compress_group<__nv_bfloat16>(d, b, s, grp, m, out);
+        else
+            compress_group<float>(d, b, s, grp, m, out);
+    } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) out[e] = 0.f;
+    }
+
+    if (d.out_dtype == V4A_FP8E4M3) {
+        // per-entry amax over the entry's `groups` consecutive lanes (a power of two <= 32)
+        float a = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) a = fmaxf(a, fabsf(out[e]));
+        for (int o = d.groups / 2; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+        if (!active) return;
+        float scale = a > 0.f ? a / 448.0f : 1.0f;
+        uint8_t* op = static_cast<uint8_t*>(d.out) + (long long)b * d.out_bs + s * d.channels + grp * 8;
+        uint32_t lo = (uint32_t)pack_e4m3x2(out[0] / scale, out[1] / scale) |
+                      ((uint32_t)pack_e4m3x2(out[2] / scale, out[3] / scale) << 16);
+        uint32_t hi = (uint32_t)pack_e4m3x2(out[4] / scale, out[5] / scale) |
+                      ((uint32_t)pack_e4m3x2(out[6] / scale, out[7] / scale) << 16);
+        *reinterpret_cast<uint2*>(op) = make_uint2(lo, hi);
+        if (grp == 0) d.out_scale[(long long)b * d.scale_bs + s] = scale;
+        return;
+    }
+    if (!active) return;
+    if (d.out_dtype == V4A_BF16) {
+        __nv_bfloat16* op = static_cast<__nv_bfloat16*>(d.out) + (long long)b * d.out_bs + s * d.channels + grp * 8;
+        Vec8<__nv_bfloat16>::store(op, out);
+    } else {
+        float* op = static_cast<float*>(d.out) + (long long)b * d.out_bs + s * d.channels + grp * 8;
+        Vec8<float>::store(op, out);
+    }
+}
+
+StreamDesc describe(const v4a_compress_io* io) {
+    StreamDesc d;
+    d.x = io->x;
+    d.gate = io->gate;
+    d.out = io->out;
+    d.out_scale = io->out_scale;
+    d.channels = io->channels;
+    d.groups = io->channels / 8;
+    d.in_dtype = io->in_dtype;
+    d.out_dtype = io->out_dtype;
+    d.x_bs = io->x_batch_stride;
+    d.gate_bs = io->gate_batch_stride;
+    d.out_bs = io->out_batch_stride;
+    d.scale_bs = io->scale_batch_stride;
+    return d;
+}
+
+}  // namespace
+
+cudaError_t launch_compress(const v4a_compress_io* kv, const v4a_compress_io* idx, int batch, long long n_tok,
+                            int m, cudaStream_t stream) {
+    long long n_ent = n_tok / m;
+    if (batch == 0 || n_ent == 0) return cudaSuccess;
+    StreamDesc s0 = describe(kv);
+    StreamDesc s1 = idx ? describe(idx) : s0;
+    long long groups = s0.groups > s1.groups ? s0.groups : s1.groups;
+    long long total = (long long)batch * n_ent * groups;
+    const int threads = 256;
+    dim3 grid((unsigned)((total + threads - 1) / threads), idx ? 2 : 1);
+    compress_kernel<<<grid, threads, 0, stream>>>(s0, s1, batch, n_ent, m);
+    return cudaGetLastError();
+}
+
+}  // namespace v4a

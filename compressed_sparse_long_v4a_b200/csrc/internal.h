@@ -1,0 +1,50 @@
+// internal.h -- host-side launchers behind the C ABI (not exported).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "v4a.h"
+
+namespace v4a {
+
+// ---- compress.cu ------------------------------------------------------
+cudaError_t launch_compress(const v4a_compress_io* kv, const v4a_compress_io* idx, int batch, long long n_tok,
+                            int m, cudaStream_t stream);
+
+// ---- indexer.cu -------------------------------------------------------
+struct IndexArgs {
+    const void* q;        // [B][n_q][HI][DI]
+    const float* w;       // [B][n_q][HI]
+    const void* k;        // [B][N][DI]
+    const float* kscale;  // [B][N] or null
+    v4a_dtype q_dtype, k_dtype;
+    int batch, n_q, m, heads_i, d_i;
+    long long ctx_len, n_ent;
+};
+
+// every score (-inf where not visible) into scores[row][N], row = b*n_q + j
+cudaError_t launch_index_scores(const IndexArgs& a, float* scores, cudaStream_t stream);
+size_t topk_workspace_bytes(const IndexArgs& a, int k);
+cudaError_t launch_topk(const IndexArgs& a, int k, int32_t* idx_out, float* score_out, void* ws, size_t ws_bytes,
+                        cudaStream_t stream);
+
+// ---- attend.cu --------------------------------------------------------
+struct AttendArgs {
+    const void* q;         // [B][n_q][H][d]
+    const void* entries;   // [B][N][d]
+    const int32_t* idx;    // [B][n_q][k] (CSA) or null (HCA: every visible entry)
+    const void* token_kv;  // [B][l_tok][d]
+    long long tok_pos0, l_tok;
+    float* out;            // [B][n_q][H][d]
+    v4a_dtype dtype;
+    int batch, n_q, heads, d, m, k, window;
+    long long ctx_len, n_ent;
+    int* dev_status;
+};
+
+size_t attend_workspace_bytes(const AttendArgs& a);
+cudaError_t launch_attend(const AttendArgs& a, void* ws, size_t ws_bytes, cudaStream_t stream);
+
+}  // namespace v4a

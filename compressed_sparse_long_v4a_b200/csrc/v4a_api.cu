@@ -1,0 +1,265 @@
+// v4a_api.cu -- the exported C ABI: argument checks, then the launchers.
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+v4a_status fail(v4a_status st, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+v4a_status from_cuda(cudaError_t e, const char* what) {
+    if (e == cudaSuccess) return V4A_OK;
+    return fail(V4A_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t dtype_size(v4a_dtype t) { return t == V4A_F32 ? 4 : t == V4A_BF16 ? 2 : 1; }
+
+v4a_status check_compress_io(const v4a_compress_io* io, const char* name, long long n_tok, int m) {
+    if (!io->x || !io->gate || !io->out) return fail(V4A_ERR_INVALID_ARG, "%s: x, gate and out are required", name);
+    if (io->channels < 8 || io->channels % 8) return fail(V4A_ERR_INVALID_ARG, "%s: channels must be a multiple of 8", name);
+    if (io->in_dtype != V4A_F32 && io->in_dtype != V4A_BF16)
+        return fail(V4A_ERR_UNSUPPORTED, "%s: input dtype must be F32 or BF16", name);
+    if (io->out_dtype != V4A_F32 && io->out_dtype != V4A_BF16 && io->out_dtype != V4A_FP8E4M3)
+        return fail(V4A_ERR_UNSUPPORTED, "%s: unknown output dtype", name);
+    if (io->out_dtype == V4A_FP8E4M3) {
+        int g = io->channels / 8;
+        if (!io->out_scale) return fail(V4A_ERR_INVALID_ARG, "%s: FP8E4M3 output needs out_scale", name);
+        if (g > 32 || (g & (g - 1))) return fail(V4A_ERR_UNSUPPORTED, "%s: FP8E4M3 output needs channels/8 a power of two <= 32", name);
+        if (!aligned(io->out_scale, 4)) return fail(V4A_ERR_INVALID_ARG, "%s: out_scale misaligned", name);
+    }
+    long long n_ent = n_tok / m;
+    if (io->x_batch_stride < n_tok * io->channels || io->gate_batch_stride < n_tok * io->channels ||
+        io->out_batch_stride < n_ent * io->channels || (io->out_scale && io->scale_batch_stride < n_ent))
+        return fail(V4A_ERR_INVALID_ARG, "%s: a batch stride is smaller than one sequence", name);
+    size_t in_sz = dtype_size(io->in_dtype), out_sz = dtype_size(io->out_dtype);
+    size_t out_al = out_sz == 1 ? 8 : 16;
+    if (!aligned(io->x, 16) || !aligned(io->gate, 16) || !aligned(io->out, out_al) ||
+        (io->x_batch_stride * in_sz) % 16 || (io->gate_batch_stride * in_sz) % 16 ||
+        (io->out_batch_stride * out_sz) % out_al)
+        return fail(V4A_ERR_INVALID_ARG, "%s: x/gate/out or their strides are not 16-byte aligned", name);
+    return V4A_OK;
+}
+
+v4a_status check_shape_common(const v4a_shape* s) {
+    if (!s) return fail(V4A_ERR_INVALID_ARG, "shape is NULL");
+    if (s->batch < 0 || s->n_q < 1 || s->m < 1 || s->ctx_len < 1)
+        return fail(V4A_ERR_INVALID_ARG, "need batch >= 0, n_q >= 1, m >= 1, ctx_len >= 1");
+    if (s->n_q > s->ctx_len) return fail(V4A_ERR_INVALID_ARG, "n_q > ctx_len");
+    if (s->ctx_len / s->m > 0x7fffffffLL) return fail(V4A_ERR_INVALID_ARG, "too many entries for int32 indices");
+    if ((long long)s->batch * s->n_q > 65535) return fail(V4A_ERR_UNSUPPORTED, "batch * n_q must be <= 65535");
+    return V4A_OK;
+}
+
+v4a_status index_args(const void* q_i, const float* w, const void* k_i, const float* k_scale, int heads_i, int d_i,
+                      v4a_dtype q_dt, v4a_dtype k_dt, const v4a_shape* s, v4a::IndexArgs* a) {
+    v4a_status st = check_shape_common(s);
+    if (st != V4A_OK) return st;
+    if (!q_i || !w || (!k_i && s->ctx_len / s->m > 0)) return fail(V4A_ERR_INVALID_ARG, "q_i, w and k_i are required");
+    if (heads_i < 1 || heads_i > 64) return fail(V4A_ERR_UNSUPPORTED, "heads_i must be in 1..64");
+    if (d_i < 8 || d_i % 8 || d_i > 1024) return fail(V4A_ERR_INVALID_ARG, "d_i must be a multiple of 8 (<= 1024)");
+    if ((long long)heads_i * d_i > 32768) return fail(V4A_ERR_UNSUPPORTED, "heads_i * d_i must be <= 32768");
+    if (q_dt != V4A_F32 && q_dt != V4A_BF16) return fail(V4A_ERR_UNSUPPORTED, "q_i dtype must be F32 or BF16");
+    if (k_dt != V4A_F32 && k_dt != V4A_BF16 && k_dt != V4A_FP8E4M3)
+        return fail(V4A_ERR_UNSUPPORTED, "k_i dtype must be F32, BF16 or FP8E4M3");
+    if (k_dt == V4A_FP8E4M3 && !k_scale) return fail(V4A_ERR_INVALID_ARG, "FP8E4M3 keys need k_scale");
+    if (!aligned(k_i, 16) || !aligned(q_i, 16) || !aligned(w, 4))
+        return fail(V4A_ERR_INVALID_ARG, "q_i/k_i must be 16-byte aligned");
+    a->q = q_i;
+    a->w = w;
+    a->k = k_i;
+    a->kscale = k_scale;
+    a->q_dtype = q_dt;
+    a->k_dtype = k_dt;
+    a->batch = s->batch;
+    a->n_q = s->n_q;
+    a->m = s->m;
+    a->heads_i = heads_i;
+    a->d_i = d_i;
+    a->ctx_len = s->ctx_len;
+    a->n_ent = s->ctx_len / s->m;
+    return V4A_OK;
+}
+
+v4a_status attend_args(const void* q, const void* entries, const int32_t* idx, const void* token_kv,
+                       long long tok_pos0, long long l_tok, float* out, v4a_dtype dt, int* dev_status,
+                       const v4a_shape* s, bool csa, v4a::AttendArgs* a) {
+    v4a_status st = check_shape_common(s);
+    if (st != V4A_OK) return st;
+    if (!q || !out) return fail(V4A_ERR_INVALID_ARG, "q and out are required");
+    if (!entries && s->ctx_len / s->m > 0) return fail(V4A_ERR_INVALID_ARG, "entries is required");
+    if (csa && !idx) return fail(V4A_ERR_INVALID_ARG, "idx is required");
+    if (csa && (s->k < 1 || s->k > 65536)) return fail(V4A_ERR_INVALID_ARG, "k must be in 1..65536");
+    if (s->heads < 1) return fail(V4A_ERR_INVALID_ARG, "heads must be >= 1");
+    if (s->d != 64 && s->d != 128 && s->d != 256 && s->d != 512)
+        return fail(V4A_ERR_UNSUPPORTED, "d must be 64, 128, 256 or 512");
+    if (s->window < 0) return fail(V4A_ERR_INVALID_ARG, "window must be >= 0");
+    if (dt != V4A_F32 && dt != V4A_BF16) return fail(V4A_ERR_UNSUPPORTED, "dtype must be F32 or BF16");
+    if (s->window > 0) {
+        if (!token_kv) return fail(V4A_ERR_INVALID_ARG, "token_kv is required when window > 0");
+        long long lo = s->ctx_len - s->n_q - s->window + 1;
+        if (lo < 0) lo = 0;
+        if (tok_pos0 > lo || tok_pos0 < 0 || tok_pos0 + l_tok < s->ctx_len)
+            return fail(V4A_ERR_INVALID_ARG, "token_kv rows [%lld, %lld) do not cover the windows [%lld, %lld)",
+                        tok_pos0, tok_pos0 + l_tok, lo, s->ctx_len);
+    }
+    if (!aligned(q, 16) || !aligned(entries, 16) || !aligned(token_kv, 16) || !aligned(out, 16) ||
+        (idx && !aligned(idx, 4)))
+        return fail(V4A_ERR_INVALID_ARG, "q/entries/token_kv/out must be 16-byte aligned");
+    a->q = q;
+    a->entries = entries;
+    a->idx = csa ? idx : nullptr;
+    a->token_kv = token_kv;
+    a->tok_pos0 = tok_pos0;
+    a->l_tok = l_tok;
+    a->out = out;
+    a->dtype = dt;
+    a->batch = s->batch;
+    a->n_q = s->n_q;
+    a->heads = s->heads;
+    a->d = s->d;
+    a->m = s->m;
+    a->k = csa ? s->k : 0;
+    a->window = s->window;
+    a->ctx_len = s->ctx_len;
+    a->n_ent = s->ctx_len / s->m;
+    a->dev_status = dev_status;
+    return V4A_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+v4a_status v4a_compress(const v4a_compress_io* kv, const v4a_compress_io* idx, int batch, long long n_tok, int m,
+                        void* stream) {
+    if (!kv) return fail(V4A_ERR_INVALID_ARG, "kv stream is NULL");
+    if (batch < 0 || n_tok < 0 || m < 1) return fail(V4A_ERR_INVALID_ARG, "need batch >= 0, n_tok >= 0, m >= 1");
+    v4a_status st = check_compress_io(kv, "kv", n_tok, m);
+    if (st != V4A_OK) return st;
+    if (idx) {
+        st = check_compress_io(idx, "idx", n_tok, m);
+        if (st != V4A_OK) return st;
+    }
+    return from_cuda(v4a::launch_compress(kv, idx, batch, n_tok, m, (cudaStream_t)stream), "v4a_compress");
+}
+
+v4a_status v4a_index_scores(const void* q_i, const float* w, const void* k_i, const float* k_scale, float* scores,
+                            int heads_i, int d_i, v4a_dtype q_dtype, v4a_dtype k_dtype, const v4a_shape* shape,
+                            void* stream) {
+    v4a::IndexArgs a;
+    v4a_status st = index_args(q_i, w, k_i, k_scale, heads_i, d_i, q_dtype, k_dtype, shape, &a);
+    if (st != V4A_OK) return st;
+    if (!scores && a.n_ent > 0) return fail(V4A_ERR_INVALID_ARG, "scores is required");
+    return from_cuda(v4a::launch_index_scores(a, scores, (cudaStream_t)stream), "v4a_index_scores");
+}
+
+v4a_status v4a_topk(const void* q_i, const float* w, const void* k_i, const float* k_scale, int32_t* idx_out,
+                    float* score_out, int heads_i, int d_i, v4a_dtype q_dtype, v4a_dtype k_dtype, void* workspace,
+                    size_t workspace_bytes, const v4a_shape* shape, void* stream) {
+    v4a::IndexArgs a;
+    v4a_status st = index_args(q_i, w, k_i, k_scale, heads_i, d_i, q_dtype, k_dtype, shape, &a);
+    if (st != V4A_OK) return st;
+    if (shape->k < 1 || shape->k > 4096) return fail(V4A_ERR_INVALID_ARG, "k must be in 1..4096");
+    if (!idx_out) return fail(V4A_ERR_INVALID_ARG, "idx_out is required");
+    size_t need = v4a::topk_workspace_bytes(a, shape->k);
+    if (!workspace || workspace_bytes < need)
+        return fail(V4A_ERR_INVALID_ARG, "workspace of %zu bytes needed, %zu given", need, workspace_bytes);
+    if (!aligned(workspace, 256)) return fail(V4A_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    return from_cuda(v4a::launch_topk(a, shape->k, idx_out, score_out, workspace, workspace_bytes,
+                                      (cudaStream_t)stream),
+                     "v4a_topk");
+}
+
+static v4a_status attend_common(const void* q, const void* entries, const int32_t* idx, const void* token_kv,
+                                long long tok_pos0, long long l_tok, float* out, v4a_dtype dtype, void* workspace,
+                                size_t workspace_bytes, int* dev_status, const v4a_shape* shape, void* stream,
+                                bool csa) {
+    v4a::AttendArgs a;
+    v4a_status st = attend_args(q, entries, idx, token_kv, tok_pos0, l_tok, out, dtype, dev_status, shape, csa, &a);
+    if (st != V4A_OK) return st;
+    size_t need = v4a::attend_workspace_bytes(a);
+    if (!workspace || workspace_bytes < need)
+        return fail(V4A_ERR_INVALID_ARG, "workspace of %zu bytes needed, %zu given", need, workspace_bytes);
+    if (!aligned(workspace, 256)) return fail(V4A_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    if (dev_status) {
+        cudaError_t e = cudaMemsetAsync(dev_status, 0, sizeof(int), (cudaStream_t)stream);
+        if (e != cudaSuccess) return from_cuda(e, "dev_status reset");
+    }
+    return from_cuda(v4a::launch_attend(a, workspace, workspace_bytes, (cudaStream_t)stream),
+                     csa ? "v4a_csa_attend" : "v4a_hca_attend");
+}
+
+v4a_status v4a_csa_attend(const void* q, const void* entries, const int32_t* idx, const void* token_kv,
+                          long long tok_pos0, long long l_tok, float* out, v4a_dtype dtype, void* workspace,
+                          size_t workspace_bytes, int* dev_status, const v4a_shape* shape, void* stream) {
+    return attend_common(q, entries, idx, token_kv, tok_pos0, l_tok, out, dtype, workspace, workspace_bytes,
+                         dev_status, shape, stream, true);
+}
+
+v4a_status v4a_hca_attend(const void* q, const void* entries, const void* token_kv, long long tok_pos0,
+                          long long l_tok, float* out, v4a_dtype dtype, void* workspace, size_t workspace_bytes,
+                          const v4a_shape* shape, void* stream) {
+    return attend_common(q, entries, nullptr, token_kv, tok_pos0, l_tok, out, dtype, workspace, workspace_bytes,
+                         nullptr, shape, stream, false);
+}
+
+size_t v4a_workspace_size(const char* op, const v4a_shape* shape, int heads_i, int d_i) {
+    if (!op || !shape) return 0;
+    if (strcmp(op, "topk") == 0) {
+        v4a::IndexArgs a = {};
+        a.batch = shape->batch;
+        a.n_q = shape->n_q;
+        a.m = shape->m > 0 ? shape->m : 1;
+        a.heads_i = heads_i;
+        a.d_i = d_i;
+        a.ctx_len = shape->ctx_len;
+        a.n_ent = shape->ctx_len / a.m;
+        return v4a::topk_workspace_bytes(a, shape->k);
+    }
+    bool csa = strcmp(op, "csa_attend") == 0;
+    if (csa || strcmp(op, "hca_attend") == 0) {
+        v4a::AttendArgs a = {};
+        a.batch = shape->batch;
+        a.n_q = shape->n_q;
+        a.heads = shape->heads > 0 ? shape->heads : 1;
+        a.d = shape->d >= 64 ? shape->d : 64;
+        a.m = shape->m > 0 ? shape->m : 1;
+        a.k = csa ? shape->k : 0;
+        a.window = shape->window;
+        a.ctx_len = shape->ctx_len;
+        a.n_ent = shape->ctx_len / a.m;
+        a.idx = csa ? reinterpret_cast<const int32_t*>(1) : nullptr;
+        return v4a::attend_workspace_bytes(a);
+    }
+    return 0;
+}
+
+const char* v4a_status_string(v4a_status st) {
+    switch (st) {
+    case V4A_OK: return "ok";
+    case V4A_ERR_INVALID_ARG: return "invalid argument";
+    case V4A_ERR_UNSUPPORTED: return "unsupported combination";
+    case V4A_ERR_CUDA: return "CUDA error";
+    case V4A_ERR_DEVICE_FAULT: return "device fault (bad data found by a kernel)";
+    default: return "unknown status";
+    }
+}
+
+const char* v4a_last_error(void) { return g_last_error; }
+
+int v4a_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,208 @@
+/*
+ * v4a.h -- C ABI of libv4a.so: the compressed-attention step of DeepSeek-V4
+ * (CSA = compressed sparse attention, HCA = heavily compressed attention,
+ * plus the raw sliding window) as hand-written CUDA kernels for sm_100a.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Pointers named in the argument lists are DEVICE pointers unless said
+ *    otherwise.  The caller owns every buffer; the library never allocates,
+ *    frees or synchronises.  Scratch memory ("workspace") is passed in; its
+ *    size comes from v4a_workspace_size().
+ *  - Every call only enqueues work on `stream` (a cudaStream_t; NULL is the
+ *    legacy default stream) and returns V4A_OK once the work is enqueued.
+ *    Argument errors are found on the host, before anything is enqueued, and
+ *    return V4A_ERR_INVALID_ARG or V4A_ERR_UNSUPPORTED; v4a_last_error()
+ *    then holds a one-line reason (per host thread).  A failed launch returns
+ *    V4A_ERR_CUDA.  Kernels never trap: data-dependent faults (an index out of
+ *    range) are skipped and reported through a device status word.
+ *  - Layouts are dense and row-major, innermost dimension last.  Sizes are in
+ *    elements unless they say bytes.
+ *  - Positions.  A sequence's context holds ctx_len tokens (positions
+ *    0 .. ctx_len-1).  The n_q query tokens are the LAST n_q positions,
+ *    t = ctx_len - n_q + j for query j (decode: n_q = 1, t = ctx_len - 1).
+ *  - Compressed entries.  With compression rate m, entry s summarises tokens
+ *    [m*s, m*s + m) and every sequence holds N = floor(ctx_len / m) entries
+ *    (only complete chunks are compressed).  Entry s is visible to query
+ *    position t iff m*(s+1) <= t+1, i.e. N_vis(t) = floor((t+1)/m): a query
+ *    never reads its own incomplete block ("1M Context != Lossless Long
+ *    Memory", section 6.1).
+ *  - Sliding window.  Query t also attends to the raw tokens (t-W, t],
+ *    clipped at 0 (same page, section 6; W = n_win = 128 in V4).  Window rows
+ *    come from a token_kv buffer [batch][l_tok][d] whose row r holds position
+ *    tok_pos0 + r; it must cover every query's window.
+ *  - K = V.  One compressed vector per entry (and one vector per window
+ *    token) serves as key and value for every query head ("DeepSeek-V4:
+ *    Million-Token Context via Hybrid Compressed Attention", CSA "Core
+ *    attention with shared KV MQA").
+ */
+#ifndef V4A_H
+#define V4A_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define V4A_API __attribute__((visibility("default")))
+#else
+#define V4A_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum v4a_status {
+    V4A_OK = 0,
+    V4A_ERR_INVALID_ARG = 1,  /* a pointer, size or layout the call cannot take */
+    V4A_ERR_UNSUPPORTED = 2,  /* a valid combination this build has no kernel for */
+    V4A_ERR_CUDA = 3,         /* the CUDA runtime refused a launch */
+    V4A_ERR_DEVICE_FAULT = 4  /* written to a device status word: bad data found by a kernel */
+} v4a_status;
+
+typedef enum v4a_dtype {
+    V4A_F32 = 0,      /* IEEE binary32 */
+    V4A_BF16 = 1,     /* bfloat16 */
+    V4A_FP8E4M3 = 2   /* float8 e4m3 ("fn": no inf, max 448), with one fp32 scale per row */
+} v4a_dtype;
+
+/* Problem shape.  Fields an entry point does not use are ignored. */
+typedef struct v4a_shape {
+    int batch;          /* B: independent sequences */
+    int n_q;            /* T: query tokens per sequence (the last T positions) */
+    int heads;          /* H: attention query heads */
+    int d;              /* K = V vector dimension */
+    int m;              /* compression rate (4 for CSA, 128 for HCA) */
+    int k;              /* top-k: entries selected per query (CSA) */
+    int window;         /* W: sliding-window length (0 = no window) */
+    long long ctx_len;  /* L: tokens in each sequence's context */
+} v4a_shape;
+
+/* ------------------------------------------------------------------ */
+/* compression                                                          */
+/* ------------------------------------------------------------------ */
+
+/* One stream of token rows to compress.  Rows are `channels` wide; row 0 of
+ * x and gate is the first token of the first chunk, row 0 of out the entry it
+ * produces.  Each sequence's rows start *_batch_stride elements apart. */
+typedef struct v4a_compress_io {
+    const void* x;                /* content rows [batch][n_tok][channels], in_dtype */
+    const void* gate;             /* gate logits, same shape, in_dtype */
+    void* out;                    /* entries [batch][n_tok/m][channels], out_dtype */
+    float* out_scale;             /* [batch][n_tok/m] per-entry scale; required iff out_dtype == FP8E4M3 */
+    int channels;                 /* multiple of 8; <= 256 for FP8E4M3 output */
+    v4a_dtype in_dtype;           /* F32 or BF16 */
+    v4a_dtype out_dtype;          /* F32, BF16 or FP8E4M3 */
+    long long x_batch_stride;     /* elements between sequences in x (>= n_tok*channels) */
+    long long gate_batch_stride;  /* elements between sequences in gate */
+    long long out_batch_stride;   /* elements between sequences in out */
+    long long scale_batch_stride; /* floats between sequences in out_scale */
+} v4a_compress_io;
+
+/* Chunk compression ("DeepSeek-V4 的暗线之一：分层记忆比输入框更关键",
+ * section 3; "DeepSeek-V4: Million-Token Context ...", HCA "How it works"):
+ * for every complete chunk s of m tokens and every channel c,
+ *     out[s][c] = sum_{i<m} softmax_i(gate[m*s+i][c]) * x[m*s+i][c],
+ * the softmax running over the chunk's tokens separately for each channel.
+ * The same single-series rule serves m = 4 (CSA) and m' = 128 (HCA).
+ * FP8E4M3 output stores, per entry, scale = amax/448 (1 for an all-zero
+ * entry) in out_scale and each value as the nearest e4m3 code of
+ * value/scale (ties to even, saturating).
+ * kv: the K=V stream (required).  idx: the indexer-key stream compressed in
+ * the same launch (may be NULL); it uses the same batch, n_tok and m.
+ * n_tok: tokens per sequence; a trailing partial chunk is ignored.
+ * Errors: V4A_ERR_INVALID_ARG for a NULL required pointer, m < 1, n_tok < 0,
+ * channels not a multiple of 8, strides too small, misaligned pointers
+ * (x/gate/out need 16-byte alignment); V4A_ERR_UNSUPPORTED for other dtype
+ * combinations. */
+V4A_API v4a_status v4a_compress(const v4a_compress_io* kv, const v4a_compress_io* idx, int batch, long long n_tok, int m,
+                        void* stream);
+
+/* ------------------------------------------------------------------ */
+/* Lightning indexer and top-k                                          */
+/* ------------------------------------------------------------------ */
+
+/* Indexer scores ("How V4 makes a million-token context actually
+ * affordable", Lightning-Indexer section):
+ *     I(t,s) = scale[s] * sum_{j<heads_i} w[j] * ReLU(q_i[j] . k_i[s]),
+ * for every entry s < N_vis(t); -inf for entries not yet visible.
+ * q_i: [batch][n_q][heads_i][d_i] (q_dtype F32 or BF16);
+ * w:   [batch][n_q][heads_i] fp32;
+ * k_i: [batch][N][d_i], N = ctx_len/m (k_dtype F32, BF16 or FP8E4M3);
+ * k_scale: [batch][N] fp32, required for FP8E4M3 keys, else NULL (= 1);
+ * scores: [batch][n_q][N] fp32 output.
+ * Uses shape->batch, n_q, m, ctx_len.  This entry point materialises every
+ * score and exists for inspection and tests; v4a_topk never does. */
+V4A_API v4a_status v4a_index_scores(const void* q_i, const float* w, const void* k_i, const float* k_scale, float* scores,
+                            int heads_i, int d_i, v4a_dtype q_dtype, v4a_dtype k_dtype, const v4a_shape* shape,
+                            void* stream);
+
+/* Indexer + top-k select ("1M Context != Lossless Long Memory", section
+ * 4.2: the query attends only to the k best-scoring entries).  For each
+ * query, the min(k, N_vis) visible entries with the largest I(t,s), ties
+ * going to the lower entry index, are written to idx_out [batch][n_q][k]
+ * (int32) in ASCENDING entry order, padded with -1.  score_out (nullable)
+ * [batch][n_q][k] receives each selected entry's fp32 score (-inf for
+ * padding).  Arguments as v4a_index_scores; workspace of
+ * v4a_workspace_size("topk", shape, heads_i, d_i) bytes.  Uses
+ * shape->batch, n_q, m, k, ctx_len.  Errors: k < 1 or k > 4096. */
+V4A_API v4a_status v4a_topk(const void* q_i, const float* w, const void* k_i, const float* k_scale, int32_t* idx_out,
+                    float* score_out, int heads_i, int d_i, v4a_dtype q_dtype, v4a_dtype k_dtype, void* workspace,
+                    size_t workspace_bytes, const v4a_shape* shape, void* stream);
+
+/* ------------------------------------------------------------------ */
+/* attention                                                            */
+/* ------------------------------------------------------------------ */
+
+/* CSA attention: for every query (b, j) at position t and head h,
+ *     out[h] = sum_r p_r * v_r,  p = softmax_r(q[h] . v_r / sqrt(d)),
+ * one joint softmax over the candidate rows v_r = the selected entries
+ * entries[idx[b][j][i]] (every idx >= 0; a value listed twice is two
+ * candidates) and the window tokens (t-W, t].  The window may repeat tokens an entry already
+ * summarises; both stay.  An empty candidate set yields zeros.
+ * q: [batch][n_q][heads][d]; entries: [batch][N][d], N = ctx_len/m;
+ * idx: [batch][n_q][k] int32, -1 = empty slot; token_kv: [batch][l_tok][d],
+ * row r = position tok_pos0 + r; q/entries/token_kv share dtype (F32 or
+ * BF16); out: [batch][n_q][heads][d] fp32.
+ * dev_status (nullable, device int): set to V4A_OK by the call, and to
+ * V4A_ERR_DEVICE_FAULT by the kernels if an idx entry is neither -1 nor a
+ * visible entry; such slots are skipped.  Workspace:
+ * v4a_workspace_size("csa_attend", shape, 0, 0) bytes.
+ * Uses every shape field.  Errors: d not a multiple of 64 or > 512, a window
+ * not covered by token_kv. */
+V4A_API v4a_status v4a_csa_attend(const void* q, const void* entries, const int32_t* idx, const void* token_kv,
+                          long long tok_pos0, long long l_tok, float* out, v4a_dtype dtype, void* workspace,
+                          size_t workspace_bytes, int* dev_status, const v4a_shape* shape, void* stream);
+
+/* HCA attention ("1M Context != Lossless Long Memory", section 5; "How V4
+ * makes ...", CSA-vs-HCA table: no selection, dense over every entry): as
+ * v4a_csa_attend with the candidate rows = every visible entry s < N_vis(t)
+ * plus the window.  Uses shape->batch, n_q, heads, d, m, window, ctx_len;
+ * workspace of v4a_workspace_size("hca_attend", shape, 0, 0) bytes. */
+V4A_API v4a_status v4a_hca_attend(const void* q, const void* entries, const void* token_kv, long long tok_pos0,
+                          long long l_tok, float* out, v4a_dtype dtype, void* workspace, size_t workspace_bytes,
+                          const v4a_shape* shape, void* stream);
+
+/* ------------------------------------------------------------------ */
+/* housekeeping                                                         */
+/* ------------------------------------------------------------------ */
+
+/* Bytes of device workspace an op needs for this shape: op is "topk",
+ * "csa_attend" or "hca_attend" (0 for anything else).  heads_i/d_i are the
+ * indexer's (used by "topk"). */
+V4A_API size_t v4a_workspace_size(const char* op, const v4a_shape* shape, int heads_i, int d_i);
+
+/* Static description of a status code. */
+V4A_API const char* v4a_status_string(v4a_status status);
+
+/* The reason for the last non-OK status returned on this host thread. */
+V4A_API const char* v4a_last_error(void);
+
+/* Library version: major*10000 + minor*100 + patch. */
+V4A_API int v4a_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* V4A_H */
