@@ -147,6 +147,7 @@ v4a_status v4a_compress(const v4a_compress_io* kv, const v4a_compress_io* idx, i
                         void* stream) {
     if (!kv) return fail(V4A_ERR_INVALID_ARG, "kv stream is NULL");
     if (batch < 0 || n_tok < 0 || m < 1) return fail(V4A_ERR_INVALID_ARG, "need batch >= 0, n_tok >= 0, m >= 1");
+    if (batch == 0 || n_tok / m == 0) return V4A_OK;  // no complete chunk: nothing to write
     v4a_status st = check_compress_io(kv, "kv", n_tok, m);
     if (st != V4A_OK) return st;
     if (idx) {
