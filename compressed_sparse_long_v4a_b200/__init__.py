@@ -16,7 +16,7 @@ import torch
 
 __all__ = [
     "V4AError", "F32", "BF16", "FP8E4M3", "lib", "library_path",
-    "v4a_compress", "v4a_index_scores", "v4a_topk", "v4a_csa_attend", "v4a_hca_attend",
+    "v4a_compress", "v4a_index_scores", "v4a_topk", "v4a_topk_noalloc", "v4a_csa_attend", "v4a_hca_attend",
     "v4a_workspace_size", "v4a_status_string", "v4a_version", "n_entries", "window_rows",
 ]
 
@@ -61,6 +61,8 @@ def _load():
     L.v4a_index_scores.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, P(Shape), vp]
     L.v4a_topk.restype = i32
     L.v4a_topk.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, sz, P(Shape), vp]
+    L.v4a_topk_noalloc.restype = i32
+    L.v4a_topk_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, P(Shape), vp]
     L.v4a_csa_attend.restype = i32
     L.v4a_csa_attend.argtypes = [vp, vp, vp, vp, ll, ll, vp, i32, vp, sz, vp, P(Shape), vp]
     L.v4a_hca_attend.restype = i32
@@ -194,6 +196,19 @@ def v4a_topk(q_i, w, k_i, k_scale, idx_out, score_out=None, *, m: int, k: int, c
     _check(lib.v4a_topk(_ptr(q_i), _ptr(w), _ptr(k_i), _ptr(k_scale), _ptr(idx_out), _ptr(score_out), HI, DI,
                         _dtype(q_i), _dtype(k_i), _ptr(workspace), workspace.numel() * workspace.element_size(),
                         ctypes.byref(s), _stream(stream)))
+
+
+def v4a_topk_noalloc(q_i, w, k_i, k_scale, idx_out, score_out=None, *, m: int, k: int, ctx_len: int,
+                     stream=None) -> None:
+    """v4a_topk with the library's built-in scratch: no workspace argument and
+    no device allocation (see include/v4a.h for the size limit)."""
+    for t, n in ((q_i, "q_i"), (w, "w"), (k_i, "k_i"), (k_scale, "k_scale"), (idx_out, "idx_out"),
+                 (score_out, "score_out")):
+        _contig(t, n)
+    B, T, HI, DI = q_i.shape
+    s = _shape(batch=B, n_q=T, m=m, k=k, ctx_len=ctx_len)
+    _check(lib.v4a_topk_noalloc(_ptr(q_i), _ptr(w), _ptr(k_i), _ptr(k_scale), _ptr(idx_out), _ptr(score_out), HI,
+                                DI, _dtype(q_i), _dtype(k_i), ctypes.byref(s), _stream(stream)))
 
 
 def v4a_csa_attend(q, entries, idx, token_kv, tok_pos0: int, out, *, m: int, window: int, ctx_len: int,

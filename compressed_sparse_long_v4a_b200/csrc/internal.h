@@ -9,6 +9,9 @@
 
 namespace v4a {
 
+// Record a one-line reason for v4a_last_error() and return st.
+v4a_status report(v4a_status st, const char* fmt, ...);
+
 // ---- compress.cu ------------------------------------------------------
 cudaError_t launch_compress(const v4a_compress_io* kv, const v4a_compress_io* idx, int batch, long long n_tok,
                             int m, cudaStream_t stream);

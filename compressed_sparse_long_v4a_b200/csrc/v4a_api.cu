@@ -141,6 +141,14 @@ v4a_status attend_args(const void* q, const void* entries, const int32_t* idx, c
 
 }  // namespace
 
+v4a_status v4a::report(v4a_status st, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+    va_end(ap);
+    return st;
+}
+
 extern "C" {
 
 v4a_status v4a_compress(const v4a_compress_io* kv, const v4a_compress_io* idx, int batch, long long n_tok, int m,

@@ -150,6 +150,30 @@ V4A_API v4a_status v4a_topk(const void* q_i, const float* w, const void* k_i, co
                     float* score_out, int heads_i, int d_i, v4a_dtype q_dtype, v4a_dtype k_dtype, void* workspace,
                     size_t workspace_bytes, const v4a_shape* shape, void* stream);
 
+/* The same operation as v4a_topk for callers that cannot allocate device
+ * memory: a plug-in inside a host framework that owns every device
+ * allocation, or a serving loop where allocating is not allowed.  (The pages
+ * have no counterpart: this is an interface convenience, not part of the
+ * method.)  Arguments, results and errors are those of v4a_topk, except that
+ * there is no workspace argument: the scratch is a fixed 16 MiB array
+ * compiled into the library, which every device that loads the library keeps
+ * in its global memory until the process exits.  It bounds the problem size:
+ * batch * n_q * (ctx_len / m) must not exceed 4,194,304 (the 1M-context
+ * decode of 4 sequences needs 1,048,576); larger shapes return
+ * V4A_ERR_INVALID_ARG with the limit in v4a_last_error().
+ * The first call made with a given device current looks up the array's
+ * device address (cudaGetSymbolAddress) and caches it; make that first call
+ * outside any stream capture.  The call itself allocates nothing: no
+ * cudaMalloc, no cudaFree, no allocating library routine.
+ * Every call on a device uses the same array, and the array keeps whatever
+ * the previous call left in it (each call writes every scratch byte before
+ * reading it).  Calls whose work may overlap on the GPU -- on different
+ * streams, or from several host threads without ordering -- race on the
+ * array and must be serialised by the caller. */
+V4A_API v4a_status v4a_topk_noalloc(const void* q_i, const float* w, const void* k_i, const float* k_scale,
+                                    int32_t* idx_out, float* score_out, int heads_i, int d_i, v4a_dtype q_dtype,
+                                    v4a_dtype k_dtype, const v4a_shape* shape, void* stream);
+
 /* ------------------------------------------------------------------ */
 /* attention                                                            */
 /* ------------------------------------------------------------------ */
