@@ -270,7 +270,7 @@ cudaError_t launch_dtype(const AttendArgs& a, const SplitPlan& plan, float* ml, 
 
 }  // namespace
 
-size_t attend_workspace_bytes(const AttendArgs& a) {
+static size_t core_workspace_bytes(const AttendArgs& a) {
     SplitPlan p = plan_for(a);
     if (p.n_splits == 1) return 256;
     size_t rows = (size_t)a.batch * a.n_q;
@@ -279,9 +279,19 @@ size_t attend_workspace_bytes(const AttendArgs& a) {
     return ml + n * a.d * sizeof(float);
 }
 
+size_t attend_workspace_bytes(const AttendArgs& a) {
+    size_t w = core_workspace_bytes(a);
+    if (attend_tc_shape_ok(a)) {
+        size_t t = attend_tc_workspace_bytes(a);
+        if (t > w) w = t;
+    }
+    return w;
+}
+
 cudaError_t launch_attend(const AttendArgs& a, void* ws, size_t ws_bytes, cudaStream_t stream) {
     if (a.batch == 0) return cudaSuccess;
     if (ws_bytes < attend_workspace_bytes(a)) return cudaErrorInvalidValue;
+    if (attend_tc_available(a)) return launch_attend_tc(a, ws, ws_bytes, stream);
     SplitPlan plan = plan_for(a);
     size_t rows = (size_t)a.batch * a.n_q;
     size_t n = rows * plan.n_splits * a.heads;

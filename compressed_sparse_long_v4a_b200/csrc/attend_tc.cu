@@ -1,0 +1,614 @@
+// attend_tc.cu -- tensor-core (tcgen05 / TMEM / TMA) CSA and HCA attention
+// for the 64-head, d = 512, bf16 shape of DeepSeek-V4's compressed layers.
+//
+// What it computes is the joint softmax of attend.cu: for query (b, j) at
+// position t and head h, softmax_r(q_h . v_r / sqrt(d)) over the candidate
+// rows (selected or all visible compressed entries, then the window tokens
+// (t-W, t]), times the same rows ("DeepSeek-V4: Million-Token Context via
+// Hybrid Compressed Attention", CSA "Core attention with shared KV MQA").
+//
+// Shape of the work.  One query has 64 heads sharing every K=V row, so per
+// 64-row tile of candidates:
+//   S  = Q K^T      tcgen05 M=64 (heads) x N=64 (rows) x K=512, Q and K in smem
+//   P  = softmax(S) (online, one thread per head)
+//   O^T += V^T P^T  tcgen05 M=128 (d chunk) x N=64 (heads) x K=64 (rows),
+//                   four d chunks, V^T read MN-major from the same smem tile
+// The accumulator O^T (512 x 64 fp32) and two S buffers live in TMEM.
+//
+// Work split: the candidate tiles of all queries form one flat sequence that
+// is cut into `grid` contiguous ranges, one per CTA (one CTA per SM).  A CTA
+// whose range covers a query's tiles completely writes that query's output;
+// a query cut between CTAs gets one partial (m, l, O) per piece, merged by
+// attend_tc_combine.  Per CTA: warp 0 loads (TMA for contiguous rows and the
+// query, cp.async gathers for CSA-selected rows) into a 2-stage ring, warp 1
+// issues the MMAs, warps 2-5 run the softmax and the output.  Every wait is
+// bounded; on a time-out the CTA records a device fault, poisons its outputs
+// with NaN and winds down.
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "tc.cuh"
+
+namespace v4a {
+namespace {
+
+constexpr int kD = 512;
+constexpr int kH = 64;
+constexpr int kTile = 64;                        // candidate rows per tile
+constexpr int kSlabs = kD / 64;                  // 64-element (128 B) column slabs
+constexpr uint32_t kSlabBytes = kTile * 128;     // 8 KB
+constexpr uint32_t kTileBytes = kSlabs * kSlabBytes;
+constexpr uint32_t kQBytes = kSlabs * kH * 128;  // 64 KB
+constexpr uint32_t kPBytes = kH * 128;           // 64 heads x 64 rows bf16
+constexpr uint32_t kColO = 0;                    // O^T: 4 chunks of 64 columns
+constexpr uint32_t kColS = 256;                  // S: 2 buffers of 64 columns
+constexpr uint32_t kTmemCols = 512;
+constexpr int kThreads = 192;
+constexpr float kRescaleSlack = 8.0f;  // keep a stale running max until the true one exceeds it by 2^8
+
+constexpr uint32_t kIdescQK = tc::idesc_f16(64, 64, 0, 0);
+constexpr uint32_t kIdescPV = tc::idesc_f16(128, 64, 1, 0);
+
+struct __align__(1024) Smem {
+    uint8_t q[kQBytes];
+    uint8_t kv[2][kTileBytes];
+    uint8_t p[2][kPBytes];
+    uint64_t kv_full[2], kv_empty[2], s_full[2], p_full[2], p_free[2];
+    uint64_t q_full, q_empty, drain;
+    uint64_t mask[2];
+    float alpha[2][kH], l_s[kH], m_s[kH];  // alpha / rescale_tag by tile parity
+    int rescale_tag[2];
+    int abort_flag;
+    uint32_t tmem_base;
+};
+
+struct TcArgs {
+    const __nv_bfloat16* q;
+    const __nv_bfloat16* entries;
+    const __nv_bfloat16* token_kv;
+    const int32_t* idx;  // CSA selections, or null for HCA
+    float* out;
+    float* part_ml;      // [2*grid][64][2]
+    float* part_o;       // [2*grid][64][512]
+    int* dev_status;
+    long long n_ent, l_tok, tok_pos0, ctx_len, total_tiles;
+    int rows, n_q, m, k, window;
+    int e_tiles, w_tiles, tpr, grid;
+    float scale_log2;
+};
+
+__device__ __forceinline__ long long range_start(int c, const TcArgs& a) {
+    return (long long)c * a.total_tiles / a.grid;
+}
+
+struct RowInfo {
+    int b;
+    long long t, nvis;
+};
+
+__device__ __forceinline__ RowInfo row_info(int row, const TcArgs& a) {
+    RowInfo r;
+    r.b = row / a.n_q;
+    const int j = row % a.n_q;
+    r.t = a.ctx_len - a.n_q + j;
+    r.nvis = n_visible(r.t, a.m);
+    if (r.nvis > a.n_ent) r.nvis = a.n_ent;
+    return r;
+}
+
+__device__ __forceinline__ void fault(Smem& sm, const TcArgs& a) {
+    sm.abort_flag = 1;
+    if (a.dev_status) atomicExch(a.dev_status, (int)V4A_ERR_DEVICE_FAULT);
+}
+
+// ---------------------------------------------------------------------
+// warp 0: loads
+// ---------------------------------------------------------------------
+__device__ void producer(Smem& sm, const TcArgs& a, const CUtensorMap* ent_map, const CUtensorMap* tok_map,
+                         const CUtensorMap* q_map, long long f0, long long f1) {
+    const int lane = threadIdx.x & 31;
+    int seg = 0;
+    for (long long f = f0; f < f1; ++f) {
+        if (sm.abort_flag) break;
+        const int jt = (int)(f - f0), s = jt & 1;
+        const int row = (int)(f / a.tpr), ti = (int)(f % a.tpr);
+        const bool seg_start = (f == f0) || (ti == 0);
+        const RowInfo ri = row_info(row, a);
+        if (seg_start) {
+            if (seg > 0 && !tc::mbar_wait(&sm.q_empty, (seg - 1) & 1)) { fault(sm, a); break; }
+            if (lane == 0) {
+                tc::mbar_arrive_expect_tx(&sm.q_full, kQBytes);
+                for (int c = 0; c < kSlabs; ++c) tc::tma_load_2d(sm.q + c * kH * 128, q_map, 64 * c, row * kH, &sm.q_full);
+            }
+            ++seg;
+        }
+        if (jt >= 2 && !tc::mbar_wait(&sm.kv_empty[s], ((jt >> 1) - 1) & 1)) { fault(sm, a); break; }
+        uint64_t mask = 0;
+        uint8_t* dst = sm.kv[s];
+        if (ti < a.e_tiles) {
+            const long long c0 = (long long)ti * kTile;
+            if (!a.idx) {
+                // HCA: rows c0..c0+63 of this sequence's entries are contiguous
+                const long long nv = ri.nvis - c0;
+                mask = nv >= 64 ? ~0ull : (nv <= 0 ? 0ull : ((1ull << nv) - 1));
+                if (lane == 0) {
+                    sm.mask[s] = mask;
+                    tc::mbar_arrive_expect_tx(&sm.kv_full[s], kTileBytes);
+                    const int y = (int)((long long)ri.b * a.n_ent + c0);
+                    for (int c = 0; c < kSlabs; ++c) tc::tma_load_2d(dst + c * kSlabBytes, ent_map, 64 * c, y, &sm.kv_full[s]);
+                }
+            } else {
+                // CSA: gather the selected rows with cp.async (128-byte swizzle written by hand)
+                const __nv_bfloat16* src[2];
+                bool ok[2];
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    const long long c = c0 + lane + 32 * h2;
+                    long long sidx = c < a.k ? (long long)a.idx[(long long)row * a.k + c] : -1;
+                    ok[h2] = sidx >= 0 && sidx < ri.nvis;
+                    if (!ok[h2] && sidx != -1 && a.dev_status) atomicExch(a.dev_status, (int)V4A_ERR_DEVICE_FAULT);
+                    // an excluded row still gets finite data: this query's head-0 row of q
+                    src[h2] = ok[h2] ? a.entries + ((long long)ri.b * a.n_ent + sidx) * kD
+                                     : a.q + (long long)row * kH * kD;
+                }
+                const uint32_t lo = __ballot_sync(0xffffffffu, ok[0]);
+                const uint32_t hi = __ballot_sync(0xffffffffu, ok[1]);
+                mask = (uint64_t)lo | ((uint64_t)hi << 32);
+                for (int r = 0; r < kTile; ++r) {
+                    const __nv_bfloat16* rs = (const __nv_bfloat16*)__shfl_sync(
+                        0xffffffffu, (unsigned long long)(r < 32 ? src[0] : src[1]), r & 31);
+#pragma unroll
+                    for (int h2 = 0; h2 < 2; ++h2) {
+                        const int u = lane + 32 * h2;  // 16-byte chunk of the 1 KB row
+                        uint8_t* d = dst + (u >> 3) * kSlabBytes + r * 128 + (((u & 7) ^ (r & 7)) << 4);
+                        tc::cp_async_16(d, rs + u * 8);
+                    }
+                }
+                if (lane == 0) {
+                    sm.mask[s] = mask;
+                    tc::mbar_arrive_expect_tx(&sm.kv_full[s], 0);
+                }
+            }
+        } else {
+            // window tokens p0 .. p0+63 (contiguous rows of token_kv)
+            const long long wi = ti - a.e_tiles;
+            const long long p0 = ri.t - a.window + 1 + wi * kTile;
+            for (int r = 0; r < kTile; ++r) {
+                const long long p = p0 + r;
+                if (wi * kTile + r < a.window && p >= 0) mask |= 1ull << r;
+            }
+            if (lane == 0) {
+                sm.mask[s] = mask;
+                tc::mbar_arrive_expect_tx(&sm.kv_full[s], kTileBytes);
+                const int y = (int)((long long)ri.b * a.l_tok + (p0 - a.tok_pos0));
+                for (int c = 0; c < kSlabs; ++c) tc::tma_load_2d(dst + c * kSlabBytes, tok_map, 64 * c, y, &sm.kv_full[s]);
+            }
+        }
+        tc::cp_async_arrive_noinc(&sm.kv_full[s]);  // 32 lanes: after their cp.async copies (if any) land
+    }
+    // make sure nothing this warp started is still in flight before the CTA retires
+    const long long n = f1 - f0;
+    for (long long jt = n - 2; jt < n; ++jt) {
+        if (jt < 0) continue;
+        tc::mbar_wait(&sm.kv_full[jt & 1], (jt >> 1) & 1);
+    }
+    if (seg > 0) tc::mbar_wait(&sm.q_full, (seg - 1) & 1);
+}
+
+// ---------------------------------------------------------------------
+// warp 1: MMA issue (one thread)
+// ---------------------------------------------------------------------
+__device__ bool issue_pv(Smem& sm, uint32_t tmem, int jp, bool first_in_seg) {
+    const int sp = jp & 1;
+    if (!tc::mbar_wait(&sm.p_full[sp], (jp >> 1) & 1)) return false;
+    tc::tc_fence_after();
+    const uint32_t kv = tc::smem_u32(sm.kv[sp]);
+    const uint32_t pb = tc::smem_u32(sm.p[sp]);
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) {
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk) {
+            // A = V^T (M = 128 d of slabs 2cc, 2cc+1; K = 16 rows), MN-major
+            const uint64_t ad = tc::sw128_desc(kv + (2 * cc) * kSlabBytes + kk * 2048, kSlabBytes, 1024);
+            // B = P^T (N = 64 heads, K = 16 rows), K-major rows of P
+            const uint64_t bd = tc::sw128_desc(pb + kk * 32, 16, 1024);
+            tc::mma_f16(tmem + kColO + 64 * cc, ad, bd, kIdescPV, (!first_in_seg || kk > 0) ? 1u : 0u);
+        }
+    }
+    tc::mma_commit(&sm.kv_empty[sp]);
+    tc::mma_commit(&sm.p_free[sp]);
+    return true;
+}
+
+__device__ void mma_issuer(Smem& sm, const TcArgs& a, uint32_t tmem, long long f0, long long f1) {
+    int seg = 0;
+    bool ok = true;
+    bool prev_first = false;  // whether the pending PV tile starts its segment
+    for (long long f = f0; f < f1 && ok; ++f) {
+        if (sm.abort_flag) { ok = false; break; }
+        const int jt = (int)(f - f0), s = jt & 1;
+        const int ti = (int)(f % a.tpr);
+        const bool seg_start = (f == f0) || (ti == 0);
+        const bool seg_end = (f == f1 - 1) || (ti == a.tpr - 1);
+        if (seg_start && jt > 0) {
+            if (!issue_pv(sm, tmem, jt - 1, prev_first)) { ok = false; break; }
+        }
+        if (seg_start) {
+            if (!tc::mbar_wait(&sm.q_full, seg & 1)) { ok = false; break; }
+            ++seg;
+        }
+        if (!tc::mbar_wait(&sm.kv_full[s], (jt >> 1) & 1)) { ok = false; break; }
+        tc::fence_proxy_async();  // rows gathered with cp.async become visible to the tensor core
+        tc::tc_fence_after();
+        const uint32_t qb = tc::smem_u32(sm.q);
+        const uint32_t kb = tc::smem_u32(sm.kv[s]);
+#pragma unroll 1
+        for (int c = 0; c < kSlabs; ++c) {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t ad = tc::sw128_desc(qb + c * kH * 128 + kk * 32, 16, 1024);
+                const uint64_t bd = tc::sw128_desc(kb + c * kSlabBytes + kk * 32, 16, 1024);
+                tc::mma_f16(tmem + kColS + 64 * s, ad, bd, kIdescQK, (c | kk) ? 1u : 0u);
+            }
+        }
+        tc::mma_commit(&sm.s_full[s]);
+        if (seg_end) tc::mma_commit(&sm.q_empty);
+        if (!seg_start && jt > 0) {
+            if (!issue_pv(sm, tmem, jt - 1, prev_first)) { ok = false; break; }
+        }
+        prev_first = seg_start;
+    }
+    if (ok && f1 > f0) ok = issue_pv(sm, tmem, (int)(f1 - f0 - 1), prev_first);
+    if (!ok) fault(sm, a);
+    // every MMA issued has completed before the CTA frees TMEM
+    tc::mma_commit(&sm.drain);
+    tc::mbar_wait(&sm.drain, 0);
+}
+
+// ---------------------------------------------------------------------
+// warps 2-5: softmax, rescale, output
+// ---------------------------------------------------------------------
+__device__ void softmax_warps(Smem& sm, const TcArgs& a, uint32_t tmem, long long f0, long long f1, int cta) {
+    const int sub = (threadIdx.x >> 5) & 3;  // TMEM sub-partition this warp may access
+    const int lane = threadIdx.x & 31;
+    const bool active = lane < 16;           // M = 64: head 16*sub + lane lives in lane (32*sub + lane)
+    const int h = 16 * sub + lane;
+    const uint32_t lane_addr = (uint32_t)(32 * sub) << 16;
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (long long f = f0; f < f1; ++f) {
+        if (sm.abort_flag) { ok = false; break; }
+        const int jt = (int)(f - f0), s = jt & 1;
+        const int row = (int)(f / a.tpr), ti = (int)(f % a.tpr);
+        const bool seg_start = (f == f0) || (ti == 0);
+        const bool seg_end = (f == f1 - 1) || (ti == a.tpr - 1);
+        if (seg_start) {
+            m_run = -INFINITY;
+            l_run = 0.f;
+        }
+        if (!tc::mbar_wait(&sm.kv_full[s], (jt >> 1) & 1)) { ok = false; break; }
+        const uint64_t mask = sm.mask[s];
+        if (!tc::mbar_wait(&sm.s_full[s], (jt >> 1) & 1)) { ok = false; break; }
+        tc::tc_fence_after();
+        uint32_t r[64];
+        tc::tmem_ld_x64(tmem + lane_addr + kColS + 64 * s, r);
+        tc::tmem_ld_wait();
+        float alpha = 1.f;
+        bool rescale = false;
+        uint32_t pk[32];  // bf16 pairs of this head's probabilities
+        if (active) {
+            float mt = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < 64; ++i) {
+                const float x = ((mask >> i) & 1) ? __uint_as_float(r[i]) * a.scale_log2 : -INFINITY;
+                r[i] = __float_as_uint(x);
+                mt = fmaxf(mt, x);
+            }
+            if (mt > m_run + kRescaleSlack) {
+                if (m_run != -INFINITY) {
+                    alpha = exp2f(m_run - mt);
+                    rescale = true;
+                    l_run *= alpha;
+                }
+                m_run = mt;
+            }
+            float lsum = 0.f;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const float x0 = __uint_as_float(r[2 * i]), x1 = __uint_as_float(r[2 * i + 1]);
+                const float p0 = m_run == -INFINITY ? 0.f : exp2f(x0 - m_run);
+                const float p1 = m_run == -INFINITY ? 0.f : exp2f(x1 - m_run);
+                const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
+                lsum += __low2float(pb) + __high2float(pb);
+                pk[i] = *reinterpret_cast<const uint32_t*>(&pb);
+            }
+            l_run += lsum;
+            sm.alpha[s][h] = alpha;
+            if (rescale) sm.rescale_tag[s] = jt + 1;
+        }
+        // the P buffer of this stage is free once PV two tiles back is done
+        if (jt >= 2 && !tc::mbar_wait(&sm.p_free[s], ((jt >> 1) - 1) & 1)) { ok = false; break; }
+        tc::named_barrier(1, 128);
+        if (sm.rescale_tag[s] == jt + 1) {
+            // O^T (lanes = d, columns = heads) was accumulated with the old maxima
+            if (!tc::mbar_wait(&sm.p_free[(jt - 1) & 1], ((jt - 1) >> 1) & 1)) { ok = false; break; }
+            tc::tc_fence_after();
+#pragma unroll 1
+            for (int cc = 0; cc < 4; ++cc) {
+                uint32_t o[64];
+                tc::tmem_ld_x64(tmem + lane_addr + kColO + 64 * cc, o);
+                tc::tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 64; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * sm.alpha[s][i]);
+                tc::tmem_st_x64(tmem + lane_addr + kColO + 64 * cc, o);
+            }
+            tc::tmem_st_wait();
+        }
+        if (active) {
+            uint8_t* prow = sm.p[s] + (h >> 3) * 1024 + (h & 7) * 128;
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                *reinterpret_cast<uint4*>(prow + ((u ^ (h & 7)) << 4)) =
+                    make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+        }
+        tc::fence_proxy_async();
+        tc::tc_fence_before();
+        tc::mbar_arrive(&sm.p_full[s]);
+
+        if (seg_end) {
+            if (!tc::mbar_wait(&sm.p_free[s], (jt >> 1) & 1)) { ok = false; break; }
+            tc::tc_fence_after();
+            if (active) {
+                sm.m_s[h] = m_run;
+                sm.l_s[h] = l_run;
+            }
+            tc::named_barrier(1, 128);
+            const long long rs = (long long)row * a.tpr;
+            const bool whole = (rs >= f0) && (rs + a.tpr <= f1);
+            // a piece of a split query: slot 2c for the CTA's first query, 2c+1 for its last
+            const int slot = 2 * cta + (row == (int)(f0 / a.tpr) ? 0 : 1);
+            float* dst;
+            long long hstride;
+            if (whole) {
+                dst = a.out + (long long)row * kH * kD;
+            } else {
+                dst = a.part_o + (long long)slot * kH * kD;
+                if (active) {
+                    a.part_ml[((long long)slot * kH + h) * 2] = m_run;
+                    a.part_ml[((long long)slot * kH + h) * 2 + 1] = l_run;
+                }
+            }
+            hstride = kD;
+#pragma unroll 1
+            for (int cc = 0; cc < 4; ++cc) {
+                uint32_t o[64];
+                tc::tmem_ld_x64(tmem + lane_addr + kColO + 64 * cc, o);
+                tc::tmem_ld_wait();
+                const int d = 128 * cc + 32 * sub + lane;
+#pragma unroll
+                for (int i = 0; i < kH; ++i) {
+                    float v = __uint_as_float(o[i]);
+                    if (whole) {
+                        const float l = sm.l_s[i];
+                        v = l > 0.f ? v / l : 0.f;
+                    }
+                    dst[i * hstride + d] = v;
+                }
+            }
+            tc::tc_fence_before();
+            tc::named_barrier(1, 128);
+        }
+    }
+    if (!ok || sm.abort_flag) {
+        fault(sm, a);
+        // poison every output this CTA contributes to
+        const int r0 = (int)(f0 / a.tpr), r1 = f1 > f0 ? (int)((f1 - 1) / a.tpr) : r0 - 1;
+        const int t = threadIdx.x - 64;
+        for (int rr = r0; rr <= r1; ++rr)
+            for (int i = t; i < kH * kD; i += 128) a.out[(long long)rr * kH * kD + i] = NAN;
+        for (int i = t; i < 2 * kH * 2; i += 128) a.part_ml[(long long)2 * cta * kH * 2 + i] = NAN;
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    attend_tc_kernel(const __grid_constant__ CUtensorMap ent_map, const __grid_constant__ CUtensorMap tok_map,
+                     const __grid_constant__ CUtensorMap q_map, TcArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5;
+    const int cta = blockIdx.x;
+    const long long f0 = range_start(cta, a), f1 = range_start(cta + 1, a);
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < 2; ++i) {
+            tc::mbar_init(&sm.kv_full[i], 33);  // 1 expect_tx arrival + 32 cp.async arrivals
+            tc::mbar_init(&sm.kv_empty[i], 1);
+            tc::mbar_init(&sm.s_full[i], 1);
+            tc::mbar_init(&sm.p_full[i], 128);
+            tc::mbar_init(&sm.p_free[i], 1);
+        }
+        tc::mbar_init(&sm.q_full, 1);
+        tc::mbar_init(&sm.q_empty, 1);
+        tc::mbar_init(&sm.drain, 1);
+        sm.rescale_tag[0] = sm.rescale_tag[1] = 0;
+        sm.abort_flag = 0;
+        tc::fence_barrier_init();
+    }
+    if (warp == 1) tc::tmem_alloc(&sm.tmem_base, kTmemCols);
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+
+    if (warp == 0) {
+        producer(sm, a, &ent_map, &tok_map, &q_map, f0, f1);
+    } else if (warp == 1) {
+        if ((threadIdx.x & 31) == 0) mma_issuer(sm, a, tmem, f0, f1);
+        __syncwarp();
+    } else {
+        softmax_warps(sm, a, tmem, f0, f1, cta);
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// Merge the partials of queries whose tiles were split between CTAs.
+// grid (rows, 64 heads), 128 threads x 4 elements.
+__global__ void attend_tc_combine(TcArgs a) {
+    const int row = blockIdx.x, h = blockIdx.y;
+    const long long rs = (long long)row * a.tpr, re = rs + a.tpr - 1;
+    // CTA holding flat tile f: the largest c with range_start(c) <= f
+    auto cta_of = [&](long long f) { return (int)(((f + 1) * a.grid - 1) / a.total_tiles); };
+    const int c0 = cta_of(rs), c1 = cta_of(re);
+    if (c0 == c1) return;  // written directly by its only CTA
+    float mmax = -INFINITY;
+    bool bad = false;
+    for (int c = c0; c <= c1; ++c) {
+        const int slot = 2 * c + ((range_start(c, a) / a.tpr == row) ? 0 : 1);
+        const float ms = a.part_ml[((long long)slot * kH + h) * 2];
+        bad |= isnan(ms);
+        mmax = fmaxf(mmax, ms);
+    }
+    const int e = threadIdx.x * 4;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float l = 0.f;
+    if (mmax != -INFINITY && !bad) {
+        for (int c = c0; c <= c1; ++c) {
+            const int slot = 2 * c + ((range_start(c, a) / a.tpr == row) ? 0 : 1);
+            const float ms = a.part_ml[((long long)slot * kH + h) * 2];
+            if (ms == -INFINITY) continue;
+            const float w = exp2f(ms - mmax);
+            l += w * a.part_ml[((long long)slot * kH + h) * 2 + 1];
+            const float4 v = *reinterpret_cast<const float4*>(a.part_o + ((long long)slot * kH + h) * kD + e);
+            acc.x = fmaf(w, v.x, acc.x);
+            acc.y = fmaf(w, v.y, acc.y);
+            acc.z = fmaf(w, v.z, acc.z);
+            acc.w = fmaf(w, v.w, acc.w);
+        }
+    }
+    const float inv = bad ? NAN : (l > 0.f ? 1.f / l : 0.f);
+    *reinterpret_cast<float4*>(a.out + ((long long)row * kH + h) * kD + e) =
+        make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// [rows][512] bf16, boxes of 64 columns x 64 rows, 128-byte swizzle
+bool make_map(CUtensorMap* map, const void* base, long long rows) {
+    auto fn = encode_fn();
+    if (!fn || rows < 1) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)kD * 2};
+    cuuint32_t box[2] = {64, 64};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct TcPlan {
+    int e_tiles, w_tiles, tpr, grid;
+    long long total;
+};
+
+TcPlan tc_plan(const AttendArgs& a) {
+    TcPlan p;
+    const long long n_sel_max = a.idx ? (long long)a.k : (a.ctx_len / a.m < a.n_ent ? a.ctx_len / a.m : a.n_ent);
+    p.e_tiles = (int)((n_sel_max + kTile - 1) / kTile);
+    p.w_tiles = (a.window + kTile - 1) / kTile;
+    p.tpr = p.e_tiles + p.w_tiles;
+    p.total = (long long)a.batch * a.n_q * p.tpr;
+    p.grid = (int)(p.total < kNumSMs ? p.total : kNumSMs);
+    return p;
+}
+
+}  // namespace
+
+bool attend_tc_shape_ok(const AttendArgs& a) {
+    if (a.dtype != V4A_BF16 || a.d != kD || a.heads != kH) return false;
+    TcPlan p = tc_plan(a);
+    if (p.tpr < 1 || p.grid < 1) return false;
+    if ((long long)a.batch * a.n_ent >= (1LL << 31) || (long long)a.batch * a.l_tok >= (1LL << 31)) return false;
+    if ((long long)a.batch * a.n_q * kH >= (1LL << 31)) return false;
+    return true;
+}
+
+bool attend_tc_available(const AttendArgs& a) { return attend_tc_shape_ok(a) && encode_fn() != nullptr; }
+
+size_t attend_tc_workspace_bytes(const AttendArgs& a) {
+    TcPlan p = tc_plan(a);
+    size_t slots = 2 * (size_t)p.grid;
+    size_t ml = (slots * kH * 2 * sizeof(float) + 255) / 256 * 256;
+    return ml + slots * kH * kD * sizeof(float);
+}
+
+cudaError_t launch_attend_tc(const AttendArgs& a, void* ws, size_t ws_bytes, cudaStream_t stream) {
+    if (ws_bytes < attend_tc_workspace_bytes(a)) return cudaErrorInvalidValue;
+    TcPlan p = tc_plan(a);
+    CUtensorMap ent_map, tok_map, q_map;
+    const long long ent_rows = (long long)a.batch * a.n_ent;
+    const long long tok_rows = (long long)a.batch * a.l_tok;
+    const void* tok = a.token_kv ? a.token_kv : a.q;  // a window of 0 never reads it
+    if (!make_map(&tok_map, tok, a.token_kv ? tok_rows : (long long)a.batch * a.n_q * kH)) return cudaErrorInvalidValue;
+    if (ent_rows > 0) {
+        if (!make_map(&ent_map, a.entries, ent_rows)) return cudaErrorInvalidValue;
+    } else {
+        ent_map = tok_map;  // no entry tiles exist
+    }
+    if (!make_map(&q_map, a.q, (long long)a.batch * a.n_q * kH)) return cudaErrorInvalidValue;
+
+    TcArgs t;
+    t.q = static_cast<const __nv_bfloat16*>(a.q);
+    t.entries = static_cast<const __nv_bfloat16*>(a.entries);
+    t.token_kv = static_cast<const __nv_bfloat16*>(tok);
+    t.idx = a.idx;
+    t.out = a.out;
+    const size_t slots = 2 * (size_t)p.grid;
+    t.part_ml = static_cast<float*>(ws);
+    t.part_o = reinterpret_cast<float*>(static_cast<char*>(ws) + (slots * kH * 2 * sizeof(float) + 255) / 256 * 256);
+    t.dev_status = a.dev_status;
+    t.n_ent = a.n_ent;
+    t.l_tok = a.l_tok;
+    t.tok_pos0 = a.tok_pos0;
+    t.ctx_len = a.ctx_len;
+    t.total_tiles = p.total;
+    t.rows = a.batch * a.n_q;
+    t.n_q = a.n_q;
+    t.m = a.m;
+    t.k = a.idx ? a.k : 0;
+    t.window = a.window;
+    t.e_tiles = p.e_tiles;
+    t.w_tiles = p.w_tiles;
+    t.tpr = p.tpr;
+    t.grid = p.grid;
+    t.scale_log2 = 1.4426950408889634f / sqrtf((float)kD);
+
+    const size_t smem = sizeof(Smem) + 1024;
+    cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    attend_tc_kernel<<<p.grid, kThreads, smem, stream>>>(ent_map, tok_map, q_map, t);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    if (p.grid > 1) {
+        attend_tc_combine<<<dim3(t.rows, kH), kD / 4, 0, stream>>>(t);
+        e = cudaGetLastError();
+    }
+    return e;
+}
+
+}  // namespace v4a

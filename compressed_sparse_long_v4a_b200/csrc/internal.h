@@ -50,4 +50,10 @@ struct AttendArgs {
 size_t attend_workspace_bytes(const AttendArgs& a);
 cudaError_t launch_attend(const AttendArgs& a, void* ws, size_t ws_bytes, cudaStream_t stream);
 
+// ---- attend_tc.cu (tcgen05 path: bf16, d = 512, 64 heads) -------------
+bool attend_tc_shape_ok(const AttendArgs& a);   // the shape this path takes
+bool attend_tc_available(const AttendArgs& a);  // ... and the driver's tensor-map encoder is present
+size_t attend_tc_workspace_bytes(const AttendArgs& a);
+cudaError_t launch_attend_tc(const AttendArgs& a, void* ws, size_t ws_bytes, cudaStream_t stream);
+
 }  // namespace v4a

@@ -251,6 +251,7 @@ size_t v4a_workspace_size(const char* op, const v4a_shape* shape, int heads_i, i
         a.ctx_len = shape->ctx_len;
         a.n_ent = shape->ctx_len / a.m;
         a.idx = csa ? reinterpret_cast<const int32_t*>(1) : nullptr;
+        a.dtype = V4A_BF16;  // no dtype argument: size for the larger (tensor-core) requirement
         return v4a::attend_workspace_bytes(a);
     }
     return 0;

@@ -337,3 +337,41 @@ def test_csa_l1m_fp8_full_size_sampled(v4a):
                       host(_sub(w["token_kv"], bs)), w["tok_pos0"], L, m, W)
     check_attention(out[bs], r, False, "csa_l1m_fp8")
     print("tie band entries:", rep["tie_band_entries"])
+
+
+# ----------------------------------------------------------------------
+# paths of the tensor-core kernel (bf16, d = 512, 64 heads)
+# ----------------------------------------------------------------------
+
+def test_attend_rescale_path_increasing_logits(v4a):
+    """Logits that grow by more than 2^8 per 64-row tile force the running
+    maximum (and the accumulated output) to be rescaled tile after tile."""
+    B, T, m, H, d, W = 2, 1, 128, 64, 512, 128
+    L = m * 192 + 5
+    g = wl._gen(31)
+    q = torch.ones((B, T, H, d), dtype=torch.bfloat16)
+    N = L // m
+    ramp = (torch.arange(N, dtype=torch.float32) * 0.005)[None, :, None]
+    ent = (ramp + 0.05 * wl.normal(g, (B, N, d))).to(torch.bfloat16)
+    p0, lt = wl.window_rows(L, T, W)
+    tok = (0.05 * wl.normal(g, (B, lt, d))).to(torch.bfloat16)
+    out = torch.empty((B, T, H, d), device="cuda")
+    v4a.v4a_hca_attend(dev(q), dev(ent), dev(tok), p0, out, m=m, window=W, ctx_len=L)
+    _sync()
+    ref = oracle.attend(host(q), host(ent), None, host(tok), p0, L, m, W)
+    check_attention(out, ref, False, "rescale path")
+
+
+def test_csa_many_queries_split_rows(v4a):
+    """Many queries (multi-query CSA): each CTA runs several queries and some
+    queries are split between CTAs and merged afterwards."""
+    B, T, L, m, H, d, W, k = 2, 200, 4 * 3000, 4, 64, 512, 128, 128
+    a = _attend_inputs(B, T, L, m, H, d, W, "bf16", seed=55, k=k, pad=0.05)
+    out = torch.empty((B, T, H, d), dtype=torch.float32, device="cuda")
+    st = torch.zeros((1,), dtype=torch.int32, device="cuda")
+    v4a.v4a_csa_attend(dev(a["q"]), dev(a["entries"]), dev(a["idx"]), dev(a["token_kv"]), a["tok_pos0"], out,
+                       m=m, window=W, ctx_len=L, dev_status=st)
+    _sync()
+    assert int(st.item()) == 0
+    ref = oracle.attend(host(a["q"]), host(a["entries"]), host(a["idx"]), host(a["token_kv"]), a["tok_pos0"], L, m, W)
+    check_attention(out, ref, False, "csa multi-query")
