@@ -13,6 +13,10 @@
 //   P  = softmax(S) (online, one thread per head)
 //   O^T += V^T P^T  tcgen05 M=128 (d chunk) x N=64 (heads) x K=64 (rows),
 //                   four d chunks, V^T read MN-major from the same smem tile
+// An MMA instruction costs about max(45, N/2) cycles at M=128 (M=64 at half
+// the rate), so tiles are as wide as shared memory allows (64 rows, two
+// stages next to the 64 KB query) and the issue loops use precomputed
+// descriptors.
 // The accumulator O^T (512 x 64 fp32) and two S buffers live in TMEM.
 //
 // Work split: the candidate tiles of all queries form one flat sequence that
@@ -36,6 +40,7 @@ namespace {
 constexpr int kD = 512;
 constexpr int kH = 64;
 constexpr int kTile = 64;                        // candidate rows per tile
+constexpr int kStages = 2;                       // tiles resident in shared memory
 constexpr int kSlabs = kD / 64;                  // 64-element (128 B) column slabs
 constexpr uint32_t kSlabBytes = kTile * 128;     // 8 KB
 constexpr uint32_t kTileBytes = kSlabs * kSlabBytes;
@@ -47,16 +52,16 @@ constexpr uint32_t kTmemCols = 512;
 constexpr int kThreads = 192;
 constexpr float kRescaleSlack = 8.0f;  // keep a stale running max until the true one exceeds it by 2^8
 
-constexpr uint32_t kIdescQK = tc::idesc_f16(64, 64, 0, 0);
+constexpr uint32_t kIdescQK = tc::idesc_f16(64, kTile, 0, 0);
 constexpr uint32_t kIdescPV = tc::idesc_f16(128, 64, 1, 0);
 
 struct __align__(1024) Smem {
     uint8_t q[kQBytes];
-    uint8_t kv[2][kTileBytes];
+    uint8_t kv[kStages][kTileBytes];
     uint8_t p[2][kPBytes];
-    uint64_t kv_full[2], kv_empty[2], s_full[2], p_full[2], p_free[2];
+    uint64_t kv_full[kStages], kv_empty[kStages], s_full[2], p_full[2], p_free[2];
     uint64_t q_full, q_empty, drain;
-    uint64_t mask[2];
+    uint64_t mask[kStages];
     float alpha[2][kH], l_s[kH], m_s[kH];  // alpha / rescale_tag by tile parity
     int rescale_tag[2];
     int abort_flag;
@@ -87,6 +92,18 @@ struct RowInfo {
     long long t, nvis;
 };
 
+// walks the flat tile sequence f0, f0+1, ... keeping (row, tile-in-row) without divisions
+struct Cursor {
+    int row, ti;
+    __device__ Cursor(long long f, int tpr) : row((int)(f / tpr)), ti((int)(f % tpr)) {}
+    __device__ void next(int tpr) {
+        if (++ti == tpr) {
+            ti = 0;
+            ++row;
+        }
+    }
+};
+
 __device__ __forceinline__ RowInfo row_info(int row, const TcArgs& a) {
     RowInfo r;
     r.b = row / a.n_q;
@@ -105,14 +122,28 @@ __device__ __forceinline__ void fault(Smem& sm, const TcArgs& a) {
 // ---------------------------------------------------------------------
 // warp 0: loads
 // ---------------------------------------------------------------------
+// candidate rows of one CSA tile: lane owns rows lane and lane+32
+__device__ __forceinline__ void csa_rows(const TcArgs& a, const RowInfo& ri, int row, long long c0, int lane,
+                                         const __nv_bfloat16* (&src)[2], bool (&ok)[2]) {
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2) {
+        const long long c = c0 + lane + 32 * h2;
+        const long long sidx = c < a.k ? (long long)a.idx[(long long)row * a.k + c] : -1;
+        ok[h2] = sidx >= 0 && sidx < ri.nvis;
+        // an excluded row still gets finite data: this query's head-0 row of q
+        src[h2] = ok[h2] ? a.entries + ((long long)ri.b * a.n_ent + sidx) * kD : a.q + (long long)row * kH * kD;
+    }
+}
+
 __device__ void producer(Smem& sm, const TcArgs& a, const CUtensorMap* ent_map, const CUtensorMap* tok_map,
                          const CUtensorMap* q_map, long long f0, long long f1) {
     const int lane = threadIdx.x & 31;
     int seg = 0;
-    for (long long f = f0; f < f1; ++f) {
+    Cursor cur(f0, a.tpr);
+    for (long long f = f0; f < f1; ++f, cur.next(a.tpr)) {
         if (sm.abort_flag) break;
-        const int jt = (int)(f - f0), s = jt & 1;
-        const int row = (int)(f / a.tpr), ti = (int)(f % a.tpr);
+        const int jt = (int)(f - f0), st = jt % kStages;
+        const int row = cur.row, ti = cur.ti;
         const bool seg_start = (f == f0) || (ti == 0);
         const RowInfo ri = row_info(row, a);
         if (seg_start) {
@@ -123,38 +154,33 @@ __device__ void producer(Smem& sm, const TcArgs& a, const CUtensorMap* ent_map, 
             }
             ++seg;
         }
-        if (jt >= 2 && !tc::mbar_wait(&sm.kv_empty[s], ((jt >> 1) - 1) & 1)) { fault(sm, a); break; }
+        if (jt >= kStages && !tc::mbar_wait(&sm.kv_empty[st], ((jt / kStages) - 1) & 1)) { fault(sm, a); break; }
         uint64_t mask = 0;
-        uint8_t* dst = sm.kv[s];
+        uint8_t* dst = sm.kv[st];
         if (ti < a.e_tiles) {
             const long long c0 = (long long)ti * kTile;
             if (!a.idx) {
-                // HCA: rows c0..c0+63 of this sequence's entries are contiguous
+                // HCA: rows c0 .. c0+63 of this sequence's entries are contiguous
                 const long long nv = ri.nvis - c0;
-                mask = nv >= 64 ? ~0ull : (nv <= 0 ? 0ull : ((1ull << nv) - 1));
+                mask = nv >= kTile ? ~0ull : (nv <= 0 ? 0ull : ((1ull << nv) - 1ull));
                 if (lane == 0) {
-                    sm.mask[s] = mask;
-                    tc::mbar_arrive_expect_tx(&sm.kv_full[s], kTileBytes);
+                    sm.mask[st] = mask;
+                    tc::mbar_arrive_expect_tx(&sm.kv_full[st], kTileBytes);
                     const int y = (int)((long long)ri.b * a.n_ent + c0);
-                    for (int c = 0; c < kSlabs; ++c) tc::tma_load_2d(dst + c * kSlabBytes, ent_map, 64 * c, y, &sm.kv_full[s]);
+                    for (int c = 0; c < kSlabs; ++c) tc::tma_load_2d(dst + c * kSlabBytes, ent_map, 64 * c, y, &sm.kv_full[st]);
                 }
             } else {
                 // CSA: gather the selected rows with cp.async (128-byte swizzle written by hand)
                 const __nv_bfloat16* src[2];
                 bool ok[2];
+                csa_rows(a, ri, row, c0, lane, src, ok);
 #pragma unroll
                 for (int h2 = 0; h2 < 2; ++h2) {
                     const long long c = c0 + lane + 32 * h2;
-                    long long sidx = c < a.k ? (long long)a.idx[(long long)row * a.k + c] : -1;
-                    ok[h2] = sidx >= 0 && sidx < ri.nvis;
+                    const long long sidx = c < a.k ? (long long)a.idx[(long long)row * a.k + c] : -1;
                     if (!ok[h2] && sidx != -1 && a.dev_status) atomicExch(a.dev_status, (int)V4A_ERR_DEVICE_FAULT);
-                    // an excluded row still gets finite data: this query's head-0 row of q
-                    src[h2] = ok[h2] ? a.entries + ((long long)ri.b * a.n_ent + sidx) * kD
-                                     : a.q + (long long)row * kH * kD;
                 }
-                const uint32_t lo = __ballot_sync(0xffffffffu, ok[0]);
-                const uint32_t hi = __ballot_sync(0xffffffffu, ok[1]);
-                mask = (uint64_t)lo | ((uint64_t)hi << 32);
+                mask = (uint64_t)__ballot_sync(0xffffffffu, ok[0]) | ((uint64_t)__ballot_sync(0xffffffffu, ok[1]) << 32);
                 for (int r = 0; r < kTile; ++r) {
                     const __nv_bfloat16* rs = (const __nv_bfloat16*)__shfl_sync(
                         0xffffffffu, (unsigned long long)(r < 32 ? src[0] : src[1]), r & 31);
@@ -166,8 +192,8 @@ __device__ void producer(Smem& sm, const TcArgs& a, const CUtensorMap* ent_map, 
                     }
                 }
                 if (lane == 0) {
-                    sm.mask[s] = mask;
-                    tc::mbar_arrive_expect_tx(&sm.kv_full[s], 0);
+                    sm.mask[st] = mask;
+                    tc::mbar_arrive_expect_tx(&sm.kv_full[st], 0);
                 }
             }
         } else {
@@ -179,19 +205,19 @@ __device__ void producer(Smem& sm, const TcArgs& a, const CUtensorMap* ent_map, 
                 if (wi * kTile + r < a.window && p >= 0) mask |= 1ull << r;
             }
             if (lane == 0) {
-                sm.mask[s] = mask;
-                tc::mbar_arrive_expect_tx(&sm.kv_full[s], kTileBytes);
+                sm.mask[st] = mask;
+                tc::mbar_arrive_expect_tx(&sm.kv_full[st], kTileBytes);
                 const int y = (int)((long long)ri.b * a.l_tok + (p0 - a.tok_pos0));
-                for (int c = 0; c < kSlabs; ++c) tc::tma_load_2d(dst + c * kSlabBytes, tok_map, 64 * c, y, &sm.kv_full[s]);
+                for (int c = 0; c < kSlabs; ++c) tc::tma_load_2d(dst + c * kSlabBytes, tok_map, 64 * c, y, &sm.kv_full[st]);
             }
         }
-        tc::cp_async_arrive_noinc(&sm.kv_full[s]);  // 32 lanes: after their cp.async copies (if any) land
+        tc::cp_async_arrive_noinc(&sm.kv_full[st]);  // 32 lanes: after their cp.async copies (if any) land
     }
     // make sure nothing this warp started is still in flight before the CTA retires
     const long long n = f1 - f0;
-    for (long long jt = n - 2; jt < n; ++jt) {
+    for (long long jt = n - kStages; jt < n; ++jt) {
         if (jt < 0) continue;
-        tc::mbar_wait(&sm.kv_full[jt & 1], (jt >> 1) & 1);
+        tc::mbar_wait(&sm.kv_full[jt % kStages], (jt / kStages) & 1);
     }
     if (seg > 0) tc::mbar_wait(&sm.q_full, (seg - 1) & 1);
 }
@@ -199,24 +225,24 @@ __device__ void producer(Smem& sm, const TcArgs& a, const CUtensorMap* ent_map, 
 // ---------------------------------------------------------------------
 // warp 1: MMA issue (one thread)
 // ---------------------------------------------------------------------
+// descriptor + byte offset (the start-address field counts 16-byte units)
+__device__ __forceinline__ uint64_t dadd(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
+
 __device__ bool issue_pv(Smem& sm, uint32_t tmem, int jp, bool first_in_seg) {
-    const int sp = jp & 1;
+    const int sp = jp & 1, st = jp % kStages;
     if (!tc::mbar_wait(&sm.p_full[sp], (jp >> 1) & 1)) return false;
     tc::tc_fence_after();
-    const uint32_t kv = tc::smem_u32(sm.kv[sp]);
-    const uint32_t pb = tc::smem_u32(sm.p[sp]);
+    // A = V^T (M = 128 d of slabs 2cc, 2cc+1; K = 16 rows), MN-major; B = P^T, K-major rows of P
+    const uint64_t a0 = tc::sw128_desc(tc::smem_u32(sm.kv[st]), kSlabBytes, 1024);
+    const uint64_t b0 = tc::sw128_desc(tc::smem_u32(sm.p[sp]), 16, 1024);
 #pragma unroll
-    for (int cc = 0; cc < 4; ++cc) {
+    for (int kk = 0; kk < kTile / 16; ++kk) {
 #pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk) {
-            // A = V^T (M = 128 d of slabs 2cc, 2cc+1; K = 16 rows), MN-major
-            const uint64_t ad = tc::sw128_desc(kv + (2 * cc) * kSlabBytes + kk * 2048, kSlabBytes, 1024);
-            // B = P^T (N = 64 heads, K = 16 rows), K-major rows of P
-            const uint64_t bd = tc::sw128_desc(pb + kk * 32, 16, 1024);
-            tc::mma_f16(tmem + kColO + 64 * cc, ad, bd, kIdescPV, (!first_in_seg || kk > 0) ? 1u : 0u);
-        }
+        for (int cc = 0; cc < 4; ++cc)
+            tc::mma_f16(tmem + kColO + 64 * cc, dadd(a0, (2 * cc) * kSlabBytes + kk * 2048), dadd(b0, kk * 32),
+                        kIdescPV, (!first_in_seg || kk > 0) ? 1u : 0u);
     }
-    tc::mma_commit(&sm.kv_empty[sp]);
+    tc::mma_commit(&sm.kv_empty[st]);
     tc::mma_commit(&sm.p_free[sp]);
     return true;
 }
@@ -225,10 +251,12 @@ __device__ void mma_issuer(Smem& sm, const TcArgs& a, uint32_t tmem, long long f
     int seg = 0;
     bool ok = true;
     bool prev_first = false;  // whether the pending PV tile starts its segment
-    for (long long f = f0; f < f1 && ok; ++f) {
+    const uint64_t q0 = tc::sw128_desc(tc::smem_u32(sm.q), 16, 1024);
+    Cursor cur(f0, a.tpr);
+    for (long long f = f0; f < f1 && ok; ++f, cur.next(a.tpr)) {
         if (sm.abort_flag) { ok = false; break; }
-        const int jt = (int)(f - f0), s = jt & 1;
-        const int ti = (int)(f % a.tpr);
+        const int jt = (int)(f - f0), s = jt & 1, st = jt % kStages;
+        const int ti = cur.ti;
         const bool seg_start = (f == f0) || (ti == 0);
         const bool seg_end = (f == f1 - 1) || (ti == a.tpr - 1);
         if (seg_start && jt > 0) {
@@ -238,19 +266,17 @@ __device__ void mma_issuer(Smem& sm, const TcArgs& a, uint32_t tmem, long long f
             if (!tc::mbar_wait(&sm.q_full, seg & 1)) { ok = false; break; }
             ++seg;
         }
-        if (!tc::mbar_wait(&sm.kv_full[s], (jt >> 1) & 1)) { ok = false; break; }
+        if (!tc::mbar_wait(&sm.kv_full[st], (jt / kStages) & 1)) { ok = false; break; }
         tc::fence_proxy_async();  // rows gathered with cp.async become visible to the tensor core
         tc::tc_fence_after();
-        const uint32_t qb = tc::smem_u32(sm.q);
-        const uint32_t kb = tc::smem_u32(sm.kv[s]);
-#pragma unroll 1
+        const uint64_t k0 = tc::sw128_desc(tc::smem_u32(sm.kv[st]), 16, 1024);
+        const uint32_t d_s = tmem + kColS + kTile * s;
+#pragma unroll
         for (int c = 0; c < kSlabs; ++c) {
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                const uint64_t ad = tc::sw128_desc(qb + c * kH * 128 + kk * 32, 16, 1024);
-                const uint64_t bd = tc::sw128_desc(kb + c * kSlabBytes + kk * 32, 16, 1024);
-                tc::mma_f16(tmem + kColS + 64 * s, ad, bd, kIdescQK, (c | kk) ? 1u : 0u);
-            }
+            for (int kk = 0; kk < 4; ++kk)
+                tc::mma_f16(d_s, dadd(q0, c * kH * 128 + kk * 32), dadd(k0, c * kSlabBytes + kk * 32), kIdescQK,
+                            (c | kk) ? 1u : 0u);
         }
         tc::mma_commit(&sm.s_full[s]);
         if (seg_end) tc::mma_commit(&sm.q_empty);
@@ -272,39 +298,46 @@ __device__ void mma_issuer(Smem& sm, const TcArgs& a, uint32_t tmem, long long f
 __device__ void softmax_warps(Smem& sm, const TcArgs& a, uint32_t tmem, long long f0, long long f1, int cta) {
     const int sub = (threadIdx.x >> 5) & 3;  // TMEM sub-partition this warp may access
     const int lane = threadIdx.x & 31;
-    const bool active = lane < 16;           // M = 64: head 16*sub + lane lives in lane (32*sub + lane)
-    const int h = 16 * sub + lane;
+    // M = 64: head 16*sub + (lane & 15) lives in TMEM lane 32*sub + (lane & 15); lanes 0-15 take the
+    // first 32 columns of each tile, lanes 16-31 the last 32
+    const int half = lane >> 4;
+    const int h = 16 * sub + (lane & 15);
     const uint32_t lane_addr = (uint32_t)(32 * sub) << 16;
-    float m_run = -INFINITY, l_run = 0.f;
+    float m_run = -INFINITY, l_run = 0.f;  // l_run: this thread's half of the row sum
     bool ok = true;
-    for (long long f = f0; f < f1; ++f) {
+    Cursor cur(f0, a.tpr);
+    const int first_row = cur.row;
+    for (long long f = f0; f < f1; ++f, cur.next(a.tpr)) {
         if (sm.abort_flag) { ok = false; break; }
-        const int jt = (int)(f - f0), s = jt & 1;
-        const int row = (int)(f / a.tpr), ti = (int)(f % a.tpr);
+        const int jt = (int)(f - f0), s = jt & 1, st = jt % kStages;
+        const int row = cur.row, ti = cur.ti;
         const bool seg_start = (f == f0) || (ti == 0);
         const bool seg_end = (f == f1 - 1) || (ti == a.tpr - 1);
         if (seg_start) {
             m_run = -INFINITY;
             l_run = 0.f;
         }
-        if (!tc::mbar_wait(&sm.kv_full[s], (jt >> 1) & 1)) { ok = false; break; }
-        const uint64_t mask = sm.mask[s];
+        if (!tc::mbar_wait(&sm.kv_full[st], (jt / kStages) & 1)) { ok = false; break; }
+        const uint32_t mask = (uint32_t)(sm.mask[st] >> (32 * half));
         if (!tc::mbar_wait(&sm.s_full[s], (jt >> 1) & 1)) { ok = false; break; }
         tc::tc_fence_after();
-        uint32_t r[64];
-        tc::tmem_ld_x64(tmem + lane_addr + kColS + 64 * s, r);
+        uint32_t r[32];
+        tc::tmem_ld_16x32bx2_x32(tmem + lane_addr + kColS + kTile * s, r);
         tc::tmem_ld_wait();
         float alpha = 1.f;
         bool rescale = false;
-        uint32_t pk[32];  // bf16 pairs of this head's probabilities
-        if (active) {
-            float mt = -INFINITY;
+        uint32_t pk[16];  // bf16 pairs of this thread's 32 probabilities
+        {
+            // independent partial maxima / sums keep the dependent chains short
+            float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-            for (int i = 0; i < 64; ++i) {
+            for (int i = 0; i < 32; ++i) {
                 const float x = ((mask >> i) & 1) ? __uint_as_float(r[i]) * a.scale_log2 : -INFINITY;
                 r[i] = __float_as_uint(x);
-                mt = fmaxf(mt, x);
+                mx4[i & 3] = fmaxf(mx4[i & 3], x);
             }
+            float mt = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+            mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));  // both halves of the row
             if (mt > m_run + kRescaleSlack) {
                 if (m_run != -INFINITY) {
                     alpha = exp2f(m_run - mt);
@@ -313,21 +346,23 @@ __device__ void softmax_warps(Smem& sm, const TcArgs& a, uint32_t tmem, long lon
                 }
                 m_run = mt;
             }
-            float lsum = 0.f;
+            const float msub = m_run == -INFINITY ? 0.f : m_run;  // all-masked so far: every x is -inf
+            float ls4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const float x0 = __uint_as_float(r[2 * i]), x1 = __uint_as_float(r[2 * i + 1]);
-                const float p0 = m_run == -INFINITY ? 0.f : exp2f(x0 - m_run);
-                const float p1 = m_run == -INFINITY ? 0.f : exp2f(x1 - m_run);
+            for (int i = 0; i < 16; ++i) {
+                const float p0 = exp2f(__uint_as_float(r[2 * i]) - msub);
+                const float p1 = exp2f(__uint_as_float(r[2 * i + 1]) - msub);
                 const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-                lsum += __low2float(pb) + __high2float(pb);
+                ls4[i & 3] += __low2float(pb) + __high2float(pb);
                 pk[i] = *reinterpret_cast<const uint32_t*>(&pb);
             }
-            l_run += lsum;
-            sm.alpha[s][h] = alpha;
-            if (rescale) sm.rescale_tag[s] = jt + 1;
+            l_run += (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
+            if (half == 0) {
+                sm.alpha[s][h] = alpha;
+                if (rescale) sm.rescale_tag[s] = jt + 1;
+            }
         }
-        // the P buffer of this stage is free once PV two tiles back is done
+        // the P buffer of this parity is free once PV two tiles back is done
         if (jt >= 2 && !tc::mbar_wait(&sm.p_free[s], ((jt >> 1) - 1) & 1)) { ok = false; break; }
         tc::named_barrier(1, 128);
         if (sm.rescale_tag[s] == jt + 1) {
@@ -345,11 +380,13 @@ __device__ void softmax_warps(Smem& sm, const TcArgs& a, uint32_t tmem, long lon
             }
             tc::tmem_st_wait();
         }
-        if (active) {
+        {
+            // head h's row of P: the tile's 64 probabilities as one 128 B swizzled row; this thread
+            // writes the 4 16-byte chunks of its half
             uint8_t* prow = sm.p[s] + (h >> 3) * 1024 + (h & 7) * 128;
 #pragma unroll
-            for (int u = 0; u < 8; ++u)
-                *reinterpret_cast<uint4*>(prow + ((u ^ (h & 7)) << 4)) =
+            for (int u = 0; u < 4; ++u)
+                *reinterpret_cast<uint4*>(prow + (((4 * half + u) ^ (h & 7)) << 4)) =
                     make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
         }
         tc::fence_proxy_async();
@@ -359,27 +396,26 @@ __device__ void softmax_warps(Smem& sm, const TcArgs& a, uint32_t tmem, long lon
         if (seg_end) {
             if (!tc::mbar_wait(&sm.p_free[s], (jt >> 1) & 1)) { ok = false; break; }
             tc::tc_fence_after();
-            if (active) {
+            const float l_row = l_run + __shfl_xor_sync(0xffffffffu, l_run, 16);
+            if (half == 0) {
                 sm.m_s[h] = m_run;
-                sm.l_s[h] = l_run;
+                sm.l_s[h] = l_row;
             }
             tc::named_barrier(1, 128);
             const long long rs = (long long)row * a.tpr;
             const bool whole = (rs >= f0) && (rs + a.tpr <= f1);
             // a piece of a split query: slot 2c for the CTA's first query, 2c+1 for its last
-            const int slot = 2 * cta + (row == (int)(f0 / a.tpr) ? 0 : 1);
+            const int slot = 2 * cta + (row == first_row ? 0 : 1);
             float* dst;
-            long long hstride;
             if (whole) {
                 dst = a.out + (long long)row * kH * kD;
             } else {
                 dst = a.part_o + (long long)slot * kH * kD;
-                if (active) {
+                if (half == 0) {
                     a.part_ml[((long long)slot * kH + h) * 2] = m_run;
-                    a.part_ml[((long long)slot * kH + h) * 2 + 1] = l_run;
+                    a.part_ml[((long long)slot * kH + h) * 2 + 1] = l_row;
                 }
             }
-            hstride = kD;
 #pragma unroll 1
             for (int cc = 0; cc < 4; ++cc) {
                 uint32_t o[64];
@@ -393,7 +429,7 @@ __device__ void softmax_warps(Smem& sm, const TcArgs& a, uint32_t tmem, long lon
                         const float l = sm.l_s[i];
                         v = l > 0.f ? v / l : 0.f;
                     }
-                    dst[i * hstride + d] = v;
+                    dst[i * kD + d] = v;
                 }
             }
             tc::tc_fence_before();
@@ -421,9 +457,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const long long f0 = range_start(cta, a), f1 = range_start(cta + 1, a);
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < kStages; ++i) {
             tc::mbar_init(&sm.kv_full[i], 33);  // 1 expect_tx arrival + 32 cp.async arrivals
             tc::mbar_init(&sm.kv_empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
             tc::mbar_init(&sm.s_full[i], 1);
             tc::mbar_init(&sm.p_full[i], 128);
             tc::mbar_init(&sm.p_free[i], 1);
@@ -508,13 +546,13 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// [rows][512] bf16, boxes of 64 columns x 64 rows, 128-byte swizzle
-bool make_map(CUtensorMap* map, const void* base, long long rows) {
+// [rows][512] bf16, boxes of 64 columns x box_rows rows, 128-byte swizzle
+bool make_map(CUtensorMap* map, const void* base, long long rows, int box_rows) {
     auto fn = encode_fn();
     if (!fn || rows < 1) return false;
     cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)kD * 2};
-    cuuint32_t box[2] = {64, 64};
+    cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
     cuuint32_t estr[2] = {1, 1};
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -564,13 +602,14 @@ cudaError_t launch_attend_tc(const AttendArgs& a, void* ws, size_t ws_bytes, cud
     const long long ent_rows = (long long)a.batch * a.n_ent;
     const long long tok_rows = (long long)a.batch * a.l_tok;
     const void* tok = a.token_kv ? a.token_kv : a.q;  // a window of 0 never reads it
-    if (!make_map(&tok_map, tok, a.token_kv ? tok_rows : (long long)a.batch * a.n_q * kH)) return cudaErrorInvalidValue;
+    if (!make_map(&tok_map, tok, a.token_kv ? tok_rows : (long long)a.batch * a.n_q * kH, kTile))
+        return cudaErrorInvalidValue;
     if (ent_rows > 0) {
-        if (!make_map(&ent_map, a.entries, ent_rows)) return cudaErrorInvalidValue;
+        if (!make_map(&ent_map, a.entries, ent_rows, kTile)) return cudaErrorInvalidValue;
     } else {
         ent_map = tok_map;  // no entry tiles exist
     }
-    if (!make_map(&q_map, a.q, (long long)a.batch * a.n_q * kH)) return cudaErrorInvalidValue;
+    if (!make_map(&q_map, a.q, (long long)a.batch * a.n_q * kH, kH)) return cudaErrorInvalidValue;
 
     TcArgs t;
     t.q = static_cast<const __nv_bfloat16*>(a.q);

@@ -5,11 +5,13 @@
 // logits Z) weighted sum of the content rows C.  One launch compresses both the
 // K=V stream and, optionally, the indexer-key stream of the same chunks.
 //
-// Mapping: one thread owns 8 consecutive channels of one entry and streams the
-// chunk's m tokens with 16-byte vector loads (two for fp32), keeping a running
-// max / denominator / numerator per channel in registers (online softmax).
-// The threads of one entry are consecutive lanes of one warp, so an FP8 output
-// finds the entry's amax with warp shuffles.
+// Mapping: S adjacent lanes (S = min(m, 16), a power of two; 1 for FP8
+// output) own 8 consecutive channels of one entry; each streams every S-th
+// token of the chunk with 16-byte vector loads (two for fp32), keeping a
+// running max / denominator / numerator per channel in registers (online
+// softmax), and the S partial states are merged with butterfly shuffles.  For
+// FP8 output the lanes of one entry are consecutive lanes of one warp, so the
+// entry's amax is found with warp shuffles too.
 #include "common.cuh"
 #include "internal.h"
 
@@ -22,23 +24,17 @@ struct StreamDesc {
     void* out;
     float* out_scale;
     int channels, groups;  // groups = channels / 8
+    int split;             // S: lanes sharing one (entry, channel group)
     int in_dtype, out_dtype;
     long long x_bs, gate_bs, out_bs, scale_bs;
 };
 
 template <typename T>
-__device__ __forceinline__ void compress_group(const StreamDesc& d, int b, long long s, int grp, int m,
-                                               float out[8]) {
+__device__ __forceinline__ void compress_group(const StreamDesc& d, int b, long long s, int grp, int m, int sub,
+                                               float mx[8], float den[8], float num[8]) {
     const T* xp = static_cast<const T*>(d.x) + (long long)b * d.x_bs + s * m * d.channels + grp * 8;
     const T* zp = static_cast<const T*>(d.gate) + (long long)b * d.gate_bs + s * m * d.channels + grp * 8;
-    float mx[8], den[8], num[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-        mx[e] = -INFINITY;
-        den[e] = 0.f;
-        num[e] = 0.f;
-    }
-    for (int i = 0; i < m; ++i) {
+    for (int i = sub; i < m; i += d.split) {
         float xv[8], zv[8];
         Vec8<T>::load_nc(xp + (long long)i * d.channels, xv);
         Vec8<T>::load_nc(zp + (long long)i * d.channels, zv);
@@ -52,32 +48,54 @@ __device__ __forceinline__ void compress_group(const StreamDesc& d, int b, long 
             mx[e] = nm;
         }
     }
-#pragma unroll
-    for (int e = 0; e < 8; ++e) out[e] = num[e] / den[e];
 }
 
 __global__ void __launch_bounds__(256) compress_kernel(StreamDesc s0, StreamDesc s1, int batch, long long n_ent,
                                                        int m) {
     const StreamDesc& d = blockIdx.y == 0 ? s0 : s1;
-    long long total = (long long)batch * n_ent * d.groups;
+    const long long per_entry = (long long)d.groups * d.split;
+    long long total = (long long)batch * n_ent * per_entry;
     long long g = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     bool active = g < total;
     long long gg = active ? g : 0;
-    int b = (int)(gg / (n_ent * d.groups));
-    long long rem = gg % (n_ent * d.groups);
+    const int sub = (int)(gg % d.split);
+    int b = (int)(gg / (n_ent * per_entry));
+    long long rem = (gg % (n_ent * per_entry)) / d.split;
     long long s = rem / d.groups;
     int grp = (int)(rem % d.groups);
 
-    float out[8];
+    float mx[8], den[8], num[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        mx[e] = -INFINITY;
+        den[e] = 0.f;
+        num[e] = 0.f;
+    }
     if (active) {
         if (d.in_dtype == V4A_BF16)
-            compress_group<__nv_bfloat16>(d, b, s, grp, m, out);
+            compress_group<__nv_bfloat16>(d, b, s, grp, m, sub, mx, den, num);
         else
-            compress_group<float>(d, b, s, grp, m, out);
-    } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) out[e] = 0.f;
+            compress_group<float>(d, b, s, grp, m, sub, mx, den, num);
     }
+    // merge the S lanes' partial softmax states (S adjacent lanes, S a power of two)
+    for (int o = d.split / 2; o > 0; o >>= 1) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const float m2 = __shfl_xor_sync(0xffffffffu, mx[e], o);
+            const float d2 = __shfl_xor_sync(0xffffffffu, den[e], o);
+            const float n2 = __shfl_xor_sync(0xffffffffu, num[e], o);
+            const float nm = fmaxf(mx[e], m2);
+            const float a1 = nm == -INFINITY ? 0.f : expf(mx[e] - nm);
+            const float a2 = nm == -INFINITY ? 0.f : expf(m2 - nm);
+            den[e] = den[e] * a1 + d2 * a2;
+            num[e] = num[e] * a1 + n2 * a2;
+            mx[e] = nm;
+        }
+    }
+    float out[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) out[e] = active ? num[e] / den[e] : 0.f;
+    if (sub != 0) return;
 
     if (d.out_dtype == V4A_FP8E4M3) {
         // per-entry amax over the entry's `groups` consecutive lanes (a power of two <= 32)
@@ -114,6 +132,7 @@ StreamDesc describe(const v4a_compress_io* io) {
     d.out_scale = io->out_scale;
     d.channels = io->channels;
     d.groups = io->channels / 8;
+    d.split = 1;
     d.in_dtype = io->in_dtype;
     d.out_dtype = io->out_dtype;
     d.x_bs = io->x_batch_stride;
@@ -131,8 +150,14 @@ cudaError_t launch_compress(const v4a_compress_io* kv, const v4a_compress_io* id
     if (batch == 0 || n_ent == 0) return cudaSuccess;
     StreamDesc s0 = describe(kv);
     StreamDesc s1 = idx ? describe(idx) : s0;
-    long long groups = s0.groups > s1.groups ? s0.groups : s1.groups;
-    long long total = (long long)batch * n_ent * groups;
+    // lanes per (entry, channel group): enough to spread long chunks, 1 for FP8 output
+    // (its per-entry amax runs over the entry's consecutive lanes)
+    int split = 1;
+    while (split < 16 && split * 2 <= m) split *= 2;
+    if (s0.out_dtype != V4A_FP8E4M3) s0.split = split;
+    if (s1.out_dtype != V4A_FP8E4M3) s1.split = split;
+    long long w0 = (long long)s0.groups * s0.split, w1 = (long long)s1.groups * s1.split;
+    long long total = (long long)batch * n_ent * (w0 > w1 ? w0 : w1);
     const int threads = 256;
     dim3 grid((unsigned)((total + threads - 1) / threads), idx ? 2 : 1);
     compress_kernel<<<grid, threads, 0, stream>>>(s0, s1, batch, n_ent, m);
