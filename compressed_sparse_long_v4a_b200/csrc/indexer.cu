@@ -132,21 +132,30 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_buf, int* t
     return r;
 }
 
-// one block per query row; scores[row][N] with -inf beyond N_vis
-__global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* scores, IndexArgs a, int k,
-                                                                   int32_t* idx_out, float* score_out) {
+// sum of v over the threads with a larger index (the block total in *total)
+__device__ __forceinline__ int block_exclusive_scan_rev(int v, int* warp_buf, int* total) {
+    // scan in reversed thread order by scanning the mirrored value
+    const int n = blockDim.x;
+    __shared__ int mirror[1024];
+    mirror[n - 1 - threadIdx.x] = v;
+    __syncthreads();
+    const int mv = mirror[threadIdx.x];
+    __syncthreads();
+    const int ex = block_exclusive_scan(mv, warp_buf, total);
+    mirror[threadIdx.x] = ex;
+    __syncthreads();
+    const int r = mirror[n - 1 - threadIdx.x];
+    __syncthreads();
+    return r;
+}
+
+// Exact radix select of one row (scores[0..nvis), -inf never selected): the
+// min(k, nvis) largest, ties to the lower entry, written in ascending entry
+// order and padded with -1.  Called by a whole block of kSelThreads threads.
+__device__ void select_row_radix(const float* sc, long long nvis, int k, int32_t* io, float* so) {
     __shared__ unsigned int hist[256];
     __shared__ int warp_buf[33];
     __shared__ unsigned int sh_digit, sh_above;
-    const int row = blockIdx.x;
-    const int j = row % a.n_q;
-    const long long t = a.ctx_len - a.n_q + j;
-    long long nvis = n_visible(t, a.m);
-    if (nvis > a.n_ent) nvis = a.n_ent;
-    const float* sc = scores + (long long)row * a.n_ent;
-    int32_t* io = idx_out + (long long)row * k;
-    float* so = score_out ? score_out + (long long)row * k : nullptr;
-
     uint32_t prefix = 0, mask = 0;
     long long need = k;  // how many entries with key == prefix (so far) are still wanted
     const bool all = nvis <= k;
@@ -203,6 +212,248 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* s
     }
 }
 
+__device__ __forceinline__ long long row_nvis(const IndexArgs& a, int row) {
+    const long long t = a.ctx_len - a.n_q + (row % a.n_q);
+    long long nvis = n_visible(t, a.m);
+    return nvis > a.n_ent ? a.n_ent : nvis;
+}
+
+// one block per query row; scores[row][N] with -inf beyond N_vis
+__global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* scores, IndexArgs a, int k,
+                                                                   int32_t* idx_out, float* score_out) {
+    const int row = blockIdx.x;
+    select_row_radix(scores + (long long)row * a.n_ent, row_nvis(a, row), k, idx_out + (long long)row * k,
+                     score_out ? score_out + (long long)row * k : nullptr);
+}
+
+// ---------------------------------------------------------------------
+// select for few query rows: histogram threshold, multi-block scan, final
+// ---------------------------------------------------------------------
+constexpr int kHistBins = 4096;  // top 12 bits of the ordered key (built by the score kernels)
+constexpr int kScanThreads = 256;
+constexpr int kMaxFastRows = 256;
+constexpr int kMaxParts = 512;
+constexpr int kCandCap = 20480;  // candidates the final kernel holds in shared memory
+
+// The bin holding the k-th largest key: its index, and how many keys lie in higher bins.
+// Every thread of the block gets the answer; `all` when at most k keys exist.
+__device__ void threshold_bin(const uint32_t* hist_row, int k, int* bin, int* above, bool* all) {
+    __shared__ int sb, sa, stot;
+    __shared__ int warp_buf[33];
+    const int per = kHistBins / blockDim.x;  // bins per thread (blockDim divides 4096)
+    const int b0 = threadIdx.x * per;
+    int local = 0;
+    for (int i = 0; i < per; ++i) local += (int)hist_row[b0 + i];
+    // exclusive scan over threads in DESCENDING bin order: reverse the thread index
+    int total;
+    const int rev = block_exclusive_scan_rev(local, warp_buf, &total);  // sum over higher-bin threads
+    if (threadIdx.x == 0) {
+        sb = -1;
+        sa = 0;
+        stot = total;
+    }
+    __syncthreads();
+    int run = rev;
+    for (int i = per - 1; i >= 0; --i) {
+        const int c = (int)hist_row[b0 + i];
+        if (run < k && run + c >= k) {
+            sb = b0 + i;
+            sa = run;
+        }
+        run += c;
+    }
+    __syncthreads();
+    *bin = sb;
+    *above = sa;
+    *all = stot <= k;
+    __syncthreads();
+}
+
+__global__ void __launch_bounds__(kScanThreads) topk_scan_kernel(const float* scores, const uint32_t* hist, IndexArgs a,
+                                                                  int k, int parts, long long chunk, int32_t* def_buf,
+                                                                  int32_t* cidx_buf, uint32_t* ckey_buf, int* counts) {
+    __shared__ int warp_buf[33];
+    const int row = blockIdx.x / parts, p = blockIdx.x % parts;
+    const long long nvis = row_nvis(a, row);
+    int tbin, above;
+    bool all;
+    threshold_bin(hist + (long long)row * kHistBins, k, &tbin, &above, &all);
+    const float* sc = scores + (long long)row * a.n_ent;
+    const long long lo = (long long)p * chunk;
+    long long hi = lo + chunk;
+    if (hi > nvis) hi = nvis;
+    int32_t* dout = def_buf + (long long)row * a.n_ent + lo;
+    int32_t* ciout = cidx_buf + (long long)row * a.n_ent + lo;
+    uint32_t* ckout = ckey_buf + (long long)row * a.n_ent + lo;
+    int n_def = 0, n_cand = 0;
+    for (long long base = lo; base < hi; base += blockDim.x) {
+        const long long s = base + threadIdx.x;
+        const bool in = s < hi;
+        const uint32_t key = in ? float_to_ordered(sc[s]) : 0u;
+        const int bin = (int)(key >> 20);
+        const int def = (in && (all || bin > tbin)) ? 1 : 0;
+        const int cand = (in && !all && bin == tbin) ? 1 : 0;
+        int tot;
+        const int packed = block_exclusive_scan(def | (cand << 16), warp_buf, &tot);
+        if (def) dout[n_def + (packed & 0xffff)] = (int32_t)s;
+        if (cand) {
+            ciout[n_cand + (packed >> 16)] = (int32_t)s;
+            ckout[n_cand + (packed >> 16)] = key;
+        }
+        n_def += tot & 0xffff;
+        n_cand += tot >> 16;
+    }
+    if (threadIdx.x == 0) {
+        counts[((long long)row * parts + p) * 2] = n_def;
+        counts[((long long)row * parts + p) * 2 + 1] = n_cand;
+    }
+}
+
+// first position in sorted v[0..n) holding a value >= x
+__device__ __forceinline__ int lower_bound(const int32_t* v, int n, int32_t x) {
+    int lo = 0, hi = n;
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (v[mid] < x) lo = mid + 1;
+        else hi = mid;
+    }
+    return lo;
+}
+
+// one block (kSelThreads) per query row
+__global__ void __launch_bounds__(kSelThreads) topk_final_kernel(const float* scores, IndexArgs a, int k, int parts,
+                                                                  long long chunk, const int32_t* def_buf,
+                                                                  const int32_t* cidx_buf, const uint32_t* ckey_buf,
+                                                                  const int* counts, int32_t* idx_out,
+                                                                  float* score_out) {
+    extern __shared__ uint32_t fs[];
+    uint32_t* ckey = fs;                                      // [kCandCap]
+    int32_t* cidx = reinterpret_cast<int32_t*>(fs + kCandCap);  // [kCandCap]
+    int32_t* defs = cidx + kCandCap;                          // [4096]
+    int32_t* sels = defs + 4096;                              // [4096]
+    __shared__ int doff[kMaxParts + 1], coff[kMaxParts + 1];
+    __shared__ unsigned int h1[1024];
+    __shared__ int warp_buf[33];
+    __shared__ uint32_t s_prefix;
+    __shared__ int s_need;
+
+    const int row = blockIdx.x;
+    const long long nvis = row_nvis(a, row);
+    int32_t* io = idx_out + (long long)row * k;
+    float* so = score_out ? score_out + (long long)row * k : nullptr;
+    const float* sc = scores + (long long)row * a.n_ent;
+    for (int p = threadIdx.x; p < parts; p += blockDim.x) {
+        doff[p + 1] = counts[((long long)row * parts + p) * 2];
+        coff[p + 1] = counts[((long long)row * parts + p) * 2 + 1];
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        doff[0] = coff[0] = 0;
+        for (int p = 1; p <= parts; ++p) {
+            doff[p] += doff[p - 1];
+            coff[p] += coff[p - 1];
+        }
+    }
+    __syncthreads();
+    const int D = doff[parts], C = coff[parts];
+    if (C > kCandCap || D > 4096) {
+        // more candidates than the fast path holds (e.g. huge blocks of equal scores): exact select over the row
+        select_row_radix(sc, nvis, k, io, so);
+        return;
+    }
+    // gather the definite entries and the candidates, both in ascending entry order; every element
+    // finds its part by binary search over the offsets, so all loads are independent
+    const long long row_off = (long long)row * a.n_ent;
+    for (int e = threadIdx.x; e < D + C; e += blockDim.x) {
+        const bool is_def = e < D;
+        const int x = is_def ? e : e - D;
+        const int* off = is_def ? doff : coff;
+        int lo = 0, hi = parts;  // largest p with off[p] <= x
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (off[mid] <= x) lo = mid;
+            else hi = mid;
+        }
+        const long long src = row_off + (long long)lo * chunk + (x - off[lo]);
+        if (is_def) {
+            defs[x] = def_buf[src];
+        } else {
+            cidx[x] = cidx_buf[src];
+            ckey[x] = ckey_buf[src];
+        }
+    }
+    const int need = (D + C) < k ? C : k - D;  // candidates to take
+    __syncthreads();
+    // radix select of the need-th largest candidate key over its low 20 bits (the top 12 are equal)
+    uint32_t prefix = C > 0 ? (ckey[0] & 0xfff00000u) : 0u, mask = 0xfff00000u;
+    int rem = need;
+    if (need > 0 && need < C) {
+        for (int shift = 10; shift >= 0; shift -= 10) {
+            for (int i = threadIdx.x; i < 1024; i += blockDim.x) h1[i] = 0;
+            __syncthreads();
+            for (int i = threadIdx.x; i < C; i += blockDim.x)
+                if ((ckey[i] & mask) == prefix) atomicAdd(&h1[(ckey[i] >> shift) & 1023u], 1u);
+            __syncthreads();
+            if (threadIdx.x == 0) {
+                unsigned int above = 0;
+                int dgt = 1023;
+                for (; dgt > 0; --dgt) {
+                    if (above + h1[dgt] >= (unsigned int)rem) break;
+                    above += h1[dgt];
+                }
+                s_prefix = prefix | ((uint32_t)dgt << shift);
+                s_need = rem - (int)above;
+            }
+            __syncthreads();
+            prefix = s_prefix;
+            rem = s_need;
+            mask |= 1023u << shift;
+            __syncthreads();
+        }
+    }
+    // mark: key > prefix, or key == prefix among the first `rem` such (in entry order)
+    const bool take_all = need >= C;
+    int out = 0, eq_seen = 0;
+    for (int base = 0; base < C; base += blockDim.x) {
+        const int i = base + threadIdx.x;
+        const bool in = i < C;
+        const uint32_t key = in ? ckey[i] : 0u;
+        const int gt = (in && (take_all || key > prefix)) ? 1 : 0;
+        const int eq = (in && !take_all && key == prefix) ? 1 : 0;
+        int eq_tot;
+        const int eq_rank = eq_seen + block_exclusive_scan(eq, warp_buf, &eq_tot);
+        const int sel = gt | ((eq && eq_rank < rem) ? 1 : 0);
+        int sel_tot;
+        const int pos = out + block_exclusive_scan(sel, warp_buf, &sel_tot);
+        if (sel) {
+            sels[pos] = cidx[i];
+            ckey[pos] = key;  // compacted in place: pos <= i
+        }
+        __syncthreads();
+        out += sel_tot;
+        eq_seen += eq_tot;
+    }
+    __syncthreads();
+    const int total = D + out;
+    // merge the two ascending lists into the output
+    for (int i = threadIdx.x; i < D; i += blockDim.x) {
+        const int32_t x = defs[i];
+        const int pos = i + lower_bound(sels, out, x);
+        io[pos] = x;
+        if (so) so[pos] = sc[x];
+    }
+    for (int j = threadIdx.x; j < out; j += blockDim.x) {
+        const int32_t y = sels[j];
+        const int pos = j + lower_bound(defs, D, y);
+        io[pos] = y;
+        if (so) so[pos] = ordered_to_float(ckey[j]);
+    }
+    for (int p = total + threadIdx.x; p < k; p += blockDim.x) {
+        io[p] = -1;
+        if (so) so[p] = -INFINITY;
+    }
+}
+
 template <int HMAX>
 cudaError_t launch_scores_h(const IndexArgs& a, float* scores, cudaStream_t stream) {
     long long nblk = (a.n_ent + kScoreThreads - 1) / kScoreThreads;
@@ -231,10 +482,62 @@ cudaError_t launch_scores_h(const IndexArgs& a, float* scores, cudaStream_t stre
     return cudaGetLastError();
 }
 
+
+// How the select is done for a shape: few query rows take the histogram /
+// multi-block scan / final path; many rows take one radix-select block per row.
+struct TopkPlan {
+    bool fast;
+    int parts;
+    long long chunk;
+    size_t off_hist, off_cnt, off_def, off_cidx, off_ckey, total;
+};
+
+static size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+static TopkPlan topk_plan(const IndexArgs& a) {
+    TopkPlan p = {};
+    const long long rows = (long long)a.batch * a.n_q;
+    const long long n = a.n_ent > 0 ? a.n_ent : 1;
+    size_t off = align256((size_t)rows * n * sizeof(float));  // scores
+    p.fast = rows >= 1 && rows <= kMaxFastRows;
+    if (!p.fast) {
+        p.total = off;
+        return p;
+    }
+    long long parts = (2LL * kNumSMs + rows - 1) / rows;
+    const long long max_parts = (n + 1023) / 1024;
+    if (parts > max_parts) parts = max_parts;
+    if (parts > kMaxParts) parts = kMaxParts;
+    if (parts < 1) parts = 1;
+    p.parts = (int)parts;
+    p.chunk = ((n + parts - 1) / parts + kScanThreads - 1) / kScanThreads * kScanThreads;
+    p.off_hist = off;
+    off = align256(off + (size_t)rows * kHistBins * sizeof(uint32_t));
+    p.off_cnt = off;
+    off = align256(off + (size_t)rows * p.parts * 2 * sizeof(int));
+    p.off_def = off;
+    off = align256(off + (size_t)rows * n * sizeof(int32_t));
+    p.off_cidx = off;
+    off = align256(off + (size_t)rows * n * sizeof(int32_t));
+    p.off_ckey = off;
+    off = align256(off + (size_t)rows * n * sizeof(uint32_t));
+    p.total = off;
+    return p;
+}
+
+// histogram of the order-preserving keys' top 12 bits, for the CUDA-core score path
+__global__ void score_hist_kernel(const float* scores, IndexArgs a, uint32_t* hist) {
+    const int row = blockIdx.y;
+    const long long nvis = row_nvis(a, row);
+    for (long long s = (long long)blockIdx.x * blockDim.x + threadIdx.x; s < nvis; s += (long long)gridDim.x * blockDim.x)
+        atomicAdd(&hist[(long long)row * kHistBins + (float_to_ordered(scores[(long long)row * a.n_ent + s]) >> 20)], 1u);
+}
+
 }  // namespace
 
 cudaError_t launch_index_scores(const IndexArgs& a, float* scores, cudaStream_t stream) {
     if (a.batch == 0 || a.n_ent == 0) return cudaSuccess;
+    if (index_tc_available(a)) return launch_index_scores_tc(a, scores, nullptr, nullptr, stream);
     if (a.heads_i <= 4) return launch_scores_h<4>(a, scores, stream);
     if (a.heads_i <= 8) return launch_scores_h<8>(a, scores, stream);
     if (a.heads_i <= 16) return launch_scores_h<16>(a, scores, stream);
@@ -244,20 +547,52 @@ cudaError_t launch_index_scores(const IndexArgs& a, float* scores, cudaStream_t 
 
 size_t topk_workspace_bytes(const IndexArgs& a, int k) {
     (void)k;
-    size_t n = (size_t)a.batch * (size_t)a.n_q * (size_t)(a.n_ent > 0 ? a.n_ent : 1);
-    return ((n * sizeof(float) + 255) / 256) * 256;
+    return topk_plan(a).total;
 }
 
 cudaError_t launch_topk(const IndexArgs& a, int k, int32_t* idx_out, float* score_out, void* ws, size_t ws_bytes,
                         cudaStream_t stream) {
     if (a.batch == 0) return cudaSuccess;
-    if (ws_bytes < topk_workspace_bytes(a, k)) return cudaErrorInvalidValue;
-    float* scores = static_cast<float*>(ws);
-    if (a.n_ent > 0) {
-        cudaError_t e = launch_index_scores(a, scores, stream);
-        if (e != cudaSuccess) return e;
+    const TopkPlan p = topk_plan(a);
+    if (ws_bytes < p.total) return cudaErrorInvalidValue;
+    char* base = static_cast<char*>(ws);
+    float* scores = reinterpret_cast<float*>(base);
+    const int rows = a.batch * a.n_q;
+    cudaError_t e;
+    if (!p.fast || a.n_ent == 0) {
+        if (a.n_ent > 0) {
+            e = launch_index_scores(a, scores, stream);
+            if (e != cudaSuccess) return e;
+        }
+        topk_select_kernel<<<rows, kSelThreads, 0, stream>>>(scores, a, k, idx_out, score_out);
+        return cudaGetLastError();
     }
-    topk_select_kernel<<<a.batch * a.n_q, kSelThreads, 0, stream>>>(scores, a, k, idx_out, score_out);
+    uint32_t* hist = reinterpret_cast<uint32_t*>(base + p.off_hist);
+    int* counts = reinterpret_cast<int*>(base + p.off_cnt);
+    int32_t* def_buf = reinterpret_cast<int32_t*>(base + p.off_def);
+    int32_t* cidx = reinterpret_cast<int32_t*>(base + p.off_cidx);
+    uint32_t* ckey = reinterpret_cast<uint32_t*>(base + p.off_ckey);
+    e = cudaMemsetAsync(hist, 0, (size_t)rows * kHistBins * sizeof(uint32_t), stream);
+    if (e != cudaSuccess) return e;
+    if (index_tc_available(a)) {
+        e = launch_index_scores_tc(a, scores, hist, nullptr, stream);
+    } else {
+        e = launch_index_scores(a, scores, stream);
+        if (e == cudaSuccess) {
+            score_hist_kernel<<<dim3(64, rows), 256, 0, stream>>>(scores, a, hist);
+            e = cudaGetLastError();
+        }
+    }
+    if (e != cudaSuccess) return e;
+    topk_scan_kernel<<<rows * p.parts, kScanThreads, 0, stream>>>(scores, hist, a, k, p.parts, p.chunk, def_buf, cidx,
+                                                                   ckey, counts);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const size_t smem = (size_t)kCandCap * 8 + 2 * 4096 * sizeof(int32_t);
+    e = cudaFuncSetAttribute(topk_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    topk_final_kernel<<<rows, kSelThreads, smem, stream>>>(scores, a, k, p.parts, p.chunk, def_buf, cidx, ckey, counts,
+                                                           idx_out, score_out);
     return cudaGetLastError();
 }
 

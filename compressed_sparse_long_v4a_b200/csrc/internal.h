@@ -29,6 +29,12 @@ struct IndexArgs {
 
 // every score (-inf where not visible) into scores[row][N], row = b*n_q + j
 cudaError_t launch_index_scores(const IndexArgs& a, float* scores, cudaStream_t stream);
+
+// ---- indexer_tc.cu (tcgen05 scores: d_i = 128, heads_i <= 32, bf16 q, bf16/fp8 keys) ----
+bool index_tc_shape_ok(const IndexArgs& a);
+bool index_tc_available(const IndexArgs& a);
+// scores as launch_index_scores; hist (nullable) [rows][4096] += counts of the scores' ordered-key top 12 bits
+cudaError_t launch_index_scores_tc(const IndexArgs& a, float* scores, uint32_t* hist, int* err, cudaStream_t stream);
 size_t topk_workspace_bytes(const IndexArgs& a, int k);
 cudaError_t launch_topk(const IndexArgs& a, int k, int32_t* idx_out, float* score_out, void* ws, size_t ws_bytes,
                         cudaStream_t stream);

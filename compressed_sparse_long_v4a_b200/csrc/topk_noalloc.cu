@@ -18,7 +18,7 @@
 
 namespace {
 
-constexpr size_t kScratchBytes = 16u << 20;  // 16 MiB: 4 Mi fp32 scores
+constexpr size_t kScratchBytes = 64u << 20;  // 64 MiB
 constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_topk_scratch[kScratchBytes];
@@ -53,9 +53,9 @@ extern "C" v4a_status v4a_topk_noalloc(const void* q_i, const float* w, const vo
     const size_t need = v4a_workspace_size("topk", shape, heads_i, d_i);
     if (need > kScratchBytes)
         return v4a::report(V4A_ERR_INVALID_ARG,
-                           "v4a_topk_noalloc: this shape needs %zu bytes of scratch but the built-in array holds "
-                           "%zu (batch * n_q * ctx_len/m must stay <= %zu); use v4a_topk with a workspace",
-                           need, kScratchBytes, kScratchBytes / sizeof(float));
+                           "v4a_topk_noalloc: this shape needs %zu bytes of scratch (v4a_workspace_size \"topk\") "
+                           "but the built-in array holds %zu; use v4a_topk with a workspace",
+                           need, kScratchBytes);
     void* scratch = nullptr;
     const cudaError_t e = scratch_address(&scratch);
     if (e != cudaSuccess)

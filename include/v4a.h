@@ -155,12 +155,13 @@ V4A_API v4a_status v4a_topk(const void* q_i, const float* w, const void* k_i, co
  * allocation, or a serving loop where allocating is not allowed.  (The pages
  * have no counterpart: this is an interface convenience, not part of the
  * method.)  Arguments, results and errors are those of v4a_topk, except that
- * there is no workspace argument: the scratch is a fixed 16 MiB array
+ * there is no workspace argument: the scratch is a fixed 64 MiB array
  * compiled into the library, which every device that loads the library keeps
  * in its global memory until the process exits.  It bounds the problem size:
- * batch * n_q * (ctx_len / m) must not exceed 4,194,304 (the 1M-context
- * decode of 4 sequences needs 1,048,576); larger shapes return
- * V4A_ERR_INVALID_ARG with the limit in v4a_last_error().
+ * a shape whose v4a_workspace_size("topk", ...) exceeds 64 MiB (about 16
+ * bytes per score, so some 4 million scores per call; the 1M-context decode
+ * of 4 sequences has 1,048,576) returns V4A_ERR_INVALID_ARG with both sizes
+ * in v4a_last_error().
  * The first call made with a given device current looks up the array's
  * device address (cudaGetSymbolAddress) and caches it; make that first call
  * outside any stream capture.  The call itself allocates nothing: no

@@ -67,9 +67,11 @@ def test_no_alloc_topk_refuses_shapes_beyond_its_scratch(v4a):
     k_i = torch.zeros((1, 1, 128), dtype=torch.uint8, device="cuda")
     k_s = torch.ones((1, 1), dtype=torch.float32, device="cuda")
     idx = torch.full((1, 1, 8), -7, dtype=torch.int32, device="cuda")
-    too_long = 4 * ((16 << 20) // 4 + 1)  # one fp32 score more than the 16 MiB scratch holds
+    # a context whose top-k scratch needs more than the built-in 64 MiB
+    too_long = 4 * (8 << 20)
+    assert v4a.v4a_workspace_size("topk", batch=1, m=4, k=8, ctx_len=too_long, heads_i=16, d_i=128) > (64 << 20)
     with pytest.raises(v4a.V4AError) as e:
         v4a.v4a_topk_noalloc(q_i, w, k_i, k_s, idx, m=4, k=8, ctx_len=too_long)
-    assert e.value.status == 1 and "v4a_topk_noalloc" in str(e.value) and "16777216" in str(e.value)
+    assert e.value.status == 1 and "v4a_topk_noalloc" in str(e.value) and str(64 << 20) in str(e.value)
     torch.cuda.synchronize()
     assert (idx == -7).all()  # nothing was launched
