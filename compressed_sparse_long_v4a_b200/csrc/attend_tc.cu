@@ -504,32 +504,62 @@ __global__ void attend_tc_combine(TcArgs a) {
     auto cta_of = [&](long long f) { return (int)(((f + 1) * a.grid - 1) / a.total_tiles); };
     const int c0 = cta_of(rs), c1 = cta_of(re);
     if (c0 == c1) return;  // written directly by its only CTA
-    float mmax = -INFINITY;
-    bool bad = false;
-    for (int c = c0; c <= c1; ++c) {
-        const int slot = 2 * c + ((range_start(c, a) / a.tpr == row) ? 0 : 1);
-        const float ms = a.part_ml[((long long)slot * kH + h) * 2];
-        bad |= isnan(ms);
-        mmax = fmaxf(mmax, ms);
-    }
-    const int e = threadIdx.x * 4;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    float l = 0.f;
-    if (mmax != -INFINITY && !bad) {
-        for (int c = c0; c <= c1; ++c) {
-            const int slot = 2 * c + ((range_start(c, a) / a.tpr == row) ? 0 : 1);
-            const float ms = a.part_ml[((long long)slot * kH + h) * 2];
-            if (ms == -INFINITY) continue;
-            const float w = exp2f(ms - mmax);
-            l += w * a.part_ml[((long long)slot * kH + h) * 2 + 1];
-            const float4 v = *reinterpret_cast<const float4*>(a.part_o + ((long long)slot * kH + h) * kD + e);
-            acc.x = fmaf(w, v.x, acc.x);
-            acc.y = fmaf(w, v.y, acc.y);
-            acc.z = fmaf(w, v.z, acc.z);
-            acc.w = fmaf(w, v.w, acc.w);
+    // the first CTA's piece is its first query only if the query starts its range; every later CTA's
+    // range starts inside this query, so the piece is that CTA's first (slot 2c)
+    constexpr int kPer = 5, kMaxPieces = 32 * kPer;  // covers a query split over every CTA (grid <= 148)
+    const int n = c1 - c0 + 1;
+    __shared__ float s_w[kMaxPieces];
+    __shared__ float s_l;
+    __shared__ int s_bad;
+    if (threadIdx.x < 32) {
+        float ms[kPer], ls[kPer];
+        float mmax = -INFINITY;
+        bool bad = false;
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) {
+            const int i = threadIdx.x + 32 * u;
+            ms[u] = -INFINITY;
+            ls[u] = 0.f;
+            if (i < n) {
+                const int c = c0 + i;
+                const int slot = 2 * c + ((i == 0 && range_start(c0, a) < rs) ? 1 : 0);
+                ms[u] = a.part_ml[((long long)slot * kH + h) * 2];
+                ls[u] = a.part_ml[((long long)slot * kH + h) * 2 + 1];
+                bad |= isnan(ms[u]) || isnan(ls[u]);
+                mmax = fmaxf(mmax, ms[u]);
+            }
+        }
+        mmax = group_max<32>(mmax);
+        bad = __any_sync(0xffffffffu, bad);
+        float l = 0.f;
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) {
+            const int i = threadIdx.x + 32 * u;
+            const float wgt = (i < n && ms[u] != -INFINITY && mmax != -INFINITY) ? exp2f(ms[u] - mmax) : 0.f;
+            if (i < n) s_w[i] = wgt;
+            l += wgt * ls[u];
+        }
+        l = group_sum<32>(l);
+        if (threadIdx.x == 0) {
+            s_l = l;
+            s_bad = bad;
         }
     }
-    const float inv = bad ? NAN : (l > 0.f ? 1.f / l : 0.f);
+    __syncthreads();
+    const int e = threadIdx.x * 4;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int i = 0; i < n; ++i) {
+        const float wgt = s_w[i];
+        if (wgt == 0.f) continue;
+        const int c = c0 + i;
+        const int slot = 2 * c + ((i == 0 && range_start(c0, a) < rs) ? 1 : 0);
+        const float4 v = *reinterpret_cast<const float4*>(a.part_o + ((long long)slot * kH + h) * kD + e);
+        acc.x = fmaf(wgt, v.x, acc.x);
+        acc.y = fmaf(wgt, v.y, acc.y);
+        acc.z = fmaf(wgt, v.z, acc.z);
+        acc.w = fmaf(wgt, v.w, acc.w);
+    }
+    const float inv = s_bad ? NAN : (s_l > 0.f ? 1.f / s_l : 0.f);
     *reinterpret_cast<float4*>(a.out + ((long long)row * kH + h) * kD + e) =
         make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
 }

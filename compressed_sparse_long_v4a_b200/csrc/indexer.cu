@@ -149,13 +149,37 @@ __device__ __forceinline__ int block_exclusive_scan_rev(int v, int* warp_buf, in
     return r;
 }
 
+// The digit d of a histogram (bins 0..nbins-1, nbins <= blockDim.x) at which
+// the count of keys in bins above d stays below `rem` while bins >= d reach it;
+// *above = count above d.  One bin per thread, block-wide suffix scan.
+__device__ void find_digit(const unsigned int* h, int nbins, long long rem, int* digit, long long* above) {
+    __shared__ int s_dgt;
+    __shared__ long long s_above;
+    __shared__ int warp_buf[33];
+    const int c = threadIdx.x < nbins ? (int)h[threadIdx.x] : 0;
+    int tot;
+    const int hi_sum = block_exclusive_scan_rev(c, warp_buf, &tot);  // keys in bins above this thread's
+    if (threadIdx.x == 0) {
+        s_dgt = 0;
+        s_above = 0;
+    }
+    __syncthreads();
+    if (threadIdx.x < nbins && hi_sum < rem && (long long)hi_sum + c >= rem) {
+        s_dgt = threadIdx.x;
+        s_above = hi_sum;
+    }
+    __syncthreads();
+    *digit = s_dgt;
+    *above = s_above;
+    __syncthreads();
+}
+
 // Exact radix select of one row (scores[0..nvis), -inf never selected): the
 // min(k, nvis) largest, ties to the lower entry, written in ascending entry
 // order and padded with -1.  Called by a whole block of kSelThreads threads.
 __device__ void select_row_radix(const float* sc, long long nvis, int k, int32_t* io, float* so) {
     __shared__ unsigned int hist[256];
     __shared__ int warp_buf[33];
-    __shared__ unsigned int sh_digit, sh_above;
     uint32_t prefix = 0, mask = 0;
     long long need = k;  // how many entries with key == prefix (so far) are still wanted
     const bool all = nvis <= k;
@@ -168,21 +192,12 @@ __device__ void select_row_radix(const float* sc, long long nvis, int k, int32_t
                 if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
             }
             __syncthreads();
-            if (threadIdx.x == 0) {
-                unsigned int above = 0;
-                int dgt = 255;
-                for (; dgt > 0; --dgt) {
-                    if (above + hist[dgt] >= (unsigned int)need) break;
-                    above += hist[dgt];
-                }
-                sh_digit = (unsigned int)dgt;
-                sh_above = above;
-            }
-            __syncthreads();
-            prefix |= sh_digit << shift;
+            int dgt;
+            long long above;
+            find_digit(hist, 256, need, &dgt, &above);
+            prefix |= (uint32_t)dgt << shift;
             mask |= 255u << shift;
-            need -= sh_above;
-            __syncthreads();
+            need -= above;
         }
     }
     // ordered compaction: key > prefix, or key == prefix among the first `need` such entries
@@ -286,22 +301,34 @@ __global__ void __launch_bounds__(kScanThreads) topk_scan_kernel(const float* sc
     int32_t* ciout = cidx_buf + (long long)row * a.n_ent + lo;
     uint32_t* ckout = ckey_buf + (long long)row * a.n_ent + lo;
     int n_def = 0, n_cand = 0;
-    for (long long base = lo; base < hi; base += blockDim.x) {
-        const long long s = base + threadIdx.x;
-        const bool in = s < hi;
-        const uint32_t key = in ? float_to_ordered(sc[s]) : 0u;
-        const int bin = (int)(key >> 20);
-        const int def = (in && (all || bin > tbin)) ? 1 : 0;
-        const int cand = (in && !all && bin == tbin) ? 1 : 0;
-        int tot;
-        const int packed = block_exclusive_scan(def | (cand << 16), warp_buf, &tot);
-        if (def) dout[n_def + (packed & 0xffff)] = (int32_t)s;
-        if (cand) {
-            ciout[n_cand + (packed >> 16)] = (int32_t)s;
-            ckout[n_cand + (packed >> 16)] = key;
+    constexpr int kPer = 16;  // scores per thread loaded ahead of the compaction
+    for (long long base0 = lo; base0 < hi; base0 += (long long)kPer * blockDim.x) {
+        uint32_t keys[kPer];
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) {
+            const long long s = base0 + (long long)i * blockDim.x + threadIdx.x;
+            keys[i] = s < hi ? float_to_ordered(sc[s]) : 0u;
         }
-        n_def += tot & 0xffff;
-        n_cand += tot >> 16;
+#pragma unroll 1
+        for (int i = 0; i < kPer; ++i) {
+            const long long base = base0 + (long long)i * blockDim.x;
+            if (base >= hi) break;
+            const long long s = base + threadIdx.x;
+            const bool in = s < hi;
+            const uint32_t key = keys[i];
+            const int bin = (int)(key >> 20);
+            const int def = (in && (all || bin > tbin)) ? 1 : 0;
+            const int cand = (in && !all && bin == tbin) ? 1 : 0;
+            int tot;
+            const int packed = block_exclusive_scan(def | (cand << 16), warp_buf, &tot);
+            if (def) dout[n_def + (packed & 0xffff)] = (int32_t)s;
+            if (cand) {
+                ciout[n_cand + (packed >> 16)] = (int32_t)s;
+                ckout[n_cand + (packed >> 16)] = key;
+            }
+            n_def += tot & 0xffff;
+            n_cand += tot >> 16;
+        }
     }
     if (threadIdx.x == 0) {
         counts[((long long)row * parts + p) * 2] = n_def;
@@ -334,8 +361,6 @@ __global__ void __launch_bounds__(kSelThreads) topk_final_kernel(const float* sc
     __shared__ int doff[kMaxParts + 1], coff[kMaxParts + 1];
     __shared__ unsigned int h1[1024];
     __shared__ int warp_buf[33];
-    __shared__ uint32_t s_prefix;
-    __shared__ int s_need;
 
     const int row = blockIdx.x;
     const long long nvis = row_nvis(a, row);
@@ -394,21 +419,12 @@ __global__ void __launch_bounds__(kSelThreads) topk_final_kernel(const float* sc
             for (int i = threadIdx.x; i < C; i += blockDim.x)
                 if ((ckey[i] & mask) == prefix) atomicAdd(&h1[(ckey[i] >> shift) & 1023u], 1u);
             __syncthreads();
-            if (threadIdx.x == 0) {
-                unsigned int above = 0;
-                int dgt = 1023;
-                for (; dgt > 0; --dgt) {
-                    if (above + h1[dgt] >= (unsigned int)rem) break;
-                    above += h1[dgt];
-                }
-                s_prefix = prefix | ((uint32_t)dgt << shift);
-                s_need = rem - (int)above;
-            }
-            __syncthreads();
-            prefix = s_prefix;
-            rem = s_need;
+            int dgt;
+            long long above;
+            find_digit(h1, 1024, rem, &dgt, &above);
+            prefix |= (uint32_t)dgt << shift;
+            rem -= (int)above;
             mask |= 1023u << shift;
-            __syncthreads();
         }
     }
     // mark: key > prefix, or key == prefix among the first `rem` such (in entry order)

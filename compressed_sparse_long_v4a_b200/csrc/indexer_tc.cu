@@ -220,8 +220,9 @@ __device__ void idx_epilogue(IdxSmem& sm, const IdxTcArgs& a, uint32_t tmem, lon
     int seg = 0;
     long long nvis = 0;
     ICursor cur(f0, a.tiles_per_row);
-    // pending epilogue (tile j-1)
+    // pending epilogue (tile j-1), with its entry's scale loaded ahead
     int p_row = -1, p_ti = 0, p_jt = -1;
+    float p_scale = 1.f;
     auto epilogue = [&](int jt, int row, int ti) -> bool {
         const int s = jt & 1;
         if (!tc::mbar_wait(&sm.d_full[s], (jt >> 1) & 1)) return false;
@@ -242,7 +243,7 @@ __device__ void idx_epilogue(IdxSmem& sm, const IdxTcArgs& a, uint32_t tmem, lon
 #pragma unroll
                 for (int h = 0; h < 32; ++h)
                     if (h < a.heads_i) acc = fmaf(sm.wq[h], fmaxf(__uint_as_float(dv[h]), 0.f), acc);
-                if (FP8) acc *= a.kscale[(long long)(row / a.n_q) * a.n_ent + e];
+                if (FP8) acc *= p_scale;
                 sc = acc + 0.0f;
                 if (a.hist) atomicAdd(&sm.hist[float_to_ordered(sc) >> 20], 1u);
             }
@@ -298,11 +299,18 @@ __device__ void idx_epilogue(IdxSmem& sm, const IdxTcArgs& a, uint32_t tmem, lon
             tc::tc_fence_before();
             tc::mbar_arrive(&sm.a_full[s]);
         }
+        // this tile's scale, used by its epilogue one iteration later
+        float scale_next = 1.f;
+        if (FP8) {
+            const long long e = (long long)cur.ti * kTileK + r;
+            if (e < a.n_ent) scale_next = __ldg(a.kscale + (long long)(cur.row / a.n_q) * a.n_ent + e);
+        }
         // epilogue of the previous tile overlaps this tile's MMA
         if (p_jt >= 0 && !epilogue(p_jt, p_row, p_ti)) { ok = false; break; }
         p_jt = jt;
         p_row = cur.row;
         p_ti = cur.ti;
+        p_scale = scale_next;
         (void)seg_end;
     }
     if (ok && p_jt >= 0) {

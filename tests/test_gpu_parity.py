@@ -375,3 +375,33 @@ def test_csa_many_queries_split_rows(v4a):
     assert int(st.item()) == 0
     ref = oracle.attend(host(a["q"]), host(a["entries"]), host(a["idx"]), host(a["token_kv"]), a["tok_pos0"], L, m, W)
     check_attention(out, ref, False, "csa multi-query")
+
+
+def test_hca_single_long_query_split_over_many_ctas(v4a):
+    """One 1M-context HCA query: its 130 tiles land on 130 CTAs and the
+    combine merges 130 pieces."""
+    B, T, L, m, H, d, W = 1, 1, 1 << 20, 128, 64, 512, 128
+    a = _attend_inputs(B, T, L, m, H, d, W, "bf16", seed=61)
+    out = torch.empty((B, T, H, d), device="cuda")
+    v4a.v4a_hca_attend(dev(a["q"]), dev(a["entries"]), dev(a["token_kv"]), a["tok_pos0"], out, m=m, window=W,
+                       ctx_len=L)
+    _sync()
+    ref = oracle.attend(host(a["q"]), host(a["entries"]), None, host(a["token_kv"]), a["tok_pos0"], L, m, W)
+    check_attention(out, ref, False, "hca one long query")
+
+
+def test_topk_all_scores_equal_takes_lowest_entries(v4a):
+    """Every entry scores the same: the candidate set exceeds what the fast
+    select holds in shared memory and the full radix select takes over; ties
+    go to the lowest entries."""
+    B, L, m, k, HI, DI = 2, 4 * 40000, 4, 777, 16, 128
+    c = wl.index_case(B, 1, L, m, HI, DI, "bf16", "bf16", seed=71)
+    c["k_i"] = c["k_i"][:, :1].expand(B, L // m, DI).contiguous()  # one key repeated everywhere
+    idx = torch.empty((B, 1, k), dtype=torch.int32, device="cuda")
+    sco = torch.empty((B, 1, k), dtype=torch.float32, device="cuda")
+    v4a.v4a_topk(dev(c["q_i"]), dev(c["w"]), dev(c["k_i"]), None, idx, sco, m=m, k=k, ctx_len=L)
+    _sync()
+    want = np.broadcast_to(np.arange(k, dtype=np.int32), (B, 1, k))
+    assert np.array_equal(idx.cpu().numpy(), want)
+    s = sco.cpu().numpy()
+    assert (s == s[:, :, :1]).all()
