@@ -44,7 +44,7 @@ WORKLOAD = ("1M-ctx decode step: CSA layer (batch 4, 262,144 entries, fp8 indexe
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=400)
+    p.add_argument("--steps", type=int, default=10000)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -109,6 +109,10 @@ class ClockSampler:
             self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
                                           "-i", str(self.gpu), "-lms", "100"], stdout=self.f,
                                          stderr=subprocess.DEVNULL)
+            # wait (bounded) for the first sample so that the timed region is covered from its start
+            t0 = time.time()
+            while time.time() - t0 < 10.0 and os.path.getsize(self.path) == 0 and self.proc.poll() is None:
+                time.sleep(0.05)
         except Exception:
             self.proc = None
         return self
@@ -243,33 +247,25 @@ class Step:
 
 
 def kernel_nodes(graph) -> int | None:
-    """Kernel nodes in a captured graph (cudaGraphGetNodes + cudaGraphNodeGetType)."""
+    """Kernel nodes in a captured graph (cuGraphGetNodes + cuGraphNodeGetType of
+    the driver API; the graph must have been made with keep_graph=True)."""
     try:
         import ctypes
-
-        import torch.cuda
-        raw = graph.raw_cuda_graph()
-        rt = None
-        for name in ("libcudart.so.12", "libcudart.so"):
-            try:
-                rt = ctypes.CDLL(name)
-                break
-            except OSError:
-                continue
-        if rt is None:
-            return None
+        drv = ctypes.CDLL("libcuda.so.1")
+        raw = ctypes.c_void_p(graph.raw_cuda_graph())
         n = ctypes.c_size_t(0)
-        if rt.cudaGraphGetNodes(ctypes.c_void_p(raw), None, ctypes.byref(n)) != 0:
+        if drv.cuGraphGetNodes(raw, None, ctypes.byref(n)) != 0:
             return None
         nodes = (ctypes.c_void_p * n.value)()
-        if rt.cudaGraphGetNodes(ctypes.c_void_p(raw), nodes, ctypes.byref(n)) != 0:
+        if drv.cuGraphGetNodes(raw, nodes, ctypes.byref(n)) != 0:
             return None
-        kinds = 0
+        kernels = 0
         for i in range(n.value):
             t = ctypes.c_int(-1)
-            rt.cudaGraphNodeGetType(ctypes.c_void_p(nodes[i]), ctypes.byref(t))
-            kinds += 1 if t.value == 0 else 0  # cudaGraphNodeTypeKernel
-        return kinds
+            if drv.cuGraphNodeGetType(ctypes.c_void_p(nodes[i]), ctypes.byref(t)) != 0:
+                return None
+            kernels += 1 if t.value == 0 else 0  # CU_GRAPH_NODE_TYPE_KERNEL
+        return kernels
     except Exception:
         return None
 
@@ -369,9 +365,10 @@ def main():
     for _ in range(args.warmup):
         step.run()
     torch.cuda.synchronize()
-    g = torch.cuda.CUDAGraph()
+    g = torch.cuda.CUDAGraph(keep_graph=True)
     with torch.cuda.graph(g):
         step.run()
+    g.instantiate()
     for _ in range(args.warmup):
         g.replay()
     torch.cuda.synchronize()
