@@ -16,9 +16,13 @@
 //    operand; q is B in f16, each head scaled by a power of two so that its
 //    largest element lies in [2^13, 2^14) (exact for every bf16 value within
 //    2^-30 of it; the head weight carries the inverse power of two).
-// Warp 0 loads key tiles into a 4-stage ring, warp 1 issues the MMAs, warps
-// 2-5 convert (FP8) and run the epilogue.  CTAs take contiguous ranges of the
-// flat (query row, tile) sequence.  Every wait is bounded.
+// Warp 0 loads key tiles into a shared-memory ring (8 x 16 KB for FP8, 4 x 32 KB
+// for bf16), warp 1 issues the MMAs, warps 2-5 stage each row's q and (FP8)
+// widen key tiles into TMEM, warps 6-9 run the epilogue; widening of tile j,
+// the MMAs of tile j-1 and the epilogue of tile j-2 overlap.  CTAs take
+// contiguous ranges of the flat (query row, tile) sequence; a run of one
+// row's tiles inside a CTA's range is a segment, with its own q buffer and
+// histogram (both double-buffered).  Every wait is bounded.
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
@@ -30,19 +34,28 @@ namespace {
 
 constexpr int kDI = 128;                 // indexer dim handled here
 constexpr int kTileK = 128;              // entries per tile
-constexpr int kStages = 4;
-constexpr int kThreads = 192;
+constexpr int kRingBytes = 131072;       // key-tile ring
+constexpr int kMaxStages = 8;
+constexpr int kThreads = 320;
 constexpr int kHistBins = 4096;          // top 12 bits of the ordered score key
-constexpr uint32_t kColA = 0;            // FP8: converted key tiles, 2 x 64 columns
-constexpr uint32_t kColD = 128;          // D: 2 x 32 columns
+constexpr int kAStages = 2;              // FP8: widened key tiles in TMEM
+constexpr int kDStages = 4;              // accumulators in TMEM
+constexpr uint32_t kColA = 0;            // 2 x 64 columns
+constexpr uint32_t kColD = 128;          // 4 x 32 columns
 constexpr uint32_t kTmemCols = 256;
 
+template <bool FP8> struct Ring {
+    static constexpr int kStageBytes = FP8 ? kTileK * kDI : kTileK * kDI * 2;
+    static constexpr int kStages = kRingBytes / kStageBytes;
+};
+
 struct __align__(1024) IdxSmem {
-    uint8_t keys[kStages][kTileK * kDI * 2];  // bf16: 2 slabs of [128][128 B]; fp8: [128][128 B]
-    uint8_t q[2][32 * 128];                   // B operand: 2 K-slabs of [32 heads][128 B]
-    float wq[32];                             // head weights (times 2^-s for FP8)
-    uint32_t hist[kHistBins];
-    uint64_t k_full[kStages], k_empty[kStages], a_full[2], d_full[2], d_free[2], q_ready, q_free, drain;
+    uint8_t ring[kRingBytes];                 // bf16: [2 slabs][128][128 B] per stage; fp8: [128][128 B]
+    uint8_t q[2][2 * 32 * 128];               // B operand per segment buffer: 2 K-slabs of [N heads][128 B]
+    float wq[2][32];                          // head weights (times 2^-s for FP8)
+    uint32_t hist[2][kHistBins];
+    uint64_t k_full[kMaxStages], k_empty[kMaxStages], a_full[kAStages], a_free[kAStages], d_full[kDStages],
+        d_free[kDStages], q_full[2], q_free[2], ep_sync, drain;
     int abort_flag;
     uint32_t tmem_base;
 };
@@ -55,7 +68,7 @@ struct IdxTcArgs {
     uint32_t* hist;          // [rows][4096]
     int* err;                // device fault word (may be null)
     long long n_ent, ctx_len, total_tiles;
-    int rows, n_q, m, heads_i, n_pad, tiles_per_row, grid;
+    int rows, n_q, m, heads_i, tiles_per_row, grid;
 };
 
 __device__ __forceinline__ void idx_fault(IdxSmem& sm, const IdxTcArgs& a) {
@@ -63,115 +76,127 @@ __device__ __forceinline__ void idx_fault(IdxSmem& sm, const IdxTcArgs& a) {
     if (a.err) atomicExch(a.err, (int)V4A_ERR_DEVICE_FAULT);
 }
 
+// bounded wait taken by a whole warp: true only if every lane saw the phase complete
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity) {
+    return __all_sync(0xffffffffu, tc::mbar_wait(bar, parity));
+}
+__device__ __forceinline__ bool warp_aborted(const IdxSmem& sm) {
+    return __any_sync(0xffffffffu, *reinterpret_cast<const volatile int*>(&sm.abort_flag) != 0);
+}
+
 __device__ __forceinline__ long long irange(int c, const IdxTcArgs& a) { return (long long)c * a.total_tiles / a.grid; }
 
+// walks (row, tile) in flat order; rq = row % n_q and bat = row / n_q kept incrementally
 struct ICursor {
-    int row, ti;
-    __device__ ICursor(long long f, int tpr) : row((int)(f / tpr)), ti((int)(f % tpr)) {}
-    __device__ void next(int tpr) {
-        if (++ti == tpr) {
+    int row, ti, rq, bat;
+    __device__ ICursor(long long f, const IdxTcArgs& a) {
+        row = (int)(f / a.tiles_per_row);
+        ti = (int)(f - (long long)row * a.tiles_per_row);
+        bat = row / a.n_q;
+        rq = row - bat * a.n_q;
+    }
+    __device__ __forceinline__ void next(const IdxTcArgs& a) {
+        if (++ti == a.tiles_per_row) {
             ti = 0;
             ++row;
+            if (++rq == a.n_q) {
+                rq = 0;
+                ++bat;
+            }
         }
     }
 };
 
-__device__ __forceinline__ long long nvis_of(int row, const IdxTcArgs& a) {
-    const long long t = a.ctx_len - a.n_q + (row % a.n_q);
-    long long nv = n_visible(t, a.m);
+__device__ __forceinline__ long long nvis_of(const ICursor& c, const IdxTcArgs& a) {
+    const long long t = a.ctx_len - a.n_q + c.rq;
+    const long long nv = n_visible(t, a.m);
     return nv > a.n_ent ? a.n_ent : nv;
 }
 
-// idesc: M=128, N = n_pad, A and B both f16 (FP8 path) or both bf16
-__device__ __forceinline__ uint32_t idx_idesc(int n_pad, bool fp8) { return tc::idesc_f16(128, n_pad, 0, 0, fp8 ? 0 : 1); }
-
 template <bool FP8>
 __device__ void idx_producer(IdxSmem& sm, const IdxTcArgs& a, const CUtensorMap* kmap, long long f0, long long f1) {
-    const int lane = threadIdx.x & 31;
-    ICursor cur(f0, a.tiles_per_row);
-    for (long long f = f0; f < f1; ++f, cur.next(a.tiles_per_row)) {
-        if (sm.abort_flag) break;
-        const int jt = (int)(f - f0), st = jt % kStages;
-        if (jt >= kStages && !tc::mbar_wait(&sm.k_empty[st], ((jt / kStages) - 1) & 1)) { idx_fault(sm, a); break; }
-        if (lane == 0) {
-            const int b = cur.row / a.n_q;
-            const int y = (int)((long long)b * a.n_ent + (long long)cur.ti * kTileK);
-            if (FP8) {
-                tc::mbar_arrive_expect_tx(&sm.k_full[st], kTileK * kDI);
-                tc::tma_load_2d(sm.keys[st], kmap, 0, y, &sm.k_full[st]);
-            } else {
-                tc::mbar_arrive_expect_tx(&sm.k_full[st], kTileK * kDI * 2);
-                tc::tma_load_2d(sm.keys[st], kmap, 0, y, &sm.k_full[st]);
-                tc::tma_load_2d(sm.keys[st] + kTileK * 128, kmap, 64, y, &sm.k_full[st]);
-            }
-        }
-    }
+    constexpr int kSt = Ring<FP8>::kStages, kBytes = Ring<FP8>::kStageBytes;
+    ICursor cur(f0, a);
     const long long n = f1 - f0;
-    for (long long jt = n - kStages; jt < n; ++jt)
-        if (jt >= 0) tc::mbar_wait(&sm.k_full[jt % kStages], (jt / kStages) & 1);
+    for (long long jt = 0; jt < n; ++jt, cur.next(a)) {
+        if (*reinterpret_cast<volatile int*>(&sm.abort_flag)) break;
+        const int st = (int)(jt % kSt);
+        if (jt >= kSt && !tc::mbar_wait(&sm.k_empty[st], (uint32_t)((jt / kSt) - 1) & 1)) { idx_fault(sm, a); break; }
+        const int y = (int)((long long)cur.bat * a.n_ent + (long long)cur.ti * kTileK);
+        uint8_t* dst = sm.ring + st * kBytes;
+        tc::mbar_arrive_expect_tx(&sm.k_full[st], kBytes);
+        tc::tma_load_2d(dst, kmap, 0, y, &sm.k_full[st]);
+        if (!FP8) tc::tma_load_2d(dst + kTileK * 128, kmap, 64, y, &sm.k_full[st]);
+    }
+    // no copy may still be in flight when the CTA exits
+    for (long long jt = n - kSt; jt < n; ++jt)
+        if (jt >= 0) tc::mbar_wait(&sm.k_full[jt % kSt], (uint32_t)(jt / kSt) & 1);
 }
 
-template <bool FP8>
+template <bool FP8, int NP>
 __device__ void idx_mma(IdxSmem& sm, const IdxTcArgs& a, uint32_t tmem, long long f0, long long f1) {
+    constexpr int kSt = Ring<FP8>::kStages, kBytes = Ring<FP8>::kStageBytes;
+    constexpr uint32_t kQSlab = NP * 128;  // bytes per K-slab of q
+    constexpr uint32_t idesc = tc::idesc_f16(128, NP, 0, 0, FP8 ? 0 : 1);
     bool ok = true;
-    int seg = 0;
-    const uint32_t idesc = idx_idesc(a.n_pad, FP8);
-    const uint64_t qd = tc::sw128_desc(tc::smem_u32(sm.q[0]), 16, 1024);
-    const uint32_t qslab = (uint32_t)a.n_pad * 128;  // bytes per K-slab of q
-    ICursor cur(f0, a.tiles_per_row);
-    for (long long f = f0; f < f1; ++f, cur.next(a.tiles_per_row)) {
-        if (sm.abort_flag) { ok = false; break; }
-        const int jt = (int)(f - f0), s = jt & 1, st = jt % kStages;
-        const bool seg_start = (f == f0) || (cur.ti == 0);
-        const bool seg_end = (f == f1 - 1) || (cur.ti == a.tiles_per_row - 1);
-        if (seg_start) {
-            if (!tc::mbar_wait(&sm.q_ready, seg & 1)) { ok = false; break; }
+    int seg = 0, b = 0;
+    uint64_t qd = 0;
+    ICursor cur(f0, a);
+    for (long long f = f0; f < f1; ++f, cur.next(a)) {
+        if (*reinterpret_cast<volatile int*>(&sm.abort_flag)) { ok = false; break; }
+        const int jt = (int)(f - f0), s = jt & 1, st = jt % kSt, sd = jt & 3;
+        if (f == f0 || cur.ti == 0) {
+            b = seg & 1;
+            if (!tc::mbar_wait(&sm.q_full[b], (seg >> 1) & 1)) { ok = false; break; }
+            qd = tc::sw128_desc(tc::smem_u32(sm.q[b]), 16, 1024);
             ++seg;
         }
+        const bool seg_end = (f == f1 - 1) || (cur.ti == a.tiles_per_row - 1);
         if (FP8) {
             if (!tc::mbar_wait(&sm.a_full[s], (jt >> 1) & 1)) { ok = false; break; }
         } else {
-            if (!tc::mbar_wait(&sm.k_full[st], (jt / kStages) & 1)) { ok = false; break; }
-            if (jt >= 2 && !tc::mbar_wait(&sm.d_free[s], ((jt >> 1) - 1) & 1)) { ok = false; break; }
+            if (!tc::mbar_wait(&sm.k_full[st], (jt / kSt) & 1)) { ok = false; break; }
         }
+        if (jt >= kDStages && !tc::mbar_wait(&sm.d_free[sd], ((jt >> 2) - 1) & 1)) { ok = false; break; }
         tc::tc_fence_after();
-        const uint32_t d = tmem + kColD + 32 * s;
+        const uint32_t d = tmem + kColD + 32 * sd;
         if (FP8) {
             const uint32_t at = tmem + kColA + 64 * s;
 #pragma unroll
             for (int kk = 0; kk < kDI / 16; ++kk) {
-                const uint64_t bd = qd + ((((kk >> 2) * qslab) + (kk & 3) * 32) >> 4);
+                const uint64_t bd = qd + ((((kk >> 2) * kQSlab) + (kk & 3) * 32) >> 4);
                 asm volatile(
                     "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
                     " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d),
                     "r"(at + 8 * kk), "l"(bd), "r"(idesc), "r"(kk ? 1u : 0u)
                     : "memory");
             }
+            tc::mma_commit(&sm.a_free[s]);
         } else {
-            const uint64_t kd = tc::sw128_desc(tc::smem_u32(sm.keys[st]), 16, 1024);
+            const uint64_t kd = tc::sw128_desc(tc::smem_u32(sm.ring + st * kBytes), 16, 1024);
 #pragma unroll
             for (int kk = 0; kk < kDI / 16; ++kk) {
                 const uint64_t ad = kd + ((((kk >> 2) * (kTileK * 128)) + (kk & 3) * 32) >> 4);
-                const uint64_t bd = qd + ((((kk >> 2) * qslab) + (kk & 3) * 32) >> 4);
+                const uint64_t bd = qd + ((((kk >> 2) * kQSlab) + (kk & 3) * 32) >> 4);
                 tc::mma_f16(d, ad, bd, idesc, kk ? 1u : 0u);
             }
             tc::mma_commit(&sm.k_empty[st]);
         }
-        tc::mma_commit(&sm.d_full[s]);
-        if (seg_end) tc::mma_commit(&sm.q_free);
+        tc::mma_commit(&sm.d_full[sd]);
+        if (seg_end) tc::mma_commit(&sm.q_free[b]);
     }
     if (!ok) idx_fault(sm, a);
     tc::mma_commit(&sm.drain);
     tc::mbar_wait(&sm.drain, 0);
 }
 
-// q of `row` into the B-operand layout (K-major, 128-byte swizzle), and the head weights
-template <bool FP8>
-__device__ void stage_query(IdxSmem& sm, const IdxTcArgs& a, int row) {
-    const int t = threadIdx.x - 64;  // 0..127
-    // one warp per head group: warp w handles heads w, w+4, ...; lane owns 4 of the 128 elements
-    const int warp = t >> 5, lane = t & 31;
-    for (int h = warp; h < a.n_pad; h += 4) {
+// q of one row into buffer b in the B-operand layout (K-major, 128-byte
+// swizzle, NP head rows per K-slab), and the head weights; ct = 0..127
+template <bool FP8, int NP>
+__device__ void stage_query(IdxSmem& sm, const IdxTcArgs& a, int row, int b, int ct) {
+    // warp w handles heads w, w+4, ...; lane owns 4 of the 128 elements
+    const int warp = ct >> 5, lane = ct & 31;
+    for (int h = warp; h < NP; h += 4) {
         float v[4] = {0.f, 0.f, 0.f, 0.f};
         if (h < a.heads_i) {
             const __nv_bfloat16* qp = a.q + ((long long)row * a.heads_i + h) * kDI + lane * 4;
@@ -203,83 +228,41 @@ __device__ void stage_query(IdxSmem& sm, const IdxTcArgs& a, int row) {
         }
         // element k = 4*lane .. 4*lane+3 of head h: K-slab k/64, 16-byte chunk (k%64)/8, 8-byte half
         const int k = lane * 4;
-        uint8_t* slab = sm.q[0] + (k >> 6) * (a.n_pad * 128);
+        uint8_t* slab = sm.q[b] + (k >> 6) * (NP * 128);
         uint8_t* dst = slab + (h >> 3) * 1024 + (h & 7) * 128 + ((((k & 63) >> 3) ^ (h & 7)) << 4) + ((k & 7) ? 8 : 0);
         *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
-        if (lane == 0) sm.wq[h] = wq;
+        if (lane == 0) sm.wq[b][h] = wq;
     }
 }
 
-template <bool FP8>
-__device__ void idx_epilogue(IdxSmem& sm, const IdxTcArgs& a, uint32_t tmem, long long f0, long long f1) {
-    const int t = threadIdx.x - 64;                 // entry within the tile
+// warps 2-5: per segment stage q; per tile (FP8) widen the key tile to f16 in TMEM
+template <bool FP8, int NP>
+__device__ void idx_convert(IdxSmem& sm, const IdxTcArgs& a, uint32_t tmem, long long f0, long long f1) {
+    constexpr int kSt = Ring<FP8>::kStages, kBytes = Ring<FP8>::kStageBytes;
+    const int ct = threadIdx.x - 64;
     const int sub = (threadIdx.x >> 5) & 3;
-    const int r = 32 * sub + (threadIdx.x & 31);    // TMEM lane = entry row of the tile
+    const int r = 32 * sub + (threadIdx.x & 31);  // TMEM lane = entry row of the tile
     const uint32_t lane_addr = (uint32_t)(32 * sub) << 16;
     bool ok = true;
     int seg = 0;
-    long long nvis = 0;
-    ICursor cur(f0, a.tiles_per_row);
-    // pending epilogue (tile j-1), with its entry's scale loaded ahead
-    int p_row = -1, p_ti = 0, p_jt = -1;
-    float p_scale = 1.f;
-    auto epilogue = [&](int jt, int row, int ti) -> bool {
-        const int s = jt & 1;
-        if (!tc::mbar_wait(&sm.d_full[s], (jt >> 1) & 1)) return false;
-        tc::tc_fence_after();
-        uint32_t dv[32];
-        tc::tmem_ld_x32(tmem + lane_addr + kColD + 32 * s, dv);
-        tc::tmem_ld_wait();
-        if (!FP8) {
-            tc::tc_fence_before();
-            tc::mbar_arrive(&sm.d_free[s]);
-        }
-        const long long e = (long long)ti * kTileK + r;
-        const long long nv = nvis_of(row, a);
-        if (e < a.n_ent) {
-            float sc = -INFINITY;
-            if (e < nv) {
-                float acc = 0.f;
-#pragma unroll
-                for (int h = 0; h < 32; ++h)
-                    if (h < a.heads_i) acc = fmaf(sm.wq[h], fmaxf(__uint_as_float(dv[h]), 0.f), acc);
-                if (FP8) acc *= p_scale;
-                sc = acc + 0.0f;
-                if (a.hist) atomicAdd(&sm.hist[float_to_ordered(sc) >> 20], 1u);
-            }
-            a.scores[(long long)row * a.n_ent + e] = sc;
-        }
-        return true;
-    };
-    for (long long f = f0; f < f1; ++f, cur.next(a.tiles_per_row)) {
-        if (sm.abort_flag) { ok = false; break; }
-        const int jt = (int)(f - f0), s = jt & 1, st = jt % kStages;
-        const bool seg_start = (f == f0) || (cur.ti == 0);
-        const bool seg_end = (f == f1 - 1) || (cur.ti == a.tiles_per_row - 1);
-        if (seg_start) {
-            // finish the previous row: its last tile's epilogue, then flush its histogram
-            if (p_jt >= 0) {
-                if (!epilogue(p_jt, p_row, p_ti)) { ok = false; break; }
-                p_jt = -1;
-                tc::named_barrier(1, 128);
-                if (a.hist)
-                    for (int i = t; i < kHistBins; i += 128)
-                        if (sm.hist[i]) atomicAdd(&a.hist[(long long)p_row * kHistBins + i], sm.hist[i]);
-            }
-            // the MMAs of the previous row no longer read q
-            if (seg > 0 && !tc::mbar_wait(&sm.q_free, (seg - 1) & 1)) { ok = false; break; }
-            tc::named_barrier(1, 128);
-            for (int i = t; i < kHistBins; i += 128) sm.hist[i] = 0;
-            stage_query<FP8>(sm, a, cur.row);
+    ICursor cur(f0, a);
+    for (long long f = f0; f < f1; ++f, cur.next(a)) {
+        if (warp_aborted(sm)) { ok = false; break; }
+        const int jt = (int)(f - f0);
+        if (f == f0 || cur.ti == 0) {
+            const int b = seg & 1;
+            if (seg >= 2 && !warp_wait(&sm.q_free[b], ((seg >> 1) - 1) & 1)) { ok = false; break; }
+            stage_query<FP8, NP>(sm, a, cur.row, b, ct);
             tc::fence_proxy_async();
-            tc::mbar_arrive(&sm.q_ready);
+            tc::mbar_arrive(&sm.q_full[b]);
             ++seg;
-            nvis = nvis_of(cur.row, a);
         }
         if (FP8) {
-            // widen this thread's entry (row r of the tile) to f16 into TMEM
-            if (!tc::mbar_wait(&sm.k_full[st], (jt / kStages) & 1)) { ok = false; break; }
-            const uint8_t* kr = sm.keys[st] + r * 128;
+            const int s = jt & 1, st = jt % kSt;
+            if (!warp_wait(&sm.k_full[st], (jt / kSt) & 1)) { ok = false; break; }
+            if (jt >= kAStages && !warp_wait(&sm.a_free[s], ((jt >> 1) - 1) & 1)) { ok = false; break; }
+            tc::tc_fence_after();
+            const uint8_t* kr = sm.ring + st * kBytes + r * 128;
             uint32_t cv[64];
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
@@ -299,66 +282,129 @@ __device__ void idx_epilogue(IdxSmem& sm, const IdxTcArgs& a, uint32_t tmem, lon
             tc::tc_fence_before();
             tc::mbar_arrive(&sm.a_full[s]);
         }
-        // this tile's scale, used by its epilogue one iteration later
-        float scale_next = 1.f;
-        if (FP8) {
-            const long long e = (long long)cur.ti * kTileK + r;
-            if (e < a.n_ent) scale_next = __ldg(a.kscale + (long long)(cur.row / a.n_q) * a.n_ent + e);
-        }
-        // epilogue of the previous tile overlaps this tile's MMA
-        if (p_jt >= 0 && !epilogue(p_jt, p_row, p_ti)) { ok = false; break; }
-        p_jt = jt;
-        p_row = cur.row;
-        p_ti = cur.ti;
-        p_scale = scale_next;
-        (void)seg_end;
-    }
-    if (ok && p_jt >= 0) {
-        ok = epilogue(p_jt, p_row, p_ti);
-        tc::named_barrier(1, 128);
-        if (ok && a.hist)
-            for (int i = t; i < kHistBins; i += 128)
-                if (sm.hist[i]) atomicAdd(&a.hist[(long long)p_row * kHistBins + i], sm.hist[i]);
     }
     if (!ok) idx_fault(sm, a);
-    (void)nvis;
 }
 
-template <bool FP8>
+// warps 6-9: per tile the score of one entry per thread, its histogram count and store
+template <bool FP8, int NP>
+__device__ void idx_epilogue(IdxSmem& sm, const IdxTcArgs& a, uint32_t tmem, long long f0, long long f1) {
+    const int et = threadIdx.x - 192;
+    const int sub = (threadIdx.x >> 5) & 3;
+    const int r = 32 * sub + (threadIdx.x & 31);  // TMEM lane = entry row of the tile
+    const uint32_t lane_addr = (uint32_t)(32 * sub) << 16;
+    bool ok = true;
+    int seg = 0, b = 0, nsync = 0;
+    long long nv = 0;
+    float* srow = nullptr;
+    ICursor cur(f0, a);
+    // scale of the current tile's entry, loaded one tile ahead
+    auto scale_of = [&](const ICursor& c) -> float {
+        const long long e = (long long)c.ti * kTileK + r;
+        return e < a.n_ent ? __ldg(a.kscale + (long long)c.bat * a.n_ent + e) : 1.f;
+    };
+    float sc_cur = FP8 ? scale_of(cur) : 1.f;
+    for (long long f = f0; f < f1; ++f) {
+        if (warp_aborted(sm)) { ok = false; break; }
+        const int jt = (int)(f - f0), sd = jt & 3;
+        if (f == f0 || cur.ti == 0) {
+            b = seg & 1;
+            if (!warp_wait(&sm.q_full[b], (seg >> 1) & 1)) { ok = false; break; }
+            ++seg;
+            nv = nvis_of(cur, a);
+            srow = a.scores + (long long)cur.row * a.n_ent;
+        }
+        const bool seg_end = (f == f1 - 1) || (cur.ti == a.tiles_per_row - 1);
+        const int ti = cur.ti, row = cur.row;
+        cur.next(a);
+        float sc_next = 1.f;
+        if (FP8 && f + 1 < f1) sc_next = scale_of(cur);
+        if (!warp_wait(&sm.d_full[sd], (jt >> 2) & 1)) { ok = false; break; }
+        tc::tc_fence_after();
+        uint32_t dv[NP];
+        if constexpr (NP == 16) tc::tmem_ld_x16(tmem + lane_addr + kColD + 32 * sd, dv);
+        else tc::tmem_ld_x32(tmem + lane_addr + kColD + 32 * sd, dv);
+        tc::tmem_ld_wait();
+        tc::tc_fence_before();
+        tc::mbar_arrive(&sm.d_free[sd]);
+        const long long e = (long long)ti * kTileK + r;
+        if (e < a.n_ent) {
+            float sc = -INFINITY;
+            if (e < nv) {
+                float acc = 0.f;
+#pragma unroll
+                for (int h = 0; h < NP; ++h) acc = fmaf(sm.wq[b][h], fmaxf(__uint_as_float(dv[h]), 0.f), acc);
+                if (FP8) acc *= sc_cur;
+                sc = acc + 0.0f;
+                if (a.hist) atomicAdd(&sm.hist[b][float_to_ordered(sc) >> 20], 1u);
+            }
+            srow[e] = sc;
+        }
+        sc_cur = sc_next;
+        if (seg_end) {
+            tc::mbar_arrive(&sm.q_free[b]);  // done with wq[b]
+            // every epilogue thread has counted this segment's scores (bounded, unlike a named barrier)
+            tc::mbar_arrive(&sm.ep_sync);
+            if (!warp_wait(&sm.ep_sync, nsync++ & 1)) { ok = false; break; }
+            if (a.hist) {
+                uint32_t* g = a.hist + (long long)row * kHistBins;
+                for (int i = et; i < kHistBins; i += 128) {
+                    const uint32_t v = sm.hist[b][i];
+                    if (v) {
+                        atomicAdd(g + i, v);
+                        sm.hist[b][i] = 0;
+                    }
+                }
+            }
+        }
+    }
+    if (!ok) idx_fault(sm, a);
+}
+
+template <bool FP8, int NP>
 __global__ void __launch_bounds__(kThreads, 1) index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, IdxTcArgs a) {
     extern __shared__ uint8_t smem_raw[];
     IdxSmem& sm = *reinterpret_cast<IdxSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const int warp = threadIdx.x >> 5;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long long f0 = irange(blockIdx.x, a), f1 = irange(blockIdx.x + 1, a);
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kStages; ++i) {
+        for (int i = 0; i < Ring<FP8>::kStages; ++i) {
             tc::mbar_init(&sm.k_full[i], 1);
             tc::mbar_init(&sm.k_empty[i], FP8 ? 128 : 1);
         }
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < kAStages; ++i) {
             tc::mbar_init(&sm.a_full[i], 128);
+            tc::mbar_init(&sm.a_free[i], 1);
+        }
+        for (int i = 0; i < kDStages; ++i) {
             tc::mbar_init(&sm.d_full[i], 1);
             tc::mbar_init(&sm.d_free[i], 128);
         }
-        tc::mbar_init(&sm.q_ready, 128);
-        tc::mbar_init(&sm.q_free, 1);
+        for (int i = 0; i < 2; ++i) {
+            tc::mbar_init(&sm.q_full[i], 128);
+            tc::mbar_init(&sm.q_free[i], 1 + 128);  // the MMAs' commit + every epilogue thread
+        }
+        tc::mbar_init(&sm.ep_sync, 128);
         tc::mbar_init(&sm.drain, 1);
         sm.abort_flag = 0;
         tc::fence_barrier_init();
     }
+    for (int i = threadIdx.x; i < 2 * kHistBins; i += kThreads) (&sm.hist[0][0])[i] = 0;
     if (warp == 1) tc::tmem_alloc(&sm.tmem_base, kTmemCols);
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
     if (warp == 0) {
-        idx_producer<FP8>(sm, a, &kmap, f0, f1);
+        if (lane == 0) idx_producer<FP8>(sm, a, &kmap, f0, f1);
     } else if (warp == 1) {
-        if ((threadIdx.x & 31) == 0) idx_mma<FP8>(sm, a, tmem, f0, f1);
-        __syncwarp();
+        if (lane == 0) idx_mma<FP8, NP>(sm, a, tmem, f0, f1);
+    } else if (warp < 6) {
+        idx_convert<FP8, NP>(sm, a, tmem, f0, f1);
     } else {
-        idx_epilogue<FP8>(sm, a, tmem, f0, f1);
+        idx_epilogue<FP8, NP>(sm, a, tmem, f0, f1);
     }
+    __syncwarp();
     tc::tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -415,7 +461,6 @@ cudaError_t launch_index_scores_tc(const IndexArgs& a, float* scores, uint32_t* 
     t.n_q = a.n_q;
     t.m = a.m;
     t.heads_i = a.heads_i;
-    t.n_pad = a.heads_i <= 16 ? 16 : 32;
     // tiles up to the last entry any query of the row block can see
     long long nv_max = n_visible(a.ctx_len - 1, a.m);
     if (nv_max > a.n_ent) nv_max = a.n_ent;
@@ -424,14 +469,14 @@ cudaError_t launch_index_scores_tc(const IndexArgs& a, float* scores, uint32_t* 
     if (t.total_tiles == 0) return cudaSuccess;
     t.grid = (int)(t.total_tiles < kNumSMs ? t.total_tiles : kNumSMs);
     const size_t smem = sizeof(IdxSmem) + 1024;
-    cudaError_t e;
-    if (fp8) {
-        e = cudaFuncSetAttribute(index_score_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e == cudaSuccess) index_score_tc_kernel<true><<<t.grid, kThreads, smem, stream>>>(kmap, t);
-    } else {
-        e = cudaFuncSetAttribute(index_score_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e == cudaSuccess) index_score_tc_kernel<false><<<t.grid, kThreads, smem, stream>>>(kmap, t);
-    }
+    auto go = [&](auto kernel) {
+        cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (err == cudaSuccess) kernel<<<t.grid, kThreads, smem, stream>>>(kmap, t);
+        return err;
+    };
+    const bool narrow = a.heads_i <= 16;
+    cudaError_t e = fp8 ? (narrow ? go(index_score_tc_kernel<true, 16>) : go(index_score_tc_kernel<true, 32>))
+                        : (narrow ? go(index_score_tc_kernel<false, 16>) : go(index_score_tc_kernel<false, 32>));
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
