@@ -228,9 +228,9 @@ __device__ void producer(Smem& sm, const TcArgs& a, const CUtensorMap* ent_map, 
 // descriptor + byte offset (the start-address field counts 16-byte units)
 __device__ __forceinline__ uint64_t dadd(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
 
-__device__ bool issue_pv(Smem& sm, uint32_t tmem, int jp, bool first_in_seg) {
+// O^T += V^T P^T for tile jp (its P is in shared memory)
+__device__ void issue_pv(Smem& sm, uint32_t tmem, int jp, bool first_in_seg) {
     const int sp = jp & 1, st = jp % kStages;
-    if (!tc::mbar_wait(&sm.p_full[sp], (jp >> 1) & 1)) return false;
     tc::tc_fence_after();
     // A = V^T (M = 128 d of slabs 2cc, 2cc+1; K = 16 rows), MN-major; B = P^T, K-major rows of P
     const uint64_t a0 = tc::sw128_desc(tc::smem_u32(sm.kv[st]), kSlabBytes, 1024);
@@ -244,48 +244,67 @@ __device__ bool issue_pv(Smem& sm, uint32_t tmem, int jp, bool first_in_seg) {
     }
     tc::mma_commit(&sm.kv_empty[st]);
     tc::mma_commit(&sm.p_free[sp]);
-    return true;
 }
 
-__device__ void mma_issuer(Smem& sm, const TcArgs& a, uint32_t tmem, long long f0, long long f1) {
-    int seg = 0;
-    bool ok = true;
-    bool prev_first = false;  // whether the pending PV tile starts its segment
-    const uint64_t q0 = tc::sw128_desc(tc::smem_u32(sm.q), 16, 1024);
-    Cursor cur(f0, a.tpr);
-    for (long long f = f0; f < f1 && ok; ++f, cur.next(a.tpr)) {
-        if (sm.abort_flag) { ok = false; break; }
-        const int jt = (int)(f - f0), s = jt & 1, st = jt % kStages;
-        const int ti = cur.ti;
-        const bool seg_start = (f == f0) || (ti == 0);
-        const bool seg_end = (f == f1 - 1) || (ti == a.tpr - 1);
-        if (seg_start && jt > 0) {
-            if (!issue_pv(sm, tmem, jt - 1, prev_first)) { ok = false; break; }
-        }
-        if (seg_start) {
-            if (!tc::mbar_wait(&sm.q_full, seg & 1)) { ok = false; break; }
-            ++seg;
-        }
-        if (!tc::mbar_wait(&sm.kv_full[st], (jt / kStages) & 1)) { ok = false; break; }
-        tc::fence_proxy_async();  // rows gathered with cp.async become visible to the tensor core
-        tc::tc_fence_after();
-        const uint64_t k0 = tc::sw128_desc(tc::smem_u32(sm.kv[st]), 16, 1024);
-        const uint32_t d_s = tmem + kColS + kTile * s;
+// S = Q K^T for tile jq (its rows are in shared memory)
+__device__ void issue_qk(Smem& sm, uint32_t tmem, int jq, bool gathered, uint64_t q0) {
+    const int s = jq & 1, st = jq % kStages;
+    if (gathered) tc::fence_proxy_async();  // rows gathered with cp.async become visible to the tensor core
+    tc::tc_fence_after();
+    const uint64_t k0 = tc::sw128_desc(tc::smem_u32(sm.kv[st]), 16, 1024);
+    const uint32_t d_s = tmem + kColS + kTile * s;
 #pragma unroll
-        for (int c = 0; c < kSlabs; ++c) {
+    for (int c = 0; c < kSlabs; ++c) {
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-                tc::mma_f16(d_s, dadd(q0, c * kH * 128 + kk * 32), dadd(k0, c * kSlabBytes + kk * 32), kIdescQK,
-                            (c | kk) ? 1u : 0u);
-        }
-        tc::mma_commit(&sm.s_full[s]);
-        if (seg_end) tc::mma_commit(&sm.q_empty);
-        if (!seg_start && jt > 0) {
-            if (!issue_pv(sm, tmem, jt - 1, prev_first)) { ok = false; break; }
-        }
-        prev_first = seg_start;
+        for (int kk = 0; kk < 4; ++kk)
+            tc::mma_f16(d_s, dadd(q0, c * kH * 128 + kk * 32), dadd(k0, c * kSlabBytes + kk * 32), kIdescQK,
+                        (c | kk) ? 1u : 0u);
     }
-    if (ok && f1 > f0) ok = issue_pv(sm, tmem, (int)(f1 - f0 - 1), prev_first);
+    tc::mma_commit(&sm.s_full[s]);
+}
+
+// No CTA-wide progress for this many cycles (about a second) counts as a fault.
+constexpr long long kStallCycles = 1LL << 31;
+
+// The two MMA groups of every tile are issued in whatever order their inputs
+// become ready: PV(j) as soon as the softmax has written P(j) (which frees
+// tile j's stage for the next load early), QK(j) as soon as tile j has
+// landed and S buffer j&1 is free (PV(j-2) issued).
+__device__ void mma_issuer(Smem& sm, const TcArgs& a, uint32_t tmem, long long f0, long long f1) {
+    const long long n = f1 - f0;
+    const uint64_t q0 = tc::sw128_desc(tc::smem_u32(sm.q), 16, 1024);
+    long long jq = 0, jp = 0;
+    int segq = 0;
+    bool ok = true;
+    Cursor cq(f0, a.tpr), cp(f0, a.tpr);
+    long long t_last = clock64();
+    while (jp < n) {
+        if (*reinterpret_cast<volatile int*>(&sm.abort_flag)) { ok = false; break; }
+        bool progressed = false;
+        if (jp < jq && tc::mbar_test(&sm.p_full[jp & 1], (uint32_t)(jp >> 1) & 1)) {
+            issue_pv(sm, tmem, (int)jp, jp == 0 || cp.ti == 0);
+            ++jp;
+            cp.next(a.tpr);
+            progressed = true;
+        } else if (jq < n && jp >= jq - 1) {
+            const bool qseg = jq == 0 || cq.ti == 0;
+            if (tc::mbar_test(&sm.kv_full[jq % kStages], (uint32_t)(jq / kStages) & 1) &&
+                (!qseg || tc::mbar_test(&sm.q_full, segq & 1))) {
+                issue_qk(sm, tmem, (int)jq, a.idx != nullptr && cq.ti < a.e_tiles, q0);
+                if (jq == n - 1 || cq.ti == a.tpr - 1) tc::mma_commit(&sm.q_empty);  // last QK of this query
+                if (qseg) ++segq;
+                ++jq;
+                cq.next(a.tpr);
+                progressed = true;
+            }
+        }
+        if (progressed) {
+            t_last = clock64();
+        } else if (clock64() - t_last > kStallCycles) {
+            ok = false;
+            break;
+        }
+    }
     if (!ok) fault(sm, a);
     // every MMA issued has completed before the CTA frees TMEM
     tc::mma_commit(&sm.drain);
