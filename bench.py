@@ -271,19 +271,32 @@ def kernel_nodes(graph) -> int | None:
 
 
 def time_op(fn, reps: int, flush: torch.Tensor) -> float:
-    """Mean device ms of one call of fn, L2 flushed (memset of a buffer larger
-    than L2) before each timed call, outside its events."""
+    """Device ms of one call of fn with L2 flushed before it (a memset of a
+    buffer larger than L2): one CUDA graph replays `reps` x (flush, fn), a
+    second replays `reps` x flush alone, and the difference of their event
+    times over `reps` is fn's share, free of launch and event overheads."""
     s = torch.cuda.current_stream()
-    evs = []
-    for _ in range(reps):
-        flush.zero_()
+
+    def timed(with_fn: bool) -> float:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(reps):
+                flush.zero_()
+                if with_fn:
+                    fn()
+        g.replay()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(s)
-        fn()
-        b.record(s)
-        evs.append((a, b))
-    torch.cuda.synchronize()
-    return statistics.mean(a.elapsed_time(b) for a, b in evs)
+        best = float("inf")
+        for _ in range(3):
+            a.record(s)
+            g.replay()
+            b.record(s)
+            torch.cuda.synchronize()
+            best = min(best, a.elapsed_time(b))
+        del g
+        return best
+
+    return max(0.0, (timed(True) - timed(False)) / reps)
 
 
 # ----------------------------------------------------------------------

@@ -5,12 +5,13 @@
 // logits Z) weighted sum of the content rows C.  One launch compresses both the
 // K=V stream and, optionally, the indexer-key stream of the same chunks.
 //
-// Mapping: S adjacent lanes (S = min(m, 16), a power of two; 1 for FP8
-// output) own 8 consecutive channels of one entry; each streams every S-th
-// token of the chunk with 16-byte vector loads (two for fp32), keeping a
-// running max / denominator / numerator per channel in registers (online
-// softmax), and the S partial states are merged with butterfly shuffles.  For
-// FP8 output the lanes of one entry are consecutive lanes of one warp, so the
+// Mapping: S adjacent lanes (S = the largest power of two <= min(m, 32); 1
+// for FP8 output) own 8 consecutive channels of one entry; each takes every
+// S-th token of the chunk with 16-byte vector loads (two for fp32), four
+// tokens per round with all loads issued first, keeping a running max /
+// denominator / numerator per channel in registers.  The S partial states are
+// merged with shuffles: common max, one rescale per lane, then sums.  For FP8
+// output the lanes of one entry are consecutive lanes of one warp, so the
 // entry's amax is found with warp shuffles too.
 #include "common.cuh"
 #include "internal.h"
@@ -29,22 +30,46 @@ struct StreamDesc {
     long long x_bs, gate_bs, out_bs, scale_bs;
 };
 
+// This lane's share of one (entry, 8-channel group): tokens sub, sub + S, ... of the chunk, in
+// rounds of kU tokens whose loads are all issued first; per round one max, one rescale of the
+// running state and one exp per element.
 template <typename T>
 __device__ __forceinline__ void compress_group(const StreamDesc& d, int b, long long s, int grp, int m, int sub,
                                                float mx[8], float den[8], float num[8]) {
     const T* xp = static_cast<const T*>(d.x) + (long long)b * d.x_bs + s * m * d.channels + grp * 8;
     const T* zp = static_cast<const T*>(d.gate) + (long long)b * d.gate_bs + s * m * d.channels + grp * 8;
-    for (int i = sub; i < m; i += d.split) {
-        float xv[8], zv[8];
-        Vec8<T>::load_nc(xp + (long long)i * d.channels, xv);
-        Vec8<T>::load_nc(zp + (long long)i * d.channels, zv);
+    constexpr int kU = 4;
+    for (int i0 = sub; i0 < m; i0 += kU * d.split) {
+        float xv[kU][8], zv[kU][8];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const int i = i0 + u * d.split;
+            if (i < m) {
+                Vec8<T>::load_nc(xp + (long long)i * d.channels, xv[u]);
+                Vec8<T>::load_nc(zp + (long long)i * d.channels, zv[u]);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    xv[u][e] = 0.f;
+                    zv[u][e] = -INFINITY;
+                }
+            }
+        }
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-            float nm = fmaxf(mx[e], zv[e]);
-            float a = expf(mx[e] - nm);  // rescale of what was accumulated so far
-            float p = expf(zv[e] - nm);
-            den[e] = den[e] * a + p;
-            num[e] = num[e] * a + p * xv[e];
+            float nm = mx[e];
+#pragma unroll
+            for (int u = 0; u < kU; ++u) nm = fmaxf(nm, zv[u][e]);
+            const float a = mx[e] == -INFINITY ? 0.f : expf(mx[e] - nm);  // rescale of the running state
+            float dn = den[e] * a, nu = num[e] * a;
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+                const float p = zv[u][e] == -INFINITY ? 0.f : expf(zv[u][e] - nm);
+                dn += p;
+                nu = fmaf(p, xv[u][e], nu);
+            }
+            den[e] = dn;
+            num[e] = nu;
             mx[e] = nm;
         }
     }
@@ -77,19 +102,21 @@ __global__ void __launch_bounds__(256) compress_kernel(StreamDesc s0, StreamDesc
         else
             compress_group<float>(d, b, s, grp, m, sub, mx, den, num);
     }
-    // merge the S lanes' partial softmax states (S adjacent lanes, S a power of two)
-    for (int o = d.split / 2; o > 0; o >>= 1) {
+    // merge the S lanes' partial states (S adjacent lanes, S a power of two): the common max,
+    // one rescale per lane, then plain sums
+    if (d.split > 1) {
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-            const float m2 = __shfl_xor_sync(0xffffffffu, mx[e], o);
-            const float d2 = __shfl_xor_sync(0xffffffffu, den[e], o);
-            const float n2 = __shfl_xor_sync(0xffffffffu, num[e], o);
-            const float nm = fmaxf(mx[e], m2);
-            const float a1 = nm == -INFINITY ? 0.f : expf(mx[e] - nm);
-            const float a2 = nm == -INFINITY ? 0.f : expf(m2 - nm);
-            den[e] = den[e] * a1 + d2 * a2;
-            num[e] = num[e] * a1 + n2 * a2;
-            mx[e] = nm;
+            float gm = mx[e];
+            for (int o = d.split / 2; o > 0; o >>= 1) gm = fmaxf(gm, __shfl_xor_sync(0xffffffffu, gm, o));
+            const float a = mx[e] == -INFINITY ? 0.f : expf(mx[e] - gm);
+            float dn = den[e] * a, nu = num[e] * a;
+            for (int o = d.split / 2; o > 0; o >>= 1) {
+                dn += __shfl_xor_sync(0xffffffffu, dn, o);
+                nu += __shfl_xor_sync(0xffffffffu, nu, o);
+            }
+            den[e] = dn;
+            num[e] = nu;
         }
     }
     float out[8];
@@ -150,10 +177,10 @@ cudaError_t launch_compress(const v4a_compress_io* kv, const v4a_compress_io* id
     if (batch == 0 || n_ent == 0) return cudaSuccess;
     StreamDesc s0 = describe(kv);
     StreamDesc s1 = idx ? describe(idx) : s0;
-    // lanes per (entry, channel group): enough to spread long chunks, 1 for FP8 output
+    // lanes per (entry, channel group): up to a warp, to spread long chunks; 1 for FP8 output
     // (its per-entry amax runs over the entry's consecutive lanes)
     int split = 1;
-    while (split < 16 && split * 2 <= m) split *= 2;
+    while (split < 32 && split * 2 <= m) split *= 2;
     if (s0.out_dtype != V4A_FP8E4M3) s0.split = split;
     if (s1.out_dtype != V4A_FP8E4M3) s1.split = split;
     long long w0 = (long long)s0.groups * s0.split, w1 = (long long)s1.groups * s1.split;

@@ -4,25 +4,30 @@
 // I(t,s) = scale_s * sum_j w_j * ReLU(q_j . k_s)   ("How V4 makes a
 // million-token context actually affordable", Lightning-Indexer section).
 //
-// Per tile of 128 entries of one query row: D[128 entries x N heads] = K Q^T
-// on tcgen05 (M=128, N=16 or 32, K=128 in 8 steps of 16), then the epilogue
-// (one thread per entry, TMEM lane = entry) forms the score, writes it as
-// fp32 and counts it in a 4096-bin histogram of its order-preserving key's
-// top 12 bits (the select step starts from that histogram).
-//  * bf16 keys: the key tile (TMA, 128-byte swizzle) is the MMA's A operand
-//    in shared memory; q is B (bf16).
-//  * FP8 keys: the tile is widened in registers, exactly, to f16
-//    (e4m3 -> f16 is exact) and stored to TMEM, where it is the MMA's A
-//    operand; q is B in f16, each head scaled by a power of two so that its
-//    largest element lies in [2^13, 2^14) (exact for every bf16 value within
-//    2^-30 of it; the head weight carries the inverse power of two).
-// Warp 0 loads key tiles into a shared-memory ring (8 x 16 KB for FP8, 4 x 32 KB
-// for bf16), warp 1 issues the MMAs, warps 2-5 stage each row's q and (FP8)
-// widen key tiles into TMEM, warps 6-9 run the epilogue; widening of tile j,
-// the MMAs of tile j-1 and the epilogue of tile j-2 overlap.  CTAs take
-// contiguous ranges of the flat (query row, tile) sequence; a run of one
-// row's tiles inside a CTA's range is a segment, with its own q buffer and
-// histogram (both double-buffered).  Every wait is bounded.
+// Per tile of 256 entries of one query row, D[256 entries x N] = K B^T on
+// tcgen05 (two M=128 halves, K=128), then the epilogue (one thread per pair
+// of entries r, r+128; TMEM lane = r) forms the scores, writes them as fp32
+// and counts them in a 4096-bin histogram of the order-preserving key's top
+// 12 bits (the select step starts from that histogram).  Tiles of 256
+// entries make 32 KB FP8 stages: a 128 KB ring of such stages streams HBM
+// at about 7 TB/s on B200, while 16 KB stages stay near 5.5 TB/s.
+//  * bf16 keys: kind::f16, B = q (N = heads, bf16), 8 MMAs of K=16.
+//  * FP8 keys: kind::f8f6f4 straight from the TMA tile, 4 MMAs of K=32.  B
+//    holds q split exactly into e4m3 pieces, four columns per head: with q
+//    scaled per head by 2^s so that its largest magnitude lies in [128, 256),
+//    an element x with |x| >= 1/4 is hi + lo (hi = nearest e4m3 of x, lo =
+//    x - hi, both exact in e4m3), and a smaller one is (hi' + lo') * 2^-10
+//    from x * 2^10 the same way (exact down to 2^-20 of the head's maximum).
+//    q_j . k = (D_hi + D_lo) + (D_hi' + D_lo') * 2^-10, times 2^-s (folded
+//    into the head weight).  These MMAs accumulate in f32 at least as
+//    precisely as a sequential f32 sum (measured on B200), so the score keeps
+//    f32 accuracy without widening the keys.
+// Warp 0 loads key tiles into a shared-memory ring (4 x 32 KB for FP8, 2 x 64
+// KB for bf16), warp 1 issues the MMAs, warps 2-5 stage each row's B
+// operand, warps 6-9 run the epilogue.  CTAs take contiguous ranges of the
+// flat (query row, tile) sequence; a run of one row's tiles inside a CTA's
+// range is a segment, with its own B buffer and histogram (both
+// double-buffered).  Every wait is bounded.
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
@@ -33,29 +38,34 @@ namespace v4a {
 namespace {
 
 constexpr int kDI = 128;                 // indexer dim handled here
-constexpr int kTileK = 128;              // entries per tile
+constexpr int kTileK = 256;              // entries per tile (two M=128 halves)
+constexpr int kHalf = 128;
 constexpr int kRingBytes = 131072;       // key-tile ring
 constexpr int kMaxStages = 8;
 constexpr int kThreads = 320;
 constexpr int kHistBins = 4096;          // top 12 bits of the ordered score key
-constexpr int kAStages = 2;              // FP8: widened key tiles in TMEM
-constexpr int kDStages = 4;              // accumulators in TMEM
-constexpr uint32_t kColA = 0;            // 2 x 64 columns
-constexpr uint32_t kColD = 128;          // 4 x 32 columns
-constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kTmemCols = 512;
+constexpr int kMaxDStages = 4;
+constexpr int kQBufBytes = 16384;        // B operand of one segment: up to 128 rows of 128 B
 
 template <bool FP8> struct Ring {
     static constexpr int kStageBytes = FP8 ? kTileK * kDI : kTileK * kDI * 2;
     static constexpr int kStages = kRingBytes / kStageBytes;
 };
+// accumulators: N columns per half (4 pieces per head for FP8), two halves per tile
+template <bool FP8, int NP> struct Acc {
+    static constexpr int kN = FP8 ? 4 * NP : NP;
+    static constexpr uint32_t kCols = 2 * kN;                                          // per tile
+    static constexpr int kStages = (int)(kTmemCols / kCols) < kMaxDStages ? (int)(kTmemCols / kCols) : kMaxDStages;
+};
 
 struct __align__(1024) IdxSmem {
     uint8_t ring[kRingBytes];                 // bf16: [2 slabs][128][128 B] per stage; fp8: [128][128 B]
-    uint8_t q[2][2 * 32 * 128];               // B operand per segment buffer: 2 K-slabs of [N heads][128 B]
+    uint8_t q[2][kQBufBytes];                 // B operand per segment buffer
     float wq[2][32];                          // head weights (times 2^-s for FP8)
     uint32_t hist[2][kHistBins];
-    uint64_t k_full[kMaxStages], k_empty[kMaxStages], a_full[kAStages], a_free[kAStages], d_full[kDStages],
-        d_free[kDStages], q_full[2], q_free[2], ep_sync, drain;
+    uint64_t k_full[kMaxStages], k_empty[kMaxStages], d_full[kMaxDStages], d_free[kMaxDStages], q_full[2], q_free[2],
+        ep_sync, drain;
     int abort_flag;
     uint32_t tmem_base;
 };
@@ -75,6 +85,7 @@ __device__ __forceinline__ void idx_fault(IdxSmem& sm, const IdxTcArgs& a) {
     sm.abort_flag = 1;
     if (a.err) atomicExch(a.err, (int)V4A_ERR_DEVICE_FAULT);
 }
+__device__ __forceinline__ bool aborted(IdxSmem& sm) { return *reinterpret_cast<volatile int*>(&sm.abort_flag) != 0; }
 
 // bounded wait taken by a whole warp: true only if every lane saw the phase complete
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity) {
@@ -119,14 +130,14 @@ __device__ void idx_producer(IdxSmem& sm, const IdxTcArgs& a, const CUtensorMap*
     ICursor cur(f0, a);
     const long long n = f1 - f0;
     for (long long jt = 0; jt < n; ++jt, cur.next(a)) {
-        if (*reinterpret_cast<volatile int*>(&sm.abort_flag)) break;
+        if (aborted(sm)) break;
         const int st = (int)(jt % kSt);
         if (jt >= kSt && !tc::mbar_wait(&sm.k_empty[st], (uint32_t)((jt / kSt) - 1) & 1)) { idx_fault(sm, a); break; }
         const int y = (int)((long long)cur.bat * a.n_ent + (long long)cur.ti * kTileK);
         uint8_t* dst = sm.ring + st * kBytes;
         tc::mbar_arrive_expect_tx(&sm.k_full[st], kBytes);
         tc::tma_load_2d(dst, kmap, 0, y, &sm.k_full[st]);
-        if (!FP8) tc::tma_load_2d(dst + kTileK * 128, kmap, 64, y, &sm.k_full[st]);
+        if (!FP8) tc::tma_load_2d(dst + kTileK * 128, kmap, 64, y, &sm.k_full[st]);  // second 64-column slab
     }
     // no copy may still be in flight when the CTA exits
     for (long long jt = n - kSt; jt < n; ++jt)
@@ -136,15 +147,16 @@ __device__ void idx_producer(IdxSmem& sm, const IdxTcArgs& a, const CUtensorMap*
 template <bool FP8, int NP>
 __device__ void idx_mma(IdxSmem& sm, const IdxTcArgs& a, uint32_t tmem, long long f0, long long f1) {
     constexpr int kSt = Ring<FP8>::kStages, kBytes = Ring<FP8>::kStageBytes;
-    constexpr uint32_t kQSlab = NP * 128;  // bytes per K-slab of q
-    constexpr uint32_t idesc = tc::idesc_f16(128, NP, 0, 0, FP8 ? 0 : 1);
+    constexpr int kDS = Acc<FP8, NP>::kStages, kN = Acc<FP8, NP>::kN;
+    constexpr uint32_t kQSlab = NP * 128;  // bf16: bytes per K-slab of q
+    constexpr uint32_t idesc = FP8 ? tc::idesc_e4m3(128, kN) : tc::idesc_f16(128, kN, 0, 0, 1);
     bool ok = true;
     int seg = 0, b = 0;
     uint64_t qd = 0;
     ICursor cur(f0, a);
     for (long long f = f0; f < f1; ++f, cur.next(a)) {
-        if (*reinterpret_cast<volatile int*>(&sm.abort_flag)) { ok = false; break; }
-        const int jt = (int)(f - f0), s = jt & 1, st = jt % kSt, sd = jt & 3;
+        if (aborted(sm)) { ok = false; break; }
+        const int jt = (int)(f - f0), st = jt % kSt, sd = jt % kDS;
         if (f == f0 || cur.ti == 0) {
             b = seg & 1;
             if (!tc::mbar_wait(&sm.q_full[b], (seg >> 1) & 1)) { ok = false; break; }
@@ -152,36 +164,35 @@ __device__ void idx_mma(IdxSmem& sm, const IdxTcArgs& a, uint32_t tmem, long lon
             ++seg;
         }
         const bool seg_end = (f == f1 - 1) || (cur.ti == a.tiles_per_row - 1);
-        if (FP8) {
-            if (!tc::mbar_wait(&sm.a_full[s], (jt >> 1) & 1)) { ok = false; break; }
-        } else {
-            if (!tc::mbar_wait(&sm.k_full[st], (jt / kSt) & 1)) { ok = false; break; }
-        }
-        if (jt >= kDStages && !tc::mbar_wait(&sm.d_free[sd], ((jt >> 2) - 1) & 1)) { ok = false; break; }
+        if (!tc::mbar_wait(&sm.k_full[st], (jt / kSt) & 1)) { ok = false; break; }
+        if (jt >= kDS && !tc::mbar_wait(&sm.d_free[sd], ((jt / kDS) - 1) & 1)) { ok = false; break; }
         tc::tc_fence_after();
-        const uint32_t d = tmem + kColD + 32 * sd;
-        if (FP8) {
-            const uint32_t at = tmem + kColA + 64 * s;
+        const uint32_t stage = tc::smem_u32(sm.ring + st * kBytes);
 #pragma unroll
-            for (int kk = 0; kk < kDI / 16; ++kk) {
-                const uint64_t bd = qd + ((((kk >> 2) * kQSlab) + (kk & 3) * 32) >> 4);
-                asm volatile(
-                    "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-                    " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d),
-                    "r"(at + 8 * kk), "l"(bd), "r"(idesc), "r"(kk ? 1u : 0u)
-                    : "memory");
-            }
-            tc::mma_commit(&sm.a_free[s]);
-        } else {
-            const uint64_t kd = tc::sw128_desc(tc::smem_u32(sm.ring + st * kBytes), 16, 1024);
+        for (int hf = 0; hf < 2; ++hf) {
+            const uint32_t d = tmem + Acc<FP8, NP>::kCols * sd + kN * hf;
+            // rows 128 hf .. 128 hf + 127 of every 128-byte slab of the tile
+            const uint64_t kd = tc::sw128_desc(stage + hf * kHalf * 128, 16, 1024);
+            if (FP8) {
+                // K = 32 e4m3 per MMA: 32 bytes along the 128-byte rows of both operands
 #pragma unroll
-            for (int kk = 0; kk < kDI / 16; ++kk) {
-                const uint64_t ad = kd + ((((kk >> 2) * (kTileK * 128)) + (kk & 3) * 32) >> 4);
-                const uint64_t bd = qd + ((((kk >> 2) * kQSlab) + (kk & 3) * 32) >> 4);
-                tc::mma_f16(d, ad, bd, idesc, kk ? 1u : 0u);
+                for (int kk = 0; kk < kDI / 32; ++kk)
+                    asm volatile(
+                        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+                        " tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n}\n" ::"r"(d),
+                        "l"(kd + (uint64_t)((kk * 32) >> 4)), "l"(qd + (uint64_t)((kk * 32) >> 4)), "r"(idesc),
+                        "r"(kk ? 1u : 0u)
+                        : "memory");
+            } else {
+#pragma unroll
+                for (int kk = 0; kk < kDI / 16; ++kk) {
+                    const uint64_t ad = kd + ((((kk >> 2) * (kTileK * 128)) + (kk & 3) * 32) >> 4);
+                    const uint64_t bd = qd + ((((kk >> 2) * kQSlab) + (kk & 3) * 32) >> 4);
+                    tc::mma_f16(d, ad, bd, idesc, kk ? 1u : 0u);
+                }
             }
-            tc::mma_commit(&sm.k_empty[st]);
         }
+        tc::mma_commit(&sm.k_empty[st]);
         tc::mma_commit(&sm.d_full[sd]);
         if (seg_end) tc::mma_commit(&sm.q_free[b]);
     }
@@ -190,16 +201,25 @@ __device__ void idx_mma(IdxSmem& sm, const IdxTcArgs& a, uint32_t tmem, long lon
     tc::mbar_wait(&sm.drain, 0);
 }
 
-// q of one row into buffer b in the B-operand layout (K-major, 128-byte
-// swizzle, NP head rows per K-slab), and the head weights; ct = 0..127
+__device__ __forceinline__ uint32_t e4m3_rn(float x) {
+    return (uint32_t)__nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3);
+}
+__device__ __forceinline__ float e4m3_value(uint32_t c) {
+    return __half2float(__half(__nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)c, __NV_E4M3)));
+}
+
+// B operand of one row into buffer b (K-major, 128-byte swizzle, 128-byte rows) and the head
+// weights; ct = 0..127.  bf16 keys: q itself (two K-slabs of NP rows).  FP8 keys: rows
+// p * NP + h hold piece p of head h (p = hi, lo, hi', lo'), one e4m3 per element.
 template <bool FP8, int NP>
 __device__ void stage_query(IdxSmem& sm, const IdxTcArgs& a, int row, int b, int ct) {
     // warp w handles heads w, w+4, ...; lane owns 4 of the 128 elements
     const int warp = ct >> 5, lane = ct & 31;
+    const int k = lane * 4;
     for (int h = warp; h < NP; h += 4) {
         float v[4] = {0.f, 0.f, 0.f, 0.f};
         if (h < a.heads_i) {
-            const __nv_bfloat16* qp = a.q + ((long long)row * a.heads_i + h) * kDI + lane * 4;
+            const __nv_bfloat16* qp = a.q + ((long long)row * a.heads_i + h) * kDI + k;
             const uint2 raw = *reinterpret_cast<const uint2*>(qp);
             v[0] = __uint_as_float(raw.x << 16);
             v[1] = __uint_as_float(raw.x & 0xffff0000u);
@@ -207,106 +227,129 @@ __device__ void stage_query(IdxSmem& sm, const IdxTcArgs& a, int row, int b, int
             v[3] = __uint_as_float(raw.y & 0xffff0000u);
         }
         float wq = h < a.heads_i ? a.w[(long long)row * a.heads_i + h] : 0.f;
-        uint32_t packed[2];
         if (FP8) {
             float amax = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
             int e = 0;
-            if (amax > 0.f) frexpf(amax, &e);  // amax = f * 2^e, f in [0.5, 1)
-            const int sh = amax > 0.f ? 14 - e : 0;  // amax * 2^sh in [2^13, 2^14)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) v[i] = ldexpf(v[i], sh);
+            if (amax > 0.f) frexpf(amax, &e);       // amax = f * 2^e, f in [0.5, 1)
+            const int sh = amax > 0.f ? 8 - e : 0;  // amax * 2^sh in [128, 256)
             wq = ldexpf(wq, -sh);
-            __half2 h0 = __floats2half2_rn(v[0], v[1]), h1 = __floats2half2_rn(v[2], v[3]);
-            packed[0] = *reinterpret_cast<uint32_t*>(&h0);
-            packed[1] = *reinterpret_cast<uint32_t*>(&h1);
+            uint32_t pc[4] = {0u, 0u, 0u, 0u};      // pieces hi, lo, hi', lo': 4 codes each
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float x = ldexpf(v[i], sh);
+                const bool big = fabsf(x) >= 0.25f;
+                const float y = big ? x : x * 1024.0f;
+                const uint32_t hi = e4m3_rn(y);
+                const uint32_t lo = e4m3_rn(y - e4m3_value(hi));
+                pc[big ? 0 : 2] |= hi << (8 * i);
+                pc[big ? 1 : 3] |= lo << (8 * i);
+            }
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+                const int n = p * NP + h;
+                uint8_t* dst = sm.q[b] + (n >> 3) * 1024 + (n & 7) * 128 + ((((k >> 4) ^ (n & 7))) << 4) + (k & 15);
+                *reinterpret_cast<uint32_t*>(dst) = pc[p];
+            }
         } else {
             __nv_bfloat162 b0 = __floats2bfloat162_rn(v[0], v[1]), b1 = __floats2bfloat162_rn(v[2], v[3]);
-            packed[0] = *reinterpret_cast<uint32_t*>(&b0);
-            packed[1] = *reinterpret_cast<uint32_t*>(&b1);
+            // element k of head h: K-slab k/64, 16-byte chunk (k%64)/8, 8-byte half
+            uint8_t* slab = sm.q[b] + (k >> 6) * (NP * 128);
+            uint8_t* dst = slab + (h >> 3) * 1024 + (h & 7) * 128 + ((((k & 63) >> 3) ^ (h & 7)) << 4) + ((k & 7) ? 8 : 0);
+            *reinterpret_cast<uint2*>(dst) =
+                make_uint2(*reinterpret_cast<uint32_t*>(&b0), *reinterpret_cast<uint32_t*>(&b1));
         }
-        // element k = 4*lane .. 4*lane+3 of head h: K-slab k/64, 16-byte chunk (k%64)/8, 8-byte half
-        const int k = lane * 4;
-        uint8_t* slab = sm.q[b] + (k >> 6) * (NP * 128);
-        uint8_t* dst = slab + (h >> 3) * 1024 + (h & 7) * 128 + ((((k & 63) >> 3) ^ (h & 7)) << 4) + ((k & 7) ? 8 : 0);
-        *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
         if (lane == 0) sm.wq[b][h] = wq;
     }
 }
 
-// warps 2-5: per segment stage q; per tile (FP8) widen the key tile to f16 in TMEM
+// warps 2-5: per segment, stage the row's B operand
 template <bool FP8, int NP>
-__device__ void idx_convert(IdxSmem& sm, const IdxTcArgs& a, uint32_t tmem, long long f0, long long f1) {
-    constexpr int kSt = Ring<FP8>::kStages, kBytes = Ring<FP8>::kStageBytes;
+__device__ void idx_stage(IdxSmem& sm, const IdxTcArgs& a, long long f0, long long f1) {
     const int ct = threadIdx.x - 64;
-    const int sub = (threadIdx.x >> 5) & 3;
-    const int r = 32 * sub + (threadIdx.x & 31);  // TMEM lane = entry row of the tile
-    const uint32_t lane_addr = (uint32_t)(32 * sub) << 16;
     bool ok = true;
     int seg = 0;
     ICursor cur(f0, a);
     for (long long f = f0; f < f1; ++f, cur.next(a)) {
+        if (f != f0 && cur.ti != 0) continue;
         if (warp_aborted(sm)) { ok = false; break; }
-        const int jt = (int)(f - f0);
-        if (f == f0 || cur.ti == 0) {
-            const int b = seg & 1;
-            if (seg >= 2 && !warp_wait(&sm.q_free[b], ((seg >> 1) - 1) & 1)) { ok = false; break; }
-            stage_query<FP8, NP>(sm, a, cur.row, b, ct);
-            tc::fence_proxy_async();
-            tc::mbar_arrive(&sm.q_full[b]);
-            ++seg;
-        }
-        if (FP8) {
-            const int s = jt & 1, st = jt % kSt;
-            if (!warp_wait(&sm.k_full[st], (jt / kSt) & 1)) { ok = false; break; }
-            if (jt >= kAStages && !warp_wait(&sm.a_free[s], ((jt >> 1) - 1) & 1)) { ok = false; break; }
-            tc::tc_fence_after();
-            const uint8_t* kr = sm.ring + st * kBytes + r * 128;
-            uint32_t cv[64];
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const uint4 raw = *reinterpret_cast<const uint4*>(kr + ((c ^ (r & 7)) << 4));
-                const uint32_t w4[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w4[i] & 0xffffu), __NV_E4M3);
-                    __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w4[i] >> 16), __NV_E4M3);
-                    cv[8 * c + 2 * i] = *reinterpret_cast<uint32_t*>(&lo);
-                    cv[8 * c + 2 * i + 1] = *reinterpret_cast<uint32_t*>(&hi);
-                }
-            }
-            tc::mbar_arrive(&sm.k_empty[st]);  // the smem tile has been read
-            tc::tmem_st_x64(tmem + lane_addr + kColA + 64 * s, cv);
-            tc::tmem_st_wait();
-            tc::tc_fence_before();
-            tc::mbar_arrive(&sm.a_full[s]);
-        }
+        const int b = seg & 1;
+        if (seg >= 2 && !warp_wait(&sm.q_free[b], ((seg >> 1) - 1) & 1)) { ok = false; break; }
+        stage_query<FP8, NP>(sm, a, cur.row, b, ct);
+        tc::fence_proxy_async();
+        tc::mbar_arrive(&sm.q_full[b]);
+        ++seg;
     }
     if (!ok) idx_fault(sm, a);
 }
 
-// warps 6-9: per tile the score of one entry per thread, its histogram count and store
+// q_j . k of the 128 entries' row of D (this thread's TMEM lane), for every head
+template <bool FP8, int NP>
+__device__ __forceinline__ float score_of(uint32_t taddr, const float* wq) {
+    float acc = 0.f;
+    if (!FP8) {
+        uint32_t dv[NP];
+        if constexpr (NP == 16) tc::tmem_ld_x16(taddr, dv);
+        else tc::tmem_ld_x32(taddr, dv);
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int h = 0; h < NP; ++h) acc = fmaf(wq[h], fmaxf(__uint_as_float(dv[h]), 0.f), acc);
+    } else if (NP == 16) {
+        uint32_t r[64];  // columns: hi | lo | hi' | lo', 16 heads each
+        tc::tmem_ld_x64(taddr, r);
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int h = 0; h < 16; ++h) {
+            const float d1 = __uint_as_float(r[h]) + __uint_as_float(r[16 + h]);
+            const float d2 = __uint_as_float(r[32 + h]) + __uint_as_float(r[48 + h]);
+            acc = fmaf(wq[h], fmaxf(fmaf(d2, 0x1p-10f, d1), 0.f), acc);
+        }
+    } else {
+        uint32_t r[64];
+        float d1[32];
+        tc::tmem_ld_x64(taddr, r);  // hi | lo of 32 heads
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int h = 0; h < 32; ++h) d1[h] = __uint_as_float(r[h]) + __uint_as_float(r[32 + h]);
+        tc::tmem_ld_x64(taddr + 64, r);  // hi' | lo'
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int h = 0; h < 32; ++h) {
+            const float d2 = __uint_as_float(r[h]) + __uint_as_float(r[32 + h]);
+            acc = fmaf(wq[h], fmaxf(fmaf(d2, 0x1p-10f, d1[h]), 0.f), acc);
+        }
+    }
+    return acc;
+}
+
+// warps 6-9: per tile the scores of entries r and r + 128 (r = this thread's TMEM lane), their
+// histogram counts and stores
 template <bool FP8, int NP>
 __device__ void idx_epilogue(IdxSmem& sm, const IdxTcArgs& a, uint32_t tmem, long long f0, long long f1) {
+    constexpr int kDS = Acc<FP8, NP>::kStages, kN = Acc<FP8, NP>::kN;
     const int et = threadIdx.x - 192;
     const int sub = (threadIdx.x >> 5) & 3;
-    const int r = 32 * sub + (threadIdx.x & 31);  // TMEM lane = entry row of the tile
+    const int r = 32 * sub + (threadIdx.x & 31);
     const uint32_t lane_addr = (uint32_t)(32 * sub) << 16;
     bool ok = true;
     int seg = 0, b = 0, nsync = 0;
     long long nv = 0;
     float* srow = nullptr;
     ICursor cur(f0, a);
-    // scale of the current tile's entry, loaded one tile ahead
-    auto scale_of = [&](const ICursor& c) -> float {
-        const long long e = (long long)c.ti * kTileK + r;
-        return e < a.n_ent ? __ldg(a.kscale + (long long)c.bat * a.n_ent + e) : 1.f;
+    // scales of the current tile's two entries, loaded one tile ahead
+    auto scales_of = [&](const ICursor& c, float (&sc)[2]) {
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+            const long long e = (long long)c.ti * kTileK + kHalf * hf + r;
+            sc[hf] = e < a.n_ent ? __ldg(a.kscale + (long long)c.bat * a.n_ent + e) : 1.f;
+        }
     };
-    float sc_cur = FP8 ? scale_of(cur) : 1.f;
+    float sc_cur[2] = {1.f, 1.f};
+    if (FP8) scales_of(cur, sc_cur);
     for (long long f = f0; f < f1; ++f) {
         if (warp_aborted(sm)) { ok = false; break; }
-        const int jt = (int)(f - f0), sd = jt & 3;
+        const int jt = (int)(f - f0), sd = jt % kDS;
         if (f == f0 || cur.ti == 0) {
             b = seg & 1;
             if (!warp_wait(&sm.q_full[b], (seg >> 1) & 1)) { ok = false; break; }
@@ -317,30 +360,32 @@ __device__ void idx_epilogue(IdxSmem& sm, const IdxTcArgs& a, uint32_t tmem, lon
         const bool seg_end = (f == f1 - 1) || (cur.ti == a.tiles_per_row - 1);
         const int ti = cur.ti, row = cur.row;
         cur.next(a);
-        float sc_next = 1.f;
-        if (FP8 && f + 1 < f1) sc_next = scale_of(cur);
-        if (!warp_wait(&sm.d_full[sd], (jt >> 2) & 1)) { ok = false; break; }
+        float sc_next[2] = {1.f, 1.f};
+        if (FP8 && f + 1 < f1) scales_of(cur, sc_next);
+        if (!warp_wait(&sm.d_full[sd], (jt / kDS) & 1)) { ok = false; break; }
         tc::tc_fence_after();
-        uint32_t dv[NP];
-        if constexpr (NP == 16) tc::tmem_ld_x16(tmem + lane_addr + kColD + 32 * sd, dv);
-        else tc::tmem_ld_x32(tmem + lane_addr + kColD + 32 * sd, dv);
-        tc::tmem_ld_wait();
+        float acc[2];
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf)
+            acc[hf] = score_of<FP8, NP>(tmem + lane_addr + Acc<FP8, NP>::kCols * sd + kN * hf, sm.wq[b]);
         tc::tc_fence_before();
         tc::mbar_arrive(&sm.d_free[sd]);
-        const long long e = (long long)ti * kTileK + r;
-        if (e < a.n_ent) {
-            float sc = -INFINITY;
-            if (e < nv) {
-                float acc = 0.f;
 #pragma unroll
-                for (int h = 0; h < NP; ++h) acc = fmaf(sm.wq[b][h], fmaxf(__uint_as_float(dv[h]), 0.f), acc);
-                if (FP8) acc *= sc_cur;
-                sc = acc + 0.0f;
-                if (a.hist) atomicAdd(&sm.hist[b][float_to_ordered(sc) >> 20], 1u);
+        for (int hf = 0; hf < 2; ++hf) {
+            const long long e = (long long)ti * kTileK + kHalf * hf + r;
+            if (e < a.n_ent) {
+                float sc = -INFINITY;
+                if (e < nv) {
+                    float v = acc[hf];
+                    if (FP8) v *= sc_cur[hf];
+                    sc = v + 0.0f;
+                    if (a.hist) atomicAdd(&sm.hist[b][float_to_ordered(sc) >> 20], 1u);
+                }
+                srow[e] = sc;
             }
-            srow[e] = sc;
         }
-        sc_cur = sc_next;
+        sc_cur[0] = sc_next[0];
+        sc_cur[1] = sc_next[1];
         if (seg_end) {
             tc::mbar_arrive(&sm.q_free[b]);  // done with wq[b]
             // every epilogue thread has counted this segment's scores (bounded, unlike a named barrier)
@@ -370,13 +415,9 @@ __global__ void __launch_bounds__(kThreads, 1) index_score_tc_kernel(const __gri
     if (threadIdx.x == 0) {
         for (int i = 0; i < Ring<FP8>::kStages; ++i) {
             tc::mbar_init(&sm.k_full[i], 1);
-            tc::mbar_init(&sm.k_empty[i], FP8 ? 128 : 1);
+            tc::mbar_init(&sm.k_empty[i], 1);
         }
-        for (int i = 0; i < kAStages; ++i) {
-            tc::mbar_init(&sm.a_full[i], 128);
-            tc::mbar_init(&sm.a_free[i], 1);
-        }
-        for (int i = 0; i < kDStages; ++i) {
+        for (int i = 0; i < Acc<FP8, NP>::kStages; ++i) {
             tc::mbar_init(&sm.d_full[i], 1);
             tc::mbar_init(&sm.d_free[i], 128);
         }
@@ -390,6 +431,8 @@ __global__ void __launch_bounds__(kThreads, 1) index_score_tc_kernel(const __gri
         tc::fence_barrier_init();
     }
     for (int i = threadIdx.x; i < 2 * kHistBins; i += kThreads) (&sm.hist[0][0])[i] = 0;
+    if (FP8)  // rows of the B buffers past 4 NP are never read, but keep them defined
+        for (int i = threadIdx.x; i < 2 * kQBufBytes / 4; i += kThreads) reinterpret_cast<uint32_t*>(sm.q)[i] = 0;
     if (warp == 1) tc::tmem_alloc(&sm.tmem_base, kTmemCols);
     tc::tc_fence_before();
     __syncthreads();
@@ -400,7 +443,7 @@ __global__ void __launch_bounds__(kThreads, 1) index_score_tc_kernel(const __gri
     } else if (warp == 1) {
         if (lane == 0) idx_mma<FP8, NP>(sm, a, tmem, f0, f1);
     } else if (warp < 6) {
-        idx_convert<FP8, NP>(sm, a, tmem, f0, f1);
+        idx_stage<FP8, NP>(sm, a, f0, f1);
     } else {
         idx_epilogue<FP8, NP>(sm, a, tmem, f0, f1);
     }

@@ -198,6 +198,10 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uin
 }
 
 // instruction descriptor: kind::f16, fp32 accumulate, A/B bf16 (fmt 1) or f16 (fmt 0)
+// instruction descriptor, kind::f8f6f4 with e4m3 A and B (format code 0), f32 accumulate, both K-major
+__host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N) {
+    return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
 __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, int a_mn, int b_mn, int ab_fmt = 1) {
     return (1u << 4) | ((uint32_t)ab_fmt << 7) | ((uint32_t)ab_fmt << 10) | ((uint32_t)a_mn << 15) |
            ((uint32_t)b_mn << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);

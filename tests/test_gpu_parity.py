@@ -102,7 +102,10 @@ def test_compress_empty_and_short(v4a):
 # ----------------------------------------------------------------------
 
 @pytest.mark.parametrize("qf,kf,HI,DI,T,L,m", [("f32", "f32", 4, 64, 1, 4096, 4), ("bf16", "bf16", 16, 128, 3, 2050, 4),
-                                              ("bf16", "e4m3", 16, 128, 5, 4099, 4), ("f32", "bf16", 1, 32, 2, 300, 8)])
+                                              ("bf16", "e4m3", 16, 128, 5, 4099, 4), ("f32", "bf16", 1, 32, 2, 300, 8),
+                                              ("bf16", "e4m3", 32, 128, 2, 4096 + 12, 4),
+                                              ("bf16", "e4m3", 5, 128, 1, 1000, 4),
+                                              ("bf16", "bf16", 24, 128, 2, 3000, 4)])
 def test_index_scores_match_oracle(v4a, qf, kf, HI, DI, T, L, m):
     c = wl.index_case(2, T, L, m, HI, DI, qf, kf, seed=11 + HI)
     N = L // m
@@ -114,9 +117,27 @@ def test_index_scores_match_oracle(v4a, qf, kf, HI, DI, T, L, m):
     check_scores(scores, ref, f"{qf}/{kf}")
 
 
+def test_index_scores_fp8_keys_tiny_query_elements(v4a):
+    """Query elements far below their head's largest one (down to 1e-9 of it)
+    must still count: the FP8-key path splits q into e4m3 pieces per magnitude
+    class, and its scores must stay within f32 rounding of the oracle."""
+    c = wl.index_case(2, 2, 4096, 4, 16, 128, "bf16", "e4m3", seed=91)
+    q = c["q_i"].float()
+    g = torch.Generator().manual_seed(92)
+    factors = torch.tensor([1.0, 1e-3, 1e-5, 1e-7, 1e-9])[torch.randint(0, 5, q.shape, generator=g)]
+    c["q_i"] = (q * factors).to(torch.bfloat16)
+    N = 4096 // 4
+    scores = torch.empty((2, 2, N), dtype=torch.float32, device="cuda")
+    v4a.v4a_index_scores(dev(c["q_i"]), dev(c["w"]), dev(c["k_i"]), dev(c["k_scale"]), scores, m=4, ctx_len=4096)
+    _sync()
+    ref = oracle.index_scores(host(c["q_i"]), host(c["w"]), host(c["k_i"]), host(c["k_scale"]), 4096, 4)
+    check_scores(scores, ref, "bf16/e4m3 tiny q elements")
+
+
 @pytest.mark.parametrize("qf,kf,HI,DI,T,L,m,k", [("f32", "f32", 4, 64, 1, 4096, 4, 64),
                                                 ("bf16", "bf16", 16, 128, 2, 8192 + 7, 4, 512),
                                                 ("bf16", "e4m3", 16, 128, 3, 16384 + 2, 4, 1024),
+                                                ("bf16", "e4m3", 32, 128, 2, 8192 + 300, 4, 256),
                                                 ("bf16", "bf16", 8, 64, 4, 40, 4, 16),   # N_vis < k: padding
                                                 ("f32", "f32", 2, 32, 1, 257, 4, 1)])
 def test_topk_matches_oracle(v4a, qf, kf, HI, DI, T, L, m, k):
