@@ -242,98 +242,154 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* s
 }
 
 // ---------------------------------------------------------------------
-// select for few query rows: histogram threshold, multi-block scan, final
+// select for few query rows: histogram threshold, then one kernel whose
+// blocks each compact one chunk of a row and whose last block per row
+// finishes that row
 // ---------------------------------------------------------------------
 constexpr int kHistBins = 4096;  // top 12 bits of the ordered key (built by the score kernels)
-constexpr int kScanThreads = 256;
+constexpr int kFastThreads = 512;
+constexpr int kFastPer = 8;                              // consecutive scores per thread per step
+constexpr int kFastStep = kFastThreads * kFastPer;       // 4096 scores per block step
 constexpr int kMaxFastRows = 256;
 constexpr int kMaxParts = 512;
-constexpr int kCandCap = 20480;  // candidates the final kernel holds in shared memory
+constexpr int kCandCap = 7168;   // candidates the finishing block holds in shared memory (two blocks fit an SM)
+constexpr size_t kFastSmem = (size_t)kCandCap * 8 + 2 * 4096 * sizeof(int32_t);
 
-// The bin holding the k-th largest key: its index, and how many keys lie in higher bins.
-// Every thread of the block gets the answer; `all` when at most k keys exist.
-__device__ void threshold_bin(const uint32_t* hist_row, int k, int* bin, int* above, bool* all) {
-    __shared__ int sb, sa, stot;
-    __shared__ int warp_buf[33];
-    const int per = kHistBins / blockDim.x;  // bins per thread (blockDim divides 4096)
-    const int b0 = threadIdx.x * per;
-    int local = 0;
-    for (int i = 0; i < per; ++i) local += (int)hist_row[b0 + i];
-    // exclusive scan over threads in DESCENDING bin order: reverse the thread index
-    int total;
-    const int rev = block_exclusive_scan_rev(local, warp_buf, &total);  // sum over higher-bin threads
-    if (threadIdx.x == 0) {
-        sb = -1;
-        sa = 0;
-        stot = total;
-    }
+// Block-wide bin search: thread t owns bins [P t, P t + P) with counts c[] (in registers).
+// Finds the bin d where the keys in bins above d number fewer than `rem` while bins >= d hold at
+// least `rem`; *above = keys above d; d = -1 when all bins together hold fewer than `rem`.
+// Per-thread sums go to shared memory, warp 0 locates the owning thread (each lane sums a run of
+// threads, read with a conflict-free swizzle, then a suffix scan over lanes), and the owner scans
+// its own P bins.  Every thread of the block gets the answer.
+template <int P>
+__device__ void block_find_bin(const int (&c)[P], long long rem, int* digit, long long* above, long long* total) {
+    __shared__ int psum[1024];
+    __shared__ int s_t, s_d;
+    __shared__ long long s_tab, s_tot, s_ab;
+    int sum = 0;
+#pragma unroll
+    for (int i = 0; i < P; ++i) sum += c[i];
+    psum[threadIdx.x] = sum;
     __syncthreads();
-    int run = rev;
-    for (int i = per - 1; i >= 0; --i) {
-        const int c = (int)hist_row[b0 + i];
-        if (run < k && run + c >= k) {
-            sb = b0 + i;
-            sa = run;
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x, nt = blockDim.x, per = (nt + 31) / 32;
+        long long local = 0;
+        for (int j = 0; j < per; ++j) {
+            const int idx = lane * per + ((j + lane / 2) % per);
+            if (idx < nt) local += psum[idx];
         }
-        run += c;
+        long long incl = local;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const long long y = __shfl_down_sync(0xffffffffu, incl, o);
+            if (lane + o < 32) incl += y;
+        }
+        const long long higher = incl - local;  // keys in threads owned by higher lanes
+        int tsel = -1;
+        long long tab = 0;
+        if (higher < rem && incl >= rem) {
+            long long run = higher;
+            for (int j = per - 1; j >= 0; --j) {
+                const int idx = lane * per + j;
+                const long long v = idx < nt ? psum[idx] : 0;
+                if (run + v >= rem) {
+                    tsel = idx;
+                    tab = run;
+                    break;
+                }
+                run += v;
+            }
+        }
+        const unsigned who = __ballot_sync(0xffffffffu, tsel >= 0);
+        const int src = who ? __ffs(who) - 1 : 0;
+        tsel = __shfl_sync(0xffffffffu, tsel, src);
+        tab = __shfl_sync(0xffffffffu, tab, src);
+        const long long tot = __shfl_sync(0xffffffffu, incl, 0);
+        if (lane == 0) {
+            s_t = who ? tsel : -1;
+            s_tab = tab;
+            s_tot = tot;
+            if (!who) {
+                s_d = -1;
+                s_ab = 0;
+            }
+        }
     }
     __syncthreads();
-    *bin = sb;
-    *above = sa;
-    *all = stot <= k;
+    if ((int)threadIdx.x == s_t) {
+        long long run = s_tab;
+        for (int i = P - 1; i >= 0; --i) {
+            if (run + c[i] >= rem) {
+                s_d = P * (int)threadIdx.x + i;
+                s_ab = run;
+                break;
+            }
+            run += c[i];
+        }
+    }
     __syncthreads();
+    *digit = s_d;
+    *above = s_ab;
+    *total = s_tot;
+    __syncthreads();  // the shared words may be reused by the next call
 }
 
-__global__ void __launch_bounds__(kScanThreads) topk_scan_kernel(const float* scores, const uint32_t* hist, IndexArgs a,
-                                                                  int k, int parts, long long chunk, int32_t* def_buf,
-                                                                  int32_t* cidx_buf, uint32_t* ckey_buf, int* counts) {
-    __shared__ int warp_buf[33];
-    const int row = blockIdx.x / parts, p = blockIdx.x % parts;
-    const long long nvis = row_nvis(a, row);
-    int tbin, above;
-    bool all;
-    threshold_bin(hist + (long long)row * kHistBins, k, &tbin, &above, &all);
-    const float* sc = scores + (long long)row * a.n_ent;
-    const long long lo = (long long)p * chunk;
-    long long hi = lo + chunk;
-    if (hi > nvis) hi = nvis;
-    int32_t* dout = def_buf + (long long)row * a.n_ent + lo;
-    int32_t* ciout = cidx_buf + (long long)row * a.n_ent + lo;
-    uint32_t* ckout = ckey_buf + (long long)row * a.n_ent + lo;
-    int n_def = 0, n_cand = 0;
-    constexpr int kPer = 16;  // scores per thread loaded ahead of the compaction
-    for (long long base0 = lo; base0 < hi; base0 += (long long)kPer * blockDim.x) {
-        uint32_t keys[kPer];
+// The bin holding the k-th largest key: its index, and how many keys lie in higher bins.
+// Every thread of the block gets the answer; `all` when at most k keys exist.  blockDim.x must
+// be kHistBins / 8 (each thread owns 8 bins).
+__device__ void threshold_bin(const uint32_t* hist_row, int k, int* bin, int* above, bool* all) {
+    const uint4* h4 = reinterpret_cast<const uint4*>(hist_row) + 2 * threadIdx.x;
+    const uint4 u = __ldcg(h4), v = __ldcg(h4 + 1);
+    const int c[8] = {(int)u.x, (int)u.y, (int)u.z, (int)u.w, (int)v.x, (int)v.y, (int)v.z, (int)v.w};
+    int d;
+    long long ab, tot;
+    block_find_bin<8>(c, k, &d, &ab, &tot);
+    *bin = d;
+    *above = (int)ab;
+    *all = tot <= k;
+}
+
+// The digit of a 1024-bin shared histogram, found by warp 0 in two levels (32 bins per lane read
+// with a conflict-free rotation, suffix scan over lanes; then the owning lane's 32 bins, one per
+// lane, scanned again) and broadcast to the block.
+__device__ void find_digit_1024(const unsigned int* h, long long rem, int* digit, long long* above) {
+    __shared__ int s_dgt;
+    __shared__ long long s_above;
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        long long local = 0;
+#pragma unroll 8
+        for (int j = 0; j < 32; ++j) local += h[32 * lane + ((j + lane) & 31)];
+        long long incl = local;
 #pragma unroll
-        for (int i = 0; i < kPer; ++i) {
-            const long long s = base0 + (long long)i * blockDim.x + threadIdx.x;
-            keys[i] = s < hi ? float_to_ordered(sc[s]) : 0u;
+        for (int o = 1; o < 32; o <<= 1) {
+            const long long y = __shfl_down_sync(0xffffffffu, incl, o);
+            if (lane + o < 32) incl += y;
         }
-#pragma unroll 1
-        for (int i = 0; i < kPer; ++i) {
-            const long long base = base0 + (long long)i * blockDim.x;
-            if (base >= hi) break;
-            const long long s = base + threadIdx.x;
-            const bool in = s < hi;
-            const uint32_t key = keys[i];
-            const int bin = (int)(key >> 20);
-            const int def = (in && (all || bin > tbin)) ? 1 : 0;
-            const int cand = (in && !all && bin == tbin) ? 1 : 0;
-            int tot;
-            const int packed = block_exclusive_scan(def | (cand << 16), warp_buf, &tot);
-            if (def) dout[n_def + (packed & 0xffff)] = (int32_t)s;
-            if (cand) {
-                ciout[n_cand + (packed >> 16)] = (int32_t)s;
-                ckout[n_cand + (packed >> 16)] = key;
-            }
-            n_def += tot & 0xffff;
-            n_cand += tot >> 16;
+        const long long higher = incl - local;
+        const unsigned who = __ballot_sync(0xffffffffu, higher < rem && incl >= rem);
+        const int L = who ? __ffs(who) - 1 : 0;
+        const long long hL = __shfl_sync(0xffffffffu, higher, L);
+        const long long v = h[32 * L + lane];
+        long long incl2 = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const long long y = __shfl_down_sync(0xffffffffu, incl2, o);
+            if (lane + o < 32) incl2 += y;
+        }
+        const long long higher2 = hL + incl2 - v;
+        const unsigned who2 = __ballot_sync(0xffffffffu, higher2 < rem && higher2 + v >= rem);
+        const int j = who2 ? __ffs(who2) - 1 : 0;
+        const long long ab = __shfl_sync(0xffffffffu, higher2, j);
+        if (lane == 0) {
+            s_dgt = who ? 32 * L + j : 0;
+            s_above = who ? ab : 0;
         }
     }
-    if (threadIdx.x == 0) {
-        counts[((long long)row * parts + p) * 2] = n_def;
-        counts[((long long)row * parts + p) * 2 + 1] = n_cand;
-    }
+    __syncthreads();
+    *digit = s_dgt;
+    *above = s_above;
+    __syncthreads();
 }
 
 // first position in sorted v[0..n) holding a value >= x
@@ -347,39 +403,37 @@ __device__ __forceinline__ int lower_bound(const int32_t* v, int n, int32_t x) {
     return lo;
 }
 
-// one block (kSelThreads) per query row
-__global__ void __launch_bounds__(kSelThreads) topk_final_kernel(const float* scores, IndexArgs a, int k, int parts,
-                                                                  long long chunk, const int32_t* def_buf,
-                                                                  const int32_t* cidx_buf, const uint32_t* ckey_buf,
-                                                                  const int* counts, int32_t* idx_out,
-                                                                  float* score_out) {
-    extern __shared__ uint32_t fs[];
-    uint32_t* ckey = fs;                                      // [kCandCap]
-    int32_t* cidx = reinterpret_cast<int32_t*>(fs + kCandCap);  // [kCandCap]
-    int32_t* defs = cidx + kCandCap;                          // [4096]
-    int32_t* sels = defs + 4096;                              // [4096]
+// The row's answer from the parts' compacted lists: every definite entry (key in a bin above the
+// threshold bin) plus the best `need` candidates (keys in the threshold bin), ties to the lower
+// entry, in ascending entry order, padded with -1.  Whole block; the parts' writes are visible.
+__device__ void finish_row(const float* sc, long long nvis, int k, int parts, long long chunk, const int32_t* def_row,
+                           const int32_t* cidx_row, const uint32_t* ckey_row, const int* counts_row, int32_t* io,
+                           float* so, uint8_t* dsm) {
+    uint32_t* ckey = reinterpret_cast<uint32_t*>(dsm);           // [kCandCap]
+    int32_t* cidx = reinterpret_cast<int32_t*>(ckey + kCandCap);  // [kCandCap]
+    int32_t* defs = cidx + kCandCap;                              // [4096]
+    int32_t* sels = defs + 4096;                                  // [4096]
     __shared__ int doff[kMaxParts + 1], coff[kMaxParts + 1];
     __shared__ unsigned int h1[1024];
     __shared__ int warp_buf[33];
-
-    const int row = blockIdx.x;
-    const long long nvis = row_nvis(a, row);
-    int32_t* io = idx_out + (long long)row * k;
-    float* so = score_out ? score_out + (long long)row * k : nullptr;
-    const float* sc = scores + (long long)row * a.n_ent;
-    for (int p = threadIdx.x; p < parts; p += blockDim.x) {
-        doff[p + 1] = counts[((long long)row * parts + p) * 2];
-        coff[p + 1] = counts[((long long)row * parts + p) * 2 + 1];
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        doff[0] = coff[0] = 0;
-        for (int p = 1; p <= parts; ++p) {
-            doff[p] += doff[p - 1];
-            coff[p] += coff[p - 1];
+    {
+        // prefix sums of the parts' counts (parts <= kMaxParts = blockDim)
+        const int p = threadIdx.x;
+        const int nd = p < parts ? __ldcg(counts_row + 2 * p) : 0;
+        const int nc = p < parts ? __ldcg(counts_row + 2 * p + 1) : 0;
+        int td, tc;
+        const int ed = block_exclusive_scan(nd, warp_buf, &td);
+        const int ec = block_exclusive_scan(nc, warp_buf, &tc);
+        if (p < parts) {
+            doff[p] = ed;
+            coff[p] = ec;
         }
+        if (p == 0) {
+            doff[parts] = td;
+            coff[parts] = tc;
+        }
+        __syncthreads();
     }
-    __syncthreads();
     const int D = doff[parts], C = coff[parts];
     if (C > kCandCap || D > 4096) {
         // more candidates than the fast path holds (e.g. huge blocks of equal scores): exact select over the row
@@ -387,24 +441,50 @@ __global__ void __launch_bounds__(kSelThreads) topk_final_kernel(const float* sc
         return;
     }
     // gather the definite entries and the candidates, both in ascending entry order; every element
-    // finds its part by binary search over the offsets, so all loads are independent
-    const long long row_off = (long long)row * a.n_ent;
-    for (int e = threadIdx.x; e < D + C; e += blockDim.x) {
-        const bool is_def = e < D;
-        const int x = is_def ? e : e - D;
-        const int* off = is_def ? doff : coff;
-        int lo = 0, hi = parts;  // largest p with off[p] <= x
-        while (hi - lo > 1) {
-            const int mid = (lo + hi) >> 1;
-            if (off[mid] <= x) lo = mid;
-            else hi = mid;
+    // finds its part by binary search over the offsets, and each thread issues the loads of up to
+    // kG elements before using any of them
+    constexpr int kG = 8;
+    for (int e0 = threadIdx.x; e0 < D + C; e0 += kG * blockDim.x) {
+        long long src[kG];
+        int32_t vi[kG];
+        uint32_t vk[kG];
+#pragma unroll
+        for (int g = 0; g < kG; ++g) {
+            const int e = e0 + g * blockDim.x;
+            src[g] = -1;
+            if (e < D + C) {
+                const bool is_def = e < D;
+                const int x = is_def ? e : e - D;
+                const int* off = is_def ? doff : coff;
+                int lo = 0, hi = parts;  // largest p with off[p] <= x
+                while (hi - lo > 1) {
+                    const int mid = (lo + hi) >> 1;
+                    if (off[mid] <= x) lo = mid;
+                    else hi = mid;
+                }
+                src[g] = (long long)lo * chunk + (x - off[lo]);
+            }
         }
-        const long long src = row_off + (long long)lo * chunk + (x - off[lo]);
-        if (is_def) {
-            defs[x] = def_buf[src];
-        } else {
-            cidx[x] = cidx_buf[src];
-            ckey[x] = ckey_buf[src];
+#pragma unroll
+        for (int g = 0; g < kG; ++g) {
+            const int e = e0 + g * blockDim.x;
+            vi[g] = 0;
+            vk[g] = 0;
+            if (src[g] >= 0) {
+                vi[g] = e < D ? __ldcg(def_row + src[g]) : __ldcg(cidx_row + src[g]);
+                if (e >= D) vk[g] = __ldcg(ckey_row + src[g]);
+            }
+        }
+#pragma unroll
+        for (int g = 0; g < kG; ++g) {
+            const int e = e0 + g * blockDim.x;
+            if (src[g] < 0) continue;
+            if (e < D) {
+                defs[e] = vi[g];
+            } else {
+                cidx[e - D] = vi[g];
+                ckey[e - D] = vk[g];
+            }
         }
     }
     const int need = (D + C) < k ? C : k - D;  // candidates to take
@@ -421,34 +501,55 @@ __global__ void __launch_bounds__(kSelThreads) topk_final_kernel(const float* sc
             __syncthreads();
             int dgt;
             long long above;
-            find_digit(h1, 1024, rem, &dgt, &above);
+            find_digit_1024(h1, rem, &dgt, &above);
             prefix |= (uint32_t)dgt << shift;
             rem -= (int)above;
             mask |= 1023u << shift;
         }
     }
-    // mark: key > prefix, or key == prefix among the first `rem` such (in entry order)
+    // mark: key > prefix, or key == prefix among the first `rem` such (in entry order).  Thread t
+    // takes candidates [t*per, t*per + per) into registers; two block scans give the equal-key ranks
+    // and the output positions; the compacted keys go back into ckey after everyone has read.
     const bool take_all = need >= C;
-    int out = 0, eq_seen = 0;
-    for (int base = 0; base < C; base += blockDim.x) {
-        const int i = base + threadIdx.x;
-        const bool in = i < C;
-        const uint32_t key = in ? ckey[i] : 0u;
-        const int gt = (in && (take_all || key > prefix)) ? 1 : 0;
-        const int eq = (in && !take_all && key == prefix) ? 1 : 0;
-        int eq_tot;
-        const int eq_rank = eq_seen + block_exclusive_scan(eq, warp_buf, &eq_tot);
-        const int sel = gt | ((eq && eq_rank < rem) ? 1 : 0);
-        int sel_tot;
-        const int pos = out + block_exclusive_scan(sel, warp_buf, &sel_tot);
-        if (sel) {
-            sels[pos] = cidx[i];
-            ckey[pos] = key;  // compacted in place: pos <= i
-        }
-        __syncthreads();
-        out += sel_tot;
-        eq_seen += eq_tot;
+    constexpr int kMaxPer = kCandCap / kFastThreads;
+    const int per = (C + (int)blockDim.x - 1) / (int)blockDim.x;
+    const int i0 = threadIdx.x * per;
+    uint32_t mk[kMaxPer];
+    int32_t mi[kMaxPer];
+    int n_eq = 0;
+#pragma unroll
+    for (int j = 0; j < kMaxPer; ++j) {
+        const int i = i0 + j;
+        const bool in = j < per && i < C;
+        mk[j] = in ? ckey[i] : 0u;
+        mi[j] = in ? cidx[i] : -1;
+        n_eq += (in && !take_all && mk[j] == prefix) ? 1 : 0;
     }
+    int eq_tot;
+    int eq_rank = block_exclusive_scan(n_eq, warp_buf, &eq_tot);
+    uint32_t selmask = 0;
+    int n_sel = 0;
+#pragma unroll
+    for (int j = 0; j < kMaxPer; ++j) {
+        const bool in = mi[j] >= 0;
+        const bool gt = in && (take_all || mk[j] > prefix);
+        const bool eq = in && !take_all && mk[j] == prefix;
+        const bool sel = gt || (eq && eq_rank < rem);
+        eq_rank += eq ? 1 : 0;
+        if (sel) {
+            selmask |= 1u << j;
+            ++n_sel;
+        }
+    }
+    int out;
+    int pos = block_exclusive_scan(n_sel, warp_buf, &out);  // ends with a barrier: all reads are done
+#pragma unroll
+    for (int j = 0; j < kMaxPer; ++j)
+        if (selmask & (1u << j)) {
+            sels[pos] = mi[j];
+            ckey[pos] = mk[j];
+            ++pos;
+        }
     __syncthreads();
     const int total = D + out;
     // merge the two ascending lists into the output
@@ -468,6 +569,75 @@ __global__ void __launch_bounds__(kSelThreads) topk_final_kernel(const float* sc
         io[p] = -1;
         if (so) so[p] = -INFINITY;
     }
+}
+
+// grid rows * parts, kFastThreads threads.  Block (row, p) compacts entries [p*chunk, (p+1)*chunk)
+// of the row: definite entries (bin above the threshold bin) and candidates (the threshold bin),
+// each in ascending entry order; the last block of the row to finish (counted on row_done, which
+// starts at zero) then finishes the row.
+__global__ void __launch_bounds__(kFastThreads) topk_fast_kernel(const float* scores, const uint32_t* hist, IndexArgs a,
+                                                                 int k, int parts, long long chunk, int32_t* def_buf,
+                                                                 int32_t* cidx_buf, uint32_t* ckey_buf, int* counts,
+                                                                 unsigned int* row_done, int32_t* idx_out,
+                                                                 float* score_out) {
+    extern __shared__ __align__(16) uint8_t dsm[];
+    __shared__ int warp_buf[33];
+    __shared__ int s_last;
+    const int row = blockIdx.x / parts, p = blockIdx.x % parts;
+    const long long nvis = row_nvis(a, row);
+    int tbin, above;
+    bool all;
+    threshold_bin(hist + (long long)row * kHistBins, k, &tbin, &above, &all);
+    const float* sc = scores + (long long)row * a.n_ent;
+    const long long row_off = (long long)row * a.n_ent;
+    const long long lo = (long long)p * chunk;
+    long long hi = lo + chunk;
+    if (hi > nvis) hi = nvis;
+    int32_t* dout = def_buf + row_off + lo;
+    int32_t* ciout = cidx_buf + row_off + lo;
+    uint32_t* ckout = ckey_buf + row_off + lo;
+    int n_def = 0, n_cand = 0;
+    for (long long base = lo; base < hi; base += kFastStep) {
+        // this thread's kFastPer consecutive scores
+        const long long s0 = base + (long long)threadIdx.x * kFastPer;
+        uint32_t keys[kFastPer];
+        int nd = 0, nc = 0;
+#pragma unroll
+        for (int i = 0; i < kFastPer; ++i) {
+            const long long s = s0 + i;
+            keys[i] = s < hi ? float_to_ordered(sc[s]) : 0u;  // L1 serves the warp's 1 KB after its first load
+            const int bin = (int)(keys[i] >> 20);
+            nd += (s < hi && (all || bin > tbin)) ? 1 : 0;
+            nc += (s < hi && !all && bin == tbin) ? 1 : 0;
+        }
+        int tot;
+        const int packed = block_exclusive_scan(nd | (nc << 16), warp_buf, &tot);
+        int od = n_def + (packed & 0xffff), oc = n_cand + (packed >> 16);
+#pragma unroll
+        for (int i = 0; i < kFastPer; ++i) {
+            const long long s = s0 + i;
+            const int bin = (int)(keys[i] >> 20);
+            if (s < hi && (all || bin > tbin)) dout[od++] = (int32_t)s;
+            if (s < hi && !all && bin == tbin) {
+                ciout[oc] = (int32_t)s;
+                ckout[oc++] = keys[i];
+            }
+        }
+        n_def += tot & 0xffff;
+        n_cand += tot >> 16;
+    }
+    if (threadIdx.x == 0) {
+        counts[((long long)row * parts + p) * 2] = n_def;
+        counts[((long long)row * parts + p) * 2 + 1] = n_cand;
+        __threadfence();  // this part's lists and counts are visible before it is counted
+        s_last = atomicAdd(row_done + row, 1u) == (unsigned)(parts - 1);
+    }
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    finish_row(sc, nvis, k, parts, chunk, def_buf + row_off, cidx_buf + row_off, ckey_buf + row_off,
+               counts + (long long)row * parts * 2, idx_out + (long long)row * k,
+               score_out ? score_out + (long long)row * k : nullptr, dsm);
 }
 
 template <int HMAX>
@@ -520,15 +690,14 @@ static TopkPlan topk_plan(const IndexArgs& a) {
         p.total = off;
         return p;
     }
-    long long parts = (2LL * kNumSMs + rows - 1) / rows;
-    const long long max_parts = (n + 1023) / 1024;
-    if (parts > max_parts) parts = max_parts;
+    // parts of kFastStep scores (more per part only if a row would need more than kMaxParts)
+    long long parts = (n + kFastStep - 1) / kFastStep;
     if (parts > kMaxParts) parts = kMaxParts;
     if (parts < 1) parts = 1;
     p.parts = (int)parts;
-    p.chunk = ((n + parts - 1) / parts + kScanThreads - 1) / kScanThreads * kScanThreads;
-    p.off_hist = off;
-    off = align256(off + (size_t)rows * kHistBins * sizeof(uint32_t));
+    p.chunk = ((n + parts - 1) / parts + kFastStep - 1) / kFastStep * kFastStep;
+    p.off_hist = off;  // histograms, then one finished-parts counter per row: zeroed together
+    off = align256(off + (size_t)rows * (kHistBins + 1) * sizeof(uint32_t));
     p.off_cnt = off;
     off = align256(off + (size_t)rows * p.parts * 2 * sizeof(int));
     p.off_def = off;
@@ -588,7 +757,8 @@ cudaError_t launch_topk(const IndexArgs& a, int k, int32_t* idx_out, float* scor
     int32_t* def_buf = reinterpret_cast<int32_t*>(base + p.off_def);
     int32_t* cidx = reinterpret_cast<int32_t*>(base + p.off_cidx);
     uint32_t* ckey = reinterpret_cast<uint32_t*>(base + p.off_ckey);
-    e = cudaMemsetAsync(hist, 0, (size_t)rows * kHistBins * sizeof(uint32_t), stream);
+    unsigned int* row_done = hist + (size_t)rows * kHistBins;
+    e = cudaMemsetAsync(hist, 0, (size_t)rows * (kHistBins + 1) * sizeof(uint32_t), stream);
     if (e != cudaSuccess) return e;
     if (index_tc_available(a)) {
         e = launch_index_scores_tc(a, scores, hist, nullptr, stream);
@@ -600,15 +770,11 @@ cudaError_t launch_topk(const IndexArgs& a, int k, int32_t* idx_out, float* scor
         }
     }
     if (e != cudaSuccess) return e;
-    topk_scan_kernel<<<rows * p.parts, kScanThreads, 0, stream>>>(scores, hist, a, k, p.parts, p.chunk, def_buf, cidx,
-                                                                   ckey, counts);
-    e = cudaGetLastError();
+    e = cudaFuncSetAttribute(topk_fast_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFastSmem);
     if (e != cudaSuccess) return e;
-    const size_t smem = (size_t)kCandCap * 8 + 2 * 4096 * sizeof(int32_t);
-    e = cudaFuncSetAttribute(topk_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    topk_final_kernel<<<rows, kSelThreads, smem, stream>>>(scores, a, k, p.parts, p.chunk, def_buf, cidx, ckey, counts,
-                                                           idx_out, score_out);
+    topk_fast_kernel<<<rows * p.parts, kFastThreads, kFastSmem, stream>>>(scores, hist, a, k, p.parts, p.chunk, def_buf,
+                                                                          cidx, ckey, counts, row_done, idx_out,
+                                                                          score_out);
     return cudaGetLastError();
 }
 
