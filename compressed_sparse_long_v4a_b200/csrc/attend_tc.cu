@@ -441,14 +441,19 @@ __device__ void softmax_warps(Smem& sm, const TcArgs& a, uint32_t tmem, long lon
                 tc::tmem_ld_x64(tmem + lane_addr + kColO + 64 * cc, o);
                 tc::tmem_ld_wait();
                 const int d = 128 * cc + 32 * sub + lane;
+                if (whole) {
 #pragma unroll
-                for (int i = 0; i < kH; ++i) {
-                    float v = __uint_as_float(o[i]);
-                    if (whole) {
+                    for (int i = 0; i < kH; ++i) {
                         const float l = sm.l_s[i];
-                        v = l > 0.f ? v / l : 0.f;
+                        dst[i * kD + d] = l > 0.f ? __uint_as_float(o[i]) / l : 0.f;
                     }
-                    dst[i * kD + d] = v;
+                } else {
+                    // a piece is stored d-major ([d][64 heads]): this thread's 64 heads are contiguous
+                    float4* pd = reinterpret_cast<float4*>(dst + (long long)d * kH);
+#pragma unroll
+                    for (int i = 0; i < kH / 4; ++i)
+                        pd[i] = make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
+                                            __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
                 }
             }
             tc::tc_fence_before();
@@ -515,9 +520,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // Merge the partials of queries whose tiles were split between CTAs.
-// grid (rows, 64 heads), 128 threads x 4 elements.
-__global__ void attend_tc_combine(TcArgs a) {
-    const int row = blockIdx.x, h = blockIdx.y;
+// grid (rows, 512 / 32 d chunks), 256 threads.  Pieces are stored d-major
+// ([d][64 heads]); each block reads its 32 d x 64 heads of every piece
+// (coalesced along heads), weights them by exp2(m_piece - m_max) per head,
+// and writes out[row][h][d0 .. d0 + 31] through a shared-memory transpose.
+__global__ void __launch_bounds__(256) attend_tc_combine(TcArgs a) {
+    constexpr int kDC = 32;  // d per block
+    const int row = blockIdx.x, d0 = blockIdx.y * kDC;
     const long long rs = (long long)row * a.tpr, re = rs + a.tpr - 1;
     // CTA holding flat tile f: the largest c with range_start(c) <= f
     auto cta_of = [&](long long f) { return (int)(((f + 1) * a.grid - 1) / a.total_tiles); };
@@ -525,62 +534,59 @@ __global__ void attend_tc_combine(TcArgs a) {
     if (c0 == c1) return;  // written directly by its only CTA
     // the first CTA's piece is its first query only if the query starts its range; every later CTA's
     // range starts inside this query, so the piece is that CTA's first (slot 2c)
-    constexpr int kPer = 5, kMaxPieces = 32 * kPer;  // covers a query split over every CTA (grid <= 148)
     const int n = c1 - c0 + 1;
-    __shared__ float s_w[kMaxPieces];
-    __shared__ float s_l;
-    __shared__ int s_bad;
-    if (threadIdx.x < 32) {
-        float ms[kPer], ls[kPer];
+    constexpr int kMaxPieces = kNumSMs;  // a query split over every CTA (grid <= 148)
+    __shared__ float s_w[kMaxPieces][kH];  // weight of piece i for head h, divided by the head's total
+    __shared__ int s_slot[kMaxPieces];
+    __shared__ float s_acc[kH][kDC + 1];
+    const int t = threadIdx.x;
+    for (int i = t; i < n; i += blockDim.x)
+        s_slot[i] = 2 * (c0 + i) + ((i == 0 && range_start(c0, a) < rs) ? 1 : 0);
+    __syncthreads();
+    if (t < kH) {
+        const int h = t;
         float mmax = -INFINITY;
         bool bad = false;
-#pragma unroll
-        for (int u = 0; u < kPer; ++u) {
-            const int i = threadIdx.x + 32 * u;
-            ms[u] = -INFINITY;
-            ls[u] = 0.f;
-            if (i < n) {
-                const int c = c0 + i;
-                const int slot = 2 * c + ((i == 0 && range_start(c0, a) < rs) ? 1 : 0);
-                ms[u] = a.part_ml[((long long)slot * kH + h) * 2];
-                ls[u] = a.part_ml[((long long)slot * kH + h) * 2 + 1];
-                bad |= isnan(ms[u]) || isnan(ls[u]);
-                mmax = fmaxf(mmax, ms[u]);
-            }
+        for (int i = 0; i < n; ++i) {
+            const float m = a.part_ml[((long long)s_slot[i] * kH + h) * 2];
+            bad |= isnan(m);
+            mmax = fmaxf(mmax, m);
         }
-        mmax = group_max<32>(mmax);
-        bad = __any_sync(0xffffffffu, bad);
         float l = 0.f;
-#pragma unroll
-        for (int u = 0; u < kPer; ++u) {
-            const int i = threadIdx.x + 32 * u;
-            const float wgt = (i < n && ms[u] != -INFINITY && mmax != -INFINITY) ? exp2f(ms[u] - mmax) : 0.f;
-            if (i < n) s_w[i] = wgt;
-            l += wgt * ls[u];
+        for (int i = 0; i < n; ++i) {
+            const float m = a.part_ml[((long long)s_slot[i] * kH + h) * 2];
+            const float li = a.part_ml[((long long)s_slot[i] * kH + h) * 2 + 1];
+            bad |= isnan(li);
+            const float wgt = (m != -INFINITY && mmax != -INFINITY) ? exp2f(m - mmax) : 0.f;
+            s_w[i][h] = wgt;
+            l += wgt * li;
         }
-        l = group_sum<32>(l);
-        if (threadIdx.x == 0) {
-            s_l = l;
-            s_bad = bad;
-        }
+        const float inv = bad ? NAN : (l > 0.f ? 1.f / l : 0.f);
+        for (int i = 0; i < n; ++i) s_w[i][h] *= inv;
+        if (bad || !(l > 0.f)) s_w[0][h] = bad ? NAN : 0.f;  // NaN poisons, an empty row stays zero
     }
     __syncthreads();
-    const int e = threadIdx.x * 4;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    // thread t: head h = t % 64, d rows dd = t / 64, + 4, ... (8 of the 32)
+    const int h = t & (kH - 1), dq = t >> 6;
+    float acc[kDC / 4];
+#pragma unroll
+    for (int j = 0; j < kDC / 4; ++j) acc[j] = 0.f;
     for (int i = 0; i < n; ++i) {
-        const float wgt = s_w[i];
+        const float wgt = s_w[i][h];
         if (wgt == 0.f) continue;
-        const int c = c0 + i;
-        const int slot = 2 * c + ((i == 0 && range_start(c0, a) < rs) ? 1 : 0);
-        const float4 v = *reinterpret_cast<const float4*>(a.part_o + ((long long)slot * kH + h) * kD + e);
-        acc.x = fmaf(wgt, v.x, acc.x);
-        acc.y = fmaf(wgt, v.y, acc.y);
-        acc.z = fmaf(wgt, v.z, acc.z);
-        acc.w = fmaf(wgt, v.w, acc.w);
+        const float* pp = a.part_o + (long long)s_slot[i] * kH * kD + (long long)d0 * kH + h;
+#pragma unroll
+        for (int j = 0; j < kDC / 4; ++j) acc[j] = fmaf(wgt, pp[(long long)(dq + 4 * j) * kH], acc[j]);
     }
-    const float inv = s_bad ? NAN : (s_l > 0.f ? 1.f / s_l : 0.f);
-    *reinterpret_cast<float4*>(a.out + ((long long)row * kH + h) * kD + e) =
-        make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+    // a poisoned head makes its whole output NaN
+    const float w0 = s_w[0][h];
+#pragma unroll
+    for (int j = 0; j < kDC / 4; ++j) s_acc[h][dq + 4 * j] = isnan(w0) ? NAN : acc[j];
+    __syncthreads();
+    // write out[row][h][d0 .. d0+31]: warp w covers heads w, w+8, ...; lane = d
+    const int lane = t & 31, w = t >> 5;
+    for (int hh = w; hh < kH; hh += 8)
+        a.out[((long long)row * kH + hh) * kD + d0 + lane] = s_acc[hh][lane];
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -693,7 +699,7 @@ cudaError_t launch_attend_tc(const AttendArgs& a, void* ws, size_t ws_bytes, cud
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     if (p.grid > 1) {
-        attend_tc_combine<<<dim3(t.rows, kH), kD / 4, 0, stream>>>(t);
+        attend_tc_combine<<<dim3(t.rows, kD / 32), 256, 0, stream>>>(t);
         e = cudaGetLastError();
     }
     return e;
