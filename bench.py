@@ -49,6 +49,8 @@ def parse():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=20.0, help="budget of the oracle sample")
+    p.add_argument("--profile-steps", action="store_true",
+                   help="run the warm-up and K steps eagerly and exit (the command ncu captures are taken on)")
     return p.parse_args()
 
 
@@ -232,6 +234,15 @@ class Step:
         self.csa_attend()
         self.hca_attend()
 
+    def csa_layer(self):
+        self.compress_csa()
+        self.topk()
+        self.csa_attend()
+
+    def hca_layer(self):
+        self.compress_hca()
+        self.hca_attend()
+
     # bytes ------------------------------------------------------------
     def algorithmic_bytes(self):
         """Bytes the method must read per step (indexer keys + scales, selected
@@ -297,6 +308,39 @@ def time_op(fn, reps: int, flush: torch.Tensor) -> float:
         return best
 
     return max(0.0, (timed(True) - timed(False)) / reps)
+
+
+def layer_times(fn, reps: int) -> list:
+    """Device ms of each of `reps` back-to-back replays of fn captured as one
+    CUDA graph (the layer's inputs are larger than L2)."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    for _ in range(3):
+        g.replay()
+    s = torch.cuda.current_stream()
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
+    evs[0].record(s)
+    for i in range(reps):
+        g.replay()
+        evs[i + 1].record(s)
+    torch.cuda.synchronize()
+    del g
+    return [evs[i].elapsed_time(evs[i + 1]) for i in range(reps)]
+
+
+def pct(xs, q):
+    xs = sorted(xs)
+    return xs[min(len(xs) - 1, max(0, int(round(q / 100.0 * (len(xs) - 1)))))]
+
+
+def source_digest(paths) -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 # ----------------------------------------------------------------------
@@ -373,6 +417,11 @@ def main():
     args.warmup = max(3, args.warmup)
     step = Step(seed_offset=rank)
     s = torch.cuda.current_stream()
+    if args.profile_steps:
+        for _ in range(args.warmup + args.steps):
+            step.run()
+        torch.cuda.synchronize()
+        return
 
     # warm-up (also loads every kernel before capture)
     for _ in range(args.warmup):
@@ -417,16 +466,43 @@ def main():
         pass
     peak = float(peaks.get("hbm_gbs", 6650.0))
     achieved = ab[dom] / (op_ms[dom] / 1000.0) / 1e9
+    # DRAM bytes per launch of the dominant op's kernels from the committed ncu capture, kept only
+    # while the kernel sources are the ones it was taken from
     traffic = None
+    traffic_note = "no capture"
     try:
         tr = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))
-        traffic = tr.get(dom)
+        ent = tr.get(dom)
+        if ent:
+            if source_digest(ent["sources"]) == ent["source_digest"]:
+                traffic = ent["bytes_per_launch"]
+                traffic_note = ent["note"]
+            else:
+                traffic_note = "kernel changed since the capture"
     except Exception:
         pass
+    nominal = 8000.0
     roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "GB/s",
-                "frac": achieved / peak, "traffic": traffic,
+                "frac": achieved / peak, "traffic": traffic, "traffic_note": traffic_note,
                 "peak_source": "measured" if "hbm_gbs" in peaks else "fallback",
+                "peak_nominal": nominal, "frac_nominal": achieved / nominal,
                 "algorithmic_bytes": ab[dom], "ms": op_ms[dom]}
+
+    # per-layer decode: >= 100 graph replays of each layer, median / p10 / p90
+    lreps = 100
+    layers = {}
+    for name, fn, seqs, nbytes in (("csa", step.csa_layer, step.Bc, ab["topk"] + ab["csa_attend"]),
+                                   ("hca", step.hca_layer, step.Bh, ab["hca_attend"])):
+        ts = layer_times(fn, lreps)
+        med = statistics.median(ts)
+        layers[name] = {"tokens_per_s_median": seqs / (med / 1000.0),
+                        "tokens_per_s_p10": seqs / (pct(ts, 90) / 1000.0),
+                        "tokens_per_s_p90": seqs / (pct(ts, 10) / 1000.0),
+                        "ms_median": med, "ms_p10": pct(ts, 10), "ms_p90": pct(ts, 90), "replays": lreps,
+                        "algorithmic_bytes": nbytes,
+                        "hbm_gbs_median": nbytes / (med / 1000.0) / 1e9,
+                        "frac_measured_peak": nbytes / (med / 1000.0) / 1e9 / peak,
+                        "frac_nominal_peak": nbytes / (med / 1000.0) / 1e9 / nominal}
 
     # end to end through the public API: per-step inputs from pinned host memory, outputs back
     hin = step.host_in
@@ -482,10 +558,7 @@ def main():
                            "step_algorithmic_bytes": ab["total"],
                            "step_hbm_gbs": total_bytes / (ms / 1000.0) / 1e9 / world,
                            "op_ms": op_ms,
-                           "per_layer_tokens_per_s": {"csa": step.Bc / (op_ms["compress_csa"] + op_ms["topk"] +
-                                                                        op_ms["csa_attend"]) * 1000.0,
-                                                      "hca": step.Bh / (op_ms["compress_hca"] +
-                                                                        op_ms["hca_attend"]) * 1000.0}},
+                           "layers": layers},
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": (launches_per_step * args.steps) if launches_per_step else None,
                 "gpu_launches_per_step": launches_per_step,
