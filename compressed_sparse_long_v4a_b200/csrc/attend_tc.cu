@@ -547,12 +547,14 @@ __global__ void __launch_bounds__(256) attend_tc_combine(TcArgs a) {
         const int h = t;
         float mmax = -INFINITY;
         bool bad = false;
+#pragma unroll 4
         for (int i = 0; i < n; ++i) {
             const float m = a.part_ml[((long long)s_slot[i] * kH + h) * 2];
             bad |= isnan(m);
             mmax = fmaxf(mmax, m);
         }
         float l = 0.f;
+#pragma unroll 4
         for (int i = 0; i < n; ++i) {
             const float m = a.part_ml[((long long)s_slot[i] * kH + h) * 2];
             const float li = a.part_ml[((long long)s_slot[i] * kH + h) * 2 + 1];
@@ -566,15 +568,32 @@ __global__ void __launch_bounds__(256) attend_tc_combine(TcArgs a) {
         if (bad || !(l > 0.f)) s_w[0][h] = bad ? NAN : 0.f;  // NaN poisons, an empty row stays zero
     }
     __syncthreads();
-    // thread t: head h = t % 64, d rows dd = t / 64, + 4, ... (8 of the 32)
+    // thread t: head h = t % 64, d rows dq, dq + 4, ... (8 of the 32); the loads of 4 pieces are
+    // issued before any of them is used (a piece of weight 0 holds finite values: it adds 0)
     const int h = t & (kH - 1), dq = t >> 6;
     float acc[kDC / 4];
 #pragma unroll
     for (int j = 0; j < kDC / 4; ++j) acc[j] = 0.f;
-    for (int i = 0; i < n; ++i) {
-        const float wgt = s_w[i][h];
-        if (wgt == 0.f) continue;
-        const float* pp = a.part_o + (long long)s_slot[i] * kH * kD + (long long)d0 * kH + h;
+    constexpr int kU = 4;
+    int i0 = 0;
+    for (; i0 + kU <= n; i0 += kU) {
+        float v[kU][kDC / 4];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const float* pp = a.part_o + (long long)s_slot[i0 + u] * kH * kD + (long long)d0 * kH + h;
+#pragma unroll
+            for (int j = 0; j < kDC / 4; ++j) v[u][j] = pp[(long long)(dq + 4 * j) * kH];
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const float wgt = s_w[i0 + u][h];
+#pragma unroll
+            for (int j = 0; j < kDC / 4; ++j) acc[j] = fmaf(wgt, v[u][j], acc[j]);
+        }
+    }
+    for (; i0 < n; ++i0) {
+        const float wgt = s_w[i0][h];
+        const float* pp = a.part_o + (long long)s_slot[i0] * kH * kD + (long long)d0 * kH + h;
 #pragma unroll
         for (int j = 0; j < kDC / 4; ++j) acc[j] = fmaf(wgt, pp[(long long)(dq + 4 * j) * kH], acc[j]);
     }
