@@ -22,6 +22,10 @@
 //    into the head weight).  These MMAs accumulate in f32 at least as
 //    precisely as a sequential f32 sum (measured on B200), so the score keeps
 //    f32 accuracy without widening the keys.
+// Several queries of one sequence (prefill) are scored together: the B operand
+// then holds G queries' heads (N = G x heads for bf16 keys, G x 4 x heads for
+// FP8), so every key tile is read once per G queries and each MMA does G
+// times the work.
 // Warp 0 loads key tiles into a shared-memory ring (4 x 32 KB for FP8, 2 x 64
 // KB for bf16), warp 1 issues the MMAs, warps 2-5 stage each row's B
 // operand, warps 6-9 run the epilogue.  CTAs take contiguous ranges of the
@@ -52,17 +56,20 @@ template <bool FP8> struct Ring {
     static constexpr int kStageBytes = FP8 ? kTileK * kDI : kTileK * kDI * 2;
     static constexpr int kStages = kRingBytes / kStageBytes;
 };
-// accumulators: N columns per half (4 pieces per head for FP8), two halves per tile
-template <bool FP8, int NP> struct Acc {
-    static constexpr int kN = FP8 ? 4 * NP : NP;
+// accumulators: N columns per half (4 pieces per head for FP8, for each of G queries), two halves
+// per tile
+template <bool FP8, int NP, int G> struct Acc {
+    static constexpr int kNq = FP8 ? 4 * NP : NP;  // columns of one query
+    static constexpr int kN = kNq * G;
     static constexpr uint32_t kCols = 2 * kN;                                          // per tile
     static constexpr int kStages = (int)(kTmemCols / kCols) < kMaxDStages ? (int)(kTmemCols / kCols) : kMaxDStages;
+    static_assert(kN <= 128 && kN * 128 * (FP8 ? 1 : 2) <= 16384, "B operand exceeds its buffer");
 };
 
 struct __align__(1024) IdxSmem {
     uint8_t ring[kRingBytes];                 // bf16: [2 slabs][128][128 B] per stage; fp8: [128][128 B]
     uint8_t q[2][kQBufBytes];                 // B operand per segment buffer
-    float wq[2][32];                          // head weights (times 2^-s for FP8)
+    float wq[2][128];                         // head weights of the G queries (times 2^-s for FP8)
     uint32_t hist[2][kHistBins];
     uint64_t k_full[kMaxStages], k_empty[kMaxStages], d_full[kMaxDStages], d_free[kMaxDStages], q_full[2], q_free[2],
         ep_sync, drain;
@@ -79,6 +86,7 @@ struct IdxTcArgs {
     int* err;                // device fault word (may be null)
     long long n_ent, ctx_len, total_tiles;
     int rows, n_q, m, heads_i, tiles_per_row, grid;
+    int ngroups;  // query groups per sequence: ceil(n_q / G)
 };
 
 __device__ __forceinline__ void idx_fault(IdxSmem& sm, const IdxTcArgs& a) {
@@ -97,37 +105,38 @@ __device__ __forceinline__ bool warp_aborted(const IdxSmem& sm) {
 
 __device__ __forceinline__ long long irange(int c, const IdxTcArgs& a) { return (long long)c * a.total_tiles / a.grid; }
 
-// walks (row, tile) in flat order; rq = row % n_q and bat = row / n_q kept incrementally
+// walks (query group, tile) in flat order: group `grp` = queries q0 .. q0 + G - 1 of sequence bat
 struct ICursor {
-    int row, ti, rq, bat;
-    __device__ ICursor(long long f, const IdxTcArgs& a) {
-        row = (int)(f / a.tiles_per_row);
-        ti = (int)(f - (long long)row * a.tiles_per_row);
-        bat = row / a.n_q;
-        rq = row - bat * a.n_q;
+    int grp, ti, q0, bat, G;
+    __device__ ICursor(long long f, const IdxTcArgs& a, int g) : G(g) {
+        grp = (int)(f / a.tiles_per_row);
+        ti = (int)(f - (long long)grp * a.tiles_per_row);
+        bat = grp / a.ngroups;
+        q0 = (grp - bat * a.ngroups) * G;
     }
     __device__ __forceinline__ void next(const IdxTcArgs& a) {
         if (++ti == a.tiles_per_row) {
             ti = 0;
-            ++row;
-            if (++rq == a.n_q) {
-                rq = 0;
+            ++grp;
+            q0 += G;
+            if (q0 >= a.n_q) {
+                q0 = 0;
                 ++bat;
             }
         }
     }
 };
 
-__device__ __forceinline__ long long nvis_of(const ICursor& c, const IdxTcArgs& a) {
-    const long long t = a.ctx_len - a.n_q + c.rq;
+__device__ __forceinline__ long long nvis_of(int qj, const IdxTcArgs& a) {
+    const long long t = a.ctx_len - a.n_q + qj;
     const long long nv = n_visible(t, a.m);
     return nv > a.n_ent ? a.n_ent : nv;
 }
 
-template <bool FP8>
+template <bool FP8, int G>
 __device__ void idx_producer(IdxSmem& sm, const IdxTcArgs& a, const CUtensorMap* kmap, long long f0, long long f1) {
     constexpr int kSt = Ring<FP8>::kStages, kBytes = Ring<FP8>::kStageBytes;
-    ICursor cur(f0, a);
+    ICursor cur(f0, a, G);
     const long long n = f1 - f0;
     for (long long jt = 0; jt < n; ++jt, cur.next(a)) {
         if (aborted(sm)) break;
@@ -144,16 +153,16 @@ __device__ void idx_producer(IdxSmem& sm, const IdxTcArgs& a, const CUtensorMap*
         if (jt >= 0) tc::mbar_wait(&sm.k_full[jt % kSt], (uint32_t)(jt / kSt) & 1);
 }
 
-template <bool FP8, int NP>
+template <bool FP8, int NP, int G>
 __device__ void idx_mma(IdxSmem& sm, const IdxTcArgs& a, uint32_t tmem, long long f0, long long f1) {
     constexpr int kSt = Ring<FP8>::kStages, kBytes = Ring<FP8>::kStageBytes;
-    constexpr int kDS = Acc<FP8, NP>::kStages, kN = Acc<FP8, NP>::kN;
-    constexpr uint32_t kQSlab = NP * 128;  // bf16: bytes per K-slab of q
+    constexpr int kDS = Acc<FP8, NP, G>::kStages, kN = Acc<FP8, NP, G>::kN;
+    constexpr uint32_t kQSlab = kN * 128;  // bf16: bytes per K-slab of q
     constexpr uint32_t idesc = FP8 ? tc::idesc_e4m3(128, kN) : tc::idesc_f16(128, kN, 0, 0, 1);
     bool ok = true;
     int seg = 0, b = 0;
     uint64_t qd = 0;
-    ICursor cur(f0, a);
+    ICursor cur(f0, a, G);
     for (long long f = f0; f < f1; ++f, cur.next(a)) {
         if (aborted(sm)) { ok = false; break; }
         const int jt = (int)(f - f0), st = jt % kSt, sd = jt % kDS;
@@ -170,7 +179,7 @@ __device__ void idx_mma(IdxSmem& sm, const IdxTcArgs& a, uint32_t tmem, long lon
         const uint32_t stage = tc::smem_u32(sm.ring + st * kBytes);
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
-            const uint32_t d = tmem + Acc<FP8, NP>::kCols * sd + kN * hf;
+            const uint32_t d = tmem + Acc<FP8, NP, G>::kCols * sd + kN * hf;
             // rows 128 hf .. 128 hf + 127 of every 128-byte slab of the tile
             const uint64_t kd = tc::sw128_desc(stage + hf * kHalf * 128, 16, 1024);
             if (FP8) {
@@ -208,25 +217,30 @@ __device__ __forceinline__ float e4m3_value(uint32_t c) {
     return __half2float(__half(__nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)c, __NV_E4M3)));
 }
 
-// B operand of one row into buffer b (K-major, 128-byte swizzle, 128-byte rows) and the head
-// weights; ct = 0..127.  bf16 keys: q itself (two K-slabs of NP rows).  FP8 keys: rows
-// p * NP + h hold piece p of head h (p = hi, lo, hi', lo'), one e4m3 per element.
-template <bool FP8, int NP>
-__device__ void stage_query(IdxSmem& sm, const IdxTcArgs& a, int row, int b, int ct) {
-    // warp w handles heads w, w+4, ...; lane owns 4 of the 128 elements
+// B operand of one query group into buffer b (K-major, 128-byte swizzle, 128-byte rows) and the
+// head weights; ct = 0..127.  Virtual head vh = g NP + h is head h of query q0 + g (zero past the
+// last query or head).  bf16 keys: q itself (two K-slabs of G NP rows).  FP8 keys: rows
+// g 4 NP + p NP + h hold piece p of that head (p = hi, lo, hi', lo'), one e4m3 per element.
+template <bool FP8, int NP, int G>
+__device__ void stage_query(IdxSmem& sm, const IdxTcArgs& a, int bat, int q0, int b, int ct) {
+    constexpr int kN = Acc<FP8, NP, G>::kN;
+    // warp w handles virtual heads w, w+4, ...; lane owns 4 of the 128 elements
     const int warp = ct >> 5, lane = ct & 31;
     const int k = lane * 4;
-    for (int h = warp; h < NP; h += 4) {
+    for (int vh = warp; vh < G * NP; vh += 4) {
+        const int g = vh / NP, h = vh - g * NP, qj = q0 + g;
+        const bool live = qj < a.n_q && h < a.heads_i;
+        const long long row = (long long)bat * a.n_q + qj;
         float v[4] = {0.f, 0.f, 0.f, 0.f};
-        if (h < a.heads_i) {
-            const __nv_bfloat16* qp = a.q + ((long long)row * a.heads_i + h) * kDI + k;
+        if (live) {
+            const __nv_bfloat16* qp = a.q + (row * a.heads_i + h) * kDI + k;
             const uint2 raw = *reinterpret_cast<const uint2*>(qp);
             v[0] = __uint_as_float(raw.x << 16);
             v[1] = __uint_as_float(raw.x & 0xffff0000u);
             v[2] = __uint_as_float(raw.y << 16);
             v[3] = __uint_as_float(raw.y & 0xffff0000u);
         }
-        float wq = h < a.heads_i ? a.w[(long long)row * a.heads_i + h] : 0.f;
+        float wq = live ? a.w[row * a.heads_i + h] : 0.f;
         if (FP8) {
             float amax = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
 #pragma unroll
@@ -248,35 +262,35 @@ __device__ void stage_query(IdxSmem& sm, const IdxTcArgs& a, int row, int b, int
             }
 #pragma unroll
             for (int p = 0; p < 4; ++p) {
-                const int n = p * NP + h;
+                const int n = g * 4 * NP + p * NP + h;
                 uint8_t* dst = sm.q[b] + (n >> 3) * 1024 + (n & 7) * 128 + ((((k >> 4) ^ (n & 7))) << 4) + (k & 15);
                 *reinterpret_cast<uint32_t*>(dst) = pc[p];
             }
         } else {
             __nv_bfloat162 b0 = __floats2bfloat162_rn(v[0], v[1]), b1 = __floats2bfloat162_rn(v[2], v[3]);
-            // element k of head h: K-slab k/64, 16-byte chunk (k%64)/8, 8-byte half
-            uint8_t* slab = sm.q[b] + (k >> 6) * (NP * 128);
-            uint8_t* dst = slab + (h >> 3) * 1024 + (h & 7) * 128 + ((((k & 63) >> 3) ^ (h & 7)) << 4) + ((k & 7) ? 8 : 0);
+            // element k of virtual head vh: K-slab k/64, 16-byte chunk (k%64)/8, 8-byte half
+            uint8_t* slab = sm.q[b] + (k >> 6) * (kN * 128);
+            uint8_t* dst = slab + (vh >> 3) * 1024 + (vh & 7) * 128 + ((((k & 63) >> 3) ^ (vh & 7)) << 4) + ((k & 7) ? 8 : 0);
             *reinterpret_cast<uint2*>(dst) =
                 make_uint2(*reinterpret_cast<uint32_t*>(&b0), *reinterpret_cast<uint32_t*>(&b1));
         }
-        if (lane == 0) sm.wq[b][h] = wq;
+        if (lane == 0) sm.wq[b][vh] = wq;
     }
 }
 
-// warps 2-5: per segment, stage the row's B operand
-template <bool FP8, int NP>
+// warps 2-5: per segment, stage the query group's B operand
+template <bool FP8, int NP, int G>
 __device__ void idx_stage(IdxSmem& sm, const IdxTcArgs& a, long long f0, long long f1) {
     const int ct = threadIdx.x - 64;
     bool ok = true;
     int seg = 0;
-    ICursor cur(f0, a);
+    ICursor cur(f0, a, G);
     for (long long f = f0; f < f1; ++f, cur.next(a)) {
         if (f != f0 && cur.ti != 0) continue;
         if (warp_aborted(sm)) { ok = false; break; }
         const int b = seg & 1;
         if (seg >= 2 && !warp_wait(&sm.q_free[b], ((seg >> 1) - 1) & 1)) { ok = false; break; }
-        stage_query<FP8, NP>(sm, a, cur.row, b, ct);
+        stage_query<FP8, NP, G>(sm, a, cur.bat, cur.q0, b, ct);
         tc::fence_proxy_async();
         tc::mbar_arrive(&sm.q_full[b]);
         ++seg;
@@ -323,20 +337,22 @@ __device__ __forceinline__ float score_of(uint32_t taddr, const float* wq) {
     return acc;
 }
 
-// warps 6-9: per tile the scores of entries r and r + 128 (r = this thread's TMEM lane), their
-// histogram counts and stores
-template <bool FP8, int NP>
+// warps 6-9: per tile the scores of entries r and r + 128 (r = this thread's TMEM lane) for each
+// query of the group, their histogram counts (single queries only) and stores
+template <bool FP8, int NP, int G>
 __device__ void idx_epilogue(IdxSmem& sm, const IdxTcArgs& a, uint32_t tmem, long long f0, long long f1) {
-    constexpr int kDS = Acc<FP8, NP>::kStages, kN = Acc<FP8, NP>::kN;
+    constexpr int kDS = Acc<FP8, NP, G>::kStages, kN = Acc<FP8, NP, G>::kN, kNq = Acc<FP8, NP, G>::kNq;
     const int et = threadIdx.x - 192;
     const int sub = (threadIdx.x >> 5) & 3;
     const int r = 32 * sub + (threadIdx.x & 31);
     const uint32_t lane_addr = (uint32_t)(32 * sub) << 16;
     bool ok = true;
     int seg = 0, b = 0, nsync = 0;
-    long long nv = 0;
-    float* srow = nullptr;
-    ICursor cur(f0, a);
+    int nv[G];            // visible entries of each query of the group (0 past the last query)
+    float* srow0 = nullptr;  // the group's first score row; query g's is g rows further
+#pragma unroll
+    for (int g = 0; g < G; ++g) nv[g] = 0;
+    ICursor cur(f0, a, G);
     // scales of the current tile's two entries, loaded one tile ahead
     auto scales_of = [&](const ICursor& c, float (&sc)[2]) {
 #pragma unroll
@@ -354,49 +370,60 @@ __device__ void idx_epilogue(IdxSmem& sm, const IdxTcArgs& a, uint32_t tmem, lon
             b = seg & 1;
             if (!warp_wait(&sm.q_full[b], (seg >> 1) & 1)) { ok = false; break; }
             ++seg;
-            nv = nvis_of(cur, a);
-            srow = a.scores + (long long)cur.row * a.n_ent;
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                const int qj = cur.q0 + g;
+                nv[g] = qj < a.n_q ? (int)nvis_of(qj, a) : 0;
+            }
+            srow0 = a.scores + ((long long)cur.bat * a.n_q + cur.q0) * a.n_ent;
         }
         const bool seg_end = (f == f1 - 1) || (cur.ti == a.tiles_per_row - 1);
-        const int ti = cur.ti, row = cur.row;
+        const int ti = cur.ti, q0t = cur.q0, row = cur.bat * a.n_q + cur.q0;  // row: the group's first query
         cur.next(a);
         float sc_next[2] = {1.f, 1.f};
         if (FP8 && f + 1 < f1) scales_of(cur, sc_next);
         if (!warp_wait(&sm.d_full[sd], (jt / kDS) & 1)) { ok = false; break; }
         tc::tc_fence_after();
-        float acc[2];
+        float acc[G][2];
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf)
-            acc[hf] = score_of<FP8, NP>(tmem + lane_addr + Acc<FP8, NP>::kCols * sd + kN * hf, sm.wq[b]);
+        for (int g = 0; g < G; ++g)
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf)
+                acc[g][hf] = score_of<FP8, NP>(tmem + lane_addr + Acc<FP8, NP, G>::kCols * sd + kN * hf + kNq * g,
+                                               sm.wq[b] + NP * g);
         tc::tc_fence_before();
         tc::mbar_arrive(&sm.d_free[sd]);
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-            const long long e = (long long)ti * kTileK + kHalf * hf + r;
-            if (e < a.n_ent) {
-                float sc = -INFINITY;
-                if (e < nv) {
-                    float v = acc[hf];
-                    if (FP8) v *= sc_cur[hf];
-                    sc = v + 0.0f;
-                    if (a.hist) atomicAdd(&sm.hist[b][float_to_ordered(sc) >> 20], 1u);
+        for (int g = 0; g < G; ++g) {
+            if (q0t + g >= a.n_q) continue;  // past the last query of the sequence
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                const long long e = (long long)ti * kTileK + kHalf * hf + r;
+                if (e < a.n_ent) {
+                    float sc = -INFINITY;
+                    if (e < nv[g]) {
+                        float v = acc[g][hf];
+                        if (FP8) v *= sc_cur[hf];
+                        sc = v + 0.0f;
+                        if (G == 1 && a.hist) atomicAdd(&sm.hist[b][float_to_ordered(sc) >> 20], 1u);
+                    }
+                    srow0[(long long)g * a.n_ent + e] = sc;
                 }
-                srow[e] = sc;
             }
         }
         sc_cur[0] = sc_next[0];
         sc_cur[1] = sc_next[1];
         if (seg_end) {
             tc::mbar_arrive(&sm.q_free[b]);  // done with wq[b]
-            // every epilogue thread has counted this segment's scores (bounded, unlike a named barrier)
-            tc::mbar_arrive(&sm.ep_sync);
-            if (!warp_wait(&sm.ep_sync, nsync++ & 1)) { ok = false; break; }
-            if (a.hist) {
-                uint32_t* g = a.hist + (long long)row * kHistBins;
+            if (G == 1 && a.hist) {
+                // every epilogue thread has counted this segment's scores (bounded, unlike a named barrier)
+                tc::mbar_arrive(&sm.ep_sync);
+                if (!warp_wait(&sm.ep_sync, nsync++ & 1)) { ok = false; break; }
+                uint32_t* gh = a.hist + (long long)row * kHistBins;
                 for (int i = et; i < kHistBins; i += 128) {
                     const uint32_t v = sm.hist[b][i];
                     if (v) {
-                        atomicAdd(g + i, v);
+                        atomicAdd(gh + i, v);
                         sm.hist[b][i] = 0;
                     }
                 }
@@ -406,7 +433,7 @@ __device__ void idx_epilogue(IdxSmem& sm, const IdxTcArgs& a, uint32_t tmem, lon
     if (!ok) idx_fault(sm, a);
 }
 
-template <bool FP8, int NP>
+template <bool FP8, int NP, int G>
 __global__ void __launch_bounds__(kThreads, 1) index_score_tc_kernel(const __grid_constant__ CUtensorMap kmap, IdxTcArgs a) {
     extern __shared__ uint8_t smem_raw[];
     IdxSmem& sm = *reinterpret_cast<IdxSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -417,7 +444,7 @@ __global__ void __launch_bounds__(kThreads, 1) index_score_tc_kernel(const __gri
             tc::mbar_init(&sm.k_full[i], 1);
             tc::mbar_init(&sm.k_empty[i], 1);
         }
-        for (int i = 0; i < Acc<FP8, NP>::kStages; ++i) {
+        for (int i = 0; i < Acc<FP8, NP, G>::kStages; ++i) {
             tc::mbar_init(&sm.d_full[i], 1);
             tc::mbar_init(&sm.d_free[i], 128);
         }
@@ -439,13 +466,13 @@ __global__ void __launch_bounds__(kThreads, 1) index_score_tc_kernel(const __gri
     tc::tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
     if (warp == 0) {
-        if (lane == 0) idx_producer<FP8>(sm, a, &kmap, f0, f1);
+        if (lane == 0) idx_producer<FP8, G>(sm, a, &kmap, f0, f1);
     } else if (warp == 1) {
-        if (lane == 0) idx_mma<FP8, NP>(sm, a, tmem, f0, f1);
+        if (lane == 0) idx_mma<FP8, NP, G>(sm, a, tmem, f0, f1);
     } else if (warp < 6) {
-        idx_stage<FP8, NP>(sm, a, f0, f1);
+        idx_stage<FP8, NP, G>(sm, a, f0, f1);
     } else {
-        idx_epilogue<FP8, NP>(sm, a, tmem, f0, f1);
+        idx_epilogue<FP8, NP, G>(sm, a, tmem, f0, f1);
     }
     __syncwarp();
     tc::tc_fence_before();
@@ -504,11 +531,16 @@ cudaError_t launch_index_scores_tc(const IndexArgs& a, float* scores, uint32_t* 
     t.n_q = a.n_q;
     t.m = a.m;
     t.heads_i = a.heads_i;
+    // queries scored together: several per key tile when there are many queries and no histogram
+    const bool narrow = a.heads_i <= 16;
+    int G = 1;
+    if (a.n_q > 1 && hist == nullptr) G = fp8 ? (narrow ? 2 : 1) : (narrow ? 4 : 2);
+    t.ngroups = (a.n_q + G - 1) / G;
     // tiles up to the last entry any query of the row block can see
     long long nv_max = n_visible(a.ctx_len - 1, a.m);
     if (nv_max > a.n_ent) nv_max = a.n_ent;
     t.tiles_per_row = (int)((nv_max + kTileK - 1) / kTileK);
-    t.total_tiles = (long long)t.rows * t.tiles_per_row;
+    t.total_tiles = (long long)a.batch * t.ngroups * t.tiles_per_row;
     if (t.total_tiles == 0) return cudaSuccess;
     t.grid = (int)(t.total_tiles < kNumSMs ? t.total_tiles : kNumSMs);
     const size_t smem = sizeof(IdxSmem) + 1024;
@@ -517,9 +549,14 @@ cudaError_t launch_index_scores_tc(const IndexArgs& a, float* scores, uint32_t* 
         if (err == cudaSuccess) kernel<<<t.grid, kThreads, smem, stream>>>(kmap, t);
         return err;
     };
-    const bool narrow = a.heads_i <= 16;
-    cudaError_t e = fp8 ? (narrow ? go(index_score_tc_kernel<true, 16>) : go(index_score_tc_kernel<true, 32>))
-                        : (narrow ? go(index_score_tc_kernel<false, 16>) : go(index_score_tc_kernel<false, 32>));
+    cudaError_t e;
+    if (fp8) {
+        if (narrow) e = G == 2 ? go(index_score_tc_kernel<true, 16, 2>) : go(index_score_tc_kernel<true, 16, 1>);
+        else e = go(index_score_tc_kernel<true, 32, 1>);
+    } else {
+        if (narrow) e = G == 4 ? go(index_score_tc_kernel<false, 16, 4>) : go(index_score_tc_kernel<false, 16, 1>);
+        else e = G == 2 ? go(index_score_tc_kernel<false, 32, 2>) : go(index_score_tc_kernel<false, 32, 1>);
+    }
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
