@@ -101,7 +101,6 @@ __global__ void __launch_bounds__(kScoreThreads) index_score_kernel(IndexArgs a,
 // ---------------------------------------------------------------------
 // select
 // ---------------------------------------------------------------------
-constexpr int kSelThreads = 1024;
 
 // exclusive block scan of one int per thread; returns the block total in *total
 __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_buf, int* total) {
@@ -176,7 +175,7 @@ __device__ void find_digit(const unsigned int* h, int nbins, long long rem, int*
 
 // Exact radix select of one row (scores[0..nvis), -inf never selected): the
 // min(k, nvis) largest, ties to the lower entry, written in ascending entry
-// order and padded with -1.  Called by a whole block of kSelThreads threads.
+// order and padded with -1.  Called by a whole block (any size of at least 256 threads).
 __device__ void select_row_radix(const float* sc, long long nvis, int k, int32_t* io, float* so) {
     __shared__ unsigned int hist[256];
     __shared__ int warp_buf[33];
@@ -233,13 +232,6 @@ __device__ __forceinline__ long long row_nvis(const IndexArgs& a, int row) {
     return nvis > a.n_ent ? a.n_ent : nvis;
 }
 
-// one block per query row; scores[row][N] with -inf beyond N_vis
-__global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const float* scores, IndexArgs a, int k,
-                                                                   int32_t* idx_out, float* score_out) {
-    const int row = blockIdx.x;
-    select_row_radix(scores + (long long)row * a.n_ent, row_nvis(a, row), k, idx_out + (long long)row * k,
-                     score_out ? score_out + (long long)row * k : nullptr);
-}
 
 // ---------------------------------------------------------------------
 // select for few query rows: histogram threshold, then one kernel whose
@@ -406,87 +398,14 @@ __device__ __forceinline__ int lower_bound(const int32_t* v, int n, int32_t x) {
 // The row's answer from the parts' compacted lists: every definite entry (key in a bin above the
 // threshold bin) plus the best `need` candidates (keys in the threshold bin), ties to the lower
 // entry, in ascending entry order, padded with -1.  Whole block; the parts' writes are visible.
-__device__ void finish_row(const float* sc, long long nvis, int k, int parts, long long chunk, const int32_t* def_row,
-                           const int32_t* cidx_row, const uint32_t* ckey_row, const int* counts_row, int32_t* io,
-                           float* so, uint8_t* dsm) {
-    uint32_t* ckey = reinterpret_cast<uint32_t*>(dsm);           // [kCandCap]
-    int32_t* cidx = reinterpret_cast<int32_t*>(ckey + kCandCap);  // [kCandCap]
-    int32_t* defs = cidx + kCandCap;                              // [4096]
-    int32_t* sels = defs + 4096;                                  // [4096]
-    __shared__ int doff[kMaxParts + 1], coff[kMaxParts + 1];
+// The row's answer from its definite entries defs[0..D) and candidates (cidx, ckey)[0..C) in
+// shared memory, both in ascending entry order: every definite entry plus the best `need` candidates
+// (radix select over the low 20 key bits, whose top 12 are equal; ties to the lower entry), merged
+// in ascending order into io (and so), padded with -1.  Whole block of kFastThreads threads.
+__device__ void finish_lists(const float* sc, int k, int D, int C, int32_t* defs, int32_t* cidx, uint32_t* ckey,
+                             int32_t* sels, int32_t* io, float* so) {
     __shared__ unsigned int h1[1024];
     __shared__ int warp_buf[33];
-    {
-        // prefix sums of the parts' counts (parts <= kMaxParts = blockDim)
-        const int p = threadIdx.x;
-        const int nd = p < parts ? __ldcg(counts_row + 2 * p) : 0;
-        const int nc = p < parts ? __ldcg(counts_row + 2 * p + 1) : 0;
-        int td, tc;
-        const int ed = block_exclusive_scan(nd, warp_buf, &td);
-        const int ec = block_exclusive_scan(nc, warp_buf, &tc);
-        if (p < parts) {
-            doff[p] = ed;
-            coff[p] = ec;
-        }
-        if (p == 0) {
-            doff[parts] = td;
-            coff[parts] = tc;
-        }
-        __syncthreads();
-    }
-    const int D = doff[parts], C = coff[parts];
-    if (C > kCandCap || D > 4096) {
-        // more candidates than the fast path holds (e.g. huge blocks of equal scores): exact select over the row
-        select_row_radix(sc, nvis, k, io, so);
-        return;
-    }
-    // gather the definite entries and the candidates, both in ascending entry order; every element
-    // finds its part by binary search over the offsets, and each thread issues the loads of up to
-    // kG elements before using any of them
-    constexpr int kG = 8;
-    for (int e0 = threadIdx.x; e0 < D + C; e0 += kG * blockDim.x) {
-        long long src[kG];
-        int32_t vi[kG];
-        uint32_t vk[kG];
-#pragma unroll
-        for (int g = 0; g < kG; ++g) {
-            const int e = e0 + g * blockDim.x;
-            src[g] = -1;
-            if (e < D + C) {
-                const bool is_def = e < D;
-                const int x = is_def ? e : e - D;
-                const int* off = is_def ? doff : coff;
-                int lo = 0, hi = parts;  // largest p with off[p] <= x
-                while (hi - lo > 1) {
-                    const int mid = (lo + hi) >> 1;
-                    if (off[mid] <= x) lo = mid;
-                    else hi = mid;
-                }
-                src[g] = (long long)lo * chunk + (x - off[lo]);
-            }
-        }
-#pragma unroll
-        for (int g = 0; g < kG; ++g) {
-            const int e = e0 + g * blockDim.x;
-            vi[g] = 0;
-            vk[g] = 0;
-            if (src[g] >= 0) {
-                vi[g] = e < D ? __ldcg(def_row + src[g]) : __ldcg(cidx_row + src[g]);
-                if (e >= D) vk[g] = __ldcg(ckey_row + src[g]);
-            }
-        }
-#pragma unroll
-        for (int g = 0; g < kG; ++g) {
-            const int e = e0 + g * blockDim.x;
-            if (src[g] < 0) continue;
-            if (e < D) {
-                defs[e] = vi[g];
-            } else {
-                cidx[e - D] = vi[g];
-                ckey[e - D] = vk[g];
-            }
-        }
-    }
     const int need = (D + C) < k ? C : k - D;  // candidates to take
     __syncthreads();
     // radix select of the need-th largest candidate key over its low 20 bits (the top 12 are equal)
@@ -571,6 +490,91 @@ __device__ void finish_row(const float* sc, long long nvis, int k, int parts, lo
     }
 }
 
+
+__device__ void finish_row(const float* sc, long long nvis, int k, int parts, long long chunk, const int32_t* def_row,
+                           const int32_t* cidx_row, const uint32_t* ckey_row, const int* counts_row, int32_t* io,
+                           float* so, uint8_t* dsm) {
+    uint32_t* ckey = reinterpret_cast<uint32_t*>(dsm);           // [kCandCap]
+    int32_t* cidx = reinterpret_cast<int32_t*>(ckey + kCandCap);  // [kCandCap]
+    int32_t* defs = cidx + kCandCap;                              // [4096]
+    int32_t* sels = defs + 4096;                                  // [4096]
+    __shared__ int doff[kMaxParts + 1], coff[kMaxParts + 1];
+    __shared__ int warp_buf[33];
+    {
+        // prefix sums of the parts' counts (parts <= kMaxParts = blockDim)
+        const int p = threadIdx.x;
+        const int nd = p < parts ? __ldcg(counts_row + 2 * p) : 0;
+        const int nc = p < parts ? __ldcg(counts_row + 2 * p + 1) : 0;
+        int td, tc;
+        const int ed = block_exclusive_scan(nd, warp_buf, &td);
+        const int ec = block_exclusive_scan(nc, warp_buf, &tc);
+        if (p < parts) {
+            doff[p] = ed;
+            coff[p] = ec;
+        }
+        if (p == 0) {
+            doff[parts] = td;
+            coff[parts] = tc;
+        }
+        __syncthreads();
+    }
+    const int D = doff[parts], C = coff[parts];
+    if (C > kCandCap || D > 4096) {
+        // more candidates than the fast path holds (e.g. huge blocks of equal scores): exact select over the row
+        select_row_radix(sc, nvis, k, io, so);
+        return;
+    }
+    // gather the definite entries and the candidates, both in ascending entry order; every element
+    // finds its part by binary search over the offsets, and each thread issues the loads of up to
+    // kG elements before using any of them
+    constexpr int kG = 8;
+    for (int e0 = threadIdx.x; e0 < D + C; e0 += kG * blockDim.x) {
+        long long src[kG];
+        int32_t vi[kG];
+        uint32_t vk[kG];
+#pragma unroll
+        for (int g = 0; g < kG; ++g) {
+            const int e = e0 + g * blockDim.x;
+            src[g] = -1;
+            if (e < D + C) {
+                const bool is_def = e < D;
+                const int x = is_def ? e : e - D;
+                const int* off = is_def ? doff : coff;
+                int lo = 0, hi = parts;  // largest p with off[p] <= x
+                while (hi - lo > 1) {
+                    const int mid = (lo + hi) >> 1;
+                    if (off[mid] <= x) lo = mid;
+                    else hi = mid;
+                }
+                src[g] = (long long)lo * chunk + (x - off[lo]);
+            }
+        }
+#pragma unroll
+        for (int g = 0; g < kG; ++g) {
+            const int e = e0 + g * blockDim.x;
+            vi[g] = 0;
+            vk[g] = 0;
+            if (src[g] >= 0) {
+                vi[g] = e < D ? __ldcg(def_row + src[g]) : __ldcg(cidx_row + src[g]);
+                if (e >= D) vk[g] = __ldcg(ckey_row + src[g]);
+            }
+        }
+#pragma unroll
+        for (int g = 0; g < kG; ++g) {
+            const int e = e0 + g * blockDim.x;
+            if (src[g] < 0) continue;
+            if (e < D) {
+                defs[e] = vi[g];
+            } else {
+                cidx[e - D] = vi[g];
+                ckey[e - D] = vk[g];
+            }
+        }
+    }
+    __syncthreads();
+    finish_lists(sc, k, D, C, defs, cidx, ckey, sels, io, so);
+}
+
 // grid rows * parts, kFastThreads threads.  Block (row, p) compacts entries [p*chunk, (p+1)*chunk)
 // of the row: definite entries (bin above the threshold bin) and candidates (the threshold bin),
 // each in ascending entry order; the last block of the row to finish (counted on row_done, which
@@ -638,6 +642,97 @@ __global__ void __launch_bounds__(kFastThreads) topk_fast_kernel(const float* sc
     finish_row(sc, nvis, k, parts, chunk, def_buf + row_off, cidx_buf + row_off, ckey_buf + row_off,
                counts + (long long)row * parts * 2, idx_out + (long long)row * k,
                score_out ? score_out + (long long)row * k : nullptr, dsm);
+}
+
+// Many query rows (prefill): one block (kFastThreads) per row.  Pass 1 builds the histogram of
+// the row's keys' top 12 bits in shared memory (warp-aggregated atomics), the threshold bin
+// follows, pass 2 compacts the definite entries and the threshold bin's candidates into shared
+// memory in entry order, and finish_lists selects and merges.  A row whose threshold bin holds
+// more than kCandCap candidates falls back to the exact radix select over the row.
+__global__ void __launch_bounds__(kFastThreads) topk_rows_kernel(const float* scores, IndexArgs a, int k,
+                                                                 int32_t* idx_out, float* score_out) {
+    extern __shared__ __align__(16) uint8_t dsm[];
+    uint32_t* ckey = reinterpret_cast<uint32_t*>(dsm);           // [kCandCap]
+    int32_t* cidx = reinterpret_cast<int32_t*>(ckey + kCandCap);  // [kCandCap]
+    int32_t* defs = cidx + kCandCap;                              // [4096]
+    int32_t* sels = defs + 4096;                                  // [4096]; the histogram before that
+    uint32_t* hist = reinterpret_cast<uint32_t*>(sels);
+    __shared__ int warp_buf[33];
+    const int row = blockIdx.x;
+    const long long nvis = row_nvis(a, row);
+    const float* sc = scores + (long long)row * a.n_ent;
+    int32_t* io = idx_out + (long long)row * k;
+    float* so = score_out ? score_out + (long long)row * k : nullptr;
+    for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    // kFastPer consecutive scores per thread per step, all loaded before any is counted; lanes of a
+    // warp that hit the same bin add once
+    for (long long base = 0; base < nvis; base += kFastStep) {
+        const long long s0 = base + (long long)threadIdx.x * kFastPer;
+        uint32_t bins[kFastPer];
+#pragma unroll
+        for (int i = 0; i < kFastPer; ++i) bins[i] = s0 + i < nvis ? float_to_ordered(sc[s0 + i]) >> 20 : 0xffffffffu;
+#pragma unroll
+        for (int i = 0; i < kFastPer; ++i) {
+            const unsigned peers = __match_any_sync(0xffffffffu, bins[i]);
+            if (bins[i] != 0xffffffffu && (threadIdx.x & 31) == (unsigned)(__ffs(peers) - 1))
+                atomicAdd(&hist[bins[i]], (uint32_t)__popc(peers));
+        }
+    }
+    __syncthreads();
+    int tbin;
+    bool all;
+    {
+        int c[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) c[j] = (int)hist[8 * threadIdx.x + j];
+        int d;
+        long long ab, tot;
+        block_find_bin<8>(c, k, &d, &ab, &tot);
+        tbin = d;
+        all = tot <= k;
+    }
+    int n_def = 0, n_cand = 0;
+    for (long long base = 0; base < nvis; base += kFastStep) {
+        const long long s0 = base + (long long)threadIdx.x * kFastPer;
+        uint32_t keys[kFastPer];
+        int nd = 0, nc = 0;
+#pragma unroll
+        for (int i = 0; i < kFastPer; ++i) {
+            const long long s = s0 + i;
+            keys[i] = s < nvis ? float_to_ordered(sc[s]) : 0u;
+            const int bin = (int)(keys[i] >> 20);
+            nd += (s < nvis && (all || bin > tbin)) ? 1 : 0;
+            nc += (s < nvis && !all && bin == tbin) ? 1 : 0;
+        }
+        int tot;
+        const int packed = block_exclusive_scan(nd | (nc << 16), warp_buf, &tot);
+        int od = n_def + (packed & 0xffff), oc = n_cand + (packed >> 16);
+#pragma unroll
+        for (int i = 0; i < kFastPer; ++i) {
+            const long long s = s0 + i;
+            const int bin = (int)(keys[i] >> 20);
+            if (s < nvis && (all || bin > tbin)) {
+                if (od < 4096) defs[od] = (int32_t)s;
+                ++od;
+            }
+            if (s < nvis && !all && bin == tbin) {
+                if (oc < kCandCap) {
+                    cidx[oc] = (int32_t)s;
+                    ckey[oc] = keys[i];
+                }
+                ++oc;
+            }
+        }
+        n_def += tot & 0xffff;
+        n_cand += tot >> 16;
+    }
+    __syncthreads();
+    if (n_cand > kCandCap || n_def > 4096) {
+        select_row_radix(sc, nvis, k, io, so);
+        return;
+    }
+    finish_lists(sc, k, n_def, n_cand, defs, cidx, ckey, sels, io, so);
 }
 
 template <int HMAX>
@@ -749,7 +844,9 @@ cudaError_t launch_topk(const IndexArgs& a, int k, int32_t* idx_out, float* scor
             e = launch_index_scores(a, scores, stream);
             if (e != cudaSuccess) return e;
         }
-        topk_select_kernel<<<rows, kSelThreads, 0, stream>>>(scores, a, k, idx_out, score_out);
+        e = cudaFuncSetAttribute(topk_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFastSmem);
+        if (e != cudaSuccess) return e;
+        topk_rows_kernel<<<rows, kFastThreads, kFastSmem, stream>>>(scores, a, k, idx_out, score_out);
         return cudaGetLastError();
     }
     uint32_t* hist = reinterpret_cast<uint32_t*>(base + p.off_hist);

@@ -411,6 +411,33 @@ def test_hca_single_long_query_split_over_many_ctas(v4a):
     check_attention(out, ref, False, "hca one long query")
 
 
+def test_topk_many_rows_matches_oracle(v4a):
+    """More query rows than the few-rows select serves (2 x 150 = 300 > 256) take the per-row
+    histogram select; the rows see different numbers of entries and include exact ties."""
+    B, T, L, m, k, HI, DI = 2, 150, 4 * 3000 + 5, 4, 200, 16, 128
+    c = wl.index_case(B, T, L, m, HI, DI, "bf16", "bf16", seed=81)
+    c["k_i"][:, 100:400] = c["k_i"][:, 100:101].clone()  # 300 copies of one key: equal scores in every row
+    idx = torch.empty((B, T, k), dtype=torch.int32, device="cuda")
+    sco = torch.empty((B, T, k), dtype=torch.float32, device="cuda")
+    v4a.v4a_topk(dev(c["q_i"]), dev(c["w"]), dev(c["k_i"]), None, idx, sco, m=m, k=k, ctx_len=L)
+    _sync()
+    ref = oracle.topk(host(c["q_i"]), host(c["w"]), host(c["k_i"]), None, L, m, k, want_scores=True)
+    check_topk(idx, ref, L, m, k, gpu_scores=sco)
+
+
+def test_topk_many_rows_all_equal_takes_lowest_entries(v4a):
+    """Many rows whose scores are all equal: the threshold bin holds every entry, more than the
+    per-row select keeps in shared memory, and the exact radix select takes the lowest entries."""
+    B, T, L, m, k, HI, DI = 1, 300, 4 * 10000, 4, 333, 16, 128
+    c = wl.index_case(B, T, L, m, HI, DI, "bf16", "bf16", seed=82)
+    c["k_i"] = c["k_i"][:, :1].expand(B, L // m, DI).contiguous()
+    idx = torch.empty((B, T, k), dtype=torch.int32, device="cuda")
+    v4a.v4a_topk(dev(c["q_i"]), dev(c["w"]), dev(c["k_i"]), None, idx, m=m, k=k, ctx_len=L)
+    _sync()
+    want = np.broadcast_to(np.arange(k, dtype=np.int32), (B, T, k))
+    assert np.array_equal(idx.cpu().numpy(), want)
+
+
 def test_topk_all_scores_equal_takes_lowest_entries(v4a):
     """Every entry scores the same: the candidate set exceeds what the fast
     select holds in shared memory and the full radix select takes over; ties
