@@ -257,6 +257,91 @@ class Step:
         return self.Bc + self.Bh
 
 
+class Prefill:
+    """The prefill-chunk workload: 4,096 causal query tokens at positions
+    126,976 .. 131,071 of a 131,072-token bf16 sequence (m = 4, 16 x 128
+    indexer, top-512, 64 heads x 512, window 128): compress the chunk, score
+    and select for every query, sparse attention for every query."""
+
+    def __init__(self):
+        import compressed_sparse_long_v4a_b200 as v4a
+        import workload as wl
+
+        self.v4a = v4a
+        w = wl.prefill_chunk()
+        c = self.c = w["cfg"]
+        self.L, self.T, self.m, self.k, self.W = c["ctx_len"], c["n_q"], c["m"], c["k"], c["window"]
+        self.n_hist, self.N = w["n_hist"], w["N"]
+        d, di = c["d"], c["d_i"]
+        self.ent = torch.zeros((1, self.N, d), dtype=torch.bfloat16, device="cuda")
+        self.keys = torch.zeros((1, self.N, di), dtype=torch.bfloat16, device="cuda")
+        self.ent[:, :self.n_hist] = w["hist_entries"].cuda()
+        self.keys[:, :self.n_hist] = w["hist_keys"].cuda()
+        dv = lambda t: t.cuda()
+        self.x, self.g, self.xi, self.gi = dv(w["x"]), dv(w["gate"]), dv(w["xi"]), dv(w["gate_i"])
+        self.q, self.qi, self.w, self.tok = dv(w["q"]), dv(w["q_i"]), dv(w["w"]), dv(w["token_kv"])
+        self.tok_pos0 = w["tok_pos0"]
+        self.idx = torch.empty((1, self.T, self.k), dtype=torch.int32, device="cuda")
+        self.out = torch.empty((1, self.T, c["heads"], d), dtype=torch.float32, device="cuda")
+        self.scores = torch.empty((1, self.T, self.N), dtype=torch.float32, device="cuda")
+        ws = lambda n: torch.empty(max(n, 256), dtype=torch.uint8, device="cuda")
+        self.ws_topk = ws(v4a.v4a_workspace_size("topk", batch=1, n_q=self.T, m=self.m, k=self.k, ctx_len=self.L,
+                                                 heads_i=c["heads_i"], d_i=di))
+        self.ws_att = ws(v4a.v4a_workspace_size("csa_attend", batch=1, n_q=self.T, heads=c["heads"], d=d, m=self.m,
+                                                k=self.k, window=self.W, ctx_len=self.L))
+
+    def compress(self):
+        self.v4a.v4a_compress(self.x, self.g, self.ent[:, self.n_hist:], m=self.m, xi=self.xi, gate_i=self.gi,
+                              out_i=self.keys[:, self.n_hist:])
+
+    def index_scores(self):
+        self.v4a.v4a_index_scores(self.qi, self.w, self.keys, None, self.scores, m=self.m, ctx_len=self.L)
+
+    def topk(self):
+        self.v4a.v4a_topk(self.qi, self.w, self.keys, None, self.idx, m=self.m, k=self.k, ctx_len=self.L,
+                          workspace=self.ws_topk)
+
+    def attend(self):
+        self.v4a.v4a_csa_attend(self.q, self.ent, self.idx, self.tok, self.tok_pos0, self.out, m=self.m,
+                                window=self.W, ctx_len=self.L, workspace=self.ws_att)
+
+    def step(self):
+        self.compress()
+        self.topk()
+        self.attend()
+
+    def flops(self):
+        c = self.c
+        nvis = sum((self.L - self.T + j + 1) // self.m for j in range(self.T))
+        idx_f = 2.0 * nvis * c["heads_i"] * c["d_i"]
+        att_f = 4.0 * self.T * c["heads"] * (self.k + self.W) * c["d"]
+        return idx_f, att_f
+
+
+def measure_prefill(peaks: dict) -> dict:
+    p = Prefill()
+    p.step()
+    torch.cuda.synchronize()
+    reps = 10
+    ms = {name: statistics.median(layer_times(getattr(p, name), reps))
+          for name in ("compress", "index_scores", "topk", "attend", "step")}
+    idx_f, att_f = p.flops()
+    sustained = float(peaks.get("bf16_tflops_sustained", 1390.0))
+    burst = float(peaks.get("bf16_tflops", 1640.0))
+    res = {"workload": "prefill chunk: 4,096 queries at positions 126,976..131,071 of a 131,072-token bf16 "
+                       "sequence, m=4, indexer 16x128 bf16, top-512, 64 heads x 512, window 128",
+           "ms_median": ms, "replays": reps,
+           "index_scores_tflops": idx_f / (ms["index_scores"] / 1000.0) / 1e12,
+           "attention_tflops": att_f / (ms["attend"] / 1000.0) / 1e12,
+           "step_tflops": (idx_f + att_f) / (ms["step"] / 1000.0) / 1e12,
+           "flops": {"index_scores": idx_f, "attention": att_f},
+           "peak_tflops_bf16": {"sustained": sustained, "burst": burst}}
+    res["step_frac_sustained"] = res["step_tflops"] / sustained
+    del p
+    torch.cuda.empty_cache()
+    return res
+
+
 def kernel_nodes(graph) -> int | None:
     """Kernel nodes in a captured graph (cuGraphGetNodes + cuGraphNodeGetType of
     the driver API; the graph must have been made with keep_graph=True)."""
@@ -542,6 +627,9 @@ def main():
            "ms_per_step": e2e_s * 1000.0, "how": "eager API calls, pinned copies in, outputs out, host wall clock"}
 
     cpu = None
+    prefill = None
+    if rank == 0 and world == 1:
+        prefill = measure_prefill(peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, threads, sample, _ = oracle_sample(args.cpu_seconds, step)
         cpu = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample}
@@ -559,7 +647,7 @@ def main():
                            "step_hbm_gbs": total_bytes / (ms / 1000.0) / 1e9 / world,
                            "op_ms": op_ms,
                            "layers": layers},
-                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "prefill": prefill,
                 "gpu_launches": (launches_per_step * args.steps) if launches_per_step else None,
                 "gpu_launches_per_step": launches_per_step,
                 "clocks": clocks}
