@@ -54,6 +54,8 @@ def _load():
     lib.v4ao_n_visible.argtypes = [ll, ll]
     lib.v4ao_compress.restype = i32
     lib.v4ao_compress.argtypes = [vp, vp, i32, ll, ll, ll, ll, vp]
+    lib.v4ao_compress_dual.restype = i32
+    lib.v4ao_compress_dual.argtypes = [vp, vp, vp, vp, vp, vp, i32, ll, ll, ll, ll, vp]
     lib.v4ao_quantize_e4m3_rows.restype = i32
     lib.v4ao_quantize_e4m3_rows.argtypes = [vp, ll, ll, vp, vp]
     lib.v4ao_index_scores.restype = i32
@@ -150,6 +152,25 @@ def compress(x, gate, m: int) -> np.ndarray:
     st = _load().v4ao_compress(_ptr(x), _ptr(gate), fmt_of(x), B, n_tok, C, m, _ptr(out))
     if st:
         raise ValueError(f"oracle compress: status {st}")
+    return out
+
+
+def compress_dual(xa, za, xb, zb, m: int, prev_xb=None, prev_zb=None) -> np.ndarray:
+    """Dual-series compression: xa, za, xb, zb [B][n_tok][C] stored bytes over the same token range
+    (starting at a block boundary); prev_xb, prev_zb [B][m][C] series b over the block before the
+    range, or None when the range starts the sequence -> entries [B][n_tok//m][C] float64."""
+    xa, za, xb, zb = _c(xa), _c(za), _c(xb), _c(zb)
+    assert xa.shape == za.shape == xb.shape == zb.shape and xa.ndim == 3
+    assert xa.dtype == za.dtype == xb.dtype == zb.dtype
+    B, n_tok, C = xa.shape
+    if prev_xb is not None:
+        prev_xb, prev_zb = _c(prev_xb), _c(prev_zb)
+        assert prev_xb.shape == prev_zb.shape == (B, m, C) and prev_xb.dtype == xa.dtype
+    out = np.zeros((B, n_tok // m, C), dtype=np.float64)
+    st = _load().v4ao_compress_dual(_ptr(xa), _ptr(za), _ptr(xb), _ptr(zb), _ptr(prev_xb), _ptr(prev_zb), fmt_of(xa),
+                                    B, n_tok, C, m, _ptr(out))
+    if st:
+        raise ValueError(f"oracle compress_dual: status {st}")
     return out
 
 

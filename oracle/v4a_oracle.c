@@ -17,6 +17,11 @@
  *    "Heavily Compressed Attention (HCA) / How it works" (single series, every
  *    m' consecutive tokens -> one entry, no overlap).  The same single-series
  *    rule is used for m = 4 and m' = 128.
+ *  - v4ao_compress_dual: "DeepSeek-V4: Million-Token Context via Hybrid
+ *    Compressed Attention", CSA, "Dual-series KV compression" -- entry i is a
+ *    weighted sum of 2m tokens, the m of series a in block i and the m of
+ *    series b in block i-1, with one softmax (per channel) over their 2m gate
+ *    logits.
  *  - v4ao_index_scores: "How V4 makes a million-token context actually
  *    affordable" (deconstructedpapers.com), Lightning-Indexer section:
  *    I(t,s) = sum_j w_j * ReLU(q_j . k_s); the key k_s carries no head index.
@@ -246,6 +251,69 @@ int v4ao_compress(const void* x, const void* gate, int dt, long long batch, long
     if (dt != OR_F32 && dt != OR_BF16) return OR_ERR_ARG;
     compress_ctx k = {x, gate, dt, n_tok, channels, m, n_tok / m, out};
     parallel_for(batch * k.n_ent, compress_item, &k);
+    return OR_OK;
+}
+
+typedef struct {
+    const void *xa, *za, *xb, *zb, *pxb, *pzb;
+    int dt;
+    long long n_tok, c, m, n_ent;
+    double* out;
+} compress_dual_ctx;
+
+static void compress_dual_item(void* vctx, long long item)
+{
+    compress_dual_ctx* k = (compress_dual_ctx*)vctx;
+    long long b = item / k->n_ent, s = item % k->n_ent;
+    const int has_b = s >= 1 || (k->pxb && k->pzb);
+    for (long long ch = 0; ch < k->c; ++ch) {
+        /* the 2m logits: series a over block s, series b over block s-1 (from the
+           previous block of the range, or from prev_* for block 0) */
+        double zv[2][1024], xv[2][1024];
+        for (long long i = 0; i < k->m; ++i) {
+            size_t at = (size_t)((b * k->n_tok + s * k->m + i) * k->c + ch);
+            zv[0][i] = load_elem(k->za, k->dt, at);
+            xv[0][i] = load_elem(k->xa, k->dt, at);
+            if (!has_b) continue;
+            if (s >= 1) {
+                size_t bt = (size_t)((b * k->n_tok + (s - 1) * k->m + i) * k->c + ch);
+                zv[1][i] = load_elem(k->zb, k->dt, bt);
+                xv[1][i] = load_elem(k->xb, k->dt, bt);
+            } else {
+                size_t bt = (size_t)((b * k->m + i) * k->c + ch);
+                zv[1][i] = load_elem(k->pzb, k->dt, bt);
+                xv[1][i] = load_elem(k->pxb, k->dt, bt);
+            }
+        }
+        double zmax = -INFINITY;
+        for (int ser = 0; ser < (has_b ? 2 : 1); ++ser)
+            for (long long i = 0; i < k->m; ++i)
+                if (zv[ser][i] > zmax) zmax = zv[ser][i];
+        double den = 0.0, num = 0.0;
+        for (int ser = 0; ser < (has_b ? 2 : 1); ++ser)
+            for (long long i = 0; i < k->m; ++i) {
+                double e = exp(zv[ser][i] - zmax);
+                den += e;
+                num += e * xv[ser][i];
+            }
+        k->out[(b * k->n_ent + s) * k->c + ch] = num / den;
+    }
+}
+
+/* xa, za, xb, zb: [batch][n_tok][channels] (dtype dt), the two series over the
+ * same token range starting at a block boundary; prev_xb, prev_zb: series b over
+ * the block before the range, [batch][m][channels], or both NULL when the range
+ * starts the sequence.  out: [batch][n_tok/m][channels] binary64.  m <= 1024. */
+int v4ao_compress_dual(const void* xa, const void* za, const void* xb, const void* zb, const void* prev_xb,
+                       const void* prev_zb, int dt, long long batch, long long n_tok, long long channels,
+                       long long m, double* out)
+{
+    if (!xa || !za || !xb || !zb || !out || batch < 0 || n_tok < 0 || channels < 1 || m < 1 || m > 1024)
+        return OR_ERR_ARG;
+    if ((prev_xb == NULL) != (prev_zb == NULL)) return OR_ERR_ARG;
+    if (dt != OR_F32 && dt != OR_BF16) return OR_ERR_ARG;
+    compress_dual_ctx k = {xa, za, xb, zb, prev_xb, prev_zb, dt, n_tok, channels, m, n_tok / m, out};
+    parallel_for(batch * k.n_ent, compress_dual_item, &k);
     return OR_OK;
 }
 

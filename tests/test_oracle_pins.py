@@ -138,6 +138,60 @@ def test_compress_shift_invariance_and_bf16_input():
     assert np.allclose(ob, of, atol=1e-12)
 
 
+# ----------------------------------------------------------------------
+# dual-series compressor ("DeepSeek-V4: Million-Token Context via Hybrid Compressed Attention",
+# CSA, "Dual-series KV compression"): entry i mixes series a over block i and series b over
+# block i-1 under one softmax of their 2m gate logits
+# ----------------------------------------------------------------------
+
+def test_compress_dual_without_series_b_is_single_series():
+    """Gate logits of series b at -inf take it out of every softmax: the single-series result of a."""
+    rng = np.random.default_rng(31)
+    xa, za, xb = (rng.normal(size=(2, 40, 16)).astype(np.float32) for _ in range(3))
+    zb = np.full_like(za, -np.inf)
+    got = oracle.compress_dual(xa, za, xb, zb, 4)
+    assert np.allclose(got, oracle.compress(xa, za, 4), rtol=1e-13, atol=1e-13)
+
+
+def test_compress_dual_same_series_is_a_sliding_2m_window():
+    """With both series equal, entry i (i >= 1) is the single-series entry over the 2m tokens
+    [m(i-1), m(i+1)); entry 0 of a sequence has only its own block."""
+    rng = np.random.default_rng(32)
+    m = 4
+    x = rng.normal(size=(3, 44, 8)).astype(np.float32)
+    z = (2.0 * rng.normal(size=(3, 44, 8))).astype(np.float32)
+    got = oracle.compress_dual(x, z, x, z, m)
+    for i in range(1, 44 // m):
+        win = slice(m * (i - 1), m * (i + 1))
+        ref = oracle.compress(x[:, win], z[:, win], 2 * m)[:, 0]
+        assert np.allclose(got[:, i], ref, rtol=1e-13, atol=1e-13), i
+    assert np.allclose(got[:, 0], oracle.compress(x[:, :m], z[:, :m], m)[:, 0], rtol=1e-13, atol=1e-13)
+
+
+def test_compress_dual_previous_block_continues_the_sequence():
+    """Compressing a range with the previous block's series b given equals compressing the longer
+    range that includes that block, minus its first entry."""
+    rng = np.random.default_rng(33)
+    m = 4
+    xa, za, xb, zb = (rng.normal(size=(2, 48, 12)).astype(np.float32) for _ in range(4))
+    full = oracle.compress_dual(xa, za, xb, zb, m)
+    part = oracle.compress_dual(xa[:, m:], za[:, m:], xb[:, m:], zb[:, m:], m, prev_xb=xb[:, :m], prev_zb=zb[:, :m])
+    assert np.allclose(part, full[:, 1:], rtol=1e-13, atol=1e-13)
+
+
+def test_compress_dual_weights_sum_to_one_and_bf16_input():
+    """Constant content gives that constant whatever the logits; bf16 codes decode before use."""
+    rng = np.random.default_rng(34)
+    za, zb = (rng.normal(size=(1, 32, 8)) * 5 for _ in range(2))
+    ones = np.ones((1, 32, 8), dtype=np.float32)
+    got = oracle.compress_dual(ones, za.astype(np.float32), ones, zb.astype(np.float32), 4)
+    assert np.allclose(got, 1.0, rtol=0, atol=1e-14)
+    xa = rng.normal(size=(1, 32, 8))
+    codes = [oracle.bf16_encode(v) for v in (xa, za, xa, zb)]
+    values = [oracle.bf16_decode(c).astype(np.float32) for c in codes]
+    assert np.array_equal(oracle.compress_dual(*codes, 4), oracle.compress_dual(*values, 4))
+
+
 def test_quantize_rows_bounds():
     rng = np.random.default_rng(6)
     v = rng.normal(size=(50, 128))
