@@ -44,6 +44,12 @@ class CompressIO(ctypes.Structure):
                 ("scale_batch_stride", ctypes.c_longlong)]
 
 
+class SeriesB(ctypes.Structure):
+    _fields_ = [("x", ctypes.c_void_p), ("gate", ctypes.c_void_p), ("prev_x", ctypes.c_void_p),
+                ("prev_gate", ctypes.c_void_p), ("x_batch_stride", ctypes.c_longlong),
+                ("gate_batch_stride", ctypes.c_longlong), ("prev_batch_stride", ctypes.c_longlong)]
+
+
 def library_path() -> str:
     return _LIB_PATH
 
@@ -57,6 +63,8 @@ def _load():
     P = ctypes.POINTER
     L.v4a_compress.restype = i32
     L.v4a_compress.argtypes = [P(CompressIO), P(CompressIO), i32, ll, i32, vp]
+    L.v4a_compress_dual.restype = i32
+    L.v4a_compress_dual.argtypes = [P(CompressIO), P(SeriesB), i32, ll, i32, vp]
     L.v4a_index_scores.restype = i32
     L.v4a_index_scores.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, P(Shape), vp]
     L.v4a_topk.restype = i32
@@ -173,6 +181,23 @@ def v4a_compress(x, gate, out, *, m: int, n_tok: int | None = None, out_scale=No
         idx = _io(xi, gate_i, out_i, out_i_scale)
     _check(lib.v4a_compress(ctypes.byref(kv), ctypes.byref(idx) if idx is not None else None, int(x.shape[0]), n,
                             int(m), _stream(stream)))
+
+
+def v4a_compress_dual(x_a, gate_a, x_b, gate_b, out, *, m: int, prev_x_b=None, prev_gate_b=None, out_scale=None,
+                      n_tok: int | None = None, stream=None) -> None:
+    """Dual-series compression: entry s of the range mixes series a over block s and series b over
+    block s-1 (prev_x_b / prev_gate_b [batch][m][channels] for block -1, or None at the start of a
+    sequence) under one per-channel softmax.  Tensors are [batch][rows][channels]."""
+    n = x_a.shape[1] if n_tok is None else int(n_tok)
+    a = _io(x_a, gate_a, out, out_scale)
+    for t, name in ((x_b, "x_b"), (gate_b, "gate_b"), (prev_x_b, "prev_x_b"), (prev_gate_b, "prev_gate_b")):
+        if t is not None and (t.dim() != 3 or t.stride(2) != 1 or t.stride(1) != t.shape[2]):
+            raise ValueError(f"{name} must be [batch][rows][channels] with dense rows")
+    prev_bs = prev_x_b.stride(0) if prev_x_b is not None else 0
+    if prev_x_b is not None and prev_gate_b is not None and prev_gate_b.stride(0) != prev_bs:
+        raise ValueError("prev_x_b and prev_gate_b must have the same batch stride")
+    b = SeriesB(_ptr(x_b), _ptr(gate_b), _ptr(prev_x_b), _ptr(prev_gate_b), x_b.stride(0), gate_b.stride(0), prev_bs)
+    _check(lib.v4a_compress_dual(ctypes.byref(a), ctypes.byref(b), int(x_a.shape[0]), n, int(m), _stream(stream)))
 
 
 def v4a_index_scores(q_i, w, k_i, k_scale, scores, *, m: int, ctx_len: int, stream=None) -> None:

@@ -4,6 +4,9 @@
 // an entry is the per-channel softmax (over the chunk's m tokens, from the gate
 // logits Z) weighted sum of the content rows C.  One launch compresses both the
 // K=V stream and, optionally, the indexer-key stream of the same chunks.
+// The dual-series form ("DeepSeek-V4: Million-Token Context via Hybrid
+// Compressed Attention", CSA, "Dual-series KV compression") adds series b's
+// rows of the previous block to the same per-channel softmax.
 //
 // Mapping: S adjacent lanes (S = the largest power of two <= min(m, 32); 1
 // for FP8 output) own 8 consecutive channels of one entry; each takes every
@@ -22,6 +25,11 @@ namespace {
 struct StreamDesc {
     const void* x;
     const void* gate;
+    const void* xb;     // dual series: series b over the range (null: single series)
+    const void* gateb;
+    const void* pxb;    // series b over the block before the range (null: none)
+    const void* pgateb;
+    long long xb_bs, gateb_bs, prev_bs;
     void* out;
     float* out_scale;
     int channels, groups;  // groups = channels / 8
@@ -34,10 +42,8 @@ struct StreamDesc {
 // rounds of kU tokens whose loads are all issued first; per round one max, one rescale of the
 // running state and one exp per element.
 template <typename T>
-__device__ __forceinline__ void compress_group(const StreamDesc& d, int b, long long s, int grp, int m, int sub,
-                                               float mx[8], float den[8], float num[8]) {
-    const T* xp = static_cast<const T*>(d.x) + (long long)b * d.x_bs + s * m * d.channels + grp * 8;
-    const T* zp = static_cast<const T*>(d.gate) + (long long)b * d.gate_bs + s * m * d.channels + grp * 8;
+__device__ __forceinline__ void compress_span(const StreamDesc& d, const T* xp, const T* zp, int m, int sub,
+                                              float mx[8], float den[8], float num[8]) {
     constexpr int kU = 4;
     for (int i0 = sub; i0 < m; i0 += kU * d.split) {
         float xv[kU][8], zv[kU][8];
@@ -97,10 +103,34 @@ __global__ void __launch_bounds__(256) compress_kernel(StreamDesc s0, StreamDesc
         num[e] = 0.f;
     }
     if (active) {
-        if (d.in_dtype == V4A_BF16)
-            compress_group<__nv_bfloat16>(d, b, s, grp, m, sub, mx, den, num);
-        else
-            compress_group<float>(d, b, s, grp, m, sub, mx, den, num);
+        // series a (or the single series) over block s; series b over block s-1 of the range, or the
+        // block before the range
+        const long long off = s * m * d.channels + grp * 8;
+        const size_t es = d.in_dtype == V4A_BF16 ? 2 : 4;
+        const char* xa = static_cast<const char*>(d.x) + ((long long)b * d.x_bs + off) * es;
+        const char* za = static_cast<const char*>(d.gate) + ((long long)b * d.gate_bs + off) * es;
+        const char* xb = nullptr;
+        const char* zb = nullptr;
+        if (d.xb && s >= 1) {
+            xb = static_cast<const char*>(d.xb) + ((long long)b * d.xb_bs + off - (long long)m * d.channels) * es;
+            zb = static_cast<const char*>(d.gateb) + ((long long)b * d.gateb_bs + off - (long long)m * d.channels) * es;
+        } else if (d.xb && d.pxb) {
+            xb = static_cast<const char*>(d.pxb) + ((long long)b * d.prev_bs + grp * 8) * es;
+            zb = static_cast<const char*>(d.pgateb) + ((long long)b * d.prev_bs + grp * 8) * es;
+        }
+        if (d.in_dtype == V4A_BF16) {
+            compress_span(d, reinterpret_cast<const __nv_bfloat16*>(xa), reinterpret_cast<const __nv_bfloat16*>(za),
+                          m, sub, mx, den, num);
+            if (xb)
+                compress_span(d, reinterpret_cast<const __nv_bfloat16*>(xb),
+                              reinterpret_cast<const __nv_bfloat16*>(zb), m, sub, mx, den, num);
+        } else {
+            compress_span(d, reinterpret_cast<const float*>(xa), reinterpret_cast<const float*>(za), m, sub, mx,
+                          den, num);
+            if (xb)
+                compress_span(d, reinterpret_cast<const float*>(xb), reinterpret_cast<const float*>(zb), m, sub, mx,
+                              den, num);
+        }
     }
     // merge the S lanes' partial states (S adjacent lanes, S a power of two): the common max,
     // one rescale per lane, then plain sums
@@ -155,6 +185,8 @@ StreamDesc describe(const v4a_compress_io* io) {
     StreamDesc d;
     d.x = io->x;
     d.gate = io->gate;
+    d.xb = d.gateb = d.pxb = d.pgateb = nullptr;
+    d.xb_bs = d.gateb_bs = d.prev_bs = 0;
     d.out = io->out;
     d.out_scale = io->out_scale;
     d.channels = io->channels;
@@ -188,6 +220,28 @@ cudaError_t launch_compress(const v4a_compress_io* kv, const v4a_compress_io* id
     const int threads = 256;
     dim3 grid((unsigned)((total + threads - 1) / threads), idx ? 2 : 1);
     compress_kernel<<<grid, threads, 0, stream>>>(s0, s1, batch, n_ent, m);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_compress_dual(const v4a_compress_io* a, const v4a_series_b* b, int batch, long long n_tok, int m,
+                                 cudaStream_t stream) {
+    long long n_ent = n_tok / m;
+    if (batch == 0 || n_ent == 0) return cudaSuccess;
+    StreamDesc s0 = describe(a);
+    s0.xb = b->x;
+    s0.gateb = b->gate;
+    s0.pxb = b->prev_x;
+    s0.pgateb = b->prev_gate;
+    s0.xb_bs = b->x_batch_stride;
+    s0.gateb_bs = b->gate_batch_stride;
+    s0.prev_bs = b->prev_batch_stride;
+    int split = 1;
+    while (split < 32 && split * 2 <= m) split *= 2;
+    if (s0.out_dtype != V4A_FP8E4M3) s0.split = split;
+    const long long total = (long long)batch * n_ent * s0.groups * s0.split;
+    const int threads = 256;
+    dim3 grid((unsigned)((total + threads - 1) / threads), 1);
+    compress_kernel<<<grid, threads, 0, stream>>>(s0, s0, batch, n_ent, m);
     return cudaGetLastError();
 }
 

@@ -15,6 +15,8 @@ v4a_status report(v4a_status st, const char* fmt, ...);
 // ---- compress.cu ------------------------------------------------------
 cudaError_t launch_compress(const v4a_compress_io* kv, const v4a_compress_io* idx, int batch, long long n_tok,
                             int m, cudaStream_t stream);
+cudaError_t launch_compress_dual(const v4a_compress_io* a, const v4a_series_b* b, int batch, long long n_tok, int m,
+                                 cudaStream_t stream);
 
 // ---- indexer.cu -------------------------------------------------------
 struct IndexArgs {

@@ -165,6 +165,27 @@ v4a_status v4a_compress(const v4a_compress_io* kv, const v4a_compress_io* idx, i
     return from_cuda(v4a::launch_compress(kv, idx, batch, n_tok, m, (cudaStream_t)stream), "v4a_compress");
 }
 
+v4a_status v4a_compress_dual(const v4a_compress_io* a, const v4a_series_b* b, int batch, long long n_tok, int m,
+                             void* stream) {
+    if (!a || !b) return fail(V4A_ERR_INVALID_ARG, "v4a_compress_dual: series a and b are required");
+    if (batch < 0 || n_tok < 0 || m < 1) return fail(V4A_ERR_INVALID_ARG, "need batch >= 0, n_tok >= 0, m >= 1");
+    if (batch == 0 || n_tok / m == 0) return V4A_OK;  // no complete chunk: nothing to write
+    v4a_status st = check_compress_io(a, "series a", n_tok, m);
+    if (st != V4A_OK) return st;
+    if (!b->x || !b->gate) return fail(V4A_ERR_INVALID_ARG, "series b: x and gate are required");
+    if ((b->prev_x == nullptr) != (b->prev_gate == nullptr))
+        return fail(V4A_ERR_INVALID_ARG, "series b: prev_x and prev_gate must both be given or both be NULL");
+    const size_t in_sz = dtype_size(a->in_dtype);
+    if (b->x_batch_stride < n_tok * a->channels || b->gate_batch_stride < n_tok * a->channels ||
+        (b->prev_x && b->prev_batch_stride < (long long)m * a->channels))
+        return fail(V4A_ERR_INVALID_ARG, "series b: a batch stride is smaller than one sequence");
+    if (!aligned(b->x, 16) || !aligned(b->gate, 16) || (b->prev_x && (!aligned(b->prev_x, 16) || !aligned(b->prev_gate, 16))) ||
+        (b->x_batch_stride * in_sz) % 16 || (b->gate_batch_stride * in_sz) % 16 ||
+        (b->prev_x && (b->prev_batch_stride * in_sz) % 16))
+        return fail(V4A_ERR_INVALID_ARG, "series b: pointers or strides are not 16-byte aligned");
+    return from_cuda(v4a::launch_compress_dual(a, b, batch, n_tok, m, (cudaStream_t)stream), "v4a_compress_dual");
+}
+
 v4a_status v4a_index_scores(const void* q_i, const float* w, const void* k_i, const float* k_scale, float* scores,
                             int heads_i, int d_i, v4a_dtype q_dtype, v4a_dtype k_dtype, const v4a_shape* shape,
                             void* stream) {

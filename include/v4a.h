@@ -118,6 +118,38 @@ typedef struct v4a_compress_io {
 V4A_API v4a_status v4a_compress(const v4a_compress_io* kv, const v4a_compress_io* idx, int batch, long long n_tok, int m,
                         void* stream);
 
+/* Series b of the dual-series compressor: its rows over the same token range
+ * as series a (the x / gate of the v4a_compress_io passed with it), and over
+ * the m tokens just before that range. */
+typedef struct v4a_series_b {
+    const void* x;                 /* content rows [batch][n_tok][channels], series a's in_dtype */
+    const void* gate;              /* gate logits, same shape and dtype */
+    const void* prev_x;            /* rows of the block before the range [batch][m][channels], or NULL
+                                      when the range starts the sequence */
+    const void* prev_gate;         /* same shape; NULL exactly when prev_x is NULL */
+    long long x_batch_stride;      /* elements between sequences in x (>= n_tok*channels) */
+    long long gate_batch_stride;   /* elements between sequences in gate */
+    long long prev_batch_stride;   /* elements between sequences in prev_x and prev_gate (>= m*channels) */
+} v4a_series_b;
+
+/* Dual-series chunk compression ("DeepSeek-V4: Million-Token Context via
+ * Hybrid Compressed Attention", CSA, "Dual-series KV compression"): entry s
+ * of the range mixes 2m token rows, the m of series a in block s and the m
+ * of series b in block s-1, under one softmax per channel over their 2m
+ * gate logits:
+ *     out[s][c] = ( sum_{i<m} e^{Za[ms+i][c]} Xa[ms+i][c]
+ *                 + sum_{i<m} e^{Zb[m(s-1)+i][c]} Xb[m(s-1)+i][c] ) / (same sums of e^Z),
+ * with block -1 of the range read from b->prev_x / prev_gate, and left out
+ * when those are NULL (the first entry of a sequence).
+ * a: series a, the output and its dtype, exactly as for v4a_compress (out,
+ * out_scale, FP8E4M3 rule).  b: series b.  n_tok: tokens per sequence in the
+ * range, which starts at a chunk boundary; a trailing partial chunk is
+ * ignored.  Errors: those of v4a_compress, plus V4A_ERR_INVALID_ARG for a
+ * NULL b->x / b->gate, exactly one of prev_x / prev_gate NULL, strides too
+ * small or misaligned series-b pointers (16 bytes). */
+V4A_API v4a_status v4a_compress_dual(const v4a_compress_io* a, const v4a_series_b* b, int batch, long long n_tok,
+                                     int m, void* stream);
+
 /* ------------------------------------------------------------------ */
 /* Lightning indexer and top-k                                          */
 /* ------------------------------------------------------------------ */

@@ -88,6 +88,53 @@ def test_compress_fused_streams_fp8_keys_and_strided_cache(v4a):
     assert (scales[:, :s0] == 0).all() and (keys[:, s0 + n_ent:] == 0).all()
 
 
+@pytest.mark.parametrize("fmt,m,n_tok,C,with_prev", [("f32", 4, 4 * 37 + 3, 128, False), ("f32", 4, 4 * 20, 64, True),
+                                                   ("bf16", 4, 4 * 300 + 1, 512, True), ("bf16", 1, 33, 128, False),
+                                                   ("bf16", 16, 16 * 9, 512, True), ("f32", 128, 128 * 3 + 5, 128, True)])
+def test_compress_dual_matches_oracle(v4a, fmt, m, n_tok, C, with_prev):
+    """Dual-series compression of a token range: series a over each block, series b over the block
+    before it (the range's previous block, or prev_* for the first entry when given)."""
+    B = 2
+    ca = wl.compress_case(B, n_tok, C, fmt, seed=200 + m)
+    cb = wl.compress_case(B, n_tok, C, fmt, seed=300 + m, gate_std=2.0)
+    pr = wl.compress_case(B, m, C, fmt, seed=400 + m) if with_prev else None
+    n_ent = n_tok // m
+    out = torch.empty((B, n_ent, C), dtype=dev(ca["x"]).dtype, device="cuda")
+    v4a.v4a_compress_dual(dev(ca["x"]), dev(ca["gate"]), dev(cb["x"]), dev(cb["gate"]), out, m=m,
+                          prev_x_b=dev(pr["x"]) if pr else None, prev_gate_b=dev(pr["gate"]) if pr else None)
+    _sync()
+    ref = oracle.compress_dual(host(ca["x"]), host(ca["gate"]), host(cb["x"]), host(cb["gate"]), m,
+                               prev_xb=host(pr["x"]) if pr else None, prev_zb=host(pr["gate"]) if pr else None)
+    g = out.double().cpu().numpy()
+    if fmt == "f32":
+        assert np.abs(g - ref).max() <= 2e-6 * max(1.0, np.abs(ref).max())
+    else:  # bf16 output: within one bf16 rounding of the fp64 value (+ fp32 slack)
+        assert (np.abs(g - ref) <= np.abs(ref) * 2.0 ** -8 + 1e-6).all()
+
+
+def test_compress_dual_fp8_output_into_cache_slice(v4a):
+    """bf16 series -> FP8 entries + scales written into the middle of a larger cache, the block before
+    the range given."""
+    B, m, n_tok, C = 3, 4, 4 * 40, 128
+    ca = wl.compress_case(B, n_tok + m, C, "bf16", seed=501)
+    cb = wl.compress_case(B, n_tok + m, C, "bf16", seed=502, gate_std=2.0)
+    cap, s0, n_ent = 60, 9, n_tok // m
+    keys = torch.zeros((B, cap, C), dtype=torch.uint8, device="cuda")
+    scales = torch.zeros((B, cap), dtype=torch.float32, device="cuda")
+    xa, za, xb, zb = (dev(t) for t in (ca["x"], ca["gate"], cb["x"], cb["gate"]))
+    v4a.v4a_compress_dual(xa[:, m:], za[:, m:], xb[:, m:], zb[:, m:], keys[:, s0:s0 + n_ent], m=m,
+                          prev_x_b=xb[:, :m], prev_gate_b=zb[:, :m], out_scale=scales[:, s0:s0 + n_ent])
+    _sync()
+    full = oracle.compress_dual(host(ca["x"]), host(ca["gate"]), host(cb["x"]), host(cb["gate"]), m)
+    ref = full[:, 1:]
+    _, ref_sc = oracle.quantize_e4m3_rows(ref)
+    sc = scales[:, s0:s0 + n_ent].double().cpu().numpy()
+    assert np.allclose(sc, ref_sc, rtol=1e-5)
+    deq = oracle.e4m3_decode(keys[:, s0:s0 + n_ent].cpu().numpy()) * sc[..., None]
+    assert np.abs(deq - ref).max() <= 0.07 * np.abs(ref).max()  # e4m3 keeps 3 mantissa bits
+    assert (keys[:, :s0] == 0).all() and (keys[:, s0 + n_ent:] == 0).all()
+
+
 def test_compress_empty_and_short(v4a):
     x = torch.randn((2, 3, 64), device="cuda")
     out = torch.full((2, 1, 64), 7.0, device="cuda")
