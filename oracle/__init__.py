@@ -54,6 +54,11 @@ def _load():
     lib.v4ao_n_visible.argtypes = [ll, ll]
     lib.v4ao_compress.restype = i32
     lib.v4ao_compress.argtypes = [vp, vp, i32, ll, ll, ll, ll, vp]
+    lib.v4ao_attend_ex.restype = i32
+    lib.v4ao_attend_ex.argtypes = [vp, vp, vp, ll, vp, ll, ll, i32, ll, ll, ll, ll, ll, ll, ll, vp, ll,
+                                   ctypes.c_double, vp]
+    lib.v4ao_rope.restype = i32
+    lib.v4ao_rope.argtypes = [vp, ll, ll, vp, ll, ctypes.c_double]
     lib.v4ao_compress_dual.restype = i32
     lib.v4ao_compress_dual.argtypes = [vp, vp, vp, vp, vp, vp, i32, ll, ll, ll, ll, vp]
     lib.v4ao_quantize_e4m3_rows.restype = i32
@@ -238,22 +243,40 @@ def topk(q_i, w, k_i, k_scale, ctx_len: int, m: int, k: int, want_scores: bool =
 
 
 def attend(q, entries, idx, token_kv, tok_pos0: int, ctx_len: int, m: int, window: int,
-           allow_bad_index: bool = False) -> np.ndarray:
+           allow_bad_index: bool = False, sink=None, rope_dims: int = 0, rope_base: float = 10000.0) -> np.ndarray:
     """Joint-softmax attention over selected (idx given: CSA) or all visible
     (idx None: HCA) compressed entries plus the window tokens.
     q [B][T][H][d], entries [B][N][d], idx [B][T][k] int32 or None,
-    token_kv [B][L_tok][d] (row r = position tok_pos0 + r) -> out [B][T][H][d] float64."""
+    token_kv [B][L_tok][d] (row r = position tok_pos0 + r) -> out [B][T][H][d] float64.
+    sink: per-head sink logits [H] (joining each head's softmax denominator as e^sink), or None;
+    rope_dims > 0: the output's last rope_dims dims rotated by RoPE at minus the query position."""
     q, entries, token_kv = _c(q), _c(entries), _c(token_kv)
     assert q.dtype == entries.dtype == token_kv.dtype
     B, T, H, d = q.shape
     ix = None if idx is None else _c(idx, np.int32)
     ksel = 0 if ix is None else ix.shape[-1]
+    sk = None if sink is None else _c(sink, np.float64)
+    assert sk is None or sk.shape == (H,)
     out = np.zeros((B, T, H, d), dtype=np.float64)
-    st = _load().v4ao_attend(_ptr(q), _ptr(entries), _ptr(ix), ksel, _ptr(token_kv), tok_pos0, token_kv.shape[1],
-                             fmt_of(q), B, T, H, d, m, window, ctx_len, _ptr(out))
+    st = _load().v4ao_attend_ex(_ptr(q), _ptr(entries), _ptr(ix), ksel, _ptr(token_kv), tok_pos0, token_kv.shape[1],
+                                fmt_of(q), B, T, H, d, m, window, ctx_len, _ptr(sk), int(rope_dims), float(rope_base),
+                                _ptr(out))
     if st and not (allow_bad_index and st == 4):
         raise ValueError(f"oracle attend: status {st}")
     return out
+
+
+def rope(x, pos, rope_dims: int, base: float = 10000.0) -> np.ndarray:
+    """RoPE on the last rope_dims dims of rows x [..][d] (float64 copy), row i at position pos[i]
+    (pos broadcast over the leading dims)."""
+    x = np.array(x, dtype=np.float64, copy=True)
+    d = x.shape[-1]
+    rows = x.reshape(-1, d)
+    p = np.ascontiguousarray(np.broadcast_to(np.asarray(pos, dtype=np.float64), x.shape[:-1]).reshape(-1))
+    st = _load().v4ao_rope(_ptr(rows), rows.shape[0], d, _ptr(p), int(rope_dims), float(base))
+    if st:
+        raise ValueError(f"oracle rope: status {st}")
+    return rows.reshape(x.shape)
 
 
 def attend_weights(q, entries, idx, token_kv, tok_pos0: int, ctx_len: int, m: int, window: int,

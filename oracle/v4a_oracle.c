@@ -36,6 +36,12 @@
  *    candidates are the selected (CSA) or all visible (HCA) compressed entries
  *    plus the raw sliding-window tokens ("1M Context != ...", section 6), in
  *    ONE joint softmax.
+ *  - Attention sink and output RoPE ("1M Context != Lossless Long Memory",
+ *    sections 7 and 8): a per-head scalar z'_h joins the softmax denominator
+ *    (read as the logit of an extra, empty candidate: the denominator gains
+ *    e^{z'_h}); RoPE acts on the last R dims of the vectors, and the attention
+ *    output of the query at position t is rotated at position -t.  RoPE pairs
+ *    adjacent dims (2k, 2k+1) of those R with frequency base^(-2k/R).
  *  - Visibility: entry s covers tokens [m*s, m*s+m) and is visible to query
  *    position t iff m*(s+1) <= t+1 ("1M Context != ...", section 6.1: a query
  *    must not read its own, still incomplete, compressed block).
@@ -507,6 +513,9 @@ typedef struct {
     long long n_q, heads, d, m, window, ctx_len, n_ent, hgroup;
     double* out;
     int bad_index; /* set when an idx entry is out of range */
+    const double* sink; /* per-head sink logits, or NULL */
+    long long rope_dims;
+    double rope_base;
 } attend_ctx;
 
 /* Candidate rows of query (b, j): pointers to element 0 of each row, as
@@ -582,8 +591,31 @@ static void head_weights(const attend_ctx* a, long long b, long long j, long lon
         wts[i] = exp(wts[i] - mx);
         den += wts[i];
     }
+    if (a->sink) den += exp(a->sink[h] - mx); /* the sink: in the denominator only */
     for (long long i = 0; i < n; ++i) wts[i] /= den;
     free(qd);
+}
+
+/* RoPE at position pos on the last rope_dims entries of x[0..d): pair k = (d - R + 2k,
+ * d - R + 2k + 1) rotates by pos * base^(-2k/R). */
+static void rope_rotate(double* x, long long d, long long rope_dims, double base, double pos)
+{
+    for (long long k = 0; k < rope_dims / 2; ++k) {
+        double ang = pos * pow(base, -2.0 * (double)k / (double)rope_dims);
+        double c = cos(ang), sn = sin(ang);
+        double* p = x + (d - rope_dims) + 2 * k;
+        double u = p[0], v = p[1];
+        p[0] = u * c - v * sn;
+        p[1] = u * sn + v * c;
+    }
+}
+
+/* rows: [n][d] binary64, rotated in place, row r at position pos[r] */
+int v4ao_rope(double* rows, long long n, long long d, const double* pos, long long rope_dims, double base)
+{
+    if (!rows || !pos || n < 0 || d < 1 || rope_dims < 0 || rope_dims > d || rope_dims % 2) return OR_ERR_ARG;
+    for (long long r = 0; r < n; ++r) rope_rotate(rows + r * d, d, rope_dims, base, pos[r]);
+    return OR_OK;
 }
 
 static void attend_item(void* vctx, long long item)
@@ -609,6 +641,7 @@ static void attend_item(void* vctx, long long item)
         head_weights(a, b, j, h, mat, n, wts);
         for (long long i = 0; i < n; ++i)
             for (long long c = 0; c < a->d; ++c) o[c] += wts[i] * mat[i * a->d + c];
+        if (a->rope_dims > 0) rope_rotate(o, a->d, a->rope_dims, a->rope_base, -(double)(a->ctx_len - a->n_q + j));
     }
     free(mat);
     free(wts);
@@ -622,19 +655,28 @@ static void attend_item(void* vctx, long long item)
  * all of q/entries/token_kv in dtype dt.  out: [batch][n_q][heads][d] binary64.
  * Returns OR_ERR_INDEX (after computing everything else) if an idx entry was
  * out of range or the window was not covered by token_kv. */
-int v4ao_attend(const void* q, const void* entries, const int32_t* idx, long long k_sel, const void* token_kv,
-                long long tok_pos0, long long l_tok, int dt, long long batch, long long n_q, long long heads,
-                long long d, long long m, long long window, long long ctx_len, double* out)
+int v4ao_attend_ex(const void* q, const void* entries, const int32_t* idx, long long k_sel, const void* token_kv,
+                   long long tok_pos0, long long l_tok, int dt, long long batch, long long n_q, long long heads,
+                   long long d, long long m, long long window, long long ctx_len, const double* sink,
+                   long long rope_dims, double rope_base, double* out)
 {
     if (!q || !entries || !token_kv || !out || batch < 0 || n_q < 1 || heads < 1 || d < 1 || m < 1 || window < 0)
         return OR_ERR_ARG;
     if (n_q > ctx_len || (idx && k_sel < 1)) return OR_ERR_ARG;
-    if (dt != OR_F32 && dt != OR_BF16) return OR_ERR_ARG;
+    if (rope_dims < 0 || rope_dims > d || rope_dims % 2 || (rope_dims > 0 && !(rope_base > 0.0))) return OR_ERR_ARG;
     attend_ctx a = {q, entries, idx, k_sel, token_kv, tok_pos0, l_tok, dt, n_q, heads, d, m, window, ctx_len,
-                    ctx_len / m, 8, out, 0};
+                    ctx_len / m, 8, out, 0, sink, rope_dims, rope_base};
     long long ngroups = (heads + a.hgroup - 1) / a.hgroup;
     parallel_for(batch * n_q * ngroups, attend_item, &a);
     return a.bad_index ? OR_ERR_INDEX : OR_OK;
+}
+
+int v4ao_attend(const void* q, const void* entries, const int32_t* idx, long long k_sel, const void* token_kv,
+                long long tok_pos0, long long l_tok, int dt, long long batch, long long n_q, long long heads,
+                long long d, long long m, long long window, long long ctx_len, double* out)
+{
+    return v4ao_attend_ex(q, entries, idx, k_sel, token_kv, tok_pos0, l_tok, dt, batch, n_q, heads, d, m, window,
+                          ctx_len, NULL, 0, 10000.0, out);
 }
 
 /* Softmax weights of one (sequence b, query j, head h) over its candidate
@@ -648,7 +690,7 @@ long long v4ao_attend_weights(const void* q, const void* entries, const int32_t*
 {
     if (!q || !entries || !token_kv || !wts || j < 0 || j >= n_q || h < 0 || h >= heads) return -1;
     attend_ctx a = {q, entries, idx, k_sel, token_kv, tok_pos0, l_tok, dt, n_q, heads, d, m, window, ctx_len,
-                    ctx_len / m, 8, NULL, 0};
+                    ctx_len / m, 8, NULL, 0, NULL, 0, 10000.0};
     long long cap = (idx ? k_sel : a.n_ent) + window + 1;
     size_t* rows = (size_t*)malloc(sizeof(size_t) * cap);
     int* src = (int*)malloc(sizeof(int) * cap);

@@ -477,3 +477,82 @@ def test_bf16_attention_matches_fp32_of_same_values():
     f = lambda a: oracle.decode(a).astype(np.float32)
     o_f = oracle.attend(f(q), f(ent), None, f(tok), p0, 256, 4, 16)
     assert np.allclose(o_b, o_f, atol=1e-12)
+
+
+# ----------------------------------------------------------------------
+# attention sink and output RoPE ("1M Context != Lossless Long Memory", sections 7 and 8)
+# ----------------------------------------------------------------------
+
+def test_rope_is_the_textbook_rotation():
+    """Pair k of the last R dims turns by pos * 10000^(-2k/R): pair 0 by pos radians; position 0
+    is the identity; rotations compose and keep norms; the first d - R dims are untouched."""
+    d, R = 12, 8
+    e = np.zeros((1, d))
+    e[0, d - R] = 1.0
+    got = oracle.rope(e, [0.7], R)
+    assert np.allclose(got[0, d - R:d - R + 2], [np.cos(0.7), np.sin(0.7)], rtol=0, atol=1e-15)
+    e2 = np.zeros((1, d))
+    e2[0, d - 2] = 1.0  # last pair: frequency 10000^(-(R-2)/R)
+    f = 10000.0 ** (-(R - 2) / R)
+    assert np.allclose(oracle.rope(e2, [3.0], R)[0, d - 2:], [np.cos(3 * f), np.sin(3 * f)], rtol=0, atol=1e-15)
+    rng = np.random.default_rng(41)
+    x = rng.normal(size=(5, d))
+    assert np.array_equal(oracle.rope(x, np.zeros(5), R), x)
+    a = oracle.rope(oracle.rope(x, [1, 2, 3, 4, 5], R), [10, 20, 30, 40, 50], R)
+    assert np.allclose(a, oracle.rope(x, [11, 22, 33, 44, 55], R), rtol=0, atol=1e-12)
+    assert np.allclose(np.linalg.norm(a, axis=1), np.linalg.norm(x, axis=1), rtol=1e-14)
+    assert np.array_equal(a[:, :d - R], x[:, :d - R])
+
+
+def _window_case(seed, L, H=4, d=16, W=8):
+    rng = np.random.default_rng(seed)
+    q = rng.normal(size=(1, 1, H, d)).astype(np.float32)
+    tok = rng.normal(size=(1, L, d)).astype(np.float32)
+    ent = np.zeros((1, max(L // 128, 1), d), dtype=np.float32)
+    return q, ent, tok
+
+
+def test_sink_at_minus_infinity_changes_nothing_and_single_row_closed_form():
+    L, W, H, d = 50, 8, 4, 16
+    q, ent, tok = _window_case(42, L, H, d, W)
+    plain = oracle.attend(q, ent, None, tok, 0, L, 128, W)
+    assert np.array_equal(oracle.attend(q, ent, None, tok, 0, L, 128, W, sink=np.full(H, -np.inf)), plain)
+    # one candidate row v (window 1, no entries): out = v * e^l / (e^l + e^z) with l = q.v / sqrt(d)
+    z = np.array([-1.0, 0.0, 0.5, 3.0])
+    got = oracle.attend(q, ent, None, tok, 0, L, 128, 1, sink=z)
+    v = tok[0, L - 1].astype(np.float64)
+    for h in range(H):
+        ell = float(q[0, 0, h].astype(np.float64) @ v) / np.sqrt(d)
+        assert np.allclose(got[0, 0, h], v / (1.0 + np.exp(z[h] - ell)), rtol=1e-13, atol=1e-15)
+
+
+def test_output_rope_is_undone_by_rope_at_the_query_position():
+    L, W, H, d, R = 70, 16, 4, 32, 8
+    q, ent, tok = _window_case(43, L, H, d, W)
+    plain = oracle.attend(q, ent, None, tok, 0, L, 128, W)
+    rot = oracle.attend(q, ent, None, tok, 0, L, 128, W, rope_dims=R)
+    assert np.array_equal(rot[..., :d - R], plain[..., :d - R])
+    assert np.allclose(oracle.rope(rot, L - 1, R), plain, rtol=0, atol=1e-12)
+
+
+def test_output_rope_turns_absolute_positions_into_distances():
+    """With RoPE at each row's own position on the last R dims of the query and of the K=V rows, the
+    rotated output depends only on distances: shifting every position by the same amount (same
+    content) leaves it unchanged ("1M Context != ...", section 8)."""
+    H, d, R, W = 4, 32, 8, 12
+    rng = np.random.default_rng(44)
+    q0 = rng.normal(size=(1, 1, H, d))
+    rows0 = rng.normal(size=(W, d))
+    outs = []
+    for L in (40, 40 + 37, 40 + 1000):  # query at t = L-1, window rows at positions L-W .. L-1
+        t = L - 1
+        pos = np.arange(L - W, L)
+        q = oracle.rope(q0, t, R).astype(np.float32)
+        tok = np.zeros((1, L, d), dtype=np.float32)
+        tok[0, L - W:] = oracle.rope(rows0, pos, R).astype(np.float32)
+        ent = np.zeros((1, 1, d), dtype=np.float32)
+        # m larger than every context here: no compressed entry is visible, only the window
+        # (the fp32 inputs round differently at each shift: compare with float32-level tolerance)
+        outs.append(oracle.attend(q, ent, None, tok, 0, L, 1 << 20, W, rope_dims=R))
+    for o in outs[1:]:
+        assert np.allclose(o, outs[0], rtol=1e-5, atol=1e-5)
