@@ -50,6 +50,10 @@ class SeriesB(ctypes.Structure):
                 ("gate_batch_stride", ctypes.c_longlong), ("prev_batch_stride", ctypes.c_longlong)]
 
 
+class AttendExt(ctypes.Structure):
+    _fields_ = [("sink", ctypes.c_void_p), ("rope_dims", ctypes.c_int), ("rope_base", ctypes.c_float)]
+
+
 def library_path() -> str:
     return _LIB_PATH
 
@@ -63,6 +67,10 @@ def _load():
     P = ctypes.POINTER
     L.v4a_compress.restype = i32
     L.v4a_compress.argtypes = [P(CompressIO), P(CompressIO), i32, ll, i32, vp]
+    L.v4a_csa_attend_ex.restype = i32
+    L.v4a_csa_attend_ex.argtypes = [vp, vp, vp, vp, ll, ll, vp, i32, vp, sz, vp, P(AttendExt), P(Shape), vp]
+    L.v4a_hca_attend_ex.restype = i32
+    L.v4a_hca_attend_ex.argtypes = [vp, vp, vp, ll, ll, vp, i32, vp, sz, P(AttendExt), P(Shape), vp]
     L.v4a_compress_dual.restype = i32
     L.v4a_compress_dual.argtypes = [P(CompressIO), P(SeriesB), i32, ll, i32, vp]
     L.v4a_index_scores.restype = i32
@@ -236,28 +244,50 @@ def v4a_topk_noalloc(q_i, w, k_i, k_scale, idx_out, score_out=None, *, m: int, k
                                 DI, _dtype(q_i), _dtype(k_i), ctypes.byref(s), _stream(stream)))
 
 
+def _ext(sink, rope_dims: int, rope_base: float):
+    """The _ex options, or None when neither the sink nor the output RoPE is asked for."""
+    if sink is None and not rope_dims:
+        return None
+    if sink is not None:
+        _contig(sink, "sink")
+        if sink.dtype != torch.float32 or sink.dim() != 1:
+            raise ValueError("sink must be a float32 vector [heads]")
+    return AttendExt(_ptr(sink), int(rope_dims), float(rope_base))
+
+
 def v4a_csa_attend(q, entries, idx, token_kv, tok_pos0: int, out, *, m: int, window: int, ctx_len: int,
-                   workspace=None, dev_status=None, stream=None) -> None:
+                   workspace=None, dev_status=None, sink=None, rope_dims: int = 0, rope_base: float = 10000.0,
+                   stream=None) -> None:
+    """CSA attention; sink ([heads] fp32 logits) and rope_dims / rope_base select the attention sink
+    and the output RoPE at minus the query position (v4a_csa_attend_ex)."""
     for t, n in ((q, "q"), (entries, "entries"), (idx, "idx"), (token_kv, "token_kv"), (out, "out")):
         _contig(t, n)
     B, T, H, d = q.shape
     s = _shape(batch=B, n_q=T, heads=H, d=d, m=m, k=idx.shape[-1], window=window, ctx_len=ctx_len)
     if workspace is None:
         workspace = _workspace(lib.v4a_workspace_size(b"csa_attend", ctypes.byref(s), 0, 0), q.device)
-    _check(lib.v4a_csa_attend(_ptr(q), _ptr(entries), _ptr(idx), _ptr(token_kv), int(tok_pos0),
-                              int(token_kv.shape[1]), _ptr(out), _dtype(q), _ptr(workspace),
-                              workspace.numel() * workspace.element_size(), _ptr(dev_status), ctypes.byref(s),
-                              _stream(stream)))
+    args = (_ptr(q), _ptr(entries), _ptr(idx), _ptr(token_kv), int(tok_pos0), int(token_kv.shape[1]), _ptr(out),
+            _dtype(q), _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(dev_status))
+    ext = _ext(sink, rope_dims, rope_base)
+    if ext is None:
+        _check(lib.v4a_csa_attend(*args, ctypes.byref(s), _stream(stream)))
+    else:
+        _check(lib.v4a_csa_attend_ex(*args, ctypes.byref(ext), ctypes.byref(s), _stream(stream)))
 
 
 def v4a_hca_attend(q, entries, token_kv, tok_pos0: int, out, *, m: int, window: int, ctx_len: int, workspace=None,
-                   stream=None) -> None:
+                   sink=None, rope_dims: int = 0, rope_base: float = 10000.0, stream=None) -> None:
+    """HCA attention; sink and rope_dims / rope_base as for v4a_csa_attend (v4a_hca_attend_ex)."""
     for t, n in ((q, "q"), (entries, "entries"), (token_kv, "token_kv"), (out, "out")):
         _contig(t, n)
     B, T, H, d = q.shape
     s = _shape(batch=B, n_q=T, heads=H, d=d, m=m, window=window, ctx_len=ctx_len)
     if workspace is None:
         workspace = _workspace(lib.v4a_workspace_size(b"hca_attend", ctypes.byref(s), 0, 0), q.device)
-    _check(lib.v4a_hca_attend(_ptr(q), _ptr(entries), _ptr(token_kv), int(tok_pos0), int(token_kv.shape[1]),
-                              _ptr(out), _dtype(q), _ptr(workspace), workspace.numel() * workspace.element_size(),
-                              ctypes.byref(s), _stream(stream)))
+    args = (_ptr(q), _ptr(entries), _ptr(token_kv), int(tok_pos0), int(token_kv.shape[1]), _ptr(out), _dtype(q),
+            _ptr(workspace), workspace.numel() * workspace.element_size())
+    ext = _ext(sink, rope_dims, rope_base)
+    if ext is None:
+        _check(lib.v4a_hca_attend(*args, ctypes.byref(s), _stream(stream)))
+    else:
+        _check(lib.v4a_hca_attend_ex(*args, ctypes.byref(ext), ctypes.byref(s), _stream(stream)))

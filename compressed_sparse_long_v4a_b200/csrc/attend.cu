@@ -179,7 +179,7 @@ __global__ void __launch_bounds__(kBlockThreads, 1) attend_split_kernel(AttendAr
     }
     if (!active) return;
 
-    if (plan.n_splits == 1) {
+    if (plan.n_splits == 1 && a.sink == nullptr && a.rope_dims == 0) {  // no combine pass: write the output
         const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
         float* op = a.out + (((long long)row * a.heads + h) * d) + part * kEpt;
 #pragma unroll
@@ -204,9 +204,11 @@ __global__ void __launch_bounds__(kBlockThreads, 1) attend_split_kernel(AttendAr
 }
 
 // grid (rows, heads); each thread merges 4 consecutive output elements
-__global__ void attend_combine_kernel(const float* part_ml, const float* part_o, float* out, int n_splits, int heads,
-                                      int d) {
+__global__ void attend_combine_kernel(const float* part_ml, const float* part_o, int n_splits, AttendArgs a) {
     const int row = blockIdx.x, h = blockIdx.y;
+    const int heads = a.heads, d = a.d;
+    float* out = a.out;
+    const long long t = a.ctx_len - a.n_q + (row % a.n_q);  // the query position (output RoPE)
     float mmax = -INFINITY;
     for (int s = 0; s < n_splits; ++s)
         mmax = fmaxf(mmax, part_ml[2 * (((long long)row * n_splits + s) * heads + h)]);
@@ -228,8 +230,23 @@ __global__ void attend_combine_kernel(const float* part_ml, const float* part_o,
                 acc.w = fmaf(wgt, v.w, acc.w);
             }
         }
+        if (a.sink && mmax != -INFINITY) l += exp2f(a.sink[h] * kLog2e - mmax);  // the sink's share
         const float inv = l > 0.f ? 1.f / l : 0.f;
-        *reinterpret_cast<float4*>(op + e) = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+        float v[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
+        if (a.rope_dims > 0) {
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {  // dims (e + 2j, e + 2j + 1) are one RoPE pair
+                const int dim = e + 2 * j;
+                if (dim >= d - a.rope_dims) {
+                    float s, c;
+                    rope_sincos(t, (dim - (d - a.rope_dims)) >> 1, a.rope_dims, a.rope_base, &s, &c);
+                    const float x = v[2 * j], y = v[2 * j + 1];
+                    v[2 * j] = fmaf(x, c, -y * s);
+                    v[2 * j + 1] = fmaf(x, s, y * c);
+                }
+            }
+        }
+        *reinterpret_cast<float4*>(op + e) = make_float4(v[0], v[1], v[2], v[3]);
     }
 }
 
@@ -272,7 +289,6 @@ cudaError_t launch_dtype(const AttendArgs& a, const SplitPlan& plan, float* ml, 
 
 static size_t core_workspace_bytes(const AttendArgs& a) {
     SplitPlan p = plan_for(a);
-    if (p.n_splits == 1) return 256;
     size_t rows = (size_t)a.batch * a.n_q;
     size_t n = rows * p.n_splits * a.heads;
     size_t ml = ((n * 2 * sizeof(float)) + 255) / 256 * 256;
@@ -299,9 +315,9 @@ cudaError_t launch_attend(const AttendArgs& a, void* ws, size_t ws_bytes, cudaSt
     float* po = reinterpret_cast<float*>(static_cast<char*>(ws) + ((n * 2 * sizeof(float)) + 255) / 256 * 256);
     cudaError_t e = a.dtype == V4A_BF16 ? launch_dtype<__nv_bfloat16>(a, plan, ml, po, stream)
                                         : launch_dtype<float>(a, plan, ml, po, stream);
-    if (e != cudaSuccess || plan.n_splits == 1) return e;
+    if (e != cudaSuccess || (plan.n_splits == 1 && a.sink == nullptr && a.rope_dims == 0)) return e;
     attend_combine_kernel<<<dim3((unsigned)rows, a.heads), a.d / 4 < 128 ? a.d / 4 : 128, 0, stream>>>(
-        ml, po, a.out, plan.n_splits, a.heads, a.d);
+        ml, po, plan.n_splits, a);
     return cudaGetLastError();
 }
 

@@ -81,6 +81,9 @@ struct TcArgs {
     int rows, n_q, m, k, window;
     int e_tiles, w_tiles, tpr, grid;
     float scale_log2;
+    const float* sink;  // [64] sink logits, or null
+    int rope_dims;      // output dims rotated at minus the query position (0: none)
+    float rope_base;
 };
 
 __device__ __forceinline__ long long range_start(int c, const TcArgs& a) {
@@ -416,13 +419,15 @@ __device__ void softmax_warps(Smem& sm, const TcArgs& a, uint32_t tmem, long lon
             if (!tc::mbar_wait(&sm.p_free[s], (jt >> 1) & 1)) { ok = false; break; }
             tc::tc_fence_after();
             const float l_row = l_run + __shfl_xor_sync(0xffffffffu, l_run, 16);
-            if (half == 0) {
-                sm.m_s[h] = m_run;
-                sm.l_s[h] = l_row;
-            }
-            tc::named_barrier(1, 128);
             const long long rs = (long long)row * a.tpr;
             const bool whole = (rs >= f0) && (rs + a.tpr <= f1);
+            if (half == 0) {
+                sm.m_s[h] = m_run;
+                // a whole row is normalised here: the sink joins its denominator (a split row's in the combine)
+                sm.l_s[h] = l_row + ((whole && a.sink && m_run != -INFINITY)
+                                         ? exp2f(a.sink[h] * 1.4426950408889634f - m_run) : 0.f);
+            }
+            tc::named_barrier(1, 128);
             // a piece of a split query: slot 2c for the CTA's first query, 2c+1 for its last
             const int slot = 2 * cta + (row == first_row ? 0 : 1);
             float* dst;
@@ -442,10 +447,21 @@ __device__ void softmax_warps(Smem& sm, const TcArgs& a, uint32_t tmem, long lon
                 tc::tmem_ld_wait();
                 const int d = 128 * cc + 32 * sub + lane;
                 if (whole) {
+                    // output RoPE: dims d and d ^ 1 are a pair held by neighbouring lanes
+                    const bool rot = a.rope_dims > 0;
+                    float rs_ = 0.f, rc_ = 1.f;
+                    if (rot && d >= kD - a.rope_dims)
+                        rope_sincos(a.ctx_len - a.n_q + (row % a.n_q), (d - (kD - a.rope_dims)) >> 1, a.rope_dims,
+                                    a.rope_base, &rs_, &rc_);
 #pragma unroll
                     for (int i = 0; i < kH; ++i) {
                         const float l = sm.l_s[i];
-                        dst[i * kD + d] = l > 0.f ? __uint_as_float(o[i]) / l : 0.f;
+                        float v = l > 0.f ? __uint_as_float(o[i]) / l : 0.f;
+                        if (rot) {
+                            const float p = __shfl_xor_sync(0xffffffffu, v, 1);
+                            if (d >= kD - a.rope_dims) v = rope_apply(d, v, p, rs_, rc_);
+                        }
+                        dst[i * kD + d] = v;
                     }
                 } else {
                     // a piece is stored d-major ([d][64 heads]): this thread's 64 heads are contiguous
@@ -563,6 +579,7 @@ __global__ void __launch_bounds__(256) attend_tc_combine(TcArgs a) {
             s_w[i][h] = wgt;
             l += wgt * li;
         }
+        if (a.sink && mmax != -INFINITY) l += exp2f(a.sink[h] * 1.4426950408889634f - mmax);  // the sink's share
         const float inv = bad ? NAN : (l > 0.f ? 1.f / l : 0.f);
         for (int i = 0; i < n; ++i) s_w[i][h] *= inv;
         if (bad || !(l > 0.f)) s_w[0][h] = bad ? NAN : 0.f;  // NaN poisons, an empty row stays zero
@@ -602,10 +619,19 @@ __global__ void __launch_bounds__(256) attend_tc_combine(TcArgs a) {
 #pragma unroll
     for (int j = 0; j < kDC / 4; ++j) s_acc[h][dq + 4 * j] = isnan(w0) ? NAN : acc[j];
     __syncthreads();
-    // write out[row][h][d0 .. d0+31]: warp w covers heads w, w+8, ...; lane = d
-    const int lane = t & 31, w = t >> 5;
-    for (int hh = w; hh < kH; hh += 8)
-        a.out[((long long)row * kH + hh) * kD + d0 + lane] = s_acc[hh][lane];
+    // write out[row][h][d0 .. d0+31]: warp w covers heads w, w+8, ...; lane = d (output RoPE: the pair
+    // partner of d is d ^ 1, in the same 32)
+    const int lane = t & 31, w = t >> 5, d = d0 + lane;
+    const bool rot = a.rope_dims > 0 && d >= kD - a.rope_dims;
+    float rs_ = 0.f, rc_ = 1.f;
+    if (rot)
+        rope_sincos(a.ctx_len - a.n_q + (row % a.n_q), (d - (kD - a.rope_dims)) >> 1, a.rope_dims, a.rope_base, &rs_,
+                    &rc_);
+    for (int hh = w; hh < kH; hh += 8) {
+        float v = s_acc[hh][lane];
+        if (rot) v = rope_apply(d, v, s_acc[hh][lane ^ 1], rs_, rc_);
+        a.out[((long long)row * kH + hh) * kD + d] = v;
+    }
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -710,6 +736,9 @@ cudaError_t launch_attend_tc(const AttendArgs& a, void* ws, size_t ws_bytes, cud
     t.tpr = p.tpr;
     t.grid = p.grid;
     t.scale_log2 = 1.4426950408889634f / sqrtf((float)kD);
+    t.sink = a.sink;
+    t.rope_dims = a.rope_dims;
+    t.rope_base = a.rope_base;
 
     const size_t smem = sizeof(Smem) + 1024;
     cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -125,4 +125,20 @@ __device__ __forceinline__ float group_sum(float v) {
 
 __host__ __device__ __forceinline__ long long n_visible(long long t, int m) { return (t + 1) / m; }
 
+// Output RoPE at minus the query position ("1M Context != Lossless Long Memory", section 8): the
+// pair k of the last R dims of a d-dim row turns by -t * base^(-2k/R).  sin/cos of that angle,
+// reduced and evaluated in double (t reaches 1M, the angle hundreds of thousands of radians).
+__device__ __forceinline__ void rope_sincos(long long t, int k, int rope_dims, float base, float* s, float* c) {
+    const double ang = -(double)t * pow((double)base, -2.0 * (double)k / (double)rope_dims);
+    const double r = remainder(ang, 6.283185307179586476925286766559);
+    double sd, cd;
+    sincos(r, &sd, &cd);
+    *s = (float)sd;
+    *c = (float)cd;
+}
+// the rotated value of output dim `dim` (in the RoPE part) from its value v and its pair partner p
+__device__ __forceinline__ float rope_apply(int dim, float v, float p, float s, float c) {
+    return (dim & 1) ? fmaf(p, s, v * c) : fmaf(v, c, -p * s);
+}
+
 }  // namespace v4a

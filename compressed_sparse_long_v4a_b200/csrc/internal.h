@@ -53,6 +53,9 @@ struct AttendArgs {
     int batch, n_q, heads, d, m, k, window;
     long long ctx_len, n_ent;
     int* dev_status;
+    const float* sink;  // [heads] sink logits, or null
+    int rope_dims;      // 0, or the output dims rotated at minus the query position
+    float rope_base;
 };
 
 size_t attend_workspace_bytes(const AttendArgs& a);

@@ -215,11 +215,23 @@ v4a_status v4a_topk(const void* q_i, const float* w, const void* k_i, const floa
 
 static v4a_status attend_common(const void* q, const void* entries, const int32_t* idx, const void* token_kv,
                                 long long tok_pos0, long long l_tok, float* out, v4a_dtype dtype, void* workspace,
-                                size_t workspace_bytes, int* dev_status, const v4a_shape* shape, void* stream,
-                                bool csa) {
+                                size_t workspace_bytes, int* dev_status, const v4a_attend_ext* ext,
+                                const v4a_shape* shape, void* stream, bool csa) {
     v4a::AttendArgs a;
     v4a_status st = attend_args(q, entries, idx, token_kv, tok_pos0, l_tok, out, dtype, dev_status, shape, csa, &a);
     if (st != V4A_OK) return st;
+    a.sink = nullptr;
+    a.rope_dims = 0;
+    a.rope_base = 10000.f;
+    if (ext) {
+        if (ext->rope_dims < 0 || ext->rope_dims > a.d || (ext->rope_dims & 1))
+            return fail(V4A_ERR_INVALID_ARG, "rope_dims must be even and in 0..d");
+        if (ext->rope_dims > 0 && !(ext->rope_base > 0.f)) return fail(V4A_ERR_INVALID_ARG, "rope_base must be > 0");
+        if (ext->sink && !aligned(ext->sink, 4)) return fail(V4A_ERR_INVALID_ARG, "sink must be 4-byte aligned");
+        a.sink = ext->sink;
+        a.rope_dims = ext->rope_dims;
+        a.rope_base = ext->rope_base;
+    }
     size_t need = v4a::attend_workspace_bytes(a);
     if (!workspace || workspace_bytes < need)
         return fail(V4A_ERR_INVALID_ARG, "workspace of %zu bytes needed, %zu given", need, workspace_bytes);
@@ -236,14 +248,29 @@ v4a_status v4a_csa_attend(const void* q, const void* entries, const int32_t* idx
                           long long tok_pos0, long long l_tok, float* out, v4a_dtype dtype, void* workspace,
                           size_t workspace_bytes, int* dev_status, const v4a_shape* shape, void* stream) {
     return attend_common(q, entries, idx, token_kv, tok_pos0, l_tok, out, dtype, workspace, workspace_bytes,
-                         dev_status, shape, stream, true);
+                         dev_status, nullptr, shape, stream, true);
+}
+
+v4a_status v4a_csa_attend_ex(const void* q, const void* entries, const int32_t* idx, const void* token_kv,
+                             long long tok_pos0, long long l_tok, float* out, v4a_dtype dtype, void* workspace,
+                             size_t workspace_bytes, int* dev_status, const v4a_attend_ext* ext,
+                             const v4a_shape* shape, void* stream) {
+    return attend_common(q, entries, idx, token_kv, tok_pos0, l_tok, out, dtype, workspace, workspace_bytes,
+                         dev_status, ext, shape, stream, true);
+}
+
+v4a_status v4a_hca_attend_ex(const void* q, const void* entries, const void* token_kv, long long tok_pos0,
+                             long long l_tok, float* out, v4a_dtype dtype, void* workspace, size_t workspace_bytes,
+                             const v4a_attend_ext* ext, const v4a_shape* shape, void* stream) {
+    return attend_common(q, entries, nullptr, token_kv, tok_pos0, l_tok, out, dtype, workspace, workspace_bytes,
+                         nullptr, ext, shape, stream, false);
 }
 
 v4a_status v4a_hca_attend(const void* q, const void* entries, const void* token_kv, long long tok_pos0,
                           long long l_tok, float* out, v4a_dtype dtype, void* workspace, size_t workspace_bytes,
                           const v4a_shape* shape, void* stream) {
     return attend_common(q, entries, nullptr, token_kv, tok_pos0, l_tok, out, dtype, workspace, workspace_bytes,
-                         nullptr, shape, stream, false);
+                         nullptr, nullptr, shape, stream, false);
 }
 
 size_t v4a_workspace_size(const char* op, const v4a_shape* shape, int heads_i, int d_i) {

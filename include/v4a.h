@@ -240,6 +240,30 @@ V4A_API v4a_status v4a_hca_attend(const void* q, const void* entries, const void
                           long long l_tok, float* out, v4a_dtype dtype, void* workspace, size_t workspace_bytes,
                           const v4a_shape* shape, void* stream);
 
+/* Options of the _ex attention calls ("1M Context != Lossless Long Memory",
+ * sections 7 and 8).  A zeroed struct (or a NULL pointer) means neither. */
+typedef struct v4a_attend_ext {
+    const float* sink;   /* [heads] fp32 per-head sink logits z'_h, or NULL: each head's softmax
+                            denominator gains e^{z'_h}, so its weights sum to less than 1 */
+    int rope_dims;       /* R: 0, or an even number <= d: the output's last R dims are rotated by
+                            RoPE at minus the query position t, pair k = dims (d-R+2k, d-R+2k+1)
+                            turning by -t * rope_base^(-2k/R) */
+    float rope_base;     /* RoPE frequency base (e.g. 10000); used when rope_dims > 0 */
+} v4a_attend_ext;
+
+/* v4a_csa_attend / v4a_hca_attend with the attention sink and the inverse
+ * output RoPE of v4a_attend_ext (ext may be NULL: then identical to the
+ * plain calls).  Errors as the plain calls, plus V4A_ERR_INVALID_ARG for an
+ * odd or too large rope_dims or a rope_base <= 0 with rope_dims > 0. */
+V4A_API v4a_status v4a_csa_attend_ex(const void* q, const void* entries, const int32_t* idx, const void* token_kv,
+                                     long long tok_pos0, long long l_tok, float* out, v4a_dtype dtype,
+                                     void* workspace, size_t workspace_bytes, int* dev_status,
+                                     const v4a_attend_ext* ext, const v4a_shape* shape, void* stream);
+V4A_API v4a_status v4a_hca_attend_ex(const void* q, const void* entries, const void* token_kv, long long tok_pos0,
+                                     long long l_tok, float* out, v4a_dtype dtype, void* workspace,
+                                     size_t workspace_bytes, const v4a_attend_ext* ext, const v4a_shape* shape,
+                                     void* stream);
+
 /* ------------------------------------------------------------------ */
 /* housekeeping                                                         */
 /* ------------------------------------------------------------------ */

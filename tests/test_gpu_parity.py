@@ -299,6 +299,34 @@ def test_hca_attend_matches_oracle(v4a, fmt, B, T, L, H, d, W):
     check_attention(out, ref, fmt == "f32", f"hca {fmt} L={L}")
 
 
+@pytest.mark.parametrize("kind,fmt,B,T,L,H,d,W", [
+    ("hca", "bf16", 2, 1, 128 * 40 + 77, 64, 512, 128),  # tensor cores, queries split between CTAs
+    ("hca", "bf16", 3, 1, 100, 64, 512, 64),             # tensor cores, one tile per query (written whole)
+    ("csa", "bf16", 2, 2, 4 * 2000 + 3, 64, 512, 128),   # tensor cores, CSA
+    ("hca", "f32", 2, 1, 128 * 30 + 5, 16, 128, 128),    # CUDA cores, several splits
+    ("csa", "f32", 1, 3, 4 * 200, 16, 128, 128),         # CUDA cores
+])
+def test_attend_sink_and_output_rope_match_oracle(v4a, kind, fmt, B, T, L, H, d, W):
+    """The attention sink (per-head logit in the softmax denominator) and the output RoPE at minus the
+    query position on the last 64 dims ("1M Context != Lossless Long Memory", sections 7 and 8)."""
+    m, k = (128, 0) if kind == "hca" else (4, 200)
+    a = _attend_inputs(B, T, L, m, H, d, W, fmt, seed=L + 7 * H, k=k if k else None, pad=0.1)
+    g = torch.Generator().manual_seed(L)
+    sink = (2.0 * torch.randn(H, generator=g)).float()
+    out = torch.empty((B, T, H, d), dtype=torch.float32, device="cuda")
+    ent = dev(a["entries"]) if a["entries"].shape[1] else None
+    if kind == "hca":
+        v4a.v4a_hca_attend(dev(a["q"]), ent, dev(a["token_kv"]), a["tok_pos0"], out, m=m, window=W, ctx_len=L,
+                           sink=sink.cuda(), rope_dims=64, rope_base=10000.0)
+    else:
+        v4a.v4a_csa_attend(dev(a["q"]), ent, dev(a["idx"]), dev(a["token_kv"]), a["tok_pos0"], out, m=m, window=W,
+                           ctx_len=L, sink=sink.cuda(), rope_dims=64, rope_base=10000.0)
+    _sync()
+    ref = oracle.attend(host(a["q"]), host(a["entries"]), host(a["idx"]) if kind == "csa" else None,
+                        host(a["token_kv"]), a["tok_pos0"], L, m, W, sink=sink.double().numpy(), rope_dims=64)
+    check_attention(out, ref, fmt == "f32", f"{kind} {fmt} L={L} with sink and output RoPE")
+
+
 def test_csa_with_every_entry_selected_equals_hca(v4a):
     B, T, L, m, H, d, W = 2, 1, 4 * 200, 4, 64, 512, 128
     a = _attend_inputs(B, T, L, m, H, d, W, "bf16", seed=9)
