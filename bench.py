@@ -243,6 +243,16 @@ class Step:
         self.compress_hca()
         self.hca_attend()
 
+    def hca_layer_sink_rope(self):
+        """The HCA layer with the attention sink and the output RoPE on the last 64 dims."""
+        h = self.hc
+        if not hasattr(self, "sink"):
+            self.sink = torch.linspace(-2.0, 2.0, h["heads"], dtype=torch.float32, device="cuda")
+        self.compress_hca()
+        self.v4a.v4a_hca_attend(self.h_q, self.h_ent, self.h_tok, self.h_pos0, self.h_out, m=h["m"],
+                                window=h["window"], ctx_len=self.Lh, workspace=self.ws_hca, sink=self.sink,
+                                rope_dims=64, rope_base=10000.0)
+
     # bytes ------------------------------------------------------------
     def algorithmic_bytes(self):
         """Bytes the method must read per step (indexer keys + scales, selected
@@ -279,6 +289,11 @@ class Prefill:
         self.keys[:, :self.n_hist] = w["hist_keys"].cuda()
         dv = lambda t: t.cuda()
         self.x, self.g, self.xi, self.gi = dv(w["x"]), dv(w["gate"]), dv(w["xi"]), dv(w["gate_i"])
+        # a second KV series for the dual-series compressor (series b, and its block before the chunk)
+        gb = wl._gen(c["seed"] + 1000)
+        self.xb = wl.store(wl.normal(gb, (1, self.T + self.m, d)), c["fmt"]).cuda()
+        self.gb = wl.store(wl.normal(gb, (1, self.T + self.m, d)), c["fmt"]).cuda()
+        self.ent_dual = torch.empty((1, self.T // self.m, d), dtype=torch.bfloat16, device="cuda")
         self.q, self.qi, self.w, self.tok = dv(w["q"]), dv(w["q_i"]), dv(w["w"]), dv(w["token_kv"])
         self.tok_pos0 = w["tok_pos0"]
         self.idx = torch.empty((1, self.T, self.k), dtype=torch.int32, device="cuda")
@@ -293,6 +308,11 @@ class Prefill:
     def compress(self):
         self.v4a.v4a_compress(self.x, self.g, self.ent[:, self.n_hist:], m=self.m, xi=self.xi, gate_i=self.gi,
                               out_i=self.keys[:, self.n_hist:])
+
+    def compress_dual(self):
+        m = self.m
+        self.v4a.v4a_compress_dual(self.x, self.g, self.xb[:, m:], self.gb[:, m:], self.ent_dual, m=m,
+                                   prev_x_b=self.xb[:, :m], prev_gate_b=self.gb[:, :m])
 
     def index_scores(self):
         self.v4a.v4a_index_scores(self.qi, self.w, self.keys, None, self.scores, m=self.m, ctx_len=self.L)
@@ -310,6 +330,10 @@ class Prefill:
         self.topk()
         self.attend()
 
+    def dual_bytes(self):
+        d = self.c["d"]
+        return 2 * (2 * self.T + 2 * (self.T + self.m)) * d + 2 * (self.T // self.m) * d  # bf16 reads + writes
+
     def flops(self):
         c = self.c
         nvis = sum((self.L - self.T + j + 1) // self.m for j in range(self.T))
@@ -324,7 +348,7 @@ def measure_prefill(peaks: dict) -> dict:
     torch.cuda.synchronize()
     reps = 10
     ms = {name: statistics.median(layer_times(getattr(p, name), reps))
-          for name in ("compress", "index_scores", "topk", "attend", "step")}
+          for name in ("compress", "compress_dual", "index_scores", "topk", "attend", "step")}
     idx_f, att_f = p.flops()
     sustained = float(peaks.get("bf16_tflops_sustained", 1390.0))
     burst = float(peaks.get("bf16_tflops", 1640.0))
@@ -335,6 +359,7 @@ def measure_prefill(peaks: dict) -> dict:
            "attention_tflops": att_f / (ms["attend"] / 1000.0) / 1e12,
            "step_tflops": (idx_f + att_f) / (ms["step"] / 1000.0) / 1e12,
            "flops": {"index_scores": idx_f, "attention": att_f},
+           "compress_dual_gbs": p.dual_bytes() / (ms["compress_dual"] / 1000.0) / 1e9,
            "peak_tflops_bf16": {"sustained": sustained, "burst": burst}}
     res["step_frac_sustained"] = res["step_tflops"] / sustained
     del p
@@ -580,6 +605,9 @@ def main():
                                    ("hca", step.hca_layer, step.Bh, ab["hca_attend"])):
         ts = layer_times(fn, lreps)
         med = statistics.median(ts)
+        if name == "hca":
+            layers["hca_with_sink_and_output_rope_ms_median"] = statistics.median(
+                layer_times(step.hca_layer_sink_rope, lreps))
         layers[name] = {"tokens_per_s_median": seqs / (med / 1000.0),
                         "tokens_per_s_p10": seqs / (pct(ts, 90) / 1000.0),
                         "tokens_per_s_p90": seqs / (pct(ts, 10) / 1000.0),
