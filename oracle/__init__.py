@@ -8,7 +8,8 @@ CUDA library and the CUDA library never touches it.
 
 Every function returns numpy arrays.  Inputs are numpy arrays (or anything
 ``numpy.ascontiguousarray`` accepts) holding the *stored* bytes: float32,
-bfloat16 as uint16 bit patterns, e4m3 as uint8 codes.
+bfloat16 as uint16 bit patterns, e4m3 as uint8 codes, binary64 values as
+float64 (the decoded operands of the MXFP4 indexer).
 """
 from __future__ import annotations
 
@@ -18,7 +19,7 @@ import subprocess
 
 import numpy as np
 
-F32, BF16, E4M3 = 0, 1, 2  # storage-format codes of the oracle's own C API
+F32, BF16, E4M3, F64 = 0, 1, 2, 3  # storage-format codes of the oracle's own C API
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "v4a_oracle.c")
@@ -48,6 +49,14 @@ def _load():
     lib.v4ao_e4m3_decode.argtypes = [ctypes.c_uint8]
     lib.v4ao_e4m3_encode.restype = ctypes.c_uint8
     lib.v4ao_e4m3_encode.argtypes = [dbl]
+    lib.v4ao_e2m1_decode.restype = dbl
+    lib.v4ao_e2m1_decode.argtypes = [ctypes.c_uint8]
+    lib.v4ao_e2m1_encode.restype = ctypes.c_uint8
+    lib.v4ao_e2m1_encode.argtypes = [dbl]
+    lib.v4ao_quantize_mxfp4.restype = i32
+    lib.v4ao_quantize_mxfp4.argtypes = [vp, ll, ll, vp, vp]
+    lib.v4ao_decode_mxfp4.restype = i32
+    lib.v4ao_decode_mxfp4.argtypes = [vp, vp, ll, ll, vp]
     lib.v4ao_set_threads.argtypes = [i32]
     lib.v4ao_get_threads.restype = i32
     lib.v4ao_n_visible.restype = ll
@@ -94,6 +103,8 @@ def fmt_of(a: np.ndarray) -> int:
         return BF16
     if a.dtype == np.uint8:
         return E4M3
+    if a.dtype == np.float64:
+        return F64
     raise TypeError(f"unsupported storage dtype {a.dtype}")
 
 
@@ -135,7 +146,7 @@ _tables: dict = {}
 def decode(a: np.ndarray) -> np.ndarray:
     """Stored bytes -> binary64 values, by the oracle's own decoders."""
     f = fmt_of(a)
-    if f == F32:
+    if f in (F32, F64):
         return a.astype(np.float64)
     if f not in _tables:
         fn = _load().v4ao_bf16_decode if f == BF16 else _load().v4ao_e4m3_decode
@@ -189,6 +200,63 @@ def quantize_e4m3_rows(values) -> tuple[np.ndarray, np.ndarray]:
     if st:
         raise ValueError(f"oracle quantize: status {st}")
     return codes, scales
+
+
+def e2m1_decode(codes) -> np.ndarray:
+    lib = _load()
+    c = np.asarray(codes, dtype=np.uint8)
+    return np.array([lib.v4ao_e2m1_decode(int(v)) for v in c.ravel()]).reshape(c.shape)
+
+
+def e2m1_encode(values) -> np.ndarray:
+    lib = _load()
+    v = np.asarray(values, dtype=np.float64)
+    return np.array([lib.v4ao_e2m1_encode(float(x)) for x in v.ravel()], dtype=np.uint8).reshape(v.shape)
+
+
+def quantize_mxfp4(values) -> tuple[np.ndarray, np.ndarray]:
+    """MXFP4 (OCP MX) quantisation along the last axis (a multiple of 32) of binary64 values:
+    returns (codes uint8 [..][cols/2], two e2m1 codes per byte with the even element in the low
+    nibble; exps uint8 [..][cols/32], the E8M0 block exponents X + 127)."""
+    v = _c(values, np.float64)
+    cols = v.shape[-1]
+    rows = int(np.prod(v.shape[:-1]))
+    codes = np.zeros(v.shape[:-1] + (cols // 2,), dtype=np.uint8)
+    exps = np.zeros(v.shape[:-1] + (cols // 32,), dtype=np.uint8)
+    st = _load().v4ao_quantize_mxfp4(_ptr(v), rows, cols, _ptr(codes), _ptr(exps))
+    if st:
+        raise ValueError(f"oracle quantize_mxfp4: status {st}")
+    return codes, exps
+
+
+def decode_mxfp4(codes, exps) -> np.ndarray:
+    """MXFP4 codes [..][cols/2] and block exponents [..][cols/32] -> binary64 values [..][cols]."""
+    c, x = _c(codes, np.uint8), _c(exps, np.uint8)
+    cols = c.shape[-1] * 2
+    assert x.shape == c.shape[:-1] + (cols // 32,)
+    rows = int(np.prod(c.shape[:-1]))
+    out = np.zeros(c.shape[:-1] + (cols,), dtype=np.float64)
+    st = _load().v4ao_decode_mxfp4(_ptr(c), _ptr(x), rows, cols, _ptr(out))
+    if st:
+        raise ValueError(f"oracle decode_mxfp4: status {st}")
+    return out
+
+
+def mxfp4_query(q_i) -> np.ndarray:
+    """The indexer query as the FP4 dot product sees it: every head's d_I values (stored bytes)
+    quantised to MXFP4 and decoded back, as binary64."""
+    return decode_mxfp4(*quantize_mxfp4(decode(_c(q_i))))
+
+
+def index_scores_mxfp4(q_i, w, k_codes, k_exps, ctx_len: int, m: int) -> np.ndarray:
+    """Indexer scores with MXFP4 keys (codes [B][N][d_I/2], exps [B][N][d_I/32]) and the query
+    quantised to MXFP4 per head: the score definition on the decoded values of both operands."""
+    return index_scores(mxfp4_query(q_i), w, decode_mxfp4(k_codes, k_exps), None, ctx_len, m)
+
+
+def topk_mxfp4(q_i, w, k_codes, k_exps, ctx_len: int, m: int, k: int, want_scores: bool = False):
+    """Indexer + top-k with MXFP4 keys and queries (see index_scores_mxfp4)."""
+    return topk(mxfp4_query(q_i), w, decode_mxfp4(k_codes, k_exps), None, ctx_len, m, k, want_scores)
 
 
 def index_scores(q_i, w, k_i, k_scale, ctx_len: int, m: int) -> np.ndarray:

@@ -47,6 +47,20 @@
  *    must not read its own, still incomplete, compressed block).
  *  - Window: tokens (t-W, t] clipped at 0 ("1M Context != ...", section 6.1,
  *    n_win = 128).  The window may overlap visible entries; both are kept.
+ *  - FP4 indexer keys ("1M Context != Lossless Long Memory", section 4.2 and
+ *    footnote 3: indexer KV in FP4, FP4 dot products; "DeepSeek-V4 ...",
+ *    "Where It Breaks": FP4 QK indexer).  The pages name no bit format; the
+ *    oracle reads it as the OCP Microscaling (MX v1.0) MXFP4 format: e2m1
+ *    elements (1 sign, 2 exponent bits with bias 1, 1 fraction bit; values
+ *    0, 0.5, 1, 1.5, 2, 3, 4, 6) in blocks of 32 sharing one power-of-two
+ *    scale 2^X stored as an E8M0 byte X + 127.  A block is quantised with
+ *    X = max(floor(log2(amax)) - 2, -127) (2 = the largest e2m1 exponent;
+ *    X = -127 for an all-zero block) and element codes = nearest e2m1 of
+ *    v / 2^X (ties to the even code, magnitudes above 6 clamp to 6, the sign
+ *    kept even when the value rounds to zero).  "FP4 QK" is read as both
+ *    operands in MXFP4: the query of each indexer head is quantised the same
+ *    way (blocks of 32 along d_I), and the score is the definition above
+ *    evaluated on the decoded values.
  */
 #include <math.h>
 #include <pthread.h>
@@ -58,6 +72,7 @@
 #define OR_F32 0
 #define OR_BF16 1
 #define OR_E4M3 2
+#define OR_F64 3 /* binary64 values (decoded MXFP4 operands) */
 
 #define OR_OK 0
 #define OR_ERR_ARG 1
@@ -143,12 +158,47 @@ uint16_t v4ao_bf16_encode(double v)
     return sign | (uint16_t)((u >> 16) & 0x7fff);
 }
 
+/* e2m1 (4 bits: sign, 2 exponent bits with bias 1, 1 fraction bit; no
+ * infinities or NaN): exponent field 0 is subnormal, 0.f * 2^0. */
+double v4ao_e2m1_decode(uint8_t c)
+{
+    int s = (c >> 3) & 1;
+    int e = (c >> 1) & 3;
+    int f = c & 1;
+    double v = e == 0 ? 0.5 * f : ldexp(1.0 + 0.5 * f, e - 1);
+    return s ? -v : v;
+}
+
+/* Nearest e2m1 code of v (ties to the code with an even fraction bit),
+ * magnitudes above 6 clamp to 6; the sign bit is the sign of v, also when
+ * the magnitude rounds to 0.  Found by searching the 8 non-negative codes,
+ * whose values increase with the code. */
+uint8_t v4ao_e2m1_encode(double v)
+{
+    uint8_t sign = signbit(v) ? 0x8 : 0x0;
+    double a = fabs(v);
+    if (a >= 6.0) return sign | 0x7;
+    int lo = 0;                                        /* largest code with value <= a */
+    for (int c = 0; c <= 7; ++c) {
+        if (v4ao_e2m1_decode((uint8_t)c) <= a) lo = c; else break;
+    }
+    int hi = lo < 7 ? lo + 1 : lo;
+    double dl = a - v4ao_e2m1_decode((uint8_t)lo);
+    double dh = v4ao_e2m1_decode((uint8_t)hi) - a;
+    int pick;
+    if (dl < dh) pick = lo;
+    else if (dh < dl) pick = hi;
+    else pick = (lo & 1) ? hi : lo;
+    return sign | (uint8_t)pick;
+}
+
 static double load_elem(const void* p, int dt, size_t i)
 {
     switch (dt) {
     case OR_F32: return (double)((const float*)p)[i];
     case OR_BF16: return v4ao_bf16_decode(((const uint16_t*)p)[i]);
     case OR_E4M3: return v4ao_e4m3_decode(((const uint8_t*)p)[i]);
+    case OR_F64: return ((const double*)p)[i];
     default: return NAN;
     }
 }
@@ -342,6 +392,54 @@ int v4ao_quantize_e4m3_rows(const double* v, long long rows, long long cols, uin
     return OR_OK;
 }
 
+/* MXFP4 quantisation (OCP MX v1.0) of rows of binary64 values, cols a
+ * multiple of 32: per block of 32, X = max(floor(log2(amax)) - 2, -127)
+ * (-127 for an all-zero block), exps[block] = X + 127, element i's code =
+ * nearest e2m1 of v_i / 2^X, two codes per byte (element 2i in the low
+ * nibble of byte i). */
+int v4ao_quantize_mxfp4(const double* v, long long rows, long long cols, uint8_t* codes, uint8_t* exps)
+{
+    if (!v || !codes || !exps || rows < 0 || cols < 32 || cols % 32) return OR_ERR_ARG;
+    for (long long r = 0; r < rows; ++r) {
+        for (long long b = 0; b < cols / 32; ++b) {
+            const double* x = v + r * cols + b * 32;
+            double amax = 0.0;
+            for (int i = 0; i < 32; ++i)
+                if (fabs(x[i]) > amax) amax = fabs(x[i]);
+            int X = -127;
+            if (amax > 0.0) {
+                int e;
+                frexp(amax, &e);                       /* amax = f * 2^e, f in [0.5, 1) */
+                X = (e - 1) - 2;                       /* floor(log2(amax)) - 2 */
+                if (X < -127) X = -127;
+                if (X > 127) return OR_ERR_ARG;
+            }
+            exps[r * (cols / 32) + b] = (uint8_t)(X + 127);
+            uint8_t* out = codes + r * (cols / 2) + b * 16;
+            for (int i = 0; i < 32; i += 2) {
+                uint8_t lo = v4ao_e2m1_encode(ldexp(x[i], -X));
+                uint8_t hi = v4ao_e2m1_encode(ldexp(x[i + 1], -X));
+                out[i / 2] = (uint8_t)(lo | (hi << 4));
+            }
+        }
+    }
+    return OR_OK;
+}
+
+/* MXFP4 rows -> binary64 values: element = e2m1 value * 2^(exp - 127). */
+int v4ao_decode_mxfp4(const uint8_t* codes, const uint8_t* exps, long long rows, long long cols, double* out)
+{
+    if (!codes || !exps || !out || rows < 0 || cols < 32 || cols % 32) return OR_ERR_ARG;
+    for (long long r = 0; r < rows; ++r)
+        for (long long i = 0; i < cols; ++i) {
+            uint8_t byte = codes[r * (cols / 2) + i / 2];
+            uint8_t c = (i & 1) ? (byte >> 4) : (byte & 0xf);
+            uint8_t xb = exps[r * (cols / 32) + i / 32];
+            out[r * cols + i] = xb == 0xff ? NAN : ldexp(v4ao_e2m1_decode(c), (int)xb - 127);  /* 0xff: NaN */
+        }
+    return OR_OK;
+}
+
 /* ------------------------------------------------------------------ */
 /* Lightning-Indexer scores                                            */
 /* ------------------------------------------------------------------ */
@@ -399,8 +497,8 @@ int v4ao_index_scores(const void* q, int q_dt, const float* w, const void* key, 
 {
     if (!q || !w || !key || !scores || batch < 0 || n_q < 1 || m < 1 || heads_i < 1 || d_i < 1) return OR_ERR_ARG;
     if (n_q > ctx_len) return OR_ERR_ARG;
-    if (q_dt != OR_F32 && q_dt != OR_BF16) return OR_ERR_ARG;
-    if (k_dt != OR_F32 && k_dt != OR_BF16 && k_dt != OR_E4M3) return OR_ERR_ARG;
+    if (q_dt != OR_F32 && q_dt != OR_BF16 && q_dt != OR_F64) return OR_ERR_ARG;
+    if (k_dt != OR_F32 && k_dt != OR_BF16 && k_dt != OR_E4M3 && k_dt != OR_F64) return OR_ERR_ARG;
     index_ctx k = {q, q_dt, w, key, k_dt, scale, n_q, ctx_len, m, heads_i, d_i, ctx_len / m, scores};
     parallel_for(batch * n_q, index_item, &k);
     return OR_OK;

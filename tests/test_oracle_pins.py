@@ -207,6 +207,128 @@ def test_quantize_rows_bounds():
 
 
 # ----------------------------------------------------------------------
+# MXFP4 (OCP MX: e2m1 elements, blocks of 32 sharing an E8M0 power of two)
+# ----------------------------------------------------------------------
+
+def _lib_e2m1_codes(vals):
+    import ml_dtypes
+    return np.asarray(vals, dtype=np.float32).astype(ml_dtypes.float4_e2m1fn).view(np.uint8) & 0xF
+
+
+def test_e2m1_decode_all_codes_match_library():
+    import ml_dtypes
+    codes = np.arange(16, dtype=np.uint8)
+    lib = codes.view(ml_dtypes.float4_e2m1fn).astype(np.float64)
+    ours = oracle.e2m1_decode(codes)
+    assert np.array_equal(ours, lib) and np.array_equal(np.signbit(ours), np.signbit(lib))
+    assert sorted(set(np.abs(ours))) == [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+
+
+def test_e2m1_encode_matches_library_rne_and_saturates():
+    grid = oracle.e2m1_decode(np.arange(8, dtype=np.uint8))
+    mids = (grid[:-1] + grid[1:]) / 2  # ties: 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5
+    rng = np.random.default_rng(40)
+    vals = np.concatenate([grid, mids, mids * (1 + 2.0 ** -20), mids * (1 - 2.0 ** -20),
+                           rng.uniform(-7, 7, 4000), [6.5, 7.99, 8.0, 100.0, 1e30, 1e-9, 0.0]])
+    vals = np.concatenate([vals, -vals]).astype(np.float32)
+    assert np.array_equal(oracle.e2m1_encode(vals.astype(np.float64)), _lib_e2m1_codes(vals))
+    assert oracle.e2m1_encode([-1e-9])[0] == 0x8  # the sign survives a round to zero
+
+
+def test_mxfp4_block_exponent_rule():
+    rng = np.random.default_rng(41)
+    v = rng.normal(size=(64, 128)) * np.exp2(rng.integers(-20, 20, size=(64, 1)))
+    v[5, 32:64] = 0.0                       # an all-zero block
+    v[6, :32] = rng.normal(size=32) * 2.0 ** -140  # below the smallest scale
+    codes, exps = oracle.quantize_mxfp4(v)
+    assert codes.shape == (64, 64) and exps.shape == (64, 4)
+    X = exps.astype(np.int64) - 127
+    amax = np.abs(v).reshape(64, 4, 32).max(axis=2)
+    normal = (amax > 0) & (X > -127)
+    # the block maximum lands in [4, 8) times the block scale: 2^(X+2) <= amax < 2^(X+3)
+    assert np.all(np.exp2(X[normal] + 2.0) <= amax[normal]) and np.all(amax[normal] < np.exp2(X[normal] + 3.0))
+    assert exps[5, 1] == 0 and np.all(codes[5, 16:32] == 0)
+    assert exps[6, 0] == 0  # clamped at X = -127
+
+
+def test_mxfp4_codes_are_the_library_cast_at_the_block_scale():
+    rng = np.random.default_rng(42)
+    v = rng.normal(size=(40, 64)) * np.exp2(rng.integers(-6, 6, size=(40, 1)))
+    codes, exps = oracle.quantize_mxfp4(v)
+    X = (exps.astype(np.int64) - 127).repeat(32, axis=1)
+    scaled = np.ldexp(v, -X)                 # exact: a power of two
+    nib = np.stack([codes & 0xF, codes >> 4], axis=-1).reshape(v.shape)
+    assert np.array_equal(nib, _lib_e2m1_codes(scaled.astype(np.float32)))
+    deq = oracle.decode_mxfp4(codes, exps)
+    # nearest-code error: at most half the widest step (2 between 4 and 6), i.e. 2^X, below
+    # saturation; above 6 * 2^X the value clamps to 6 * 2^X
+    sat = np.abs(v) > 6 * np.exp2(X)
+    assert np.all(np.abs(deq - v)[~sat] <= np.exp2(X)[~sat])
+    assert np.array_equal(np.abs(deq[sat]), 6 * np.exp2(X[sat]))
+
+
+def test_mxfp4_roundtrip_on_the_grid():
+    rng = np.random.default_rng(43)
+    codes = rng.integers(0, 256, size=(16, 64), dtype=np.uint8)
+    # each block needs a code of magnitude 4 or 6 so that its own exponent is reproduced
+    codes[:, ::16] = (codes[:, ::16] & 0xF0) | rng.choice(np.array([0x6, 0x7, 0xE, 0xF], dtype=np.uint8), size=(16, 4))
+    exps = rng.integers(100, 150, size=(16, 4), dtype=np.uint8)
+    v = oracle.decode_mxfp4(codes, exps)
+    c2, x2 = oracle.quantize_mxfp4(v)
+    assert np.array_equal(x2, exps)
+    # equal values: only a signed zero may come back with the other sign
+    assert np.array_equal(oracle.decode_mxfp4(c2, x2), v)
+    same = (c2 == codes) | (((c2 ^ codes) & 0x77) == 0)
+    assert same.all()
+
+
+def _on_grid(rng, shape):
+    """Values on the MXFP4 grid: each 32-block holds e2m1 values times 2^X with a 4 or 6 in it."""
+    rows = int(np.prod(shape[:-1]))
+    codes = rng.integers(0, 256, size=(rows, shape[-1] // 2), dtype=np.uint8)
+    codes[:, ::16] = (codes[:, ::16] & 0xF0) | 0x7
+    exps = rng.integers(120, 130, size=(rows, shape[-1] // 32), dtype=np.uint8)
+    return oracle.decode_mxfp4(codes, exps).reshape(shape), codes.reshape(shape[:-1] + (-1,)), \
+        exps.reshape(shape[:-1] + (-1,))
+
+
+def test_mxfp4_scores_on_the_grid_equal_the_f32_scores():
+    """Quantising values that are already on the MXFP4 grid changes nothing, so the FP4 score of
+    such operands is the (pinned) f32 score of the same values."""
+    rng = np.random.default_rng(44)
+    B, T, L, m, HI, DI = 2, 3, 256, 4, 4, 64
+    q, _, _ = _on_grid(rng, (B, T, HI, DI))
+    k, kc, kx = _on_grid(rng, (B, L // m, DI))
+    w = rng.uniform(size=(B, T, HI)).astype(np.float32)
+    s4 = oracle.index_scores_mxfp4(q.astype(np.float32), w, kc, kx, ctx_len=L, m=m)
+    s32 = oracle.index_scores(q.astype(np.float32), w, k.astype(np.float32), None, ctx_len=L, m=m)
+    assert np.array_equal(s4, s32)
+
+
+def test_mxfp4_scores_scale_with_powers_of_two_and_quantise_q_per_head():
+    rng = np.random.default_rng(45)
+    B, T, L, m, HI, DI = 1, 2, 512, 4, 3, 64
+    q = rng.normal(size=(B, T, HI, DI)).astype(np.float32)
+    w = rng.uniform(size=(B, T, HI)).astype(np.float32)
+    kc, kx = oracle.quantize_mxfp4(rng.normal(size=(B, L // m, DI)))
+    s = oracle.index_scores_mxfp4(q, w, kc, kx, ctx_len=L, m=m)
+    # keys times 2^5: every block exponent + 5, every score times 32, exactly
+    assert np.array_equal(oracle.index_scores_mxfp4(q, w, kc, kx + 5, ctx_len=L, m=m), 32 * s)
+    # the query quantiser commutes with powers of two
+    assert np.array_equal(oracle.index_scores_mxfp4(q * np.float32(0.125), w, kc, kx, ctx_len=L, m=m), s / 8)
+    # each head's query is quantised on its own: a large value in head 2 leaves heads 0 and 1 alone
+    q2 = q.copy()
+    q2[:, :, 2, 0] = 1e6
+    w01 = w.copy()
+    w01[:, :, 2] = 0
+    assert np.array_equal(oracle.index_scores_mxfp4(q2, w01, kc, kx, ctx_len=L, m=m),
+                          oracle.index_scores_mxfp4(q, w01, kc, kx, ctx_len=L, m=m))
+    # ... while the dequantised query of that head shows the block scale of its own block only
+    qd = oracle.mxfp4_query(q2)
+    assert np.array_equal(qd[:, :, 2, 32:], oracle.mxfp4_query(q)[:, :, 2, 32:])
+
+
+# ----------------------------------------------------------------------
 # visibility and counts
 # ----------------------------------------------------------------------
 
