@@ -367,6 +367,52 @@ def measure_prefill(peaks: dict) -> dict:
     return res
 
 
+def measure_fp4_indexer(step: "Step", flush: torch.Tensor, peak_gbs: float) -> dict:
+    """The 1M-context CSA indexer with MXFP4 keys (FP4 dot products): the same 4 sequences x
+    262,144 entries x 16 heads x 128, top-1024, with the keys drawn N(0,1) on the device (seeded)
+    and quantised by the library.  The keys (68 B per entry, 71 MB) fit in the 126 MB L2, so every
+    timing flushes L2 first (time_op)."""
+    v4a, c = step.v4a, step.cc
+    B, N, DI = step.Bc, step.Nc, c["d_i"]
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(c["seed"] + 4)
+    master = torch.randn((B, N, DI), generator=gen, device="cuda", dtype=torch.float32).to(torch.bfloat16)
+    kc = torch.empty((B, N, DI // 2), dtype=torch.uint8, device="cuda")
+    kx = torch.empty((B, N, DI // 32), dtype=torch.uint8, device="cuda")
+    v4a.v4a_quantize_mxfp4(master, kc, kx)
+    del master
+    scores = torch.empty((B, 1, N), dtype=torch.float32, device="cuda")
+    idx = torch.empty((B, 1, c["k"]), dtype=torch.int32, device="cuda")
+
+    def scores_fp4():
+        v4a.v4a_index_scores_mxfp4(step.c_qi, step.c_w, kc, kx, scores, m=c["m"], ctx_len=step.Lc)
+
+    def topk_fp4():
+        v4a.v4a_topk_mxfp4(step.c_qi, step.c_w, kc, kx, idx, m=c["m"], k=c["k"], ctx_len=step.Lc,
+                           workspace=step.ws_topk)
+
+    def scores_fp8():
+        v4a.v4a_index_scores(step.c_qi, step.c_w, step.c_ki, step.c_ks, scores, m=c["m"], ctx_len=step.Lc)
+
+    for fn in (scores_fp4, topk_fp4, scores_fp8):
+        fn()
+    torch.cuda.synchronize()
+    reps = 20
+    ms = {"index_scores_mxfp4": time_op(scores_fp4, reps, flush), "topk_mxfp4": time_op(topk_fp4, reps, flush),
+          "index_scores_fp8": time_op(scores_fp8, reps, flush), "topk_fp8": time_op(step.topk, reps, flush)}
+    key_bytes = B * N * (DI // 2 + DI // 32)
+    out = {"workload": "CSA decode indexer at 1M context: 4 x 262,144 MXFP4 keys (e2m1 codes, 32-element "
+                       "blocks with E8M0 exponents; N(0,1) before quantisation), query quantised to MXFP4 per "
+                       "head, 16 heads x 128, top-1024",
+           "ms": ms, "replays": reps, "l2": "flushed before each timed call",
+           "key_bytes": key_bytes, "key_bytes_per_entry": DI // 2 + DI // 32,
+           "index_scores_gbs": key_bytes / (ms["index_scores_mxfp4"] / 1000.0) / 1e9}
+    out["index_scores_frac_measured_peak"] = out["index_scores_gbs"] / peak_gbs
+    out["topk_speedup_vs_fp8"] = ms["topk_fp8"] / ms["topk_mxfp4"] if ms["topk_mxfp4"] > 0 else None
+    del kc, kx, scores, idx
+    return out
+
+
 def kernel_nodes(graph) -> int | None:
     """Kernel nodes in a captured graph (cuGraphGetNodes + cuGraphNodeGetType of
     the driver API; the graph must have been made with keep_graph=True)."""
@@ -656,7 +702,9 @@ def main():
 
     cpu = None
     prefill = None
+    fp4 = None
     if rank == 0 and world == 1:
+        fp4 = measure_fp4_indexer(step, flush, peak)
         prefill = measure_prefill(peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, threads, sample, _ = oracle_sample(args.cpu_seconds, step)
@@ -675,7 +723,7 @@ def main():
                            "step_hbm_gbs": total_bytes / (ms / 1000.0) / 1e9 / world,
                            "op_ms": op_ms,
                            "layers": layers},
-                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "prefill": prefill,
+                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "prefill": prefill, "fp4_indexer": fp4,
                 "gpu_launches": (launches_per_step * args.steps) if launches_per_step else None,
                 "gpu_launches_per_step": launches_per_step,
                 "clocks": clocks}

@@ -15,12 +15,13 @@ import os
 import torch
 
 __all__ = [
-    "V4AError", "F32", "BF16", "FP8E4M3", "lib", "library_path",
-    "v4a_compress", "v4a_index_scores", "v4a_topk", "v4a_topk_noalloc", "v4a_csa_attend", "v4a_hca_attend",
+    "V4AError", "F32", "BF16", "FP8E4M3", "MXFP4", "lib", "library_path",
+    "v4a_compress", "v4a_compress_dual", "v4a_quantize_mxfp4", "v4a_index_scores", "v4a_index_scores_mxfp4",
+    "v4a_topk", "v4a_topk_mxfp4", "v4a_topk_noalloc", "v4a_csa_attend", "v4a_hca_attend",
     "v4a_workspace_size", "v4a_status_string", "v4a_version", "n_entries", "window_rows",
 ]
 
-F32, BF16, FP8E4M3 = 0, 1, 2
+F32, BF16, FP8E4M3, MXFP4 = 0, 1, 2, 3
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libv4a.so")
 
@@ -41,7 +42,8 @@ class CompressIO(ctypes.Structure):
                 ("out_scale", ctypes.c_void_p), ("channels", ctypes.c_int), ("in_dtype", ctypes.c_int),
                 ("out_dtype", ctypes.c_int), ("x_batch_stride", ctypes.c_longlong),
                 ("gate_batch_stride", ctypes.c_longlong), ("out_batch_stride", ctypes.c_longlong),
-                ("scale_batch_stride", ctypes.c_longlong)]
+                ("scale_batch_stride", ctypes.c_longlong), ("out_exp", ctypes.c_void_p),
+                ("exp_batch_stride", ctypes.c_longlong)]
 
 
 class SeriesB(ctypes.Structure):
@@ -77,6 +79,12 @@ def _load():
     L.v4a_index_scores.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, P(Shape), vp]
     L.v4a_topk.restype = i32
     L.v4a_topk.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, sz, P(Shape), vp]
+    L.v4a_quantize_mxfp4.restype = i32
+    L.v4a_quantize_mxfp4.argtypes = [vp, i32, ll, i32, vp, vp, vp]
+    L.v4a_index_scores_mxfp4.restype = i32
+    L.v4a_index_scores_mxfp4.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, P(Shape), vp]
+    L.v4a_topk_mxfp4.restype = i32
+    L.v4a_topk_mxfp4.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, vp, sz, P(Shape), vp]
     L.v4a_topk_noalloc.restype = i32
     L.v4a_topk_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, P(Shape), vp]
     L.v4a_csa_attend.restype = i32
@@ -163,7 +171,9 @@ def _workspace(nbytes: int, device) -> torch.Tensor:
     return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
 
 
-def _io(x, gate, out, out_scale) -> CompressIO:
+def _io(x, gate, out, out_scale, out_exp=None) -> CompressIO:
+    """One compress stream.  out_exp given: MXFP4 output, out holding [batch][entries][channels/2]
+    code bytes and out_exp [batch][entries][channels/32] block exponents."""
     for t, name in ((x, "x"), (gate, "gate"), (out, "out")):
         if t.dim() != 3 or t.stride(2) != 1 or t.stride(1) != t.shape[2]:
             raise ValueError(f"{name} must be [batch][rows][channels] with dense rows")
@@ -172,21 +182,31 @@ def _io(x, gate, out, out_scale) -> CompressIO:
         if out_scale.dim() != 2 or out_scale.stride(1) != 1:
             raise ValueError("out_scale must be [batch][entries] with dense rows")
         sc_stride = out_scale.stride(0)
-    return CompressIO(_ptr(x), _ptr(gate), _ptr(out), _ptr(out_scale), int(x.shape[2]), _dtype(x), _dtype(out),
-                      x.stride(0), gate.stride(0), out.stride(0), sc_stride)
+    if out_exp is None:
+        return CompressIO(_ptr(x), _ptr(gate), _ptr(out), _ptr(out_scale), int(x.shape[2]), _dtype(x), _dtype(out),
+                          x.stride(0), gate.stride(0), out.stride(0), sc_stride, None, 0)
+    if out.dtype != torch.uint8 or out.shape[2] * 2 != x.shape[2]:
+        raise ValueError("MXFP4 out must be uint8 [batch][entries][channels/2]")
+    if out_exp.dtype != torch.uint8 or out_exp.dim() != 3 or out_exp.stride(2) != 1 or \
+            out_exp.stride(1) != out_exp.shape[2] or out_exp.shape[2] * 32 != x.shape[2]:
+        raise ValueError("out_exp must be uint8 [batch][entries][channels/32] with dense rows")
+    return CompressIO(_ptr(x), _ptr(gate), _ptr(out), None, int(x.shape[2]), _dtype(x), MXFP4, x.stride(0),
+                      gate.stride(0), 2 * out.stride(0), 0, _ptr(out_exp), out_exp.stride(0))
 
 
 def v4a_compress(x, gate, out, *, m: int, n_tok: int | None = None, out_scale=None, xi=None, gate_i=None,
-                 out_i=None, out_i_scale=None, stream=None) -> None:
+                 out_i=None, out_i_scale=None, out_i_exp=None, stream=None) -> None:
     """Compress complete m-token chunks of x (gated by `gate`) into `out`;
     optionally the indexer-key stream (xi, gate_i -> out_i [, out_i_scale]) in
-    the same launch.  Tensors are [batch][rows][channels] (views into larger
-    buffers are fine: the batch stride is read off the tensor)."""
+    the same launch; out_i_exp given: the indexer keys are written as MXFP4
+    (codes in out_i, block exponents in out_i_exp).  Tensors are
+    [batch][rows][channels] (views into larger buffers are fine: the batch
+    stride is read off the tensor)."""
     n = x.shape[1] if n_tok is None else int(n_tok)
     kv = _io(x, gate, out, out_scale)
     idx = None
     if xi is not None:
-        idx = _io(xi, gate_i, out_i, out_i_scale)
+        idx = _io(xi, gate_i, out_i, out_i_scale, out_i_exp)
     _check(lib.v4a_compress(ctypes.byref(kv), ctypes.byref(idx) if idx is not None else None, int(x.shape[0]), n,
                             int(m), _stream(stream)))
 
@@ -206,6 +226,45 @@ def v4a_compress_dual(x_a, gate_a, x_b, gate_b, out, *, m: int, prev_x_b=None, p
         raise ValueError("prev_x_b and prev_gate_b must have the same batch stride")
     b = SeriesB(_ptr(x_b), _ptr(gate_b), _ptr(prev_x_b), _ptr(prev_gate_b), x_b.stride(0), gate_b.stride(0), prev_bs)
     _check(lib.v4a_compress_dual(ctypes.byref(a), ctypes.byref(b), int(x_a.shape[0]), n, int(m), _stream(stream)))
+
+
+def v4a_quantize_mxfp4(x, codes, exps, stream=None) -> None:
+    """MXFP4 quantisation of x [..][cols] (fp32 or bf16, cols a multiple of 32) into codes
+    [..][cols/2] and exps [..][cols/32] (uint8)."""
+    for t, n in ((x, "x"), (codes, "codes"), (exps, "exps")):
+        _contig(t, n)
+    cols = int(x.shape[-1])
+    rows = x.numel() // cols if cols else 0
+    if codes.dtype != torch.uint8 or exps.dtype != torch.uint8 or codes.numel() * 2 != x.numel() or \
+            exps.numel() * 32 != x.numel():
+        raise ValueError("codes / exps must be uint8 with numel x/2 and x/32")
+    _check(lib.v4a_quantize_mxfp4(_ptr(x), _dtype(x), rows, cols, _ptr(codes), _ptr(exps), _stream(stream)))
+
+
+def v4a_index_scores_mxfp4(q_i, w, k_codes, k_exp, scores, *, m: int, ctx_len: int, stream=None) -> None:
+    """Indexer scores with MXFP4 keys (k_codes [B][N][d_i/2], k_exp [B][N][d_i/32]) and the query
+    quantised to MXFP4 per head inside the call."""
+    for t, n in ((q_i, "q_i"), (w, "w"), (k_codes, "k_codes"), (k_exp, "k_exp"), (scores, "scores")):
+        _contig(t, n)
+    B, T, HI, DI = q_i.shape
+    s = _shape(batch=B, n_q=T, m=m, ctx_len=ctx_len)
+    _check(lib.v4a_index_scores_mxfp4(_ptr(q_i), _ptr(w), _ptr(k_codes), _ptr(k_exp), _ptr(scores), HI, DI,
+                                      _dtype(q_i), ctypes.byref(s), _stream(stream)))
+
+
+def v4a_topk_mxfp4(q_i, w, k_codes, k_exp, idx_out, score_out=None, *, m: int, k: int, ctx_len: int,
+                   workspace=None, stream=None) -> None:
+    """Indexer + top-k with MXFP4 keys and FP4 dot products (see v4a_index_scores_mxfp4)."""
+    for t, n in ((q_i, "q_i"), (w, "w"), (k_codes, "k_codes"), (k_exp, "k_exp"), (idx_out, "idx_out"),
+                 (score_out, "score_out")):
+        _contig(t, n)
+    B, T, HI, DI = q_i.shape
+    s = _shape(batch=B, n_q=T, m=m, k=k, ctx_len=ctx_len)
+    if workspace is None:
+        workspace = _workspace(lib.v4a_workspace_size(b"topk", ctypes.byref(s), HI, DI), q_i.device)
+    _check(lib.v4a_topk_mxfp4(_ptr(q_i), _ptr(w), _ptr(k_codes), _ptr(k_exp), _ptr(idx_out), _ptr(score_out), HI, DI,
+                              _dtype(q_i), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                              ctypes.byref(s), _stream(stream)))
 
 
 def v4a_index_scores(q_i, w, k_i, k_scale, scores, *, m: int, ctx_len: int, stream=None) -> None:

@@ -93,6 +93,58 @@ __device__ __forceinline__ uint16_t pack_e4m3x2(float a, float b) {
 }
 
 // ---------------------------------------------------------------------
+// MXFP4 (OCP Microscaling v1.0): e2m1 codes, blocks of 32 sharing 2^X, X
+// stored as the E8M0 byte X + 127
+// ---------------------------------------------------------------------
+
+// X = max(floor(log2(amax)) - 2, -127) for a block with largest magnitude amax (-127 if amax is 0
+// or below the normal range); read off the binary32 exponent field, so exact
+__device__ __forceinline__ int mx_block_exp(float amax) {
+    const int ef = (int)((__float_as_uint(amax) >> 23) & 0xff);  // amax >= 0
+    const int x = ef - 127 - 2;
+    return (ef == 0 || x < -127) ? -127 : x;
+}
+// 2^k for k in [-126, 127] as a binary32 bit pattern (exact)
+__device__ __forceinline__ float pow2i(int k) { return __uint_as_float((uint32_t)(k + 127) << 23); }
+// 2^(e - 127) for an E8M0 byte e (e = 0 is the subnormal 2^-127; 255, NaN in the format, is not
+// produced by the quantiser and gives +inf here)
+__device__ __forceinline__ float e8m0_value(uint32_t e) { return e ? __uint_as_float(e << 23) : 0x1p-127f; }
+// nearest e2m1 code of x (ties to the even code, |x| > 6 clamps to 6, the sign kept even when the
+// magnitude rounds to 0): the magnitude code counts the rounding thresholds that |x| passes, the
+// strict ones being ties that go down to an even code
+__device__ __forceinline__ uint32_t e2m1_code(float x) {
+    const float a = fabsf(x);
+    const uint32_t m = (uint32_t)(a > 0.25f) + (uint32_t)(a >= 0.75f) + (uint32_t)(a > 1.25f) +
+                       (uint32_t)(a >= 1.75f) + (uint32_t)(a > 2.5f) + (uint32_t)(a >= 3.5f) + (uint32_t)(a > 5.0f);
+    return m | ((__float_as_uint(x) >> 28) & 0x8u);
+}
+// value of an e2m1 code
+__device__ __forceinline__ float e2m1_value(uint32_t c) {
+    const uint32_t e = (c >> 1) & 3u, f = c & 1u;
+    const float mag = e ? __uint_as_float(((e + 126u) << 23) | (f << 22)) : 0.5f * (float)f;
+    return (c & 8u) ? -mag : mag;
+}
+// Quantise 8 consecutive elements of a 32-element block held by 4 consecutive lanes (lanes 4k ..
+// 4k+3 of the warp, in element order; all 32 lanes take part): returns the 8 codes packed in a
+// 32-bit word (element 2i in the low nibble of byte i) and the block's X in *x_out.
+__device__ __forceinline__ uint32_t mx_quantize8(const float v[8], int* x_out) {
+    float a = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) a = fmaxf(a, fabsf(v[i]));
+    a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
+    a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
+    const int x = mx_block_exp(a);
+    // v * 2^-X: exact (a power of two) except for results below the normal range, which are far
+    // below the smallest e2m1 step and round to 0 either way.  2^-X for X = -127 is 2^127.
+    const float inv = pow2i(-x);
+    uint32_t w = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w |= e2m1_code(v[i] * inv) << (4 * i);
+    *x_out = x;
+    return w;
+}
+
+// ---------------------------------------------------------------------
 // order-preserving float -> uint32 (larger float -> larger key); -0 == +0
 // ---------------------------------------------------------------------
 __device__ __forceinline__ uint32_t float_to_ordered(float f) {

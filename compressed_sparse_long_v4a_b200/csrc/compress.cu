@@ -9,13 +9,14 @@
 // rows of the previous block to the same per-channel softmax.
 //
 // Mapping: S adjacent lanes (S = the largest power of two <= min(m, 32); 1
-// for FP8 output) own 8 consecutive channels of one entry; each takes every
+// for FP8 and MXFP4 output) own 8 consecutive channels of one entry; each takes every
 // S-th token of the chunk with 16-byte vector loads (two for fp32), four
 // tokens per round with all loads issued first, keeping a running max /
 // denominator / numerator per channel in registers.  The S partial states are
 // merged with shuffles: common max, one rescale per lane, then sums.  For FP8
 // output the lanes of one entry are consecutive lanes of one warp, so the
-// entry's amax is found with warp shuffles too.
+// entry's amax is found with warp shuffles too; for MXFP4 output (OCP MX,
+// the FP4 indexer keys) each block of 32 channels is 4 consecutive lanes.
 #include "common.cuh"
 #include "internal.h"
 
@@ -32,6 +33,8 @@ struct StreamDesc {
     long long xb_bs, gateb_bs, prev_bs;
     void* out;
     float* out_scale;
+    uint8_t* out_exp;      // MXFP4 output: block exponents
+    long long exp_bs;
     int channels, groups;  // groups = channels / 8
     int split;             // S: lanes sharing one (entry, channel group)
     int in_dtype, out_dtype;
@@ -171,6 +174,16 @@ __global__ void __launch_bounds__(256) compress_kernel(StreamDesc s0, StreamDesc
         if (grp == 0) d.out_scale[(long long)b * d.scale_bs + s] = scale;
         return;
     }
+    if (d.out_dtype == V4A_MXFP4) {
+        // blocks of 32 channels = 4 consecutive lanes (groups is a multiple of 4)
+        int x;
+        const uint32_t w = mx_quantize8(out, &x);
+        if (!active) return;
+        uint8_t* op = static_cast<uint8_t*>(d.out) + ((long long)b * d.out_bs + s * d.channels + grp * 8) / 2;
+        *reinterpret_cast<uint32_t*>(op) = w;
+        if ((grp & 3) == 0) d.out_exp[(long long)b * d.exp_bs + s * (d.channels / 32) + grp / 4] = (uint8_t)(x + 127);
+        return;
+    }
     if (!active) return;
     if (d.out_dtype == V4A_BF16) {
         __nv_bfloat16* op = static_cast<__nv_bfloat16*>(d.out) + (long long)b * d.out_bs + s * d.channels + grp * 8;
@@ -181,6 +194,32 @@ __global__ void __launch_bounds__(256) compress_kernel(StreamDesc s0, StreamDesc
     }
 }
 
+// quantised outputs need every lane of an entry's block (or entry) to hold a finished value
+bool quantised(int dt) { return dt == V4A_FP8E4M3 || dt == V4A_MXFP4; }
+
+// MXFP4 quantisation of rows: one thread per 8 elements, 4 lanes per 32-element block
+template <typename T>
+__global__ void __launch_bounds__(256) quantize_mxfp4_kernel(const T* x, long long rows, int cols, uint8_t* codes,
+                                                             uint8_t* exps) {
+    const int groups = cols / 8;
+    const long long g = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const bool active = g < rows * groups;
+    const long long row = active ? g / groups : 0;
+    const int grp = active ? (int)(g - row * groups) : 0;
+    float v[8];
+    if (active) {
+        Vec8<T>::load_nc(x + row * cols + grp * 8, v);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = 0.f;
+    }
+    int xe;
+    const uint32_t w = mx_quantize8(v, &xe);
+    if (!active) return;
+    *reinterpret_cast<uint32_t*>(codes + row * (cols / 2) + grp * 4) = w;
+    if ((grp & 3) == 0) exps[row * (cols / 32) + grp / 4] = (uint8_t)(xe + 127);
+}
+
 StreamDesc describe(const v4a_compress_io* io) {
     StreamDesc d;
     d.x = io->x;
@@ -189,6 +228,8 @@ StreamDesc describe(const v4a_compress_io* io) {
     d.xb_bs = d.gateb_bs = d.prev_bs = 0;
     d.out = io->out;
     d.out_scale = io->out_scale;
+    d.out_exp = io->out_exp;
+    d.exp_bs = io->exp_batch_stride;
     d.channels = io->channels;
     d.groups = io->channels / 8;
     d.split = 1;
@@ -213,13 +254,27 @@ cudaError_t launch_compress(const v4a_compress_io* kv, const v4a_compress_io* id
     // (its per-entry amax runs over the entry's consecutive lanes)
     int split = 1;
     while (split < 32 && split * 2 <= m) split *= 2;
-    if (s0.out_dtype != V4A_FP8E4M3) s0.split = split;
-    if (s1.out_dtype != V4A_FP8E4M3) s1.split = split;
+    if (!quantised(s0.out_dtype)) s0.split = split;
+    if (!quantised(s1.out_dtype)) s1.split = split;
     long long w0 = (long long)s0.groups * s0.split, w1 = (long long)s1.groups * s1.split;
     long long total = (long long)batch * n_ent * (w0 > w1 ? w0 : w1);
     const int threads = 256;
     dim3 grid((unsigned)((total + threads - 1) / threads), idx ? 2 : 1);
     compress_kernel<<<grid, threads, 0, stream>>>(s0, s1, batch, n_ent, m);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_mxfp4(const void* x, v4a_dtype dt, long long rows, int cols, uint8_t* codes,
+                                  uint8_t* exps, cudaStream_t stream) {
+    const long long total = rows * (cols / 8);
+    if (total == 0) return cudaSuccess;
+    const int threads = 256;
+    const unsigned blocks = (unsigned)((total + threads - 1) / threads);
+    if (dt == V4A_BF16)
+        quantize_mxfp4_kernel<<<blocks, threads, 0, stream>>>(static_cast<const __nv_bfloat16*>(x), rows, cols,
+                                                              codes, exps);
+    else
+        quantize_mxfp4_kernel<<<blocks, threads, 0, stream>>>(static_cast<const float*>(x), rows, cols, codes, exps);
     return cudaGetLastError();
 }
 
@@ -237,7 +292,7 @@ cudaError_t launch_compress_dual(const v4a_compress_io* a, const v4a_series_b* b
     s0.prev_bs = b->prev_batch_stride;
     int split = 1;
     while (split < 32 && split * 2 <= m) split *= 2;
-    if (s0.out_dtype != V4A_FP8E4M3) s0.split = split;
+    if (!quantised(s0.out_dtype)) s0.split = split;
     const long long total = (long long)batch * n_ent * s0.groups * s0.split;
     const int threads = 256;
     dim3 grid((unsigned)((total + threads - 1) / threads), 1);

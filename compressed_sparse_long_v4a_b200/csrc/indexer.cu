@@ -7,8 +7,9 @@
 //
 // CUDA-core path, any (heads_i <= 64, d_i % 8 == 0) and key format: one thread
 // per entry streams the entry's key with 16-byte loads (fp8 keys: 8 bytes at a
-// time, widened exactly to fp32) and accumulates every head's dot product in
-// registers against the query held in shared memory (broadcast reads).
+// time, MXFP4 keys 4 bytes, widened exactly to fp32) and accumulates every
+// head's dot product in registers against the query held in shared memory
+// (broadcast reads; for MXFP4 keys the query is quantised to MXFP4 first).
 //
 // Select: per query row, an exact radix select over order-preserving 32-bit
 // keys of the fp32 scores (four 8-bit digits, most significant first) finds
@@ -23,15 +24,21 @@ namespace {
 
 constexpr int kScoreThreads = 256;
 
+// 8 key elements starting at element `off` of the key array (decoded exactly to fp32)
 template <int KFMT>
-__device__ __forceinline__ void load_key8(const void* k, long long off, float f[8]) {
+__device__ __forceinline__ void load_key8(const IndexArgs& a, long long off, float f[8]) {
     if constexpr (KFMT == V4A_F32) {
-        Vec8<float>::load_nc(static_cast<const float*>(k) + off, f);
+        Vec8<float>::load_nc(static_cast<const float*>(a.k) + off, f);
     } else if constexpr (KFMT == V4A_BF16) {
-        Vec8<__nv_bfloat16>::load_nc(static_cast<const __nv_bfloat16*>(k) + off, f);
-    } else {
-        uint2 v = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint8_t*>(k) + off));
+        Vec8<__nv_bfloat16>::load_nc(static_cast<const __nv_bfloat16*>(a.k) + off, f);
+    } else if constexpr (KFMT == V4A_FP8E4M3) {
+        uint2 v = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint8_t*>(a.k) + off));
         unpack_e4m3x8(v, f);
+    } else {  // MXFP4: 4 bytes of codes and their block's exponent
+        const uint32_t cw = __ldg(reinterpret_cast<const uint32_t*>(static_cast<const uint8_t*>(a.k) + off / 2));
+        const float sc = e8m0_value(__ldg(a.kexp + off / 32));
+#pragma unroll
+        for (int i = 0; i < 8; ++i) f[i] = e2m1_value((cw >> (4 * i)) & 0xfu) * sc;
     }
 }
 
@@ -56,6 +63,19 @@ __global__ void __launch_bounds__(kScoreThreads) index_score_kernel(IndexArgs a,
         for (int i = threadIdx.x; i < qn; i += blockDim.x) q_s[i] = qp[i];
     }
     for (int i = threadIdx.x; i < a.heads_i; i += blockDim.x) w_s[i] = a.w[(long long)row * a.heads_i + i];
+    if constexpr (KFMT == V4A_MXFP4) {
+        // FP4 dot products: the query of every head is quantised to MXFP4 (blocks of 32 along d_i)
+        // and replaced by its decoded values
+        __syncthreads();
+        for (int i = threadIdx.x; i < qn / 32; i += blockDim.x) {
+            float* p = q_s + 32 * i;
+            float am = 0.f;
+            for (int j = 0; j < 32; ++j) am = fmaxf(am, fabsf(p[j]));
+            const int x = mx_block_exp(am);
+            const float inv = pow2i(-x), sc = e8m0_value((uint32_t)(x + 127));
+            for (int j = 0; j < 32; ++j) p[j] = e2m1_value(e2m1_code(p[j] * inv)) * sc;
+        }
+    }
     __syncthreads();
 
     const long long s = (long long)blockIdx.x * blockDim.x + threadIdx.x;
@@ -71,7 +91,7 @@ __global__ void __launch_bounds__(kScoreThreads) index_score_kernel(IndexArgs a,
     const long long koff = ((long long)b * a.n_ent + s) * a.d_i;
     for (int c = 0; c < a.d_i; c += 8) {
         float kv[8];
-        load_key8<KFMT>(a.k, koff + c, kv);
+        load_key8<KFMT>(a, koff + c, kv);
 #pragma unroll
         for (int h = 0; h < HMAX; ++h) {
             if (h < a.heads_i) {
@@ -749,6 +769,12 @@ cudaError_t launch_scores_h(const IndexArgs& a, float* scores, cudaStream_t stre
     }
     case V4A_BF16: {
         auto kern = index_score_kernel<HMAX, V4A_BF16>;
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        kern<<<grid, kScoreThreads, smem, stream>>>(a, scores);
+        break;
+    }
+    case V4A_MXFP4: {
+        auto kern = index_score_kernel<HMAX, V4A_MXFP4>;
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         kern<<<grid, kScoreThreads, smem, stream>>>(a, scores);
         break;

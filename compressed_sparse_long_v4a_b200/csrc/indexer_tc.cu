@@ -1,5 +1,5 @@
 // indexer_tc.cu -- tensor-core Lightning-Indexer scores for d_I = 128 keys
-// (bf16, or FP8 e4m3 with one fp32 scale per entry) and up to 32 heads.
+// (bf16, FP8 e4m3 with one fp32 scale per entry, or MXFP4) and up to 32 heads.
 //
 // I(t,s) = scale_s * sum_j w_j * ReLU(q_j . k_s)   ("How V4 makes a
 // million-token context actually affordable", Lightning-Indexer section).
@@ -26,6 +26,8 @@
 // then holds G queries' heads (N = G x heads for bf16 keys, G x 4 x heads for
 // FP8), so every key tile is read once per G queries and each MMA does G
 // times the work.
+//  * MXFP4 keys (and the query quantised to MXFP4 per head): see the section
+//    "MXFP4 keys and queries" below.
 // Warp 0 loads key tiles into a shared-memory ring (4 x 32 KB for FP8, 2 x 64
 // KB for bf16), warp 1 issues the MMAs, warps 2-5 stage each row's B
 // operand, warps 6-9 run the epilogue.  CTAs take contiguous ranges of the
@@ -71,8 +73,9 @@ struct __align__(1024) IdxSmem {
     uint8_t q[2][kQBufBytes];                 // B operand per segment buffer
     float wq[2][128];                         // head weights of the G queries (times 2^-s for FP8)
     uint32_t hist[2][kHistBins];
+    float fq[2][4][32];                       // MXFP4: 2^X of each (block, head) of the query
     uint64_t k_full[kMaxStages], k_empty[kMaxStages], d_full[kMaxDStages], d_free[kMaxDStages], q_full[2], q_free[2],
-        ep_sync, drain;
+        a_full[2], a_free[2], ep_sync, drain;
     int abort_flag;
     uint32_t tmem_base;
 };
@@ -81,6 +84,7 @@ struct IdxTcArgs {
     const __nv_bfloat16* q;  // [rows][HI][128] bf16
     const float* w;          // [rows][HI]
     const float* kscale;     // [B][N] (FP8) or null
+    const uint8_t* kexp;     // [B][N][4] MXFP4 block exponents or null
     float* scores;           // [rows][N]
     uint32_t* hist;          // [rows][4096]
     int* err;                // device fault word (may be null)
@@ -483,6 +487,359 @@ __global__ void __launch_bounds__(kThreads, 1) index_score_tc_kernel(const __gri
     }
 }
 
+// ---------------------------------------------------------------------
+// MXFP4 keys and queries (FP4 dot products)
+// ---------------------------------------------------------------------
+// Key rows are 64 bytes of packed e2m1 codes (plus 4 E8M0 block exponents in a
+// separate array).  TMA brings 256-entry tiles (16 KB, 64-byte swizzle) into
+// 32 KB stages of two tiles.  Warps 2-5 turn each tile's codes into the MMA's
+// A operand in tensor memory: an e2m1 code s.e1e0.f becomes the e4m3 byte
+// s.000.e1e0.f.00, whose value is exactly the e2m1 value times 2^-6 (normal
+// codes keep their exponent relative to bias 7; the subnormal e2m1 0.5 lands
+// on the e4m3 subnormal 4/8 * 2^-6), so two shifts and two masks per word.
+// The 8 codes of a 32-bit code word go out as two words, even elements then
+// odd ones; the query is staged with the same permutation, which leaves every
+// 32-element block in its own 8 columns.  One K = 32 MMA per (half, block)
+// writes that block's partial dots into its own accumulator: products of
+// e2m1 values are multiples of 1/4, so each block sum is exact, and the
+// epilogue applies the two blocks' powers of two (2^Xk * 2^Xq, and 2^12 for
+// the two 2^-6) before the ReLU and the head weights.
+
+constexpr int kMxTileBytes = kTileK * 64;                 // packed codes of one 256-entry tile
+constexpr int kMxStageBytes = 2 * kMxTileBytes;           // two tiles per stage
+constexpr int kMxStages = kRingBytes / kMxStageBytes;     // 4
+constexpr uint32_t kMxACols = 64;                         // A operand of one tile: 2 halves x 32 columns
+constexpr uint32_t kMxABase = 0;                          // two A slots at columns [0, 128)
+template <int NP> struct MxAcc {
+    static constexpr uint32_t kCols = 2 * 4 * NP;         // per tile: 2 halves x 4 blocks x NP heads
+    static constexpr uint32_t kBase = 2 * kMxACols;
+    static constexpr int kStages =
+        (int)((kTmemCols - kBase) / kCols) < kMaxDStages ? (int)((kTmemCols - kBase) / kCols) : kMaxDStages;
+    static_assert(kStages >= 1, "accumulators exceed tensor memory");
+};
+static_assert(kMxStages <= kMaxStages, "ring stages");
+
+// even elements (low nibbles) / odd elements (high nibbles) of 8 packed e2m1 codes -> 4 e4m3 bytes
+__device__ __forceinline__ uint32_t e2m1x4_even_to_e4m3(uint32_t cw) {
+    return ((cw << 2) & 0x1C1C1C1Cu) | ((cw << 4) & 0x80808080u);
+}
+__device__ __forceinline__ uint32_t e2m1x4_odd_to_e4m3(uint32_t cw) {
+    return ((cw >> 2) & 0x1C1C1C1Cu) | (cw & 0x80808080u);
+}
+
+__device__ void mx_producer(IdxSmem& sm, const IdxTcArgs& a, const CUtensorMap* kmap, long long f0, long long f1) {
+    ICursor cur(f0, a, 1);
+    const long long n = f1 - f0, nst = (n + 1) / 2;
+    for (long long i = 0; i < nst; ++i) {
+        if (aborted(sm)) break;
+        const int st = (int)(i % kMxStages);
+        if (i >= kMxStages && !tc::mbar_wait(&sm.k_empty[st], (uint32_t)((i / kMxStages) - 1) & 1)) {
+            idx_fault(sm, a);
+            break;
+        }
+        const int nt = (2 * i + 1 < n) ? 2 : 1;
+        tc::mbar_arrive_expect_tx(&sm.k_full[st], (uint32_t)(nt * kMxTileBytes));
+        for (int u = 0; u < nt; ++u, cur.next(a)) {
+            const int y = (int)((long long)cur.bat * a.n_ent + (long long)cur.ti * kTileK);
+            tc::tma_load_2d(sm.ring + st * kMxStageBytes + u * kMxTileBytes, kmap, 0, y, &sm.k_full[st]);
+        }
+    }
+    // no copy may still be in flight when the CTA exits
+    for (long long i = nst - kMxStages; i < nst; ++i)
+        if (i >= 0) tc::mbar_wait(&sm.k_full[i % kMxStages], (uint32_t)(i / kMxStages) & 1);
+}
+
+template <int NP>
+__device__ void mx_mma(IdxSmem& sm, const IdxTcArgs& a, uint32_t tmem, long long f0, long long f1) {
+    using Acc = MxAcc<NP>;
+    constexpr int kDS = Acc::kStages;
+    constexpr uint32_t idesc = tc::idesc_e4m3(128, NP);
+    bool ok = true;
+    int seg = 0, b = 0;
+    uint64_t qd = 0;
+    ICursor cur(f0, a, 1);
+    for (long long f = f0; f < f1; ++f, cur.next(a)) {
+        if (aborted(sm)) { ok = false; break; }
+        const long long jt = f - f0;
+        const int slot = (int)(jt & 1), sd = (int)(jt % kDS);
+        if (f == f0 || cur.ti == 0) {
+            b = seg & 1;
+            if (!tc::mbar_wait(&sm.q_full[b], (seg >> 1) & 1)) { ok = false; break; }
+            qd = tc::sw128_desc(tc::smem_u32(sm.q[b]), 16, 1024);
+            ++seg;
+        }
+        const bool seg_end = (f == f1 - 1) || (cur.ti == a.tiles_per_row - 1);
+        if (!tc::mbar_wait(&sm.a_full[slot], (uint32_t)(jt >> 1) & 1)) { ok = false; break; }
+        if (jt >= kDS && !tc::mbar_wait(&sm.d_free[sd], (uint32_t)((jt / kDS) - 1) & 1)) { ok = false; break; }
+        tc::tc_fence_after();
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+            for (int blk = 0; blk < 4; ++blk)
+                tc::mma_f8_ts(tmem + Acc::kBase + Acc::kCols * sd + (4 * hf + blk) * NP,
+                              tmem + kMxABase + slot * kMxACols + 32 * hf + 8 * blk,
+                              qd + (uint64_t)((32 * blk) >> 4), idesc, 0u);
+        tc::mma_commit(&sm.a_free[slot]);
+        tc::mma_commit(&sm.d_full[sd]);
+        if (seg_end) tc::mma_commit(&sm.q_free[b]);
+    }
+    if (!ok) idx_fault(sm, a);
+    tc::mma_commit(&sm.drain);
+    tc::mbar_wait(&sm.drain, 0);
+}
+
+// B operand of one query (NP rows of 128 e4m3 bytes, K-major, 128-byte swizzle) from its MXFP4
+// quantisation, with the even/odd element order of the keys; fq = 2^X per (block, head) and the
+// head weights times 2^12.  A half-warp takes one head, lane l its elements 8l .. 8l+7.
+template <int NP>
+__device__ void stage_query_mx(IdxSmem& sm, const IdxTcArgs& a, int bat, int qj, int b, int ct) {
+    const int warp = ct >> 5, lane = ct & 31, l = lane & 15;
+    const long long row = (long long)bat * a.n_q + qj;
+    for (int h = 2 * warp + (lane >> 4); h < NP; h += 8) {  // NP is a multiple of 8: whole warps iterate
+        const bool live = h < a.heads_i;
+        float v[8];
+        if (live) {
+            Vec8<__nv_bfloat16>::load_nc(a.q + (row * a.heads_i + h) * kDI + 8 * l, v);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[i] = 0.f;
+        }
+        int x;
+        const uint32_t cw = mx_quantize8(v, &x);  // lanes 4k .. 4k+3 of the half-warp share block k
+        const int k = 8 * l;
+        uint8_t* dst = sm.q[b] + (h >> 3) * 1024 + (h & 7) * 128 + ((((k >> 4) ^ (h & 7))) << 4) + (k & 15);
+        *reinterpret_cast<uint2*>(dst) = make_uint2(e2m1x4_even_to_e4m3(cw), e2m1x4_odd_to_e4m3(cw));
+        if ((l & 3) == 0) sm.fq[b][l >> 2][h] = live ? e8m0_value((uint32_t)(x + 127)) : 0.f;
+        if (l == 0) sm.wq[b][h] = live ? a.w[row * a.heads_i + h] * 4096.0f : 0.f;
+    }
+}
+
+// warps 2-5: per segment the query's B operand; per tile the keys' A operand in tensor memory
+// (thread = TMEM lane r: entries r and r + 128 of the tile)
+template <int NP>
+__device__ void mx_convert(IdxSmem& sm, const IdxTcArgs& a, uint32_t tmem, long long f0, long long f1) {
+    const int ct = threadIdx.x - 64;
+    const int sub = (threadIdx.x >> 5) & 3;
+    const int r = 32 * sub + (threadIdx.x & 31);
+    const uint32_t lane_addr = (uint32_t)(32 * sub) << 16;
+    bool ok = true;
+    int seg = 0;
+    ICursor cur(f0, a, 1);
+    for (long long f = f0; f < f1; ++f, cur.next(a)) {
+        if (warp_aborted(sm)) { ok = false; break; }
+        const long long jt = f - f0;
+        if (f == f0 || cur.ti == 0) {
+            const int b = seg & 1;
+            if (seg >= 2 && !warp_wait(&sm.q_free[b], ((seg >> 1) - 1) & 1)) { ok = false; break; }
+            stage_query_mx<NP>(sm, a, cur.bat, cur.q0, b, ct);
+            tc::fence_proxy_async();
+            tc::mbar_arrive(&sm.q_full[b]);
+            ++seg;
+        }
+        const int st = (int)((jt >> 1) % kMxStages), u = (int)(jt & 1), slot = (int)(jt & 1);
+        if (u == 0 && !warp_wait(&sm.k_full[st], (uint32_t)((jt >> 1) / kMxStages) & 1)) { ok = false; break; }
+        if (jt >= 2 && !warp_wait(&sm.a_free[slot], (uint32_t)((jt >> 1) - 1) & 1)) { ok = false; break; }
+        const uint8_t* tile = sm.ring + st * kMxStageBytes + u * kMxTileBytes;
+        uint32_t wv[64];
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+            const int y = hf * kHalf + r;
+            const uint8_t* rowp = tile + y * 64;
+            const int sw = (y >> 1) & 3;  // 64-byte swizzle: 16-byte chunk c of row y sits at chunk c ^ sw
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const uint4 v = *reinterpret_cast<const uint4*>(rowp + ((c ^ sw) << 4));
+                const uint32_t cw[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    wv[32 * hf + 8 * c + 2 * i] = e2m1x4_even_to_e4m3(cw[i]);
+                    wv[32 * hf + 8 * c + 2 * i + 1] = e2m1x4_odd_to_e4m3(cw[i]);
+                }
+            }
+        }
+        // the stage's codes are in registers: release it after its second tile (or the range's last)
+        if (u == 1 || f == f1 - 1) tc::mbar_arrive(&sm.k_empty[st]);
+        tc::tmem_st_x64(tmem + lane_addr + kMxABase + slot * kMxACols, wv);
+        tc::tmem_st_wait();
+        tc::tc_fence_before();
+        tc::mbar_arrive(&sm.a_full[slot]);
+    }
+    if (!ok) idx_fault(sm, a);
+}
+
+// one entry's score from its 4 x NP block dots (columns blk * NP + h of this thread's lane)
+template <int NP>
+__device__ __forceinline__ float mx_score(uint32_t taddr, const float (*fq)[32], const float* wq, uint32_t ex) {
+    const float k0 = e8m0_value(ex & 0xffu), k1 = e8m0_value((ex >> 8) & 0xffu), k2 = e8m0_value((ex >> 16) & 0xffu),
+                k3 = e8m0_value(ex >> 24);
+    float acc = 0.f;
+    uint32_t r[64];
+    if constexpr (NP == 16) {
+        tc::tmem_ld_x64(taddr, r);
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int h = 0; h < 16; ++h) {
+            float dot = __uint_as_float(r[h]) * fq[0][h] * k0;
+            dot = fmaf(__uint_as_float(r[16 + h]) * fq[1][h], k1, dot);
+            dot = fmaf(__uint_as_float(r[32 + h]) * fq[2][h], k2, dot);
+            dot = fmaf(__uint_as_float(r[48 + h]) * fq[3][h], k3, dot);
+            acc = fmaf(wq[h], fmaxf(dot, 0.f), acc);
+        }
+    } else {
+        // 16 heads at a time: columns blk * 32 + 16 * hg + (0 .. 15)
+#pragma unroll
+        for (int hg = 0; hg < 2; ++hg) {
+            uint32_t (&q4)[4][16] = *reinterpret_cast<uint32_t(*)[4][16]>(r);
+#pragma unroll
+            for (int blk = 0; blk < 4; ++blk) tc::tmem_ld_x16(taddr + 32 * blk + 16 * hg, q4[blk]);
+            tc::tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const int h = 16 * hg + i;
+                float dot = __uint_as_float(q4[0][i]) * fq[0][h] * k0;
+                dot = fmaf(__uint_as_float(q4[1][i]) * fq[1][h], k1, dot);
+                dot = fmaf(__uint_as_float(q4[2][i]) * fq[2][h], k2, dot);
+                dot = fmaf(__uint_as_float(q4[3][i]) * fq[3][h], k3, dot);
+                acc = fmaf(wq[h], fmaxf(dot, 0.f), acc);
+            }
+        }
+    }
+    return acc;
+}
+
+// warps 6-9: scores of entries r and r + 128 of each tile, histogram counts and stores
+template <int NP>
+__device__ void mx_epilogue(IdxSmem& sm, const IdxTcArgs& a, uint32_t tmem, long long f0, long long f1) {
+    using Acc = MxAcc<NP>;
+    constexpr int kDS = Acc::kStages;
+    const int et = threadIdx.x - 192;
+    const int sub = (threadIdx.x >> 5) & 3;
+    const int r = 32 * sub + (threadIdx.x & 31);
+    const uint32_t lane_addr = (uint32_t)(32 * sub) << 16;
+    bool ok = true;
+    int seg = 0, b = 0, nsync = 0;
+    long long nv = 0;
+    float* srow = nullptr;
+    ICursor cur(f0, a, 1);
+    // block exponents of the current tile's two entries, loaded one tile ahead
+    auto exps_of = [&](const ICursor& c, uint32_t (&ex)[2]) {
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+            const long long e = (long long)c.ti * kTileK + kHalf * hf + r;
+            ex[hf] = e < a.n_ent ? __ldg(reinterpret_cast<const uint32_t*>(a.kexp) + (long long)c.bat * a.n_ent + e)
+                                 : 0x7f7f7f7fu;
+        }
+    };
+    uint32_t ex_cur[2];
+    exps_of(cur, ex_cur);
+    for (long long f = f0; f < f1; ++f) {
+        if (warp_aborted(sm)) { ok = false; break; }
+        const int jt = (int)(f - f0), sd = jt % kDS;
+        if (f == f0 || cur.ti == 0) {
+            b = seg & 1;
+            if (!warp_wait(&sm.q_full[b], (seg >> 1) & 1)) { ok = false; break; }
+            ++seg;
+            nv = nvis_of(cur.q0, a);
+            srow = a.scores + ((long long)cur.bat * a.n_q + cur.q0) * a.n_ent;
+        }
+        const bool seg_end = (f == f1 - 1) || (cur.ti == a.tiles_per_row - 1);
+        const int ti = cur.ti, row = cur.bat * a.n_q + cur.q0;
+        cur.next(a);
+        uint32_t ex_next[2] = {0x7f7f7f7fu, 0x7f7f7f7fu};
+        if (f + 1 < f1) exps_of(cur, ex_next);
+        if (!warp_wait(&sm.d_full[sd], (jt / kDS) & 1)) { ok = false; break; }
+        tc::tc_fence_after();
+        float acc[2];
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf)
+            acc[hf] = mx_score<NP>(tmem + lane_addr + Acc::kBase + Acc::kCols * sd + 4 * NP * hf, sm.fq[b], sm.wq[b],
+                                   ex_cur[hf]);
+        tc::tc_fence_before();
+        tc::mbar_arrive(&sm.d_free[sd]);
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+            const long long e = (long long)ti * kTileK + kHalf * hf + r;
+            if (e < a.n_ent) {
+                float sc = -INFINITY;
+                if (e < nv) {
+                    sc = acc[hf] + 0.0f;
+                    if (a.hist) atomicAdd(&sm.hist[b][float_to_ordered(sc) >> 20], 1u);
+                }
+                srow[e] = sc;
+            }
+        }
+        ex_cur[0] = ex_next[0];
+        ex_cur[1] = ex_next[1];
+        if (seg_end) {
+            tc::mbar_arrive(&sm.q_free[b]);  // done with wq[b] and fq[b]
+            if (a.hist) {
+                tc::mbar_arrive(&sm.ep_sync);
+                if (!warp_wait(&sm.ep_sync, nsync++ & 1)) { ok = false; break; }
+                uint32_t* gh = a.hist + (long long)row * kHistBins;
+                for (int i = et; i < kHistBins; i += 128) {
+                    const uint32_t v = sm.hist[b][i];
+                    if (v) {
+                        atomicAdd(gh + i, v);
+                        sm.hist[b][i] = 0;
+                    }
+                }
+            }
+        }
+    }
+    if (!ok) idx_fault(sm, a);
+}
+
+template <int NP>
+__global__ void __launch_bounds__(kThreads, 1) index_score_mx_kernel(const __grid_constant__ CUtensorMap kmap, IdxTcArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    IdxSmem& sm = *reinterpret_cast<IdxSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long f0 = irange(blockIdx.x, a), f1 = irange(blockIdx.x + 1, a);
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kMxStages; ++i) {
+            tc::mbar_init(&sm.k_full[i], 1);
+            tc::mbar_init(&sm.k_empty[i], 128);  // every converter thread
+        }
+        for (int i = 0; i < MxAcc<NP>::kStages; ++i) {
+            tc::mbar_init(&sm.d_full[i], 1);
+            tc::mbar_init(&sm.d_free[i], 128);
+        }
+        for (int i = 0; i < 2; ++i) {
+            tc::mbar_init(&sm.q_full[i], 128);
+            tc::mbar_init(&sm.q_free[i], 1 + 128);
+            tc::mbar_init(&sm.a_full[i], 128);
+            tc::mbar_init(&sm.a_free[i], 1);
+        }
+        tc::mbar_init(&sm.ep_sync, 128);
+        tc::mbar_init(&sm.drain, 1);
+        sm.abort_flag = 0;
+        tc::fence_barrier_init();
+    }
+    for (int i = threadIdx.x; i < 2 * kHistBins; i += kThreads) (&sm.hist[0][0])[i] = 0;
+    for (int i = threadIdx.x; i < 2 * kQBufBytes / 4; i += kThreads) reinterpret_cast<uint32_t*>(sm.q)[i] = 0;
+    if (warp == 1) tc::tmem_alloc(&sm.tmem_base, kTmemCols);
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    if (warp == 0) {
+        if (lane == 0) mx_producer(sm, a, &kmap, f0, f1);
+    } else if (warp == 1) {
+        if (lane == 0) mx_mma<NP>(sm, a, tmem, f0, f1);
+    } else if (warp < 6) {
+        mx_convert<NP>(sm, a, tmem, f0, f1);
+    } else {
+        mx_epilogue<NP>(sm, a, tmem, f0, f1);
+    }
+    __syncwarp();
+    tc::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 idx_encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
     if (!fn) {
@@ -495,12 +852,56 @@ PFN_cuTensorMapEncodeTiled_v12000 idx_encode_fn() {
     return fn;
 }
 
+// MXFP4 keys: one query row per segment (no multi-query grouping); tiles of 256 entries
+cudaError_t launch_index_scores_mx(const IndexArgs& a, float* scores, uint32_t* hist, int* err, cudaStream_t stream,
+                                   PFN_cuTensorMapEncodeTiled_v12000 fn) {
+    CUtensorMap kmap;
+    cuuint64_t dims[2] = {64, (cuuint64_t)((long long)a.batch * a.n_ent)};
+    cuuint64_t strides[1] = {64};
+    cuuint32_t box[2] = {64u, (cuuint32_t)kTileK};
+    cuuint32_t estr[2] = {1, 1};
+    if (fn(&kmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(a.k), dims, strides, box, estr,
+           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    IdxTcArgs t;
+    t.q = static_cast<const __nv_bfloat16*>(a.q);
+    t.w = a.w;
+    t.kscale = nullptr;
+    t.kexp = a.kexp;
+    t.scores = scores;
+    t.hist = hist;
+    t.err = err;
+    t.n_ent = a.n_ent;
+    t.ctx_len = a.ctx_len;
+    t.rows = a.batch * a.n_q;
+    t.n_q = a.n_q;
+    t.m = a.m;
+    t.heads_i = a.heads_i;
+    t.ngroups = a.n_q;
+    long long nv_max = n_visible(a.ctx_len - 1, a.m);
+    if (nv_max > a.n_ent) nv_max = a.n_ent;
+    t.tiles_per_row = (int)((nv_max + kTileK - 1) / kTileK);
+    t.total_tiles = (long long)a.batch * t.ngroups * t.tiles_per_row;
+    if (t.total_tiles == 0) return cudaSuccess;
+    t.grid = (int)(t.total_tiles < kNumSMs ? t.total_tiles : kNumSMs);
+    const size_t smem = sizeof(IdxSmem) + 1024;
+    auto go = [&](auto kernel) {
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e == cudaSuccess) kernel<<<t.grid, kThreads, smem, stream>>>(kmap, t);
+        return e;
+    };
+    cudaError_t e = a.heads_i <= 16 ? go(index_score_mx_kernel<16>) : go(index_score_mx_kernel<32>);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 bool index_tc_shape_ok(const IndexArgs& a) {
     return a.d_i == kDI && a.heads_i <= 32 && a.q_dtype == V4A_BF16 &&
-           (a.k_dtype == V4A_BF16 || a.k_dtype == V4A_FP8E4M3) && a.n_ent >= 1 &&
-           (long long)a.batch * a.n_ent < (1LL << 31);
+           (a.k_dtype == V4A_BF16 || a.k_dtype == V4A_FP8E4M3 || (a.k_dtype == V4A_MXFP4 && a.kexp)) &&
+           a.n_ent >= 1 && (long long)a.batch * a.n_ent < (1LL << 31);
 }
 
 bool index_tc_available(const IndexArgs& a) { return index_tc_shape_ok(a) && idx_encode_fn() != nullptr; }
@@ -508,6 +909,7 @@ bool index_tc_available(const IndexArgs& a) { return index_tc_shape_ok(a) && idx
 cudaError_t launch_index_scores_tc(const IndexArgs& a, float* scores, uint32_t* hist, int* err, cudaStream_t stream) {
     auto fn = idx_encode_fn();
     if (!fn) return cudaErrorNotSupported;
+    if (a.k_dtype == V4A_MXFP4) return launch_index_scores_mx(a, scores, hist, err, stream, fn);
     const bool fp8 = a.k_dtype == V4A_FP8E4M3;
     CUtensorMap kmap;
     cuuint64_t dims[2] = {(cuuint64_t)kDI, (cuuint64_t)((long long)a.batch * a.n_ent)};
@@ -522,6 +924,7 @@ cudaError_t launch_index_scores_tc(const IndexArgs& a, float* scores, uint32_t* 
     t.q = static_cast<const __nv_bfloat16*>(a.q);
     t.w = a.w;
     t.kscale = a.kscale;
+    t.kexp = nullptr;
     t.scores = scores;
     t.hist = hist;
     t.err = err;

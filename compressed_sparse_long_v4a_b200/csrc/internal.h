@@ -17,6 +17,8 @@ cudaError_t launch_compress(const v4a_compress_io* kv, const v4a_compress_io* id
                             int m, cudaStream_t stream);
 cudaError_t launch_compress_dual(const v4a_compress_io* a, const v4a_series_b* b, int batch, long long n_tok, int m,
                                  cudaStream_t stream);
+cudaError_t launch_quantize_mxfp4(const void* x, v4a_dtype dt, long long rows, int cols, uint8_t* codes,
+                                  uint8_t* exps, cudaStream_t stream);
 
 // ---- indexer.cu -------------------------------------------------------
 struct IndexArgs {
@@ -24,6 +26,7 @@ struct IndexArgs {
     const float* w;       // [B][n_q][HI]
     const void* k;        // [B][N][DI]
     const float* kscale;  // [B][N] or null
+    const uint8_t* kexp;  // [B][N][DI/32] MXFP4 block exponents (k_dtype MXFP4), else null
     v4a_dtype q_dtype, k_dtype;
     int batch, n_q, m, heads_i, d_i;
     long long ctx_len, n_ent;

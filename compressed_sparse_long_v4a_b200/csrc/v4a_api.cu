@@ -32,8 +32,24 @@ v4a_status check_compress_io(const v4a_compress_io* io, const char* name, long l
     if (io->channels < 8 || io->channels % 8) return fail(V4A_ERR_INVALID_ARG, "%s: channels must be a multiple of 8", name);
     if (io->in_dtype != V4A_F32 && io->in_dtype != V4A_BF16)
         return fail(V4A_ERR_UNSUPPORTED, "%s: input dtype must be F32 or BF16", name);
-    if (io->out_dtype != V4A_F32 && io->out_dtype != V4A_BF16 && io->out_dtype != V4A_FP8E4M3)
+    if (io->out_dtype != V4A_F32 && io->out_dtype != V4A_BF16 && io->out_dtype != V4A_FP8E4M3 &&
+        io->out_dtype != V4A_MXFP4)
         return fail(V4A_ERR_UNSUPPORTED, "%s: unknown output dtype", name);
+    if (io->out_dtype == V4A_MXFP4) {
+        if (io->channels % 32) return fail(V4A_ERR_INVALID_ARG, "%s: MXFP4 output needs channels % 32 == 0", name);
+        if (!io->out_exp) return fail(V4A_ERR_INVALID_ARG, "%s: MXFP4 output needs out_exp", name);
+        const long long n_ent = n_tok / m;
+        if (io->out_batch_stride < n_ent * io->channels || io->out_batch_stride % 8 ||
+            io->exp_batch_stride < n_ent * (io->channels / 32))
+            return fail(V4A_ERR_INVALID_ARG, "%s: MXFP4 out/out_exp batch stride too small or out stride not a multiple of 8",
+                        name);
+        if (!aligned(io->x, 16) || !aligned(io->gate, 16) || !aligned(io->out, 4) ||
+            (io->x_batch_stride * dtype_size(io->in_dtype)) % 16 || (io->gate_batch_stride * dtype_size(io->in_dtype)) % 16)
+            return fail(V4A_ERR_INVALID_ARG, "%s: x/gate (16 bytes) or out (4 bytes) misaligned", name);
+        if (io->x_batch_stride < n_tok * io->channels || io->gate_batch_stride < n_tok * io->channels)
+            return fail(V4A_ERR_INVALID_ARG, "%s: a batch stride is smaller than one sequence", name);
+        return V4A_OK;
+    }
     if (io->out_dtype == V4A_FP8E4M3) {
         int g = io->channels / 8;
         if (!io->out_scale) return fail(V4A_ERR_INVALID_ARG, "%s: FP8E4M3 output needs out_scale", name);
@@ -63,8 +79,8 @@ v4a_status check_shape_common(const v4a_shape* s) {
     return V4A_OK;
 }
 
-v4a_status index_args(const void* q_i, const float* w, const void* k_i, const float* k_scale, int heads_i, int d_i,
-                      v4a_dtype q_dt, v4a_dtype k_dt, const v4a_shape* s, v4a::IndexArgs* a) {
+v4a_status index_args(const void* q_i, const float* w, const void* k_i, const float* k_scale, const uint8_t* k_exp,
+                      int heads_i, int d_i, v4a_dtype q_dt, v4a_dtype k_dt, const v4a_shape* s, v4a::IndexArgs* a) {
     v4a_status st = check_shape_common(s);
     if (st != V4A_OK) return st;
     if (!q_i || !w || (!k_i && s->ctx_len / s->m > 0)) return fail(V4A_ERR_INVALID_ARG, "q_i, w and k_i are required");
@@ -72,15 +88,21 @@ v4a_status index_args(const void* q_i, const float* w, const void* k_i, const fl
     if (d_i < 8 || d_i % 8 || d_i > 1024) return fail(V4A_ERR_INVALID_ARG, "d_i must be a multiple of 8 (<= 1024)");
     if ((long long)heads_i * d_i > 32768) return fail(V4A_ERR_UNSUPPORTED, "heads_i * d_i must be <= 32768");
     if (q_dt != V4A_F32 && q_dt != V4A_BF16) return fail(V4A_ERR_UNSUPPORTED, "q_i dtype must be F32 or BF16");
-    if (k_dt != V4A_F32 && k_dt != V4A_BF16 && k_dt != V4A_FP8E4M3)
-        return fail(V4A_ERR_UNSUPPORTED, "k_i dtype must be F32, BF16 or FP8E4M3");
+    if (k_dt == V4A_MXFP4) {
+        if (!k_exp && s->ctx_len / s->m > 0) return fail(V4A_ERR_INVALID_ARG, "MXFP4 keys need k_exp");
+        if (d_i % 32) return fail(V4A_ERR_INVALID_ARG, "MXFP4 keys need d_i % 32 == 0");
+        if (!aligned(k_exp, 4)) return fail(V4A_ERR_INVALID_ARG, "k_exp must be 4-byte aligned");
+    } else if (k_dt != V4A_F32 && k_dt != V4A_BF16 && k_dt != V4A_FP8E4M3) {
+        return fail(V4A_ERR_UNSUPPORTED, "k_i dtype must be F32, BF16 or FP8E4M3 (MXFP4 keys: the _mxfp4 calls)");
+    }
     if (k_dt == V4A_FP8E4M3 && !k_scale) return fail(V4A_ERR_INVALID_ARG, "FP8E4M3 keys need k_scale");
     if (!aligned(k_i, 16) || !aligned(q_i, 16) || !aligned(w, 4))
         return fail(V4A_ERR_INVALID_ARG, "q_i/k_i must be 16-byte aligned");
     a->q = q_i;
     a->w = w;
     a->k = k_i;
-    a->kscale = k_scale;
+    a->kscale = k_dt == V4A_MXFP4 ? nullptr : k_scale;
+    a->kexp = k_dt == V4A_MXFP4 ? k_exp : nullptr;
     a->q_dtype = q_dt;
     a->k_dtype = k_dt;
     a->batch = s->batch;
@@ -149,6 +171,19 @@ v4a_status v4a::report(v4a_status st, const char* fmt, ...) {
     return st;
 }
 
+static v4a_status topk_common(const v4a::IndexArgs& a, int32_t* idx_out, float* score_out, void* workspace,
+                              size_t workspace_bytes, const v4a_shape* shape, void* stream, const char* what) {
+    if (shape->k < 1 || shape->k > 4096) return fail(V4A_ERR_INVALID_ARG, "k must be in 1..4096");
+    if (!idx_out) return fail(V4A_ERR_INVALID_ARG, "idx_out is required");
+    size_t need = v4a::topk_workspace_bytes(a, shape->k);
+    if (!workspace || workspace_bytes < need)
+        return fail(V4A_ERR_INVALID_ARG, "workspace of %zu bytes needed, %zu given", need, workspace_bytes);
+    if (!aligned(workspace, 256)) return fail(V4A_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    return from_cuda(v4a::launch_topk(a, shape->k, idx_out, score_out, workspace, workspace_bytes,
+                                      (cudaStream_t)stream),
+                     what);
+}
+
 extern "C" {
 
 v4a_status v4a_compress(const v4a_compress_io* kv, const v4a_compress_io* idx, int batch, long long n_tok, int m,
@@ -189,28 +224,55 @@ v4a_status v4a_compress_dual(const v4a_compress_io* a, const v4a_series_b* b, in
 v4a_status v4a_index_scores(const void* q_i, const float* w, const void* k_i, const float* k_scale, float* scores,
                             int heads_i, int d_i, v4a_dtype q_dtype, v4a_dtype k_dtype, const v4a_shape* shape,
                             void* stream) {
+    if (k_dtype == V4A_MXFP4) return fail(V4A_ERR_UNSUPPORTED, "MXFP4 keys: use v4a_index_scores_mxfp4");
     v4a::IndexArgs a;
-    v4a_status st = index_args(q_i, w, k_i, k_scale, heads_i, d_i, q_dtype, k_dtype, shape, &a);
+    v4a_status st = index_args(q_i, w, k_i, k_scale, nullptr, heads_i, d_i, q_dtype, k_dtype, shape, &a);
     if (st != V4A_OK) return st;
     if (!scores && a.n_ent > 0) return fail(V4A_ERR_INVALID_ARG, "scores is required");
     return from_cuda(v4a::launch_index_scores(a, scores, (cudaStream_t)stream), "v4a_index_scores");
 }
 
+v4a_status v4a_index_scores_mxfp4(const void* q_i, const float* w, const uint8_t* k_codes, const uint8_t* k_exp,
+                                  float* scores, int heads_i, int d_i, v4a_dtype q_dtype, const v4a_shape* shape,
+                                  void* stream) {
+    v4a::IndexArgs a;
+    v4a_status st = index_args(q_i, w, k_codes, nullptr, k_exp, heads_i, d_i, q_dtype, V4A_MXFP4, shape, &a);
+    if (st != V4A_OK) return st;
+    if (!scores && a.n_ent > 0) return fail(V4A_ERR_INVALID_ARG, "scores is required");
+    return from_cuda(v4a::launch_index_scores(a, scores, (cudaStream_t)stream), "v4a_index_scores_mxfp4");
+}
+
 v4a_status v4a_topk(const void* q_i, const float* w, const void* k_i, const float* k_scale, int32_t* idx_out,
                     float* score_out, int heads_i, int d_i, v4a_dtype q_dtype, v4a_dtype k_dtype, void* workspace,
                     size_t workspace_bytes, const v4a_shape* shape, void* stream) {
+    if (k_dtype == V4A_MXFP4) return fail(V4A_ERR_UNSUPPORTED, "MXFP4 keys: use v4a_topk_mxfp4");
     v4a::IndexArgs a;
-    v4a_status st = index_args(q_i, w, k_i, k_scale, heads_i, d_i, q_dtype, k_dtype, shape, &a);
+    v4a_status st = index_args(q_i, w, k_i, k_scale, nullptr, heads_i, d_i, q_dtype, k_dtype, shape, &a);
     if (st != V4A_OK) return st;
-    if (shape->k < 1 || shape->k > 4096) return fail(V4A_ERR_INVALID_ARG, "k must be in 1..4096");
-    if (!idx_out) return fail(V4A_ERR_INVALID_ARG, "idx_out is required");
-    size_t need = v4a::topk_workspace_bytes(a, shape->k);
-    if (!workspace || workspace_bytes < need)
-        return fail(V4A_ERR_INVALID_ARG, "workspace of %zu bytes needed, %zu given", need, workspace_bytes);
-    if (!aligned(workspace, 256)) return fail(V4A_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
-    return from_cuda(v4a::launch_topk(a, shape->k, idx_out, score_out, workspace, workspace_bytes,
-                                      (cudaStream_t)stream),
-                     "v4a_topk");
+    return topk_common(a, idx_out, score_out, workspace, workspace_bytes, shape, stream, "v4a_topk");
+}
+
+v4a_status v4a_topk_mxfp4(const void* q_i, const float* w, const uint8_t* k_codes, const uint8_t* k_exp,
+                          int32_t* idx_out, float* score_out, int heads_i, int d_i, v4a_dtype q_dtype,
+                          void* workspace, size_t workspace_bytes, const v4a_shape* shape, void* stream) {
+    v4a::IndexArgs a;
+    v4a_status st = index_args(q_i, w, k_codes, nullptr, k_exp, heads_i, d_i, q_dtype, V4A_MXFP4, shape, &a);
+    if (st != V4A_OK) return st;
+    return topk_common(a, idx_out, score_out, workspace, workspace_bytes, shape, stream, "v4a_topk_mxfp4");
+}
+
+
+v4a_status v4a_quantize_mxfp4(const void* x, v4a_dtype dtype, long long rows, int cols, uint8_t* codes,
+                              uint8_t* exps, void* stream) {
+    if (rows < 0 || cols < 32 || cols % 32)
+        return fail(V4A_ERR_INVALID_ARG, "v4a_quantize_mxfp4: need rows >= 0 and cols a positive multiple of 32");
+    if (dtype != V4A_F32 && dtype != V4A_BF16) return fail(V4A_ERR_UNSUPPORTED, "v4a_quantize_mxfp4: dtype must be F32 or BF16");
+    if (rows == 0) return V4A_OK;
+    if (!x || !codes || !exps) return fail(V4A_ERR_INVALID_ARG, "v4a_quantize_mxfp4: x, codes and exps are required");
+    if (!aligned(x, 16) || !aligned(codes, 4))
+        return fail(V4A_ERR_INVALID_ARG, "v4a_quantize_mxfp4: x must be 16-byte and codes 4-byte aligned");
+    return from_cuda(v4a::launch_quantize_mxfp4(x, dtype, rows, cols, codes, exps, (cudaStream_t)stream),
+                     "v4a_quantize_mxfp4");
 }
 
 static v4a_status attend_common(const void* q, const void* entries, const int32_t* idx, const void* token_kv,
@@ -318,6 +380,6 @@ const char* v4a_status_string(v4a_status st) {
 
 const char* v4a_last_error(void) { return g_last_error; }
 
-int v4a_version(void) { return 100; }
+int v4a_version(void) { return 200; }
 
 }  // extern "C"

@@ -63,7 +63,11 @@ typedef enum v4a_status {
 typedef enum v4a_dtype {
     V4A_F32 = 0,      /* IEEE binary32 */
     V4A_BF16 = 1,     /* bfloat16 */
-    V4A_FP8E4M3 = 2   /* float8 e4m3 ("fn": no inf, max 448), with one fp32 scale per row */
+    V4A_FP8E4M3 = 2,  /* float8 e4m3 ("fn": no inf, max 448), with one fp32 scale per row */
+    V4A_MXFP4 = 3     /* OCP Microscaling MXFP4: e2m1 codes (1 sign, 2 exponent bits with bias 1,
+                         1 fraction bit: 0, 0.5, 1, 1.5, 2, 3, 4, 6), two per byte with element 2i
+                         in the low nibble of byte i, and one E8M0 exponent byte e per 32
+                         consecutive elements of a row, scaling them by 2^(e-127) (e = 255 is NaN) */
 } v4a_dtype;
 
 /* Problem shape.  Fields an entry point does not use are ignored. */
@@ -95,8 +99,11 @@ typedef struct v4a_compress_io {
     v4a_dtype out_dtype;          /* F32, BF16 or FP8E4M3 */
     long long x_batch_stride;     /* elements between sequences in x (>= n_tok*channels) */
     long long gate_batch_stride;  /* elements between sequences in gate */
-    long long out_batch_stride;   /* elements between sequences in out */
+    long long out_batch_stride;   /* elements between sequences in out (MXFP4: even; bytes = elements/2) */
     long long scale_batch_stride; /* floats between sequences in out_scale */
+    uint8_t* out_exp;             /* [batch][n_tok/m][channels/32] E8M0 block exponents; required iff
+                                     out_dtype == MXFP4 */
+    long long exp_batch_stride;   /* bytes between sequences in out_exp */
 } v4a_compress_io;
 
 /* Chunk compression ("DeepSeek-V4 的暗线之一：分层记忆比输入框更关键",
@@ -107,7 +114,9 @@ typedef struct v4a_compress_io {
  * The same single-series rule serves m = 4 (CSA) and m' = 128 (HCA).
  * FP8E4M3 output stores, per entry, scale = amax/448 (1 for an all-zero
  * entry) in out_scale and each value as the nearest e4m3 code of
- * value/scale (ties to even, saturating).
+ * value/scale (ties to even, saturating).  MXFP4 output quantises each
+ * block of 32 channels as v4a_quantize_mxfp4 does (channels a multiple of
+ * 32; codes in out, exponents in out_exp).
  * kv: the K=V stream (required).  idx: the indexer-key stream compressed in
  * the same launch (may be NULL); it uses the same batch, n_tok and m.
  * n_tok: tokens per sequence; a trailing partial chunk is ignored.
@@ -154,6 +163,21 @@ V4A_API v4a_status v4a_compress_dual(const v4a_compress_io* a, const v4a_series_
 /* Lightning indexer and top-k                                          */
 /* ------------------------------------------------------------------ */
 
+/* MXFP4 quantisation (the OCP Microscaling v1.0 conversion; the FP4 indexer
+ * keys of "1M Context != Lossless Long Memory", section 4.2 and footnote 3,
+ * whose bit format the pages leave open).  Each row of x [rows][cols] (dtype
+ * F32 or BF16, cols a multiple of 32) is cut into blocks of 32; a block with
+ * largest magnitude amax gets X = max(floor(log2(amax)) - 2, -127) (-127 for
+ * an all-zero block), exps[row][block] = X + 127, and element v the nearest
+ * e2m1 code of v / 2^X (ties to the even code, magnitudes above 6 clamp to
+ * 6, the sign bit kept even when the magnitude rounds to 0).
+ * codes: [rows][cols/2] bytes; exps: [rows][cols/32] bytes.  Inputs are
+ * taken to be finite.  Errors: V4A_ERR_INVALID_ARG for NULL pointers,
+ * rows < 0, cols not a positive multiple of 32, x not 16-byte aligned or
+ * codes not 4-byte aligned; V4A_ERR_UNSUPPORTED for another dtype. */
+V4A_API v4a_status v4a_quantize_mxfp4(const void* x, v4a_dtype dtype, long long rows, int cols, uint8_t* codes,
+                                      uint8_t* exps, void* stream);
+
 /* Indexer scores ("How V4 makes a million-token context actually
  * affordable", Lightning-Indexer section):
  *     I(t,s) = scale[s] * sum_{j<heads_i} w[j] * ReLU(q_i[j] . k_i[s]),
@@ -181,6 +205,27 @@ V4A_API v4a_status v4a_index_scores(const void* q_i, const float* w, const void*
 V4A_API v4a_status v4a_topk(const void* q_i, const float* w, const void* k_i, const float* k_scale, int32_t* idx_out,
                     float* score_out, int heads_i, int d_i, v4a_dtype q_dtype, v4a_dtype k_dtype, void* workspace,
                     size_t workspace_bytes, const v4a_shape* shape, void* stream);
+
+/* Indexer scores and top-k with FP4 keys and FP4 dot products ("1M Context
+ * != Lossless Long Memory", section 4.2: indexer KV in FP4, FP4 dot
+ * products; "DeepSeek-V4: Million-Token Context ...", "Where It Breaks":
+ * the FP4 QK indexer).  Keys are MXFP4: k_codes [batch][N][d_i/2] and
+ * k_exp [batch][N][d_i/32] as v4a_quantize_mxfp4 writes them.  The query of
+ * every indexer head (d_i values, F32 or BF16) is quantised to MXFP4 the same
+ * way inside the call, and
+ *     I(t,s) = sum_{j<heads_i} w[j] * ReLU(qhat_j . khat_s)
+ * with qhat, khat the decoded MXFP4 values: the products of e2m1 codes are
+ * exact, each 32-element block's partial sum is exact, and the blocks'
+ * powers of two are applied in fp32.  There is no per-entry k_scale.
+ * Otherwise arguments, results, workspace (v4a_workspace_size("topk", ...))
+ * and errors are those of v4a_index_scores / v4a_topk; d_i must be a
+ * multiple of 32, k_codes 16-byte and k_exp 4-byte aligned. */
+V4A_API v4a_status v4a_index_scores_mxfp4(const void* q_i, const float* w, const uint8_t* k_codes,
+                                          const uint8_t* k_exp, float* scores, int heads_i, int d_i,
+                                          v4a_dtype q_dtype, const v4a_shape* shape, void* stream);
+V4A_API v4a_status v4a_topk_mxfp4(const void* q_i, const float* w, const uint8_t* k_codes, const uint8_t* k_exp,
+                                  int32_t* idx_out, float* score_out, int heads_i, int d_i, v4a_dtype q_dtype,
+                                  void* workspace, size_t workspace_bytes, const v4a_shape* shape, void* stream);
 
 /* The same operation as v4a_topk for callers that cannot allocate device
  * memory: a plug-in inside a host framework that owns every device

@@ -84,6 +84,30 @@ def test_host_side_argument_errors(v4a):
     assert b"workspace" in L.v4a_last_error()
 
 
+def test_mxfp4_host_side_argument_errors(v4a):
+    L = v4a.lib
+    # quantiser: cols not a multiple of 32, then an unsupported dtype
+    assert L.v4a_quantize_mxfp4(16, 0, 4, 48, 16, 16, None) == 1
+    assert L.v4a_quantize_mxfp4(16, 2, 4, 64, 16, 16, None) == 2
+    assert L.v4a_quantize_mxfp4(None, 0, 0, 64, None, None, None) == 0  # nothing to do
+    shape = v4a.Shape(1, 1, 4, 64, 4, 8, 0, 64)
+    # MXFP4 keys go through the _mxfp4 calls only
+    assert L.v4a_index_scores(16, 16, 16, None, 16, 4, 64, 1, 3, ctypes.byref(shape), None) == 2
+    assert b"mxfp4" in L.v4a_last_error()
+    assert L.v4a_topk(16, 16, 16, None, 16, None, 4, 64, 1, 3, 256, 1 << 20, ctypes.byref(shape), None) == 2
+    # d_i not a multiple of 32; block exponents missing
+    assert L.v4a_index_scores_mxfp4(16, 16, 16, 16, 16, 4, 48, 1, ctypes.byref(shape), None) == 1
+    assert L.v4a_index_scores_mxfp4(16, 16, 16, None, 16, 4, 64, 1, ctypes.byref(shape), None) == 1
+    assert b"k_exp" in L.v4a_last_error()
+    assert L.v4a_topk_mxfp4(16, 16, 16, None, 16, None, 4, 64, 1, 256, 1 << 20, ctypes.byref(shape), None) == 1
+    # compress with MXFP4 output: channels must be a multiple of 32 and out_exp is required
+    io = v4a.CompressIO(16, 16, 16, None, 16, 1, 3, 64, 64, 16, 0, 16, 1)
+    assert L.v4a_compress(ctypes.byref(io), None, 1, 4, 4, None) == 1
+    io = v4a.CompressIO(16, 16, 16, None, 64, 1, 3, 256, 256, 64, 0, None, 2)
+    assert L.v4a_compress(ctypes.byref(io), None, 1, 4, 4, None) == 1
+    assert b"out_exp" in L.v4a_last_error()
+
+
 def test_workspace_sizes(v4a):
     assert v4a.v4a_workspace_size("nonsense", batch=1) == 0
     ws = v4a.v4a_workspace_size("topk", batch=4, m=4, k=1024, ctx_len=1 << 20, heads_i=16, d_i=128)

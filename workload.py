@@ -172,13 +172,17 @@ def fp32_l4096(seed: int | None = None):
                 token_kv=x, tok_pos0=0)
 
 
-def csa_decode(name: str, seed: int | None = None, with_tail: bool = True):
+def csa_decode(name: str, seed: int | None = None, with_tail: bool = True, key_fmt: str | None = None):
     """CSA decode at the last position t = L-1 of each sequence.  History
     entries and indexer keys for s < N-1 are drawn; with_tail additionally
     draws the raw inputs of the chunk that completes at t (its token rows are
     the last m window rows, plus gate logits and the indexer's token keys and
-    gates), whose entry N-1 the path compresses itself."""
-    c = CONFIGS[name]
+    gates), whose entry N-1 the path compresses itself.  key_fmt overrides the
+    stored format of the indexer keys (e.g. 'bf16' masters that a caller then
+    quantises to MXFP4); the draws are the same N(0,1) values either way."""
+    c = dict(CONFIGS[name])
+    if key_fmt is not None:
+        c["key_fmt"] = key_fmt
     g = _gen(c["seed"] if seed is None else seed)
     B, L, H, d, m = c["batch"], c["ctx_len"], c["heads"], c["d"], c["m"]
     N = L // m
