@@ -30,7 +30,10 @@
 //    "MXFP4 keys and queries" below.
 // Warp 0 loads key tiles into a shared-memory ring (4 x 32 KB for FP8, 2 x 64
 // KB for bf16), warp 1 issues the MMAs, warps 2-5 stage each row's B
-// operand, warps 6-9 run the epilogue.  CTAs take contiguous ranges of the
+// operand, warps 6-13 run the epilogue: two warps per TMEM sub-partition, one
+// per half of the tile, so each scheduler has two to switch between while one
+// waits on tensor memory.  Per-entry scales are fetched 8 tiles ahead (HBM
+// latency under load spans several tiles).  CTAs take contiguous ranges of the
 // flat (query row, tile) sequence; a run of one row's tiles inside a CTA's
 // range is a segment, with its own B buffer and histogram (both
 // double-buffered).  Every wait is bounded.
@@ -48,11 +51,17 @@ constexpr int kTileK = 256;              // entries per tile (two M=128 halves)
 constexpr int kHalf = 128;
 constexpr int kRingBytes = 131072;       // key-tile ring
 constexpr int kMaxStages = 8;
-constexpr int kThreads = 320;
+constexpr int kThreads = 448;              // producer, MMA, 4 staging / converter warps, 8 epilogue warps
+constexpr int kEpiFirst = 192;             // first epilogue thread (warp 6)
+constexpr int kEpiThreads = 256;           // warps 6-9 score half 0 of a tile, warps 10-13 half 1
+constexpr int kXAhead = 8;                 // tiles of per-entry scale words each epilogue thread fetches ahead
+constexpr int kXSlots = kXAhead + 1;
 constexpr int kHistBins = 4096;          // top 12 bits of the ordered score key
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxDStages = 4;
 constexpr int kQBufBytes = 16384;        // B operand of one segment: up to 128 rows of 128 B
+constexpr int kMxXAhead = 6;               // MXFP4: tiles of block exponents each staging thread fetches ahead
+constexpr int kMxXSlots = kMxXAhead + 1;
 
 template <bool FP8> struct Ring {
     static constexpr int kStageBytes = FP8 ? kTileK * kDI : kTileK * kDI * 2;
@@ -73,9 +82,12 @@ struct __align__(1024) IdxSmem {
     uint8_t q[2][kQBufBytes];                 // B operand per segment buffer
     float wq[2][128];                         // head weights of the G queries (times 2^-s for FP8)
     uint32_t hist[2][kHistBins];
-    float fq[2][4][32];                       // MXFP4: 2^X of each (block, head) of the query
+    union {
+        uint32_t xring[kXSlots][kEpiThreads];  // FP8: per-entry scales, per epilogue thread
+        uint32_t mx_xring[kMxXSlots][8][128];  // MXFP4: block-exponent words, per staging thread
+    };
     uint64_t k_full[kMaxStages], k_empty[kMaxStages], d_full[kMaxDStages], d_free[kMaxDStages], q_full[2], q_free[2],
-        a_full[2], a_free[2], ep_sync, drain;
+        sf_full[2], sf_free[2], ep_sync, drain;
     int abort_flag;
     uint32_t tmem_base;
 };
@@ -324,29 +336,64 @@ __device__ __forceinline__ float score_of(uint32_t taddr, const float* wq) {
             acc = fmaf(wq[h], fmaxf(fmaf(d2, 0x1p-10f, d1), 0.f), acc);
         }
     } else {
-        uint32_t r[64];
-        float d1[32];
-        tc::tmem_ld_x64(taddr, r);  // hi | lo of 32 heads
-        tc::tmem_ld_wait();
+        // 16 heads at a time: pieces hi | lo | hi' | lo' of heads 16 hg .. 16 hg + 15
 #pragma unroll
-        for (int h = 0; h < 32; ++h) d1[h] = __uint_as_float(r[h]) + __uint_as_float(r[32 + h]);
-        tc::tmem_ld_x64(taddr + 64, r);  // hi' | lo'
-        tc::tmem_ld_wait();
+        for (int hg = 0; hg < 2; ++hg) {
+            uint32_t p4[4][16];
 #pragma unroll
-        for (int h = 0; h < 32; ++h) {
-            const float d2 = __uint_as_float(r[h]) + __uint_as_float(r[32 + h]);
-            acc = fmaf(wq[h], fmaxf(fmaf(d2, 0x1p-10f, d1[h]), 0.f), acc);
+            for (int p = 0; p < 4; ++p) tc::tmem_ld_x16(taddr + 32 * p + 16 * hg, p4[p]);
+            tc::tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const float d1 = __uint_as_float(p4[0][i]) + __uint_as_float(p4[1][i]);
+                const float d2 = __uint_as_float(p4[2][i]) + __uint_as_float(p4[3][i]);
+                acc = fmaf(wq[16 * hg + i], fmaxf(fmaf(d2, 0x1p-10f, d1), 0.f), acc);
+            }
         }
     }
     return acc;
 }
 
-// warps 6-9: per tile the scores of entries r and r + 128 (r = this thread's TMEM lane) for each
-// query of the group, their histogram counts (single queries only) and stores
+// This epilogue thread's per-entry scale word (FP8 scale, MXFP4 exponents) for every tile of its
+// range, fetched kXAhead tiles ahead with 4-byte cp.async into a ring of shared memory only this
+// thread touches: HBM latency under load (2-4 us) is several tiles long, so a load issued one tile
+// ahead would stall the epilogue.  One commit group per tile, so wait_group<kXAhead> leaves the
+// current tile's word landed.
+struct XPrefetch {
+    ICursor cur;
+    long long f, f0, f1;
+    const uint32_t* src;  // [B][N] words
+    int et, hf, r;
+    __device__ XPrefetch(long long f0_, long long f1_, const IdxTcArgs& a, int G, const uint32_t* src_, int et_,
+                         int hf_, int r_)
+        : cur(f0_, a, G), f(f0_), f0(f0_), f1(f1_), src(src_), et(et_), hf(hf_), r(r_) {}
+    __device__ __forceinline__ void issue(IdxSmem& sm, const IdxTcArgs& a) {
+        if (f < f1) {
+            const long long e = (long long)cur.ti * kTileK + kHalf * hf + r;
+            if (e < a.n_ent) tc::cp_async_4(&sm.xring[(int)((f - f0) % kXSlots)][et], src + (long long)cur.bat * a.n_ent + e);
+            cur.next(a);
+            ++f;
+        }
+        tc::cp_async_commit();
+    }
+    __device__ __forceinline__ void start(IdxSmem& sm, const IdxTcArgs& a) {
+        for (int i = 0; i < kXAhead; ++i) issue(sm, a);
+    }
+    // the word of tile jt (local index), once its copy has landed; issues the copy kXAhead tiles on
+    __device__ __forceinline__ uint32_t take(IdxSmem& sm, const IdxTcArgs& a, int jt) {
+        issue(sm, a);
+        tc::cp_async_wait<kXAhead>();
+        return sm.xring[jt % kXSlots][et];
+    }
+};
+
+// warps 6-13: per tile the scores of entry 128 hf + r (r = this thread's TMEM lane, hf = which four
+// warps) for each query of the group, their histogram counts (single queries only) and stores
 template <bool FP8, int NP, int G>
 __device__ void idx_epilogue(IdxSmem& sm, const IdxTcArgs& a, uint32_t tmem, long long f0, long long f1) {
     constexpr int kDS = Acc<FP8, NP, G>::kStages, kN = Acc<FP8, NP, G>::kN, kNq = Acc<FP8, NP, G>::kNq;
-    const int et = threadIdx.x - 192;
+    const int et = threadIdx.x - kEpiFirst;
+    const int hf = et >> 7;
     const int sub = (threadIdx.x >> 5) & 3;
     const int r = 32 * sub + (threadIdx.x & 31);
     const uint32_t lane_addr = (uint32_t)(32 * sub) << 16;
@@ -357,16 +404,8 @@ __device__ void idx_epilogue(IdxSmem& sm, const IdxTcArgs& a, uint32_t tmem, lon
 #pragma unroll
     for (int g = 0; g < G; ++g) nv[g] = 0;
     ICursor cur(f0, a, G);
-    // scales of the current tile's two entries, loaded one tile ahead
-    auto scales_of = [&](const ICursor& c, float (&sc)[2]) {
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-            const long long e = (long long)c.ti * kTileK + kHalf * hf + r;
-            sc[hf] = e < a.n_ent ? __ldg(a.kscale + (long long)c.bat * a.n_ent + e) : 1.f;
-        }
-    };
-    float sc_cur[2] = {1.f, 1.f};
-    if (FP8) scales_of(cur, sc_cur);
+    XPrefetch xp(f0, f1, a, G, reinterpret_cast<const uint32_t*>(a.kscale), et, hf, r);
+    if (FP8) xp.start(sm, a);
     for (long long f = f0; f < f1; ++f) {
         if (warp_aborted(sm)) { ok = false; break; }
         const int jt = (int)(f - f0), sd = jt % kDS;
@@ -384,39 +423,29 @@ __device__ void idx_epilogue(IdxSmem& sm, const IdxTcArgs& a, uint32_t tmem, lon
         const bool seg_end = (f == f1 - 1) || (cur.ti == a.tiles_per_row - 1);
         const int ti = cur.ti, q0t = cur.q0, row = cur.bat * a.n_q + cur.q0;  // row: the group's first query
         cur.next(a);
-        float sc_next[2] = {1.f, 1.f};
-        if (FP8 && f + 1 < f1) scales_of(cur, sc_next);
         if (!warp_wait(&sm.d_full[sd], (jt / kDS) & 1)) { ok = false; break; }
         tc::tc_fence_after();
-        float acc[G][2];
+        float acc[G];
 #pragma unroll
         for (int g = 0; g < G; ++g)
-#pragma unroll
-            for (int hf = 0; hf < 2; ++hf)
-                acc[g][hf] = score_of<FP8, NP>(tmem + lane_addr + Acc<FP8, NP, G>::kCols * sd + kN * hf + kNq * g,
-                                               sm.wq[b] + NP * g);
+            acc[g] = score_of<FP8, NP>(tmem + lane_addr + Acc<FP8, NP, G>::kCols * sd + kN * hf + kNq * g,
+                                       sm.wq[b] + NP * g);
         tc::tc_fence_before();
         tc::mbar_arrive(&sm.d_free[sd]);
+        const float sc_e = FP8 ? __uint_as_float(xp.take(sm, a, jt)) : 1.f;
+        const long long e = (long long)ti * kTileK + kHalf * hf + r;
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-            if (q0t + g >= a.n_q) continue;  // past the last query of the sequence
-#pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                const long long e = (long long)ti * kTileK + kHalf * hf + r;
-                if (e < a.n_ent) {
-                    float sc = -INFINITY;
-                    if (e < nv[g]) {
-                        float v = acc[g][hf];
-                        if (FP8) v *= sc_cur[hf];
-                        sc = v + 0.0f;
-                        if (G == 1 && a.hist) atomicAdd(&sm.hist[b][float_to_ordered(sc) >> 20], 1u);
-                    }
-                    srow0[(long long)g * a.n_ent + e] = sc;
-                }
+            if (q0t + g >= a.n_q || e >= a.n_ent) continue;  // past the last query of the sequence / entry
+            float sc = -INFINITY;
+            if (e < nv[g]) {
+                float v = acc[g];
+                if (FP8) v *= sc_e;
+                sc = v + 0.0f;
+                if (G == 1 && a.hist) atomicAdd(&sm.hist[b][float_to_ordered(sc) >> 20], 1u);
             }
+            srow0[(long long)g * a.n_ent + e] = sc;
         }
-        sc_cur[0] = sc_next[0];
-        sc_cur[1] = sc_next[1];
         if (seg_end) {
             tc::mbar_arrive(&sm.q_free[b]);  // done with wq[b]
             if (G == 1 && a.hist) {
@@ -424,7 +453,7 @@ __device__ void idx_epilogue(IdxSmem& sm, const IdxTcArgs& a, uint32_t tmem, lon
                 tc::mbar_arrive(&sm.ep_sync);
                 if (!warp_wait(&sm.ep_sync, nsync++ & 1)) { ok = false; break; }
                 uint32_t* gh = a.hist + (long long)row * kHistBins;
-                for (int i = et; i < kHistBins; i += 128) {
+                for (int i = et; i < kHistBins; i += kEpiThreads) {
                     const uint32_t v = sm.hist[b][i];
                     if (v) {
                         atomicAdd(gh + i, v);
@@ -434,6 +463,7 @@ __device__ void idx_epilogue(IdxSmem& sm, const IdxTcArgs& a, uint32_t tmem, lon
             }
         }
     }
+    tc::cp_async_wait<0>();  // no copy into shared memory may be in flight at exit
     if (!ok) idx_fault(sm, a);
 }
 
@@ -450,13 +480,13 @@ __global__ void __launch_bounds__(kThreads, 1) index_score_tc_kernel(const __gri
         }
         for (int i = 0; i < Acc<FP8, NP, G>::kStages; ++i) {
             tc::mbar_init(&sm.d_full[i], 1);
-            tc::mbar_init(&sm.d_free[i], 128);
+            tc::mbar_init(&sm.d_free[i], kEpiThreads);
         }
         for (int i = 0; i < 2; ++i) {
             tc::mbar_init(&sm.q_full[i], 128);
-            tc::mbar_init(&sm.q_free[i], 1 + 128);  // the MMAs' commit + every epilogue thread
+            tc::mbar_init(&sm.q_free[i], 1 + kEpiThreads);  // the MMAs' commit + every epilogue thread
         }
-        tc::mbar_init(&sm.ep_sync, 128);
+        tc::mbar_init(&sm.ep_sync, kEpiThreads);
         tc::mbar_init(&sm.drain, 1);
         sm.abort_flag = 0;
         tc::fence_barrier_init();
@@ -488,44 +518,35 @@ __global__ void __launch_bounds__(kThreads, 1) index_score_tc_kernel(const __gri
 }
 
 // ---------------------------------------------------------------------
-// MXFP4 keys and queries (FP4 dot products)
+// MXFP4 keys and queries: FP4 dot products on the block-scaled tensor cores
 // ---------------------------------------------------------------------
-// Key rows are 64 bytes of packed e2m1 codes (plus 4 E8M0 block exponents in a
-// separate array).  TMA brings 256-entry tiles (16 KB, 64-byte swizzle) into
-// 32 KB stages of two tiles.  Warps 2-5 turn each tile's codes into the MMA's
-// A operand in tensor memory: an e2m1 code s.e1e0.f becomes the e4m3 byte
-// s.000.e1e0.f.00, whose value is exactly the e2m1 value times 2^-6 (normal
-// codes keep their exponent relative to bias 7; the subnormal e2m1 0.5 lands
-// on the e4m3 subnormal 4/8 * 2^-6), so two shifts and two masks per word.
-// The 8 codes of a 32-bit code word go out as two words, even elements then
-// odd ones; the query is staged with the same permutation, which leaves every
-// 32-element block in its own 8 columns.  One K = 32 MMA per (half, block)
-// writes that block's partial dots into its own accumulator: products of
-// e2m1 values are multiples of 1/4, so each block sum is exact, and the
-// epilogue applies the two blocks' powers of two (2^Xk * 2^Xq, and 2^12 for
-// the two 2^-6) before the ReLU and the head weights.
+// Key rows are 64 bytes of packed e2m1 codes; their 4 E8M0 block exponents
+// live in a separate array, one 32-bit word per entry whose byte j scales
+// elements 32j .. 32j+31.  TMA brings 256-entry tiles (16 KB, 64-byte
+// swizzle) into 32 KB stages of two tiles, and those tiles ARE the MMA's A
+// operand: tcgen05 kind::mxf4 (block32) reads packed e2m1 from shared memory
+// and applies one E8M0 scale per 32 K-elements from tensor memory, so a
+// 256-entry tile is 4 MMAs (2 halves x K = 2 x 64) with f32 accumulation.
+// The scale words need no repacking: row m of a 128-row half reads the word
+// at lane m % 32 (of every sub-partition), column m / 32, bytes 0-1 for
+// K 0..63 and bytes 2-3 for K 64..127.  Warps 2-5 (one per sub-partition)
+// write each tile's words there with tcgen05.st, from a ring of 4-byte
+// cp.async copies fetched kMxXAhead tiles ahead; per query they also quantise
+// q to MXFP4 (the B operand, same layout) and write its scale words.  The
+// epilogue is the bf16-key one: each accumulator column is already
+// q_h . k_s with both block scales applied.
 
 constexpr int kMxTileBytes = kTileK * 64;                 // packed codes of one 256-entry tile
 constexpr int kMxStageBytes = 2 * kMxTileBytes;           // two tiles per stage
 constexpr int kMxStages = kRingBytes / kMxStageBytes;     // 4
-constexpr uint32_t kMxACols = 64;                         // A operand of one tile: 2 halves x 32 columns
-constexpr uint32_t kMxABase = 0;                          // two A slots at columns [0, 128)
+constexpr uint32_t kMxSfaCol = 256;                       // two A-scale slots of 8 columns, 16 apart
+constexpr uint32_t kMxSfbCol = 320;                       // two B-scale columns (query buffers), 16 apart
 template <int NP> struct MxAcc {
-    static constexpr uint32_t kCols = 2 * 4 * NP;         // per tile: 2 halves x 4 blocks x NP heads
-    static constexpr uint32_t kBase = 2 * kMxACols;
-    static constexpr int kStages =
-        (int)((kTmemCols - kBase) / kCols) < kMaxDStages ? (int)((kTmemCols - kBase) / kCols) : kMaxDStages;
-    static_assert(kStages >= 1, "accumulators exceed tensor memory");
+    static constexpr uint32_t kCols = 2 * NP;             // per tile: 2 halves x NP heads
+    static constexpr int kStages = kMaxDStages;
+    static_assert(kStages * kCols <= kMxSfaCol, "accumulators overlap the scale columns");
 };
 static_assert(kMxStages <= kMaxStages, "ring stages");
-
-// even elements (low nibbles) / odd elements (high nibbles) of 8 packed e2m1 codes -> 4 e4m3 bytes
-__device__ __forceinline__ uint32_t e2m1x4_even_to_e4m3(uint32_t cw) {
-    return ((cw << 2) & 0x1C1C1C1Cu) | ((cw << 4) & 0x80808080u);
-}
-__device__ __forceinline__ uint32_t e2m1x4_odd_to_e4m3(uint32_t cw) {
-    return ((cw >> 2) & 0x1C1C1C1Cu) | (cw & 0x80808080u);
-}
 
 __device__ void mx_producer(IdxSmem& sm, const IdxTcArgs& a, const CUtensorMap* kmap, long long f0, long long f1) {
     ICursor cur(f0, a, 1);
@@ -553,34 +574,38 @@ template <int NP>
 __device__ void mx_mma(IdxSmem& sm, const IdxTcArgs& a, uint32_t tmem, long long f0, long long f1) {
     using Acc = MxAcc<NP>;
     constexpr int kDS = Acc::kStages;
-    constexpr uint32_t idesc = tc::idesc_e4m3(128, NP);
     bool ok = true;
     int seg = 0, b = 0;
-    uint64_t qd = 0;
+    uint32_t qaddr = 0;
     ICursor cur(f0, a, 1);
     for (long long f = f0; f < f1; ++f, cur.next(a)) {
         if (aborted(sm)) { ok = false; break; }
         const long long jt = f - f0;
-        const int slot = (int)(jt & 1), sd = (int)(jt % kDS);
+        const int st = (int)((jt >> 1) % kMxStages), u = (int)(jt & 1), slot = (int)(jt & 1), sd = (int)(jt % kDS);
         if (f == f0 || cur.ti == 0) {
             b = seg & 1;
             if (!tc::mbar_wait(&sm.q_full[b], (seg >> 1) & 1)) { ok = false; break; }
-            qd = tc::sw128_desc(tc::smem_u32(sm.q[b]), 16, 1024);
+            qaddr = tc::smem_u32(sm.q[b]);
             ++seg;
         }
         const bool seg_end = (f == f1 - 1) || (cur.ti == a.tiles_per_row - 1);
-        if (!tc::mbar_wait(&sm.a_full[slot], (uint32_t)(jt >> 1) & 1)) { ok = false; break; }
+        if (u == 0 && !tc::mbar_wait(&sm.k_full[st], (uint32_t)((jt >> 1) / kMxStages) & 1)) { ok = false; break; }
+        if (!tc::mbar_wait(&sm.sf_full[slot], (uint32_t)(jt >> 1) & 1)) { ok = false; break; }
         if (jt >= kDS && !tc::mbar_wait(&sm.d_free[sd], (uint32_t)((jt / kDS) - 1) & 1)) { ok = false; break; }
         tc::tc_fence_after();
+        const uint32_t tile = tc::smem_u32(sm.ring + st * kMxStageBytes + u * kMxTileBytes);
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf)
 #pragma unroll
-            for (int blk = 0; blk < 4; ++blk)
-                tc::mma_f8_ts(tmem + Acc::kBase + Acc::kCols * sd + (4 * hf + blk) * NP,
-                              tmem + kMxABase + slot * kMxACols + 32 * hf + 8 * blk,
-                              qd + (uint64_t)((32 * blk) >> 4), idesc, 0u);
-        tc::mma_commit(&sm.a_free[slot]);
+            for (int kk = 0; kk < 2; ++kk)
+                tc::mma_mxf4(tmem + Acc::kCols * sd + NP * hf,
+                             tc::sw64_desc(tile + hf * kHalf * 64 + 32 * kk), tc::sw64_desc(qaddr + 32 * kk),
+                             tc::idesc_mxf4(128, NP, 2 * kk, 2 * kk),
+                             (tmem + kMxSfaCol + 16 * slot + 4 * hf) | ((uint32_t)(2 * kk) << 30),
+                             (tmem + kMxSfbCol + 16 * b) | ((uint32_t)(2 * kk) << 30), kk ? 1u : 0u);
+        tc::mma_commit(&sm.sf_free[slot]);
         tc::mma_commit(&sm.d_full[sd]);
+        if (u == 1 || f == f1 - 1) tc::mma_commit(&sm.k_empty[st]);
         if (seg_end) tc::mma_commit(&sm.q_free[b]);
     }
     if (!ok) idx_fault(sm, a);
@@ -588,11 +613,12 @@ __device__ void mx_mma(IdxSmem& sm, const IdxTcArgs& a, uint32_t tmem, long long
     tc::mbar_wait(&sm.drain, 0);
 }
 
-// B operand of one query (NP rows of 128 e4m3 bytes, K-major, 128-byte swizzle) from its MXFP4
-// quantisation, with the even/odd element order of the keys; fq = 2^X per (block, head) and the
-// head weights times 2^12.  A half-warp takes one head, lane l its elements 8l .. 8l+7.
+// Query of one segment: its B operand (NP rows of 64 bytes of packed e2m1, 64-byte swizzle), its
+// scale words in tensor memory and the head weights.  A half-warp quantises one head, lane l
+// elements 8l .. 8l+7; then every lane h (< NP) of every staging warp writes head h's 4 block
+// exponents to its sub-partition's copy of the B scales.
 template <int NP>
-__device__ void stage_query_mx(IdxSmem& sm, const IdxTcArgs& a, int bat, int qj, int b, int ct) {
+__device__ void stage_query_mx(IdxSmem& sm, const IdxTcArgs& a, uint32_t tmem, int bat, int qj, int b, int ct) {
     const int warp = ct >> 5, lane = ct & 31, l = lane & 15;
     const long long row = (long long)bat * a.n_q + qj;
     for (int h = 2 * warp + (lane >> 4); h < NP; h += 8) {  // NP is a multiple of 8: whole warps iterate
@@ -606,24 +632,62 @@ __device__ void stage_query_mx(IdxSmem& sm, const IdxTcArgs& a, int bat, int qj,
         }
         int x;
         const uint32_t cw = mx_quantize8(v, &x);  // lanes 4k .. 4k+3 of the half-warp share block k
-        const int k = 8 * l;
-        uint8_t* dst = sm.q[b] + (h >> 3) * 1024 + (h & 7) * 128 + ((((k >> 4) ^ (h & 7))) << 4) + (k & 15);
-        *reinterpret_cast<uint2*>(dst) = make_uint2(e2m1x4_even_to_e4m3(cw), e2m1x4_odd_to_e4m3(cw));
-        if ((l & 3) == 0) sm.fq[b][l >> 2][h] = live ? e8m0_value((uint32_t)(x + 127)) : 0.f;
-        if (l == 0) sm.wq[b][h] = live ? a.w[row * a.heads_i + h] * 4096.0f : 0.f;
+        const int j = 4 * l;                       // byte of the row
+        *reinterpret_cast<uint32_t*>(sm.q[b] + h * 64 + ((((j >> 4) ^ ((h >> 1) & 3))) << 4) + (j & 15)) = cw;
+        if (l == 0) sm.wq[b][h] = live ? a.w[row * a.heads_i + h] : 0.f;
     }
+    // B scale words: lane h of this warp's sub-partition, column kMxSfbCol + 16 b
+    uint32_t word = 0x7f7f7f7fu;  // 2^0 for rows past the last head (their codes are 0)
+    if (lane < NP && lane < a.heads_i) {
+        const __nv_bfloat16* qp = a.q + (row * a.heads_i + lane) * kDI;
+        word = 0;
+#pragma unroll
+        for (int blk = 0; blk < 4; ++blk) {
+            float am = 0.f;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                float v[8];
+                Vec8<__nv_bfloat16>::load_nc(qp + 32 * blk + 8 * c, v);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) am = fmaxf(am, fabsf(v[i]));
+            }
+            word |= (uint32_t)(mx_block_exp(am) + 127) << (8 * blk);
+        }
+    }
+    const int sub = (threadIdx.x >> 5) & 3;
+    tc::tmem_st_x1(tmem + ((uint32_t)(32 * sub) << 16) + kMxSfbCol + 16 * b, word);
+    tc::tmem_st_wait();
 }
 
-// warps 2-5: per segment the query's B operand; per tile the keys' A operand in tensor memory
-// (thread = TMEM lane r: entries r and r + 128 of the tile)
+// warps 2-5: per segment the query (B operand and scales); per tile the keys' scale words (A
+// scales) in tensor memory: thread (sub-partition p, lane t) writes, in its sub-partition, column
+// 16 slot + 4 hf + c the word of entry 128 hf + 32 c + t
 template <int NP>
-__device__ void mx_convert(IdxSmem& sm, const IdxTcArgs& a, uint32_t tmem, long long f0, long long f1) {
+__device__ void mx_stage(IdxSmem& sm, const IdxTcArgs& a, uint32_t tmem, long long f0, long long f1) {
     const int ct = threadIdx.x - 64;
+    const int lane = threadIdx.x & 31;
     const int sub = (threadIdx.x >> 5) & 3;
-    const int r = 32 * sub + (threadIdx.x & 31);
     const uint32_t lane_addr = (uint32_t)(32 * sub) << 16;
+    const uint32_t* src = reinterpret_cast<const uint32_t*>(a.kexp);
     bool ok = true;
     int seg = 0;
+    // block-exponent words fetched kMxXAhead tiles ahead (one commit group per tile)
+    ICursor pre(f0, a, 1);
+    long long fp = f0;
+    auto prefetch = [&]() {
+        if (fp < f1) {
+            const int slot = (int)((fp - f0) % kMxXSlots);
+#pragma unroll
+            for (int w = 0; w < 8; ++w) {
+                const long long e = (long long)pre.ti * kTileK + kHalf * (w >> 2) + 32 * (w & 3) + lane;
+                if (e < a.n_ent) tc::cp_async_4(&sm.mx_xring[slot][w][ct], src + (long long)pre.bat * a.n_ent + e);
+            }
+            pre.next(a);
+            ++fp;
+        }
+        tc::cp_async_commit();
+    };
+    for (int i = 0; i < kMxXAhead; ++i) prefetch();
     ICursor cur(f0, a, 1);
     for (long long f = f0; f < f1; ++f, cur.next(a)) {
         if (warp_aborted(sm)) { ok = false; break; }
@@ -631,88 +695,37 @@ __device__ void mx_convert(IdxSmem& sm, const IdxTcArgs& a, uint32_t tmem, long 
         if (f == f0 || cur.ti == 0) {
             const int b = seg & 1;
             if (seg >= 2 && !warp_wait(&sm.q_free[b], ((seg >> 1) - 1) & 1)) { ok = false; break; }
-            stage_query_mx<NP>(sm, a, cur.bat, cur.q0, b, ct);
+            stage_query_mx<NP>(sm, a, tmem, cur.bat, cur.q0, b, ct);
             tc::fence_proxy_async();
+            tc::tc_fence_before();
             tc::mbar_arrive(&sm.q_full[b]);
             ++seg;
         }
-        const int st = (int)((jt >> 1) % kMxStages), u = (int)(jt & 1), slot = (int)(jt & 1);
-        if (u == 0 && !warp_wait(&sm.k_full[st], (uint32_t)((jt >> 1) / kMxStages) & 1)) { ok = false; break; }
-        if (jt >= 2 && !warp_wait(&sm.a_free[slot], (uint32_t)((jt >> 1) - 1) & 1)) { ok = false; break; }
-        const uint8_t* tile = sm.ring + st * kMxStageBytes + u * kMxTileBytes;
-        uint32_t wv[64];
+        prefetch();  // tile f + kMxXAhead
+        const int slot = (int)(jt & 1);
+        if (jt >= 2 && !warp_wait(&sm.sf_free[slot], (uint32_t)((jt >> 1) - 1) & 1)) { ok = false; break; }
+        tc::cp_async_wait<kMxXAhead>();
+        const int xs = (int)(jt % kMxXSlots);
+        uint32_t wv[8];
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-            const int y = hf * kHalf + r;
-            const uint8_t* rowp = tile + y * 64;
-            const int sw = (y >> 1) & 3;  // 64-byte swizzle: 16-byte chunk c of row y sits at chunk c ^ sw
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const uint4 v = *reinterpret_cast<const uint4*>(rowp + ((c ^ sw) << 4));
-                const uint32_t cw[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    wv[32 * hf + 8 * c + 2 * i] = e2m1x4_even_to_e4m3(cw[i]);
-                    wv[32 * hf + 8 * c + 2 * i + 1] = e2m1x4_odd_to_e4m3(cw[i]);
-                }
-            }
-        }
-        // the stage's codes are in registers: release it after its second tile (or the range's last)
-        if (u == 1 || f == f1 - 1) tc::mbar_arrive(&sm.k_empty[st]);
-        tc::tmem_st_x64(tmem + lane_addr + kMxABase + slot * kMxACols, wv);
+        for (int w = 0; w < 8; ++w) wv[w] = sm.mx_xring[xs][w][ct];
+        tc::tc_fence_after();
+        tc::tmem_st_x8(tmem + lane_addr + kMxSfaCol + 16 * slot, wv);
         tc::tmem_st_wait();
         tc::tc_fence_before();
-        tc::mbar_arrive(&sm.a_full[slot]);
+        tc::mbar_arrive(&sm.sf_full[slot]);
     }
+    tc::cp_async_wait<0>();  // no copy into shared memory may be in flight at exit
     if (!ok) idx_fault(sm, a);
 }
 
-// one entry's score from its 4 x NP block dots (columns blk * NP + h of this thread's lane)
-template <int NP>
-__device__ __forceinline__ float mx_score(uint32_t taddr, const float (*fq)[32], const float* wq, uint32_t ex) {
-    const float k0 = e8m0_value(ex & 0xffu), k1 = e8m0_value((ex >> 8) & 0xffu), k2 = e8m0_value((ex >> 16) & 0xffu),
-                k3 = e8m0_value(ex >> 24);
-    float acc = 0.f;
-    uint32_t r[64];
-    if constexpr (NP == 16) {
-        tc::tmem_ld_x64(taddr, r);
-        tc::tmem_ld_wait();
-#pragma unroll
-        for (int h = 0; h < 16; ++h) {
-            float dot = __uint_as_float(r[h]) * fq[0][h] * k0;
-            dot = fmaf(__uint_as_float(r[16 + h]) * fq[1][h], k1, dot);
-            dot = fmaf(__uint_as_float(r[32 + h]) * fq[2][h], k2, dot);
-            dot = fmaf(__uint_as_float(r[48 + h]) * fq[3][h], k3, dot);
-            acc = fmaf(wq[h], fmaxf(dot, 0.f), acc);
-        }
-    } else {
-        // 16 heads at a time: columns blk * 32 + 16 * hg + (0 .. 15)
-#pragma unroll
-        for (int hg = 0; hg < 2; ++hg) {
-            uint32_t (&q4)[4][16] = *reinterpret_cast<uint32_t(*)[4][16]>(r);
-#pragma unroll
-            for (int blk = 0; blk < 4; ++blk) tc::tmem_ld_x16(taddr + 32 * blk + 16 * hg, q4[blk]);
-            tc::tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const int h = 16 * hg + i;
-                float dot = __uint_as_float(q4[0][i]) * fq[0][h] * k0;
-                dot = fmaf(__uint_as_float(q4[1][i]) * fq[1][h], k1, dot);
-                dot = fmaf(__uint_as_float(q4[2][i]) * fq[2][h], k2, dot);
-                dot = fmaf(__uint_as_float(q4[3][i]) * fq[3][h], k3, dot);
-                acc = fmaf(wq[h], fmaxf(dot, 0.f), acc);
-            }
-        }
-    }
-    return acc;
-}
-
-// warps 6-9: scores of entries r and r + 128 of each tile, histogram counts and stores
+// warps 6-13: the score of entry 128 hf + r of each tile, histogram counts and stores
 template <int NP>
 __device__ void mx_epilogue(IdxSmem& sm, const IdxTcArgs& a, uint32_t tmem, long long f0, long long f1) {
     using Acc = MxAcc<NP>;
     constexpr int kDS = Acc::kStages;
-    const int et = threadIdx.x - 192;
+    const int et = threadIdx.x - kEpiFirst;
+    const int hf = et >> 7;
     const int sub = (threadIdx.x >> 5) & 3;
     const int r = 32 * sub + (threadIdx.x & 31);
     const uint32_t lane_addr = (uint32_t)(32 * sub) << 16;
@@ -721,17 +734,6 @@ __device__ void mx_epilogue(IdxSmem& sm, const IdxTcArgs& a, uint32_t tmem, long
     long long nv = 0;
     float* srow = nullptr;
     ICursor cur(f0, a, 1);
-    // block exponents of the current tile's two entries, loaded one tile ahead
-    auto exps_of = [&](const ICursor& c, uint32_t (&ex)[2]) {
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-            const long long e = (long long)c.ti * kTileK + kHalf * hf + r;
-            ex[hf] = e < a.n_ent ? __ldg(reinterpret_cast<const uint32_t*>(a.kexp) + (long long)c.bat * a.n_ent + e)
-                                 : 0x7f7f7f7fu;
-        }
-    };
-    uint32_t ex_cur[2];
-    exps_of(cur, ex_cur);
     for (long long f = f0; f < f1; ++f) {
         if (warp_aborted(sm)) { ok = false; break; }
         const int jt = (int)(f - f0), sd = jt % kDS;
@@ -745,38 +747,27 @@ __device__ void mx_epilogue(IdxSmem& sm, const IdxTcArgs& a, uint32_t tmem, long
         const bool seg_end = (f == f1 - 1) || (cur.ti == a.tiles_per_row - 1);
         const int ti = cur.ti, row = cur.bat * a.n_q + cur.q0;
         cur.next(a);
-        uint32_t ex_next[2] = {0x7f7f7f7fu, 0x7f7f7f7fu};
-        if (f + 1 < f1) exps_of(cur, ex_next);
         if (!warp_wait(&sm.d_full[sd], (jt / kDS) & 1)) { ok = false; break; }
         tc::tc_fence_after();
-        float acc[2];
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf)
-            acc[hf] = mx_score<NP>(tmem + lane_addr + Acc::kBase + Acc::kCols * sd + 4 * NP * hf, sm.fq[b], sm.wq[b],
-                                   ex_cur[hf]);
+        const float acc = score_of<false, NP>(tmem + lane_addr + Acc::kCols * sd + NP * hf, sm.wq[b]);
         tc::tc_fence_before();
         tc::mbar_arrive(&sm.d_free[sd]);
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-            const long long e = (long long)ti * kTileK + kHalf * hf + r;
-            if (e < a.n_ent) {
-                float sc = -INFINITY;
-                if (e < nv) {
-                    sc = acc[hf] + 0.0f;
-                    if (a.hist) atomicAdd(&sm.hist[b][float_to_ordered(sc) >> 20], 1u);
-                }
-                srow[e] = sc;
+        const long long e = (long long)ti * kTileK + kHalf * hf + r;
+        if (e < a.n_ent) {
+            float sc = -INFINITY;
+            if (e < nv) {
+                sc = acc + 0.0f;
+                if (a.hist) atomicAdd(&sm.hist[b][float_to_ordered(sc) >> 20], 1u);
             }
+            srow[e] = sc;
         }
-        ex_cur[0] = ex_next[0];
-        ex_cur[1] = ex_next[1];
         if (seg_end) {
-            tc::mbar_arrive(&sm.q_free[b]);  // done with wq[b] and fq[b]
+            tc::mbar_arrive(&sm.q_free[b]);  // done with wq[b]
             if (a.hist) {
                 tc::mbar_arrive(&sm.ep_sync);
                 if (!warp_wait(&sm.ep_sync, nsync++ & 1)) { ok = false; break; }
                 uint32_t* gh = a.hist + (long long)row * kHistBins;
-                for (int i = et; i < kHistBins; i += 128) {
+                for (int i = et; i < kHistBins; i += kEpiThreads) {
                     const uint32_t v = sm.hist[b][i];
                     if (v) {
                         atomicAdd(gh + i, v);
@@ -798,19 +789,19 @@ __global__ void __launch_bounds__(kThreads, 1) index_score_mx_kernel(const __gri
     if (threadIdx.x == 0) {
         for (int i = 0; i < kMxStages; ++i) {
             tc::mbar_init(&sm.k_full[i], 1);
-            tc::mbar_init(&sm.k_empty[i], 128);  // every converter thread
+            tc::mbar_init(&sm.k_empty[i], 1);
         }
         for (int i = 0; i < MxAcc<NP>::kStages; ++i) {
             tc::mbar_init(&sm.d_full[i], 1);
-            tc::mbar_init(&sm.d_free[i], 128);
+            tc::mbar_init(&sm.d_free[i], kEpiThreads);
         }
         for (int i = 0; i < 2; ++i) {
             tc::mbar_init(&sm.q_full[i], 128);
-            tc::mbar_init(&sm.q_free[i], 1 + 128);
-            tc::mbar_init(&sm.a_full[i], 128);
-            tc::mbar_init(&sm.a_free[i], 1);
+            tc::mbar_init(&sm.q_free[i], 1 + kEpiThreads);
+            tc::mbar_init(&sm.sf_full[i], 128);
+            tc::mbar_init(&sm.sf_free[i], 1);
         }
-        tc::mbar_init(&sm.ep_sync, 128);
+        tc::mbar_init(&sm.ep_sync, kEpiThreads);
         tc::mbar_init(&sm.drain, 1);
         sm.abort_flag = 0;
         tc::fence_barrier_init();
@@ -827,7 +818,7 @@ __global__ void __launch_bounds__(kThreads, 1) index_score_mx_kernel(const __gri
     } else if (warp == 1) {
         if (lane == 0) mx_mma<NP>(sm, a, tmem, f0, f1);
     } else if (warp < 6) {
-        mx_convert<NP>(sm, a, tmem, f0, f1);
+        mx_stage<NP>(sm, a, tmem, f0, f1);
     } else {
         mx_epilogue<NP>(sm, a, tmem, f0, f1);
     }

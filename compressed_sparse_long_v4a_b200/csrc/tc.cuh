@@ -88,6 +88,14 @@ __device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
 __device__ __forceinline__ void cp_async_16(void* dst, const void* src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
 }
+// 4-byte copy global -> shared through L1 (completion tracked per thread by commit / wait groups)
+__device__ __forceinline__ void cp_async_4(void* dst, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// wait until at most N of this thread's committed groups are still in flight
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 // arrive on `bar` once this thread's earlier cp.async copies have landed (counts against the init count)
 __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
@@ -113,17 +121,6 @@ __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64
         "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
         " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-// D[tmem] (+)= A[tmem] * B[smem desc]^T, kind::f8f6f4, issued by one thread.  A is read from
-// tensor memory: lane = row, each 32-bit column holds 4 consecutive K elements, the lowest in the
-// low byte (measured on B200).
-__device__ __forceinline__ void mma_f8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                          uint32_t accumulate) {
-    asm volatile(
-        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-        " tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
 // arrive on `bar` when every MMA issued so far by this thread has completed
@@ -206,6 +203,47 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uin
     d |= (uint64_t)1 << 46;  // descriptor version for tcgen05
     d |= (uint64_t)2 << 61;  // 128-byte swizzle
     return d;
+}
+
+// UMMA shared-memory matrix descriptor, 64-byte swizzle, K-major rows of 64 bytes (8-row atoms of
+// 512 bytes, tiles 512-byte aligned): the layout a TMA load with CU_TENSOR_MAP_SWIZZLE_64B writes
+__device__ __forceinline__ uint64_t sw64_desc(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFF);
+    d |= (uint64_t)(16u >> 4) << 16;   // leading byte offset (unused for swizzled K-major)
+    d |= (uint64_t)(512u >> 4) << 32;  // 8-row atoms 512 bytes apart
+    d |= (uint64_t)1 << 46;            // descriptor version for tcgen05
+    d |= (uint64_t)4 << 61;            // 64-byte swizzle
+    return d;
+}
+
+// D[tmem] (+)= (A * 2^SFA) * (B * 2^SFB)^T, kind::mxf4 block32: A and B packed e2m1 (two per byte)
+// in shared memory, K = 64 per instruction, one E8M0 scale per 32 K-elements read from tensor
+// memory.  A row m's scales are the bytes of the 32-bit word at lane m % 32 (of every
+// sub-partition), column sfa + m / 32, starting at byte `sf_id` (B the same with its rows);
+// the byte offset travels in the address' top two bits and in the instruction descriptor
+// (layout measured on B200).
+__host__ __device__ constexpr uint32_t idesc_mxf4(int M, int N, int a_sf_id, int b_sf_id) {
+    return ((uint32_t)b_sf_id << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | (1u << 23) |
+           ((uint32_t)(M >> 4) << 24) | ((uint32_t)a_sf_id << 29);
+}
+__device__ __forceinline__ void mma_mxf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n}\n" ::"r"(
+            d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
+// 32 lanes x N columns of 32-bit stores from this warp's sub-partition (thread t -> lane sub*32 + t)
+__device__ __forceinline__ void tmem_st_x8(uint32_t taddr, const uint32_t (&r)[8]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
+                 "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_st_x1(uint32_t taddr, uint32_t r) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(r) : "memory");
 }
 
 // instruction descriptor: kind::f16, fp32 accumulate, A/B bf16 (fmt 1) or f16 (fmt 0)
