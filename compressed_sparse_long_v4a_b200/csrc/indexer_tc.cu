@@ -60,7 +60,7 @@ constexpr int kHistBins = 4096;          // top 12 bits of the ordered score key
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxDStages = 4;
 constexpr int kQBufBytes = 16384;        // B operand of one segment: up to 128 rows of 128 B
-constexpr int kMxXAhead = 6;               // MXFP4: tiles of block exponents each staging thread fetches ahead
+constexpr int kMxXAhead = 3;               // MXFP4: 512-entry tiles of block exponents each staging thread fetches ahead
 constexpr int kMxXSlots = kMxXAhead + 1;
 
 template <bool FP8> struct Ring {
@@ -84,13 +84,15 @@ struct __align__(1024) IdxSmem {
     uint32_t hist[2][kHistBins];
     union {
         uint32_t xring[kXSlots][kEpiThreads];  // FP8: per-entry scales, per epilogue thread
-        uint32_t mx_xring[kMxXSlots][8][128];  // MXFP4: block-exponent words, per staging thread
+        uint32_t mx_xring[kMxXSlots][16][128]; // MXFP4: block-exponent words, per staging thread
     };
     uint64_t k_full[kMaxStages], k_empty[kMaxStages], d_full[kMaxDStages], d_free[kMaxDStages], q_full[2], q_free[2],
         sf_full[2], sf_free[2], ep_sync, drain;
     int abort_flag;
     uint32_t tmem_base;
 };
+
+static_assert(sizeof(IdxSmem) + 1024 <= 232448, "shared memory beyond the 227 KB a block can have");
 
 struct IdxTcArgs {
     const __nv_bfloat16* q;  // [rows][HI][128] bf16
@@ -522,90 +524,91 @@ __global__ void __launch_bounds__(kThreads, 1) index_score_tc_kernel(const __gri
 // ---------------------------------------------------------------------
 // Key rows are 64 bytes of packed e2m1 codes; their 4 E8M0 block exponents
 // live in a separate array, one 32-bit word per entry whose byte j scales
-// elements 32j .. 32j+31.  TMA brings 256-entry tiles (16 KB, 64-byte
-// swizzle) into 32 KB stages of two tiles, and those tiles ARE the MMA's A
+// elements 32j .. 32j+31.  A tile is 512 entries: two TMA boxes of 256 rows
+// (64-byte swizzle) fill one 32 KB stage, and the stage IS the MMA's A
 // operand: tcgen05 kind::mxf4 (block32) reads packed e2m1 from shared memory
-// and applies one E8M0 scale per 32 K-elements from tensor memory, so a
-// 256-entry tile is 4 MMAs (2 halves x K = 2 x 64) with f32 accumulation.
-// The scale words need no repacking: row m of a 128-row half reads the word
-// at lane m % 32 (of every sub-partition), column m / 32, bytes 0-1 for
-// K 0..63 and bytes 2-3 for K 64..127.  Warps 2-5 (one per sub-partition)
-// write each tile's words there with tcgen05.st, from a ring of 4-byte
-// cp.async copies fetched kMxXAhead tiles ahead; per query they also quantise
-// q to MXFP4 (the B operand, same layout) and write its scale words.  The
-// epilogue is the bf16-key one: each accumulator column is already
-// q_h . k_s with both block scales applied.
+// and applies one E8M0 scale per 32 K-elements from tensor memory, so a tile
+// is 8 MMAs (4 quarters of 128 rows x K = 2 x 64) with f32 accumulation, and
+// one set of waits and commits.  The scale words need no repacking: row m of
+// a 128-row quarter reads the word at lane m % 32 (of every sub-partition),
+// column m / 32, bytes 0-1 for K 0..63 and bytes 2-3 for K 64..127.  Warps
+// 2-5 (one per sub-partition) write each tile's words there with
+// tcgen05.st, from a ring of 4-byte cp.async copies fetched kMxXAhead tiles
+// ahead; per query they also quantise q to MXFP4 (the B operand, same
+// layout) and write its scale words.  The epilogue is the bf16-key one: each
+// accumulator column is already q_h . k_s with both block scales applied.
 
-constexpr int kMxTileBytes = kTileK * 64;                 // packed codes of one 256-entry tile
-constexpr int kMxStageBytes = 2 * kMxTileBytes;           // two tiles per stage
+constexpr int kMxTile = 512;                              // entries per tile
+constexpr int kMxQuarterBytes = kHalf * 64;               // 128 rows of packed codes
+constexpr int kMxStageBytes = kMxTile * 64;               // one tile per 32 KB stage
 constexpr int kMxStages = kRingBytes / kMxStageBytes;     // 4
-constexpr uint32_t kMxSfaCol = 256;                       // two A-scale slots of 8 columns, 16 apart
+constexpr uint32_t kMxSfaCol = 256;                       // two A-scale slots of 16 columns
 constexpr uint32_t kMxSfbCol = 320;                       // two B-scale columns (query buffers), 16 apart
 template <int NP> struct MxAcc {
-    static constexpr uint32_t kCols = 2 * NP;             // per tile: 2 halves x NP heads
-    static constexpr int kStages = kMaxDStages;
-    static_assert(kStages * kCols <= kMxSfaCol, "accumulators overlap the scale columns");
+    static constexpr uint32_t kCols = 4 * NP;             // per tile: 4 quarters x NP heads
+    static constexpr int kStages = (int)(kMxSfaCol / kCols) < kMaxDStages ? (int)(kMxSfaCol / kCols) : kMaxDStages;
+    static_assert(kStages >= 2, "accumulators");
 };
 static_assert(kMxStages <= kMaxStages, "ring stages");
 
 __device__ void mx_producer(IdxSmem& sm, const IdxTcArgs& a, const CUtensorMap* kmap, long long f0, long long f1) {
     ICursor cur(f0, a, 1);
-    const long long n = f1 - f0, nst = (n + 1) / 2;
-    for (long long i = 0; i < nst; ++i) {
+    const long long n = f1 - f0;
+    for (long long jt = 0; jt < n; ++jt, cur.next(a)) {
         if (aborted(sm)) break;
-        const int st = (int)(i % kMxStages);
-        if (i >= kMxStages && !tc::mbar_wait(&sm.k_empty[st], (uint32_t)((i / kMxStages) - 1) & 1)) {
+        const int st = (int)(jt % kMxStages);
+        if (jt >= kMxStages && !tc::mbar_wait(&sm.k_empty[st], (uint32_t)((jt / kMxStages) - 1) & 1)) {
             idx_fault(sm, a);
             break;
         }
-        const int nt = (2 * i + 1 < n) ? 2 : 1;
-        tc::mbar_arrive_expect_tx(&sm.k_full[st], (uint32_t)(nt * kMxTileBytes));
-        for (int u = 0; u < nt; ++u, cur.next(a)) {
-            const int y = (int)((long long)cur.bat * a.n_ent + (long long)cur.ti * kTileK);
-            tc::tma_load_2d(sm.ring + st * kMxStageBytes + u * kMxTileBytes, kmap, 0, y, &sm.k_full[st]);
-        }
+        const int y = (int)((long long)cur.bat * a.n_ent + (long long)cur.ti * kMxTile);
+        tc::mbar_arrive_expect_tx(&sm.k_full[st], (uint32_t)kMxStageBytes);
+        // boxes of 256 rows; rows past the tensor's end are filled with zeros (and still counted)
+        tc::tma_load_2d(sm.ring + st * kMxStageBytes, kmap, 0, y, &sm.k_full[st]);
+        tc::tma_load_2d(sm.ring + st * kMxStageBytes + kMxStageBytes / 2, kmap, 0, y + 256, &sm.k_full[st]);
     }
     // no copy may still be in flight when the CTA exits
-    for (long long i = nst - kMxStages; i < nst; ++i)
-        if (i >= 0) tc::mbar_wait(&sm.k_full[i % kMxStages], (uint32_t)(i / kMxStages) & 1);
+    for (long long jt = n - kMxStages; jt < n; ++jt)
+        if (jt >= 0) tc::mbar_wait(&sm.k_full[jt % kMxStages], (uint32_t)(jt / kMxStages) & 1);
 }
 
 template <int NP>
 __device__ void mx_mma(IdxSmem& sm, const IdxTcArgs& a, uint32_t tmem, long long f0, long long f1) {
     using Acc = MxAcc<NP>;
     constexpr int kDS = Acc::kStages;
+    // descriptors: the ring's first stage and both query buffers; every operand is a fixed offset
+    // from one of them (start addresses count 16-byte units in the low 14 bits; no carry here)
+    const uint64_t ring_desc = tc::sw64_desc(tc::smem_u32(sm.ring));
+    const uint64_t q_desc0 = tc::sw64_desc(tc::smem_u32(sm.q[0])), q_desc1 = tc::sw64_desc(tc::smem_u32(sm.q[1]));
+    constexpr uint32_t id0 = tc::idesc_mxf4(128, NP, 0, 0), id1 = tc::idesc_mxf4(128, NP, 2, 2);
     bool ok = true;
     int seg = 0, b = 0;
-    uint32_t qaddr = 0;
     ICursor cur(f0, a, 1);
     for (long long f = f0; f < f1; ++f, cur.next(a)) {
         if (aborted(sm)) { ok = false; break; }
-        const long long jt = f - f0;
-        const int st = (int)((jt >> 1) % kMxStages), u = (int)(jt & 1), slot = (int)(jt & 1), sd = (int)(jt % kDS);
+        const int jt = (int)(f - f0);
+        const int st = jt % kMxStages, slot = jt & 1, sd = jt % kDS;
         if (f == f0 || cur.ti == 0) {
             b = seg & 1;
             if (!tc::mbar_wait(&sm.q_full[b], (seg >> 1) & 1)) { ok = false; break; }
-            qaddr = tc::smem_u32(sm.q[b]);
             ++seg;
         }
         const bool seg_end = (f == f1 - 1) || (cur.ti == a.tiles_per_row - 1);
-        if (u == 0 && !tc::mbar_wait(&sm.k_full[st], (uint32_t)((jt >> 1) / kMxStages) & 1)) { ok = false; break; }
+        if (!tc::mbar_wait(&sm.k_full[st], (uint32_t)(jt / kMxStages) & 1)) { ok = false; break; }
         if (!tc::mbar_wait(&sm.sf_full[slot], (uint32_t)(jt >> 1) & 1)) { ok = false; break; }
         if (jt >= kDS && !tc::mbar_wait(&sm.d_free[sd], (uint32_t)((jt / kDS) - 1) & 1)) { ok = false; break; }
         tc::tc_fence_after();
-        const uint32_t tile = tc::smem_u32(sm.ring + st * kMxStageBytes + u * kMxTileBytes);
+        const uint64_t a0 = ring_desc + (uint64_t)((st * kMxStageBytes) >> 4), b0 = b ? q_desc1 : q_desc0;
+        const uint32_t d0 = tmem + Acc::kCols * sd, sfa = tmem + kMxSfaCol + 16 * slot, sfb = tmem + kMxSfbCol + 16 * b;
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf)
-#pragma unroll
-            for (int kk = 0; kk < 2; ++kk)
-                tc::mma_mxf4(tmem + Acc::kCols * sd + NP * hf,
-                             tc::sw64_desc(tile + hf * kHalf * 64 + 32 * kk), tc::sw64_desc(qaddr + 32 * kk),
-                             tc::idesc_mxf4(128, NP, 2 * kk, 2 * kk),
-                             (tmem + kMxSfaCol + 16 * slot + 4 * hf) | ((uint32_t)(2 * kk) << 30),
-                             (tmem + kMxSfbCol + 16 * b) | ((uint32_t)(2 * kk) << 30), kk ? 1u : 0u);
+        for (int qq = 0; qq < 4; ++qq) {
+            tc::mma_mxf4(d0 + NP * qq, a0 + (uint64_t)((qq * kMxQuarterBytes) >> 4), b0, id0, sfa + 4 * qq, sfb, 0u);
+            tc::mma_mxf4(d0 + NP * qq, a0 + (uint64_t)((qq * kMxQuarterBytes + 32) >> 4), b0 + 2, id1,
+                         (sfa + 4 * qq) | (2u << 30), sfb | (2u << 30), 1u);
+        }
+        tc::mma_commit(&sm.k_empty[st]);
         tc::mma_commit(&sm.sf_free[slot]);
         tc::mma_commit(&sm.d_full[sd]);
-        if (u == 1 || f == f1 - 1) tc::mma_commit(&sm.k_empty[st]);
         if (seg_end) tc::mma_commit(&sm.q_free[b]);
     }
     if (!ok) idx_fault(sm, a);
@@ -661,7 +664,7 @@ __device__ void stage_query_mx(IdxSmem& sm, const IdxTcArgs& a, uint32_t tmem, i
 
 // warps 2-5: per segment the query (B operand and scales); per tile the keys' scale words (A
 // scales) in tensor memory: thread (sub-partition p, lane t) writes, in its sub-partition, column
-// 16 slot + 4 hf + c the word of entry 128 hf + 32 c + t
+// 16 slot + 4 q + c the word of entry 128 q + 32 c + t (quarter q, c < 4)
 template <int NP>
 __device__ void mx_stage(IdxSmem& sm, const IdxTcArgs& a, uint32_t tmem, long long f0, long long f1) {
     const int ct = threadIdx.x - 64;
@@ -676,11 +679,12 @@ __device__ void mx_stage(IdxSmem& sm, const IdxTcArgs& a, uint32_t tmem, long lo
     long long fp = f0;
     auto prefetch = [&]() {
         if (fp < f1) {
-            const int slot = (int)((fp - f0) % kMxXSlots);
+            const int xs = (int)((fp - f0) % kMxXSlots);
+            const long long e0 = (long long)pre.ti * kMxTile + lane, base = (long long)pre.bat * a.n_ent;
 #pragma unroll
-            for (int w = 0; w < 8; ++w) {
-                const long long e = (long long)pre.ti * kTileK + kHalf * (w >> 2) + 32 * (w & 3) + lane;
-                if (e < a.n_ent) tc::cp_async_4(&sm.mx_xring[slot][w][ct], src + (long long)pre.bat * a.n_ent + e);
+            for (int w = 0; w < 16; ++w) {
+                const long long e = e0 + 32 * w;  // word w: quarter w / 4, column w % 4
+                if (e < a.n_ent) tc::cp_async_4(&sm.mx_xring[xs][w][ct], src + base + e);
             }
             pre.next(a);
             ++fp;
@@ -691,7 +695,7 @@ __device__ void mx_stage(IdxSmem& sm, const IdxTcArgs& a, uint32_t tmem, long lo
     ICursor cur(f0, a, 1);
     for (long long f = f0; f < f1; ++f, cur.next(a)) {
         if (warp_aborted(sm)) { ok = false; break; }
-        const long long jt = f - f0;
+        const int jt = (int)(f - f0);
         if (f == f0 || cur.ti == 0) {
             const int b = seg & 1;
             if (seg >= 2 && !warp_wait(&sm.q_free[b], ((seg >> 1) - 1) & 1)) { ok = false; break; }
@@ -702,15 +706,15 @@ __device__ void mx_stage(IdxSmem& sm, const IdxTcArgs& a, uint32_t tmem, long lo
             ++seg;
         }
         prefetch();  // tile f + kMxXAhead
-        const int slot = (int)(jt & 1);
+        const int slot = jt & 1;
         if (jt >= 2 && !warp_wait(&sm.sf_free[slot], (uint32_t)((jt >> 1) - 1) & 1)) { ok = false; break; }
         tc::cp_async_wait<kMxXAhead>();
-        const int xs = (int)(jt % kMxXSlots);
-        uint32_t wv[8];
+        const int xs = jt % kMxXSlots;
+        uint32_t wv[16];
 #pragma unroll
-        for (int w = 0; w < 8; ++w) wv[w] = sm.mx_xring[xs][w][ct];
+        for (int w = 0; w < 16; ++w) wv[w] = sm.mx_xring[xs][w][ct];
         tc::tc_fence_after();
-        tc::tmem_st_x8(tmem + lane_addr + kMxSfaCol + 16 * slot, wv);
+        tc::tmem_st_x16(tmem + lane_addr + kMxSfaCol + 16 * slot, wv);
         tc::tmem_st_wait();
         tc::tc_fence_before();
         tc::mbar_arrive(&sm.sf_full[slot]);
@@ -719,13 +723,14 @@ __device__ void mx_stage(IdxSmem& sm, const IdxTcArgs& a, uint32_t tmem, long lo
     if (!ok) idx_fault(sm, a);
 }
 
-// warps 6-13: the score of entry 128 hf + r of each tile, histogram counts and stores
+// warps 6-13: the scores of entries 128 q + r of each tile (q = g, g + 2 for warp group g),
+// histogram counts and stores
 template <int NP>
 __device__ void mx_epilogue(IdxSmem& sm, const IdxTcArgs& a, uint32_t tmem, long long f0, long long f1) {
     using Acc = MxAcc<NP>;
     constexpr int kDS = Acc::kStages;
     const int et = threadIdx.x - kEpiFirst;
-    const int hf = et >> 7;
+    const int g = et >> 7;
     const int sub = (threadIdx.x >> 5) & 3;
     const int r = 32 * sub + (threadIdx.x & 31);
     const uint32_t lane_addr = (uint32_t)(32 * sub) << 16;
@@ -749,17 +754,23 @@ __device__ void mx_epilogue(IdxSmem& sm, const IdxTcArgs& a, uint32_t tmem, long
         cur.next(a);
         if (!warp_wait(&sm.d_full[sd], (jt / kDS) & 1)) { ok = false; break; }
         tc::tc_fence_after();
-        const float acc = score_of<false, NP>(tmem + lane_addr + Acc::kCols * sd + NP * hf, sm.wq[b]);
+        float acc[2];
+#pragma unroll
+        for (int i = 0; i < 2; ++i)
+            acc[i] = score_of<false, NP>(tmem + lane_addr + Acc::kCols * sd + NP * (g + 2 * i), sm.wq[b]);
         tc::tc_fence_before();
         tc::mbar_arrive(&sm.d_free[sd]);
-        const long long e = (long long)ti * kTileK + kHalf * hf + r;
-        if (e < a.n_ent) {
-            float sc = -INFINITY;
-            if (e < nv) {
-                sc = acc + 0.0f;
-                if (a.hist) atomicAdd(&sm.hist[b][float_to_ordered(sc) >> 20], 1u);
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const long long e = (long long)ti * kMxTile + kHalf * (g + 2 * i) + r;
+            if (e < a.n_ent) {
+                float sc = -INFINITY;
+                if (e < nv) {
+                    sc = acc[i] + 0.0f;
+                    if (a.hist) atomicAdd(&sm.hist[b][float_to_ordered(sc) >> 20], 1u);
+                }
+                srow[e] = sc;
             }
-            srow[e] = sc;
         }
         if (seg_end) {
             tc::mbar_arrive(&sm.q_free[b]);  // done with wq[b]
@@ -872,7 +883,7 @@ cudaError_t launch_index_scores_mx(const IndexArgs& a, float* scores, uint32_t* 
     t.ngroups = a.n_q;
     long long nv_max = n_visible(a.ctx_len - 1, a.m);
     if (nv_max > a.n_ent) nv_max = a.n_ent;
-    t.tiles_per_row = (int)((nv_max + kTileK - 1) / kTileK);
+    t.tiles_per_row = (int)((nv_max + kMxTile - 1) / kMxTile);
     t.total_tiles = (long long)a.batch * t.ngroups * t.tiles_per_row;
     if (t.total_tiles == 0) return cudaSuccess;
     t.grid = (int)(t.total_tiles < kNumSMs ? t.total_tiles : kNumSMs);
