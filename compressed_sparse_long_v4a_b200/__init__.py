@@ -18,6 +18,8 @@ __all__ = [
     "V4AError", "F32", "BF16", "FP8E4M3", "MXFP4", "lib", "library_path",
     "v4a_compress", "v4a_compress_dual", "v4a_quantize_mxfp4", "v4a_index_scores", "v4a_index_scores_mxfp4",
     "v4a_topk", "v4a_topk_mxfp4", "v4a_topk_noalloc", "v4a_csa_attend", "v4a_hca_attend",
+    "v4a_ring_append", "v4a_compress_paged", "v4a_topk_paged", "v4a_topk_mxfp4_paged", "v4a_csa_attend_paged",
+    "v4a_hca_attend_paged",
     "v4a_workspace_size", "v4a_status_string", "v4a_version", "n_entries", "window_rows",
 ]
 
@@ -56,6 +58,16 @@ class AttendExt(ctypes.Structure):
     _fields_ = [("sink", ctypes.c_void_p), ("rope_dims", ctypes.c_int), ("rope_base", ctypes.c_float)]
 
 
+class Paged(ctypes.Structure):
+    _fields_ = [("block_table", ctypes.c_void_p), ("bt_stride", ctypes.c_int), ("block_tokens", ctypes.c_int),
+                ("n_blocks", ctypes.c_longlong), ("ring_rows", ctypes.c_int)]
+
+
+class RingIO(ctypes.Structure):
+    _fields_ = [("src", ctypes.c_void_p), ("ring", ctypes.c_void_p), ("channels", ctypes.c_int),
+                ("ring_rows", ctypes.c_int), ("dtype", ctypes.c_int), ("src_batch_stride", ctypes.c_longlong)]
+
+
 def library_path() -> str:
     return _LIB_PATH
 
@@ -85,6 +97,18 @@ def _load():
     L.v4a_index_scores_mxfp4.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, P(Shape), vp]
     L.v4a_topk_mxfp4.restype = i32
     L.v4a_topk_mxfp4.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, vp, sz, P(Shape), vp]
+    L.v4a_ring_append.restype = i32
+    L.v4a_ring_append.argtypes = [P(RingIO), i32, i32, ll, vp]
+    L.v4a_compress_paged.restype = i32
+    L.v4a_compress_paged.argtypes = [P(CompressIO), P(CompressIO), i32, ll, i32, ll, P(Paged), vp]
+    L.v4a_topk_paged.restype = i32
+    L.v4a_topk_paged.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, sz, vp, P(Paged), P(Shape), vp]
+    L.v4a_topk_mxfp4_paged.restype = i32
+    L.v4a_topk_mxfp4_paged.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, vp, sz, vp, P(Paged), P(Shape), vp]
+    L.v4a_csa_attend_paged.restype = i32
+    L.v4a_csa_attend_paged.argtypes = [vp, vp, vp, vp, vp, i32, vp, sz, vp, P(AttendExt), P(Paged), P(Shape), vp]
+    L.v4a_hca_attend_paged.restype = i32
+    L.v4a_hca_attend_paged.argtypes = [vp, vp, vp, vp, i32, vp, sz, vp, P(AttendExt), P(Paged), P(Shape), vp]
     L.v4a_topk_noalloc.restype = i32
     L.v4a_topk_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, P(Shape), vp]
     L.v4a_csa_attend.restype = i32
@@ -350,3 +374,132 @@ def v4a_hca_attend(q, entries, token_kv, tok_pos0: int, out, *, m: int, window: 
         _check(lib.v4a_hca_attend(*args, ctypes.byref(s), _stream(stream)))
     else:
         _check(lib.v4a_hca_attend_ex(*args, ctypes.byref(ext), ctypes.byref(s), _stream(stream)))
+
+
+# ----------------------------------------------------------------------
+# heterogeneous KV cache: paged classical cache + token rings
+# ----------------------------------------------------------------------
+
+def _paged(block_table, block_tokens: int, n_blocks: int, ring_rows: int = 0) -> Paged:
+    _contig(block_table, "block_table")
+    if block_table.dtype != torch.int32 or block_table.dim() != 2:
+        raise ValueError("block_table must be int32 [batch][blocks]")
+    return Paged(_ptr(block_table), int(block_table.shape[1]), int(block_tokens), int(n_blocks), int(ring_rows))
+
+
+def v4a_ring_append(pairs, pos: int, stream=None) -> None:
+    """Append the token at position `pos`: for each (src [batch][channels], ring [batch][ring_rows][channels])
+    pair, src row b goes to ring row pos % ring_rows of sequence b (one launch for up to 8 pairs)."""
+    ios = (RingIO * max(1, len(pairs)))()
+    batch = None
+    for i, (src, ring) in enumerate(pairs):
+        if src.dim() != 2 or src.stride(1) != 1 or ring.dim() != 3 or not ring.is_contiguous():
+            raise ValueError("src must be [batch][channels] with dense rows, ring [batch][rows][channels] contiguous")
+        if src.dtype != ring.dtype or src.shape[1] != ring.shape[2] or src.shape[0] != ring.shape[0]:
+            raise ValueError("src and ring disagree")
+        batch = int(src.shape[0]) if batch is None else batch
+        ios[i] = RingIO(_ptr(src), _ptr(ring), int(ring.shape[2]), int(ring.shape[1]), _dtype(src), src.stride(0))
+    _check(lib.v4a_ring_append(ios, len(pairs), batch or 0, int(pos), _stream(stream)))
+
+
+def _pool_io(x, gate, out, out_scale=None, out_exp=None) -> CompressIO:
+    """A compress stream whose output is a pool of rows [pool_rows][channels] (codes [pool_rows][channels/2]
+    with exps [pool_rows][channels/32] for MXFP4)."""
+    for t, name in ((x, "x"), (gate, "gate")):
+        if t.dim() != 3 or t.stride(2) != 1 or t.stride(1) != t.shape[2]:
+            raise ValueError(f"{name} must be [batch][rows][channels] with dense rows")
+    _contig(out, "out")
+    C = int(x.shape[2])
+    if out_exp is not None:
+        _contig(out_exp, "out_exp")
+        return CompressIO(_ptr(x), _ptr(gate), _ptr(out), None, C, _dtype(x), MXFP4, x.stride(0), gate.stride(0), 0, 0,
+                          _ptr(out_exp), 0)
+    if out_scale is not None:
+        _contig(out_scale, "out_scale")
+    return CompressIO(_ptr(x), _ptr(gate), _ptr(out), _ptr(out_scale), C, _dtype(x), _dtype(out), x.stride(0),
+                      gate.stride(0), 0, 0, None, 0)
+
+
+def v4a_compress_paged(x, gate, out_pool, *, m: int, first_entry: int, block_table, block_tokens: int,
+                       n_tok: int | None = None, out_scale=None, xi=None, gate_i=None, out_i=None, out_i_scale=None,
+                       out_i_exp=None, stream=None) -> None:
+    """Compress complete chunks of x (e.g. a slice of the token rings) into pool rows through the block
+    table: entry first_entry + s of sequence b -> row block_table[b][e // epb] * epb + e % epb (epb =
+    block_tokens // m).  The indexer-key stream (xi, gate_i -> out_i pools) rides in the same launch."""
+    n = x.shape[1] if n_tok is None else int(n_tok)
+    epb = block_tokens // m
+    kv = _pool_io(x, gate, out_pool, out_scale)
+    idx = _pool_io(xi, gate_i, out_i, out_i_scale, out_i_exp) if xi is not None else None
+    pg = _paged(block_table, block_tokens, out_pool.shape[0] // epb)
+    _check(lib.v4a_compress_paged(ctypes.byref(kv), ctypes.byref(idx) if idx is not None else None, int(x.shape[0]),
+                                  n, int(m), int(first_entry), ctypes.byref(pg), _stream(stream)))
+
+
+def v4a_topk_paged(q_i, w, k_pool, k_scale_pool, idx_out, score_out=None, *, m: int, k: int, ctx_len: int,
+                   block_table, block_tokens: int, workspace=None, dev_status=None, stream=None) -> None:
+    """v4a_topk over key pools [pool_rows][d_i] (+ scales [pool_rows]) addressed through the block table."""
+    for t, n in ((q_i, "q_i"), (w, "w"), (k_pool, "k_pool"), (k_scale_pool, "k_scale_pool"), (idx_out, "idx_out"),
+                 (score_out, "score_out")):
+        _contig(t, n)
+    B, T, HI, DI = q_i.shape
+    s = _shape(batch=B, n_q=T, m=m, k=k, ctx_len=ctx_len)
+    pg = _paged(block_table, block_tokens, k_pool.shape[0] // (block_tokens // m))
+    if workspace is None:
+        workspace = _workspace(lib.v4a_workspace_size(b"topk", ctypes.byref(s), HI, DI), q_i.device)
+    _check(lib.v4a_topk_paged(_ptr(q_i), _ptr(w), _ptr(k_pool), _ptr(k_scale_pool), _ptr(idx_out), _ptr(score_out),
+                              HI, DI, _dtype(q_i), _dtype(k_pool), _ptr(workspace),
+                              workspace.numel() * workspace.element_size(), _ptr(dev_status), ctypes.byref(pg),
+                              ctypes.byref(s), _stream(stream)))
+
+
+def v4a_topk_mxfp4_paged(q_i, w, k_codes_pool, k_exp_pool, idx_out, score_out=None, *, m: int, k: int, ctx_len: int,
+                         block_table, block_tokens: int, workspace=None, dev_status=None, stream=None) -> None:
+    """v4a_topk_mxfp4 over MXFP4 key pools (codes [pool_rows][d_i/2], exps [pool_rows][d_i/32])."""
+    for t, n in ((q_i, "q_i"), (w, "w"), (k_codes_pool, "k_codes_pool"), (k_exp_pool, "k_exp_pool"),
+                 (idx_out, "idx_out"), (score_out, "score_out")):
+        _contig(t, n)
+    B, T, HI, DI = q_i.shape
+    s = _shape(batch=B, n_q=T, m=m, k=k, ctx_len=ctx_len)
+    pg = _paged(block_table, block_tokens, k_codes_pool.shape[0] // (block_tokens // m))
+    if workspace is None:
+        workspace = _workspace(lib.v4a_workspace_size(b"topk", ctypes.byref(s), HI, DI), q_i.device)
+    _check(lib.v4a_topk_mxfp4_paged(_ptr(q_i), _ptr(w), _ptr(k_codes_pool), _ptr(k_exp_pool), _ptr(idx_out),
+                                    _ptr(score_out), HI, DI, _dtype(q_i), _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), _ptr(dev_status), ctypes.byref(pg),
+                                    ctypes.byref(s), _stream(stream)))
+
+
+def v4a_csa_attend_paged(q, ent_pool, idx, ring, out, *, m: int, window: int, ctx_len: int, block_table,
+                         block_tokens: int, workspace=None, dev_status=None, sink=None, rope_dims: int = 0,
+                         rope_base: float = 10000.0, stream=None) -> None:
+    """CSA attention over an entry pool [pool_rows][d] (block table) and the K=V ring [batch][ring_rows][d]."""
+    for t, n in ((q, "q"), (ent_pool, "ent_pool"), (idx, "idx"), (ring, "ring"), (out, "out")):
+        _contig(t, n)
+    B, T, H, d = q.shape
+    s = _shape(batch=B, n_q=T, heads=H, d=d, m=m, k=idx.shape[-1], window=window, ctx_len=ctx_len)
+    pg = _paged(block_table, block_tokens, ent_pool.shape[0] // (block_tokens // m), ring.shape[1])
+    if workspace is None:
+        workspace = _workspace(lib.v4a_workspace_size(b"csa_attend", ctypes.byref(s), 0, 0), q.device)
+    ext = _ext(sink, rope_dims, rope_base)
+    _check(lib.v4a_csa_attend_paged(_ptr(q), _ptr(ent_pool), _ptr(idx), _ptr(ring), _ptr(out), _dtype(q),
+                                    _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(dev_status),
+                                    ctypes.byref(ext) if ext is not None else None, ctypes.byref(pg), ctypes.byref(s),
+                                    _stream(stream)))
+
+
+def v4a_hca_attend_paged(q, ent_pool, ring, out, *, m: int, window: int, ctx_len: int, block_table,
+                         block_tokens: int, workspace=None, dev_status=None, sink=None, rope_dims: int = 0,
+                         rope_base: float = 10000.0, stream=None) -> None:
+    """HCA attention over an entry pool [pool_rows][d] (block table) and the K=V ring."""
+    for t, n in ((q, "q"), (ent_pool, "ent_pool"), (ring, "ring"), (out, "out")):
+        _contig(t, n)
+    B, T, H, d = q.shape
+    s = _shape(batch=B, n_q=T, heads=H, d=d, m=m, window=window, ctx_len=ctx_len)
+    pg = _paged(block_table, block_tokens, ent_pool.shape[0] // (block_tokens // m), ring.shape[1])
+    if workspace is None:
+        workspace = _workspace(lib.v4a_workspace_size(b"hca_attend", ctypes.byref(s), 0, 0), q.device)
+    ext = _ext(sink, rope_dims, rope_base)
+    _check(lib.v4a_hca_attend_paged(_ptr(q), _ptr(ent_pool), _ptr(ring), _ptr(out), _dtype(q), _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), _ptr(dev_status),
+                                    ctypes.byref(ext) if ext is not None else None, ctypes.byref(pg), ctypes.byref(s),
+                                    _stream(stream)))

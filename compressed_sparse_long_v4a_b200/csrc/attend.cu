@@ -115,10 +115,23 @@ __global__ void __launch_bounds__(kBlockThreads, 1) attend_split_kernel(AttendAr
                             if (c8 == 0 && a.dev_status) atomicExch(a.dev_status, (int)V4A_ERR_DEVICE_FAULT);
                         }
                     }
-                    if (ok) src = static_cast<const T*>(a.entries) + ((long long)b * a.n_ent + s) * d;
+                    if (ok) {
+                        long long er = (long long)b * a.n_ent + s;
+                        if (a.bt) {
+                            const long long blk = a.bt[(long long)b * a.bt_stride + s / a.epb];
+                            er = blk * a.epb + s % a.epb;
+                            if (blk < 0 || er >= a.pool_rows) {  // a block id outside the pool
+                                ok = false;
+                                if (c8 == 0 && a.dev_status) atomicExch(a.dev_status, (int)V4A_ERR_DEVICE_FAULT);
+                            }
+                        }
+                        if (ok) src = static_cast<const T*>(a.entries) + er * d;
+                    }
                 } else {
                     const long long p = win_lo + (c - n_sel);
-                    src = static_cast<const T*>(a.token_kv) + ((long long)b * a.l_tok + (p - a.tok_pos0)) * d;
+                    const long long tr = a.ring_rows > 0 ? (long long)b * a.ring_rows + p % a.ring_rows
+                                                         : (long long)b * a.l_tok + (p - a.tok_pos0);
+                    src = static_cast<const T*>(a.token_kv) + tr * d;
                 }
             }
             float f[8];

@@ -84,7 +84,25 @@ struct TcArgs {
     const float* sink;  // [64] sink logits, or null
     int rope_dims;      // output dims rotated at minus the query position (0: none)
     float rope_base;
+    const int32_t* bt;  // paged entries: block table [B][bt_stride] (epb entries per block), or null
+    int bt_stride, epb;
+    long long n_blocks;
+    int ring_rows;      // > 0: window rows come from a ring [B][ring_rows][512] (position p in row p % ring_rows)
 };
+
+// tiles whose rows the producer gathers with cp.async (CSA selections, paged entries, ring windows)
+__device__ __forceinline__ bool tile_gathered(const TcArgs& a, int ti) {
+    return ti < a.e_tiles ? (a.idx != nullptr || a.bt != nullptr) : a.ring_rows > 0;
+}
+// row of visible entry s of sequence b; null for a block id outside the pool
+__device__ __forceinline__ const __nv_bfloat16* entry_row(const TcArgs& a, int b, long long s) {
+    if (a.bt) {
+        const long long blk = a.bt[(long long)b * a.bt_stride + s / a.epb];
+        if (blk < 0 || blk >= a.n_blocks) return nullptr;
+        return a.entries + (blk * a.epb + s % a.epb) * kD;
+    }
+    return a.entries + ((long long)b * a.n_ent + s) * kD;
+}
 
 __device__ __forceinline__ long long range_start(int c, const TcArgs& a) {
     return (long long)c * a.total_tiles / a.grid;
@@ -133,9 +151,33 @@ __device__ __forceinline__ void csa_rows(const TcArgs& a, const RowInfo& ri, int
         const long long c = c0 + lane + 32 * h2;
         const long long sidx = c < a.k ? (long long)a.idx[(long long)row * a.k + c] : -1;
         ok[h2] = sidx >= 0 && sidx < ri.nvis;
+        const __nv_bfloat16* er = ok[h2] ? entry_row(a, ri.b, sidx) : nullptr;
+        if (ok[h2] && !er) {  // a block id outside the pool: skipped and reported
+            ok[h2] = false;
+            if (a.dev_status) atomicExch(a.dev_status, (int)V4A_ERR_DEVICE_FAULT);
+        }
         // an excluded row still gets finite data: this query's head-0 row of q
-        src[h2] = ok[h2] ? a.entries + ((long long)ri.b * a.n_ent + sidx) * kD : a.q + (long long)row * kH * kD;
+        src[h2] = ok[h2] ? er : a.q + (long long)row * kH * kD;
     }
+}
+
+// cp.async all 64 rows of a tile (lane owns rows lane and lane+32: src / ok) into the 128-byte-swizzled
+// stage; returns the tile's row mask
+__device__ __forceinline__ uint64_t gather_tile(uint8_t* dst, const __nv_bfloat16* const (&src)[2], const bool (&ok)[2],
+                                                int lane) {
+    const uint64_t mask =
+        (uint64_t)__ballot_sync(0xffffffffu, ok[0]) | ((uint64_t)__ballot_sync(0xffffffffu, ok[1]) << 32);
+    for (int r = 0; r < kTile; ++r) {
+        const __nv_bfloat16* rs =
+            (const __nv_bfloat16*)__shfl_sync(0xffffffffu, (unsigned long long)(r < 32 ? src[0] : src[1]), r & 31);
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+            const int u = lane + 32 * h2;  // 16-byte chunk of the 1 KB row
+            uint8_t* d = dst + (u >> 3) * kSlabBytes + r * 128 + (((u & 7) ^ (r & 7)) << 4);
+            tc::cp_async_16(d, rs + u * 8);
+        }
+    }
+    return mask;
 }
 
 __device__ void producer(Smem& sm, const TcArgs& a, const CUtensorMap* ent_map, const CUtensorMap* tok_map,
@@ -162,7 +204,24 @@ __device__ void producer(Smem& sm, const TcArgs& a, const CUtensorMap* ent_map, 
         uint8_t* dst = sm.kv[st];
         if (ti < a.e_tiles) {
             const long long c0 = (long long)ti * kTile;
-            if (!a.idx) {
+            if (!a.idx && a.bt) {
+                // HCA over a paged pool: rows c0 .. c0+63 through the block table
+                const __nv_bfloat16* src[2];
+                bool ok[2];
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    const long long s = c0 + lane + 32 * h2;
+                    const __nv_bfloat16* er = s < ri.nvis ? entry_row(a, ri.b, s) : nullptr;
+                    if (s < ri.nvis && !er && a.dev_status) atomicExch(a.dev_status, (int)V4A_ERR_DEVICE_FAULT);
+                    ok[h2] = er != nullptr;
+                    src[h2] = ok[h2] ? er : a.q + (long long)row * kH * kD;
+                }
+                mask = gather_tile(dst, src, ok, lane);
+                if (lane == 0) {
+                    sm.mask[st] = mask;
+                    tc::mbar_arrive_expect_tx(&sm.kv_full[st], 0);
+                }
+            } else if (!a.idx) {
                 // HCA: rows c0 .. c0+63 of this sequence's entries are contiguous
                 const long long nv = ri.nvis - c0;
                 mask = nv >= kTile ? ~0ull : (nv <= 0 ? 0ull : ((1ull << nv) - 1ull));
@@ -183,21 +242,30 @@ __device__ void producer(Smem& sm, const TcArgs& a, const CUtensorMap* ent_map, 
                     const long long sidx = c < a.k ? (long long)a.idx[(long long)row * a.k + c] : -1;
                     if (!ok[h2] && sidx != -1 && a.dev_status) atomicExch(a.dev_status, (int)V4A_ERR_DEVICE_FAULT);
                 }
-                mask = (uint64_t)__ballot_sync(0xffffffffu, ok[0]) | ((uint64_t)__ballot_sync(0xffffffffu, ok[1]) << 32);
-                for (int r = 0; r < kTile; ++r) {
-                    const __nv_bfloat16* rs = (const __nv_bfloat16*)__shfl_sync(
-                        0xffffffffu, (unsigned long long)(r < 32 ? src[0] : src[1]), r & 31);
-#pragma unroll
-                    for (int h2 = 0; h2 < 2; ++h2) {
-                        const int u = lane + 32 * h2;  // 16-byte chunk of the 1 KB row
-                        uint8_t* d = dst + (u >> 3) * kSlabBytes + r * 128 + (((u & 7) ^ (r & 7)) << 4);
-                        tc::cp_async_16(d, rs + u * 8);
-                    }
-                }
+                mask = gather_tile(dst, src, ok, lane);
                 if (lane == 0) {
                     sm.mask[st] = mask;
                     tc::mbar_arrive_expect_tx(&sm.kv_full[st], 0);
                 }
+            }
+        } else if (a.ring_rows > 0) {
+            // window tokens p0 .. p0+63 from the ring (they may wrap around its end)
+            const long long wi = ti - a.e_tiles;
+            const long long p0 = ri.t - a.window + 1 + wi * kTile;
+            const __nv_bfloat16* src[2];
+            bool ok[2];
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+                const int r = lane + 32 * h2;
+                const long long p = p0 + r;
+                ok[h2] = wi * kTile + r < a.window && p >= 0;
+                src[h2] = ok[h2] ? a.token_kv + ((long long)ri.b * a.ring_rows + p % a.ring_rows) * kD
+                                 : a.q + (long long)row * kH * kD;
+            }
+            mask = gather_tile(dst, src, ok, lane);
+            if (lane == 0) {
+                sm.mask[st] = mask;
+                tc::mbar_arrive_expect_tx(&sm.kv_full[st], 0);
             }
         } else {
             // window tokens p0 .. p0+63 (contiguous rows of token_kv)
@@ -293,7 +361,7 @@ __device__ void mma_issuer(Smem& sm, const TcArgs& a, uint32_t tmem, long long f
             const bool qseg = jq == 0 || cq.ti == 0;
             if (tc::mbar_test(&sm.kv_full[jq % kStages], (uint32_t)(jq / kStages) & 1) &&
                 (!qseg || tc::mbar_test(&sm.q_full, segq & 1))) {
-                issue_qk(sm, tmem, (int)jq, a.idx != nullptr && cq.ti < a.e_tiles, q0);
+                issue_qk(sm, tmem, (int)jq, tile_gathered(a, cq.ti), q0);
                 if (jq == n - 1 || cq.ti == a.tpr - 1) tc::mma_commit(&sm.q_empty);  // last QK of this query
                 if (qseg) ++segq;
                 ++jq;
@@ -682,6 +750,7 @@ bool attend_tc_shape_ok(const AttendArgs& a) {
     TcPlan p = tc_plan(a);
     if (p.tpr < 1 || p.grid < 1) return false;
     if ((long long)a.batch * a.n_ent >= (1LL << 31) || (long long)a.batch * a.l_tok >= (1LL << 31)) return false;
+    if (a.bt && a.pool_rows >= (1LL << 31)) return false;
     if ((long long)a.batch * a.n_q * kH >= (1LL << 31)) return false;
     return true;
 }
@@ -699,8 +768,8 @@ cudaError_t launch_attend_tc(const AttendArgs& a, void* ws, size_t ws_bytes, cud
     if (ws_bytes < attend_tc_workspace_bytes(a)) return cudaErrorInvalidValue;
     TcPlan p = tc_plan(a);
     CUtensorMap ent_map, tok_map, q_map;
-    const long long ent_rows = (long long)a.batch * a.n_ent;
-    const long long tok_rows = (long long)a.batch * a.l_tok;
+    const long long ent_rows = a.bt ? a.pool_rows : (long long)a.batch * a.n_ent;
+    const long long tok_rows = (long long)a.batch * (a.ring_rows > 0 ? a.ring_rows : a.l_tok);
     const void* tok = a.token_kv ? a.token_kv : a.q;  // a window of 0 never reads it
     if (!make_map(&tok_map, tok, a.token_kv ? tok_rows : (long long)a.batch * a.n_q * kH, kTile))
         return cudaErrorInvalidValue;
@@ -739,6 +808,11 @@ cudaError_t launch_attend_tc(const AttendArgs& a, void* ws, size_t ws_bytes, cud
     t.sink = a.sink;
     t.rope_dims = a.rope_dims;
     t.rope_base = a.rope_base;
+    t.bt = a.bt;
+    t.bt_stride = a.bt_stride;
+    t.epb = a.epb;
+    t.n_blocks = a.epb > 0 ? a.pool_rows / a.epb : 0;
+    t.ring_rows = a.ring_rows;
 
     const size_t smem = sizeof(Smem) + 1024;
     cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -23,6 +23,8 @@
 namespace v4a {
 namespace {
 
+constexpr int kMaxRingStreams = 8;
+
 struct StreamDesc {
     const void* x;
     const void* gate;
@@ -39,6 +41,11 @@ struct StreamDesc {
     int split;             // S: lanes sharing one (entry, channel group)
     int in_dtype, out_dtype;
     long long x_bs, gate_bs, out_bs, scale_bs;
+    // paged output: entry first + s of sequence b goes to pool row bt[b*bt_stride + (first+s)/epb]*epb +
+    // (first+s)%epb (null: the sequence's own rows)
+    const int32_t* bt;
+    int bt_stride, epb;
+    long long first, n_blocks;  // a block id outside [0, n_blocks): the entry is not written
 };
 
 // This lane's share of one (entry, 8-channel group): tokens sub, sub + S, ... of the chunk, in
@@ -156,6 +163,19 @@ __global__ void __launch_bounds__(256) compress_kernel(StreamDesc s0, StreamDesc
 #pragma unroll
     for (int e = 0; e < 8; ++e) out[e] = active ? num[e] / den[e] : 0.f;
     if (sub != 0) return;
+    // output row (in entries of `channels` elements) and its block-scale slot
+    long long orow, srow;
+    if (d.bt) {
+        const long long es = d.first + s;
+        const long long blk = d.bt[(long long)b * d.bt_stride + es / d.epb];
+        if (blk < 0 || blk >= d.n_blocks) active = false;  // nowhere to write it (shuffles are done)
+        orow = blk * d.epb + es % d.epb;
+        srow = orow;
+    } else {
+        orow = -1;
+        srow = (long long)b * d.scale_bs + s;
+    }
+    const long long obase = d.bt ? orow * d.channels : (long long)b * d.out_bs + s * d.channels;
 
     if (d.out_dtype == V4A_FP8E4M3) {
         // per-entry amax over the entry's `groups` consecutive lanes (a power of two <= 32)
@@ -165,13 +185,13 @@ __global__ void __launch_bounds__(256) compress_kernel(StreamDesc s0, StreamDesc
         for (int o = d.groups / 2; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
         if (!active) return;
         float scale = a > 0.f ? a / 448.0f : 1.0f;
-        uint8_t* op = static_cast<uint8_t*>(d.out) + (long long)b * d.out_bs + s * d.channels + grp * 8;
+        uint8_t* op = static_cast<uint8_t*>(d.out) + obase + grp * 8;
         uint32_t lo = (uint32_t)pack_e4m3x2(out[0] / scale, out[1] / scale) |
                       ((uint32_t)pack_e4m3x2(out[2] / scale, out[3] / scale) << 16);
         uint32_t hi = (uint32_t)pack_e4m3x2(out[4] / scale, out[5] / scale) |
                       ((uint32_t)pack_e4m3x2(out[6] / scale, out[7] / scale) << 16);
         *reinterpret_cast<uint2*>(op) = make_uint2(lo, hi);
-        if (grp == 0) d.out_scale[(long long)b * d.scale_bs + s] = scale;
+        if (grp == 0) d.out_scale[srow] = scale;
         return;
     }
     if (d.out_dtype == V4A_MXFP4) {
@@ -179,17 +199,18 @@ __global__ void __launch_bounds__(256) compress_kernel(StreamDesc s0, StreamDesc
         int x;
         const uint32_t w = mx_quantize8(out, &x);
         if (!active) return;
-        uint8_t* op = static_cast<uint8_t*>(d.out) + ((long long)b * d.out_bs + s * d.channels + grp * 8) / 2;
+        uint8_t* op = static_cast<uint8_t*>(d.out) + (obase + grp * 8) / 2;
         *reinterpret_cast<uint32_t*>(op) = w;
-        if ((grp & 3) == 0) d.out_exp[(long long)b * d.exp_bs + s * (d.channels / 32) + grp / 4] = (uint8_t)(x + 127);
+        const long long xb = d.bt ? orow * (d.channels / 32) : (long long)b * d.exp_bs + s * (d.channels / 32);
+        if ((grp & 3) == 0) d.out_exp[xb + grp / 4] = (uint8_t)(x + 127);
         return;
     }
     if (!active) return;
     if (d.out_dtype == V4A_BF16) {
-        __nv_bfloat16* op = static_cast<__nv_bfloat16*>(d.out) + (long long)b * d.out_bs + s * d.channels + grp * 8;
+        __nv_bfloat16* op = static_cast<__nv_bfloat16*>(d.out) + obase + grp * 8;
         Vec8<__nv_bfloat16>::store(op, out);
     } else {
-        float* op = static_cast<float*>(d.out) + (long long)b * d.out_bs + s * d.channels + grp * 8;
+        float* op = static_cast<float*>(d.out) + obase + grp * 8;
         Vec8<float>::store(op, out);
     }
 }
@@ -239,7 +260,38 @@ StreamDesc describe(const v4a_compress_io* io) {
     d.gate_bs = io->gate_batch_stride;
     d.out_bs = io->out_batch_stride;
     d.scale_bs = io->scale_batch_stride;
+    d.bt = nullptr;
+    d.bt_stride = d.epb = 0;
+    d.first = d.n_blocks = 0;
     return d;
+}
+
+// one 16-byte chunk per thread: the new row of each stream into its ring slot pos % ring_rows
+struct RingArgs {
+    v4a_ring_io io[kMaxRingStreams];
+    int n, batch;
+    long long pos;
+    int chunks[kMaxRingStreams];  // 16-byte chunks per row of each stream
+};
+
+__global__ void __launch_bounds__(256) ring_append_kernel(RingArgs r) {
+    int g = blockIdx.x * blockDim.x + threadIdx.x;
+    for (int i = 0; i < r.n; ++i) {
+        const int per = r.batch * r.chunks[i];
+        if (g < per) {
+            const v4a_ring_io& io = r.io[i];
+            const int b = g / r.chunks[i], c = g - b * r.chunks[i];
+            const size_t es = io.dtype == V4A_F32 ? 4 : io.dtype == V4A_BF16 ? 2 : 1;
+            const uint4* src = reinterpret_cast<const uint4*>(static_cast<const char*>(io.src) +
+                                                              (size_t)b * io.src_batch_stride * es) + c;
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<char*>(io.ring) +
+                                                  ((size_t)b * io.ring_rows + (size_t)(r.pos % io.ring_rows)) *
+                                                      io.channels * es) + c;
+            *dst = __ldg(src);
+            return;
+        }
+        g -= per;
+    }
 }
 
 }  // namespace
@@ -275,6 +327,50 @@ cudaError_t launch_quantize_mxfp4(const void* x, v4a_dtype dt, long long rows, i
                                                               codes, exps);
     else
         quantize_mxfp4_kernel<<<blocks, threads, 0, stream>>>(static_cast<const float*>(x), rows, cols, codes, exps);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_compress_paged(const v4a_compress_io* kv, const v4a_compress_io* idx, int batch, long long n_tok,
+                                  int m, long long first_entry, const int32_t* bt, int bt_stride, int epb,
+                                  long long n_blocks, cudaStream_t stream) {
+    long long n_ent = n_tok / m;
+    if (batch == 0 || n_ent == 0) return cudaSuccess;
+    StreamDesc s0 = describe(kv);
+    StreamDesc s1 = idx ? describe(idx) : s0;
+    for (StreamDesc* d : {&s0, &s1}) {
+        d->bt = bt;
+        d->bt_stride = bt_stride;
+        d->epb = epb;
+        d->first = first_entry;
+        d->n_blocks = n_blocks;
+    }
+    int split = 1;
+    while (split < 32 && split * 2 <= m) split *= 2;
+    if (!quantised(s0.out_dtype)) s0.split = split;
+    if (!quantised(s1.out_dtype)) s1.split = split;
+    long long w0 = (long long)s0.groups * s0.split, w1 = (long long)s1.groups * s1.split;
+    long long total = (long long)batch * n_ent * (w0 > w1 ? w0 : w1);
+    const int threads = 256;
+    dim3 grid((unsigned)((total + threads - 1) / threads), idx ? 2 : 1);
+    compress_kernel<<<grid, threads, 0, stream>>>(s0, s1, batch, n_ent, m);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_ring_append(const v4a_ring_io* io, int n, int batch, long long pos, cudaStream_t stream) {
+    if (n == 0 || batch == 0) return cudaSuccess;
+    RingArgs r;
+    r.n = n;
+    r.batch = batch;
+    r.pos = pos;
+    long long total = 0;
+    for (int i = 0; i < n; ++i) {
+        r.io[i] = io[i];
+        const size_t es = io[i].dtype == V4A_F32 ? 4 : io[i].dtype == V4A_BF16 ? 2 : 1;
+        r.chunks[i] = (int)((size_t)io[i].channels * es / 16);
+        total += (long long)batch * r.chunks[i];
+    }
+    const int threads = 256;
+    ring_append_kernel<<<(unsigned)((total + threads - 1) / threads), threads, 0, stream>>>(r);
     return cudaGetLastError();
 }
 

@@ -88,7 +88,16 @@ __global__ void __launch_bounds__(kScoreThreads) index_score_kernel(IndexArgs a,
     float acc[HMAX];
 #pragma unroll
     for (int h = 0; h < HMAX; ++h) acc[h] = 0.f;
-    const long long koff = ((long long)b * a.n_ent + s) * a.d_i;
+    long long krow = (long long)b * a.n_ent + s;
+    if (a.bt) {
+        const long long blk = a.bt[(long long)b * a.bt_stride + s / a.epb];
+        krow = (blk >= 0 && blk * a.epb < a.pool_rows) ? blk * a.epb + s % a.epb : -1;  // -1: outside the pool
+    }
+    if (krow < 0) {  // reads as a key of zeros
+        *out = 0.0f;
+        return;
+    }
+    const long long koff = krow * a.d_i;
     for (int c = 0; c < a.d_i; c += 8) {
         float kv[8];
         load_key8<KFMT>(a, koff + c, kv);
@@ -114,7 +123,7 @@ __global__ void __launch_bounds__(kScoreThreads) index_score_kernel(IndexArgs a,
 #pragma unroll
     for (int h = 0; h < HMAX; ++h)
         if (h < a.heads_i) sc = fmaf(w_s[h], fmaxf(acc[h], 0.f), sc);
-    if (a.kscale) sc *= a.kscale[(long long)b * a.n_ent + s];
+    if (a.kscale) sc *= a.kscale[krow];
     *out = sc + 0.0f;  // -0 -> +0
 }
 
@@ -843,7 +852,7 @@ __global__ void score_hist_kernel(const float* scores, IndexArgs a, uint32_t* hi
 
 cudaError_t launch_index_scores(const IndexArgs& a, float* scores, cudaStream_t stream) {
     if (a.batch == 0 || a.n_ent == 0) return cudaSuccess;
-    if (index_tc_available(a)) return launch_index_scores_tc(a, scores, nullptr, nullptr, stream);
+    if (index_tc_available(a)) return launch_index_scores_tc(a, scores, nullptr, a.dev_status, stream);
     if (a.heads_i <= 4) return launch_scores_h<4>(a, scores, stream);
     if (a.heads_i <= 8) return launch_scores_h<8>(a, scores, stream);
     if (a.heads_i <= 16) return launch_scores_h<16>(a, scores, stream);
@@ -884,7 +893,7 @@ cudaError_t launch_topk(const IndexArgs& a, int k, int32_t* idx_out, float* scor
     e = cudaMemsetAsync(hist, 0, (size_t)rows * (kHistBins + 1) * sizeof(uint32_t), stream);
     if (e != cudaSuccess) return e;
     if (index_tc_available(a)) {
-        e = launch_index_scores_tc(a, scores, hist, nullptr, stream);
+        e = launch_index_scores_tc(a, scores, hist, a.dev_status, stream);
     } else {
         e = launch_index_scores(a, scores, stream);
         if (e == cudaSuccess) {

@@ -99,6 +99,9 @@ struct IdxTcArgs {
     const float* w;          // [rows][HI]
     const float* kscale;     // [B][N] (FP8) or null
     const uint8_t* kexp;     // [B][N][4] MXFP4 block exponents or null
+    const int32_t* bt;       // paged keys: block table [B][bt_stride], epb entries per block; null = contiguous
+    int bt_stride, epb;
+    long long n_blocks;      // blocks in the pools; an id outside [0, n_blocks) reads as zero keys
     float* scores;           // [rows][N]
     uint32_t* hist;          // [rows][4096]
     int* err;                // device fault word (may be null)
@@ -151,6 +154,22 @@ __device__ __forceinline__ long long nvis_of(int qj, const IdxTcArgs& a) {
     return nv > a.n_ent ? a.n_ent : nv;
 }
 
+// pool row of entry e (< n_ent) of sequence bat, or -1 for a block id outside the pool
+__device__ __forceinline__ long long key_row(const IdxTcArgs& a, int bat, long long e) {
+    if (!a.bt) return (long long)bat * a.n_ent + e;
+    const long long blk = a.bt[(long long)bat * a.bt_stride + e / a.epb];
+    return (blk >= 0 && blk < a.n_blocks) ? blk * a.epb + e % a.epb : -1;
+}
+// first pool row of the block holding entries e .. e+epb-1, or -epb (a box the TMA fills with zeros)
+// past the last entry or for a block id outside the pool (reported)
+__device__ __forceinline__ int block_row(const IdxTcArgs& a, int bat, long long e) {
+    if (e >= a.n_ent) return -a.epb;
+    const long long blk = a.bt[(long long)bat * a.bt_stride + e / a.epb];
+    if (blk >= 0 && blk < a.n_blocks) return (int)(blk * a.epb);
+    if (a.err) atomicExch(a.err, (int)V4A_ERR_DEVICE_FAULT);
+    return -a.epb;
+}
+
 template <bool FP8, int G>
 __device__ void idx_producer(IdxSmem& sm, const IdxTcArgs& a, const CUtensorMap* kmap, long long f0, long long f1) {
     constexpr int kSt = Ring<FP8>::kStages, kBytes = Ring<FP8>::kStageBytes;
@@ -163,8 +182,17 @@ __device__ void idx_producer(IdxSmem& sm, const IdxTcArgs& a, const CUtensorMap*
         const int y = (int)((long long)cur.bat * a.n_ent + (long long)cur.ti * kTileK);
         uint8_t* dst = sm.ring + st * kBytes;
         tc::mbar_arrive_expect_tx(&sm.k_full[st], kBytes);
-        tc::tma_load_2d(dst, kmap, 0, y, &sm.k_full[st]);
-        if (!FP8) tc::tma_load_2d(dst + kTileK * 128, kmap, 64, y, &sm.k_full[st]);  // second 64-column slab
+        if (a.bt) {
+            // paged keys: one box of epb rows per block of the tile
+            for (int j = 0; j < kTileK / a.epb; ++j) {
+                const int yb = block_row(a, cur.bat, (long long)cur.ti * kTileK + (long long)j * a.epb);
+                tc::tma_load_2d(dst + j * a.epb * 128, kmap, 0, yb, &sm.k_full[st]);
+                if (!FP8) tc::tma_load_2d(dst + kTileK * 128 + j * a.epb * 128, kmap, 64, yb, &sm.k_full[st]);
+            }
+        } else {
+            tc::tma_load_2d(dst, kmap, 0, y, &sm.k_full[st]);
+            if (!FP8) tc::tma_load_2d(dst + kTileK * 128, kmap, 64, y, &sm.k_full[st]);  // second 64-column slab
+        }
     }
     // no copy may still be in flight when the CTA exits
     for (long long jt = n - kSt; jt < n; ++jt)
@@ -372,7 +400,8 @@ struct XPrefetch {
     __device__ __forceinline__ void issue(IdxSmem& sm, const IdxTcArgs& a) {
         if (f < f1) {
             const long long e = (long long)cur.ti * kTileK + kHalf * hf + r;
-            if (e < a.n_ent) tc::cp_async_4(&sm.xring[(int)((f - f0) % kXSlots)][et], src + (long long)cur.bat * a.n_ent + e);
+            const long long kr = e < a.n_ent ? key_row(a, cur.bat, e) : -1;
+            if (kr >= 0) tc::cp_async_4(&sm.xring[(int)((f - f0) % kXSlots)][et], src + kr);
             cur.next(a);
             ++f;
         }
@@ -563,9 +592,17 @@ __device__ void mx_producer(IdxSmem& sm, const IdxTcArgs& a, const CUtensorMap* 
         }
         const int y = (int)((long long)cur.bat * a.n_ent + (long long)cur.ti * kMxTile);
         tc::mbar_arrive_expect_tx(&sm.k_full[st], (uint32_t)kMxStageBytes);
-        // boxes of 256 rows; rows past the tensor's end are filled with zeros (and still counted)
-        tc::tma_load_2d(sm.ring + st * kMxStageBytes, kmap, 0, y, &sm.k_full[st]);
-        tc::tma_load_2d(sm.ring + st * kMxStageBytes + kMxStageBytes / 2, kmap, 0, y + 256, &sm.k_full[st]);
+        if (a.bt) {
+            // paged keys: one box of epb rows per block of the tile
+            for (int j = 0; j < kMxTile / a.epb; ++j) {
+                const int yb = block_row(a, cur.bat, (long long)cur.ti * kMxTile + (long long)j * a.epb);
+                tc::tma_load_2d(sm.ring + st * kMxStageBytes + j * a.epb * 64, kmap, 0, yb, &sm.k_full[st]);
+            }
+        } else {
+            // boxes of 256 rows; rows past the tensor's end are filled with zeros (and still counted)
+            tc::tma_load_2d(sm.ring + st * kMxStageBytes, kmap, 0, y, &sm.k_full[st]);
+            tc::tma_load_2d(sm.ring + st * kMxStageBytes + kMxStageBytes / 2, kmap, 0, y + 256, &sm.k_full[st]);
+        }
     }
     // no copy may still be in flight when the CTA exits
     for (long long jt = n - kMxStages; jt < n; ++jt)
@@ -680,11 +717,12 @@ __device__ void mx_stage(IdxSmem& sm, const IdxTcArgs& a, uint32_t tmem, long lo
     auto prefetch = [&]() {
         if (fp < f1) {
             const int xs = (int)((fp - f0) % kMxXSlots);
-            const long long e0 = (long long)pre.ti * kMxTile + lane, base = (long long)pre.bat * a.n_ent;
+            const long long e0 = (long long)pre.ti * kMxTile + lane;
 #pragma unroll
             for (int w = 0; w < 16; ++w) {
                 const long long e = e0 + 32 * w;  // word w: quarter w / 4, column w % 4
-                if (e < a.n_ent) tc::cp_async_4(&sm.mx_xring[xs][w][ct], src + base + e);
+                const long long kr = e < a.n_ent ? key_row(a, pre.bat, e) : -1;
+                if (kr >= 0) tc::cp_async_4(&sm.mx_xring[xs][w][ct], src + kr);
             }
             pre.next(a);
             ++fp;
@@ -858,9 +896,9 @@ PFN_cuTensorMapEncodeTiled_v12000 idx_encode_fn() {
 cudaError_t launch_index_scores_mx(const IndexArgs& a, float* scores, uint32_t* hist, int* err, cudaStream_t stream,
                                    PFN_cuTensorMapEncodeTiled_v12000 fn) {
     CUtensorMap kmap;
-    cuuint64_t dims[2] = {64, (cuuint64_t)((long long)a.batch * a.n_ent)};
+    cuuint64_t dims[2] = {64, (cuuint64_t)(a.bt ? a.pool_rows : (long long)a.batch * a.n_ent)};
     cuuint64_t strides[1] = {64};
-    cuuint32_t box[2] = {64u, (cuuint32_t)kTileK};
+    cuuint32_t box[2] = {64u, (cuuint32_t)(a.bt ? a.epb : kTileK)};
     cuuint32_t estr[2] = {1, 1};
     if (fn(&kmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(a.k), dims, strides, box, estr,
            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -871,6 +909,10 @@ cudaError_t launch_index_scores_mx(const IndexArgs& a, float* scores, uint32_t* 
     t.w = a.w;
     t.kscale = nullptr;
     t.kexp = a.kexp;
+    t.bt = a.bt;
+    t.bt_stride = a.bt_stride;
+    t.epb = a.epb;
+    t.n_blocks = a.epb > 0 ? a.pool_rows / a.epb : 0;
     t.scores = scores;
     t.hist = hist;
     t.err = err;
@@ -901,9 +943,11 @@ cudaError_t launch_index_scores_mx(const IndexArgs& a, float* scores, uint32_t* 
 }  // namespace
 
 bool index_tc_shape_ok(const IndexArgs& a) {
+    // paged keys: blocks of 8 .. 256 entries (a power of two), so a tile is whole blocks
+    const bool paged_ok = !a.bt || (a.epb >= 8 && a.epb <= 256 && (a.epb & (a.epb - 1)) == 0 && a.pool_rows < (1LL << 31));
     return a.d_i == kDI && a.heads_i <= 32 && a.q_dtype == V4A_BF16 &&
            (a.k_dtype == V4A_BF16 || a.k_dtype == V4A_FP8E4M3 || (a.k_dtype == V4A_MXFP4 && a.kexp)) &&
-           a.n_ent >= 1 && (long long)a.batch * a.n_ent < (1LL << 31);
+           a.n_ent >= 1 && (long long)a.batch * a.n_ent < (1LL << 31) && paged_ok;
 }
 
 bool index_tc_available(const IndexArgs& a) { return index_tc_shape_ok(a) && idx_encode_fn() != nullptr; }
@@ -914,9 +958,9 @@ cudaError_t launch_index_scores_tc(const IndexArgs& a, float* scores, uint32_t* 
     if (a.k_dtype == V4A_MXFP4) return launch_index_scores_mx(a, scores, hist, err, stream, fn);
     const bool fp8 = a.k_dtype == V4A_FP8E4M3;
     CUtensorMap kmap;
-    cuuint64_t dims[2] = {(cuuint64_t)kDI, (cuuint64_t)((long long)a.batch * a.n_ent)};
+    cuuint64_t dims[2] = {(cuuint64_t)kDI, (cuuint64_t)(a.bt ? a.pool_rows : (long long)a.batch * a.n_ent)};
     cuuint64_t strides[1] = {(cuuint64_t)kDI * (fp8 ? 1 : 2)};
-    cuuint32_t box[2] = {fp8 ? 128u : 64u, (cuuint32_t)kTileK};
+    cuuint32_t box[2] = {fp8 ? 128u : 64u, (cuuint32_t)(a.bt ? a.epb : kTileK)};
     cuuint32_t estr[2] = {1, 1};
     if (fn(&kmap, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(a.k),
            dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -927,6 +971,10 @@ cudaError_t launch_index_scores_tc(const IndexArgs& a, float* scores, uint32_t* 
     t.w = a.w;
     t.kscale = a.kscale;
     t.kexp = nullptr;
+    t.bt = a.bt;
+    t.bt_stride = a.bt_stride;
+    t.epb = a.epb;
+    t.n_blocks = a.epb > 0 ? a.pool_rows / a.epb : 0;
     t.scores = scores;
     t.hist = hist;
     t.err = err;

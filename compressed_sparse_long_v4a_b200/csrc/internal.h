@@ -19,6 +19,12 @@ cudaError_t launch_compress_dual(const v4a_compress_io* a, const v4a_series_b* b
                                  cudaStream_t stream);
 cudaError_t launch_quantize_mxfp4(const void* x, v4a_dtype dt, long long rows, int cols, uint8_t* codes,
                                   uint8_t* exps, cudaStream_t stream);
+// compression whose outputs go to a paged pool: entry first_entry + s of sequence b -> pool row
+// bt[b*bt_stride + (first_entry+s)/epb]*epb + (first_entry+s)%epb (out_batch_stride ignored)
+cudaError_t launch_compress_paged(const v4a_compress_io* kv, const v4a_compress_io* idx, int batch, long long n_tok,
+                                  int m, long long first_entry, const int32_t* bt, int bt_stride, int epb,
+                                  long long n_blocks, cudaStream_t stream);
+cudaError_t launch_ring_append(const v4a_ring_io* io, int n, int batch, long long pos, cudaStream_t stream);
 
 // ---- indexer.cu -------------------------------------------------------
 struct IndexArgs {
@@ -27,6 +33,12 @@ struct IndexArgs {
     const void* k;        // [B][N][DI]
     const float* kscale;  // [B][N] or null
     const uint8_t* kexp;  // [B][N][DI/32] MXFP4 block exponents (k_dtype MXFP4), else null
+    // paged classical cache (as AttendArgs): keys, scales and exponents are pools of pool_rows rows; a
+    // block id outside the pool reads as a block of zero keys
+    const int32_t* bt;
+    int bt_stride, epb;
+    long long pool_rows;
+    int* dev_status;  // nullable: V4A_ERR_DEVICE_FAULT for a block id outside the pool
     v4a_dtype q_dtype, k_dtype;
     int batch, n_q, m, heads_i, d_i;
     long long ctx_len, n_ent;
@@ -59,6 +71,12 @@ struct AttendArgs {
     const float* sink;  // [heads] sink logits, or null
     int rope_dims;      // 0, or the output dims rotated at minus the query position
     float rope_base;
+    // paged classical cache: entry s of sequence b is row bt[b*bt_stride + s/epb]*epb + s%epb of
+    // `entries` (a pool of pool_rows rows); bt null = contiguous [B][N][d]
+    const int32_t* bt;
+    int bt_stride, epb;
+    long long pool_rows;  // n_blocks * epb; a block id outside [0, n_blocks) is a bad index
+    int ring_rows;  // > 0: token_kv is a ring [B][ring_rows][d] holding position p in row p % ring_rows
 };
 
 size_t attend_workspace_bytes(const AttendArgs& a);

@@ -103,6 +103,10 @@ v4a_status index_args(const void* q_i, const float* w, const void* k_i, const fl
     a->k = k_i;
     a->kscale = k_dt == V4A_MXFP4 ? nullptr : k_scale;
     a->kexp = k_dt == V4A_MXFP4 ? k_exp : nullptr;
+    a->bt = nullptr;
+    a->bt_stride = a->epb = 0;
+    a->pool_rows = 0;
+    a->dev_status = nullptr;
     a->q_dtype = q_dt;
     a->k_dtype = k_dt;
     a->batch = s->batch;
@@ -158,6 +162,25 @@ v4a_status attend_args(const void* q, const void* entries, const int32_t* idx, c
     a->ctx_len = s->ctx_len;
     a->n_ent = s->ctx_len / s->m;
     a->dev_status = dev_status;
+    a->bt = nullptr;
+    a->bt_stride = a->epb = 0;
+    a->pool_rows = 0;
+    a->ring_rows = 0;
+    return V4A_OK;
+}
+
+// checks a heterogeneous-cache descriptor for compression rate m and `entries` entries per sequence
+v4a_status paged_check(const v4a_paged* pg, int m, long long entries, const char* what) {
+    if (!pg || !pg->block_table) return fail(V4A_ERR_INVALID_ARG, "%s: a block table is required", what);
+    if (!aligned(pg->block_table, 4)) return fail(V4A_ERR_INVALID_ARG, "%s: block_table misaligned", what);
+    if (pg->block_tokens < m || pg->block_tokens % m)
+        return fail(V4A_ERR_INVALID_ARG, "%s: block_tokens must be a positive multiple of m", what);
+    if (pg->n_blocks < 1) return fail(V4A_ERR_INVALID_ARG, "%s: n_blocks must be >= 1", what);
+    const long long epb = pg->block_tokens / m;
+    if (pg->bt_stride < 0 || (long long)pg->bt_stride * epb < entries)
+        return fail(V4A_ERR_INVALID_ARG, "%s: the block table holds %lld entries per sequence, %lld needed", what,
+                    (long long)pg->bt_stride * epb, entries);
+    if (pg->n_blocks * epb >= (1LL << 31)) return fail(V4A_ERR_UNSUPPORTED, "%s: pool too large", what);
     return V4A_OK;
 }
 
@@ -262,6 +285,87 @@ v4a_status v4a_topk_mxfp4(const void* q_i, const float* w, const uint8_t* k_code
 }
 
 
+static v4a_status topk_paged_common(v4a::IndexArgs& a, int32_t* idx_out, float* score_out, void* workspace,
+                                    size_t workspace_bytes, int* dev_status, const v4a_paged* pg,
+                                    const v4a_shape* shape, void* stream, const char* what) {
+    v4a_status st = paged_check(pg, shape->m, a.n_ent, what);
+    if (st != V4A_OK) return st;
+    if (dev_status && !aligned(dev_status, 4)) return fail(V4A_ERR_INVALID_ARG, "%s: dev_status misaligned", what);
+    a.bt = pg->block_table;
+    a.bt_stride = pg->bt_stride;
+    a.epb = pg->block_tokens / shape->m;
+    a.pool_rows = pg->n_blocks * a.epb;
+    a.dev_status = dev_status;
+    if (dev_status) {
+        cudaError_t e = cudaMemsetAsync(dev_status, 0, sizeof(int), (cudaStream_t)stream);
+        if (e != cudaSuccess) return from_cuda(e, "dev_status reset");
+    }
+    return topk_common(a, idx_out, score_out, workspace, workspace_bytes, shape, stream, what);
+}
+
+v4a_status v4a_topk_paged(const void* q_i, const float* w, const void* k_i, const float* k_scale, int32_t* idx_out,
+                          float* score_out, int heads_i, int d_i, v4a_dtype q_dtype, v4a_dtype k_dtype,
+                          void* workspace, size_t workspace_bytes, int* dev_status, const v4a_paged* pg,
+                          const v4a_shape* shape, void* stream) {
+    if (k_dtype == V4A_MXFP4) return fail(V4A_ERR_UNSUPPORTED, "MXFP4 keys: use v4a_topk_mxfp4_paged");
+    v4a::IndexArgs a;
+    v4a_status st = index_args(q_i, w, k_i, k_scale, nullptr, heads_i, d_i, q_dtype, k_dtype, shape, &a);
+    if (st != V4A_OK) return st;
+    return topk_paged_common(a, idx_out, score_out, workspace, workspace_bytes, dev_status, pg, shape, stream,
+                             "v4a_topk_paged");
+}
+
+v4a_status v4a_topk_mxfp4_paged(const void* q_i, const float* w, const uint8_t* k_codes, const uint8_t* k_exp,
+                                int32_t* idx_out, float* score_out, int heads_i, int d_i, v4a_dtype q_dtype,
+                                void* workspace, size_t workspace_bytes, int* dev_status, const v4a_paged* pg,
+                                const v4a_shape* shape, void* stream) {
+    v4a::IndexArgs a;
+    v4a_status st = index_args(q_i, w, k_codes, nullptr, k_exp, heads_i, d_i, q_dtype, V4A_MXFP4, shape, &a);
+    if (st != V4A_OK) return st;
+    return topk_paged_common(a, idx_out, score_out, workspace, workspace_bytes, dev_status, pg, shape, stream,
+                             "v4a_topk_mxfp4_paged");
+}
+
+v4a_status v4a_compress_paged(const v4a_compress_io* kv, const v4a_compress_io* idx, int batch, long long n_tok, int m,
+                              long long first_entry, const v4a_paged* pg, void* stream) {
+    if (!kv) return fail(V4A_ERR_INVALID_ARG, "kv stream is NULL");
+    if (batch < 0 || n_tok < 0 || m < 1 || first_entry < 0)
+        return fail(V4A_ERR_INVALID_ARG, "need batch >= 0, n_tok >= 0, m >= 1, first_entry >= 0");
+    const long long n_ent = n_tok / m;
+    if (batch == 0 || n_ent == 0) return V4A_OK;
+    v4a_status st = paged_check(pg, m, first_entry + n_ent, "v4a_compress_paged");
+    if (st != V4A_OK) return st;
+    // the pools take the place of per-sequence outputs: check each stream as if its output rows were its own
+    for (const v4a_compress_io* io : {kv, idx}) {
+        if (!io) continue;
+        v4a_compress_io c = *io;
+        c.out_batch_stride = n_ent * c.channels;
+        c.scale_batch_stride = n_ent;
+        c.exp_batch_stride = n_ent * (c.channels / 32);
+        st = check_compress_io(&c, io == kv ? "kv" : "idx", n_tok, m);
+        if (st != V4A_OK) return st;
+    }
+    return from_cuda(v4a::launch_compress_paged(kv, idx, batch, n_tok, m, first_entry, pg->block_table, pg->bt_stride,
+                                                pg->block_tokens / m, pg->n_blocks, (cudaStream_t)stream),
+                     "v4a_compress_paged");
+}
+
+v4a_status v4a_ring_append(const v4a_ring_io* io, int n_streams, int batch, long long pos, void* stream) {
+    if (n_streams < 0 || n_streams > 8) return fail(V4A_ERR_INVALID_ARG, "v4a_ring_append: 0 .. 8 streams");
+    if (batch < 0 || pos < 0) return fail(V4A_ERR_INVALID_ARG, "v4a_ring_append: need batch >= 0, pos >= 0");
+    if (n_streams == 0 || batch == 0) return V4A_OK;
+    if (!io) return fail(V4A_ERR_INVALID_ARG, "v4a_ring_append: io is NULL");
+    for (int i = 0; i < n_streams; ++i) {
+        const v4a_ring_io& r = io[i];
+        const size_t es = dtype_size(r.dtype);
+        if (!r.src || !r.ring || r.channels < 1 || r.ring_rows < 1 || ((size_t)r.channels * es) % 16 ||
+            !aligned(r.src, 16) || !aligned(r.ring, 16) || ((size_t)r.src_batch_stride * es) % 16 ||
+            r.src_batch_stride < r.channels)
+            return fail(V4A_ERR_INVALID_ARG, "v4a_ring_append: stream %d: pointers, sizes or strides", i);
+    }
+    return from_cuda(v4a::launch_ring_append(io, n_streams, batch, pos, (cudaStream_t)stream), "v4a_ring_append");
+}
+
 v4a_status v4a_quantize_mxfp4(const void* x, v4a_dtype dtype, long long rows, int cols, uint8_t* codes,
                               uint8_t* exps, void* stream) {
     if (rows < 0 || cols < 32 || cols % 32)
@@ -278,10 +382,19 @@ v4a_status v4a_quantize_mxfp4(const void* x, v4a_dtype dtype, long long rows, in
 static v4a_status attend_common(const void* q, const void* entries, const int32_t* idx, const void* token_kv,
                                 long long tok_pos0, long long l_tok, float* out, v4a_dtype dtype, void* workspace,
                                 size_t workspace_bytes, int* dev_status, const v4a_attend_ext* ext,
-                                const v4a_shape* shape, void* stream, bool csa) {
+                                const v4a_shape* shape, void* stream, bool csa, const v4a_paged* pg = nullptr) {
     v4a::AttendArgs a;
     v4a_status st = attend_args(q, entries, idx, token_kv, tok_pos0, l_tok, out, dtype, dev_status, shape, csa, &a);
     if (st != V4A_OK) return st;
+    if (pg) {
+        a.bt = pg->block_table;
+        a.bt_stride = pg->bt_stride;
+        a.epb = pg->block_tokens / shape->m;
+        a.pool_rows = pg->n_blocks * a.epb;
+        a.ring_rows = pg->ring_rows;
+        a.l_tok = pg->ring_rows;
+        a.tok_pos0 = 0;
+    }
     a.sink = nullptr;
     a.rope_dims = 0;
     a.rope_base = 10000.f;
@@ -333,6 +446,35 @@ v4a_status v4a_hca_attend(const void* q, const void* entries, const void* token_
                           const v4a_shape* shape, void* stream) {
     return attend_common(q, entries, nullptr, token_kv, tok_pos0, l_tok, out, dtype, workspace, workspace_bytes,
                          nullptr, nullptr, shape, stream, false);
+}
+
+static v4a_status attend_paged(const void* q, const void* entries, const int32_t* idx, const void* token_kv, float* out,
+                               v4a_dtype dtype, void* workspace, size_t workspace_bytes, int* dev_status,
+                               const v4a_attend_ext* ext, const v4a_paged* pg, const v4a_shape* shape, void* stream,
+                               bool csa) {
+    const char* what = csa ? "v4a_csa_attend_paged" : "v4a_hca_attend_paged";
+    if (!shape) return fail(V4A_ERR_INVALID_ARG, "shape is NULL");
+    v4a_status st = paged_check(pg, shape->m > 0 ? shape->m : 1, shape->m > 0 ? shape->ctx_len / shape->m : 0, what);
+    if (st != V4A_OK) return st;
+    if (shape->window > 0 && (pg->ring_rows < 1 || (long long)pg->ring_rows < (long long)shape->window + shape->n_q - 1))
+        return fail(V4A_ERR_INVALID_ARG, "%s: the ring of %d rows cannot hold the window (%d + %d - 1)", what,
+                    pg->ring_rows, shape->window, shape->n_q);
+    return attend_common(q, entries, idx, token_kv, 0, shape->ctx_len, out, dtype, workspace, workspace_bytes,
+                         dev_status, ext, shape, stream, csa, pg);
+}
+
+v4a_status v4a_csa_attend_paged(const void* q, const void* entries, const int32_t* idx, const void* token_kv, float* out,
+                                v4a_dtype dtype, void* workspace, size_t workspace_bytes, int* dev_status,
+                                const v4a_attend_ext* ext, const v4a_paged* pg, const v4a_shape* shape, void* stream) {
+    return attend_paged(q, entries, idx, token_kv, out, dtype, workspace, workspace_bytes, dev_status, ext, pg, shape,
+                        stream, true);
+}
+
+v4a_status v4a_hca_attend_paged(const void* q, const void* entries, const void* token_kv, float* out, v4a_dtype dtype,
+                                void* workspace, size_t workspace_bytes, int* dev_status, const v4a_attend_ext* ext,
+                                const v4a_paged* pg, const v4a_shape* shape, void* stream) {
+    return attend_paged(q, entries, nullptr, token_kv, out, dtype, workspace, workspace_bytes, dev_status, ext, pg,
+                        shape, stream, false);
 }
 
 size_t v4a_workspace_size(const char* op, const v4a_shape* shape, int heads_i, int d_i) {

@@ -310,6 +310,95 @@ V4A_API v4a_status v4a_hca_attend_ex(const void* q, const void* entries, const v
                                      void* stream);
 
 /* ------------------------------------------------------------------ */
+/* heterogeneous KV cache: paged classical cache + token rings          */
+/* ------------------------------------------------------------------ */
+
+/* "DeepSeek-V4: Million-Token Context via Hybrid Compressed Attention",
+ * "KV Cache Management" / "KV Cache Layout": the cache is split into a
+ * classical cache of compressed entries (CSA / HCA), allocated in blocks that
+ * each cover lcm(m, m') original tokens (128 in V4: 32 CSA entries with their
+ * indexer keys, or 1 HCA entry), and a state cache pre-allocated per sequence
+ * for the sliding window and the tokens of the still incomplete chunks.
+ * Here the classical cache of a layer is a pool of n_blocks blocks: entries
+ * (and keys, scales, exponents) are pools of n_blocks * epb rows, epb =
+ * block_tokens / m, and entry s of sequence b is pool row
+ *     block_table[b * bt_stride + s / epb] * epb + s % epb.
+ * The state cache is a ring of ring_rows token rows per sequence for each
+ * stream (K = V rows, gate logits, indexer rows): position p is row
+ * p % ring_rows.  A decode step appends the new token to the rings
+ * (v4a_ring_append), compresses a chunk into its block once its last token
+ * has arrived (v4a_compress_paged, reading the chunk's rows from the rings),
+ * and attends through the block table and the ring (the _paged calls).  All
+ * sequences of a call are at the same position (ctx_len).
+ * A block id outside [0, n_blocks) is a bad index: attention skips those
+ * entries and reports V4A_ERR_DEVICE_FAULT in dev_status, the indexer scores
+ * them as all-zero keys, compression does not write them. */
+typedef struct v4a_paged {
+    const int32_t* block_table;  /* [batch][bt_stride] block ids (device) */
+    int bt_stride;               /* block-table entries per sequence (>= the blocks the context needs) */
+    int block_tokens;            /* tokens per block, a multiple of m: lcm(m, m') = 128 in V4 */
+    long long n_blocks;          /* blocks in the pools */
+    int ring_rows;               /* rows of each sequence's token ring (attention calls; a multiple of m for
+                                    compression), >= window + n_q - 1 */
+} v4a_paged;
+
+/* One stream of a ring append: the new token's row of each sequence. */
+typedef struct v4a_ring_io {
+    const void* src;             /* [batch] rows of `channels` elements, src_batch_stride elements apart */
+    void* ring;                  /* [batch][ring_rows][channels] */
+    int channels;                /* channels * element size a multiple of 16 bytes */
+    int ring_rows;
+    v4a_dtype dtype;             /* F32, BF16 (or FP8E4M3 / MXFP4 bytes copied as such) */
+    long long src_batch_stride;  /* elements */
+} v4a_ring_io;
+
+/* Append the token at position pos to up to 8 rings in one launch: row b of
+ * io[i].src goes to ring row pos % ring_rows of sequence b.  Pointers
+ * 16-byte aligned.  Errors: V4A_ERR_INVALID_ARG for n_streams outside 0..8,
+ * NULL or misaligned pointers, rows not a multiple of 16 bytes, pos < 0. */
+V4A_API v4a_status v4a_ring_append(const v4a_ring_io* io, int n_streams, int batch, long long pos, void* stream);
+
+/* v4a_compress whose entries go to paged pools: for each stream the chunk
+ * rows are read as for v4a_compress (x / gate with their batch strides, e.g.
+ * a slice of the rings), and entry first_entry + s of sequence b (s <
+ * n_tok / m) is written to pool row block_table[b * bt_stride + e / epb] *
+ * epb + e % epb, e = first_entry + s, epb = pg->block_tokens / m (out,
+ * out_scale and out_exp are pools; their batch strides are ignored).
+ * Errors: those of v4a_compress, plus V4A_ERR_INVALID_ARG for a NULL
+ * block table, block_tokens not a multiple of m, n_blocks < 1 or entries
+ * beyond bt_stride * epb. */
+V4A_API v4a_status v4a_compress_paged(const v4a_compress_io* kv, const v4a_compress_io* idx, int batch, long long n_tok,
+                                      int m, long long first_entry, const v4a_paged* pg, void* stream);
+
+/* v4a_topk over paged keys: k_i (and k_scale for FP8E4M3) are pools of
+ * n_blocks * epb rows addressed through pg's block table; everything else
+ * as v4a_topk.  dev_status (nullable, device int) is set to V4A_OK and to
+ * V4A_ERR_DEVICE_FAULT if a block id lies outside the pool. */
+V4A_API v4a_status v4a_topk_paged(const void* q_i, const float* w, const void* k_i, const float* k_scale,
+                                  int32_t* idx_out, float* score_out, int heads_i, int d_i, v4a_dtype q_dtype,
+                                  v4a_dtype k_dtype, void* workspace, size_t workspace_bytes, int* dev_status,
+                                  const v4a_paged* pg, const v4a_shape* shape, void* stream);
+/* The same with MXFP4 keys (k_codes / k_exp pools, see v4a_topk_mxfp4). */
+V4A_API v4a_status v4a_topk_mxfp4_paged(const void* q_i, const float* w, const uint8_t* k_codes, const uint8_t* k_exp,
+                                        int32_t* idx_out, float* score_out, int heads_i, int d_i, v4a_dtype q_dtype,
+                                        void* workspace, size_t workspace_bytes, int* dev_status,
+                                        const v4a_paged* pg, const v4a_shape* shape, void* stream);
+
+/* v4a_csa_attend_ex / v4a_hca_attend_ex over the heterogeneous cache:
+ * entries is a pool addressed through pg's block table (epb =
+ * block_tokens / m) and token_kv is the K = V ring ([batch][ring_rows][d],
+ * position p in row p % ring_rows; pg->ring_rows >= window + n_q - 1).
+ * Everything else (ext included) as the _ex calls. */
+V4A_API v4a_status v4a_csa_attend_paged(const void* q, const void* entries, const int32_t* idx, const void* token_kv,
+                                        float* out, v4a_dtype dtype, void* workspace, size_t workspace_bytes,
+                                        int* dev_status, const v4a_attend_ext* ext, const v4a_paged* pg,
+                                        const v4a_shape* shape, void* stream);
+V4A_API v4a_status v4a_hca_attend_paged(const void* q, const void* entries, const void* token_kv, float* out,
+                                        v4a_dtype dtype, void* workspace, size_t workspace_bytes, int* dev_status,
+                                        const v4a_attend_ext* ext, const v4a_paged* pg, const v4a_shape* shape,
+                                        void* stream);
+
+/* ------------------------------------------------------------------ */
 /* housekeeping                                                         */
 /* ------------------------------------------------------------------ */
 

@@ -108,6 +108,38 @@ def test_mxfp4_host_side_argument_errors(v4a):
     assert b"out_exp" in L.v4a_last_error()
 
 
+def test_paged_host_side_argument_errors(v4a):
+    L = v4a.lib
+    shape = v4a.Shape(1, 1, 64, 512, 4, 8, 128, 1024)
+    bt = ctypes.c_int32 * 8
+    tab = bt()
+    # no block table
+    pg = v4a.Paged(None, 8, 128, 4, 256)
+    assert L.v4a_topk_paged(16, 16, 16, None, 16, None, 4, 64, 1, 1, 256, 1 << 20, None, ctypes.byref(pg),
+                            ctypes.byref(shape), None) == 1
+    assert b"block table" in L.v4a_last_error()
+    # block_tokens not a multiple of m, then a table too short for the context (1024/4 = 256 entries)
+    fake = 1 << 20  # a device-looking pointer that is never dereferenced on the host
+    pg = v4a.Paged(fake, 8, 130, 4, 256)
+    assert L.v4a_topk_paged(16, 16, 16, None, 16, None, 4, 64, 1, 1, 256, 1 << 20, None, ctypes.byref(pg),
+                            ctypes.byref(shape), None) == 1
+    pg = v4a.Paged(fake, 4, 128, 4, 256)
+    assert L.v4a_topk_paged(16, 16, 16, None, 16, None, 4, 64, 1, 1, 256, 1 << 20, None, ctypes.byref(pg),
+                            ctypes.byref(shape), None) == 1
+    assert b"block table" in L.v4a_last_error()
+    # a ring that cannot hold the window
+    pg = v4a.Paged(fake, 8, 128, 4, 100)
+    assert L.v4a_csa_attend_paged(16, 16, 16, 16, 16, 1, 256, 1 << 20, None, None, ctypes.byref(pg),
+                                  ctypes.byref(shape), None) == 1
+    assert b"ring" in L.v4a_last_error()
+    # ring append: too many streams, misaligned rows
+    ios = (v4a.RingIO * 9)()
+    assert L.v4a_ring_append(ios, 9, 1, 0, None) == 1
+    ios[0] = v4a.RingIO(16, 16, 12, 256, 1, 12)  # 24-byte rows
+    assert L.v4a_ring_append(ios, 1, 1, 0, None) == 1
+    del tab
+
+
 def test_workspace_sizes(v4a):
     assert v4a.v4a_workspace_size("nonsense", batch=1) == 0
     ws = v4a.v4a_workspace_size("topk", batch=4, m=4, k=1024, ctx_len=1 << 20, heads_i=16, d_i=128)
