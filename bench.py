@@ -367,6 +367,106 @@ def measure_prefill(peaks: dict) -> dict:
     return res
 
 
+class PagedStep:
+    """The decode step over the heterogeneous cache: the same 1M-context CSA and HCA layers with their
+    compressed entries (and indexer keys) in pools of 128-token blocks (lcm(4, 128)) handed out in
+    shuffled order, and the window and the chunk tails in per-sequence token rings of 256 rows.  One
+    layer step: append the new token to the rings, compress the chunks that complete at t = L-1 into
+    their blocks, top-k through the block table, attend through the block table and the ring."""
+
+    BLOCK, RING = 128, 256
+
+    def __init__(self, step: "Step"):
+        v4a, c, h = step.v4a, step.cc, step.hc
+        self.v4a, self.step = v4a, step
+        g = torch.Generator().manual_seed(97)
+        dv = "cuda"
+
+        def pools(B, N, m):
+            epb = self.BLOCK // m
+            nb = (N + epb - 1) // epb
+            perm = torch.randperm(B * nb, generator=g).to(torch.int32)
+            bt = perm.view(B, nb).contiguous().to(dv)
+            s = torch.arange(N, device=dv)
+            rows = (bt[:, s // epb].long() * epb + (s % epb)).contiguous()  # [B][N] pool row of each entry
+            return bt, rows, B * nb * epb
+
+        self.bt_c, rows_c, P_c = pools(step.Bc, step.Nc, c["m"])
+        self.bt_h, rows_h, P_h = pools(step.Bh, step.Nh, h["m"])
+        d, di = c["d"], c["d_i"]
+        self.ent_c = torch.zeros((P_c, d), dtype=torch.bfloat16, device=dv)
+        self.ent_c[rows_c.view(-1)] = step.c_ent.view(-1, d)
+        self.key_c = torch.zeros((P_c, di), dtype=torch.uint8, device=dv)
+        self.key_c[rows_c.view(-1)] = step.c_ki.view(-1, di)
+        self.ksc_c = torch.ones((P_c,), dtype=torch.float32, device=dv)
+        self.ksc_c[rows_c.view(-1)] = step.c_ks.view(-1)
+        self.ent_h = torch.zeros((P_h, h["d"]), dtype=torch.bfloat16, device=dv)
+        self.ent_h[rows_h.view(-1)] = step.h_ent.view(-1, h["d"])
+        R = self.RING
+        # token rings: the window rows (and the completing chunks) at their positions p % R
+        def ring(rows_src, p_last, C, B):
+            r = torch.zeros((B, R, C), dtype=torch.bfloat16, device=dv)
+            n = rows_src.shape[1]
+            pos = torch.arange(p_last - n + 1, p_last + 1, device=dv) % R
+            r[:, pos] = rows_src
+            return r
+        Lc, Lh = step.Lc, step.Lh
+        self.r_kv_c = ring(step.c_tok, Lc - 1, d, step.Bc)
+        self.r_gc = ring(step.c_gate, Lc - 1, d, step.Bc)
+        self.r_xi = ring(step.c_xi, Lc - 1, di, step.Bc)
+        self.r_gi = ring(step.c_gi, Lc - 1, di, step.Bc)
+        self.r_kv_h = ring(step.h_tok, Lh - 1, h["d"], step.Bh)
+        self.r_gh = ring(step.h_gate, Lh - 1, h["d"], step.Bh)
+        # the newest token's rows (appended again each step: same bytes, the cost is the point)
+        self.new_c = [(step.c_tok[:, -1], self.r_kv_c), (step.c_gate[:, -1], self.r_gc), (step.c_xi[:, -1], self.r_xi),
+                      (step.c_gi[:, -1], self.r_gi)]
+        self.new_h = [(step.h_tok[:, -1], self.r_kv_h), (step.h_gate[:, -1], self.r_gh)]
+
+    def csa_layer(self):
+        st, c, v, R = self.step, self.step.cc, self.v4a, self.RING
+        m, L = c["m"], st.Lc
+        v.v4a_ring_append(self.new_c, L - 1)
+        r0 = (L - m) % R
+        v.v4a_compress_paged(self.r_kv_c[:, r0:r0 + m], self.r_gc[:, r0:r0 + m], self.ent_c, m=m,
+                             first_entry=L // m - 1, block_table=self.bt_c, block_tokens=self.BLOCK,
+                             xi=self.r_xi[:, r0:r0 + m], gate_i=self.r_gi[:, r0:r0 + m], out_i=self.key_c,
+                             out_i_scale=self.ksc_c)
+        v.v4a_topk_paged(st.c_qi, st.c_w, self.key_c, self.ksc_c, st.idx, m=m, k=c["k"], ctx_len=L,
+                         block_table=self.bt_c, block_tokens=self.BLOCK, workspace=st.ws_topk)
+        v.v4a_csa_attend_paged(st.c_q, self.ent_c, st.idx, self.r_kv_c, st.c_out, m=m, window=c["window"], ctx_len=L,
+                               block_table=self.bt_c, block_tokens=self.BLOCK, workspace=st.ws_csa,
+                               dev_status=st.status)
+
+    def hca_layer(self):
+        st, h, v, R = self.step, self.step.hc, self.v4a, self.RING
+        m, L = h["m"], st.Lh
+        v.v4a_ring_append(self.new_h, L - 1)
+        r0 = (L - m) % R
+        v.v4a_compress_paged(self.r_kv_h[:, r0:r0 + m], self.r_gh[:, r0:r0 + m], self.ent_h, m=m,
+                             first_entry=L // m - 1, block_table=self.bt_h, block_tokens=self.BLOCK)
+        v.v4a_hca_attend_paged(st.h_q, self.ent_h, self.r_kv_h, st.h_out, m=m, window=h["window"], ctx_len=L,
+                               block_table=self.bt_h, block_tokens=self.BLOCK, workspace=st.ws_hca,
+                               dev_status=st.status)
+
+
+def measure_paged(step: "Step", contiguous_ms: dict) -> dict:
+    ps = PagedStep(step)
+    ps.csa_layer()
+    ps.hca_layer()
+    torch.cuda.synchronize()
+    reps = 100
+    ms = {"csa": statistics.median(layer_times(ps.csa_layer, reps)),
+          "hca": statistics.median(layer_times(ps.hca_layer, reps))}
+    res = {"workload": "the 1M-context decode layers over the heterogeneous cache: entries and indexer keys in "
+                       "pools of 128-token blocks (shuffled block ids), window and chunk tails in 256-row token "
+                       "rings; one step = ring append + compress of the completing chunks + top-k + attention",
+           "ms_median": ms, "replays": reps, "contiguous_ms_median": contiguous_ms,
+           "tokens_per_s_median": {"csa": step.Bc / (ms["csa"] / 1000.0), "hca": step.Bh / (ms["hca"] / 1000.0)}}
+    del ps
+    torch.cuda.empty_cache()
+    return res
+
+
 def measure_fp4_indexer(step: "Step", flush: torch.Tensor, peak_gbs: float) -> dict:
     """The 1M-context CSA indexer with MXFP4 keys (FP4 dot products): the same 4 sequences x
     262,144 entries x 16 heads x 128, top-1024, with the keys drawn N(0,1) on the device (seeded)
@@ -703,8 +803,10 @@ def main():
     cpu = None
     prefill = None
     fp4 = None
+    paged = None
     if rank == 0 and world == 1:
         fp4 = measure_fp4_indexer(step, flush, peak)
+        paged = measure_paged(step, {"csa": layers["csa"]["ms_median"], "hca": layers["hca"]["ms_median"]})
         prefill = measure_prefill(peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, threads, sample, _ = oracle_sample(args.cpu_seconds, step)
@@ -724,6 +826,7 @@ def main():
                            "op_ms": op_ms,
                            "layers": layers},
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "prefill": prefill, "fp4_indexer": fp4,
+                "paged_cache": paged,
                 "gpu_launches": (launches_per_step * args.steps) if launches_per_step else None,
                 "gpu_launches_per_step": launches_per_step,
                 "clocks": clocks}

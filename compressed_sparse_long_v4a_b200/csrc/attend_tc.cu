@@ -180,17 +180,73 @@ __device__ __forceinline__ uint64_t gather_tile(uint8_t* dst, const __nv_bfloat1
     return mask;
 }
 
+// Rows of a gathered tile (CSA selections, paged entries, ring windows) for this lane: rows lane and
+// lane + 32 (src, ok).  False for tiles loaded with TMA.  Bad selections and block ids are reported here.
+__device__ __forceinline__ bool tile_rows(const TcArgs& a, int row, int ti, int lane, const __nv_bfloat16* (&src)[2],
+                                          bool (&ok)[2]) {
+    if (!tile_gathered(a, ti)) return false;
+    const RowInfo ri = row_info(row, a);
+    const __nv_bfloat16* fallback = a.q + (long long)row * kH * kD;  // finite data for excluded rows
+    if (ti < a.e_tiles) {
+        const long long c0 = (long long)ti * kTile;
+        if (a.idx) {
+            csa_rows(a, ri, row, c0, lane, src, ok);
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+                const long long c = c0 + lane + 32 * h2;
+                const long long sidx = c < a.k ? (long long)a.idx[(long long)row * a.k + c] : -1;
+                if (!ok[h2] && sidx != -1 && a.dev_status) atomicExch(a.dev_status, (int)V4A_ERR_DEVICE_FAULT);
+            }
+        } else {
+            // HCA over a paged pool: rows c0 .. c0+63 through the block table
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+                const long long s = c0 + lane + 32 * h2;
+                const __nv_bfloat16* er = s < ri.nvis ? entry_row(a, ri.b, s) : nullptr;
+                if (s < ri.nvis && !er && a.dev_status) atomicExch(a.dev_status, (int)V4A_ERR_DEVICE_FAULT);
+                ok[h2] = er != nullptr;
+                src[h2] = ok[h2] ? er : fallback;
+            }
+        }
+    } else {
+        // window tokens p0 .. p0+63 from the ring (they may wrap around its end)
+        const long long wi = ti - a.e_tiles;
+        const long long p0 = ri.t - a.window + 1 + wi * kTile;
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+            const int r = lane + 32 * h2;
+            const long long p = p0 + r;
+            ok[h2] = wi * kTile + r < a.window && p >= 0;
+            src[h2] = ok[h2] ? a.token_kv + ((long long)ri.b * a.ring_rows + p % a.ring_rows) * kD : fallback;
+        }
+    }
+    return true;
+}
+
 __device__ void producer(Smem& sm, const TcArgs& a, const CUtensorMap* ent_map, const CUtensorMap* tok_map,
                          const CUtensorMap* q_map, long long f0, long long f1) {
     const int lane = threadIdx.x & 31;
     int seg = 0;
     Cursor cur(f0, a.tpr);
+    // the rows of gathered tiles are worked out a tile ahead, so their index / block-table loads overlap
+    // the current tile's copies
+    const __nv_bfloat16* nsrc[2] = {a.q, a.q};
+    bool nok[2] = {false, false};
+    bool ngath = f0 < f1 && tile_rows(a, cur.row, cur.ti, lane, nsrc, nok);
     for (long long f = f0; f < f1; ++f, cur.next(a.tpr)) {
         if (sm.abort_flag) break;
         const int jt = (int)(f - f0), st = jt % kStages;
         const int row = cur.row, ti = cur.ti;
         const bool seg_start = (f == f0) || (ti == 0);
         const RowInfo ri = row_info(row, a);
+        const bool gath = ngath;
+        const __nv_bfloat16* src[2] = {nsrc[0], nsrc[1]};
+        const bool ok[2] = {nok[0], nok[1]};
+        if (f + 1 < f1) {
+            Cursor nx = cur;
+            nx.next(a.tpr);
+            ngath = tile_rows(a, nx.row, nx.ti, lane, nsrc, nok);
+        }
         if (seg_start) {
             if (seg > 0 && !tc::mbar_wait(&sm.q_empty, (seg - 1) & 1)) { fault(sm, a); break; }
             if (lane == 0) {
@@ -202,70 +258,22 @@ __device__ void producer(Smem& sm, const TcArgs& a, const CUtensorMap* ent_map, 
         if (jt >= kStages && !tc::mbar_wait(&sm.kv_empty[st], ((jt / kStages) - 1) & 1)) { fault(sm, a); break; }
         uint64_t mask = 0;
         uint8_t* dst = sm.kv[st];
-        if (ti < a.e_tiles) {
-            const long long c0 = (long long)ti * kTile;
-            if (!a.idx && a.bt) {
-                // HCA over a paged pool: rows c0 .. c0+63 through the block table
-                const __nv_bfloat16* src[2];
-                bool ok[2];
-#pragma unroll
-                for (int h2 = 0; h2 < 2; ++h2) {
-                    const long long s = c0 + lane + 32 * h2;
-                    const __nv_bfloat16* er = s < ri.nvis ? entry_row(a, ri.b, s) : nullptr;
-                    if (s < ri.nvis && !er && a.dev_status) atomicExch(a.dev_status, (int)V4A_ERR_DEVICE_FAULT);
-                    ok[h2] = er != nullptr;
-                    src[h2] = ok[h2] ? er : a.q + (long long)row * kH * kD;
-                }
-                mask = gather_tile(dst, src, ok, lane);
-                if (lane == 0) {
-                    sm.mask[st] = mask;
-                    tc::mbar_arrive_expect_tx(&sm.kv_full[st], 0);
-                }
-            } else if (!a.idx) {
-                // HCA: rows c0 .. c0+63 of this sequence's entries are contiguous
-                const long long nv = ri.nvis - c0;
-                mask = nv >= kTile ? ~0ull : (nv <= 0 ? 0ull : ((1ull << nv) - 1ull));
-                if (lane == 0) {
-                    sm.mask[st] = mask;
-                    tc::mbar_arrive_expect_tx(&sm.kv_full[st], kTileBytes);
-                    const int y = (int)((long long)ri.b * a.n_ent + c0);
-                    for (int c = 0; c < kSlabs; ++c) tc::tma_load_2d(dst + c * kSlabBytes, ent_map, 64 * c, y, &sm.kv_full[st]);
-                }
-            } else {
-                // CSA: gather the selected rows with cp.async (128-byte swizzle written by hand)
-                const __nv_bfloat16* src[2];
-                bool ok[2];
-                csa_rows(a, ri, row, c0, lane, src, ok);
-#pragma unroll
-                for (int h2 = 0; h2 < 2; ++h2) {
-                    const long long c = c0 + lane + 32 * h2;
-                    const long long sidx = c < a.k ? (long long)a.idx[(long long)row * a.k + c] : -1;
-                    if (!ok[h2] && sidx != -1 && a.dev_status) atomicExch(a.dev_status, (int)V4A_ERR_DEVICE_FAULT);
-                }
-                mask = gather_tile(dst, src, ok, lane);
-                if (lane == 0) {
-                    sm.mask[st] = mask;
-                    tc::mbar_arrive_expect_tx(&sm.kv_full[st], 0);
-                }
-            }
-        } else if (a.ring_rows > 0) {
-            // window tokens p0 .. p0+63 from the ring (they may wrap around its end)
-            const long long wi = ti - a.e_tiles;
-            const long long p0 = ri.t - a.window + 1 + wi * kTile;
-            const __nv_bfloat16* src[2];
-            bool ok[2];
-#pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-                const int r = lane + 32 * h2;
-                const long long p = p0 + r;
-                ok[h2] = wi * kTile + r < a.window && p >= 0;
-                src[h2] = ok[h2] ? a.token_kv + ((long long)ri.b * a.ring_rows + p % a.ring_rows) * kD
-                                 : a.q + (long long)row * kH * kD;
-            }
+        if (gath) {
             mask = gather_tile(dst, src, ok, lane);
             if (lane == 0) {
                 sm.mask[st] = mask;
                 tc::mbar_arrive_expect_tx(&sm.kv_full[st], 0);
+            }
+        } else if (ti < a.e_tiles) {
+            // HCA: rows c0 .. c0+63 of this sequence's entries are contiguous
+            const long long c0 = (long long)ti * kTile;
+            const long long nv = ri.nvis - c0;
+            mask = nv >= kTile ? ~0ull : (nv <= 0 ? 0ull : ((1ull << nv) - 1ull));
+            if (lane == 0) {
+                sm.mask[st] = mask;
+                tc::mbar_arrive_expect_tx(&sm.kv_full[st], kTileBytes);
+                const int y = (int)((long long)ri.b * a.n_ent + c0);
+                for (int c = 0; c < kSlabs; ++c) tc::tma_load_2d(dst + c * kSlabBytes, ent_map, 64 * c, y, &sm.kv_full[st]);
             }
         } else {
             // window tokens p0 .. p0+63 (contiguous rows of token_kv)

@@ -60,6 +60,7 @@ constexpr int kHistBins = 4096;          // top 12 bits of the ordered score key
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxDStages = 4;
 constexpr int kQBufBytes = 16384;        // B operand of one segment: up to 128 rows of 128 B
+constexpr int kMinEpb = 32;                // paged keys on this path: blocks of at least 32 entries
 constexpr int kMxXAhead = 3;               // MXFP4: 512-entry tiles of block exponents each staging thread fetches ahead
 constexpr int kMxXSlots = kMxXAhead + 1;
 
@@ -100,7 +101,7 @@ struct IdxTcArgs {
     const float* kscale;     // [B][N] (FP8) or null
     const uint8_t* kexp;     // [B][N][4] MXFP4 block exponents or null
     const int32_t* bt;       // paged keys: block table [B][bt_stride], epb entries per block; null = contiguous
-    int bt_stride, epb;
+    int bt_stride, epb, epb_shift;  // epb = 1 << epb_shift (this path takes power-of-two blocks)
     long long n_blocks;      // blocks in the pools; an id outside [0, n_blocks) reads as zero keys
     float* scores;           // [rows][N]
     uint32_t* hist;          // [rows][4096]
@@ -154,28 +155,50 @@ __device__ __forceinline__ long long nvis_of(int qj, const IdxTcArgs& a) {
     return nv > a.n_ent ? a.n_ent : nv;
 }
 
-// pool row of entry e (< n_ent) of sequence bat, or -1 for a block id outside the pool
-__device__ __forceinline__ long long key_row(const IdxTcArgs& a, int bat, long long e) {
-    if (!a.bt) return (long long)bat * a.n_ent + e;
-    const long long blk = a.bt[(long long)bat * a.bt_stride + e / a.epb];
-    return (blk >= 0 && blk < a.n_blocks) ? blk * a.epb + e % a.epb : -1;
+// pool row of entry e (< n_ent) of sequence bat through the block table, or -1 for a block id outside
+// the pool (pool rows fit in 31 bits on this path)
+__device__ __forceinline__ int paged_row(const IdxTcArgs& a, int bat, int e) {
+    const int blk = a.bt[(long long)bat * a.bt_stride + (e >> a.epb_shift)];
+    return (blk >= 0 && blk < a.n_blocks) ? (blk << a.epb_shift) + (e & (a.epb - 1)) : -1;
 }
 // first pool row of the block holding entries e .. e+epb-1, or -epb (a box the TMA fills with zeros)
 // past the last entry or for a block id outside the pool (reported)
 __device__ __forceinline__ int block_row(const IdxTcArgs& a, int bat, long long e) {
     if (e >= a.n_ent) return -a.epb;
-    const long long blk = a.bt[(long long)bat * a.bt_stride + e / a.epb];
-    if (blk >= 0 && blk < a.n_blocks) return (int)(blk * a.epb);
+    const int blk = a.bt[(long long)bat * a.bt_stride + (int)(e >> a.epb_shift)];
+    if (blk >= 0 && blk < a.n_blocks) return blk << a.epb_shift;
     if (a.err) atomicExch(a.err, (int)V4A_ERR_DEVICE_FAULT);
     return -a.epb;
+}
+
+// the first pool rows of the nb blocks of a tile that starts at entry e0 (paged keys), loaded together so
+// their latencies overlap; the producer fetches them one tile ahead
+template <int kMaxB>
+__device__ __forceinline__ void fetch_block_rows(const IdxTcArgs& a, int bat, long long e0, int nb, int (&rows)[kMaxB]) {
+#pragma unroll
+    for (int j = 0; j < kMaxB; ++j)
+        if (j < nb) rows[j] = block_row(a, bat, e0 + (long long)j * a.epb);
 }
 
 template <bool FP8, int G>
 __device__ void idx_producer(IdxSmem& sm, const IdxTcArgs& a, const CUtensorMap* kmap, long long f0, long long f1) {
     constexpr int kSt = Ring<FP8>::kStages, kBytes = Ring<FP8>::kStageBytes;
+    constexpr int kMaxB = kTileK / kMinEpb;  // blocks per tile at the smallest block
     ICursor cur(f0, a, G);
     const long long n = f1 - f0;
+    const int nb = a.bt ? kTileK / a.epb : 0;
+    int rows[kMaxB], next_rows[kMaxB];
+    if (a.bt && n > 0) fetch_block_rows<kMaxB>(a, cur.bat, (long long)cur.ti * kTileK, nb, next_rows);
     for (long long jt = 0; jt < n; ++jt, cur.next(a)) {
+        if (a.bt) {
+#pragma unroll
+            for (int j = 0; j < kMaxB; ++j) rows[j] = next_rows[j];
+            if (jt + 1 < n) {  // the next tile's block rows, a tile ahead
+                ICursor nx = cur;
+                nx.next(a);
+                fetch_block_rows<kMaxB>(a, nx.bat, (long long)nx.ti * kTileK, nb, next_rows);
+            }
+        }
         if (aborted(sm)) break;
         const int st = (int)(jt % kSt);
         if (jt >= kSt && !tc::mbar_wait(&sm.k_empty[st], (uint32_t)((jt / kSt) - 1) & 1)) { idx_fault(sm, a); break; }
@@ -184,10 +207,11 @@ __device__ void idx_producer(IdxSmem& sm, const IdxTcArgs& a, const CUtensorMap*
         tc::mbar_arrive_expect_tx(&sm.k_full[st], kBytes);
         if (a.bt) {
             // paged keys: one box of epb rows per block of the tile
-            for (int j = 0; j < kTileK / a.epb; ++j) {
-                const int yb = block_row(a, cur.bat, (long long)cur.ti * kTileK + (long long)j * a.epb);
-                tc::tma_load_2d(dst + j * a.epb * 128, kmap, 0, yb, &sm.k_full[st]);
-                if (!FP8) tc::tma_load_2d(dst + kTileK * 128 + j * a.epb * 128, kmap, 64, yb, &sm.k_full[st]);
+#pragma unroll
+            for (int j = 0; j < kMaxB; ++j) {
+                if (j >= nb) break;
+                tc::tma_load_2d(dst + j * a.epb * 128, kmap, 0, rows[j], &sm.k_full[st]);
+                if (!FP8) tc::tma_load_2d(dst + kTileK * 128 + j * a.epb * 128, kmap, 64, rows[j], &sm.k_full[st]);
             }
         } else {
             tc::tma_load_2d(dst, kmap, 0, y, &sm.k_full[st]);
@@ -400,8 +424,10 @@ struct XPrefetch {
     __device__ __forceinline__ void issue(IdxSmem& sm, const IdxTcArgs& a) {
         if (f < f1) {
             const long long e = (long long)cur.ti * kTileK + kHalf * hf + r;
-            const long long kr = e < a.n_ent ? key_row(a, cur.bat, e) : -1;
-            if (kr >= 0) tc::cp_async_4(&sm.xring[(int)((f - f0) % kXSlots)][et], src + kr);
+            if (e < a.n_ent) {
+                const long long kr = a.bt ? (long long)paged_row(a, cur.bat, (int)e) : (long long)cur.bat * a.n_ent + e;
+                if (kr >= 0) tc::cp_async_4(&sm.xring[(int)((f - f0) % kXSlots)][et], src + kr);
+            }
             cur.next(a);
             ++f;
         }
@@ -581,9 +607,22 @@ template <int NP> struct MxAcc {
 static_assert(kMxStages <= kMaxStages, "ring stages");
 
 __device__ void mx_producer(IdxSmem& sm, const IdxTcArgs& a, const CUtensorMap* kmap, long long f0, long long f1) {
+    constexpr int kMaxB = kMxTile / kMinEpb;  // blocks per tile at the smallest block
     ICursor cur(f0, a, 1);
     const long long n = f1 - f0;
+    const int nb = a.bt ? kMxTile / a.epb : 0;
+    int rows[kMaxB], next_rows[kMaxB];
+    if (a.bt && n > 0) fetch_block_rows<kMaxB>(a, cur.bat, (long long)cur.ti * kMxTile, nb, next_rows);
     for (long long jt = 0; jt < n; ++jt, cur.next(a)) {
+        if (a.bt) {
+#pragma unroll
+            for (int j = 0; j < kMaxB; ++j) rows[j] = next_rows[j];
+            if (jt + 1 < n) {  // the next tile's block rows, a tile ahead
+                ICursor nx = cur;
+                nx.next(a);
+                fetch_block_rows<kMaxB>(a, nx.bat, (long long)nx.ti * kMxTile, nb, next_rows);
+            }
+        }
         if (aborted(sm)) break;
         const int st = (int)(jt % kMxStages);
         if (jt >= kMxStages && !tc::mbar_wait(&sm.k_empty[st], (uint32_t)((jt / kMxStages) - 1) & 1)) {
@@ -594,9 +633,10 @@ __device__ void mx_producer(IdxSmem& sm, const IdxTcArgs& a, const CUtensorMap* 
         tc::mbar_arrive_expect_tx(&sm.k_full[st], (uint32_t)kMxStageBytes);
         if (a.bt) {
             // paged keys: one box of epb rows per block of the tile
-            for (int j = 0; j < kMxTile / a.epb; ++j) {
-                const int yb = block_row(a, cur.bat, (long long)cur.ti * kMxTile + (long long)j * a.epb);
-                tc::tma_load_2d(sm.ring + st * kMxStageBytes + j * a.epb * 64, kmap, 0, yb, &sm.k_full[st]);
+#pragma unroll
+            for (int j = 0; j < kMaxB; ++j) {
+                if (j >= nb) break;
+                tc::tma_load_2d(sm.ring + st * kMxStageBytes + j * a.epb * 64, kmap, 0, rows[j], &sm.k_full[st]);
             }
         } else {
             // boxes of 256 rows; rows past the tensor's end are filled with zeros (and still counted)
@@ -718,11 +758,18 @@ __device__ void mx_stage(IdxSmem& sm, const IdxTcArgs& a, uint32_t tmem, long lo
         if (fp < f1) {
             const int xs = (int)((fp - f0) % kMxXSlots);
             const long long e0 = (long long)pre.ti * kMxTile + lane;
+            if (!a.bt) {
+                const uint32_t* sp = src + (long long)pre.bat * a.n_ent + e0;
 #pragma unroll
-            for (int w = 0; w < 16; ++w) {
-                const long long e = e0 + 32 * w;  // word w: quarter w / 4, column w % 4
-                const long long kr = e < a.n_ent ? key_row(a, pre.bat, e) : -1;
-                if (kr >= 0) tc::cp_async_4(&sm.mx_xring[xs][w][ct], src + kr);
+                for (int w = 0; w < 16; ++w)  // word w: quarter w / 4, column w % 4
+                    if (e0 + 32 * w < a.n_ent) tc::cp_async_4(&sm.mx_xring[xs][w][ct], sp + 32 * w);
+            } else {
+#pragma unroll
+                for (int w = 0; w < 16; ++w) {
+                    const long long e = e0 + 32 * w;
+                    const int kr = e < a.n_ent ? paged_row(a, pre.bat, (int)e) : -1;
+                    if (kr >= 0) tc::cp_async_4(&sm.mx_xring[xs][w][ct], src + kr);
+                }
             }
             pre.next(a);
             ++fp;
@@ -912,6 +959,7 @@ cudaError_t launch_index_scores_mx(const IndexArgs& a, float* scores, uint32_t* 
     t.bt = a.bt;
     t.bt_stride = a.bt_stride;
     t.epb = a.epb;
+    t.epb_shift = a.epb > 0 ? __builtin_ctz((unsigned)a.epb) : 0;
     t.n_blocks = a.epb > 0 ? a.pool_rows / a.epb : 0;
     t.scores = scores;
     t.hist = hist;
@@ -943,8 +991,9 @@ cudaError_t launch_index_scores_mx(const IndexArgs& a, float* scores, uint32_t* 
 }  // namespace
 
 bool index_tc_shape_ok(const IndexArgs& a) {
-    // paged keys: blocks of 8 .. 256 entries (a power of two), so a tile is whole blocks
-    const bool paged_ok = !a.bt || (a.epb >= 8 && a.epb <= 256 && (a.epb & (a.epb - 1)) == 0 && a.pool_rows < (1LL << 31));
+    // paged keys: blocks of kMinEpb .. 256 entries (a power of two), so a tile is whole blocks
+    const bool paged_ok =
+        !a.bt || (a.epb >= kMinEpb && a.epb <= 256 && (a.epb & (a.epb - 1)) == 0 && a.pool_rows < (1LL << 31));
     return a.d_i == kDI && a.heads_i <= 32 && a.q_dtype == V4A_BF16 &&
            (a.k_dtype == V4A_BF16 || a.k_dtype == V4A_FP8E4M3 || (a.k_dtype == V4A_MXFP4 && a.kexp)) &&
            a.n_ent >= 1 && (long long)a.batch * a.n_ent < (1LL << 31) && paged_ok;
@@ -974,6 +1023,7 @@ cudaError_t launch_index_scores_tc(const IndexArgs& a, float* scores, uint32_t* 
     t.bt = a.bt;
     t.bt_stride = a.bt_stride;
     t.epb = a.epb;
+    t.epb_shift = a.epb > 0 ? __builtin_ctz((unsigned)a.epb) : 0;
     t.n_blocks = a.epb > 0 ? a.pool_rows / a.epb : 0;
     t.scores = scores;
     t.hist = hist;
