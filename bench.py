@@ -51,6 +51,9 @@ def parse():
     p.add_argument("--cpu-seconds", type=float, default=20.0, help="budget of the oracle sample")
     p.add_argument("--profile-steps", action="store_true",
                    help="run the warm-up and K steps eagerly and exit (the command ncu captures are taken on)")
+    p.add_argument("--profile-fp4", action="store_true",
+                   help="run the MXFP4 indexer (scores and top-k of the 1M-context CSA keys) warm-up + K times "
+                        "eagerly and exit (the command ncu captures of the FP4 kernels are taken on)")
     return p.parse_args()
 
 
@@ -467,11 +470,9 @@ def measure_paged(step: "Step", contiguous_ms: dict) -> dict:
     return res
 
 
-def measure_fp4_indexer(step: "Step", flush: torch.Tensor, peak_gbs: float) -> dict:
-    """The 1M-context CSA indexer with MXFP4 keys (FP4 dot products): the same 4 sequences x
-    262,144 entries x 16 heads x 128, top-1024, with the keys drawn N(0,1) on the device (seeded)
-    and quantised by the library.  The keys (68 B per entry, 71 MB) fit in the 126 MB L2, so every
-    timing flushes L2 first (time_op)."""
+def fp4_inputs(step: "Step"):
+    """MXFP4 keys of the 1M-context CSA workload: N(0,1) drawn on the device (seeded), quantised by the
+    library; plus score / index outputs."""
     v4a, c = step.v4a, step.cc
     B, N, DI = step.Bc, step.Nc, c["d_i"]
     gen = torch.Generator(device="cuda")
@@ -483,6 +484,27 @@ def measure_fp4_indexer(step: "Step", flush: torch.Tensor, peak_gbs: float) -> d
     del master
     scores = torch.empty((B, 1, N), dtype=torch.float32, device="cuda")
     idx = torch.empty((B, 1, c["k"]), dtype=torch.int32, device="cuda")
+    return kc, kx, scores, idx
+
+
+def fp4_profile_run(step: "Step", n: int) -> None:
+    v4a, c = step.v4a, step.cc
+    kc, kx, scores, idx = fp4_inputs(step)
+    for _ in range(n):
+        v4a.v4a_index_scores_mxfp4(step.c_qi, step.c_w, kc, kx, scores, m=c["m"], ctx_len=step.Lc)
+        v4a.v4a_topk_mxfp4(step.c_qi, step.c_w, kc, kx, idx, m=c["m"], k=c["k"], ctx_len=step.Lc,
+                           workspace=step.ws_topk)
+    torch.cuda.synchronize()
+
+
+def measure_fp4_indexer(step: "Step", flush: torch.Tensor, peak_gbs: float) -> dict:
+    """The 1M-context CSA indexer with MXFP4 keys (FP4 dot products): the same 4 sequences x
+    262,144 entries x 16 heads x 128, top-1024, with the keys drawn N(0,1) on the device (seeded)
+    and quantised by the library.  The keys (68 B per entry, 71 MB) fit in the 126 MB L2, so every
+    timing flushes L2 first (time_op)."""
+    v4a, c = step.v4a, step.cc
+    B, N, DI = step.Bc, step.Nc, c["d_i"]
+    kc, kx, scores, idx = fp4_inputs(step)
 
     def scores_fp4():
         v4a.v4a_index_scores_mxfp4(step.c_qi, step.c_w, kc, kx, scores, m=c["m"], ctx_len=step.Lc)
@@ -673,6 +695,9 @@ def main():
     args.warmup = max(3, args.warmup)
     step = Step(seed_offset=rank)
     s = torch.cuda.current_stream()
+    if args.profile_fp4:
+        fp4_profile_run(step, args.warmup + args.steps)
+        return
     if args.profile_steps:
         for _ in range(args.warmup + args.steps):
             step.run()
