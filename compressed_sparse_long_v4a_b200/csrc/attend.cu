@@ -38,6 +38,8 @@ struct SplitPlan {
 template <typename T, int P>
 __global__ void __launch_bounds__(kBlockThreads, 1) attend_split_kernel(AttendArgs a, SplitPlan plan, float* part_ml,
                                                                      float* part_o) {
+    griddep_wait();  // everything before this kernel on the stream has finished
+    griddep_launch_dependents();
     __shared__ __align__(16) float rows_s[kRows * kEpt * P];
     __shared__ int valid_s[kRows];
     __shared__ float lg_s[kBlockThreads * kRows];  // per head-in-block logits of the tile
@@ -218,6 +220,8 @@ __global__ void __launch_bounds__(kBlockThreads, 1) attend_split_kernel(AttendAr
 
 // grid (rows, heads); each thread merges 4 consecutive output elements
 __global__ void attend_combine_kernel(const float* part_ml, const float* part_o, int n_splits, AttendArgs a) {
+    griddep_wait();  // everything before this kernel on the stream has finished
+    griddep_launch_dependents();
     const int row = blockIdx.x, h = blockIdx.y;
     const int heads = a.heads, d = a.d;
     float* out = a.out;
@@ -284,7 +288,8 @@ SplitPlan plan_for(const AttendArgs& a) {
 template <typename T, int P>
 cudaError_t launch_t(const AttendArgs& a, const SplitPlan& plan, float* ml, float* po, cudaStream_t stream) {
     dim3 grid(plan.n_splits, a.batch * a.n_q, plan.head_groups);
-    attend_split_kernel<T, P><<<grid, plan.threads, 0, stream>>>(a, plan, ml, po);
+    cudaError_t le = launch_pdl(attend_split_kernel<T, P>, grid, dim3(plan.threads), 0, stream, a, plan, ml, po);
+    if (le != cudaSuccess) return le;
     return cudaGetLastError();
 }
 
@@ -329,8 +334,9 @@ cudaError_t launch_attend(const AttendArgs& a, void* ws, size_t ws_bytes, cudaSt
     cudaError_t e = a.dtype == V4A_BF16 ? launch_dtype<__nv_bfloat16>(a, plan, ml, po, stream)
                                         : launch_dtype<float>(a, plan, ml, po, stream);
     if (e != cudaSuccess || (plan.n_splits == 1 && a.sink == nullptr && a.rope_dims == 0)) return e;
-    attend_combine_kernel<<<dim3((unsigned)rows, a.heads), a.d / 4 < 128 ? a.d / 4 : 128, 0, stream>>>(
-        ml, po, plan.n_splits, a);
+    e = launch_pdl(attend_combine_kernel, dim3((unsigned)rows, a.heads), dim3(a.d / 4 < 128 ? a.d / 4 : 128), 0,
+                   stream, (const float*)ml, (const float*)po, plan.n_splits, a);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

@@ -593,6 +593,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
+    griddep_wait();  // the prologue above touched only shared and tensor memory
+    griddep_launch_dependents();
     const uint32_t tmem = sm.tmem_base;
 
     if (warp == 0) {
@@ -617,6 +619,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 // (coalesced along heads), weights them by exp2(m_piece - m_max) per head,
 // and writes out[row][h][d0 .. d0 + 31] through a shared-memory transpose.
 __global__ void __launch_bounds__(256) attend_tc_combine(TcArgs a) {
+    griddep_wait();  // everything before this kernel on the stream has finished
+    griddep_launch_dependents();
     constexpr int kDC = 32;  // d per block
     const int row = blockIdx.x, d0 = blockIdx.y * kDC;
     const long long rs = (long long)row * a.tpr, re = rs + a.tpr - 1;
@@ -825,12 +829,12 @@ cudaError_t launch_attend_tc(const AttendArgs& a, void* ws, size_t ws_bytes, cud
     const size_t smem = sizeof(Smem) + 1024;
     cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    attend_tc_kernel<<<p.grid, kThreads, smem, stream>>>(ent_map, tok_map, q_map, t);
-    e = cudaGetLastError();
+    e = launch_pdl(attend_tc_kernel, dim3(p.grid), dim3(kThreads), smem, stream, ent_map, tok_map, q_map, t);
+    if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     if (p.grid > 1) {
-        attend_tc_combine<<<dim3(t.rows, kD / 32), 256, 0, stream>>>(t);
-        e = cudaGetLastError();
+        e = launch_pdl(attend_tc_combine, dim3(t.rows, kD / 32), dim3(256), 0, stream, t);
+        if (e == cudaSuccess) e = cudaGetLastError();
     }
     return e;
 }

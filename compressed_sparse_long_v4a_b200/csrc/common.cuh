@@ -177,6 +177,15 @@ __device__ __forceinline__ float group_sum(float v) {
 
 __host__ __device__ __forceinline__ long long n_visible(long long t, int m) { return (t + 1) / m; }
 
+// Programmatic dependent launch.  Every kernel of the library is launched with launch_pdl(), so it may
+// be scheduled while the kernel before it on the stream is still finishing; griddep_wait() then
+// blocks until that kernel has completed and its memory is visible (a no-op when there is no such
+// dependency), so every thread calls it before its first global memory access (reads and writes);
+// griddep_launch_dependents() lets the next kernel's blocks be scheduled once every block of this
+// grid has called it, so they can set up (shared memory, barriers, tensor memory) meanwhile.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // Output RoPE at minus the query position ("1M Context != Lossless Long Memory", section 8): the
 // pair k of the last R dims of a d-dim row turns by -t * base^(-2k/R).  sin/cos of that angle,
 // reduced and evaluated in double (t reaches 1M, the angle hundreds of thousands of radians).

@@ -93,6 +93,8 @@ __device__ __forceinline__ void compress_span(const StreamDesc& d, const T* xp, 
 
 __global__ void __launch_bounds__(256) compress_kernel(StreamDesc s0, StreamDesc s1, int batch, long long n_ent,
                                                        int m) {
+    griddep_wait();  // everything before this kernel on the stream has finished
+    griddep_launch_dependents();
     const StreamDesc& d = blockIdx.y == 0 ? s0 : s1;
     const long long per_entry = (long long)d.groups * d.split;
     long long total = (long long)batch * n_ent * per_entry;
@@ -222,6 +224,8 @@ bool quantised(int dt) { return dt == V4A_FP8E4M3 || dt == V4A_MXFP4; }
 template <typename T>
 __global__ void __launch_bounds__(256) quantize_mxfp4_kernel(const T* x, long long rows, int cols, uint8_t* codes,
                                                              uint8_t* exps) {
+    griddep_wait();  // everything before this kernel on the stream has finished
+    griddep_launch_dependents();
     const int groups = cols / 8;
     const long long g = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     const bool active = g < rows * groups;
@@ -275,6 +279,8 @@ struct RingArgs {
 };
 
 __global__ void __launch_bounds__(256) ring_append_kernel(RingArgs r) {
+    griddep_wait();  // everything before this kernel on the stream has finished
+    griddep_launch_dependents();
     int g = blockIdx.x * blockDim.x + threadIdx.x;
     for (int i = 0; i < r.n; ++i) {
         const int per = r.batch * r.chunks[i];
@@ -312,8 +318,8 @@ cudaError_t launch_compress(const v4a_compress_io* kv, const v4a_compress_io* id
     long long total = (long long)batch * n_ent * (w0 > w1 ? w0 : w1);
     const int threads = 256;
     dim3 grid((unsigned)((total + threads - 1) / threads), idx ? 2 : 1);
-    compress_kernel<<<grid, threads, 0, stream>>>(s0, s1, batch, n_ent, m);
-    return cudaGetLastError();
+    const cudaError_t e = launch_pdl(compress_kernel, grid, dim3(threads), 0, stream, s0, s1, batch, n_ent, m);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_quantize_mxfp4(const void* x, v4a_dtype dt, long long rows, int cols, uint8_t* codes,
@@ -322,12 +328,12 @@ cudaError_t launch_quantize_mxfp4(const void* x, v4a_dtype dt, long long rows, i
     if (total == 0) return cudaSuccess;
     const int threads = 256;
     const unsigned blocks = (unsigned)((total + threads - 1) / threads);
-    if (dt == V4A_BF16)
-        quantize_mxfp4_kernel<<<blocks, threads, 0, stream>>>(static_cast<const __nv_bfloat16*>(x), rows, cols,
-                                                              codes, exps);
-    else
-        quantize_mxfp4_kernel<<<blocks, threads, 0, stream>>>(static_cast<const float*>(x), rows, cols, codes, exps);
-    return cudaGetLastError();
+    const cudaError_t e =
+        dt == V4A_BF16 ? launch_pdl(quantize_mxfp4_kernel<__nv_bfloat16>, dim3(blocks), dim3(threads), 0, stream,
+                                    static_cast<const __nv_bfloat16*>(x), rows, cols, codes, exps)
+                       : launch_pdl(quantize_mxfp4_kernel<float>, dim3(blocks), dim3(threads), 0, stream,
+                                    static_cast<const float*>(x), rows, cols, codes, exps);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_compress_paged(const v4a_compress_io* kv, const v4a_compress_io* idx, int batch, long long n_tok,
@@ -352,8 +358,8 @@ cudaError_t launch_compress_paged(const v4a_compress_io* kv, const v4a_compress_
     long long total = (long long)batch * n_ent * (w0 > w1 ? w0 : w1);
     const int threads = 256;
     dim3 grid((unsigned)((total + threads - 1) / threads), idx ? 2 : 1);
-    compress_kernel<<<grid, threads, 0, stream>>>(s0, s1, batch, n_ent, m);
-    return cudaGetLastError();
+    const cudaError_t e = launch_pdl(compress_kernel, grid, dim3(threads), 0, stream, s0, s1, batch, n_ent, m);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_ring_append(const v4a_ring_io* io, int n, int batch, long long pos, cudaStream_t stream) {
@@ -370,8 +376,9 @@ cudaError_t launch_ring_append(const v4a_ring_io* io, int n, int batch, long lon
         total += (long long)batch * r.chunks[i];
     }
     const int threads = 256;
-    ring_append_kernel<<<(unsigned)((total + threads - 1) / threads), threads, 0, stream>>>(r);
-    return cudaGetLastError();
+    const cudaError_t e =
+        launch_pdl(ring_append_kernel, dim3((unsigned)((total + threads - 1) / threads)), dim3(threads), 0, stream, r);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_compress_dual(const v4a_compress_io* a, const v4a_series_b* b, int batch, long long n_tok, int m,
@@ -392,8 +399,8 @@ cudaError_t launch_compress_dual(const v4a_compress_io* a, const v4a_series_b* b
     const long long total = (long long)batch * n_ent * s0.groups * s0.split;
     const int threads = 256;
     dim3 grid((unsigned)((total + threads - 1) / threads), 1);
-    compress_kernel<<<grid, threads, 0, stream>>>(s0, s0, batch, n_ent, m);
-    return cudaGetLastError();
+    const cudaError_t e = launch_pdl(compress_kernel, grid, dim3(threads), 0, stream, s0, s0, batch, n_ent, m);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace v4a

@@ -45,6 +45,8 @@ __device__ __forceinline__ void load_key8(const IndexArgs& a, long long off, flo
 // grid: (ceil(N / 256), B * n_q); q of the block's query staged in shared memory
 template <int HMAX, int KFMT>
 __global__ void __launch_bounds__(kScoreThreads) index_score_kernel(IndexArgs a, float* scores) {
+    griddep_wait();  // everything before this kernel on the stream has finished
+    griddep_launch_dependents();
     extern __shared__ float smem[];
     float* q_s = smem;                         // [HI][DI]
     float* w_s = smem + a.heads_i * a.d_i;     // [HI]
@@ -613,6 +615,8 @@ __global__ void __launch_bounds__(kFastThreads) topk_fast_kernel(const float* sc
                                                                  int32_t* cidx_buf, uint32_t* ckey_buf, int* counts,
                                                                  unsigned int* row_done, int32_t* idx_out,
                                                                  float* score_out) {
+    griddep_wait();  // everything before this kernel on the stream has finished
+    griddep_launch_dependents();
     extern __shared__ __align__(16) uint8_t dsm[];
     __shared__ int warp_buf[33];
     __shared__ int s_last;
@@ -680,6 +684,8 @@ __global__ void __launch_bounds__(kFastThreads) topk_fast_kernel(const float* sc
 // more than kCandCap candidates falls back to the exact radix select over the row.
 __global__ void __launch_bounds__(kFastThreads) topk_rows_kernel(const float* scores, IndexArgs a, int k,
                                                                  int32_t* idx_out, float* score_out) {
+    griddep_wait();  // everything before this kernel on the stream has finished
+    griddep_launch_dependents();
     extern __shared__ __align__(16) uint8_t dsm[];
     uint32_t* ckey = reinterpret_cast<uint32_t*>(dsm);           // [kCandCap]
     int32_t* cidx = reinterpret_cast<int32_t*>(ckey + kCandCap);  // [kCandCap]
@@ -773,25 +779,29 @@ cudaError_t launch_scores_h(const IndexArgs& a, float* scores, cudaStream_t stre
     case V4A_F32: {
         auto kern = index_score_kernel<HMAX, V4A_F32>;
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        kern<<<grid, kScoreThreads, smem, stream>>>(a, scores);
+        const cudaError_t le = launch_pdl(kern, grid, dim3(kScoreThreads), smem, stream, a, scores);
+        if (le != cudaSuccess) return le;
         break;
     }
     case V4A_BF16: {
         auto kern = index_score_kernel<HMAX, V4A_BF16>;
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        kern<<<grid, kScoreThreads, smem, stream>>>(a, scores);
+        const cudaError_t le = launch_pdl(kern, grid, dim3(kScoreThreads), smem, stream, a, scores);
+        if (le != cudaSuccess) return le;
         break;
     }
     case V4A_MXFP4: {
         auto kern = index_score_kernel<HMAX, V4A_MXFP4>;
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        kern<<<grid, kScoreThreads, smem, stream>>>(a, scores);
+        const cudaError_t le = launch_pdl(kern, grid, dim3(kScoreThreads), smem, stream, a, scores);
+        if (le != cudaSuccess) return le;
         break;
     }
     default: {
         auto kern = index_score_kernel<HMAX, V4A_FP8E4M3>;
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        kern<<<grid, kScoreThreads, smem, stream>>>(a, scores);
+        const cudaError_t le = launch_pdl(kern, grid, dim3(kScoreThreads), smem, stream, a, scores);
+        if (le != cudaSuccess) return le;
         break;
     }
     }
@@ -842,6 +852,8 @@ static TopkPlan topk_plan(const IndexArgs& a) {
 
 // histogram of the order-preserving keys' top 12 bits, for the CUDA-core score path
 __global__ void score_hist_kernel(const float* scores, IndexArgs a, uint32_t* hist) {
+    griddep_wait();  // everything before this kernel on the stream has finished
+    griddep_launch_dependents();
     const int row = blockIdx.y;
     const long long nvis = row_nvis(a, row);
     for (long long s = (long long)blockIdx.x * blockDim.x + threadIdx.x; s < nvis; s += (long long)gridDim.x * blockDim.x)
@@ -881,8 +893,9 @@ cudaError_t launch_topk(const IndexArgs& a, int k, int32_t* idx_out, float* scor
         }
         e = cudaFuncSetAttribute(topk_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFastSmem);
         if (e != cudaSuccess) return e;
-        topk_rows_kernel<<<rows, kFastThreads, kFastSmem, stream>>>(scores, a, k, idx_out, score_out);
-        return cudaGetLastError();
+        e = launch_pdl(topk_rows_kernel, dim3(rows), dim3(kFastThreads), kFastSmem, stream, (const float*)scores, a, k,
+                       idx_out, score_out);
+        return e != cudaSuccess ? e : cudaGetLastError();
     }
     uint32_t* hist = reinterpret_cast<uint32_t*>(base + p.off_hist);
     int* counts = reinterpret_cast<int*>(base + p.off_cnt);
@@ -897,16 +910,17 @@ cudaError_t launch_topk(const IndexArgs& a, int k, int32_t* idx_out, float* scor
     } else {
         e = launch_index_scores(a, scores, stream);
         if (e == cudaSuccess) {
-            score_hist_kernel<<<dim3(64, rows), 256, 0, stream>>>(scores, a, hist);
-            e = cudaGetLastError();
+            e = launch_pdl(score_hist_kernel, dim3(64, rows), dim3(256), 0, stream, (const float*)scores, a, hist);
+            if (e == cudaSuccess) e = cudaGetLastError();
         }
     }
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(topk_fast_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFastSmem);
     if (e != cudaSuccess) return e;
-    topk_fast_kernel<<<rows * p.parts, kFastThreads, kFastSmem, stream>>>(scores, hist, a, k, p.parts, p.chunk, def_buf,
-                                                                          cidx, ckey, counts, row_done, idx_out,
-                                                                          score_out);
+    e = launch_pdl(topk_fast_kernel, dim3(rows * p.parts), dim3(kFastThreads), kFastSmem, stream, (const float*)scores,
+                   (const uint32_t*)hist, a, k, p.parts, p.chunk, def_buf, cidx, ckey, counts, row_done, idx_out,
+                   score_out);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

@@ -555,6 +555,8 @@ __global__ void __launch_bounds__(kThreads, 1) index_score_tc_kernel(const __gri
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
+    griddep_wait();  // the prologue above touched only shared and tensor memory
+    griddep_launch_dependents();
     const uint32_t tmem = sm.tmem_base;
     if (warp == 0) {
         if (lane == 0) idx_producer<FP8, G>(sm, a, &kmap, f0, f1);
@@ -908,6 +910,8 @@ __global__ void __launch_bounds__(kThreads, 1) index_score_mx_kernel(const __gri
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
+    griddep_wait();  // the prologue above touched only shared and tensor memory
+    griddep_launch_dependents();
     const uint32_t tmem = sm.tmem_base;
     if (warp == 0) {
         if (lane == 0) mx_producer(sm, a, &kmap, f0, f1);
@@ -980,7 +984,7 @@ cudaError_t launch_index_scores_mx(const IndexArgs& a, float* scores, uint32_t* 
     const size_t smem = sizeof(IdxSmem) + 1024;
     auto go = [&](auto kernel) {
         cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e == cudaSuccess) kernel<<<t.grid, kThreads, smem, stream>>>(kmap, t);
+        if (e == cudaSuccess) e = launch_pdl(kernel, dim3(t.grid), dim3(kThreads), smem, stream, kmap, t);
         return e;
     };
     cudaError_t e = a.heads_i <= 16 ? go(index_score_mx_kernel<16>) : go(index_score_mx_kernel<32>);
@@ -1049,7 +1053,7 @@ cudaError_t launch_index_scores_tc(const IndexArgs& a, float* scores, uint32_t* 
     const size_t smem = sizeof(IdxSmem) + 1024;
     auto go = [&](auto kernel) {
         cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (err == cudaSuccess) kernel<<<t.grid, kThreads, smem, stream>>>(kmap, t);
+        if (err == cudaSuccess) err = launch_pdl(kernel, dim3(t.grid), dim3(kThreads), smem, stream, kmap, t);
         return err;
     };
     cudaError_t e;
