@@ -88,6 +88,7 @@ struct TcArgs {
     int bt_stride, epb;
     long long n_blocks;
     int ring_rows;      // > 0: window rows come from a ring [B][ring_rows][512] (position p in row p % ring_rows)
+    int comb_pieces;    // bound on the pieces of one query (attend_tc_combine's shared memory)
 };
 
 // tiles whose rows the producer gathers with cp.async (CSA selections, paged entries, ring windows)
@@ -614,14 +615,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // Merge the partials of queries whose tiles were split between CTAs.
-// grid (rows, 512 / 32 d chunks), 256 threads.  Pieces are stored d-major
-// ([d][64 heads]); each block reads its 32 d x 64 heads of every piece
-// (coalesced along heads), weights them by exp2(m_piece - m_max) per head,
-// and writes out[row][h][d0 .. d0 + 31] through a shared-memory transpose.
+// grid (rows, 512 / 16 d chunks), 256 threads, a.comb_pieces * 64 floats of dynamic shared memory
+// (at least the pieces of any query).  Pieces are stored d-major ([d][64 heads]), so a block's
+// 16 d x 64 heads of one piece are 4 KB in one run: each thread loads 16 bytes of it (one d, four
+// heads) for up to 8 pieces before using any of them.  The per-head weights exp2(m_piece - m_max)
+// come first, from four groups of 64 threads each taking every fourth piece; the weighted sum is
+// scaled by 1 / l at the end and written to out[row][h][d0 .. d0 + 15] through a shared-memory
+// transpose.
 __global__ void __launch_bounds__(256) attend_tc_combine(TcArgs a) {
     griddep_wait();  // everything before this kernel on the stream has finished
     griddep_launch_dependents();
-    constexpr int kDC = 32;  // d per block
+    constexpr int kDC = 16;  // d per block
+    constexpr int kU = 8;    // pieces whose loads are in flight together
     const int row = blockIdx.x, d0 = blockIdx.y * kDC;
     const long long rs = (long long)row * a.tpr, re = rs + a.tpr - 1;
     // CTA holding flat tile f: the largest c with range_start(c) <= f
@@ -631,83 +636,94 @@ __global__ void __launch_bounds__(256) attend_tc_combine(TcArgs a) {
     // the first CTA's piece is its first query only if the query starts its range; every later CTA's
     // range starts inside this query, so the piece is that CTA's first (slot 2c)
     const int n = c1 - c0 + 1;
-    constexpr int kMaxPieces = kNumSMs;  // a query split over every CTA (grid <= 148)
-    __shared__ float s_w[kMaxPieces][kH];  // weight of piece i for head h, divided by the head's total
-    __shared__ int s_slot[kMaxPieces];
+    if (n > a.comb_pieces) {  // the host's bound on pieces per query does not hold
+        if (threadIdx.x == 0 && a.dev_status) atomicExch(a.dev_status, (int)V4A_ERR_DEVICE_FAULT);
+        return;
+    }
+    extern __shared__ __align__(16) float s_w[];  // [n][64]: weight of piece i for head h
+    __shared__ int s_slot[kNumSMs + kU];
+    __shared__ float s_red[4][kH];
+    __shared__ __align__(16) float s_inv[kH];
     __shared__ float s_acc[kH][kDC + 1];
-    const int t = threadIdx.x;
+    const int t = threadIdx.x, g = t >> 6, h = t & (kH - 1);
     for (int i = t; i < n; i += blockDim.x)
         s_slot[i] = 2 * (c0 + i) + ((i == 0 && range_start(c0, a) < rs) ? 1 : 0);
     __syncthreads();
+    // per head: the largest piece max, then the weights and the total l; NaN anywhere poisons the head
+    const float2* ml = reinterpret_cast<const float2*>(a.part_ml);  // [slot][64] of (m, l)
+    bool bad = false;
+    float mg = -INFINITY;
+#pragma unroll 4
+    for (int i = g; i < n; i += 4) {
+        const float m = ml[(long long)s_slot[i] * kH + h].x;
+        bad |= isnan(m);
+        mg = fmaxf(mg, m);
+    }
+    s_red[g][h] = bad ? NAN : mg;
+    __syncthreads();
+    float mmax = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const float x = s_red[j][h];
+        bad |= isnan(x);
+        mmax = fmaxf(mmax, x);
+    }
+    float lg = 0.f;
+#pragma unroll 4
+    for (int i = g; i < n; i += 4) {
+        const float2 p = ml[(long long)s_slot[i] * kH + h];
+        bad |= isnan(p.y);
+        const float wgt = (p.x != -INFINITY && mmax != -INFINITY) ? exp2f(p.x - mmax) : 0.f;
+        s_w[i * kH + h] = wgt;
+        lg += wgt * p.y;
+    }
+    __syncthreads();  // every group has read s_red
+    s_red[g][h] = bad ? NAN : lg;
+    __syncthreads();
     if (t < kH) {
-        const int h = t;
-        float mmax = -INFINITY;
-        bool bad = false;
-#pragma unroll 4
-        for (int i = 0; i < n; ++i) {
-            const float m = a.part_ml[((long long)s_slot[i] * kH + h) * 2];
-            bad |= isnan(m);
-            mmax = fmaxf(mmax, m);
-        }
-        float l = 0.f;
-#pragma unroll 4
-        for (int i = 0; i < n; ++i) {
-            const float m = a.part_ml[((long long)s_slot[i] * kH + h) * 2];
-            const float li = a.part_ml[((long long)s_slot[i] * kH + h) * 2 + 1];
-            bad |= isnan(li);
-            const float wgt = (m != -INFINITY && mmax != -INFINITY) ? exp2f(m - mmax) : 0.f;
-            s_w[i][h] = wgt;
-            l += wgt * li;
-        }
+        float l = (s_red[0][h] + s_red[1][h]) + (s_red[2][h] + s_red[3][h]);
         if (a.sink && mmax != -INFINITY) l += exp2f(a.sink[h] * 1.4426950408889634f - mmax);  // the sink's share
-        const float inv = bad ? NAN : (l > 0.f ? 1.f / l : 0.f);
-        for (int i = 0; i < n; ++i) s_w[i][h] *= inv;
-        if (bad || !(l > 0.f)) s_w[0][h] = bad ? NAN : 0.f;  // NaN poisons, an empty row stays zero
+        s_inv[h] = isnan(l) ? NAN : (l > 0.f ? 1.f / l : 0.f);  // an empty row stays zero
     }
-    __syncthreads();
-    // thread t: head h = t % 64, d rows dq, dq + 4, ... (8 of the 32); the loads of 4 pieces are
-    // issued before any of them is used (a piece of weight 0 holds finite values: it adds 0)
-    const int h = t & (kH - 1), dq = t >> 6;
-    float acc[kDC / 4];
+    // thread t: d row dr = t / 16 of the chunk, heads hq .. hq + 3 (a piece of weight 0 holds finite
+    // values: it adds 0)
+    const int dr = t >> 4, hq = (t & 15) * 4;
+    const float* src = a.part_o + (long long)(d0 + dr) * kH + hq;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int i0 = 0; i0 < n; i0 += kU) {
+        float4 v[kU];
 #pragma unroll
-    for (int j = 0; j < kDC / 4; ++j) acc[j] = 0.f;
-    constexpr int kU = 4;
-    int i0 = 0;
-    for (; i0 + kU <= n; i0 += kU) {
-        float v[kU][kDC / 4];
+        for (int u = 0; u < kU; ++u)
+            v[u] = i0 + u < n ? __ldcg(reinterpret_cast<const float4*>(src + (long long)s_slot[i0 + u] * kH * kD))
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
         for (int u = 0; u < kU; ++u) {
-            const float* pp = a.part_o + (long long)s_slot[i0 + u] * kH * kD + (long long)d0 * kH + h;
-#pragma unroll
-            for (int j = 0; j < kDC / 4; ++j) v[u][j] = pp[(long long)(dq + 4 * j) * kH];
-        }
-#pragma unroll
-        for (int u = 0; u < kU; ++u) {
-            const float wgt = s_w[i0 + u][h];
-#pragma unroll
-            for (int j = 0; j < kDC / 4; ++j) acc[j] = fmaf(wgt, v[u][j], acc[j]);
+            if (i0 + u >= n) break;
+            const float4 w = *reinterpret_cast<const float4*>(s_w + (i0 + u) * kH + hq);
+            acc.x = fmaf(w.x, v[u].x, acc.x);
+            acc.y = fmaf(w.y, v[u].y, acc.y);
+            acc.z = fmaf(w.z, v[u].z, acc.z);
+            acc.w = fmaf(w.w, v[u].w, acc.w);
         }
     }
-    for (; i0 < n; ++i0) {
-        const float wgt = s_w[i0][h];
-        const float* pp = a.part_o + (long long)s_slot[i0] * kH * kD + (long long)d0 * kH + h;
-#pragma unroll
-        for (int j = 0; j < kDC / 4; ++j) acc[j] = fmaf(wgt, pp[(long long)(dq + 4 * j) * kH], acc[j]);
+    __syncthreads();  // s_inv is written
+    {
+        const float4 inv = *reinterpret_cast<const float4*>(s_inv + hq);  // NaN for a poisoned head
+        s_acc[hq][dr] = acc.x * inv.x;
+        s_acc[hq + 1][dr] = acc.y * inv.y;
+        s_acc[hq + 2][dr] = acc.z * inv.z;
+        s_acc[hq + 3][dr] = acc.w * inv.w;
     }
-    // a poisoned head makes its whole output NaN
-    const float w0 = s_w[0][h];
-#pragma unroll
-    for (int j = 0; j < kDC / 4; ++j) s_acc[h][dq + 4 * j] = isnan(w0) ? NAN : acc[j];
     __syncthreads();
-    // write out[row][h][d0 .. d0+31]: warp w covers heads w, w+8, ...; lane = d (output RoPE: the pair
-    // partner of d is d ^ 1, in the same 32)
-    const int lane = t & 31, w = t >> 5, d = d0 + lane;
+    // write out[row][h][d0 .. d0+15]: thread t takes d = d0 + t % 16 of heads t / 16, t / 16 + 16, ...
+    // (output RoPE: the pair partner of d is d ^ 1, in the same 16)
+    const int lane = t & (kDC - 1), hg = t >> 4, d = d0 + lane;
     const bool rot = a.rope_dims > 0 && d >= kD - a.rope_dims;
     float rs_ = 0.f, rc_ = 1.f;
     if (rot)
         rope_sincos(a.ctx_len - a.n_q + (row % a.n_q), (d - (kD - a.rope_dims)) >> 1, a.rope_dims, a.rope_base, &rs_,
                     &rc_);
-    for (int hh = w; hh < kH; hh += 8) {
+    for (int hh = hg; hh < kH; hh += 256 / kDC) {
         float v = s_acc[hh][lane];
         if (rot) v = rope_apply(d, v, s_acc[hh][lane ^ 1], rs_, rc_);
         a.out[((long long)row * kH + hh) * kD + d] = v;
@@ -825,6 +841,13 @@ cudaError_t launch_attend_tc(const AttendArgs& a, void* ws, size_t ws_bytes, cud
     t.epb = a.epb;
     t.n_blocks = a.epb > 0 ? a.pool_rows / a.epb : 0;
     t.ring_rows = a.ring_rows;
+    {
+        // CTA c covers flat tiles [c T / G, (c+1) T / G), at least floor(T / G) of them, so a query's tpr
+        // tiles meet at most ceil(tpr / floor(T / G)) + 1 CTAs
+        const long long per = p.total / p.grid;
+        const long long bound = (p.tpr + per - 1) / per + 1;
+        t.comb_pieces = (int)(bound < p.grid ? bound : p.grid);
+    }
 
     const size_t smem = sizeof(Smem) + 1024;
     cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -833,7 +856,8 @@ cudaError_t launch_attend_tc(const AttendArgs& a, void* ws, size_t ws_bytes, cud
     if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     if (p.grid > 1) {
-        e = launch_pdl(attend_tc_combine, dim3(t.rows, kD / 32), dim3(256), 0, stream, t);
+        e = launch_pdl(attend_tc_combine, dim3(t.rows, kD / 16), dim3(256), (size_t)t.comb_pieces * kH * sizeof(float),
+                       stream, t);
         if (e == cudaSuccess) e = cudaGetLastError();
     }
     return e;
