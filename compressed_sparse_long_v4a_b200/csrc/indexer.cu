@@ -903,7 +903,7 @@ cudaError_t launch_topk(const IndexArgs& a, int k, int32_t* idx_out, float* scor
     int32_t* cidx = reinterpret_cast<int32_t*>(base + p.off_cidx);
     uint32_t* ckey = reinterpret_cast<uint32_t*>(base + p.off_ckey);
     unsigned int* row_done = hist + (size_t)rows * kHistBins;
-    e = cudaMemsetAsync(hist, 0, (size_t)rows * (kHistBins + 1) * sizeof(uint32_t), stream);
+    e = launch_zero_words(hist, (long long)rows * (kHistBins + 1), stream);
     if (e != cudaSuccess) return e;
     if (index_tc_available(a)) {
         e = launch_index_scores_tc(a, scores, hist, a.dev_status, stream);

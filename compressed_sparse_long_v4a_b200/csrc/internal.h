@@ -29,6 +29,11 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
 // Record a one-line reason for v4a_last_error() and return st.
 v4a_status report(v4a_status st, const char* fmt, ...);
 
+// ---- v4a_api.cu -------------------------------------------------------
+// Zero n 32-bit words with a kernel launched like every other kernel here, after the previous
+// work on the stream (a memset node in its place would end the chain of overlapped launches).
+cudaError_t launch_zero_words(uint32_t* p, long long n, cudaStream_t stream);
+
 // ---- compress.cu ------------------------------------------------------
 cudaError_t launch_compress(const v4a_compress_io* kv, const v4a_compress_io* idx, int batch, long long n_tok,
                             int m, cudaStream_t stream);
