@@ -25,7 +25,7 @@
 // a query cut between CTAs gets one partial (m, l, O) per piece, merged by
 // attend_tc_combine.  Per CTA: warp 0 loads (TMA for contiguous rows and the
 // query, cp.async gathers for CSA-selected rows) into a 2-stage ring, warp 1
-// issues the MMAs, warps 2-5 run the softmax and the output.  Every wait is
+// (all lanes; one elected lane) issues the MMAs, warps 2-5 run the softmax and the output.  Every wait is
 // bounded; on a time-out the CTA records a device fault, poisons its outputs
 // with NaN and winds down.
 #include <cudaTypedefs.h>
@@ -346,10 +346,11 @@ __device__ void issue_qk(Smem& sm, uint32_t tmem, int jq, bool gathered, uint64_
 // No CTA-wide progress for this many cycles (about a second) counts as a fault.
 constexpr long long kStallCycles = 1LL << 31;
 
-// The two MMA groups of every tile are issued in whatever order their inputs
-// become ready: PV(j) as soon as the softmax has written P(j) (which frees
-// tile j's stage for the next load early), QK(j) as soon as tile j has
-// landed and S buffer j&1 is free (PV(j-2) issued).
+// Warp 1, all 32 lanes (one elected lane issues each MMA and commit; every decision below is taken
+// on lane 0's view, so the warp stays converged).  The two MMA groups of every tile are issued in
+// whatever order their inputs become ready: PV(j) as soon as the softmax has written P(j) (which frees
+// tile j's stage for the next load early), QK(j) as soon as tile j has landed and S buffer j&1 is free
+// (PV(j-2) issued).
 __device__ void mma_issuer(Smem& sm, const TcArgs& a, uint32_t tmem, long long f0, long long f1) {
     const long long n = f1 - f0;
     const uint64_t q0 = tc::sw128_desc(tc::smem_u32(sm.q), 16, 1024);
@@ -359,17 +360,17 @@ __device__ void mma_issuer(Smem& sm, const TcArgs& a, uint32_t tmem, long long f
     Cursor cq(f0, a.tpr), cp(f0, a.tpr);
     long long t_last = clock64();
     while (jp < n) {
-        if (*reinterpret_cast<volatile int*>(&sm.abort_flag)) { ok = false; break; }
+        if (__shfl_sync(0xffffffffu, *reinterpret_cast<volatile int*>(&sm.abort_flag), 0)) { ok = false; break; }
         bool progressed = false;
-        if (jp < jq && tc::mbar_test(&sm.p_full[jp & 1], (uint32_t)(jp >> 1) & 1)) {
+        if (jp < jq && tc::mbar_test_warp(&sm.p_full[jp & 1], (uint32_t)(jp >> 1) & 1)) {
             issue_pv(sm, tmem, (int)jp, jp == 0 || cp.ti == 0);
             ++jp;
             cp.next(a.tpr);
             progressed = true;
         } else if (jq < n && jp >= jq - 1) {
             const bool qseg = jq == 0 || cq.ti == 0;
-            if (tc::mbar_test(&sm.kv_full[jq % kStages], (uint32_t)(jq / kStages) & 1) &&
-                (!qseg || tc::mbar_test(&sm.q_full, segq & 1))) {
+            if (tc::mbar_test_warp(&sm.kv_full[jq % kStages], (uint32_t)(jq / kStages) & 1) &&
+                (!qseg || tc::mbar_test_warp(&sm.q_full, segq & 1))) {
                 issue_qk(sm, tmem, (int)jq, tile_gathered(a, cq.ti), q0);
                 if (jq == n - 1 || cq.ti == a.tpr - 1) tc::mma_commit(&sm.q_empty);  // last QK of this query
                 if (qseg) ++segq;
@@ -380,7 +381,7 @@ __device__ void mma_issuer(Smem& sm, const TcArgs& a, uint32_t tmem, long long f
         }
         if (progressed) {
             t_last = clock64();
-        } else if (clock64() - t_last > kStallCycles) {
+        } else if (__shfl_sync(0xffffffffu, (int)(clock64() - t_last > kStallCycles), 0)) {
             ok = false;
             break;
         }
@@ -603,8 +604,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0) {
         producer(sm, a, &ent_map, &tok_map, &q_map, f0, f1);
     } else if (warp == 1) {
-        if ((threadIdx.x & 31) == 0) mma_issuer(sm, a, tmem, f0, f1);
-        __syncwarp();
+        mma_issuer(sm, a, tmem, f0, f1);
     } else {
         softmax_warps(sm, a, tmem, f0, f1, cta);
     }

@@ -29,7 +29,7 @@
 //  * MXFP4 keys (and the query quantised to MXFP4 per head): see the section
 //    "MXFP4 keys and queries" below.
 // Warp 0 loads key tiles into a shared-memory ring (4 x 32 KB for FP8, 2 x 64
-// KB for bf16), warp 1 issues the MMAs, warps 2-5 stage each row's B
+// KB for bf16), warp 1 (all lanes, one elected lane issuing) issues the MMAs, warps 2-5 stage each row's B
 // operand, warps 6-13 run the epilogue: two warps per TMEM sub-partition, one
 // per half of the tile, so each scheduler has two to switch between while one
 // waits on tensor memory.  Per-entry scales are fetched 8 tiles ahead (HBM
@@ -234,17 +234,17 @@ __device__ void idx_mma(IdxSmem& sm, const IdxTcArgs& a, uint32_t tmem, long lon
     uint64_t qd = 0;
     ICursor cur(f0, a, G);
     for (long long f = f0; f < f1; ++f, cur.next(a)) {
-        if (aborted(sm)) { ok = false; break; }
+        if (warp_aborted(sm)) { ok = false; break; }
         const int jt = (int)(f - f0), st = jt % kSt, sd = jt % kDS;
         if (f == f0 || cur.ti == 0) {
             b = seg & 1;
-            if (!tc::mbar_wait(&sm.q_full[b], (seg >> 1) & 1)) { ok = false; break; }
+            if (!warp_wait(&sm.q_full[b], (seg >> 1) & 1)) { ok = false; break; }
             qd = tc::sw128_desc(tc::smem_u32(sm.q[b]), 16, 1024);
             ++seg;
         }
         const bool seg_end = (f == f1 - 1) || (cur.ti == a.tiles_per_row - 1);
-        if (!tc::mbar_wait(&sm.k_full[st], (jt / kSt) & 1)) { ok = false; break; }
-        if (jt >= kDS && !tc::mbar_wait(&sm.d_free[sd], ((jt / kDS) - 1) & 1)) { ok = false; break; }
+        if (!warp_wait(&sm.k_full[st], (jt / kSt) & 1)) { ok = false; break; }
+        if (jt >= kDS && !warp_wait(&sm.d_free[sd], ((jt / kDS) - 1) & 1)) { ok = false; break; }
         tc::tc_fence_after();
         const uint32_t stage = tc::smem_u32(sm.ring + st * kBytes);
 #pragma unroll
@@ -256,12 +256,8 @@ __device__ void idx_mma(IdxSmem& sm, const IdxTcArgs& a, uint32_t tmem, long lon
                 // K = 32 e4m3 per MMA: 32 bytes along the 128-byte rows of both operands
 #pragma unroll
                 for (int kk = 0; kk < kDI / 32; ++kk)
-                    asm volatile(
-                        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-                        " tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n}\n" ::"r"(d),
-                        "l"(kd + (uint64_t)((kk * 32) >> 4)), "l"(qd + (uint64_t)((kk * 32) >> 4)), "r"(idesc),
-                        "r"(kk ? 1u : 0u)
-                        : "memory");
+                    tc::mma_f8f6f4(d, kd + (uint64_t)((kk * 32) >> 4), qd + (uint64_t)((kk * 32) >> 4), idesc,
+                                   kk ? 1u : 0u);
             } else {
 #pragma unroll
                 for (int kk = 0; kk < kDI / 16; ++kk) {
@@ -561,7 +557,7 @@ __global__ void __launch_bounds__(kThreads, 1) index_score_tc_kernel(const __gri
     if (warp == 0) {
         if (lane == 0) idx_producer<FP8, G>(sm, a, &kmap, f0, f1);
     } else if (warp == 1) {
-        if (lane == 0) idx_mma<FP8, NP, G>(sm, a, tmem, f0, f1);
+        idx_mma<FP8, NP, G>(sm, a, tmem, f0, f1);  // the whole warp (one elected lane issues)
     } else if (warp < 6) {
         idx_stage<FP8, NP, G>(sm, a, f0, f1);
     } else {
@@ -664,18 +660,18 @@ __device__ void mx_mma(IdxSmem& sm, const IdxTcArgs& a, uint32_t tmem, long long
     int seg = 0, b = 0;
     ICursor cur(f0, a, 1);
     for (long long f = f0; f < f1; ++f, cur.next(a)) {
-        if (aborted(sm)) { ok = false; break; }
+        if (warp_aborted(sm)) { ok = false; break; }
         const int jt = (int)(f - f0);
         const int st = jt % kMxStages, slot = jt & 1, sd = jt % kDS;
         if (f == f0 || cur.ti == 0) {
             b = seg & 1;
-            if (!tc::mbar_wait(&sm.q_full[b], (seg >> 1) & 1)) { ok = false; break; }
+            if (!warp_wait(&sm.q_full[b], (seg >> 1) & 1)) { ok = false; break; }
             ++seg;
         }
         const bool seg_end = (f == f1 - 1) || (cur.ti == a.tiles_per_row - 1);
-        if (!tc::mbar_wait(&sm.k_full[st], (uint32_t)(jt / kMxStages) & 1)) { ok = false; break; }
-        if (!tc::mbar_wait(&sm.sf_full[slot], (uint32_t)(jt >> 1) & 1)) { ok = false; break; }
-        if (jt >= kDS && !tc::mbar_wait(&sm.d_free[sd], (uint32_t)((jt / kDS) - 1) & 1)) { ok = false; break; }
+        if (!warp_wait(&sm.k_full[st], (uint32_t)(jt / kMxStages) & 1)) { ok = false; break; }
+        if (!warp_wait(&sm.sf_full[slot], (uint32_t)(jt >> 1) & 1)) { ok = false; break; }
+        if (jt >= kDS && !warp_wait(&sm.d_free[sd], (uint32_t)((jt / kDS) - 1) & 1)) { ok = false; break; }
         tc::tc_fence_after();
         const uint64_t a0 = ring_desc + (uint64_t)((st * kMxStageBytes) >> 4), b0 = b ? q_desc1 : q_desc0;
         const uint32_t d0 = tmem + Acc::kCols * sd, sfa = tmem + kMxSfaCol + 16 * slot, sfb = tmem + kMxSfbCol + 16 * b;
@@ -916,7 +912,7 @@ __global__ void __launch_bounds__(kThreads, 1) index_score_mx_kernel(const __gri
     if (warp == 0) {
         if (lane == 0) mx_producer(sm, a, &kmap, f0, f1);
     } else if (warp == 1) {
-        if (lane == 0) mx_mma<NP>(sm, a, tmem, f0, f1);
+        mx_mma<NP>(sm, a, tmem, f0, f1);  // the whole warp (one elected lane issues)
     } else if (warp < 6) {
         mx_stage<NP>(sm, a, tmem, f0, f1);
     } else {
