@@ -51,6 +51,12 @@ constexpr uint32_t kColS = 256;                  // S: 2 buffers of 64 columns
 constexpr uint32_t kTmemCols = 512;
 constexpr int kThreads = 192;
 constexpr float kRescaleSlack = 8.0f;  // keep a stale running max until the true one exceeds it by 2^8
+// Piece layout: a piece (partial O of a query split between CTAs) holds O[h][d] for 64 heads x 512
+// dims as float4 groups of four heads: the group of heads 4i .. 4i+3 at dim d is float4 number
+// ((d / 32) * 16 + i) * 32 + d % 32.  This is the order the epilogue's threads hold O^T in (thread
+// = TMEM lane = dim, its registers = heads), so each warp store is 512 contiguous bytes, and the
+// combine reads it back in the same 512-byte runs.  (Stored d-major, [d][64 heads], a warp store
+// touched 32 cache lines and a 128 KB piece took ~9,900 cycles to write on B200.)
 
 constexpr uint32_t kIdescQK = tc::idesc_f16(64, kTile, 0, 0);
 constexpr uint32_t kIdescPV = tc::idesc_f16(128, 64, 1, 0);
@@ -75,7 +81,7 @@ struct TcArgs {
     const int32_t* idx;  // CSA selections, or null for HCA
     float* out;
     float* part_ml;      // [2*grid][64][2]
-    float* part_o;       // [2*grid][64][512]
+    float* part_o;       // [2*grid] pieces of 64 x 512 floats (piece layout above)
     int* dev_status;
     long long n_ent, l_tok, tok_pos0, ctx_len, total_tiles;
     int rows, n_q, m, k, window;
@@ -542,12 +548,13 @@ __device__ void softmax_warps(Smem& sm, const TcArgs& a, uint32_t tmem, long lon
                         dst[i * kD + d] = v;
                     }
                 } else {
-                    // a piece is stored d-major ([d][64 heads]): this thread's 64 heads are contiguous
-                    float4* pd = reinterpret_cast<float4*>(dst + (long long)d * kH);
+                    // a piece is stored in the order the threads hold it (piece layout): one warp store
+                    // writes 512 contiguous bytes, heads 4i .. 4i+3 of this warp's 32 dims
+                    float4* pd = reinterpret_cast<float4*>(dst) + (long long)(4 * cc + sub) * (16 * 32) + lane;
 #pragma unroll
                     for (int i = 0; i < kH / 4; ++i)
-                        pd[i] = make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
-                                            __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
+                        pd[32 * i] = make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
+                                                 __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
                 }
             }
             tc::tc_fence_before();
@@ -617,22 +624,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // Merge the partials of queries whose tiles were split between CTAs.
-// grid (rows, 512 / kDC d chunks), 256 threads, a.comb_pieces * 64 floats of dynamic shared memory
-// (at least the pieces of any query).  Pieces are stored d-major ([d][64 heads]), so a block's
-// kDC d x 64 heads of one piece are one run of kDC * 256 bytes: each thread loads 16 bytes of it
-// (one d, four heads) per 16 d, for up to kU pieces before using any of them.  kDC = 16 gives few
-// queries many blocks; kDC = 64 gives many queries few enough blocks to be resident at once.  The
-// per-head weights exp2(m_piece - m_max) come first, from four groups of 64 threads each taking
-// every fourth piece; the weighted sum is scaled by 1 / l at the end and written to
-// out[row][h][d0 .. d0 + kDC - 1] through a shared-memory transpose.
-template <int kDC>
+// grid (rows, 16 groups of 32 dims), 256 threads, a.comb_pieces * 64 floats of dynamic shared memory
+// (at least the pieces of any query).  The per-head weights exp2(m_piece - m_max) come first, from
+// four groups of 64 threads each taking every fourth piece.  Then warp w sums heads 4w .. 4w+3 and
+// 4w+32 .. 4w+35 of the block's 32 dims (lane = dim) over the pieces: per piece two float4 loads, each
+// warp-wide load one 512-byte run of the piece (piece layout), up to kU pieces in flight.  The sums
+// are scaled by 1 / l and written to out[row][h][d], 32 consecutive dims (128 bytes) per warp store.
 __global__ void __launch_bounds__(256) attend_tc_combine(TcArgs a) {
     griddep_wait();  // everything before this kernel on the stream has finished
     griddep_launch_dependents();
-    static_assert(kDC % 16 == 0 && 256 % kDC == 0, "d chunk");
-    constexpr int kR = kDC / 16;          // d rows per thread
-    constexpr int kU = kR == 1 ? 8 : 4;   // pieces whose loads are in flight together
-    const int row = blockIdx.x, d0 = blockIdx.y * kDC;
+    constexpr int kU = 4;  // pieces whose loads are in flight together
+    const int row = blockIdx.x, dg = blockIdx.y;
     const long long rs = (long long)row * a.tpr, re = rs + a.tpr - 1;
     // CTA holding flat tile f: the largest c with range_start(c) <= f
     auto cta_of = [&](long long f) { return (int)(((f + 1) * a.grid - 1) / a.total_tiles); };
@@ -649,7 +651,6 @@ __global__ void __launch_bounds__(256) attend_tc_combine(TcArgs a) {
     __shared__ int s_slot[kNumSMs + kU];
     __shared__ float s_red[4][kH];
     __shared__ __align__(16) float s_inv[kH];
-    __shared__ float s_acc[kH][kDC + 1];
     const int t = threadIdx.x, g = t >> 6, h = t & (kH - 1);
     for (int i = t; i < n; i += blockDim.x)
         s_slot[i] = 2 * (c0 + i) + ((i == 0 && range_start(c0, a) < rs) ? 1 : 0);
@@ -690,59 +691,52 @@ __global__ void __launch_bounds__(256) attend_tc_combine(TcArgs a) {
         if (a.sink && mmax != -INFINITY) l += exp2f(a.sink[h] * 1.4426950408889634f - mmax);  // the sink's share
         s_inv[h] = isnan(l) ? NAN : (l > 0.f ? 1.f / l : 0.f);  // an empty row stays zero
     }
-    // thread t: d rows t / 16 + 16 r (r < kR) of the chunk, heads hq .. hq + 3 (a piece of weight 0
-    // holds finite values: it adds 0)
-    const int dr = t >> 4, hq = (t & 15) * 4;
-    const float* src = a.part_o + (long long)(d0 + dr) * kH + hq;
-    float4 acc[kR];
-#pragma unroll
-    for (int r = 0; r < kR; ++r) acc[r] = make_float4(0.f, 0.f, 0.f, 0.f);
+    __syncthreads();  // s_w and s_inv are written
+    // thread (warp w, lane): dim 32 dg + lane, head quads w and w + 8 (a piece of weight 0 holds finite
+    // values: it adds 0)
+    const int w = t >> 5, lane = t & 31, d = 32 * dg + lane;
+    const float4* src = reinterpret_cast<const float4*>(a.part_o) + (long long)dg * (16 * 32) + lane;
+    float4 acc[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
     for (int i0 = 0; i0 < n; i0 += kU) {
-        float4 v[kU][kR];
+        float4 v[kU][2];
 #pragma unroll
         for (int u = 0; u < kU; ++u)
 #pragma unroll
-            for (int r = 0; r < kR; ++r)
-                v[u][r] = i0 + u < n ? __ldcg(reinterpret_cast<const float4*>(src + (long long)s_slot[i0 + u] * kH * kD +
-                                                                                16 * r * kH))
+            for (int r = 0; r < 2; ++r)
+                v[u][r] = i0 + u < n ? __ldcg(src + (long long)s_slot[i0 + u] * (kH * kD / 4) + 32 * (w + 8 * r))
                                      : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
         for (int u = 0; u < kU; ++u) {
             if (i0 + u >= n) break;
-            const float4 w = *reinterpret_cast<const float4*>(s_w + (i0 + u) * kH + hq);
 #pragma unroll
-            for (int r = 0; r < kR; ++r) {
-                acc[r].x = fmaf(w.x, v[u][r].x, acc[r].x);
-                acc[r].y = fmaf(w.y, v[u][r].y, acc[r].y);
-                acc[r].z = fmaf(w.z, v[u][r].z, acc[r].z);
-                acc[r].w = fmaf(w.w, v[u][r].w, acc[r].w);
+            for (int r = 0; r < 2; ++r) {
+                const float4 wt = *reinterpret_cast<const float4*>(s_w + (i0 + u) * kH + 4 * (w + 8 * r));
+                acc[r].x = fmaf(wt.x, v[u][r].x, acc[r].x);
+                acc[r].y = fmaf(wt.y, v[u][r].y, acc[r].y);
+                acc[r].z = fmaf(wt.z, v[u][r].z, acc[r].z);
+                acc[r].w = fmaf(wt.w, v[u][r].w, acc[r].w);
             }
         }
     }
-    __syncthreads();  // s_inv is written
-    {
-        const float4 inv = *reinterpret_cast<const float4*>(s_inv + hq);  // NaN for a poisoned head
-#pragma unroll
-        for (int r = 0; r < kR; ++r) {
-            s_acc[hq][dr + 16 * r] = acc[r].x * inv.x;
-            s_acc[hq + 1][dr + 16 * r] = acc[r].y * inv.y;
-            s_acc[hq + 2][dr + 16 * r] = acc[r].z * inv.z;
-            s_acc[hq + 3][dr + 16 * r] = acc[r].w * inv.w;
-        }
-    }
-    __syncthreads();
-    // write out[row][h][d0 .. d0 + kDC - 1]: thread t takes d = d0 + t % kDC of heads t / kDC,
-    // t / kDC + 256 / kDC, ... (output RoPE: the pair partner of d is d ^ 1, in the same chunk)
-    const int lane = t & (kDC - 1), hg = t / kDC, d = d0 + lane;
+    // out[row][h][d] (output RoPE: the pair partner of d is d ^ 1, the neighbouring lane)
     const bool rot = a.rope_dims > 0 && d >= kD - a.rope_dims;
     float rs_ = 0.f, rc_ = 1.f;
     if (rot)
         rope_sincos(a.ctx_len - a.n_q + (row % a.n_q), (d - (kD - a.rope_dims)) >> 1, a.rope_dims, a.rope_base, &rs_,
                     &rc_);
-    for (int hh = hg; hh < kH; hh += 256 / kDC) {
-        float v = s_acc[hh][lane];
-        if (rot) v = rope_apply(d, v, s_acc[hh][lane ^ 1], rs_, rc_);
-        a.out[((long long)row * kH + hh) * kD + d] = v;
+    float* orow = a.out + (long long)row * kH * kD + d;
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        const int h0 = 4 * (w + 8 * r);
+        const float4 inv = *reinterpret_cast<const float4*>(s_inv + h0);  // NaN for a poisoned head
+        const float vals[4] = {acc[r].x * inv.x, acc[r].y * inv.y, acc[r].z * inv.z, acc[r].w * inv.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            float vv = vals[j];
+            const float pp = __shfl_xor_sync(0xffffffffu, vv, 1);
+            if (rot) vv = rope_apply(d, vv, pp, rs_, rc_);
+            orow[(long long)(h0 + j) * kD] = vv;
+        }
     }
 }
 
@@ -872,11 +866,8 @@ cudaError_t launch_attend_tc(const AttendArgs& a, void* ws, size_t ws_bytes, cud
     if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     if (p.grid > 1) {
-        // 16-d chunks while rows x 32 blocks stay within two per SM, else 64-d chunks
         const size_t csm = (size_t)t.comb_pieces * kH * sizeof(float);
-        e = (long long)t.rows * (kD / 16) <= 2LL * kNumSMs
-                ? launch_pdl(attend_tc_combine<16>, dim3(t.rows, kD / 16), dim3(256), csm, stream, t)
-                : launch_pdl(attend_tc_combine<64>, dim3(t.rows, kD / 64), dim3(256), csm, stream, t);
+        e = launch_pdl(attend_tc_combine, dim3(t.rows, kD / 32), dim3(256), csm, stream, t);
         if (e == cudaSuccess) e = cudaGetLastError();
     }
     return e;
