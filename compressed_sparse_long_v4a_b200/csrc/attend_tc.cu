@@ -230,6 +230,24 @@ __device__ __forceinline__ bool tile_rows(const TcArgs& a, int row, int ti, int 
     return true;
 }
 
+// Warp 0 lane 0, before the grid dependency wait: the query of the CTA's first segment and an L2
+// prefetch of its first contiguous (TMA-loaded) entry tiles.  Both only read.  No kernel of this library
+// writes attention queries, and a kernel before this one on the stream that is not programmatically
+// launched has completed before this one starts, so the query is complete; the prefetch only warms L2,
+// the point of coherence, so an entry still being written is read afresh by the load after the wait.
+__device__ void early_loads(Smem& sm, const TcArgs& a, const CUtensorMap* ent_map, const CUtensorMap* q_map,
+                            long long f0, long long f1) {
+    const Cursor cur(f0, a.tpr);
+    tc::mbar_arrive_expect_tx(&sm.q_full, kQBytes);
+    for (int c = 0; c < kSlabs; ++c) tc::tma_load_2d(sm.q + c * kH * 128, q_map, 64 * c, cur.row * kH, &sm.q_full);
+    if (a.idx || a.bt) return;
+    const RowInfo ri = row_info(cur.row, a);
+    for (int j = 0; j < kStages && f0 + j < f1 && cur.ti + j < a.e_tiles; ++j) {
+        const int y = (int)((long long)ri.b * a.n_ent + (long long)(cur.ti + j) * kTile);
+        for (int c = 0; c < kSlabs; ++c) tc::tma_prefetch_2d(ent_map, 64 * c, y);
+    }
+}
+
 __device__ void producer(Smem& sm, const TcArgs& a, const CUtensorMap* ent_map, const CUtensorMap* tok_map,
                          const CUtensorMap* q_map, long long f0, long long f1) {
     const int lane = threadIdx.x & 31;
@@ -256,7 +274,7 @@ __device__ void producer(Smem& sm, const TcArgs& a, const CUtensorMap* ent_map, 
         }
         if (seg_start) {
             if (seg > 0 && !tc::mbar_wait(&sm.q_empty, (seg - 1) & 1)) { fault(sm, a); break; }
-            if (lane == 0) {
+            if (lane == 0 && seg > 0) {  // the first segment's query was requested before the dependency wait
                 tc::mbar_arrive_expect_tx(&sm.q_full, kQBytes);
                 for (int c = 0; c < kSlabs; ++c) tc::tma_load_2d(sm.q + c * kH * 128, q_map, 64 * c, row * kH, &sm.q_full);
             }
@@ -305,7 +323,9 @@ __device__ void producer(Smem& sm, const TcArgs& a, const CUtensorMap* ent_map, 
         if (jt < 0) continue;
         tc::mbar_wait(&sm.kv_full[jt % kStages], (jt / kStages) & 1);
     }
-    if (seg > 0) tc::mbar_wait(&sm.q_full, (seg - 1) & 1);
+    // ... nor a query load (the first segment's was issued before the loop)
+    const int q_loads = seg > 0 ? seg : (f0 < f1 ? 1 : 0);
+    if (q_loads > 0) tc::mbar_wait(&sm.q_full, (q_loads - 1) & 1);
 }
 
 // ---------------------------------------------------------------------
@@ -602,7 +622,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
-    griddep_wait();  // the prologue above touched only shared and tensor memory
+    if (warp == 0 && (threadIdx.x & 31) == 0 && f0 < f1) early_loads(sm, a, &ent_map, &q_map, f0, f1);
+    griddep_wait();  // the prologue above touched only shared and tensor memory (and read the query)
     // No early griddep_launch_dependents here: the next kernel (the combine, or the next call) is let
     // in as this grid's CTAs exit, so its blocks spread over every SM instead of packing onto the first
     // SMs to free up (measured on B200: the 32-query combine ran 1.8 us faster, the step 2 us faster).

@@ -274,9 +274,13 @@ constexpr int kFastThreads = 512;
 constexpr int kFastPer = 8;                              // consecutive scores per thread per step
 constexpr int kFastStep = kFastThreads * kFastPer;       // 4096 scores per block step
 constexpr int kMaxFastRows = 256;
-constexpr int kMaxParts = 512;
+constexpr int kMaxFastParts = 512;
 constexpr int kCandCap = 7168;   // candidates the finishing block holds in shared memory (two blocks fit an SM)
 constexpr size_t kFastSmem = (size_t)kCandCap * 8 + 2 * 4096 * sizeof(int32_t);
+constexpr int kMaxK = 4096;      // largest k the API takes
+constexpr int kSelCap = 4096;    // threshold-bin candidates of a row the few-rows select holds
+constexpr size_t kSelSmem = (size_t)kSelCap * 8 + 2 * kMaxK * sizeof(int32_t);
+
 
 // Block-wide bin search: thread t owns bins [P t, P t + P) with counts c[] (in registers).
 // Finds the bin d where the keys in bins above d number fewer than `rem` while bins >= d hold at
@@ -522,159 +526,280 @@ __device__ void finish_lists(const float* sc, int k, int D, int C, int32_t* defs
 }
 
 
-__device__ void finish_row(const float* sc, long long nvis, int k, int parts, long long chunk, const int32_t* def_row,
-                           const int32_t* cidx_row, const uint32_t* ckey_row, const int* counts_row, int32_t* io,
-                           float* so, uint8_t* dsm) {
-    uint32_t* ckey = reinterpret_cast<uint32_t*>(dsm);           // [kCandCap]
-    int32_t* cidx = reinterpret_cast<int32_t*>(ckey + kCandCap);  // [kCandCap]
-    int32_t* defs = cidx + kCandCap;                              // [4096]
-    int32_t* sels = defs + 4096;                                  // [4096]
-    __shared__ int doff[kMaxParts + 1], coff[kMaxParts + 1];
-    __shared__ int warp_buf[33];
-    {
-        // prefix sums of the parts' counts (parts <= kMaxParts = blockDim)
-        const int p = threadIdx.x;
-        const int nd = p < parts ? __ldcg(counts_row + 2 * p) : 0;
-        const int nc = p < parts ? __ldcg(counts_row + 2 * p + 1) : 0;
-        int td, tc;
-        const int ed = block_exclusive_scan(nd, warp_buf, &td);
-        const int ec = block_exclusive_scan(nc, warp_buf, &tc);
-        if (p < parts) {
-            doff[p] = ed;
-            coff[p] = ec;
+// Bitonic sort of v[0 .. n2) ascending in shared memory (n2 a power of two; padded with 0x7fffffff).
+// Whole block.
+__device__ void bitonic_sort(int32_t* v, int n2) {
+    for (int size = 2; size <= n2; size <<= 1) {
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            for (int i = threadIdx.x; i < (n2 >> 1); i += blockDim.x) {
+                const int lo = 2 * i - (i & (stride - 1)), hi = lo + stride;
+                const int32_t x = v[lo], y = v[hi];
+                if ((x > y) == ((lo & size) == 0)) {
+                    v[lo] = y;
+                    v[hi] = x;
+                }
+            }
+            __syncthreads();
         }
-        if (p == 0) {
-            doff[parts] = td;
-            coff[parts] = tc;
-        }
-        __syncthreads();
     }
-    const int D = doff[parts], C = coff[parts];
-    if (C > kCandCap || D > 4096) {
-        // more candidates than the fast path holds (e.g. huge blocks of equal scores): exact select over the row
+}
+
+__device__ __forceinline__ int pow2_at_least(int n) {
+    int p = 1;
+    while (p < n) p <<= 1;
+    return p;
+}
+
+// ---------------------------------------------------------------------
+// select for few query rows: kFastThreads-thread blocks, `parts` per row
+// ---------------------------------------------------------------------
+// Block (row, p) finds the threshold bin (the 12-bit bin of the row's k-th largest key, from the
+// histogram the scoring kernel built) and compacts entries [p chunk, (p+1) chunk) of the row into the
+// row's two lists in global memory: definite entries (keys in higher bins; fewer than k in the row)
+// and candidates (keys in the threshold bin, with their keys), reserving its span of both with one
+// 64-bit atomic per step.  The last block of the row to finish (an atomic ticket; nothing waits)
+// finishes the row: a radix select over the candidates' low 20 key bits picks the best `need`
+// (ties to the lower entries), and the chosen entries are marked in a bitmap over the row whose
+// prefix counts give each its place in the ascending output (rows longer than the bitmap sort the
+// chosen entries instead).  Loops are kept rolled: these blocks run briefly, and on B200 a short
+// kernel's time went largely to fetching its instructions (a step streams more than L2 holds), at
+// about 120 cycles per element for an unrolled 32-element loop.
+constexpr int kBitmapWords = kSelCap * 2;  // the candidate arrays, reused: rows of up to 262,144 entries
+
+__device__ void finish_row(const float* sc, long long nvis, int k, int D, int C, const int32_t* def_row,
+                           const int32_t* cidx_row, const uint32_t* ckey_row, int32_t* io, float* so, uint8_t* dsm) {
+    uint32_t* ckey = reinterpret_cast<uint32_t*>(dsm);          // [kSelCap]
+    int32_t* cidx = reinterpret_cast<int32_t*>(ckey + kSelCap);  // [kSelCap]
+    int32_t* sel = cidx + kSelCap;                               // [kMaxK]: the answer
+    int32_t* eqv = sel + kMaxK;                                  // [kMaxK]: candidates equal to the threshold key
+    uint32_t* bits = ckey;                                       // [kBitmapWords] once the candidates are used
+    __shared__ unsigned int h1[1024];
+    __shared__ int s_ngt, s_neq, warp_buf[33];
+    if (C > kSelCap || D > k) {
+        // more candidates than the finish holds (e.g. huge blocks of equal scores): exact select over the row
         select_row_radix(sc, nvis, k, io, so);
         return;
     }
-    // gather the definite entries and the candidates, both in ascending entry order; every element
-    // finds its part by binary search over the offsets, and each thread issues the loads of up to
-    // kG elements before using any of them
-    constexpr int kG = 8;
-    for (int e0 = threadIdx.x; e0 < D + C; e0 += kG * blockDim.x) {
-        long long src[kG];
-        int32_t vi[kG];
-        uint32_t vk[kG];
+    // the lists, four loads in flight per thread
+#pragma unroll 1
+    for (int i0 = threadIdx.x; i0 < C; i0 += 4 * kFastThreads) {
+        uint32_t kk[4];
+        int32_t ii[4];
 #pragma unroll
-        for (int g = 0; g < kG; ++g) {
-            const int e = e0 + g * blockDim.x;
-            src[g] = -1;
-            if (e < D + C) {
-                const bool is_def = e < D;
-                const int x = is_def ? e : e - D;
-                const int* off = is_def ? doff : coff;
-                int lo = 0, hi = parts;  // largest p with off[p] <= x
-                while (hi - lo > 1) {
-                    const int mid = (lo + hi) >> 1;
-                    if (off[mid] <= x) lo = mid;
-                    else hi = mid;
-                }
-                src[g] = (long long)lo * chunk + (x - off[lo]);
-            }
+        for (int u = 0; u < 4; ++u) {
+            const int i = i0 + u * kFastThreads;
+            kk[u] = i < C ? __ldcg(ckey_row + i) : 0u;
+            ii[u] = i < C ? __ldcg(cidx_row + i) : 0;
         }
 #pragma unroll
-        for (int g = 0; g < kG; ++g) {
-            const int e = e0 + g * blockDim.x;
-            vi[g] = 0;
-            vk[g] = 0;
-            if (src[g] >= 0) {
-                vi[g] = e < D ? __ldcg(def_row + src[g]) : __ldcg(cidx_row + src[g]);
-                if (e >= D) vk[g] = __ldcg(ckey_row + src[g]);
-            }
-        }
-#pragma unroll
-        for (int g = 0; g < kG; ++g) {
-            const int e = e0 + g * blockDim.x;
-            if (src[g] < 0) continue;
-            if (e < D) {
-                defs[e] = vi[g];
-            } else {
-                cidx[e - D] = vi[g];
-                ckey[e - D] = vk[g];
+        for (int u = 0; u < 4; ++u) {
+            const int i = i0 + u * kFastThreads;
+            if (i < C) {
+                ckey[i] = kk[u];
+                cidx[i] = ii[u];
             }
         }
     }
+#pragma unroll 1
+    for (int i0 = threadIdx.x; i0 < D; i0 += 4 * kFastThreads) {
+        int32_t dd[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) dd[u] = i0 + u * kFastThreads < D ? __ldcg(def_row + i0 + u * kFastThreads) : 0;
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if (i0 + u * kFastThreads < D) sel[i0 + u * kFastThreads] = dd[u];
+    }
+    if (threadIdx.x == 0) {
+        s_ngt = D;
+        s_neq = 0;
+    }
+    const int need = (D + C) <= k ? C : k - D;  // candidates to take
+    const bool take_all = need >= C;
     __syncthreads();
-    finish_lists(sc, k, D, C, defs, cidx, ckey, sels, io, so);
+    // radix select of the need-th largest candidate key over its low 20 bits (the top 12 are equal)
+    uint32_t prefix = C > 0 ? (ckey[0] & 0xfff00000u) : 0u, mask = 0xfff00000u;
+    int rem = need;
+    if (!take_all) {
+#pragma unroll 1
+        for (int shift = 10; shift >= 0; shift -= 10) {
+            for (int i = threadIdx.x; i < 1024; i += blockDim.x) h1[i] = 0;
+            __syncthreads();
+#pragma unroll 1
+            for (int i = threadIdx.x; i < C; i += blockDim.x)
+                if ((ckey[i] & mask) == prefix) atomicAdd(&h1[(ckey[i] >> shift) & 1023u], 1u);
+            __syncthreads();
+            int dgt;
+            long long above;
+            find_digit_1024(h1, rem, &dgt, &above);
+            prefix |= (uint32_t)dgt << shift;
+            rem -= (int)above;
+            mask |= 1023u << shift;
+        }
+    }
+    // candidates above the threshold key join the answer; those equal to it are collected (rem of them
+    // are taken, the lowest entries)
+#pragma unroll 1
+    for (int i0 = 0; i0 < C; i0 += blockDim.x) {  // warp-uniform trip count (ballots below)
+        const int i = i0 + threadIdx.x;
+        const uint32_t key = i < C ? ckey[i] : 0u;
+        const bool gt = i < C && (take_all || key > prefix);
+        const bool eq = i < C && !take_all && key == prefix;
+        const unsigned mg = __ballot_sync(0xffffffffu, gt), me = __ballot_sync(0xffffffffu, eq);
+        const int lane = threadIdx.x & 31;
+        int bg = 0, be = 0;
+        if (lane == 0) {
+            bg = mg ? atomicAdd(&s_ngt, __popc(mg)) : 0;
+            be = me ? atomicAdd(&s_neq, __popc(me)) : 0;
+        }
+        bg = __shfl_sync(0xffffffffu, bg, 0);
+        be = __shfl_sync(0xffffffffu, be, 0);
+        const unsigned below = (1u << lane) - 1u;
+        if (gt) sel[bg + __popc(mg & below)] = cidx[i];
+        if (eq && be + __popc(me & below) < kMaxK) eqv[be + __popc(me & below)] = cidx[i];
+    }
+    __syncthreads();
+    const int ngt = s_ngt, neq = s_neq;
+    if (!take_all && rem > 0) {
+        if (neq > kMaxK) {  // (at most k - D tied keys are wanted; a larger tie goes the exact way)
+            select_row_radix(sc, nvis, k, io, so);
+            return;
+        }
+        if (rem < neq) {  // the lowest entries among the tied candidates
+            const int n2 = pow2_at_least(neq);
+            for (int i = neq + threadIdx.x; i < n2; i += blockDim.x) eqv[i] = 0x7fffffff;
+            __syncthreads();
+            bitonic_sort(eqv, n2);
+        }
+        for (int i = threadIdx.x; i < rem; i += blockDim.x) sel[ngt + i] = eqv[i];
+    }
+    const int total = ngt + (take_all ? 0 : rem);
+    __syncthreads();
+    const int words = (int)((nvis + 31) >> 5);
+    if (words <= kBitmapWords) {
+        // bitmap over the row; thread t owns words [t per, t per + per), its set bits go out in order after
+        // those of lower threads
+        for (int i = threadIdx.x; i < words; i += blockDim.x) bits[i] = 0u;
+        __syncthreads();
+        for (int i = threadIdx.x; i < total; i += blockDim.x) atomicOr(&bits[sel[i] >> 5], 1u << (sel[i] & 31));
+        __syncthreads();
+        const int per = (words + (int)blockDim.x - 1) / (int)blockDim.x, w0 = threadIdx.x * per;
+        int cnt = 0;
+#pragma unroll 1
+        for (int j = 0; j < per; ++j)
+            if (w0 + j < words) cnt += __popc(bits[w0 + j]);
+        int tot;
+        int pos = block_exclusive_scan(cnt, warp_buf, &tot);
+#pragma unroll 1
+        for (int j = 0; j < per; ++j) {
+            uint32_t b = w0 + j < words ? bits[w0 + j] : 0u;
+            while (b) {
+                const int32_t x = (int32_t)((w0 + j) * 32 + __ffs(b) - 1);
+                b &= b - 1;
+                io[pos++] = x;
+            }
+        }
+    } else {
+        const int n2 = pow2_at_least(total < 2 ? 2 : total);
+        for (int i = total + threadIdx.x; i < n2; i += blockDim.x) sel[i] = 0x7fffffff;
+        __syncthreads();
+        bitonic_sort(sel, n2);
+        for (int p = threadIdx.x; p < total; p += blockDim.x) io[p] = sel[p];
+    }
+    for (int p = total + threadIdx.x; p < k; p += blockDim.x) io[p] = -1;
+    if (so) {
+        __syncthreads();  // io is written (by this block; read back below)
+#pragma unroll 1
+        for (int p = threadIdx.x; p < k; p += blockDim.x) {
+            const int32_t x = __ldcg(io + p);
+            so[p] = x >= 0 ? __ldcg(sc + x) : -INFINITY;
+        }
+    }
 }
 
-// grid rows * parts, kFastThreads threads.  Block (row, p) compacts entries [p*chunk, (p+1)*chunk)
-// of the row: definite entries (bin above the threshold bin) and candidates (the threshold bin),
-// each in ascending entry order; the last block of the row to finish (counted on row_done, which
-// starts at zero) then finishes the row.
+// grid rows * parts, kFastThreads threads (see above).  ctr: per row one 64-bit word (definite entries
+// in its low half, candidates in its high half) and one finished-parts count, all starting at zero.
 __global__ void __launch_bounds__(kFastThreads) topk_fast_kernel(const float* scores, const uint32_t* hist, IndexArgs a,
                                                                  int k, int parts, long long chunk, int32_t* def_buf,
-                                                                 int32_t* cidx_buf, uint32_t* ckey_buf, int* counts,
-                                                                 unsigned int* row_done, int32_t* idx_out,
+                                                                 int32_t* cidx_buf, uint32_t* ckey_buf,
+                                                                 unsigned long long* ctr, int32_t* idx_out,
                                                                  float* score_out) {
     griddep_wait();  // everything before this kernel on the stream has finished
     griddep_launch_dependents();
     extern __shared__ __align__(16) uint8_t dsm[];
     __shared__ int warp_buf[33];
     __shared__ int s_last;
+    __shared__ unsigned long long s_base;
     const int row = blockIdx.x / parts, p = blockIdx.x % parts;
     const long long nvis = row_nvis(a, row);
     int tbin, above;
     bool all;
     threshold_bin(hist + (long long)row * kHistBins, k, &tbin, &above, &all);
     const float* sc = scores + (long long)row * a.n_ent;
-    const long long row_off = (long long)row * a.n_ent;
     const long long lo = (long long)p * chunk;
     long long hi = lo + chunk;
     if (hi > nvis) hi = nvis;
-    int32_t* dout = def_buf + row_off + lo;
-    int32_t* ciout = cidx_buf + row_off + lo;
-    uint32_t* ckout = ckey_buf + row_off + lo;
-    int n_def = 0, n_cand = 0;
+    int32_t* dout = def_buf + (long long)row * k;
+    int32_t* ciout = cidx_buf + (long long)row * kSelCap;
+    uint32_t* ckout = ckey_buf + (long long)row * kSelCap;
+    unsigned long long* rc = ctr + 2LL * row;
+    const bool vec = (reinterpret_cast<uintptr_t>(sc) & 15) == 0;
+#pragma unroll 1
     for (long long base = lo; base < hi; base += kFastStep) {
-        // this thread's kFastPer consecutive scores
+        // this thread's kFastPer consecutive scores (16-byte loads when the row is 16-byte aligned)
         const long long s0 = base + (long long)threadIdx.x * kFastPer;
-        uint32_t keys[kFastPer];
+        float v[kFastPer];
+        if (vec && s0 + kFastPer <= hi) {
+            const float4 x0 = __ldcg(reinterpret_cast<const float4*>(sc + s0));
+            const float4 x1 = __ldcg(reinterpret_cast<const float4*>(sc + s0) + 1);
+            v[0] = x0.x; v[1] = x0.y; v[2] = x0.z; v[3] = x0.w;
+            v[4] = x1.x; v[5] = x1.y; v[6] = x1.z; v[7] = x1.w;
+        } else {
+#pragma unroll
+            for (int i = 0; i < kFastPer; ++i) v[i] = s0 + i < hi ? __ldcg(sc + s0 + i) : 0.f;
+        }
         int nd = 0, nc = 0;
 #pragma unroll
         for (int i = 0; i < kFastPer; ++i) {
-            const long long s = s0 + i;
-            keys[i] = s < hi ? float_to_ordered(sc[s]) : 0u;  // L1 serves the warp's 1 KB after its first load
-            const int bin = (int)(keys[i] >> 20);
-            nd += (s < hi && (all || bin > tbin)) ? 1 : 0;
-            nc += (s < hi && !all && bin == tbin) ? 1 : 0;
+            const int bin = (int)(float_to_ordered(v[i]) >> 20);
+            const bool in = s0 + i < hi;
+            nd += (in && (all || bin > tbin)) ? 1 : 0;
+            nc += (in && !all && bin == tbin) ? 1 : 0;
         }
         int tot;
         const int packed = block_exclusive_scan(nd | (nc << 16), warp_buf, &tot);
-        int od = n_def + (packed & 0xffff), oc = n_cand + (packed >> 16);
-#pragma unroll
+        if (threadIdx.x == 0)
+            s_base = atomicAdd(rc, (unsigned long long)(tot & 0xffff) | ((unsigned long long)(tot >> 16) << 32));
+        __syncthreads();
+        int od = (int)(s_base & 0xffffffffu) + (packed & 0xffff), oc = (int)(s_base >> 32) + (packed >> 16);
+#pragma unroll 1
         for (int i = 0; i < kFastPer; ++i) {
-            const long long s = s0 + i;
-            const int bin = (int)(keys[i] >> 20);
-            if (s < hi && (all || bin > tbin)) dout[od++] = (int32_t)s;
-            if (s < hi && !all && bin == tbin) {
-                ciout[oc] = (int32_t)s;
-                ckout[oc++] = keys[i];
+            const uint32_t key = float_to_ordered(v[i]);
+            const int bin = (int)(key >> 20);
+            const bool in = s0 + i < hi;
+            if (in && (all || bin > tbin)) {
+                if (od < k) dout[od] = (int32_t)(s0 + i);  // fewer than k entries lie above the threshold bin
+                ++od;
+            }
+            if (in && !all && bin == tbin) {
+                if (oc < kSelCap) {
+                    ciout[oc] = (int32_t)(s0 + i);
+                    ckout[oc] = key;
+                }
+                ++oc;
             }
         }
-        n_def += tot & 0xffff;
-        n_cand += tot >> 16;
+        __syncthreads();  // s_base is read before the next step overwrites it
     }
-    if (threadIdx.x == 0) {
-        counts[((long long)row * parts + p) * 2] = n_def;
-        counts[((long long)row * parts + p) * 2 + 1] = n_cand;
-        __threadfence();  // this part's lists and counts are visible before it is counted
-        s_last = atomicAdd(row_done + row, 1u) == (unsigned)(parts - 1);
-    }
+    __threadfence();  // this block's list entries are visible before it is counted
+    __syncthreads();
+    if (threadIdx.x == 0)
+        s_last = atomicAdd(reinterpret_cast<unsigned int*>(rc + 1), 1u) == (unsigned)(parts - 1);
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    finish_row(sc, nvis, k, parts, chunk, def_buf + row_off, cidx_buf + row_off, ckey_buf + row_off,
-               counts + (long long)row * parts * 2, idx_out + (long long)row * k,
-               score_out ? score_out + (long long)row * k : nullptr, dsm);
+    const unsigned long long dc = __ldcg(rc);
+    finish_row(sc, nvis, k, (int)(dc & 0xffffffffu), (int)(dc >> 32), dout, ciout, ckout,
+               idx_out + (long long)row * k, score_out ? score_out + (long long)row * k : nullptr, dsm);
 }
 
 // Many query rows (prefill): one block (kFastThreads) per row.  Pass 1 builds the histogram of
@@ -815,12 +940,12 @@ struct TopkPlan {
     bool fast;
     int parts;
     long long chunk;
-    size_t off_hist, off_cnt, off_def, off_cidx, off_ckey, total;
+    size_t off_hist, off_def, off_cidx, off_ckey, total;
 };
 
 static size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
-static TopkPlan topk_plan(const IndexArgs& a) {
+static TopkPlan topk_plan(const IndexArgs& a, int k) {
     TopkPlan p = {};
     const long long rows = (long long)a.batch * a.n_q;
     const long long n = a.n_ent > 0 ? a.n_ent : 1;
@@ -830,22 +955,22 @@ static TopkPlan topk_plan(const IndexArgs& a) {
         p.total = off;
         return p;
     }
-    // parts of kFastStep scores (more per part only if a row would need more than kMaxParts)
+    if (k < 1) k = 1;
+    // parts of kFastStep scores (more per part only if a row would need more than kMaxFastParts)
     long long parts = (n + kFastStep - 1) / kFastStep;
-    if (parts > kMaxParts) parts = kMaxParts;
+    if (parts > kMaxFastParts) parts = kMaxFastParts;
     if (parts < 1) parts = 1;
     p.parts = (int)parts;
     p.chunk = ((n + parts - 1) / parts + kFastStep - 1) / kFastStep * kFastStep;
-    p.off_hist = off;  // histograms, then one finished-parts counter per row: zeroed together
-    off = align256(off + (size_t)rows * (kHistBins + 1) * sizeof(uint32_t));
-    p.off_cnt = off;
-    off = align256(off + (size_t)rows * p.parts * 2 * sizeof(int));
+    // histograms, then per row a 64-bit list counter and a finished-parts counter: zeroed together
+    p.off_hist = off;
+    off = align256(off + (size_t)rows * (kHistBins * sizeof(uint32_t) + 2 * sizeof(unsigned long long)));
     p.off_def = off;
-    off = align256(off + (size_t)rows * n * sizeof(int32_t));
+    off = align256(off + (size_t)rows * k * sizeof(int32_t));
     p.off_cidx = off;
-    off = align256(off + (size_t)rows * n * sizeof(int32_t));
+    off = align256(off + (size_t)rows * kSelCap * sizeof(int32_t));
     p.off_ckey = off;
-    off = align256(off + (size_t)rows * n * sizeof(uint32_t));
+    off = align256(off + (size_t)rows * kSelCap * sizeof(uint32_t));
     p.total = off;
     return p;
 }
@@ -872,15 +997,12 @@ cudaError_t launch_index_scores(const IndexArgs& a, float* scores, cudaStream_t 
     return launch_scores_h<64>(a, scores, stream);
 }
 
-size_t topk_workspace_bytes(const IndexArgs& a, int k) {
-    (void)k;
-    return topk_plan(a).total;
-}
+size_t topk_workspace_bytes(const IndexArgs& a, int k) { return topk_plan(a, k).total; }
 
 cudaError_t launch_topk(const IndexArgs& a, int k, int32_t* idx_out, float* score_out, void* ws, size_t ws_bytes,
                         cudaStream_t stream) {
     if (a.batch == 0) return cudaSuccess;
-    const TopkPlan p = topk_plan(a);
+    const TopkPlan p = topk_plan(a, k);
     if (ws_bytes < p.total) return cudaErrorInvalidValue;
     char* base = static_cast<char*>(ws);
     float* scores = reinterpret_cast<float*>(base);
@@ -898,12 +1020,11 @@ cudaError_t launch_topk(const IndexArgs& a, int k, int32_t* idx_out, float* scor
         return e != cudaSuccess ? e : cudaGetLastError();
     }
     uint32_t* hist = reinterpret_cast<uint32_t*>(base + p.off_hist);
-    int* counts = reinterpret_cast<int*>(base + p.off_cnt);
+    unsigned long long* ctr = reinterpret_cast<unsigned long long*>(hist + (size_t)rows * kHistBins);
     int32_t* def_buf = reinterpret_cast<int32_t*>(base + p.off_def);
     int32_t* cidx = reinterpret_cast<int32_t*>(base + p.off_cidx);
     uint32_t* ckey = reinterpret_cast<uint32_t*>(base + p.off_ckey);
-    unsigned int* row_done = hist + (size_t)rows * kHistBins;
-    e = launch_zero_words(hist, (long long)rows * (kHistBins + 1), stream);
+    e = launch_zero_words(hist, (long long)rows * (kHistBins + 4), stream);
     if (e != cudaSuccess) return e;
     if (index_tc_available(a)) {
         e = launch_index_scores_tc(a, scores, hist, a.dev_status, stream);
@@ -915,11 +1036,10 @@ cudaError_t launch_topk(const IndexArgs& a, int k, int32_t* idx_out, float* scor
         }
     }
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(topk_fast_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFastSmem);
+    e = cudaFuncSetAttribute(topk_fast_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSelSmem);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(topk_fast_kernel, dim3(rows * p.parts), dim3(kFastThreads), kFastSmem, stream, (const float*)scores,
-                   (const uint32_t*)hist, a, k, p.parts, p.chunk, def_buf, cidx, ckey, counts, row_done, idx_out,
-                   score_out);
+    e = launch_pdl(topk_fast_kernel, dim3(rows * p.parts), dim3(kFastThreads), kSelSmem, stream, (const float*)scores,
+                   (const uint32_t*)hist, a, k, p.parts, p.chunk, def_buf, cidx, ckey, ctr, idx_out, score_out);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

@@ -180,6 +180,32 @@ __device__ __forceinline__ void fetch_block_rows(const IdxTcArgs& a, int bat, lo
         if (j < nb) rows[j] = block_row(a, bat, e0 + (long long)j * a.epb);
 }
 
+// Lane 0 of warp 0, before the grid dependency wait: an L2 prefetch of this CTA's first `tiles` key
+// tiles of `rows` entries (boxes of the key tensor map, `xboxes` 64-column boxes across for bf16 keys)
+// and of their per-entry words (FP8 scales or MXFP4 exponents, `wbytes` bytes per entry), so that the
+// first loads' DRAM and address-translation latency overlaps the previous kernel's tail.  A prefetch
+// only warms L2, the point of coherence: a key the previous kernel is still writing (the newest entry)
+// is read afresh by the load after the wait.  Contiguous keys only.
+__device__ void prefetch_first_tiles(const IdxTcArgs& a, const CUtensorMap* kmap, long long f0, long long f1,
+                                     int rows, int boxes, int xboxes, int tiles, const void* words, int wbytes) {
+    ICursor cur(f0, a, 1);
+    for (int j = 0; j < tiles && f0 + j < f1; ++j, cur.next(a)) {
+        const long long e0 = (long long)cur.ti * rows;
+        const int y = (int)((long long)cur.bat * a.n_ent + e0);
+        for (int bx = 0; bx < boxes; ++bx)
+            for (int x = 0; x < xboxes; ++x) tc::tma_prefetch_2d(kmap, 64 * x, y + bx * (rows / boxes));
+        if (words && (reinterpret_cast<uintptr_t>(words) & 15) == 0) {
+            // the tile's words, trimmed to 16-byte boundaries (the bulk prefetch's alignment rule); the base
+            // being 16-byte aligned keeps the trimmed range inside the array
+            long long ne = a.n_ent - e0;
+            if (ne > rows) ne = rows;
+            const uintptr_t lo = reinterpret_cast<uintptr_t>(words) + ((long long)cur.bat * a.n_ent + e0) * wbytes;
+            const uintptr_t b0 = (lo + 15) & ~(uintptr_t)15, b1 = (lo + ne * wbytes) & ~(uintptr_t)15;
+            if (b1 > b0) tc::prefetch_l2(reinterpret_cast<const void*>(b0), (uint32_t)(b1 - b0));
+        }
+    }
+}
+
 template <bool FP8, int G>
 __device__ void idx_producer(IdxSmem& sm, const IdxTcArgs& a, const CUtensorMap* kmap, long long f0, long long f1) {
     constexpr int kSt = Ring<FP8>::kStages, kBytes = Ring<FP8>::kStageBytes;
@@ -551,7 +577,9 @@ __global__ void __launch_bounds__(kThreads, 1) index_score_tc_kernel(const __gri
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
-    griddep_wait();  // the prologue above touched only shared and tensor memory
+    if (threadIdx.x == 0 && !a.bt && G == 1)
+        prefetch_first_tiles(a, &kmap, f0, f1, kTileK, 1, FP8 ? 1 : 2, Ring<FP8>::kStages + 2, a.kscale, 4);
+    griddep_wait();  // the prologue above touched only shared and tensor memory (and prefetched into L2)
     griddep_launch_dependents();
     const uint32_t tmem = sm.tmem_base;
     if (warp == 0) {
@@ -906,7 +934,8 @@ __global__ void __launch_bounds__(kThreads, 1) index_score_mx_kernel(const __gri
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
-    griddep_wait();  // the prologue above touched only shared and tensor memory
+    if (threadIdx.x == 0 && !a.bt) prefetch_first_tiles(a, &kmap, f0, f1, kMxTile, 2, 1, kMxStages + 2, a.kexp, 4);
+    griddep_wait();  // the prologue above touched only shared and tensor memory (and prefetched into L2)
     griddep_launch_dependents();
     const uint32_t tmem = sm.tmem_base;
     if (warp == 0) {

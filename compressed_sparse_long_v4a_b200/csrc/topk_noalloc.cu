@@ -10,7 +10,8 @@
 //
 // The array lives in device global memory for as long as the library is
 // loaded on a device; its host-side name is only a stand-in, so its device
-// address is looked up once per device with cudaGetSymbolAddress and cached.
+// address is looked up once per device with cudaGetSymbolAddress and cached
+// (for the device's current context: a cudaDeviceReset makes it stale).
 #include <mutex>
 
 #include "common.cuh"
@@ -50,6 +51,11 @@ extern "C" v4a_status v4a_topk_noalloc(const void* q_i, const float* w, const vo
                                        int32_t* idx_out, float* score_out, int heads_i, int d_i, v4a_dtype q_dtype,
                                        v4a_dtype k_dtype, const v4a_shape* shape, void* stream) {
     if (!shape) return v4a::report(V4A_ERR_INVALID_ARG, "shape is NULL");
+    if (shape->batch < 0 || shape->n_q < 1 || shape->ctx_len < 0 || shape->m < 1 || shape->k < 1)
+        // not a shape v4a_topk takes, so no scratch size applies: v4a_topk's own checks say why (it
+        // rejects the shape before looking at the scratch, and launches nothing)
+        return v4a_topk(q_i, w, k_i, k_scale, idx_out, score_out, heads_i, d_i, q_dtype, k_dtype, nullptr, 0, shape,
+                        stream);
     const size_t need = v4a_workspace_size("topk", shape, heads_i, d_i);
     if (need > kScratchBytes)
         return v4a::report(V4A_ERR_INVALID_ARG,

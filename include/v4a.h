@@ -235,14 +235,18 @@ V4A_API v4a_status v4a_topk_mxfp4(const void* q_i, const float* w, const uint8_t
  * there is no workspace argument: the scratch is a fixed 64 MiB array
  * compiled into the library, which every device that loads the library keeps
  * in its global memory until the process exits.  It bounds the problem size:
- * a shape whose v4a_workspace_size("topk", ...) exceeds 64 MiB (about 16
- * bytes per score, so some 4 million scores per call; the 1M-context decode
- * of 4 sequences has 1,048,576) returns V4A_ERR_INVALID_ARG with both sizes
- * in v4a_last_error().
+ * a shape whose v4a_workspace_size("topk", ...) exceeds 64 MiB (4 bytes per
+ * score plus 16 KB per query row for the decode select, so some 16 million
+ * scores per call; the 1M-context decode of 4 sequences has 1,048,576)
+ * returns V4A_ERR_INVALID_ARG with both sizes in v4a_last_error().  A shape
+ * that v4a_topk itself rejects gets v4a_topk's error.
  * The first call made with a given device current looks up the array's
  * device address (cudaGetSymbolAddress) and caches it; make that first call
- * outside any stream capture.  The call itself allocates nothing: no
- * cudaMalloc, no cudaFree, no allocating library routine.
+ * outside any stream capture.  The cached address belongs to the device's
+ * current context: after cudaDeviceReset on that device, do not call
+ * v4a_topk_noalloc there again in the same process.  The call itself
+ * allocates nothing: no cudaMalloc, no cudaFree, no allocating library
+ * routine.
  * Every call on a device uses the same array, and the array keeps whatever
  * the previous call left in it (each call writes every scratch byte before
  * reading it).  Calls whose work may overlap on the GPU -- on different

@@ -67,11 +67,42 @@ def test_no_alloc_topk_refuses_shapes_beyond_its_scratch(v4a):
     k_i = torch.zeros((1, 1, 128), dtype=torch.uint8, device="cuda")
     k_s = torch.ones((1, 1), dtype=torch.float32, device="cuda")
     idx = torch.full((1, 1, 8), -7, dtype=torch.int32, device="cuda")
-    # a context whose top-k scratch needs more than the built-in 64 MiB
-    too_long = 4 * (8 << 20)
+    # a context whose top-k scratch needs more than the built-in 64 MiB (4 bytes per score)
+    too_long = 4 * (20 << 20)
     assert v4a.v4a_workspace_size("topk", batch=1, m=4, k=8, ctx_len=too_long, heads_i=16, d_i=128) > (64 << 20)
     with pytest.raises(v4a.V4AError) as e:
         v4a.v4a_topk_noalloc(q_i, w, k_i, k_s, idx, m=4, k=8, ctx_len=too_long)
     assert e.value.status == 1 and "v4a_topk_noalloc" in str(e.value) and str(64 << 20) in str(e.value)
     torch.cuda.synchronize()
     assert (idx == -7).all()  # nothing was launched
+
+
+def test_no_alloc_topk_many_rows_matches_workspace_topk(v4a):
+    # more query rows than the few-rows select takes (a prefill-like block of 512 queries): the per-row
+    # select path also works out of the built-in scratch, bit-equal to the workspace call
+    c = wl.index_case(1, 512, 4096, 4, 16, 128, "bf16", "bf16", seed=43)
+    c = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in c.items()}
+    k = 64
+    ref_idx = torch.empty((1, 512, k), dtype=torch.int32, device="cuda")
+    ref_sco = torch.empty((1, 512, k), dtype=torch.float32, device="cuda")
+    v4a.v4a_topk(c["q_i"], c["w"], c["k_i"], c["k_scale"], ref_idx, ref_sco, m=4, k=k, ctx_len=4096)
+    for _ in range(2):
+        idx = torch.full((1, 512, k), -7, dtype=torch.int32, device="cuda")
+        sco = torch.full((1, 512, k), 7.0, dtype=torch.float32, device="cuda")
+        v4a.v4a_topk_noalloc(c["q_i"], c["w"], c["k_i"], c["k_scale"], idx, sco, m=4, k=k, ctx_len=4096)
+        torch.cuda.synchronize()
+        assert torch.equal(idx, ref_idx)
+        assert torch.equal(sco, ref_sco)
+
+
+def test_no_alloc_topk_reports_bad_shapes_as_argument_errors(v4a):
+    q_i = torch.zeros((1, 1, 16, 128), dtype=torch.bfloat16, device="cuda")
+    w = torch.zeros((1, 1, 16), dtype=torch.float32, device="cuda")
+    k_i = torch.zeros((1, 1, 128), dtype=torch.uint8, device="cuda")
+    k_s = torch.ones((1, 1), dtype=torch.float32, device="cuda")
+    idx = torch.full((1, 1, 8), -7, dtype=torch.int32, device="cuda")
+    with pytest.raises(v4a.V4AError) as e:
+        v4a.v4a_topk_noalloc(q_i, w, k_i, k_s, idx, m=4, k=8, ctx_len=-5)
+    assert e.value.status == 1 and "scratch" not in str(e.value)
+    torch.cuda.synchronize()
+    assert (idx == -7).all()
