@@ -49,6 +49,8 @@ def parse():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=20.0, help="budget of the oracle sample")
+    p.add_argument("--clocks-out", default=None, help="where the nvidia-smi clock samples of the timed region go "
+                                                      "(default: a temporary directory)")
     p.add_argument("--profile-steps", action="store_true",
                    help="run the warm-up and K steps eagerly and exit (the command ncu captures are taken on)")
     p.add_argument("--profile-fp4", action="store_true",
@@ -102,10 +104,12 @@ class ClockSampler:
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, out_path: str | None = None):
+        import tempfile
+
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+        self.path = out_path or os.path.join(tempfile.mkdtemp(prefix="v4a_clocks_"), f"clocks_rank{gpu_index}.csv")
 
     def __enter__(self):
         try:
@@ -343,6 +347,47 @@ class Prefill:
         idx_f = 2.0 * nvis * c["heads_i"] * c["d_i"]
         att_f = 4.0 * self.T * c["heads"] * (self.k + self.W) * c["d"]
         return idx_f, att_f
+
+
+def measure_csa64k(flush: torch.Tensor, peak_gbs: float) -> dict:
+    """The 64K-context CSA decode (batch 8, bf16 keys and entries, top-512): the layer (compress of the
+    completing chunk, indexer + top-k, sparse attention) timed with L2 flushed before every call, since
+    its algorithmic bytes (38.8 MB) fit in L2."""
+    import compressed_sparse_long_v4a_b200 as v4a
+    import workload as wl
+
+    w = wl.csa_decode("csa_l64k")
+    c = w["cfg"]
+    dv = lambda t: None if t is None else t.cuda()
+    q, tok, ent, qi, ww, ki = (dv(w[k]) for k in ("q", "token_kv", "entries", "q_i", "w", "k_i"))
+    gate, xi, gi = dv(w["gate_tail"]), dv(w["xi_tail"]), dv(w["gate_i_tail"])
+    B, L, m, k = c["batch"], c["ctx_len"], c["m"], c["k"]
+    N = L // m
+    idx = torch.empty((B, 1, k), dtype=torch.int32, device="cuda")
+    out = torch.empty((B, 1, c["heads"], c["d"]), dtype=torch.float32, device="cuda")
+    st = torch.zeros((1,), dtype=torch.int32, device="cuda")
+    ws = lambda n: torch.empty(max(n, 256), dtype=torch.uint8, device="cuda")
+    ws_k = ws(v4a.v4a_workspace_size("topk", batch=B, m=m, k=k, ctx_len=L, heads_i=c["heads_i"], d_i=c["d_i"]))
+    ws_a = ws(v4a.v4a_workspace_size("csa_attend", batch=B, heads=c["heads"], d=c["d"], m=m, k=k,
+                                     window=c["window"], ctx_len=L))
+    lt = tok.shape[1]
+
+    def layer():
+        v4a.v4a_compress(tok[:, lt - m:], gate, ent[:, N - 1:], m=m, xi=xi, gate_i=gi, out_i=ki[:, N - 1:])
+        v4a.v4a_topk(qi, ww, ki, None, idx, m=m, k=k, ctx_len=L, workspace=ws_k)
+        v4a.v4a_csa_attend(q, ent, idx, tok, w["tok_pos0"], out, m=m, window=c["window"], ctx_len=L, workspace=ws_a,
+                           dev_status=st)
+
+    layer()
+    torch.cuda.synchronize()
+    ms = statistics.median(time_op(layer, 20, flush) for _ in range(5))
+    nbytes = B * N * c["d_i"] * 2 + B * (k + c["window"]) * c["d"] * 2
+    return {"workload": "CSA decode, batch 8, 65,536-token context, bf16 keys and entries, indexer 16 x 128, "
+                        "top-512, 64 heads x 512, window 128",
+            "config": "csa_l64k", "ms": ms, "tokens_per_s": B / (ms / 1000.0), "algorithmic_bytes": nbytes,
+            "hbm_gbs": nbytes / (ms / 1000.0) / 1e9, "frac_measured_peak": nbytes / (ms / 1000.0) / 1e9 / peak_gbs,
+            "l2": "flushed before every call (the 38.8 MB working set fits in L2)",
+            "how": "median of 5 CUDA graphs of 20 x (L2 flush + layer) minus 20 x flush"}
 
 
 def measure_prefill(peaks: dict) -> dict:
@@ -625,57 +670,65 @@ def source_digest(paths) -> str:
 # CPU oracle (the reference arm and the cpu_baseline object)
 # ----------------------------------------------------------------------
 
-def oracle_sample(budget_s: float, step: "Step | None" = None):
-    """Time the CPU oracle on a bounded sample of the same workload: all 4 CSA
-    sequences (indexer + top-k + attention) and as many HCA sequences as fit the
-    budget.  Returns (tokens/s for the workload's 4:32 mix, threads, sample text)."""
-    import numpy as np
-
+def reference_step_fn():
+    """One reference step: the oracle (fp64 C, all host threads) on a bounded sample of the decode step's
+    work, one CSA sequence (indexer + top-k + attention) and eight HCA sequences, the workload's 4:32
+    mix in miniature; successive steps take successive sequences.  Returns (fn, tokens per step)."""
     import oracle
     import workload as wl
 
-    if step is not None:
-        cw, hw = step.cw_host, step.hw_host
-    else:
-        cw = wl.csa_decode("csa_l1m_fp8", with_tail=False)
-        hw = wl.hca_decode("hca_l1m", with_tail=False)
+    cw = wl.csa_decode("csa_l1m_fp8", with_tail=False)
+    hw = wl.hca_decode("hca_l1m", with_tail=False)
     c, h = cw["cfg"], hw["cfg"]
     h_ = wl.stored_numpy
-    t0 = time.perf_counter()
-    top = oracle.topk(h_(cw["q_i"]), h_(cw["w"]), h_(cw["k_i"]), h_(cw["k_scale"]), c["ctx_len"], c["m"], c["k"])
-    oracle.attend(h_(cw["q"]), h_(cw["entries"]), top["idx"], h_(cw["token_kv"]), cw["tok_pos0"], c["ctx_len"],
-                  c["m"], c["window"])
-    t_csa = (time.perf_counter() - t0) / c["batch"]
-    n_h = 0
-    t1 = time.perf_counter()
-    per = max(1, oracle.get_threads() // 8)
-    while n_h < h["batch"]:
-        bs = list(range(n_h, min(h["batch"], n_h + per)))
-        oracle.attend(h_(hw["q"][bs]), h_(hw["entries"][bs]), None, h_(hw["token_kv"][bs]), hw["tok_pos0"],
+    per = h["batch"] // c["batch"]  # HCA sequences per CSA sequence
+    state = {"i": 0}
+
+    def step():
+        b = state["i"] % c["batch"]
+        state["i"] += 1
+        top = oracle.topk(h_(cw["q_i"][b:b + 1]), h_(cw["w"][b:b + 1]), h_(cw["k_i"][b:b + 1]),
+                          h_(cw["k_scale"][b:b + 1]), c["ctx_len"], c["m"], c["k"])
+        oracle.attend(h_(cw["q"][b:b + 1]), h_(cw["entries"][b:b + 1]), top["idx"], h_(cw["token_kv"][b:b + 1]),
+                      cw["tok_pos0"], c["ctx_len"], c["m"], c["window"])
+        hs = list(range(b * per, (b + 1) * per))
+        oracle.attend(h_(hw["q"][hs]), h_(hw["entries"][hs]), None, h_(hw["token_kv"][hs]), hw["tok_pos0"],
                       h["ctx_len"], h["m"], h["window"])
-        n_h += len(bs)
-        if time.perf_counter() - t1 > budget_s:
-            break
-    t_hca = (time.perf_counter() - t1) / n_h
-    step_s = c["batch"] * t_csa + h["batch"] * t_hca
-    value = (c["batch"] + h["batch"]) / step_s
-    sample = (f"oracle (fp64 C, {oracle.get_threads()} threads) on all {c['batch']} CSA sequences "
-              f"(indexer+top-k+attention) and {n_h} of {h['batch']} HCA sequences; per-sequence times "
-              f"{t_csa:.3f} s (CSA) / {t_hca:.3f} s (HCA) combined in the step's 4:32 mix")
-    return value, oracle.get_threads(), sample, dict(csa_s_per_seq=t_csa, hca_s_per_seq=t_hca, hca_seqs=n_h)
+
+    return step, 1 + per
 
 
 def run_reference(args, world, rank):
+    """The reference arm: the oracle timed on the host cores, rank 0 only.  Each step is one bounded
+    sample (reference_step_fn); at most as many steps run as fit --cpu-seconds, and the line reports the
+    steps and the time per step that were actually measured."""
     if rank != 0:
         return
-    import numpy as np  # noqa: F401
+    import oracle
 
-    value, threads, sample, detail = oracle_sample(args.cpu_seconds)
-    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": 1000.0 * 36 / value, "higher_is_better": True,
+    step, tokens = reference_step_fn()
+    warm = min(args.warmup, 1)
+    for _ in range(warm):
+        step()
+    n, t_total = 0, 0.0
+    while n < args.steps:
+        t0 = time.perf_counter()
+        step()
+        t_total += time.perf_counter() - t0
+        n += 1
+        if t_total > args.cpu_seconds:
+            break
+    value = tokens * n / t_total
+    threads = oracle.get_threads()
+    sample = (f"oracle (fp64 C, {threads} threads): {n} steps, each one CSA sequence (indexer + top-k + "
+              f"attention at 1M context) and {tokens - 1} HCA sequences (dense attention at 1M context), "
+              f"{tokens} sequence-layer decodes per step")
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": n,
+            "warmup": warm, "ms_per_step": 1000.0 * t_total / n, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "impl": "reference",
-            "config": {"workload": WORKLOAD, "parallelism": "replicas", "sample": sample},
+            "config": {"workload": WORKLOAD, "parallelism": "replicas", "sample": sample,
+                       "steps_requested": args.steps, "warmup_requested": args.warmup},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -720,7 +773,7 @@ def main():
     # timed region: K graph replays, inputs (416 MB streamed per step) larger than L2
     barrier(world)
     torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
+    with ClockSampler(local, args.clocks_out) as clk:
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(s)
         for _ in range(args.steps):
@@ -829,13 +882,25 @@ def main():
     prefill = None
     fp4 = None
     paged = None
+    csa64k = None
     if rank == 0 and world == 1:
+        csa64k = measure_csa64k(flush, peak)
         fp4 = measure_fp4_indexer(step, flush, peak)
         paged = measure_paged(step, {"csa": layers["csa"]["ms_median"], "hca": layers["hca"]["ms_median"]})
         prefill = measure_prefill(peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, threads, sample, _ = oracle_sample(args.cpu_seconds, step)
-        cpu = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample}
+        import oracle
+
+        ref_step, tokens = reference_step_fn()
+        n, t_total = 0, 0.0
+        while t_total < args.cpu_seconds and n < 64:
+            t0 = time.perf_counter()
+            ref_step()
+            t_total += time.perf_counter() - t0
+            n += 1
+        cpu = {"value": tokens * n / t_total, "unit": UNIT, "cores": oracle.get_threads(), "kind": "oracle",
+               "sample": f"{n} reference steps of {tokens} sequence-layer decodes (one CSA sequence, "
+                         f"{tokens - 1} HCA sequences, 1M context), {t_total:.1f} s"}
 
     clocks = clk.summary()
     if rank == 0:
@@ -850,7 +915,8 @@ def main():
                            "step_hbm_gbs": total_bytes / (ms / 1000.0) / 1e9 / world,
                            "op_ms": op_ms,
                            "layers": layers},
-                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "prefill": prefill, "fp4_indexer": fp4,
+                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "csa_l64k": csa64k, "prefill": prefill,
+                "fp4_indexer": fp4,
                 "paged_cache": paged,
                 "gpu_launches": (launches_per_step * args.steps) if launches_per_step else None,
                 "gpu_launches_per_step": launches_per_step,

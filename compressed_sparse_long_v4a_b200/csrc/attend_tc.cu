@@ -171,7 +171,7 @@ __device__ __forceinline__ void csa_rows(const TcArgs& a, const RowInfo& ri, int
 // cp.async all 64 rows of a tile (lane owns rows lane and lane+32: src / ok) into the 128-byte-swizzled
 // stage; returns the tile's row mask
 __device__ __forceinline__ uint64_t gather_tile(uint8_t* dst, const __nv_bfloat16* const (&src)[2], const bool (&ok)[2],
-                                                int lane) {
+                                                int lane, uint64_t policy) {
     const uint64_t mask =
         (uint64_t)__ballot_sync(0xffffffffu, ok[0]) | ((uint64_t)__ballot_sync(0xffffffffu, ok[1]) << 32);
     for (int r = 0; r < kTile; ++r) {
@@ -181,7 +181,7 @@ __device__ __forceinline__ uint64_t gather_tile(uint8_t* dst, const __nv_bfloat1
         for (int h2 = 0; h2 < 2; ++h2) {
             const int u = lane + 32 * h2;  // 16-byte chunk of the 1 KB row
             uint8_t* d = dst + (u >> 3) * kSlabBytes + r * 128 + (((u & 7) ^ (r & 7)) << 4);
-            tc::cp_async_16(d, rs + u * 8);
+            tc::cp_async_16_hint(d, rs + u * 8, policy);
         }
     }
     return mask;
@@ -253,6 +253,7 @@ __device__ void producer(Smem& sm, const TcArgs& a, const CUtensorMap* ent_map, 
     const int lane = threadIdx.x & 31;
     int seg = 0;
     Cursor cur(f0, a.tpr);
+    const uint64_t stream_policy = tc::l2_evict_first();  // candidate rows are read once per call
     // the rows of gathered tiles are worked out a tile ahead, so their index / block-table loads overlap
     // the current tile's copies
     const __nv_bfloat16* nsrc[2] = {a.q, a.q};
@@ -284,7 +285,7 @@ __device__ void producer(Smem& sm, const TcArgs& a, const CUtensorMap* ent_map, 
         uint64_t mask = 0;
         uint8_t* dst = sm.kv[st];
         if (gath) {
-            mask = gather_tile(dst, src, ok, lane);
+            mask = gather_tile(dst, src, ok, lane, stream_policy);
             if (lane == 0) {
                 sm.mask[st] = mask;
                 tc::mbar_arrive_expect_tx(&sm.kv_full[st], 0);
@@ -298,7 +299,8 @@ __device__ void producer(Smem& sm, const TcArgs& a, const CUtensorMap* ent_map, 
                 sm.mask[st] = mask;
                 tc::mbar_arrive_expect_tx(&sm.kv_full[st], kTileBytes);
                 const int y = (int)((long long)ri.b * a.n_ent + c0);
-                for (int c = 0; c < kSlabs; ++c) tc::tma_load_2d(dst + c * kSlabBytes, ent_map, 64 * c, y, &sm.kv_full[st]);
+                for (int c = 0; c < kSlabs; ++c)
+                    tc::tma_load_2d_hint(dst + c * kSlabBytes, ent_map, 64 * c, y, &sm.kv_full[st], stream_policy);
             }
         } else {
             // window tokens p0 .. p0+63 (contiguous rows of token_kv)
@@ -312,7 +314,8 @@ __device__ void producer(Smem& sm, const TcArgs& a, const CUtensorMap* ent_map, 
                 sm.mask[st] = mask;
                 tc::mbar_arrive_expect_tx(&sm.kv_full[st], kTileBytes);
                 const int y = (int)((long long)ri.b * a.l_tok + (p0 - a.tok_pos0));
-                for (int c = 0; c < kSlabs; ++c) tc::tma_load_2d(dst + c * kSlabBytes, tok_map, 64 * c, y, &sm.kv_full[st]);
+                for (int c = 0; c < kSlabs; ++c)
+                    tc::tma_load_2d_hint(dst + c * kSlabBytes, tok_map, 64 * c, y, &sm.kv_full[st], stream_policy);
             }
         }
         tc::cp_async_arrive_noinc(&sm.kv_full[st]);  // 32 lanes: after their cp.async copies (if any) land

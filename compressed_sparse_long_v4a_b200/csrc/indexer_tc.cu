@@ -214,6 +214,7 @@ __device__ void idx_producer(IdxSmem& sm, const IdxTcArgs& a, const CUtensorMap*
     const long long n = f1 - f0;
     const int nb = a.bt ? kTileK / a.epb : 0;
     int rows[kMaxB], next_rows[kMaxB];
+    const uint64_t pol = tc::l2_evict_first();  // key tiles are read once per call
     if (a.bt && n > 0) fetch_block_rows<kMaxB>(a, cur.bat, (long long)cur.ti * kTileK, nb, next_rows);
     for (long long jt = 0; jt < n; ++jt, cur.next(a)) {
         if (a.bt) {
@@ -236,12 +237,12 @@ __device__ void idx_producer(IdxSmem& sm, const IdxTcArgs& a, const CUtensorMap*
 #pragma unroll
             for (int j = 0; j < kMaxB; ++j) {
                 if (j >= nb) break;
-                tc::tma_load_2d(dst + j * a.epb * 128, kmap, 0, rows[j], &sm.k_full[st]);
-                if (!FP8) tc::tma_load_2d(dst + kTileK * 128 + j * a.epb * 128, kmap, 64, rows[j], &sm.k_full[st]);
+                tc::tma_load_2d_hint(dst + j * a.epb * 128, kmap, 0, rows[j], &sm.k_full[st], pol);
+                if (!FP8) tc::tma_load_2d_hint(dst + kTileK * 128 + j * a.epb * 128, kmap, 64, rows[j], &sm.k_full[st], pol);
             }
         } else {
-            tc::tma_load_2d(dst, kmap, 0, y, &sm.k_full[st]);
-            if (!FP8) tc::tma_load_2d(dst + kTileK * 128, kmap, 64, y, &sm.k_full[st]);  // second 64-column slab
+            tc::tma_load_2d_hint(dst, kmap, 0, y, &sm.k_full[st], pol);
+            if (!FP8) tc::tma_load_2d_hint(dst + kTileK * 128, kmap, 64, y, &sm.k_full[st], pol);  // second 64-column slab
         }
     }
     // no copy may still be in flight when the CTA exits
@@ -638,6 +639,7 @@ __device__ void mx_producer(IdxSmem& sm, const IdxTcArgs& a, const CUtensorMap* 
     const long long n = f1 - f0;
     const int nb = a.bt ? kMxTile / a.epb : 0;
     int rows[kMaxB], next_rows[kMaxB];
+    const uint64_t pol = tc::l2_evict_first();  // key tiles are read once per call
     if (a.bt && n > 0) fetch_block_rows<kMaxB>(a, cur.bat, (long long)cur.ti * kMxTile, nb, next_rows);
     for (long long jt = 0; jt < n; ++jt, cur.next(a)) {
         if (a.bt) {
@@ -662,12 +664,12 @@ __device__ void mx_producer(IdxSmem& sm, const IdxTcArgs& a, const CUtensorMap* 
 #pragma unroll
             for (int j = 0; j < kMaxB; ++j) {
                 if (j >= nb) break;
-                tc::tma_load_2d(sm.ring + st * kMxStageBytes + j * a.epb * 64, kmap, 0, rows[j], &sm.k_full[st]);
+                tc::tma_load_2d_hint(sm.ring + st * kMxStageBytes + j * a.epb * 64, kmap, 0, rows[j], &sm.k_full[st], pol);
             }
         } else {
             // boxes of 256 rows; rows past the tensor's end are filled with zeros (and still counted)
-            tc::tma_load_2d(sm.ring + st * kMxStageBytes, kmap, 0, y, &sm.k_full[st]);
-            tc::tma_load_2d(sm.ring + st * kMxStageBytes + kMxStageBytes / 2, kmap, 0, y + 256, &sm.k_full[st]);
+            tc::tma_load_2d_hint(sm.ring + st * kMxStageBytes, kmap, 0, y, &sm.k_full[st], pol);
+            tc::tma_load_2d_hint(sm.ring + st * kMxStageBytes + kMxStageBytes / 2, kmap, 0, y + 256, &sm.k_full[st], pol);
         }
     }
     // no copy may still be in flight when the CTA exits
