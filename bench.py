@@ -53,6 +53,9 @@ def parse():
                                                       "(default: a temporary directory)")
     p.add_argument("--profile-steps", action="store_true",
                    help="run the warm-up and K steps eagerly and exit (the command ncu captures are taken on)")
+    p.add_argument("--profile-prefill", action="store_true",
+                   help="run the prefill chunk (compress, scores + top-k, attention) warm-up + K times eagerly and exit "
+                        "(the command ncu captures of the prefill kernels are taken on)")
     p.add_argument("--profile-fp4", action="store_true",
                    help="run the MXFP4 indexer (scores and top-k of the 1M-context CSA keys) warm-up + K times "
                         "eagerly and exit (the command ncu captures of the FP4 kernels are taken on)")
@@ -746,6 +749,12 @@ def main():
         return
     assert torch.cuda.is_available(), "bench.py needs a CUDA device"
     args.warmup = max(3, args.warmup)
+    if args.profile_prefill:
+        pf = Prefill()
+        for _ in range(args.warmup + args.steps):
+            pf.step()
+        torch.cuda.synchronize()
+        return
     step = Step(seed_offset=rank)
     s = torch.cuda.current_stream()
     if args.profile_fp4:

@@ -39,8 +39,10 @@ namespace {
 
 constexpr int kD = 512;
 constexpr int kH = 64;
-constexpr int kTile = 64;                        // candidate rows per tile
-constexpr int kStages = 2;                       // tiles resident in shared memory
+constexpr int kTile = 48;                        // candidate rows per tile
+constexpr int kStages = 3;                       // tiles resident in shared memory
+constexpr uint64_t kTileMask = (1ull << kTile) - 1;
+constexpr uint32_t kSCols = 64;                  // TMEM columns between the two S buffers
 constexpr int kSlabs = kD / 64;                  // 64-element (128 B) column slabs
 constexpr uint32_t kSlabBytes = kTile * 128;     // 8 KB
 constexpr uint32_t kTileBytes = kSlabs * kSlabBytes;
@@ -95,6 +97,12 @@ struct TcArgs {
     long long n_blocks;
     int ring_rows;      // > 0: window rows come from a ring [B][ring_rows][512] (position p in row p % ring_rows)
     int comb_pieces;    // bound on the pieces of one query (attend_tc_combine's shared memory)
+    // bounded-wait limits (polls of an mbarrier; cycles without progress for the MMA warp) and the
+    // fault-injection switch of the test hook (v4a_test_attend_fault): a CTA withholds its tile
+    // `withhold` (local index; -1: never), issuing no copy and no arrival for it
+    uint32_t wait_polls;
+    long long stall_cycles;
+    int withhold;
 };
 
 // tiles whose rows the producer gathers with cp.async (CSA selections, paged entries, ring windows)
@@ -156,7 +164,7 @@ __device__ __forceinline__ void csa_rows(const TcArgs& a, const RowInfo& ri, int
 #pragma unroll
     for (int h2 = 0; h2 < 2; ++h2) {
         const long long c = c0 + lane + 32 * h2;
-        const long long sidx = c < a.k ? (long long)a.idx[(long long)row * a.k + c] : -1;
+        const long long sidx = (c < a.k && lane + 32 * h2 < kTile) ? (long long)a.idx[(long long)row * a.k + c] : -1;
         ok[h2] = sidx >= 0 && sidx < ri.nvis;
         const __nv_bfloat16* er = ok[h2] ? entry_row(a, ri.b, sidx) : nullptr;
         if (ok[h2] && !er) {  // a block id outside the pool: skipped and reported
@@ -201,7 +209,7 @@ __device__ __forceinline__ bool tile_rows(const TcArgs& a, int row, int ti, int 
 #pragma unroll
             for (int h2 = 0; h2 < 2; ++h2) {
                 const long long c = c0 + lane + 32 * h2;
-                const long long sidx = c < a.k ? (long long)a.idx[(long long)row * a.k + c] : -1;
+                const long long sidx = (c < a.k && lane + 32 * h2 < kTile) ? (long long)a.idx[(long long)row * a.k + c] : -1;
                 if (!ok[h2] && sidx != -1 && a.dev_status) atomicExch(a.dev_status, (int)V4A_ERR_DEVICE_FAULT);
             }
         } else {
@@ -209,7 +217,7 @@ __device__ __forceinline__ bool tile_rows(const TcArgs& a, int row, int ti, int 
 #pragma unroll
             for (int h2 = 0; h2 < 2; ++h2) {
                 const long long s = c0 + lane + 32 * h2;
-                const __nv_bfloat16* er = s < ri.nvis ? entry_row(a, ri.b, s) : nullptr;
+                const __nv_bfloat16* er = (s < ri.nvis && lane + 32 * h2 < kTile) ? entry_row(a, ri.b, s) : nullptr;
                 if (s < ri.nvis && !er && a.dev_status) atomicExch(a.dev_status, (int)V4A_ERR_DEVICE_FAULT);
                 ok[h2] = er != nullptr;
                 src[h2] = ok[h2] ? er : fallback;
@@ -223,7 +231,7 @@ __device__ __forceinline__ bool tile_rows(const TcArgs& a, int row, int ti, int 
         for (int h2 = 0; h2 < 2; ++h2) {
             const int r = lane + 32 * h2;
             const long long p = p0 + r;
-            ok[h2] = wi * kTile + r < a.window && p >= 0;
+            ok[h2] = r < kTile && wi * kTile + r < a.window && p >= 0;
             src[h2] = ok[h2] ? a.token_kv + ((long long)ri.b * a.ring_rows + p % a.ring_rows) * kD : fallback;
         }
     }
@@ -254,6 +262,8 @@ __device__ void producer(Smem& sm, const TcArgs& a, const CUtensorMap* ent_map, 
     int seg = 0;
     Cursor cur(f0, a.tpr);
     const uint64_t stream_policy = tc::l2_evict_first();  // candidate rows are read once per call
+    int last_load[kStages];  // the last tile whose copies went into each stage (-1: none)
+    for (int i = 0; i < kStages; ++i) last_load[i] = -1;
     // the rows of gathered tiles are worked out a tile ahead, so their index / block-table loads overlap
     // the current tile's copies
     const __nv_bfloat16* nsrc[2] = {a.q, a.q};
@@ -274,16 +284,18 @@ __device__ void producer(Smem& sm, const TcArgs& a, const CUtensorMap* ent_map, 
             ngath = tile_rows(a, nx.row, nx.ti, lane, nsrc, nok);
         }
         if (seg_start) {
-            if (seg > 0 && !tc::mbar_wait(&sm.q_empty, (seg - 1) & 1)) { fault(sm, a); break; }
+            if (seg > 0 && !tc::mbar_wait(&sm.q_empty, (seg - 1) & 1, a.wait_polls)) { fault(sm, a); break; }
             if (lane == 0 && seg > 0) {  // the first segment's query was requested before the dependency wait
                 tc::mbar_arrive_expect_tx(&sm.q_full, kQBytes);
                 for (int c = 0; c < kSlabs; ++c) tc::tma_load_2d(sm.q + c * kH * 128, q_map, 64 * c, row * kH, &sm.q_full);
             }
             ++seg;
         }
-        if (jt >= kStages && !tc::mbar_wait(&sm.kv_empty[st], ((jt / kStages) - 1) & 1)) { fault(sm, a); break; }
+        if (jt >= kStages && !tc::mbar_wait(&sm.kv_empty[st], ((jt / kStages) - 1) & 1, a.wait_polls)) { fault(sm, a); break; }
         uint64_t mask = 0;
         uint8_t* dst = sm.kv[st];
+        if (jt == a.withhold) continue;  // test hook: this stage never fills (no copy, no arrival)
+        last_load[st] = jt;
         if (gath) {
             mask = gather_tile(dst, src, ok, lane, stream_policy);
             if (lane == 0) {
@@ -294,7 +306,7 @@ __device__ void producer(Smem& sm, const TcArgs& a, const CUtensorMap* ent_map, 
             // HCA: rows c0 .. c0+63 of this sequence's entries are contiguous
             const long long c0 = (long long)ti * kTile;
             const long long nv = ri.nvis - c0;
-            mask = nv >= kTile ? ~0ull : (nv <= 0 ? 0ull : ((1ull << nv) - 1ull));
+            mask = nv >= kTile ? kTileMask : (nv <= 0 ? 0ull : ((1ull << nv) - 1ull));
             if (lane == 0) {
                 sm.mask[st] = mask;
                 tc::mbar_arrive_expect_tx(&sm.kv_full[st], kTileBytes);
@@ -320,15 +332,13 @@ __device__ void producer(Smem& sm, const TcArgs& a, const CUtensorMap* ent_map, 
         }
         tc::cp_async_arrive_noinc(&sm.kv_full[st]);  // 32 lanes: after their cp.async copies (if any) land
     }
-    // make sure nothing this warp started is still in flight before the CTA retires
-    const long long n = f1 - f0;
-    for (long long jt = n - kStages; jt < n; ++jt) {
-        if (jt < 0) continue;
-        tc::mbar_wait(&sm.kv_full[jt % kStages], (jt / kStages) & 1);
-    }
+    // make sure nothing this warp started is still in flight before the CTA retires (also after an abort
+    // or a withheld stage: the last copies issued into each stage)
+    for (int st = 0; st < kStages; ++st)
+        if (last_load[st] >= 0) tc::mbar_wait(&sm.kv_full[st], (last_load[st] / kStages) & 1, a.wait_polls);
     // ... nor a query load (the first segment's was issued before the loop)
     const int q_loads = seg > 0 ? seg : (f0 < f1 ? 1 : 0);
-    if (q_loads > 0) tc::mbar_wait(&sm.q_full, (q_loads - 1) & 1);
+    if (q_loads > 0) tc::mbar_wait(&sm.q_full, (q_loads - 1) & 1, a.wait_polls);
 }
 
 // ---------------------------------------------------------------------
@@ -361,7 +371,7 @@ __device__ void issue_qk(Smem& sm, uint32_t tmem, int jq, bool gathered, uint64_
     if (gathered) tc::fence_proxy_async();  // rows gathered with cp.async become visible to the tensor core
     tc::tc_fence_after();
     const uint64_t k0 = tc::sw128_desc(tc::smem_u32(sm.kv[st]), 16, 1024);
-    const uint32_t d_s = tmem + kColS + kTile * s;
+    const uint32_t d_s = tmem + kColS + kSCols * s;
 #pragma unroll
     for (int c = 0; c < kSlabs; ++c) {
 #pragma unroll
@@ -410,7 +420,7 @@ __device__ void mma_issuer(Smem& sm, const TcArgs& a, uint32_t tmem, long long f
         }
         if (progressed) {
             t_last = clock64();
-        } else if (__shfl_sync(0xffffffffu, (int)(clock64() - t_last > kStallCycles), 0)) {
+        } else if (__shfl_sync(0xffffffffu, (int)(clock64() - t_last > a.stall_cycles), 0)) {
             ok = false;
             break;
         }
@@ -446,21 +456,23 @@ __device__ void softmax_warps(Smem& sm, const TcArgs& a, uint32_t tmem, long lon
             m_run = -INFINITY;
             l_run = 0.f;
         }
-        if (!tc::mbar_wait(&sm.kv_full[st], (jt / kStages) & 1)) { ok = false; break; }
-        const uint32_t mask = (uint32_t)(sm.mask[st] >> (32 * half));
-        if (!tc::mbar_wait(&sm.s_full[s], (jt >> 1) & 1)) { ok = false; break; }
+        if (!tc::mbar_wait(&sm.kv_full[st], (jt / kStages) & 1, a.wait_polls)) { ok = false; break; }
+        const uint64_t tmask = sm.mask[st];
+        const uint32_t mask = (uint32_t)((tmask >> (16 * half)) & 0xffffu) | ((uint32_t)((tmask >> (32 + 8 * half)) & 0xffu) << 16);
+        if (!tc::mbar_wait(&sm.s_full[s], (jt >> 1) & 1, a.wait_polls)) { ok = false; break; }
         tc::tc_fence_after();
-        uint32_t r[32];
-        tc::tmem_ld_16x32bx2_x32(tmem + lane_addr + kColS + kTile * s, r);
+        uint32_t r[24];
+        tc::tmem_ld_16x32bx2_x16(tmem + lane_addr + kColS + kSCols * s, r);
+        tc::tmem_ld_16x32bx2_x8(tmem + lane_addr + kColS + kSCols * s + 32, r + 16);
         tc::tmem_ld_wait();
         float alpha = 1.f;
         bool rescale = false;
-        uint32_t pk[16];  // bf16 pairs of this thread's 32 probabilities
+        uint32_t pk[12];  // bf16 pairs of this thread's 24 probabilities
         {
             // independent partial maxima / sums keep the dependent chains short
             float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
+            for (int i = 0; i < 24; ++i) {
                 const float x = ((mask >> i) & 1) ? __uint_as_float(r[i]) * a.scale_log2 : -INFINITY;
                 r[i] = __float_as_uint(x);
                 mx4[i & 3] = fmaxf(mx4[i & 3], x);
@@ -478,7 +490,7 @@ __device__ void softmax_warps(Smem& sm, const TcArgs& a, uint32_t tmem, long lon
             const float msub = m_run == -INFINITY ? 0.f : m_run;  // all-masked so far: every x is -inf
             float ls4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
+            for (int i = 0; i < 12; ++i) {
                 const float p0 = exp2f(__uint_as_float(r[2 * i]) - msub);
                 const float p1 = exp2f(__uint_as_float(r[2 * i + 1]) - msub);
                 const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
@@ -492,11 +504,11 @@ __device__ void softmax_warps(Smem& sm, const TcArgs& a, uint32_t tmem, long lon
             }
         }
         // the P buffer of this parity is free once PV two tiles back is done
-        if (jt >= 2 && !tc::mbar_wait(&sm.p_free[s], ((jt >> 1) - 1) & 1)) { ok = false; break; }
+        if (jt >= 2 && !tc::mbar_wait(&sm.p_free[s], ((jt >> 1) - 1) & 1, a.wait_polls)) { ok = false; break; }
         tc::named_barrier(1, 128);
         if (sm.rescale_tag[s] == jt + 1) {
             // O^T (lanes = d, columns = heads) was accumulated with the old maxima
-            if (!tc::mbar_wait(&sm.p_free[(jt - 1) & 1], ((jt - 1) >> 1) & 1)) { ok = false; break; }
+            if (!tc::mbar_wait(&sm.p_free[(jt - 1) & 1], ((jt - 1) >> 1) & 1, a.wait_polls)) { ok = false; break; }
             tc::tc_fence_after();
 #pragma unroll 1
             for (int cc = 0; cc < 4; ++cc) {
@@ -514,16 +526,18 @@ __device__ void softmax_warps(Smem& sm, const TcArgs& a, uint32_t tmem, long lon
             // writes the 4 16-byte chunks of its half
             uint8_t* prow = sm.p[s] + (h >> 3) * 1024 + (h & 7) * 128;
 #pragma unroll
-            for (int u = 0; u < 4; ++u)
-                *reinterpret_cast<uint4*>(prow + (((4 * half + u) ^ (h & 7)) << 4)) =
+            for (int u = 0; u < 3; ++u) {
+                const int chunk = u < 2 ? 2 * half + u : 4 + half;  // rows 8 chunk .. 8 chunk + 7
+                *reinterpret_cast<uint4*>(prow + ((chunk ^ (h & 7)) << 4)) =
                     make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+            }
         }
         tc::fence_proxy_async();
         tc::tc_fence_before();
         tc::mbar_arrive(&sm.p_full[s]);
 
         if (seg_end) {
-            if (!tc::mbar_wait(&sm.p_free[s], (jt >> 1) & 1)) { ok = false; break; }
+            if (!tc::mbar_wait(&sm.p_free[s], (jt >> 1) & 1, a.wait_polls)) { ok = false; break; }
             tc::tc_fence_after();
             const float l_row = l_run + __shfl_xor_sync(0xffffffffu, l_run, 16);
             const long long rs = (long long)row * a.tpr;
@@ -807,6 +821,8 @@ TcPlan tc_plan(const AttendArgs& a) {
 
 }  // namespace
 
+AttendFaultTest g_test_fault = {-1, 0, 0};
+
 bool attend_tc_shape_ok(const AttendArgs& a) {
     if (a.dtype != V4A_BF16 || a.d != kD || a.heads != kH) return false;
     TcPlan p = tc_plan(a);
@@ -870,6 +886,9 @@ cudaError_t launch_attend_tc(const AttendArgs& a, void* ws, size_t ws_bytes, cud
     t.sink = a.sink;
     t.rope_dims = a.rope_dims;
     t.rope_base = a.rope_base;
+    t.wait_polls = g_test_fault.withhold >= 0 ? g_test_fault.wait_polls : tc::kWaitPolls;
+    t.stall_cycles = g_test_fault.withhold >= 0 ? g_test_fault.stall_cycles : kStallCycles;
+    t.withhold = g_test_fault.withhold;
     t.bt = a.bt;
     t.bt_stride = a.bt_stride;
     t.epb = a.epb;
@@ -883,6 +902,7 @@ cudaError_t launch_attend_tc(const AttendArgs& a, void* ws, size_t ws_bytes, cud
         t.comb_pieces = (int)(bound < p.grid ? bound : p.grid);
     }
 
+    static_assert(sizeof(Smem) + 1024 <= 232448, "shared memory");
     const size_t smem = sizeof(Smem) + 1024;
     cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;

@@ -105,6 +105,16 @@ size_t attend_workspace_bytes(const AttendArgs& a);
 cudaError_t launch_attend(const AttendArgs& a, void* ws, size_t ws_bytes, cudaStream_t stream);
 
 // ---- attend_tc.cu (tcgen05 path: bf16, d = 512, 64 heads) -------------
+// Fault injection for the tensor-core attention's bounded waits (set by v4a_test_attend_fault only;
+// withhold = -1 in normal use): every CTA withholds its local tile `withhold`, and the waits give up
+// after wait_polls polls / stall_cycles cycles without progress.
+struct AttendFaultTest {
+    int withhold;
+    uint32_t wait_polls;
+    long long stall_cycles;
+};
+extern AttendFaultTest g_test_fault;
+
 bool attend_tc_shape_ok(const AttendArgs& a);   // the shape this path takes
 bool attend_tc_available(const AttendArgs& a);  // ... and the driver's tensor-map encoder is present
 size_t attend_tc_workspace_bytes(const AttendArgs& a);

@@ -548,6 +548,12 @@ const char* v4a_status_string(v4a_status st) {
 
 const char* v4a_last_error(void) { return g_last_error; }
 
+void v4a_test_attend_fault(int withhold_tile, int wait_polls) {
+    v4a::g_test_fault.withhold = withhold_tile >= 0 ? withhold_tile : -1;
+    v4a::g_test_fault.wait_polls = (uint32_t)(wait_polls > 0 ? wait_polls : 1);
+    v4a::g_test_fault.stall_cycles = 1LL << 22;  // ~2 ms of no progress at 1.9 GHz
+}
+
 int v4a_version(void) { return 200; }
 
 }  // extern "C"

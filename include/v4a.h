@@ -420,6 +420,24 @@ V4A_API const char* v4a_last_error(void);
 /* Library version: major*10000 + minor*100 + patch. */
 V4A_API int v4a_version(void);
 
+/* ------------------------------------------------------------------ */
+/* test hook                                                            */
+/* ------------------------------------------------------------------ */
+
+/* Fault injection for tests of the bounded waits (not part of the method;
+ * never needed in normal use).  With withhold_tile >= 0, every later launch
+ * of the tensor-core attention kernel (the bf16, d = 512, 64-head path of
+ * the CSA and HCA attention calls) makes each CTA skip the copies of its
+ * local tile withhold_tile -- no copy is issued and no arrival made, so that
+ * stage never fills -- and gives every wait of the kernel wait_polls polls
+ * (each suspends for at most ~20 us) and the MMA warp ~2 ms without progress.
+ * The waits then give up: the kernel records V4A_ERR_DEVICE_FAULT in the
+ * call's dev_status, writes NaN to every output it contributes to, frees its
+ * tensor memory and returns; nothing traps and nothing is left in flight.
+ * withhold_tile = -1 restores normal launches.  Host-side global state: not
+ * for concurrent use. */
+V4A_API void v4a_test_attend_fault(int withhold_tile, int wait_polls);
+
 #ifdef __cplusplus
 }
 #endif

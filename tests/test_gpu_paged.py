@@ -208,6 +208,18 @@ def test_paged_tensor_core_path_equals_contiguous(v4a, key_fmt):
         assert torch.equal(idx_p, idx_c) and torch.equal(sc_p, sc_c), f"top-k at ctx {ctx}"
         assert torch.equal(out_p, out_c), f"csa at ctx {ctx}"
         assert torch.equal(outh_p, outh_c), f"hca at ctx {ctx}"
+        if ctx == 900:
+            # and straight against the oracle on the bytes the cache holds: top-k (tie band), CSA and HCA
+            # attention (bf16 tolerance), not only transitively through the contiguous calls
+            if key_fmt == "mxfp4":
+                r_top = oracle.topk_mxfp4(host(qi), host(w), host(key), host(kexp), ctx, 4, k, want_scores=True)
+            else:
+                r_top = oracle.topk(host(qi), host(w), host(key), host(ksc), ctx, 4, k, want_scores=True)
+            check_topk(idx_p, r_top, ctx, 4, k)
+            r_c = oracle.attend(host(q), host(ent), r_top["idx"], host(tok), p0, ctx, 4, W)
+            check_attention(out_p, r_c, False, f"paged csa vs oracle at ctx {ctx}")
+            r_h = oracle.attend(host(q), host(hent[:, :Nh].contiguous()), None, host(tokh), p0, ctx, 128, W)
+            check_attention(outh_p, r_h, False, f"paged hca vs oracle at ctx {ctx}")
 
 
 def test_paged_bad_block_id_is_skipped_and_reported(v4a):

@@ -131,7 +131,12 @@ def test_compress_dual_fp8_output_into_cache_slice(v4a):
     sc = scales[:, s0:s0 + n_ent].double().cpu().numpy()
     assert np.allclose(sc, ref_sc, rtol=1e-5)
     deq = oracle.e4m3_decode(keys[:, s0:s0 + n_ent].cpu().numpy()) * sc[..., None]
-    assert np.abs(deq - ref).max() <= 0.07 * np.abs(ref).max()  # e4m3 keeps 3 mantissa bits
+    # each code is the nearest e4m3 grid point of value/scale (half a grid step), up to the fp32 arithmetic
+    # of the compressed value, as for the single-series FP8 output
+    v = ref / ref_sc[..., None]
+    step = np.maximum(2.0 ** (np.floor(np.log2(np.maximum(np.abs(v), 2.0 ** -6))) - 3), 2.0 ** -9)
+    err = np.abs(deq / sc[..., None] - v)
+    assert (err <= 0.5 * step * (1 + 1e-4) + 1e-5 * np.abs(v)).all()
     assert (keys[:, :s0] == 0).all() and (keys[:, s0 + n_ent:] == 0).all()
 
 
