@@ -8,15 +8,14 @@
 // Hybrid Compressed Attention", CSA "Core attention with shared KV MQA").
 //
 // Shape of the work.  One query has 64 heads sharing every K=V row, so per
-// 64-row tile of candidates:
-//   S  = Q K^T      tcgen05 M=64 (heads) x N=64 (rows) x K=512, Q and K in smem
-//   P  = softmax(S) (online, one thread per head)
-//   O^T += V^T P^T  tcgen05 M=128 (d chunk) x N=64 (heads) x K=64 (rows),
+// tile of T candidate rows (T = 64, or 48 for long rows: see Tiles):
+//   S  = Q K^T      tcgen05 M=64 (heads) x N=T (rows) x K=512, Q and K in smem
+//   P  = softmax(S) (online, two threads per head)
+//   O^T += V^T P^T  tcgen05 M=128 (d chunk) x N=64 (heads) x K=T (rows),
 //                   four d chunks, V^T read MN-major from the same smem tile
-// An MMA instruction costs about max(45, N/2) cycles at M=128 (M=64 at half
-// the rate), so tiles are as wide as shared memory allows (64 rows, two
-// stages next to the 64 KB query) and the issue loops use precomputed
-// descriptors.
+// One warp issues the MMAs (an elected lane per instruction, descriptors in
+// uniform registers); the issue rate, not the tensor pipe, bounds small MMAs,
+// so tiles are as wide as shared memory allows next to the 64 KB query.
 // The accumulator O^T (512 x 64 fp32) and two S buffers live in TMEM.
 //
 // Work split: the candidate tiles of all queries form one flat sequence that
@@ -24,7 +23,7 @@
 // whose range covers a query's tiles completely writes that query's output;
 // a query cut between CTAs gets one partial (m, l, O) per piece, merged by
 // attend_tc_combine.  Per CTA: warp 0 loads (TMA for contiguous rows and the
-// query, cp.async gathers for CSA-selected rows) into a 2-stage ring, warp 1
+// query, cp.async gathers for CSA-selected rows) into a ring of 2 or 3 stages, warp 1
 // (all lanes; one elected lane) issues the MMAs, warps 2-5 run the softmax and the output.  Every wait is
 // bounded; on a time-out the CTA records a device fault, poisons its outputs
 // with NaN and winds down.
@@ -39,15 +38,10 @@ namespace {
 
 constexpr int kD = 512;
 constexpr int kH = 64;
-constexpr int kTile = 48;                        // candidate rows per tile
-constexpr int kStages = 3;                       // tiles resident in shared memory
-constexpr uint64_t kTileMask = (1ull << kTile) - 1;
 constexpr uint32_t kSCols = 64;                  // TMEM columns between the two S buffers
 constexpr int kSlabs = kD / 64;                  // 64-element (128 B) column slabs
-constexpr uint32_t kSlabBytes = kTile * 128;     // 8 KB
-constexpr uint32_t kTileBytes = kSlabs * kSlabBytes;
 constexpr uint32_t kQBytes = kSlabs * kH * 128;  // 64 KB
-constexpr uint32_t kPBytes = kH * 128;           // 64 heads x 64 rows bf16
+constexpr uint32_t kPBytes = kH * 128;           // 64 heads x up to 64 rows bf16
 constexpr uint32_t kColO = 0;                    // O^T: 4 chunks of 64 columns
 constexpr uint32_t kColS = 256;                  // S: 2 buffers of 64 columns
 constexpr uint32_t kTmemCols = 512;
@@ -60,16 +54,36 @@ constexpr float kRescaleSlack = 8.0f;  // keep a stale running max until the tru
 // combine reads it back in the same 512-byte runs.  (Stored d-major, [d][64 heads], a warp store
 // touched 32 cache lines and a 128 KB piece took ~9,900 cycles to write on B200.)
 
-constexpr uint32_t kIdescQK = tc::idesc_f16(64, kTile, 0, 0);
 constexpr uint32_t kIdescPV = tc::idesc_f16(128, 64, 1, 0);
 
+// Tile shapes.  A tile is T candidate rows; its 8 column slabs of T x 128 bytes sit in one of C::kStages
+// stages beside the 64 KB query.  T = 64 with two stages keeps one tile load in flight while a tile is
+// processed and spends the fewest MMA instructions per row; T = 48 fits a third stage, so two loads
+// are in flight, at a third more QK instructions per row.  Long rows (HCA: thousands of entries per
+// query, streamed) take 48; short ones (CSA selections, prefill rows) take 64 (measured on B200: HCA
+// attention at 1M context 81 -> 77 us with 48; the prefill chunk's attention 1.72 -> 2.10 ms with 48).
+template <int T>
+struct Tiles {
+    static_assert(T == 48 || T == 64, "tile rows");
+    static constexpr int kTile = T;
+    static constexpr int kStages = T == 64 ? 2 : 3;
+    static constexpr uint64_t kTileMask = T == 64 ? ~0ull : ((1ull << T) - 1ull);
+    static constexpr uint32_t kSlabBytes = T * 128;
+    static constexpr uint32_t kTileBytes = kSlabs * kSlabBytes;
+    static constexpr uint32_t kIdescQK = tc::idesc_f16(64, T, 0, 0);
+    static constexpr int kHalfRows = T / 2;          // S values per softmax thread
+    static constexpr int kHiRows = T / 2 - 16;       // ... of which from the second 16x32bx2 load
+};
+
+template <int T>
 struct __align__(1024) Smem {
+    using C = Tiles<T>;
     uint8_t q[kQBytes];
-    uint8_t kv[kStages][kTileBytes];
+    uint8_t kv[C::kStages][C::kTileBytes];
     uint8_t p[2][kPBytes];
-    uint64_t kv_full[kStages], kv_empty[kStages], s_full[2], p_full[2], p_free[2];
+    uint64_t kv_full[C::kStages], kv_empty[C::kStages], s_full[2], p_full[2], p_free[2];
     uint64_t q_full, q_empty, drain;
-    uint64_t mask[kStages];
+    uint64_t mask[C::kStages];
     float alpha[2][kH], l_s[kH], m_s[kH];  // alpha / rescale_tag by tile parity
     int rescale_tag[2];
     int abort_flag;
@@ -150,7 +164,8 @@ __device__ __forceinline__ RowInfo row_info(int row, const TcArgs& a) {
     return r;
 }
 
-__device__ __forceinline__ void fault(Smem& sm, const TcArgs& a) {
+template <int T>
+__device__ __forceinline__ void fault(Smem<T>& sm, const TcArgs& a) {
     sm.abort_flag = 1;
     if (a.dev_status) atomicExch(a.dev_status, (int)V4A_ERR_DEVICE_FAULT);
 }
@@ -159,12 +174,14 @@ __device__ __forceinline__ void fault(Smem& sm, const TcArgs& a) {
 // warp 0: loads
 // ---------------------------------------------------------------------
 // candidate rows of one CSA tile: lane owns rows lane and lane+32
+template <int T>
 __device__ __forceinline__ void csa_rows(const TcArgs& a, const RowInfo& ri, int row, long long c0, int lane,
                                          const __nv_bfloat16* (&src)[2], bool (&ok)[2]) {
+    using C = Tiles<T>;
 #pragma unroll
     for (int h2 = 0; h2 < 2; ++h2) {
         const long long c = c0 + lane + 32 * h2;
-        const long long sidx = (c < a.k && lane + 32 * h2 < kTile) ? (long long)a.idx[(long long)row * a.k + c] : -1;
+        const long long sidx = (c < a.k && lane + 32 * h2 < C::kTile) ? (long long)a.idx[(long long)row * a.k + c] : -1;
         ok[h2] = sidx >= 0 && sidx < ri.nvis;
         const __nv_bfloat16* er = ok[h2] ? entry_row(a, ri.b, sidx) : nullptr;
         if (ok[h2] && !er) {  // a block id outside the pool: skipped and reported
@@ -176,19 +193,21 @@ __device__ __forceinline__ void csa_rows(const TcArgs& a, const RowInfo& ri, int
     }
 }
 
-// cp.async all 64 rows of a tile (lane owns rows lane and lane+32: src / ok) into the 128-byte-swizzled
+// cp.async all T rows of a tile (lane owns rows lane and lane+32: src / ok) into the 128-byte-swizzled
 // stage; returns the tile's row mask
+template <int T>
 __device__ __forceinline__ uint64_t gather_tile(uint8_t* dst, const __nv_bfloat16* const (&src)[2], const bool (&ok)[2],
                                                 int lane, uint64_t policy) {
+    using C = Tiles<T>;
     const uint64_t mask =
         (uint64_t)__ballot_sync(0xffffffffu, ok[0]) | ((uint64_t)__ballot_sync(0xffffffffu, ok[1]) << 32);
-    for (int r = 0; r < kTile; ++r) {
+    for (int r = 0; r < C::kTile; ++r) {
         const __nv_bfloat16* rs =
             (const __nv_bfloat16*)__shfl_sync(0xffffffffu, (unsigned long long)(r < 32 ? src[0] : src[1]), r & 31);
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
             const int u = lane + 32 * h2;  // 16-byte chunk of the 1 KB row
-            uint8_t* d = dst + (u >> 3) * kSlabBytes + r * 128 + (((u & 7) ^ (r & 7)) << 4);
+            uint8_t* d = dst + (u >> 3) * C::kSlabBytes + r * 128 + (((u & 7) ^ (r & 7)) << 4);
             tc::cp_async_16_hint(d, rs + u * 8, policy);
         }
     }
@@ -197,19 +216,21 @@ __device__ __forceinline__ uint64_t gather_tile(uint8_t* dst, const __nv_bfloat1
 
 // Rows of a gathered tile (CSA selections, paged entries, ring windows) for this lane: rows lane and
 // lane + 32 (src, ok).  False for tiles loaded with TMA.  Bad selections and block ids are reported here.
+template <int T>
 __device__ __forceinline__ bool tile_rows(const TcArgs& a, int row, int ti, int lane, const __nv_bfloat16* (&src)[2],
                                           bool (&ok)[2]) {
+    using C = Tiles<T>;
     if (!tile_gathered(a, ti)) return false;
     const RowInfo ri = row_info(row, a);
     const __nv_bfloat16* fallback = a.q + (long long)row * kH * kD;  // finite data for excluded rows
     if (ti < a.e_tiles) {
-        const long long c0 = (long long)ti * kTile;
+        const long long c0 = (long long)ti * C::kTile;
         if (a.idx) {
-            csa_rows(a, ri, row, c0, lane, src, ok);
+            csa_rows<T>(a, ri, row, c0, lane, src, ok);
 #pragma unroll
             for (int h2 = 0; h2 < 2; ++h2) {
                 const long long c = c0 + lane + 32 * h2;
-                const long long sidx = (c < a.k && lane + 32 * h2 < kTile) ? (long long)a.idx[(long long)row * a.k + c] : -1;
+                const long long sidx = (c < a.k && lane + 32 * h2 < C::kTile) ? (long long)a.idx[(long long)row * a.k + c] : -1;
                 if (!ok[h2] && sidx != -1 && a.dev_status) atomicExch(a.dev_status, (int)V4A_ERR_DEVICE_FAULT);
             }
         } else {
@@ -217,7 +238,7 @@ __device__ __forceinline__ bool tile_rows(const TcArgs& a, int row, int ti, int 
 #pragma unroll
             for (int h2 = 0; h2 < 2; ++h2) {
                 const long long s = c0 + lane + 32 * h2;
-                const __nv_bfloat16* er = (s < ri.nvis && lane + 32 * h2 < kTile) ? entry_row(a, ri.b, s) : nullptr;
+                const __nv_bfloat16* er = (s < ri.nvis && lane + 32 * h2 < C::kTile) ? entry_row(a, ri.b, s) : nullptr;
                 if (s < ri.nvis && !er && a.dev_status) atomicExch(a.dev_status, (int)V4A_ERR_DEVICE_FAULT);
                 ok[h2] = er != nullptr;
                 src[h2] = ok[h2] ? er : fallback;
@@ -226,12 +247,12 @@ __device__ __forceinline__ bool tile_rows(const TcArgs& a, int row, int ti, int 
     } else {
         // window tokens p0 .. p0+63 from the ring (they may wrap around its end)
         const long long wi = ti - a.e_tiles;
-        const long long p0 = ri.t - a.window + 1 + wi * kTile;
+        const long long p0 = ri.t - a.window + 1 + wi * C::kTile;
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
             const int r = lane + 32 * h2;
             const long long p = p0 + r;
-            ok[h2] = r < kTile && wi * kTile + r < a.window && p >= 0;
+            ok[h2] = r < C::kTile && wi * C::kTile + r < a.window && p >= 0;
             src[h2] = ok[h2] ? a.token_kv + ((long long)ri.b * a.ring_rows + p % a.ring_rows) * kD : fallback;
         }
     }
@@ -243,35 +264,39 @@ __device__ __forceinline__ bool tile_rows(const TcArgs& a, int row, int ti, int 
 // writes attention queries, and a kernel before this one on the stream that is not programmatically
 // launched has completed before this one starts, so the query is complete; the prefetch only warms L2,
 // the point of coherence, so an entry still being written is read afresh by the load after the wait.
-__device__ void early_loads(Smem& sm, const TcArgs& a, const CUtensorMap* ent_map, const CUtensorMap* q_map,
+template <int T>
+__device__ void early_loads(Smem<T>& sm, const TcArgs& a, const CUtensorMap* ent_map, const CUtensorMap* q_map,
                             long long f0, long long f1) {
+    using C = Tiles<T>;
     const Cursor cur(f0, a.tpr);
     tc::mbar_arrive_expect_tx(&sm.q_full, kQBytes);
     for (int c = 0; c < kSlabs; ++c) tc::tma_load_2d(sm.q + c * kH * 128, q_map, 64 * c, cur.row * kH, &sm.q_full);
     if (a.idx || a.bt) return;
     const RowInfo ri = row_info(cur.row, a);
-    for (int j = 0; j < kStages && f0 + j < f1 && cur.ti + j < a.e_tiles; ++j) {
-        const int y = (int)((long long)ri.b * a.n_ent + (long long)(cur.ti + j) * kTile);
+    for (int j = 0; j < C::kStages && f0 + j < f1 && cur.ti + j < a.e_tiles; ++j) {
+        const int y = (int)((long long)ri.b * a.n_ent + (long long)(cur.ti + j) * C::kTile);
         for (int c = 0; c < kSlabs; ++c) tc::tma_prefetch_2d(ent_map, 64 * c, y);
     }
 }
 
-__device__ void producer(Smem& sm, const TcArgs& a, const CUtensorMap* ent_map, const CUtensorMap* tok_map,
+template <int T>
+__device__ void producer(Smem<T>& sm, const TcArgs& a, const CUtensorMap* ent_map, const CUtensorMap* tok_map,
                          const CUtensorMap* q_map, long long f0, long long f1) {
+    using C = Tiles<T>;
     const int lane = threadIdx.x & 31;
     int seg = 0;
     Cursor cur(f0, a.tpr);
     const uint64_t stream_policy = tc::l2_evict_first();  // candidate rows are read once per call
-    int last_load[kStages];  // the last tile whose copies went into each stage (-1: none)
-    for (int i = 0; i < kStages; ++i) last_load[i] = -1;
+    int last_load[C::kStages];  // the last tile whose copies went into each stage (-1: none)
+    for (int i = 0; i < C::kStages; ++i) last_load[i] = -1;
     // the rows of gathered tiles are worked out a tile ahead, so their index / block-table loads overlap
     // the current tile's copies
     const __nv_bfloat16* nsrc[2] = {a.q, a.q};
     bool nok[2] = {false, false};
-    bool ngath = f0 < f1 && tile_rows(a, cur.row, cur.ti, lane, nsrc, nok);
+    bool ngath = f0 < f1 && tile_rows<T>(a, cur.row, cur.ti, lane, nsrc, nok);
     for (long long f = f0; f < f1; ++f, cur.next(a.tpr)) {
         if (sm.abort_flag) break;
-        const int jt = (int)(f - f0), st = jt % kStages;
+        const int jt = (int)(f - f0), st = jt % C::kStages;
         const int row = cur.row, ti = cur.ti;
         const bool seg_start = (f == f0) || (ti == 0);
         const RowInfo ri = row_info(row, a);
@@ -281,7 +306,7 @@ __device__ void producer(Smem& sm, const TcArgs& a, const CUtensorMap* ent_map, 
         if (f + 1 < f1) {
             Cursor nx = cur;
             nx.next(a.tpr);
-            ngath = tile_rows(a, nx.row, nx.ti, lane, nsrc, nok);
+            ngath = tile_rows<T>(a, nx.row, nx.ti, lane, nsrc, nok);
         }
         if (seg_start) {
             if (seg > 0 && !tc::mbar_wait(&sm.q_empty, (seg - 1) & 1, a.wait_polls)) { fault(sm, a); break; }
@@ -291,51 +316,51 @@ __device__ void producer(Smem& sm, const TcArgs& a, const CUtensorMap* ent_map, 
             }
             ++seg;
         }
-        if (jt >= kStages && !tc::mbar_wait(&sm.kv_empty[st], ((jt / kStages) - 1) & 1, a.wait_polls)) { fault(sm, a); break; }
+        if (jt >= C::kStages && !tc::mbar_wait(&sm.kv_empty[st], ((jt / C::kStages) - 1) & 1, a.wait_polls)) { fault(sm, a); break; }
         uint64_t mask = 0;
         uint8_t* dst = sm.kv[st];
         if (jt == a.withhold) continue;  // test hook: this stage never fills (no copy, no arrival)
         last_load[st] = jt;
         if (gath) {
-            mask = gather_tile(dst, src, ok, lane, stream_policy);
+            mask = gather_tile<T>(dst, src, ok, lane, stream_policy);
             if (lane == 0) {
                 sm.mask[st] = mask;
                 tc::mbar_arrive_expect_tx(&sm.kv_full[st], 0);
             }
         } else if (ti < a.e_tiles) {
             // HCA: rows c0 .. c0+63 of this sequence's entries are contiguous
-            const long long c0 = (long long)ti * kTile;
+            const long long c0 = (long long)ti * C::kTile;
             const long long nv = ri.nvis - c0;
-            mask = nv >= kTile ? kTileMask : (nv <= 0 ? 0ull : ((1ull << nv) - 1ull));
+            mask = nv >= C::kTile ? C::kTileMask : (nv <= 0 ? 0ull : ((1ull << nv) - 1ull));
             if (lane == 0) {
                 sm.mask[st] = mask;
-                tc::mbar_arrive_expect_tx(&sm.kv_full[st], kTileBytes);
+                tc::mbar_arrive_expect_tx(&sm.kv_full[st], C::kTileBytes);
                 const int y = (int)((long long)ri.b * a.n_ent + c0);
                 for (int c = 0; c < kSlabs; ++c)
-                    tc::tma_load_2d_hint(dst + c * kSlabBytes, ent_map, 64 * c, y, &sm.kv_full[st], stream_policy);
+                    tc::tma_load_2d_hint(dst + c * C::kSlabBytes, ent_map, 64 * c, y, &sm.kv_full[st], stream_policy);
             }
         } else {
             // window tokens p0 .. p0+63 (contiguous rows of token_kv)
             const long long wi = ti - a.e_tiles;
-            const long long p0 = ri.t - a.window + 1 + wi * kTile;
-            for (int r = 0; r < kTile; ++r) {
+            const long long p0 = ri.t - a.window + 1 + wi * C::kTile;
+            for (int r = 0; r < C::kTile; ++r) {
                 const long long p = p0 + r;
-                if (wi * kTile + r < a.window && p >= 0) mask |= 1ull << r;
+                if (wi * C::kTile + r < a.window && p >= 0) mask |= 1ull << r;
             }
             if (lane == 0) {
                 sm.mask[st] = mask;
-                tc::mbar_arrive_expect_tx(&sm.kv_full[st], kTileBytes);
+                tc::mbar_arrive_expect_tx(&sm.kv_full[st], C::kTileBytes);
                 const int y = (int)((long long)ri.b * a.l_tok + (p0 - a.tok_pos0));
                 for (int c = 0; c < kSlabs; ++c)
-                    tc::tma_load_2d_hint(dst + c * kSlabBytes, tok_map, 64 * c, y, &sm.kv_full[st], stream_policy);
+                    tc::tma_load_2d_hint(dst + c * C::kSlabBytes, tok_map, 64 * c, y, &sm.kv_full[st], stream_policy);
             }
         }
         tc::cp_async_arrive_noinc(&sm.kv_full[st]);  // 32 lanes: after their cp.async copies (if any) land
     }
     // make sure nothing this warp started is still in flight before the CTA retires (also after an abort
     // or a withheld stage: the last copies issued into each stage)
-    for (int st = 0; st < kStages; ++st)
-        if (last_load[st] >= 0) tc::mbar_wait(&sm.kv_full[st], (last_load[st] / kStages) & 1, a.wait_polls);
+    for (int st = 0; st < C::kStages; ++st)
+        if (last_load[st] >= 0) tc::mbar_wait(&sm.kv_full[st], (last_load[st] / C::kStages) & 1, a.wait_polls);
     // ... nor a query load (the first segment's was issued before the loop)
     const int q_loads = seg > 0 ? seg : (f0 < f1 ? 1 : 0);
     if (q_loads > 0) tc::mbar_wait(&sm.q_full, (q_loads - 1) & 1, a.wait_polls);
@@ -348,17 +373,19 @@ __device__ void producer(Smem& sm, const TcArgs& a, const CUtensorMap* ent_map, 
 __device__ __forceinline__ uint64_t dadd(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
 
 // O^T += V^T P^T for tile jp (its P is in shared memory)
-__device__ void issue_pv(Smem& sm, uint32_t tmem, int jp, bool first_in_seg) {
-    const int sp = jp & 1, st = jp % kStages;
+template <int T>
+__device__ void issue_pv(Smem<T>& sm, uint32_t tmem, int jp, bool first_in_seg) {
+    using C = Tiles<T>;
+    const int sp = jp & 1, st = jp % C::kStages;
     tc::tc_fence_after();
     // A = V^T (M = 128 d of slabs 2cc, 2cc+1; K = 16 rows), MN-major; B = P^T, K-major rows of P
-    const uint64_t a0 = tc::sw128_desc(tc::smem_u32(sm.kv[st]), kSlabBytes, 1024);
+    const uint64_t a0 = tc::sw128_desc(tc::smem_u32(sm.kv[st]), C::kSlabBytes, 1024);
     const uint64_t b0 = tc::sw128_desc(tc::smem_u32(sm.p[sp]), 16, 1024);
 #pragma unroll
-    for (int kk = 0; kk < kTile / 16; ++kk) {
+    for (int kk = 0; kk < C::kTile / 16; ++kk) {
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc)
-            tc::mma_f16(tmem + kColO + 64 * cc, dadd(a0, (2 * cc) * kSlabBytes + kk * 2048), dadd(b0, kk * 32),
+            tc::mma_f16(tmem + kColO + 64 * cc, dadd(a0, (2 * cc) * C::kSlabBytes + kk * 2048), dadd(b0, kk * 32),
                         kIdescPV, (!first_in_seg || kk > 0) ? 1u : 0u);
     }
     tc::mma_commit(&sm.kv_empty[st]);
@@ -366,8 +393,10 @@ __device__ void issue_pv(Smem& sm, uint32_t tmem, int jp, bool first_in_seg) {
 }
 
 // S = Q K^T for tile jq (its rows are in shared memory)
-__device__ void issue_qk(Smem& sm, uint32_t tmem, int jq, bool gathered, uint64_t q0) {
-    const int s = jq & 1, st = jq % kStages;
+template <int T>
+__device__ void issue_qk(Smem<T>& sm, uint32_t tmem, int jq, bool gathered, uint64_t q0) {
+    using C = Tiles<T>;
+    const int s = jq & 1, st = jq % C::kStages;
     if (gathered) tc::fence_proxy_async();  // rows gathered with cp.async become visible to the tensor core
     tc::tc_fence_after();
     const uint64_t k0 = tc::sw128_desc(tc::smem_u32(sm.kv[st]), 16, 1024);
@@ -376,7 +405,7 @@ __device__ void issue_qk(Smem& sm, uint32_t tmem, int jq, bool gathered, uint64_
     for (int c = 0; c < kSlabs; ++c) {
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-            tc::mma_f16(d_s, dadd(q0, c * kH * 128 + kk * 32), dadd(k0, c * kSlabBytes + kk * 32), kIdescQK,
+            tc::mma_f16(d_s, dadd(q0, c * kH * 128 + kk * 32), dadd(k0, c * C::kSlabBytes + kk * 32), C::kIdescQK,
                         (c | kk) ? 1u : 0u);
     }
     tc::mma_commit(&sm.s_full[s]);
@@ -390,7 +419,9 @@ constexpr long long kStallCycles = 1LL << 31;
 // whatever order their inputs become ready: PV(j) as soon as the softmax has written P(j) (which frees
 // tile j's stage for the next load early), QK(j) as soon as tile j has landed and S buffer j&1 is free
 // (PV(j-2) issued).
-__device__ void mma_issuer(Smem& sm, const TcArgs& a, uint32_t tmem, long long f0, long long f1) {
+template <int T>
+__device__ void mma_issuer(Smem<T>& sm, const TcArgs& a, uint32_t tmem, long long f0, long long f1) {
+    using C = Tiles<T>;
     const long long n = f1 - f0;
     const uint64_t q0 = tc::sw128_desc(tc::smem_u32(sm.q), 16, 1024);
     long long jq = 0, jp = 0;
@@ -408,9 +439,9 @@ __device__ void mma_issuer(Smem& sm, const TcArgs& a, uint32_t tmem, long long f
             progressed = true;
         } else if (jq < n && jp >= jq - 1) {
             const bool qseg = jq == 0 || cq.ti == 0;
-            if (tc::mbar_test_warp(&sm.kv_full[jq % kStages], (uint32_t)(jq / kStages) & 1) &&
+            if (tc::mbar_test_warp(&sm.kv_full[jq % C::kStages], (uint32_t)(jq / C::kStages) & 1) &&
                 (!qseg || tc::mbar_test_warp(&sm.q_full, segq & 1))) {
-                issue_qk(sm, tmem, (int)jq, tile_gathered(a, cq.ti), q0);
+                issue_qk<T>(sm, tmem, (int)jq, tile_gathered(a, cq.ti), q0);
                 if (jq == n - 1 || cq.ti == a.tpr - 1) tc::mma_commit(&sm.q_empty);  // last QK of this query
                 if (qseg) ++segq;
                 ++jq;
@@ -434,7 +465,9 @@ __device__ void mma_issuer(Smem& sm, const TcArgs& a, uint32_t tmem, long long f
 // ---------------------------------------------------------------------
 // warps 2-5: softmax, rescale, output
 // ---------------------------------------------------------------------
-__device__ void softmax_warps(Smem& sm, const TcArgs& a, uint32_t tmem, long long f0, long long f1, int cta) {
+template <int T>
+__device__ void softmax_warps(Smem<T>& sm, const TcArgs& a, uint32_t tmem, long long f0, long long f1, int cta) {
+    using C = Tiles<T>;
     const int sub = (threadIdx.x >> 5) & 3;  // TMEM sub-partition this warp may access
     const int lane = threadIdx.x & 31;
     // M = 64: head 16*sub + (lane & 15) lives in TMEM lane 32*sub + (lane & 15); lanes 0-15 take the
@@ -448,7 +481,7 @@ __device__ void softmax_warps(Smem& sm, const TcArgs& a, uint32_t tmem, long lon
     const int first_row = cur.row;
     for (long long f = f0; f < f1; ++f, cur.next(a.tpr)) {
         if (sm.abort_flag) { ok = false; break; }
-        const int jt = (int)(f - f0), s = jt & 1, st = jt % kStages;
+        const int jt = (int)(f - f0), s = jt & 1, st = jt % C::kStages;
         const int row = cur.row, ti = cur.ti;
         const bool seg_start = (f == f0) || (ti == 0);
         const bool seg_end = (f == f1 - 1) || (ti == a.tpr - 1);
@@ -456,23 +489,28 @@ __device__ void softmax_warps(Smem& sm, const TcArgs& a, uint32_t tmem, long lon
             m_run = -INFINITY;
             l_run = 0.f;
         }
-        if (!tc::mbar_wait(&sm.kv_full[st], (jt / kStages) & 1, a.wait_polls)) { ok = false; break; }
+        if (!tc::mbar_wait(&sm.kv_full[st], (jt / C::kStages) & 1, a.wait_polls)) { ok = false; break; }
+        // this thread's kHalfRows rows of the tile: 16 from S columns [0, 32) (rows 16 half .. 16 half + 15)
+        // and kHiRows from columns [32, T) (rows 32 + kHiRows half ..), the two halves of each 16x32bx2 load
+        constexpr int kNR = C::kHalfRows, kHi = C::kHiRows;
         const uint64_t tmask = sm.mask[st];
-        const uint32_t mask = (uint32_t)((tmask >> (16 * half)) & 0xffffu) | ((uint32_t)((tmask >> (32 + 8 * half)) & 0xffu) << 16);
+        const uint32_t mask = (uint32_t)((tmask >> (16 * half)) & 0xffffu) |
+                              ((uint32_t)((tmask >> (32 + kHi * half)) & ((1ull << kHi) - 1ull)) << 16);
         if (!tc::mbar_wait(&sm.s_full[s], (jt >> 1) & 1, a.wait_polls)) { ok = false; break; }
         tc::tc_fence_after();
-        uint32_t r[24];
+        uint32_t r[kNR];
         tc::tmem_ld_16x32bx2_x16(tmem + lane_addr + kColS + kSCols * s, r);
-        tc::tmem_ld_16x32bx2_x8(tmem + lane_addr + kColS + kSCols * s + 32, r + 16);
+        if constexpr (kHi == 16) tc::tmem_ld_16x32bx2_x16(tmem + lane_addr + kColS + kSCols * s + 32, r + 16);
+        else tc::tmem_ld_16x32bx2_x8(tmem + lane_addr + kColS + kSCols * s + 32, r + 16);
         tc::tmem_ld_wait();
         float alpha = 1.f;
         bool rescale = false;
-        uint32_t pk[12];  // bf16 pairs of this thread's 24 probabilities
+        uint32_t pk[kNR / 2];  // bf16 pairs of this thread's probabilities
         {
             // independent partial maxima / sums keep the dependent chains short
             float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-            for (int i = 0; i < 24; ++i) {
+            for (int i = 0; i < kNR; ++i) {
                 const float x = ((mask >> i) & 1) ? __uint_as_float(r[i]) * a.scale_log2 : -INFINITY;
                 r[i] = __float_as_uint(x);
                 mx4[i & 3] = fmaxf(mx4[i & 3], x);
@@ -490,7 +528,7 @@ __device__ void softmax_warps(Smem& sm, const TcArgs& a, uint32_t tmem, long lon
             const float msub = m_run == -INFINITY ? 0.f : m_run;  // all-masked so far: every x is -inf
             float ls4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int i = 0; i < 12; ++i) {
+            for (int i = 0; i < kNR / 2; ++i) {
                 const float p0 = exp2f(__uint_as_float(r[2 * i]) - msub);
                 const float p1 = exp2f(__uint_as_float(r[2 * i + 1]) - msub);
                 const __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
@@ -522,12 +560,13 @@ __device__ void softmax_warps(Smem& sm, const TcArgs& a, uint32_t tmem, long lon
             tc::tmem_st_wait();
         }
         {
-            // head h's row of P: the tile's 64 probabilities as one 128 B swizzled row; this thread
-            // writes the 4 16-byte chunks of its half
+            // head h's row of P: the tile's probabilities as one 128 B swizzled row (the first 2 T bytes
+            // used); this thread writes the 16-byte chunks of its rows: 8-row chunks 2 half, 2 half + 1 (rows
+            // 16 half ..) and then 4 + (kHi / 8) half .. (rows 32 + kHi half ..)
             uint8_t* prow = sm.p[s] + (h >> 3) * 1024 + (h & 7) * 128;
 #pragma unroll
-            for (int u = 0; u < 3; ++u) {
-                const int chunk = u < 2 ? 2 * half + u : 4 + half;  // rows 8 chunk .. 8 chunk + 7
+            for (int u = 0; u < kNR / 8; ++u) {
+                const int chunk = u < 2 ? 2 * half + u : 4 + (kHi / 8) * half + (u - 2);
                 *reinterpret_cast<uint4*>(prow + ((chunk ^ (h & 7)) << 4)) =
                     make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
             }
@@ -609,17 +648,19 @@ __device__ void softmax_warps(Smem& sm, const TcArgs& a, uint32_t tmem, long lon
     }
 }
 
+template <int T>
 __global__ void __launch_bounds__(kThreads, 1)
     attend_tc_kernel(const __grid_constant__ CUtensorMap ent_map, const __grid_constant__ CUtensorMap tok_map,
                      const __grid_constant__ CUtensorMap q_map, TcArgs a) {
+    using C = Tiles<T>;
     extern __shared__ uint8_t smem_raw[];
-    Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Smem<T>& sm = *reinterpret_cast<Smem<T>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5;
     const int cta = blockIdx.x;
     const long long f0 = range_start(cta, a), f1 = range_start(cta + 1, a);
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kStages; ++i) {
+        for (int i = 0; i < C::kStages; ++i) {
             tc::mbar_init(&sm.kv_full[i], 33);  // 1 expect_tx arrival + 32 cp.async arrivals
             tc::mbar_init(&sm.kv_empty[i], 1);
         }
@@ -804,6 +845,7 @@ bool make_map(CUtensorMap* map, const void* base, long long rows, int box_rows) 
 }
 
 struct TcPlan {
+    int tile;  // rows per tile: 48 for rows of more than 2,048 candidates, else 64 (see Tiles)
     int e_tiles, w_tiles, tpr, grid;
     long long total;
 };
@@ -811,8 +853,9 @@ struct TcPlan {
 TcPlan tc_plan(const AttendArgs& a) {
     TcPlan p;
     const long long n_sel_max = a.idx ? (long long)a.k : (a.ctx_len / a.m < a.n_ent ? a.ctx_len / a.m : a.n_ent);
-    p.e_tiles = (int)((n_sel_max + kTile - 1) / kTile);
-    p.w_tiles = (a.window + kTile - 1) / kTile;
+    p.tile = n_sel_max > 2048 ? 48 : 64;
+    p.e_tiles = (int)((n_sel_max + p.tile - 1) / p.tile);
+    p.w_tiles = (a.window + p.tile - 1) / p.tile;
     p.tpr = p.e_tiles + p.w_tiles;
     p.total = (long long)a.batch * a.n_q * p.tpr;
     p.grid = (int)(p.total < kNumSMs ? p.total : kNumSMs);
@@ -849,10 +892,10 @@ cudaError_t launch_attend_tc(const AttendArgs& a, void* ws, size_t ws_bytes, cud
     const long long ent_rows = a.bt ? a.pool_rows : (long long)a.batch * a.n_ent;
     const long long tok_rows = (long long)a.batch * (a.ring_rows > 0 ? a.ring_rows : a.l_tok);
     const void* tok = a.token_kv ? a.token_kv : a.q;  // a window of 0 never reads it
-    if (!make_map(&tok_map, tok, a.token_kv ? tok_rows : (long long)a.batch * a.n_q * kH, kTile))
+    if (!make_map(&tok_map, tok, a.token_kv ? tok_rows : (long long)a.batch * a.n_q * kH, p.tile))
         return cudaErrorInvalidValue;
     if (ent_rows > 0) {
-        if (!make_map(&ent_map, a.entries, ent_rows, kTile)) return cudaErrorInvalidValue;
+        if (!make_map(&ent_map, a.entries, ent_rows, p.tile)) return cudaErrorInvalidValue;
     } else {
         ent_map = tok_map;  // no entry tiles exist
     }
@@ -902,12 +945,15 @@ cudaError_t launch_attend_tc(const AttendArgs& a, void* ws, size_t ws_bytes, cud
         t.comb_pieces = (int)(bound < p.grid ? bound : p.grid);
     }
 
-    static_assert(sizeof(Smem) + 1024 <= 232448, "shared memory");
-    const size_t smem = sizeof(Smem) + 1024;
-    cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    e = launch_pdl(attend_tc_kernel, dim3(p.grid), dim3(kThreads), smem, stream, ent_map, tok_map, q_map, t);
-    if (e == cudaSuccess) e = cudaGetLastError();
+    auto go = [&](auto kernel, size_t smem) {
+        cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (err == cudaSuccess)
+            err = launch_pdl(kernel, dim3(p.grid), dim3(kThreads), smem, stream, ent_map, tok_map, q_map, t);
+        return err == cudaSuccess ? cudaGetLastError() : err;
+    };
+    static_assert(sizeof(Smem<48>) + 1024 <= 232448 && sizeof(Smem<64>) + 1024 <= 232448, "shared memory");
+    cudaError_t e = p.tile == 48 ? go(attend_tc_kernel<48>, sizeof(Smem<48>) + 1024)
+                                 : go(attend_tc_kernel<64>, sizeof(Smem<64>) + 1024);
     if (e != cudaSuccess) return e;
     if (p.grid > 1) {
         const size_t csm = (size_t)t.comb_pieces * kH * sizeof(float);

@@ -248,6 +248,7 @@ def _attend_inputs(B, T, L, m, H, d, W, fmt, seed, k=None, pad=0.0, dup=False):
     ("bf16", 3, 2, 5000, 4, 64, 512, 128, 300),
     ("bf16", 1, 4, 100, 4, 16, 256, 128, 64),      # short context: window clipped at 0, k > N_vis
     ("bf16", 2, 1, 2048, 4, 32, 512, 0, 128),      # no window
+    ("bf16", 2, 1, 4 * 3000, 4, 64, 512, 128, 2500),  # k > 2048: the 48-row-tile kernel
 ])
 def test_csa_attend_matches_oracle(v4a, fmt, B, T, L, m, H, d, W, k):
     a = _attend_inputs(B, T, L, m, H, d, W, fmt, seed=L + k, k=k, pad=0.1)
@@ -292,6 +293,7 @@ def test_csa_attend_duplicates_and_bad_indices(v4a):
     ("f32", 2, 2, 100, 8, 64, 128),      # shorter than one chunk: pure sliding window
     ("bf16", 1, 1, 127, 64, 512, 128),
     ("bf16", 2, 1, 128 * 40, 32, 256, 0),  # no window
+    ("bf16", 1, 1, 128 * 2100 + 77, 64, 512, 128),  # more than 2,048 entries: the 48-row-tile kernel
 ])
 def test_hca_attend_matches_oracle(v4a, fmt, B, T, L, H, d, W):
     m = 128
