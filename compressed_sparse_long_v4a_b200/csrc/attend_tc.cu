@@ -84,7 +84,7 @@ struct __align__(1024) Smem {
     uint64_t kv_full[C::kStages], kv_empty[C::kStages], s_full[2], p_full[2], p_free[2];
     uint64_t q_full, q_empty, drain;
     uint64_t mask[C::kStages];
-    float alpha[2][kH], l_s[kH], m_s[kH];  // alpha / rescale_tag by tile parity
+    float alpha[2][kH], inv_l[kH];  // alpha / rescale_tag by tile parity; 1 / l of a whole row's heads
     int rescale_tag[2];
     int abort_flag;
     uint32_t tmem_base;
@@ -581,11 +581,11 @@ __device__ void softmax_warps(Smem<T>& sm, const TcArgs& a, uint32_t tmem, long 
             const float l_row = l_run + __shfl_xor_sync(0xffffffffu, l_run, 16);
             const long long rs = (long long)row * a.tpr;
             const bool whole = (rs >= f0) && (rs + a.tpr <= f1);
-            if (half == 0) {
-                sm.m_s[h] = m_run;
+            if (half == 0 && whole) {
                 // a whole row is normalised here: the sink joins its denominator (a split row's in the combine)
-                sm.l_s[h] = l_row + ((whole && a.sink && m_run != -INFINITY)
-                                         ? exp2f(a.sink[h] * 1.4426950408889634f - m_run) : 0.f);
+                const float l = l_row + ((a.sink && m_run != -INFINITY)
+                                             ? exp2f(a.sink[h] * 1.4426950408889634f - m_run) : 0.f);
+                sm.inv_l[h] = l > 0.f ? 1.f / l : 0.f;  // an empty row stays zero
             }
             tc::named_barrier(1, 128);
             // a piece of a split query: slot 2c for the CTA's first query, 2c+1 for its last
@@ -615,13 +615,34 @@ __device__ void softmax_warps(Smem<T>& sm, const TcArgs& a, uint32_t tmem, long 
                                     a.rope_base, &rs_, &rc_);
 #pragma unroll
                     for (int i = 0; i < kH; ++i) {
-                        const float l = sm.l_s[i];
-                        float v = l > 0.f ? __uint_as_float(o[i]) / l : 0.f;
+                        float v = __uint_as_float(o[i]) * sm.inv_l[i];
                         if (rot) {
                             const float p = __shfl_xor_sync(0xffffffffu, v, 1);
                             if (d >= kD - a.rope_dims) v = rope_apply(d, v, p, rs_, rc_);
                         }
-                        dst[i * kD + d] = v;
+                        o[i] = __float_as_uint(v);
+                    }
+                    // out[row][h][d]: lanes 4q .. 4q+3 exchange their 4 x 4 blocks (heads 4g .. 4g+3 at dims
+                    // d - j .. d - j + 3, j = lane % 4) in two xor steps, so that lane 4q + j holds head 4g + j
+                    // at those 4 dims: one 16-byte store per head group instead of four 4-byte ones
+                    const int j = lane & 3;
+#pragma unroll
+                    for (int g = 0; g < kH / 4; ++g) {
+                        float x[4] = {__uint_as_float(o[4 * g]), __uint_as_float(o[4 * g + 1]),
+                                      __uint_as_float(o[4 * g + 2]), __uint_as_float(o[4 * g + 3])};
+#pragma unroll
+                        for (int msk = 1; msk <= 2; msk <<= 1) {
+                            const bool hi = (j & msk) != 0;
+#pragma unroll
+                            for (int k = 0; k < 4; ++k) {
+                                if (k & msk) continue;
+                                const float send = hi ? x[k] : x[k + msk];
+                                const float recv = __shfl_xor_sync(0xffffffffu, send, msk);
+                                if (hi) x[k] = recv;
+                                else x[k + msk] = recv;
+                            }
+                        }
+                        *reinterpret_cast<float4*>(dst + (4 * g + j) * kD + (d - j)) = make_float4(x[0], x[1], x[2], x[3]);
                     }
                 } else {
                     // a piece is stored in the order the threads hold it (piece layout): one warp store
