@@ -173,90 +173,103 @@ __device__ __forceinline__ void fault(Smem<T>& sm, const TcArgs& a) {
 // ---------------------------------------------------------------------
 // warp 0: loads
 // ---------------------------------------------------------------------
-// candidate rows of one CSA tile: lane owns rows lane and lane+32
+// The rows of a gathered tile are worked out in two steps, so the index (or block-table) loads of the
+// next tile are in flight while this tile's copies are issued: fetch_rows issues them (rows lane and
+// lane + 32 of the tile), resolve_rows turns what they returned into row pointers.  RowInfo is the
+// query row's, taken once per query row.
+struct RowFetch {
+    long long v[2];  // CSA: the selection (-1: none); paged HCA: the block id; ring: unused
+    bool gath;       // the tile is gathered (false: loaded as a contiguous box)
+};
+
 template <int T>
-__device__ __forceinline__ void csa_rows(const TcArgs& a, const RowInfo& ri, int row, long long c0, int lane,
-                                         const __nv_bfloat16* (&src)[2], bool (&ok)[2]) {
+__device__ __forceinline__ RowFetch fetch_rows(const TcArgs& a, const RowInfo& ri, int row, int ti, int lane) {
     using C = Tiles<T>;
+    RowFetch f;
+    f.gath = tile_gathered(a, ti);
+    f.v[0] = f.v[1] = -1;
+    if (!f.gath || ti >= a.e_tiles) return f;
 #pragma unroll
     for (int h2 = 0; h2 < 2; ++h2) {
-        const long long c = c0 + lane + 32 * h2;
-        const long long sidx = (c < a.k && lane + 32 * h2 < C::kTile) ? (long long)a.idx[(long long)row * a.k + c] : -1;
-        ok[h2] = sidx >= 0 && sidx < ri.nvis;
-        const __nv_bfloat16* er = ok[h2] ? entry_row(a, ri.b, sidx) : nullptr;
-        if (ok[h2] && !er) {  // a block id outside the pool: skipped and reported
-            ok[h2] = false;
-            if (a.dev_status) atomicExch(a.dev_status, (int)V4A_ERR_DEVICE_FAULT);
+        const int r = lane + 32 * h2;
+        const long long c = (long long)ti * C::kTile + r;
+        if (r >= C::kTile) continue;
+        if (a.idx) {
+            if (c < a.k) f.v[h2] = a.idx[(long long)row * a.k + c];
+        } else if (c < ri.nvis) {  // HCA over a paged pool: entries c0 .. c0 + T - 1 through the block table
+            f.v[h2] = a.bt[(long long)ri.b * a.bt_stride + c / a.epb];
         }
-        // an excluded row still gets finite data: this query's head-0 row of q
-        src[h2] = ok[h2] ? er : a.q + (long long)row * kH * kD;
+    }
+    return f;
+}
+
+// Row pointers (src) and participation (ok) of this lane's rows of a gathered tile from fetch_rows'
+// values.  Bad selections and block ids are reported; an excluded row still gets finite data (this
+// query's head-0 row of q).
+template <int T>
+__device__ __forceinline__ void resolve_rows(const TcArgs& a, const RowInfo& ri, int row, int ti, int lane,
+                                             const RowFetch& f, const __nv_bfloat16* (&src)[2], bool (&ok)[2]) {
+    using C = Tiles<T>;
+    const __nv_bfloat16* fallback = a.q + (long long)row * kH * kD;
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2) {
+        const int r = lane + 32 * h2;
+        const __nv_bfloat16* er = nullptr;
+        bool bad = false;
+        if (r < C::kTile) {
+            if (ti < a.e_tiles) {
+                if (a.idx) {
+                    const long long sidx = f.v[h2];
+                    if (sidx >= 0 && sidx < ri.nvis) {
+                        er = entry_row(a, ri.b, sidx);
+                        bad = er == nullptr;  // a block id outside the pool
+                    } else {
+                        bad = sidx != -1;  // neither a selection nor the -1 filler
+                    }
+                } else {
+                    const long long s = (long long)ti * C::kTile + r;
+                    if (s < ri.nvis) {
+                        const long long blk = f.v[h2];
+                        if (blk >= 0 && blk < a.n_blocks) er = a.entries + (blk * a.epb + s % a.epb) * kD;
+                        else bad = true;
+                    }
+                }
+            } else {
+                // window tokens p0 .. p0 + T - 1 from the ring (they may wrap around its end)
+                const long long wi = ti - a.e_tiles;
+                const long long p = ri.t - a.window + 1 + wi * C::kTile + r;
+                if (wi * C::kTile + r < a.window && p >= 0)
+                    er = a.token_kv + ((long long)ri.b * a.ring_rows + p % a.ring_rows) * kD;
+            }
+        }
+        if (bad && a.dev_status) atomicExch(a.dev_status, (int)V4A_ERR_DEVICE_FAULT);
+        ok[h2] = er != nullptr;
+        src[h2] = ok[h2] ? er : fallback;
     }
 }
 
-// cp.async all T rows of a tile (lane owns rows lane and lane+32: src / ok) into the 128-byte-swizzled
-// stage; returns the tile's row mask
+// cp.async all T rows of a tile (lane owns the pointers of rows lane and lane + 32: src / ok) into the
+// 128-byte-swizzled stage, eight lanes per row: lane l copies 16-byte chunk l % 8 of every slab of rows
+// l / 8, l / 8 + 4, ..., so each warp copy is four whole 128-byte lines and each row pointer is shuffled
+// once for eight copies.  Returns the tile's row mask.
 template <int T>
 __device__ __forceinline__ uint64_t gather_tile(uint8_t* dst, const __nv_bfloat16* const (&src)[2], const bool (&ok)[2],
                                                 int lane, uint64_t policy) {
     using C = Tiles<T>;
     const uint64_t mask =
         (uint64_t)__ballot_sync(0xffffffffu, ok[0]) | ((uint64_t)__ballot_sync(0xffffffffu, ok[1]) << 32);
-    for (int r = 0; r < C::kTile; ++r) {
-        const __nv_bfloat16* rs =
-            (const __nv_bfloat16*)__shfl_sync(0xffffffffu, (unsigned long long)(r < 32 ? src[0] : src[1]), r & 31);
+    const int rl = lane >> 3, k = lane & 7;
+#pragma unroll 4
+    for (int i = 0; i < C::kTile / 4; ++i) {
+        const int r = 4 * i + rl;
+        // rows 0..31 are the lanes' first rows, rows 32..63 their second (i is the same in every lane)
+        const unsigned long long pr = __shfl_sync(0xffffffffu, (unsigned long long)(i < 8 ? src[0] : src[1]), r & 31);
+        const __nv_bfloat16* rs = (const __nv_bfloat16*)pr + k * 8;
+        uint8_t* d = dst + r * 128 + ((k ^ (r & 7)) << 4);
 #pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-            const int u = lane + 32 * h2;  // 16-byte chunk of the 1 KB row
-            uint8_t* d = dst + (u >> 3) * C::kSlabBytes + r * 128 + (((u & 7) ^ (r & 7)) << 4);
-            tc::cp_async_16_hint(d, rs + u * 8, policy);
-        }
+        for (int c = 0; c < kSlabs; ++c) tc::cp_async_16_hint(d + c * C::kSlabBytes, rs + c * 64, policy);
     }
     return mask;
-}
-
-// Rows of a gathered tile (CSA selections, paged entries, ring windows) for this lane: rows lane and
-// lane + 32 (src, ok).  False for tiles loaded with TMA.  Bad selections and block ids are reported here.
-template <int T>
-__device__ __forceinline__ bool tile_rows(const TcArgs& a, int row, int ti, int lane, const __nv_bfloat16* (&src)[2],
-                                          bool (&ok)[2]) {
-    using C = Tiles<T>;
-    if (!tile_gathered(a, ti)) return false;
-    const RowInfo ri = row_info(row, a);
-    const __nv_bfloat16* fallback = a.q + (long long)row * kH * kD;  // finite data for excluded rows
-    if (ti < a.e_tiles) {
-        const long long c0 = (long long)ti * C::kTile;
-        if (a.idx) {
-            csa_rows<T>(a, ri, row, c0, lane, src, ok);
-#pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-                const long long c = c0 + lane + 32 * h2;
-                const long long sidx = (c < a.k && lane + 32 * h2 < C::kTile) ? (long long)a.idx[(long long)row * a.k + c] : -1;
-                if (!ok[h2] && sidx != -1 && a.dev_status) atomicExch(a.dev_status, (int)V4A_ERR_DEVICE_FAULT);
-            }
-        } else {
-            // HCA over a paged pool: rows c0 .. c0+63 through the block table
-#pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-                const long long s = c0 + lane + 32 * h2;
-                const __nv_bfloat16* er = (s < ri.nvis && lane + 32 * h2 < C::kTile) ? entry_row(a, ri.b, s) : nullptr;
-                if (s < ri.nvis && !er && a.dev_status) atomicExch(a.dev_status, (int)V4A_ERR_DEVICE_FAULT);
-                ok[h2] = er != nullptr;
-                src[h2] = ok[h2] ? er : fallback;
-            }
-        }
-    } else {
-        // window tokens p0 .. p0+63 from the ring (they may wrap around its end)
-        const long long wi = ti - a.e_tiles;
-        const long long p0 = ri.t - a.window + 1 + wi * C::kTile;
-#pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-            const int r = lane + 32 * h2;
-            const long long p = p0 + r;
-            ok[h2] = r < C::kTile && wi * C::kTile + r < a.window && p >= 0;
-            src[h2] = ok[h2] ? a.token_kv + ((long long)ri.b * a.ring_rows + p % a.ring_rows) * kD : fallback;
-        }
-    }
-    return true;
 }
 
 // Warp 0 lane 0, before the grid dependency wait: the query of the CTA's first segment and an L2
@@ -286,28 +299,33 @@ __device__ void producer(Smem<T>& sm, const TcArgs& a, const CUtensorMap* ent_ma
     const int lane = threadIdx.x & 31;
     int seg = 0;
     Cursor cur(f0, a.tpr);
-    const uint64_t stream_policy = tc::l2_evict_first();  // candidate rows are read once per call
+    // candidate rows: read once per call in decode, shared by the queries of a chunk in prefill
+    const uint64_t stream_policy = tc::l2_stream_policy(a.n_q);
     int last_load[C::kStages];  // the last tile whose copies went into each stage (-1: none)
     for (int i = 0; i < C::kStages; ++i) last_load[i] = -1;
-    // the rows of gathered tiles are worked out a tile ahead, so their index / block-table loads overlap
-    // the current tile's copies
-    const __nv_bfloat16* nsrc[2] = {a.q, a.q};
-    bool nok[2] = {false, false};
-    bool ngath = f0 < f1 && tile_rows<T>(a, cur.row, cur.ti, lane, nsrc, nok);
+    // the rows of gathered tiles are fetched a tile ahead and resolved once this tile's copies are issued,
+    // so the index / block-table loads overlap the copies
+    RowInfo ri = {0, 0, 0};
+    RowFetch fc = {{-1, -1}, false};
+    const __nv_bfloat16* src[2] = {a.q, a.q};
+    bool ok[2] = {false, false};
+    if (f0 < f1) {
+        ri = row_info(cur.row, a);
+        fc = fetch_rows<T>(a, ri, cur.row, cur.ti, lane);
+        if (fc.gath) resolve_rows<T>(a, ri, cur.row, cur.ti, lane, fc, src, ok);
+    }
     for (long long f = f0; f < f1; ++f, cur.next(a.tpr)) {
         if (sm.abort_flag) break;
         const int jt = (int)(f - f0), st = jt % C::kStages;
         const int row = cur.row, ti = cur.ti;
         const bool seg_start = (f == f0) || (ti == 0);
-        const RowInfo ri = row_info(row, a);
-        const bool gath = ngath;
-        const __nv_bfloat16* src[2] = {nsrc[0], nsrc[1]};
-        const bool ok[2] = {nok[0], nok[1]};
-        if (f + 1 < f1) {
-            Cursor nx = cur;
-            nx.next(a.tpr);
-            ngath = tile_rows<T>(a, nx.row, nx.ti, lane, nsrc, nok);
-        }
+        const bool gath = fc.gath;
+        Cursor nx = cur;
+        nx.next(a.tpr);
+        const bool more = f + 1 < f1;
+        const RowInfo nri = (more && nx.row != row) ? row_info(nx.row, a) : ri;
+        RowFetch fn = {{-1, -1}, false};
+        if (more) fn = fetch_rows<T>(a, nri, nx.row, nx.ti, lane);
         if (seg_start) {
             if (seg > 0 && !tc::mbar_wait(&sm.q_empty, (seg - 1) & 1, a.wait_polls)) { fault(sm, a); break; }
             if (lane == 0 && seg > 0) {  // the first segment's query was requested before the dependency wait
@@ -317,45 +335,49 @@ __device__ void producer(Smem<T>& sm, const TcArgs& a, const CUtensorMap* ent_ma
             ++seg;
         }
         if (jt >= C::kStages && !tc::mbar_wait(&sm.kv_empty[st], ((jt / C::kStages) - 1) & 1, a.wait_polls)) { fault(sm, a); break; }
-        uint64_t mask = 0;
         uint8_t* dst = sm.kv[st];
-        if (jt == a.withhold) continue;  // test hook: this stage never fills (no copy, no arrival)
-        last_load[st] = jt;
-        if (gath) {
-            mask = gather_tile<T>(dst, src, ok, lane, stream_policy);
-            if (lane == 0) {
-                sm.mask[st] = mask;
-                tc::mbar_arrive_expect_tx(&sm.kv_full[st], 0);
+        if (jt != a.withhold) {  // test hook: the withheld stage never fills (no copy, no arrival)
+            last_load[st] = jt;
+            uint64_t mask = 0;
+            if (gath) {
+                mask = gather_tile<T>(dst, src, ok, lane, stream_policy);
+                if (lane == 0) {
+                    sm.mask[st] = mask;
+                    tc::mbar_arrive_expect_tx(&sm.kv_full[st], 0);
+                }
+            } else if (ti < a.e_tiles) {
+                // HCA: rows c0 .. c0+T-1 of this sequence's entries are contiguous
+                const long long c0 = (long long)ti * C::kTile;
+                const long long nv = ri.nvis - c0;
+                mask = nv >= C::kTile ? C::kTileMask : (nv <= 0 ? 0ull : ((1ull << nv) - 1ull));
+                if (lane == 0) {
+                    sm.mask[st] = mask;
+                    tc::mbar_arrive_expect_tx(&sm.kv_full[st], C::kTileBytes);
+                    const int y = (int)((long long)ri.b * a.n_ent + c0);
+                    for (int c = 0; c < kSlabs; ++c)
+                        tc::tma_load_2d_hint(dst + c * C::kSlabBytes, ent_map, 64 * c, y, &sm.kv_full[st], stream_policy);
+                }
+            } else {
+                // window tokens p0 .. p0+T-1 (contiguous rows of token_kv)
+                const long long wi = ti - a.e_tiles;
+                const long long p0 = ri.t - a.window + 1 + wi * C::kTile;
+                for (int r = 0; r < C::kTile; ++r) {
+                    const long long p = p0 + r;
+                    if (wi * C::kTile + r < a.window && p >= 0) mask |= 1ull << r;
+                }
+                if (lane == 0) {
+                    sm.mask[st] = mask;
+                    tc::mbar_arrive_expect_tx(&sm.kv_full[st], C::kTileBytes);
+                    const int y = (int)((long long)ri.b * a.l_tok + (p0 - a.tok_pos0));
+                    for (int c = 0; c < kSlabs; ++c)
+                        tc::tma_load_2d_hint(dst + c * C::kSlabBytes, tok_map, 64 * c, y, &sm.kv_full[st], stream_policy);
+                }
             }
-        } else if (ti < a.e_tiles) {
-            // HCA: rows c0 .. c0+63 of this sequence's entries are contiguous
-            const long long c0 = (long long)ti * C::kTile;
-            const long long nv = ri.nvis - c0;
-            mask = nv >= C::kTile ? C::kTileMask : (nv <= 0 ? 0ull : ((1ull << nv) - 1ull));
-            if (lane == 0) {
-                sm.mask[st] = mask;
-                tc::mbar_arrive_expect_tx(&sm.kv_full[st], C::kTileBytes);
-                const int y = (int)((long long)ri.b * a.n_ent + c0);
-                for (int c = 0; c < kSlabs; ++c)
-                    tc::tma_load_2d_hint(dst + c * C::kSlabBytes, ent_map, 64 * c, y, &sm.kv_full[st], stream_policy);
-            }
-        } else {
-            // window tokens p0 .. p0+63 (contiguous rows of token_kv)
-            const long long wi = ti - a.e_tiles;
-            const long long p0 = ri.t - a.window + 1 + wi * C::kTile;
-            for (int r = 0; r < C::kTile; ++r) {
-                const long long p = p0 + r;
-                if (wi * C::kTile + r < a.window && p >= 0) mask |= 1ull << r;
-            }
-            if (lane == 0) {
-                sm.mask[st] = mask;
-                tc::mbar_arrive_expect_tx(&sm.kv_full[st], C::kTileBytes);
-                const int y = (int)((long long)ri.b * a.l_tok + (p0 - a.tok_pos0));
-                for (int c = 0; c < kSlabs; ++c)
-                    tc::tma_load_2d_hint(dst + c * C::kSlabBytes, tok_map, 64 * c, y, &sm.kv_full[st], stream_policy);
-            }
+            tc::cp_async_arrive_noinc(&sm.kv_full[st]);  // 32 lanes: after their cp.async copies (if any) land
         }
-        tc::cp_async_arrive_noinc(&sm.kv_full[st]);  // 32 lanes: after their cp.async copies (if any) land
+        if (more && fn.gath) resolve_rows<T>(a, nri, nx.row, nx.ti, lane, fn, src, ok);
+        ri = nri;
+        fc = fn;
     }
     // make sure nothing this warp started is still in flight before the CTA retires (also after an abort
     // or a withheld stage: the last copies issued into each stage)

@@ -214,7 +214,8 @@ __device__ void idx_producer(IdxSmem& sm, const IdxTcArgs& a, const CUtensorMap*
     const long long n = f1 - f0;
     const int nb = a.bt ? kTileK / a.epb : 0;
     int rows[kMaxB], next_rows[kMaxB];
-    const uint64_t pol = tc::l2_evict_first();  // key tiles are read once per call
+    // key tiles: read once per call unless several query groups of a sequence share them
+    const uint64_t pol = tc::l2_stream_policy(a.ngroups);
     if (a.bt && n > 0) fetch_block_rows<kMaxB>(a, cur.bat, (long long)cur.ti * kTileK, nb, next_rows);
     for (long long jt = 0; jt < n; ++jt, cur.next(a)) {
         if (a.bt) {
@@ -639,7 +640,8 @@ __device__ void mx_producer(IdxSmem& sm, const IdxTcArgs& a, const CUtensorMap* 
     const long long n = f1 - f0;
     const int nb = a.bt ? kMxTile / a.epb : 0;
     int rows[kMaxB], next_rows[kMaxB];
-    const uint64_t pol = tc::l2_evict_first();  // key tiles are read once per call
+    // key tiles: read once per call unless several query groups of a sequence share them
+    const uint64_t pol = tc::l2_stream_policy(a.ngroups);
     if (a.bt && n > 0) fetch_block_rows<kMaxB>(a, cur.bat, (long long)cur.ti * kMxTile, nb, next_rows);
     for (long long jt = 0; jt < n; ++jt, cur.next(a)) {
         if (a.bt) {

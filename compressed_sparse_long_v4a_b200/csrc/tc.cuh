@@ -87,6 +87,17 @@ __device__ __forceinline__ uint64_t l2_evict_first() {
     asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
     return p;
 }
+// L2 policy for data that other CTAs of the same call read again (the keys and entries of a prefill
+// chunk, shared by all its queries): plain LRU
+__device__ __forceinline__ uint64_t l2_evict_normal() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+// the policy for an operand read by `readers` query groups of one call
+__device__ __forceinline__ uint64_t l2_stream_policy(int readers) {
+    return readers > 1 ? l2_evict_normal() : l2_evict_first();
+}
 // tma_load_2d with an L2 cache policy
 __device__ __forceinline__ void tma_load_2d_hint(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar,
                                                  uint64_t policy) {
