@@ -45,7 +45,9 @@ constexpr uint32_t kPBytes = kH * 128;           // 64 heads x up to 64 rows bf1
 constexpr uint32_t kColO = 0;                    // O^T: 4 chunks of 64 columns
 constexpr uint32_t kColS = 256;                  // S: 2 buffers of 64 columns
 constexpr uint32_t kTmemCols = 512;
-constexpr int kThreads = 192;
+// Warps: 0 (and 6, when two warps gather) loads, 1 issues the MMAs, 2-5 run the softmax and the output.
+template <int G>
+constexpr int threads_for() { return 32 * (5 + G); }
 constexpr float kRescaleSlack = 8.0f;  // keep a stale running max until the true one exceeds it by 2^8
 // Piece layout: a piece (partial O of a query split between CTAs) holds O[h][d] for 64 heads x 512
 // dims as float4 groups of four heads: the group of heads 4i .. 4i+3 at dim d is float4 number
@@ -174,24 +176,25 @@ __device__ __forceinline__ void fault(Smem<T>& sm, const TcArgs& a) {
 // warp 0: loads
 // ---------------------------------------------------------------------
 // The rows of a gathered tile are worked out in two steps, so the index (or block-table) loads of the
-// next tile are in flight while this tile's copies are issued: fetch_rows issues them (rows lane and
-// lane + 32 of the tile), resolve_rows turns what they returned into row pointers.  RowInfo is the
-// query row's, taken once per query row.
+// next tiles are in flight while this tile's copies are issued: fetch_rows issues them, resolve_rows
+// turns what they returned into row pointers.  RowInfo is the query row's, taken once per query row.
+// With G loading warps, warp `part` owns rows 32 (h2 + part) + lane, h2 < 2 / G, of every tile: one
+// warp owns rows lane and lane + 32, two warps own 32 rows each.
 struct RowFetch {
     long long v[2];  // CSA: the selection (-1: none); paged HCA: the block id; ring: unused
     bool gath;       // the tile is gathered (false: loaded as a contiguous box)
 };
 
-template <int T>
-__device__ __forceinline__ RowFetch fetch_rows(const TcArgs& a, const RowInfo& ri, int row, int ti, int lane) {
+template <int T, int G>
+__device__ __forceinline__ RowFetch fetch_rows(const TcArgs& a, const RowInfo& ri, int row, int ti, int lane, int part) {
     using C = Tiles<T>;
     RowFetch f;
     f.gath = tile_gathered(a, ti);
     f.v[0] = f.v[1] = -1;
     if (!f.gath || ti >= a.e_tiles) return f;
 #pragma unroll
-    for (int h2 = 0; h2 < 2; ++h2) {
-        const int r = lane + 32 * h2;
+    for (int h2 = 0; h2 < 2 / G; ++h2) {
+        const int r = lane + 32 * (h2 + part);
         const long long c = (long long)ti * C::kTile + r;
         if (r >= C::kTile) continue;
         if (a.idx) {
@@ -206,14 +209,14 @@ __device__ __forceinline__ RowFetch fetch_rows(const TcArgs& a, const RowInfo& r
 // Row pointers (src) and participation (ok) of this lane's rows of a gathered tile from fetch_rows'
 // values.  Bad selections and block ids are reported; an excluded row still gets finite data (this
 // query's head-0 row of q).
-template <int T>
-__device__ __forceinline__ void resolve_rows(const TcArgs& a, const RowInfo& ri, int row, int ti, int lane,
+template <int T, int G>
+__device__ __forceinline__ void resolve_rows(const TcArgs& a, const RowInfo& ri, int row, int ti, int lane, int part,
                                              const RowFetch& f, const __nv_bfloat16* (&src)[2], bool (&ok)[2]) {
     using C = Tiles<T>;
     const __nv_bfloat16* fallback = a.q + (long long)row * kH * kD;
 #pragma unroll
-    for (int h2 = 0; h2 < 2; ++h2) {
-        const int r = lane + 32 * h2;
+    for (int h2 = 0; h2 < 2 / G; ++h2) {
+        const int r = lane + 32 * (h2 + part);
         const __nv_bfloat16* er = nullptr;
         bool bad = false;
         if (r < C::kTile) {
@@ -248,22 +251,25 @@ __device__ __forceinline__ void resolve_rows(const TcArgs& a, const RowInfo& ri,
     }
 }
 
-// cp.async all T rows of a tile (lane owns the pointers of rows lane and lane + 32: src / ok) into the
-// 128-byte-swizzled stage, eight lanes per row: lane l copies 16-byte chunk l % 8 of every slab of rows
-// l / 8, l / 8 + 4, ..., so each warp copy is four whole 128-byte lines and each row pointer is shuffled
-// once for eight copies.  Returns the tile's row mask.
-template <int T>
+// cp.async this warp's rows of a tile (src / ok from resolve_rows) into the 128-byte-swizzled stage,
+// eight lanes per row: lane l copies 16-byte chunk l % 8 of every slab of rows 4 i + l / 8, so each warp
+// copy is four whole 128-byte lines and each row pointer is shuffled once for eight copies.  Returns the
+// warp's rows' bits of the tile's row mask.
+template <int T, int G>
 __device__ __forceinline__ uint64_t gather_tile(uint8_t* dst, const __nv_bfloat16* const (&src)[2], const bool (&ok)[2],
-                                                int lane, uint64_t policy) {
+                                                int lane, int part, uint64_t policy) {
     using C = Tiles<T>;
-    const uint64_t mask =
-        (uint64_t)__ballot_sync(0xffffffffu, ok[0]) | ((uint64_t)__ballot_sync(0xffffffffu, ok[1]) << 32);
+    uint64_t mask = 0;
+#pragma unroll
+    for (int h2 = 0; h2 < 2 / G; ++h2) mask |= (uint64_t)__ballot_sync(0xffffffffu, ok[h2]) << (32 * (h2 + part));
     const int rl = lane >> 3, k = lane & 7;
+    const int i0 = 8 * part, i1 = (8 * (part + 2 / G) < C::kTile / 4) ? 8 * (part + 2 / G) : C::kTile / 4;
 #pragma unroll 4
-    for (int i = 0; i < C::kTile / 4; ++i) {
+    for (int i = i0; i < i1; ++i) {
         const int r = 4 * i + rl;
-        // rows 0..31 are the lanes' first rows, rows 32..63 their second (i is the same in every lane)
-        const unsigned long long pr = __shfl_sync(0xffffffffu, (unsigned long long)(i < 8 ? src[0] : src[1]), r & 31);
+        // row r is lane r % 32's row number r / 32 - part (i is the same in every lane)
+        const unsigned long long pr =
+            __shfl_sync(0xffffffffu, (unsigned long long)((i >> 3) == part ? src[0] : src[1]), r & 31);
         const __nv_bfloat16* rs = (const __nv_bfloat16*)pr + k * 8;
         uint8_t* d = dst + r * 128 + ((k ^ (r & 7)) << 4);
 #pragma unroll
@@ -292,9 +298,11 @@ __device__ void early_loads(Smem<T>& sm, const TcArgs& a, const CUtensorMap* ent
     }
 }
 
-template <int T>
+// Loading warp `part` of G.  Part 0 also loads the queries and the contiguous tiles; with two loading
+// warps each gathers its 32 rows of a gathered tile and writes its half of the row mask.
+template <int T, int G>
 __device__ void producer(Smem<T>& sm, const TcArgs& a, const CUtensorMap* ent_map, const CUtensorMap* tok_map,
-                         const CUtensorMap* q_map, long long f0, long long f1) {
+                         const CUtensorMap* q_map, long long f0, long long f1, int part) {
     using C = Tiles<T>;
     const int lane = threadIdx.x & 31;
     int seg = 0;
@@ -303,36 +311,38 @@ __device__ void producer(Smem<T>& sm, const TcArgs& a, const CUtensorMap* ent_ma
     const uint64_t stream_policy = tc::l2_stream_policy(a.n_q);
     int last_load[C::kStages];  // the last tile whose copies went into each stage (-1: none)
     for (int i = 0; i < C::kStages; ++i) last_load[i] = -1;
-    // the rows of gathered tiles are fetched a tile ahead and resolved once this tile's copies are issued,
-    // so the index / block-table loads overlap the copies
-    RowInfo ri = {0, 0, 0};
-    RowFetch fc = {{-1, -1}, false};
+    // The rows of gathered tiles are fetched two tiles ahead (their index / block-table loads queue behind
+    // a whole tile's copies) and resolved into row pointers once the current tile's copies are issued.
+    // c1, c2: the next two tiles; ri, ri1, ri2: their query rows' info.
+    Cursor c1 = cur, c2 = cur;
+    c1.next(a.tpr);
+    c2.next(a.tpr);
+    c2.next(a.tpr);
+    RowInfo ri = {0, 0, 0}, ri1 = {0, 0, 0};
+    RowFetch fn1 = {{-1, -1}, false};
+    bool gath = false;  // the current tile is gathered
     const __nv_bfloat16* src[2] = {a.q, a.q};
     bool ok[2] = {false, false};
     if (f0 < f1) {
         ri = row_info(cur.row, a);
-        fc = fetch_rows<T>(a, ri, cur.row, cur.ti, lane);
-        if (fc.gath) resolve_rows<T>(a, ri, cur.row, cur.ti, lane, fc, src, ok);
+        const RowFetch fc = fetch_rows<T, G>(a, ri, cur.row, cur.ti, lane, part);
+        if (f0 + 1 < f1) {
+            ri1 = c1.row != cur.row ? row_info(c1.row, a) : ri;
+            fn1 = fetch_rows<T, G>(a, ri1, c1.row, c1.ti, lane, part);
+        }
+        gath = fc.gath;
+        if (gath) resolve_rows<T, G>(a, ri, cur.row, cur.ti, lane, part, fc, src, ok);
     }
-    for (long long f = f0; f < f1; ++f, cur.next(a.tpr)) {
+    for (long long f = f0; f < f1; ++f) {
         if (sm.abort_flag) break;
         const int jt = (int)(f - f0), st = jt % C::kStages;
         const int row = cur.row, ti = cur.ti;
         const bool seg_start = (f == f0) || (ti == 0);
-        const bool gath = fc.gath;
-        Cursor nx = cur;
-        nx.next(a.tpr);
-        const bool more = f + 1 < f1;
-        const RowInfo nri = (more && nx.row != row) ? row_info(nx.row, a) : ri;
-        RowFetch fn = {{-1, -1}, false};
-        if (more) fn = fetch_rows<T>(a, nri, nx.row, nx.ti, lane);
-        if (seg_start) {
-            if (seg > 0 && !tc::mbar_wait(&sm.q_empty, (seg - 1) & 1, a.wait_polls)) { fault(sm, a); break; }
-            if (lane == 0 && seg > 0) {  // the first segment's query was requested before the dependency wait
-                tc::mbar_arrive_expect_tx(&sm.q_full, kQBytes);
-                for (int c = 0; c < kSlabs; ++c) tc::tma_load_2d(sm.q + c * kH * 128, q_map, 64 * c, row * kH, &sm.q_full);
-            }
-            ++seg;
+        RowInfo ri2 = ri1;
+        RowFetch fn2 = {{-1, -1}, false};
+        if (f + 2 < f1) {
+            if (c2.row != c1.row) ri2 = row_info(c2.row, a);
+            fn2 = fetch_rows<T, G>(a, ri2, c2.row, c2.ti, lane, part);
         }
         if (jt >= C::kStages && !tc::mbar_wait(&sm.kv_empty[st], ((jt / C::kStages) - 1) & 1, a.wait_polls)) { fault(sm, a); break; }
         uint8_t* dst = sm.kv[st];
@@ -340,11 +350,15 @@ __device__ void producer(Smem<T>& sm, const TcArgs& a, const CUtensorMap* ent_ma
             last_load[st] = jt;
             uint64_t mask = 0;
             if (gath) {
-                mask = gather_tile<T>(dst, src, ok, lane, stream_policy);
+                mask = gather_tile<T, G>(dst, src, ok, lane, part, stream_policy);
                 if (lane == 0) {
-                    sm.mask[st] = mask;
-                    tc::mbar_arrive_expect_tx(&sm.kv_full[st], 0);
+                    if (G == 1) sm.mask[st] = mask;
+                    else reinterpret_cast<uint32_t*>(&sm.mask[st])[part] = (uint32_t)(mask >> (32 * part));
+                    if (part == 0) tc::mbar_arrive_expect_tx(&sm.kv_full[st], 0);
+                    else tc::mbar_arrive(&sm.kv_full[st]);
                 }
+            } else if (part > 0) {
+                if (lane == 0) tc::mbar_arrive(&sm.kv_full[st]);  // part 0 loads a contiguous tile alone
             } else if (ti < a.e_tiles) {
                 // HCA: rows c0 .. c0+T-1 of this sequence's entries are contiguous
                 const long long c0 = (long long)ti * C::kTile;
@@ -375,9 +389,23 @@ __device__ void producer(Smem<T>& sm, const TcArgs& a, const CUtensorMap* ent_ma
             }
             tc::cp_async_arrive_noinc(&sm.kv_full[st]);  // 32 lanes: after their cp.async copies (if any) land
         }
-        if (more && fn.gath) resolve_rows<T>(a, nri, nx.row, nx.ti, lane, fn, src, ok);
-        ri = nri;
-        fc = fn;
+        // a new query's rows are on their way; its query replaces the last one's once that one's last QK is done
+        if (seg_start && part == 0) {
+            if (seg > 0 && !tc::mbar_wait(&sm.q_empty, (seg - 1) & 1, a.wait_polls)) { fault(sm, a); break; }
+            if (lane == 0 && seg > 0) {  // the first segment's query was requested before the dependency wait
+                tc::mbar_arrive_expect_tx(&sm.q_full, kQBytes);
+                for (int c = 0; c < kSlabs; ++c) tc::tma_load_2d(sm.q + c * kH * 128, q_map, 64 * c, row * kH, &sm.q_full);
+            }
+            ++seg;
+        }
+        gath = fn1.gath;
+        if (f + 1 < f1 && gath) resolve_rows<T, G>(a, ri1, c1.row, c1.ti, lane, part, fn1, src, ok);
+        ri = ri1;
+        ri1 = ri2;
+        fn1 = fn2;
+        cur = c1;
+        c1 = c2;
+        c2.next(a.tpr);
     }
     // make sure nothing this warp started is still in flight before the CTA retires (also after an abort
     // or a withheld stage: the last copies issued into each stage)
@@ -385,7 +413,7 @@ __device__ void producer(Smem<T>& sm, const TcArgs& a, const CUtensorMap* ent_ma
         if (last_load[st] >= 0) tc::mbar_wait(&sm.kv_full[st], (last_load[st] / C::kStages) & 1, a.wait_polls);
     // ... nor a query load (the first segment's was issued before the loop)
     const int q_loads = seg > 0 ? seg : (f0 < f1 ? 1 : 0);
-    if (q_loads > 0) tc::mbar_wait(&sm.q_full, (q_loads - 1) & 1, a.wait_polls);
+    if (part == 0 && q_loads > 0) tc::mbar_wait(&sm.q_full, (q_loads - 1) & 1, a.wait_polls);
 }
 
 // ---------------------------------------------------------------------
@@ -664,7 +692,9 @@ __device__ void softmax_warps(Smem<T>& sm, const TcArgs& a, uint32_t tmem, long 
                                 else x[k + msk] = recv;
                             }
                         }
-                        *reinterpret_cast<float4*>(dst + (4 * g + j) * kD + (d - j)) = make_float4(x[0], x[1], x[2], x[3]);
+                        // streaming store: the output is not read again here, so it should not push the
+                        // entries that other queries gather out of L2
+                        __stcs(reinterpret_cast<float4*>(dst + (4 * g + j) * kD + (d - j)), make_float4(x[0], x[1], x[2], x[3]));
                     }
                 } else {
                     // a piece is stored in the order the threads hold it (piece layout): one warp store
@@ -691,8 +721,8 @@ __device__ void softmax_warps(Smem<T>& sm, const TcArgs& a, uint32_t tmem, long 
     }
 }
 
-template <int T>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int T, int G>
+__global__ void __launch_bounds__(threads_for<G>(), 1)
     attend_tc_kernel(const __grid_constant__ CUtensorMap ent_map, const __grid_constant__ CUtensorMap tok_map,
                      const __grid_constant__ CUtensorMap q_map, TcArgs a) {
     using C = Tiles<T>;
@@ -704,7 +734,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < C::kStages; ++i) {
-            tc::mbar_init(&sm.kv_full[i], 33);  // 1 expect_tx arrival + 32 cp.async arrivals
+            tc::mbar_init(&sm.kv_full[i], 33 * G);  // per loading warp: lane 0's arrival + 32 cp.async arrivals
             tc::mbar_init(&sm.kv_empty[i], 1);
         }
         for (int i = 0; i < 2; ++i) {
@@ -730,8 +760,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // SMs to free up (measured on B200: the 32-query combine ran 1.8 us faster, the step 2 us faster).
     const uint32_t tmem = sm.tmem_base;
 
-    if (warp == 0) {
-        producer(sm, a, &ent_map, &tok_map, &q_map, f0, f1);
+    if (warp == 0 || warp == 6) {
+        producer<T, G>(sm, a, &ent_map, &tok_map, &q_map, f0, f1, warp == 0 ? 0 : 1);
     } else if (warp == 1) {
         mma_issuer(sm, a, tmem, f0, f1);
     } else {
@@ -988,15 +1018,22 @@ cudaError_t launch_attend_tc(const AttendArgs& a, void* ws, size_t ws_bytes, cud
         t.comb_pieces = (int)(bound < p.grid ? bound : p.grid);
     }
 
-    auto go = [&](auto kernel, size_t smem) {
+    auto go = [&](auto kernel, size_t smem, int threads) {
         cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (err == cudaSuccess)
-            err = launch_pdl(kernel, dim3(p.grid), dim3(kThreads), smem, stream, ent_map, tok_map, q_map, t);
+            err = launch_pdl(kernel, dim3(p.grid), dim3(threads), smem, stream, ent_map, tok_map, q_map, t);
         return err == cudaSuccess ? cudaGetLastError() : err;
     };
     static_assert(sizeof(Smem<48>) + 1024 <= 232448 && sizeof(Smem<64>) + 1024 <= 232448, "shared memory");
-    cudaError_t e = p.tile == 48 ? go(attend_tc_kernel<48>, sizeof(Smem<48>) + 1024)
-                                 : go(attend_tc_kernel<64>, sizeof(Smem<64>) + 1024);
+    // tiles gathered row by row get a second loading warp
+    const bool gathered = a.idx != nullptr || a.bt != nullptr || a.ring_rows > 0;
+    cudaError_t e;
+    if (p.tile == 48)
+        e = gathered ? go(attend_tc_kernel<48, 2>, sizeof(Smem<48>) + 1024, threads_for<2>())
+                     : go(attend_tc_kernel<48, 1>, sizeof(Smem<48>) + 1024, threads_for<1>());
+    else
+        e = gathered ? go(attend_tc_kernel<64, 2>, sizeof(Smem<64>) + 1024, threads_for<2>())
+                     : go(attend_tc_kernel<64, 1>, sizeof(Smem<64>) + 1024, threads_for<1>());
     if (e != cudaSuccess) return e;
     if (p.grid > 1) {
         const size_t csm = (size_t)t.comb_pieces * kH * sizeof(float);
