@@ -289,12 +289,12 @@ __device__ void early_loads(Smem<T>& sm, const TcArgs& a, const CUtensorMap* ent
     using C = Tiles<T>;
     const Cursor cur(f0, a.tpr);
     tc::mbar_arrive_expect_tx(&sm.q_full, kQBytes);
-    for (int c = 0; c < kSlabs; ++c) tc::tma_load_2d(sm.q + c * kH * 128, q_map, 64 * c, cur.row * kH, &sm.q_full);
+    tc::tma_load_3d(sm.q, q_map, 0, cur.row * kH, 0, &sm.q_full);
     if (a.idx || a.bt) return;
     const RowInfo ri = row_info(cur.row, a);
     for (int j = 0; j < C::kStages && f0 + j < f1 && cur.ti + j < a.e_tiles; ++j) {
         const int y = (int)((long long)ri.b * a.n_ent + (long long)(cur.ti + j) * C::kTile);
-        for (int c = 0; c < kSlabs; ++c) tc::tma_prefetch_2d(ent_map, 64 * c, y);
+        tc::tma_prefetch_3d(ent_map, 0, y, 0);
     }
 }
 
@@ -368,8 +368,7 @@ __device__ void producer(Smem<T>& sm, const TcArgs& a, const CUtensorMap* ent_ma
                     sm.mask[st] = mask;
                     tc::mbar_arrive_expect_tx(&sm.kv_full[st], C::kTileBytes);
                     const int y = (int)((long long)ri.b * a.n_ent + c0);
-                    for (int c = 0; c < kSlabs; ++c)
-                        tc::tma_load_2d_hint(dst + c * C::kSlabBytes, ent_map, 64 * c, y, &sm.kv_full[st], stream_policy);
+                    tc::tma_load_3d_hint(dst, ent_map, 0, y, 0, &sm.kv_full[st], stream_policy);
                 }
             } else {
                 // window tokens p0 .. p0+T-1 (contiguous rows of token_kv)
@@ -383,8 +382,7 @@ __device__ void producer(Smem<T>& sm, const TcArgs& a, const CUtensorMap* ent_ma
                     sm.mask[st] = mask;
                     tc::mbar_arrive_expect_tx(&sm.kv_full[st], C::kTileBytes);
                     const int y = (int)((long long)ri.b * a.l_tok + (p0 - a.tok_pos0));
-                    for (int c = 0; c < kSlabs; ++c)
-                        tc::tma_load_2d_hint(dst + c * C::kSlabBytes, tok_map, 64 * c, y, &sm.kv_full[st], stream_policy);
+                    tc::tma_load_3d_hint(dst, tok_map, 0, y, 0, &sm.kv_full[st], stream_policy);
                 }
             }
             tc::cp_async_arrive_noinc(&sm.kv_full[st]);  // 32 lanes: after their cp.async copies (if any) land
@@ -394,7 +392,7 @@ __device__ void producer(Smem<T>& sm, const TcArgs& a, const CUtensorMap* ent_ma
             if (seg > 0 && !tc::mbar_wait(&sm.q_empty, (seg - 1) & 1, a.wait_polls)) { fault(sm, a); break; }
             if (lane == 0 && seg > 0) {  // the first segment's query was requested before the dependency wait
                 tc::mbar_arrive_expect_tx(&sm.q_full, kQBytes);
-                for (int c = 0; c < kSlabs; ++c) tc::tma_load_2d(sm.q + c * kH * 128, q_map, 64 * c, row * kH, &sm.q_full);
+                tc::tma_load_3d(sm.q, q_map, 0, row * kH, 0, &sm.q_full);
             }
             ++seg;
         }
@@ -904,15 +902,18 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// [rows][512] bf16, boxes of 64 columns x box_rows rows, 128-byte swizzle
+// [rows][512] bf16 viewed as (64 columns, rows, 8 slabs of 64 columns): the row stride is 1 KB and the
+// slab stride 128 bytes, so every address the view reaches lies inside the [rows][512] array.  One box of
+// 64 columns x box_rows rows x 8 slabs lands in shared memory as 8 slabs of box_rows 128-byte rows, the
+// tile layout (128-byte swizzle), in one TMA instruction.
 bool make_map(CUtensorMap* map, const void* base, long long rows, int box_rows) {
     auto fn = encode_fn();
     if (!fn || rows < 1) return false;
-    cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)kD * 2};
-    cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+    cuuint64_t dims[3] = {64, (cuuint64_t)rows, (cuuint64_t)kSlabs};
+    cuuint64_t strides[2] = {(cuuint64_t)kD * 2, 128};
+    cuuint32_t box[3] = {64, (cuuint32_t)box_rows, (cuuint32_t)kSlabs};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
