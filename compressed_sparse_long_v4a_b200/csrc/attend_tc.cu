@@ -780,10 +780,13 @@ __global__ void __launch_bounds__(threads_for<G>(), 1)
 // 4w+32 .. 4w+35 of the block's 32 dims (lane = dim) over the pieces: per piece two float4 loads, each
 // warp-wide load one 512-byte run of the piece (piece layout), up to kU pieces in flight.  The sums
 // are scaled by 1 / l and written to out[row][h][d], 32 consecutive dims (128 bytes) per warp store.
+// KU: pieces whose loads are in flight together.  8 for a few queries with many pieces each (CSA decode:
+// up to 18), 4 for many queries with few pieces (fewer registers, more blocks resident).
+template <int KU>
 __global__ void __launch_bounds__(256) attend_tc_combine(TcArgs a) {
     griddep_wait();  // everything before this kernel on the stream has finished
     griddep_launch_dependents();
-    constexpr int kU = 4;  // pieces whose loads are in flight together
+    constexpr int kU = KU;
     const int row = blockIdx.x, dg = blockIdx.y;
     const long long rs = (long long)row * a.tpr, re = rs + a.tpr - 1;
     // CTA holding flat tile f: the largest c with range_start(c) <= f
@@ -1038,7 +1041,8 @@ cudaError_t launch_attend_tc(const AttendArgs& a, void* ws, size_t ws_bytes, cud
     if (e != cudaSuccess) return e;
     if (p.grid > 1) {
         const size_t csm = (size_t)t.comb_pieces * kH * sizeof(float);
-        e = launch_pdl(attend_tc_combine, dim3(t.rows, kD / 32), dim3(256), csm, stream, t);
+        e = t.comb_pieces > 8 ? launch_pdl(attend_tc_combine<8>, dim3(t.rows, kD / 32), dim3(256), csm, stream, t)
+                              : launch_pdl(attend_tc_combine<4>, dim3(t.rows, kD / 32), dim3(256), csm, stream, t);
         if (e == cudaSuccess) e = cudaGetLastError();
     }
     return e;

@@ -17,6 +17,8 @@
 // output the lanes of one entry are consecutive lanes of one warp, so the
 // entry's amax is found with warp shuffles too; for MXFP4 output (OCP MX,
 // the FP4 indexer keys) each block of 32 channels is 4 consecutive lanes.
+// Long chunks of one unquantised stream (the HCA chunk) go to
+// compress_wide_kernel instead, whose warp loads are coalesced across channels.
 #include "common.cuh"
 #include "internal.h"
 
@@ -217,8 +219,114 @@ __global__ void __launch_bounds__(256) compress_kernel(StreamDesc s0, StreamDesc
     }
 }
 
+// Long chunks (m >= 32: the HCA chunk of 128 tokens) of one stream with bf16 / fp32 output: a block
+// per (entry, 16 channel groups = 128 channels), kWideThreads threads.  Lane l of warp w owns channel
+// group 16 blockIdx.y + l % 16 and token slot 2 w + l / 16, i.e. tokens slot, slot + 32, ... of the
+// chunk (compress_span with a stride of 32), so each warp load reads 256 contiguous bytes of two
+// adjacent token rows.  The two slots of a group within a warp merge with one shuffle, the 16 warps'
+// states through shared memory, and 128 threads (group x channel) finish.  (The lanes-per-entry
+// mapping of compress_kernel has each warp load touch 32 token rows, 16 bytes each.)
+constexpr int kWideGroups = 16;
+constexpr int kWideThreads = 512;
+
+__global__ void __launch_bounds__(kWideThreads) compress_wide_kernel(StreamDesc d, long long n_ent, int m) {
+    griddep_wait();  // everything before this kernel on the stream has finished
+    griddep_launch_dependents();
+    __shared__ float s_st[kWideThreads / 32][kWideGroups][25];  // (max, den, num) x 8 channels, padded
+    __shared__ __align__(16) float s_out[kWideGroups][8];
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int b = (int)(blockIdx.x / n_ent);
+    const long long s = blockIdx.x - (long long)b * n_ent;
+    const int gl = lane & 15, grp = blockIdx.y * kWideGroups + gl;
+    const int slot = 2 * w + (lane >> 4);
+    float mx[8], den[8], num[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        mx[e] = -INFINITY;
+        den[e] = 0.f;
+        num[e] = 0.f;
+    }
+    if (grp < d.groups) {
+        StreamDesc dd = d;
+        dd.split = 32;  // token stride of compress_span
+        const long long off = s * m * d.channels + grp * 8;
+        if (d.in_dtype == V4A_BF16) {
+            compress_span(dd, static_cast<const __nv_bfloat16*>(d.x) + (long long)b * d.x_bs + off,
+                          static_cast<const __nv_bfloat16*>(d.gate) + (long long)b * d.gate_bs + off, m, slot, mx,
+                          den, num);
+        } else {
+            compress_span(dd, static_cast<const float*>(d.x) + (long long)b * d.x_bs + off,
+                          static_cast<const float*>(d.gate) + (long long)b * d.gate_bs + off, m, slot, mx, den, num);
+        }
+    }
+    // lanes l and l ^ 16: the same group, two token slots
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        const float gm = fmaxf(mx[e], __shfl_xor_sync(0xffffffffu, mx[e], 16));
+        const float a = mx[e] == -INFINITY ? 0.f : expf(mx[e] - gm);
+        float dn = den[e] * a, nu = num[e] * a;
+        dn += __shfl_xor_sync(0xffffffffu, dn, 16);
+        nu += __shfl_xor_sync(0xffffffffu, nu, 16);
+        mx[e] = gm;
+        den[e] = dn;
+        num[e] = nu;
+    }
+    if (lane < 16) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            s_st[w][gl][3 * e] = mx[e];
+            s_st[w][gl][3 * e + 1] = den[e];
+            s_st[w][gl][3 * e + 2] = num[e];
+        }
+    }
+    __syncthreads();
+    if (threadIdx.x < kWideGroups * 8) {
+        const int gi = threadIdx.x >> 3, ch = threadIdx.x & 7;
+        float gm = -INFINITY;
+#pragma unroll 4
+        for (int v = 0; v < kWideThreads / 32; ++v) gm = fmaxf(gm, s_st[v][gi][3 * ch]);
+        float dn = 0.f, nu = 0.f;
+#pragma unroll 4
+        for (int v = 0; v < kWideThreads / 32; ++v) {
+            const float mv = s_st[v][gi][3 * ch];
+            const float a = mv == -INFINITY ? 0.f : expf(mv - gm);
+            dn = fmaf(s_st[v][gi][3 * ch + 1], a, dn);
+            nu = fmaf(s_st[v][gi][3 * ch + 2], a, nu);
+        }
+        s_out[gi][ch] = nu / dn;
+    }
+    __syncthreads();
+    if (threadIdx.x >= kWideGroups) return;
+    const int og = blockIdx.y * kWideGroups + threadIdx.x;
+    if (og >= d.groups) return;
+    long long obase;
+    if (d.bt) {
+        const long long es = d.first + s;
+        const long long blk = d.bt[(long long)b * d.bt_stride + es / d.epb];
+        if (blk < 0 || blk >= d.n_blocks) return;  // nowhere to write it
+        obase = (blk * d.epb + es % d.epb) * d.channels;
+    } else {
+        obase = (long long)b * d.out_bs + s * d.channels;
+    }
+    float out[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) out[e] = s_out[threadIdx.x][e];
+    if (d.out_dtype == V4A_BF16) Vec8<__nv_bfloat16>::store(static_cast<__nv_bfloat16*>(d.out) + obase + og * 8, out);
+    else Vec8<float>::store(static_cast<float*>(d.out) + obase + og * 8, out);
+}
+
 // quantised outputs need every lane of an entry's block (or entry) to hold a finished value
 bool quantised(int dt) { return dt == V4A_FP8E4M3 || dt == V4A_MXFP4; }
+
+// one stream, unquantised, chunks of at least 32 tokens: compress_wide_kernel
+bool wide(const StreamDesc& s0, bool two_streams, int m) {
+    return !two_streams && m >= 32 && !quantised(s0.out_dtype) && s0.xb == nullptr;
+}
+cudaError_t launch_wide(const StreamDesc& s0, int batch, long long n_ent, int m, cudaStream_t stream) {
+    const dim3 grid((unsigned)((long long)batch * n_ent), (unsigned)((s0.groups + kWideGroups - 1) / kWideGroups));
+    const cudaError_t e = launch_pdl(compress_wide_kernel, grid, dim3(kWideThreads), 0, stream, s0, n_ent, m);
+    return e != cudaSuccess ? e : cudaGetLastError();
+}
 
 // MXFP4 quantisation of rows: one thread per 8 elements, 4 lanes per 32-element block
 template <typename T>
@@ -308,6 +416,7 @@ cudaError_t launch_compress(const v4a_compress_io* kv, const v4a_compress_io* id
     if (batch == 0 || n_ent == 0) return cudaSuccess;
     StreamDesc s0 = describe(kv);
     StreamDesc s1 = idx ? describe(idx) : s0;
+    if (wide(s0, idx != nullptr, m)) return launch_wide(s0, batch, n_ent, m, stream);
     // lanes per (entry, channel group): up to a warp, to spread long chunks; 1 for FP8 output
     // (its per-entry amax runs over the entry's consecutive lanes)
     int split = 1;
@@ -350,6 +459,7 @@ cudaError_t launch_compress_paged(const v4a_compress_io* kv, const v4a_compress_
         d->first = first_entry;
         d->n_blocks = n_blocks;
     }
+    if (wide(s0, idx != nullptr, m)) return launch_wide(s0, batch, n_ent, m, stream);
     int split = 1;
     while (split < 32 && split * 2 <= m) split *= 2;
     if (!quantised(s0.out_dtype)) s0.split = split;

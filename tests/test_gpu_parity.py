@@ -38,7 +38,9 @@ def _sync():
 # ----------------------------------------------------------------------
 
 @pytest.mark.parametrize("fmt,m,n_tok,C", [("f32", 4, 4 * 37 + 3, 128), ("f32", 1, 29, 64), ("f32", 128, 128 * 5 + 17, 128),
-                                         ("bf16", 4, 4 * 300 + 1, 512), ("bf16", 128, 128 * 3, 512)])
+                                         ("bf16", 4, 4 * 300 + 1, 512), ("bf16", 128, 128 * 3, 512),
+                                         # long chunks with a partial channel tile and a chunk not a multiple of 32
+                                         ("bf16", 40, 40 * 7 + 3, 72), ("f32", 64, 64 * 4, 264)])
 def test_compress_matches_oracle(v4a, fmt, m, n_tok, C):
     case = wl.compress_case(2, n_tok, C, fmt, seed=100 + m + C)
     x, z = dev(case["x"]), dev(case["gate"])
