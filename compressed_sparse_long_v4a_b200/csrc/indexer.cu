@@ -676,26 +676,34 @@ __device__ void finish_row(const float* sc, long long nvis, int k, int D, int C,
     __syncthreads();
     const int words = (int)((nvis + 31) >> 5);
     if (words <= kBitmapWords) {
-        // bitmap over the row; thread t owns words [t per, t per + per), its set bits go out in order after
-        // those of lower threads
-        for (int i = threadIdx.x; i < words; i += blockDim.x) bits[i] = 0u;
+        // bitmap over the row; thread t owns words [16 t, 16 t + 16) (kBitmapWords = 16 x kFastThreads), held
+        // in registers from four 16-byte loads, and its set bits go out in order after those of lower threads
+        static_assert(kBitmapWords == 16 * kFastThreads, "bitmap words per thread");
+        uint4* b4 = reinterpret_cast<uint4*>(bits);
+        for (int i = threadIdx.x; i < kBitmapWords / 4; i += blockDim.x) b4[i] = make_uint4(0u, 0u, 0u, 0u);
         __syncthreads();
         for (int i = threadIdx.x; i < total; i += blockDim.x) atomicOr(&bits[sel[i] >> 5], 1u << (sel[i] & 31));
         __syncthreads();
-        const int per = (words + (int)blockDim.x - 1) / (int)blockDim.x, w0 = threadIdx.x * per;
+        uint32_t wv[16];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const uint4 x = b4[4 * threadIdx.x + q];
+            wv[4 * q] = x.x;
+            wv[4 * q + 1] = x.y;
+            wv[4 * q + 2] = x.z;
+            wv[4 * q + 3] = x.w;
+        }
         int cnt = 0;
-#pragma unroll 1
-        for (int j = 0; j < per; ++j)
-            if (w0 + j < words) cnt += __popc(bits[w0 + j]);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) cnt += __popc(wv[j]);
         int tot;
         int pos = block_exclusive_scan(cnt, warp_buf, &tot);
-#pragma unroll 1
-        for (int j = 0; j < per; ++j) {
-            uint32_t b = w0 + j < words ? bits[w0 + j] : 0u;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {  // unrolled: wv stays in registers
+            uint32_t b = wv[j];
             while (b) {
-                const int32_t x = (int32_t)((w0 + j) * 32 + __ffs(b) - 1);
+                io[pos++] = (int32_t)((16 * (int)threadIdx.x + j) * 32 + __ffs(b) - 1);
                 b &= b - 1;
-                io[pos++] = x;
             }
         }
     } else {
