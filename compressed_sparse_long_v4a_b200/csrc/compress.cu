@@ -318,9 +318,11 @@ __global__ void __launch_bounds__(kWideThreads) compress_wide_kernel(StreamDesc 
 // quantised outputs need every lane of an entry's block (or entry) to hold a finished value
 bool quantised(int dt) { return dt == V4A_FP8E4M3 || dt == V4A_MXFP4; }
 
-// one stream, unquantised, chunks of at least 32 tokens: compress_wide_kernel
-bool wide(const StreamDesc& s0, bool two_streams, int m) {
-    return !two_streams && m >= 32 && !quantised(s0.out_dtype) && s0.xb == nullptr;
+// one stream, unquantised, chunks of at least 32 tokens: compress_wide_kernel (a block per entry: the
+// entries of a launch must fit the grid's x dimension)
+bool wide(const StreamDesc& s0, bool two_streams, int batch, long long n_ent, int m) {
+    return !two_streams && m >= 32 && !quantised(s0.out_dtype) && s0.xb == nullptr &&
+           (long long)batch * n_ent <= 0x7fffffffLL;
 }
 cudaError_t launch_wide(const StreamDesc& s0, int batch, long long n_ent, int m, cudaStream_t stream) {
     const dim3 grid((unsigned)((long long)batch * n_ent), (unsigned)((s0.groups + kWideGroups - 1) / kWideGroups));
@@ -416,7 +418,7 @@ cudaError_t launch_compress(const v4a_compress_io* kv, const v4a_compress_io* id
     if (batch == 0 || n_ent == 0) return cudaSuccess;
     StreamDesc s0 = describe(kv);
     StreamDesc s1 = idx ? describe(idx) : s0;
-    if (wide(s0, idx != nullptr, m)) return launch_wide(s0, batch, n_ent, m, stream);
+    if (wide(s0, idx != nullptr, batch, n_ent, m)) return launch_wide(s0, batch, n_ent, m, stream);
     // lanes per (entry, channel group): up to a warp, to spread long chunks; 1 for FP8 output
     // (its per-entry amax runs over the entry's consecutive lanes)
     int split = 1;
@@ -459,7 +461,7 @@ cudaError_t launch_compress_paged(const v4a_compress_io* kv, const v4a_compress_
         d->first = first_entry;
         d->n_blocks = n_blocks;
     }
-    if (wide(s0, idx != nullptr, m)) return launch_wide(s0, batch, n_ent, m, stream);
+    if (wide(s0, idx != nullptr, batch, n_ent, m)) return launch_wide(s0, batch, n_ent, m, stream);
     int split = 1;
     while (split < 32 && split * 2 <= m) split *= 2;
     if (!quantised(s0.out_dtype)) s0.split = split;
