@@ -22,11 +22,12 @@
 // is cut into `grid` contiguous ranges, one per CTA (one CTA per SM).  A CTA
 // whose range covers a query's tiles completely writes that query's output;
 // a query cut between CTAs gets one partial (m, l, O) per piece, merged by
-// attend_tc_combine.  Per CTA: warp 0 loads (TMA for contiguous rows and the
-// query, cp.async gathers for CSA-selected rows) into a ring of 2 or 3 stages, warp 1
-// (all lanes; one elected lane) issues the MMAs, warps 2-5 run the softmax and the output.  Every wait is
-// bounded; on a time-out the CTA records a device fault, poisons its outputs
-// with NaN and winds down.
+// attend_tc_combine.  Per CTA: warp 0 loads into a ring of 2 or 3 stages -- one
+// TMA box per tile for contiguous rows and per query, or, with warp 6 (G = 2),
+// cp.async gathers of selected, paged or ring rows, 32 rows per warp -- warp 1
+// (all lanes; one elected lane) issues the MMAs, warps 2-5 run the softmax and
+// the output.  Every wait is bounded; on a time-out the CTA records a device
+// fault, poisons its outputs with NaN and winds down.
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
